@@ -1,0 +1,417 @@
+"""Float64 CPU oracle for SAS gated block-sparse causal attention.
+
+TEST INFRASTRUCTURE. Only the test suite, the package's smoke check and the
+benchmark's CPU-baseline leg may import this module. The product path (the
+C-ABI library and its Python binding) never calls it, and it shares no code
+with that path: nothing here imports the package, and the package imports
+nothing from here.
+
+What it computes, in the pages' notation (sources named by page title and
+section; none of the pages prints code for this path):
+
+* [Methodology, Eq. 4] and [Gradient Analysis, Eq. 6] of the picx.dev summary
+  of "SAS: Simple Attention Sparsification via End-to-End Optimization of
+  Context Ranking", and [Core equations] of the reproduction README "SAS:
+  End-to-end learning of sparse attention rankings from language-model loss":
+  history gates g = softmax(s) over the history blocks of a query block,
+  log g_m = s_m - LSE(s); the always-retained current block has g0 = 1.
+* [Theoretical Foundation, Eq. 3] (picx.dev) and [Core equations] (README):
+  I = Top-K(s, K) over the history blocks, S = union of the selected blocks.
+* [Methodology, Eq. 9] (picx.dev) with the 1/sqrt(d) scale from [Core
+  equations] (README): o = softmax(q K_S^T / sqrt(d) + log g_S) V_S over the
+  selected blocks plus the causally masked current block.
+* [Gradient Analysis, Eq. 5, inner form] (picx.dev): the gradient reaching a
+  gate; composed here with the Jacobian of Eq. 6 to give d loss / d scores.
+
+Readings where the pages leave a step open (each is listed in the design
+notes with its reason):
+  - the 1/sqrt(d) scale multiplies q.k only, never log g;
+  - the LSE of Eq. 6 runs over all history blocks m < j of query block j
+    (not only the selected ones), so selected gates are not renormalised;
+  - Top-K is taken over the fp32 scores, descending, ties to the lower block
+    index, and returned in that rank order, padded with -1;
+  - K counts history blocks only; block j has n_j = min(K, j) selections;
+  - one selection and one gate vector per (batch, KV head, query block),
+    shared by the G = Hq/Hkv query heads of that KV head;
+  - no gradient flows through the hard selection (idx is piecewise constant);
+  - decode: the query sits at position L-1 and its key is already in the
+    cache; the block holding L-1 is the current block (fully visible), and
+    the C = floor((L-1)/b) blocks before it are the history.
+
+All arithmetic is float64; inputs (fp32 or bf16 values) convert to float64
+exactly. Parity of every function here is pinned by tests against closed
+forms, brute force, library special cases and finite differences.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+
+def _f64(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Gate softmax (Eq. 4 with phi = softmax; Eq. 6) and Top-K (Eq. 3)
+# ---------------------------------------------------------------------------
+
+def log_gates_row(s_row, n: int) -> np.ndarray:
+    """Eq. 6: log g_m = s_m - LSE(s_0 .. s_{n-1}) for the n history blocks."""
+    s = _f64(s_row[:n])
+    if n == 0:
+        return s
+    mx = s.max()
+    lse = mx + math.log(np.exp(s - mx).sum())
+    return s - lse
+
+
+def topk_row(s_row_f32, n: int, K: int) -> list[int]:
+    """Eq. 3: the min(K, n) history blocks with the largest fp32 score.
+
+    A full stable sort by (-score, index): ties go to the lower block index,
+    and the result is in rank order. Scores compare as fp32 values (so -0.0
+    and +0.0 are equal). Returns exactly K entries, padded with -1.
+    """
+    vals = [float(np.float32(x)) for x in s_row_f32[:n]]
+    order = sorted(range(n), key=lambda m: (-vals[m], m))
+    sel = order[:min(K, n)]
+    return sel + [-1] * (K - len(sel))
+
+
+def gate_topk(scores, K: int, causal: bool = True):
+    """Gates and Top-K indices for every row of ``scores``.
+
+    scores: [B, Hkv, R, C] fp32. causal=True: R = C = N and row j has j valid
+    entries (the history of query block j). causal=False: every row has C
+    valid entries (decode). Returns (gates float64 [B,Hkv,R,C], zero past the
+    valid length; log_gates float64, -inf past it; idx int32 [B,Hkv,R,K]).
+    """
+    s = np.asarray(scores)
+    B, H, R, C = s.shape
+    gates = np.zeros((B, H, R, C), dtype=np.float64)
+    logg = np.full((B, H, R, C), -np.inf, dtype=np.float64)
+    idx = np.full((B, H, R, K), -1, dtype=np.int32)
+    for bi in range(B):
+        for h in range(H):
+            for r in range(R):
+                n = min(r, C) if causal else C
+                lg = log_gates_row(s[bi, h, r], n)
+                logg[bi, h, r, :n] = lg
+                gates[bi, h, r, :n] = np.exp(lg)
+                idx[bi, h, r] = topk_row(s[bi, h, r], n, K)
+    return gates, logg, idx
+
+
+# ---------------------------------------------------------------------------
+# Key set of one query block (Eq. 3 selection + the always-retained block)
+# ---------------------------------------------------------------------------
+
+def _key_set(j: int, b: int, T: int, sel_row, logg_row, use_gates: bool):
+    """Columns and additive biases for query block j.
+
+    The selected history blocks contribute all their b keys with bias
+    log g_m (Eq. 9) or 0 (Eq. 2, gates off); the current block j contributes
+    its keys with bias 0 (g0 = 1, Eq. 4). Returns (cols, bias, n_hist_cols).
+    """
+    cols, bias = [], []
+    for m in sel_row:
+        m = int(m)
+        if m < 0:
+            continue
+        cols.extend(range(m * b, (m + 1) * b))
+        bias.extend([float(logg_row[m]) if use_gates else 0.0] * b)
+    nh = len(cols)
+    cur = list(range(j * b, min(T, (j + 1) * b)))
+    cols.extend(cur)
+    bias.extend([0.0] * len(cur))
+    return np.asarray(cols, dtype=np.int64), np.asarray(bias, dtype=np.float64), nh
+
+
+def _block_logits(Qb, Kc, bias, nh, scale, row0, col0_cur):
+    """Gated logits for the rows of one query block against its key set.
+
+    Row r (global position row0 + r) may see current-block key c (global
+    position col0_cur + c) only when col0_cur + c <= row0 + r (causal mask).
+    """
+    X = scale * (Qb @ Kc.T) + bias[None, :]
+    ncur = Kc.shape[0] - nh
+    if ncur:
+        rows = row0 + np.arange(Qb.shape[0])[:, None]
+        keys = col0_cur + np.arange(ncur)[None, :]
+        X[:, nh:] = np.where(keys <= rows, X[:, nh:], -np.inf)
+    return X
+
+
+def _lse_rows(X):
+    mx = X.max(axis=1, keepdims=True)
+    return (mx + np.log(np.exp(X - mx).sum(axis=1, keepdims=True)))[:, 0]
+
+
+def _default_scale(d, scale):
+    return 1.0 / math.sqrt(d) if not scale else float(scale)
+
+
+# ---------------------------------------------------------------------------
+# Forward (Eq. 9)
+# ---------------------------------------------------------------------------
+
+def attn_fwd_block(q, k, v, idx, logg, bi, kvh, j, b, scale=0.0, use_gates=True):
+    """Eq. 9 for the G query heads of KV head ``kvh`` and the rows of block j.
+
+    Returns (o [G, rows, d], lse [G, rows]) in float64.
+    """
+    q, k, v = np.asarray(q), np.asarray(k), np.asarray(v)
+    Hq, T, d = q.shape[1], q.shape[2], q.shape[3]
+    G = Hq // k.shape[1]
+    scale = _default_scale(d, scale)
+    cols, bias, nh = _key_set(j, b, T, idx[bi, kvh, j],
+                              logg[bi, kvh, j] if logg is not None else None, use_gates)
+    Kc = _f64(k[bi, kvh, cols])
+    Vc = _f64(v[bi, kvh, cols])
+    r0, r1 = j * b, min(T, (j + 1) * b)
+    O = np.empty((G, r1 - r0, d))
+    L = np.empty((G, r1 - r0))
+    for g in range(G):
+        h = kvh * G + g
+        X = _block_logits(_f64(q[bi, h, r0:r1]), Kc, bias, nh, scale, r0, j * b)
+        lse = _lse_rows(X)
+        P = np.exp(X - lse[:, None])
+        O[g] = P @ Vc
+        L[g] = lse
+    return O, L
+
+
+def attn_fwd(q, k, v, idx, logg, b, scale=0.0, use_gates=True):
+    """Eq. 9 over every query block. Returns (o [B,Hq,T,d], lse [B,Hq,T])."""
+    B, Hq, T, d = np.shape(q)
+    Hkv = np.shape(k)[1]
+    G = Hq // Hkv
+    N = (T + b - 1) // b
+    o = np.empty((B, Hq, T, d))
+    lse = np.empty((B, Hq, T))
+    for bi in range(B):
+        for kvh in range(Hkv):
+            for j in range(N):
+                O, L = attn_fwd_block(q, k, v, idx, logg, bi, kvh, j, b, scale, use_gates)
+                r0, r1 = j * b, min(T, (j + 1) * b)
+                o[bi, kvh * G:(kvh + 1) * G, r0:r1] = O
+                lse[bi, kvh * G:(kvh + 1) * G, r0:r1] = L
+    return o, lse
+
+
+# ---------------------------------------------------------------------------
+# Backward: chain rule through Eq. 9, then Eq. 5 (inner) and the Eq. 6 Jacobian
+# ---------------------------------------------------------------------------
+
+def attn_bwd_block(q, k, v, dO, idx, logg, bi, kvh, j, b, scale=0.0, use_gates=True):
+    """Gradients contributed by query block j of KV head ``kvh``.
+
+    For the loss L = sum(o * dO): returns a dict with
+      dq   [G, rows, d]        gradient for the block's query rows (complete),
+      cols, dk_c, dv_c         key columns touched and their partial dk/dv,
+      da   {m: value}          dL/d log g_m for every selected history block m,
+    where dL/dX = P * (dP - rowsum(P * dP)) is the softmax Jacobian applied to
+    dP = dO V^T, and da_m sums dL/dX over block m's columns, all rows and all
+    G heads (log g_m enters every logit of block m, shared by the group).
+    """
+    q, k, v, dO = np.asarray(q), np.asarray(k), np.asarray(v), np.asarray(dO)
+    Hq, T, d = q.shape[1], q.shape[2], q.shape[3]
+    G = Hq // k.shape[1]
+    scale = _default_scale(d, scale)
+    cols, bias, nh = _key_set(j, b, T, idx[bi, kvh, j],
+                              logg[bi, kvh, j] if logg is not None else None, use_gates)
+    Kc = _f64(k[bi, kvh, cols])
+    Vc = _f64(v[bi, kvh, cols])
+    r0, r1 = j * b, min(T, (j + 1) * b)
+    dq = np.zeros((G, r1 - r0, d))
+    dk_c = np.zeros_like(Kc)
+    dv_c = np.zeros_like(Vc)
+    dX_hist = np.zeros(nh)
+    for g in range(G):
+        h = kvh * G + g
+        Qb = _f64(q[bi, h, r0:r1])
+        dOb = _f64(dO[bi, h, r0:r1])
+        X = _block_logits(Qb, Kc, bias, nh, scale, r0, j * b)
+        P = np.exp(X - _lse_rows(X)[:, None])
+        dP = dOb @ Vc.T
+        dX = P * (dP - (P * dP).sum(axis=1, keepdims=True))
+        dq[g] = scale * (dX @ Kc)
+        dk_c += scale * (dX.T @ Qb)
+        dv_c += P.T @ dOb
+        dX_hist += dX[:, :nh].sum(axis=0)
+    da = {}
+    pos = 0
+    for m in idx[bi, kvh, j]:
+        m = int(m)
+        if m < 0:
+            continue
+        da[m] = dX_hist[pos:pos + b].sum()
+        pos += b
+    return {"dq": dq, "cols": cols, "dk_c": dk_c, "dv_c": dv_c, "da": da}
+
+
+def dscores_row(da: dict, gates_row, n: int) -> np.ndarray:
+    """Eq. 6 Jacobian: dL/ds_k = [k in I] da_k - g_k * sum_{m in I} da_m, k < n.
+
+    d log g_m / d s_k = delta_mk - g_k, so only the selected blocks' da enter;
+    no gradient flows through the (piecewise constant) selection itself.
+    """
+    out = np.zeros(n)
+    tot = sum(da.values())
+    g = _f64(gates_row[:n])
+    out[:] = -g * tot
+    for m, a in da.items():
+        out[m] += a
+    return out
+
+
+def attn_bwd(q, k, v, dO, idx, gates, logg, b, scale=0.0, use_gates=True):
+    """Full backward. Returns (dq, dk, dv, dscores) in float64.
+
+    dscores has the shape of the training score tensor [B, Hkv, N, N]: row j
+    holds dL/ds_{j,k} for k < j and zero elsewhere; all zero when gates are off.
+    """
+    B, Hq, T, d = np.shape(q)
+    Hkv = np.shape(k)[1]
+    G = Hq // Hkv
+    N = (T + b - 1) // b
+    dq = np.zeros((B, Hq, T, d))
+    dk = np.zeros((B, Hkv, T, d))
+    dv = np.zeros((B, Hkv, T, d))
+    ds = np.zeros((B, Hkv, N, N))
+    for bi in range(B):
+        for kvh in range(Hkv):
+            for j in range(N):
+                r = attn_bwd_block(q, k, v, dO, idx, logg, bi, kvh, j, b, scale, use_gates)
+                r0, r1 = j * b, min(T, (j + 1) * b)
+                dq[bi, kvh * G:(kvh + 1) * G, r0:r1] = r["dq"]
+                np.add.at(dk[bi, kvh], r["cols"], r["dk_c"])
+                np.add.at(dv[bi, kvh], r["cols"], r["dv_c"])
+                if use_gates:
+                    ds[bi, kvh, j, :j] = dscores_row(r["da"], gates[bi, kvh, j], j)
+    return dq, dk, dv, ds
+
+
+def gate_grad_eq5(q, k, v, dO, idx, gates, logg, bi, kvh, j, b, scale=0.0):
+    """Eq. 5, inner form, literally: dg_m = sum_i (p~_i / g_m) dO^T (v_i - o).
+
+    The sum runs over the keys i of selected block m, for every row and every
+    head of the group, with p~ the gated attention probability and o that
+    row's output. Returns {m: dg_m}. Used as an independent pin: g_m * dg_m
+    must equal da_m of ``attn_bwd_block``.
+    """
+    q, k, v, dO = np.asarray(q), np.asarray(k), np.asarray(v), np.asarray(dO)
+    Hq, T, d = q.shape[1], q.shape[2], q.shape[3]
+    G = Hq // k.shape[1]
+    scale = _default_scale(d, scale)
+    cols, bias, nh = _key_set(j, b, T, idx[bi, kvh, j], logg[bi, kvh, j], True)
+    Kc = _f64(k[bi, kvh, cols])
+    Vc = _f64(v[bi, kvh, cols])
+    r0, r1 = j * b, min(T, (j + 1) * b)
+    out = {}
+    sel = [int(m) for m in idx[bi, kvh, j] if m >= 0]
+    for g in range(G):
+        h = kvh * G + g
+        X = _block_logits(_f64(q[bi, h, r0:r1]), Kc, bias, nh, scale, r0, j * b)
+        P = np.exp(X - _lse_rows(X)[:, None])
+        O = P @ Vc
+        dOb = _f64(dO[bi, h, r0:r1])
+        for pos, m in enumerate(sel):
+            blk = slice(pos * b, (pos + 1) * b)
+            term = (P[:, blk] / gates[bi, kvh, j, m]) * (dOb @ Vc[blk].T - (dOb * O).sum(1)[:, None])
+            out[m] = out.get(m, 0.0) + term.sum()
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Decode (Eq. 2 with gates dropped, or Eq. 9) for one query token
+# ---------------------------------------------------------------------------
+
+def decode(q, kcache, vcache, idx, logg, b, scale=0.0, use_gates=False):
+    """One query token per (batch, q head) at position L-1 of the cache.
+
+    q [B,Hq,d]; kcache/vcache [B,Hkv,L,d]; idx [B,Hkv,K] over the
+    C = floor((L-1)/b) history blocks; logg [B,Hkv,C] (used when use_gates).
+    Keys: the selected history blocks (bias log g_m, or 0 with gates off)
+    plus every position of the current block up to L-1 (bias 0).
+    Returns o [B,Hq,d] float64.
+    """
+    q, kc, vc = np.asarray(q), np.asarray(kcache), np.asarray(vcache)
+    B, Hq, d = q.shape
+    Hkv, L = kc.shape[1], kc.shape[2]
+    G = Hq // Hkv
+    scale = _default_scale(d, scale)
+    cb = (L - 1) // b
+    o = np.empty((B, Hq, d))
+    for bi in range(B):
+        for kvh in range(Hkv):
+            cols, bias = [], []
+            for m in idx[bi, kvh]:
+                m = int(m)
+                if m < 0:
+                    continue
+                cols.extend(range(m * b, (m + 1) * b))
+                bias.extend([float(logg[bi, kvh, m]) if use_gates else 0.0] * b)
+            cols.extend(range(cb * b, L))
+            bias.extend([0.0] * (L - cb * b))
+            Kc = _f64(kc[bi, kvh, cols])
+            Vc = _f64(vc[bi, kvh, cols])
+            bias = np.asarray(bias)
+            for g in range(G):
+                h = kvh * G + g
+                x = scale * (Kc @ _f64(q[bi, h])) + bias
+                mx = x.max()
+                p = np.exp(x - mx)
+                o[bi, h] = (p @ Vc) / p.sum()
+    return o
+
+
+# ---------------------------------------------------------------------------
+# Dense comparison (Eq. 1 with a causal mask): every block, gates off
+# ---------------------------------------------------------------------------
+
+def all_blocks_idx(B, Hkv, N):
+    """Selection of every history block (rank order = ascending index)."""
+    idx = np.full((B, Hkv, N, max(N - 1, 1)), -1, dtype=np.int32)
+    for j in range(N):
+        idx[:, :, j, :j] = np.arange(j, dtype=np.int32)
+    return idx
+
+
+def dense_fwd(q, k, v, b, scale=0.0):
+    B, Hq, T, d = np.shape(q)
+    N = (T + b - 1) // b
+    return attn_fwd(q, k, v, all_blocks_idx(B, np.shape(k)[1], N), None, b, scale,
+                    use_gates=False)
+
+
+def dense_decode(q, kcache, vcache, scale=0.0):
+    """Every cache position 0..L-1 attends, gates off."""
+    q, kc, vc = np.asarray(q), np.asarray(kcache), np.asarray(vcache)
+    B, Hq, d = q.shape
+    G = Hq // kc.shape[1]
+    scale = _default_scale(d, scale)
+    o = np.empty((B, Hq, d))
+    for bi in range(B):
+        for h in range(Hq):
+            Kc = _f64(kc[bi, h // G])
+            x = scale * (Kc @ _f64(q[bi, h]))
+            p = np.exp(x - x.max())
+            o[bi, h] = (p @ _f64(vc[bi, h // G])) / p.sum()
+    return o
+
+
+# ---------------------------------------------------------------------------
+# Algorithmic work counts (for throughput figures, not for any result)
+# ---------------------------------------------------------------------------
+
+def attended_pairs(B, Hq, T, b, K):
+    """Sum over query rows of the number of keys each row attends."""
+    N = (T + b - 1) // b
+    total = 0
+    for j in range(N):
+        rows = min(T, (j + 1) * b) - j * b
+        total += rows * b * min(K, j) + rows * (rows + 1) // 2
+    return total * B * Hq
