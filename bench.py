@@ -1,0 +1,441 @@
+"""Benchmark of the SAS gated block-sparse attention library on B200.
+
+One step = one pass of the training hot path over one synthetic batch of the
+Qwen3-4B-shaped layer (B=1, 32 q heads / 8 KV heads, d=128, T=16384, b=64,
+K=16): gate softmax + Top-K (sas_gate_topk), the gated sparse forward
+(sas_attn_fwd) and its backward into q, k, v and the selector scores
+(sas_attn_bwd). `value` is the algorithmic fwd+bwd TFLOP/s of the whole job
+(14*d FLOPs per attended (query, key) pair per query head; dense and skipped
+work never counted). Beside it the line reports the decode hot path (one token
+per sequence over 64K and 512K caches, gates off and on) in GB/s of selected
+K/V bytes, the same library's dense kernels, the roofline of the dominant
+kernel, an end-to-end figure through host buffers and the float64 oracle's
+CPU throughput.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs its own batch (weak scaling, no
+collective on the data path); the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_attention_sas_b200 import dist as D  # noqa: E402
+from block_sparse_attention_sas_b200 import workloads as W  # noqa: E402
+
+TRAIN = W.QWEN3_4B_TRAIN
+DECODES = [(W.QWEN3_4B_DECODE, 0), (W.QWEN3_4B_DECODE, 1), (W.QWEN3_14B_DECODE, 0)]
+METRIC = "gated sparse attn fwd+bwd TFLOP/s & decode GB/s; % of B200 roofline"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def attended_pairs(B, Hq, T, b, K):
+    """Sum over query rows of the keys each row attends (selected blocks + causal current)."""
+    N = (T + b - 1) // b
+    tot = 0
+    for j in range(N):
+        rows = min(T, (j + 1) * b) - j * b
+        tot += rows * b * min(K, j) + rows * (rows + 1) // 2
+    return tot * B * Hq
+
+
+def train_flops(cfg):
+    pairs = attended_pairs(cfg.B, cfg.Hq, cfg.T, cfg.b, cfg.K)
+    return 4 * cfg.d * pairs, 10 * cfg.d * pairs
+
+
+def decode_bytes(cfg, dense=False):
+    """Algorithmic bytes of one decode call: the attended K and V rows
+    (selected history blocks + the current block) plus q, o, idx and gates."""
+    e = 2 if cfg.dtype == "bf16" else 4
+    n_blocks = (cfg.C + 1) if dense else (min(cfg.K, cfg.C) + 1)
+    cur = cfg.L - cfg.C * cfg.b
+    rows = (n_blocks - 1) * cfg.b + cur
+    kv = 2 * rows * cfg.d * e * cfg.B * cfg.Hkv
+    small = 2 * cfg.B * cfg.Hq * cfg.d * e + (0 if dense else cfg.B * cfg.Hkv * cfg.K * 4)
+    return kv + small
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ---------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.proc = None
+        self.path = None
+        self.gpu_id = gpu_id
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            cmd = ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                   "-lms", "200"]
+            if self.gpu_id:
+                cmd += ["-i", self.gpu_id]
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_pci_id(torch, dev):
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        return "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        return vis.split(",")[dev.index or 0] if vis else str(dev.index or 0)
+
+
+# ------------------------------------------------------------------ CPU side
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_sample(cfg, kv_heads=(0,), x=None):
+    """The float64 oracle on a bounded sample of the training layer: every query
+    block of the given KV heads (gates, Top-K, forward, backward). Returns
+    (seconds, algorithmic FLOPs of the sample)."""
+    from oracle import sas_oracle as O
+    if x is None:
+        x = W.make_train_inputs(cfg)
+    t0 = time.perf_counter()
+    for kvh in kv_heads:
+        sl = slice(kvh, kvh + 1)
+        g, lg, ix = O.gate_topk(x.scores[:, sl], cfg.K)
+        q = x.q[:, kvh * cfg.G:(kvh + 1) * cfg.G]
+        k, v = x.k[:, sl], x.v[:, sl]
+        dO = x.dO[:, kvh * cfg.G:(kvh + 1) * cfg.G]
+        O.attn_fwd(q, k, v, ix, lg, cfg.b)
+        O.attn_bwd(q, k, v, dO, ix, g, lg, cfg.b)
+    dt = time.perf_counter() - t0
+    f, b = train_flops(cfg)
+    return dt, (f + b) * len(kv_heads) / (cfg.B * cfg.Hkv)
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args):
+    import torch
+    from block_sparse_attention_sas_b200 import _lib as S
+
+    rank, local_rank, world = D.env_rank()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    D.init("nccl", timeout_s=300)
+    peaks = load_peaks()
+    cfg = TRAIN
+    seed = D.rank_seed(cfg.seed, rank)
+
+    # ---- inputs: host (pinned) and device copies
+    x = W.make_train_inputs(cfg, seed=seed)
+    bf = torch.bfloat16
+
+    def pin(a, dt):
+        t = torch.from_numpy(a)
+        if dt is not None:
+            t = t.to(dt)
+        return t.pin_memory()
+
+    h = dict(q=pin(x.q, bf), k=pin(x.k, bf), v=pin(x.v, bf), dO=pin(x.dO, bf),
+             scores=pin(x.scores, None))
+    d = {n: t.to(dev, non_blocking=False) for n, t in h.items()}
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    f_fwd, f_bwd = train_flops(cfg)
+
+    def step(inp, ev=None):
+        if ev:
+            ev[0].record(stream)
+        gates, idx = S.gate_topk(inp["scores"], cfg.K, causal=True)
+        if ev:
+            ev[1].record(stream)
+        o, lse = S.attn_fwd(inp["q"], inp["k"], inp["v"], idx, gates, cfg.b)
+        if ev:
+            ev[2].record(stream)
+        dq, dk, dv, ds = S.attn_bwd(inp["q"], inp["k"], inp["v"], o, lse, inp["dO"], idx, gates,
+                                    cfg.b)
+        if ev:
+            ev[3].record(stream)
+        return o, dq, dk, dv, ds
+
+    for _ in range(args.warmup):
+        step(d)
+    torch.cuda.synchronize(dev)
+    st, raw = S.device_error()
+    if st != 0:
+        raise SystemExit(f"device error during warm-up: {raw:#x}")
+
+    # ---- timed region: K steps, L2 flushed before each, CUDA events per step
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    n_launch0 = S.launch_count()
+    with ClockSampler(gpu_pci_id(torch, dev)) as clk:
+        D.barrier(dev)
+        torch.cuda.synchronize(dev)
+        t_wall = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()
+            step(d, evs[i])
+        torch.cuda.synchronize(dev)
+        t_wall = time.perf_counter() - t_wall
+        D.barrier(dev)
+    launches = S.launch_count() - n_launch0
+    clocks = clk.summary()
+    per = [[e[a].elapsed_time(e[a + 1]) for a in range(3)] for e in evs]  # ms
+    step_ms = sum(sum(p) for p in per) / args.steps
+    k_ms = {n: sum(p[i] for p in per) / args.steps for i, n in
+            enumerate(("sas_gate_topk", "sas_attn_fwd", "sas_attn_bwd"))}
+    step_ms_max = D.max_over_ranks(step_ms, dev)
+    value = world * (f_fwd + f_bwd) / (step_ms_max * 1e-3) / 1e12
+
+    # ---- e2e: host buffers in, result (dscores, the selector gradient) out
+    out_h = torch.empty((cfg.B, cfg.Hkv, cfg.N, cfg.N), dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in h.values())
+    d2h = out_h.numel() * out_h.element_size()
+    e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    D.barrier(dev)
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()
+        e_ev[i][0].record(stream)
+        for n in d:
+            d[n].copy_(h[n], non_blocking=True)
+        ds = step(d)[4]
+        out_h.copy_(ds, non_blocking=True)
+        e_ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = D.max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev) / args.steps, dev)
+    e2e_val = world * (f_fwd + f_bwd) / (e2e_ms * 1e-3) / 1e12
+
+    # ---- decode lines (one call per timing, L2 flushed before each)
+    decode_lines = []
+    if not args.no_decode:
+        decode_lines = bench_decode(S, torch, dev, stream, flush, peaks, args, rank)
+
+    # ---- roofline of the dominant call of the training step
+    dom = max(k_ms, key=k_ms.get)
+    dom_flops = {"sas_attn_fwd": f_fwd, "sas_attn_bwd": f_bwd}.get(dom, 0.0)
+    achieved = dom_flops / (k_ms[dom] * 1e-3) / 1e12 if dom_flops else None
+    roof = {"kernel": dom, "bound": "tensor", "achieved": achieved,
+            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": (achieved / peaks["bf16_tflops"]) if achieved else None,
+            "traffic": None, "peak_source": peaks["source"] + " (burst bf16 dense)"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded numpy PCG64; shapes and distributions of the Qwen3-4B layer)",
+        "config": {"workload": cfg.name, "model": "qwen3-4b attention layer (synthetic)",
+                   "global_batch": cfg.B * world, "seq_len": cfg.T, "parallelism": f"dp{world}",
+                   "heads": f"{cfg.Hq}/{cfg.Hkv}", "head_dim": cfg.d, "block": cfg.b,
+                   "K": cfg.K, "l2": "flushed (256 MB write) before every timed step",
+                   "algorithmic_tflop_per_step": (f_fwd + f_bwd) / 1e12},
+        "kernels_ms": k_ms,
+        "roofline": roof,
+        "e2e": {"value": e2e_val, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "decode": decode_lines,
+        "wall_s_timed": t_wall,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu:
+        kvh = tuple(range(args.cpu_heads))
+        secs, fl = oracle_sample(cfg, kvh, x)
+        line["cpu_baseline"] = {"value": fl / secs / 1e12, "unit": "TFLOP/s",
+                                "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"float64 oracle, gates+top-k+fwd+bwd of {len(kvh)} of "
+                                          f"{cfg.Hkv} KV heads of {cfg.name} ({secs:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    D.shutdown()
+
+
+def bench_decode(S, torch, dev, stream, flush, peaks, args, rank):
+    out = []
+    cache = {}
+    for cfg, use_gates in DECODES:
+        if cfg.name not in cache:
+            cache.clear()
+            torch.cuda.empty_cache()
+            x = W.make_decode_inputs(cfg, seed=D.rank_seed(cfg.seed, rank))
+            bf = torch.bfloat16
+            cache[cfg.name] = dict(
+                q=torch.from_numpy(x.q).to(bf).to(dev),
+                kc=torch.from_numpy(x.kcache).to(bf).to(dev),
+                vc=torch.from_numpy(x.vcache).to(bf).to(dev),
+                s=torch.from_numpy(x.scores[:, :, None, :].copy()).to(dev))
+            del x
+        t = cache[cfg.name]
+
+        def one(ev=None):
+            if ev:
+                ev[0].record(stream)
+            gates, idx = S.gate_topk(t["s"], cfg.K, causal=False)
+            if ev:
+                ev[1].record(stream)
+            o = S.decode(t["q"], t["kc"], t["vc"], idx[:, :, 0], gates[:, :, 0], use_gates, cfg.b,
+                         L=cfg.L)
+            if ev:
+                ev[2].record(stream)
+            return o
+
+        for _ in range(max(3, args.warmup)):
+            one()
+        reps = max(10, args.steps)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+        for i in range(reps):
+            flush.zero_()
+            one(evs[i])
+        torch.cuda.synchronize(dev)
+        topk_us = 1e3 * statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+        dec_us = 1e3 * statistics.median(e[1].elapsed_time(e[2]) for e in evs)
+        nbytes = decode_bytes(cfg)
+        gbs = nbytes / (dec_us * 1e-6) / 1e9
+        line = {"workload": cfg.name, "use_gates": use_gates, "decode_us": dec_us,
+                "gate_topk_us": topk_us, "step_us": dec_us + topk_us,
+                "selected_bytes": nbytes, "GB/s": gbs,
+                "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                             "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                             "peak_source": peaks["source"] + " (copy bandwidth)"}}
+        if use_gates == 0:
+            dev_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(5)]
+            for i in range(5):
+                flush.zero_()
+                dev_ev[i][0].record(stream)
+                S.dense_decode(t["q"], t["kc"], t["vc"], L=cfg.L)
+                dev_ev[i][1].record(stream)
+            torch.cuda.synchronize(dev)
+            dense_us = 1e3 * statistics.median(a.elapsed_time(b) for a, b in dev_ev)
+            dbytes = decode_bytes(cfg, dense=True)
+            line["dense"] = {"decode_us": dense_us, "bytes": dbytes,
+                             "GB/s": dbytes / (dense_us * 1e-6) / 1e9,
+                             "speedup_sparse_step": dense_us / (dec_us + topk_us)}
+        out.append(line)
+    return out
+
+
+# ----------------------------------------------------------- reference arm
+
+def run_reference(args):
+    """The float64 oracle as it stands, on the host cores: each step is a
+    bounded sample (one KV head of the Qwen3-4B layer: gates, Top-K, forward,
+    backward), reported in the same metric and unit."""
+    rank, _, world = D.env_rank()
+    if rank != 0:
+        return
+    cfg = TRAIN
+    x = W.make_train_inputs(cfg)
+    for _ in range(args.warmup if args.warmup < 2 else 1):
+        oracle_sample(cfg, (0,), x)
+    secs, fl = 0.0, 0.0
+    for i in range(args.steps):
+        s, f = oracle_sample(cfg, (i % cfg.Hkv,), x)
+        secs += s
+        fl += f
+    val = fl / secs / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "sample_per_step": "1 of 8 KV heads"},
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": blas_threads(),
+                             "kind": "oracle",
+                             "sample": "one KV head of the Qwen3-4B layer per step"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-heads", type=int, default=2)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,248 @@
+"""Python binding of the SAS C-ABI library (libsas_b200.so), through ctypes.
+
+Argument marshalling only: every function takes CUDA tensors, allocates the
+outputs (and cached workspaces) with torch, passes raw device pointers, the
+sizes and torch's current stream to the C entry point of the same name, and
+raises SasError on a non-OK status. All computation happens in the library's
+CUDA kernels; there is no other implementation behind these calls, and
+importing this module fails loudly when the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsas_b200.so")
+
+SAS_F32, SAS_BF16 = 0, 1
+STATUS = {0: "SAS_OK", 1: "SAS_ERR_INVALID_ARG", 2: "SAS_ERR_UNSUPPORTED", 3: "SAS_ERR_CUDA",
+          4: "SAS_ERR_TIMEOUT", 5: "SAS_ERR_WORKSPACE", 6: "SAS_ERR_DEVICE"}
+
+
+class SasError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} returned {STATUS.get(status, status)}")
+
+
+_i, _f, _p, _sz = ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+
+# name -> (restype, argtypes); mirrors include/sas.h
+SIGNATURES = {
+    "sas_status_string": (ctypes.c_char_p, [_i]),
+    "sas_version": (_i, []),
+    "sas_launch_count": (ctypes.c_uint64, []),
+    "sas_gate_topk": (_i, [_p, _i, _i, _i, _i, _i, _i, _p, _p, _p]),
+    "sas_attn_fwd": (_i, [_i, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p]),
+    "sas_attn_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "sas_attn_bwd": (_i, [_i, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f,
+                          _p, _p, _p, _p, _p, _sz, _p]),
+    "sas_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "sas_decode": (_i, [_i, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p,
+                        _sz, _p]),
+    "sas_dense_fwd": (_i, [_i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p]),
+    "sas_dense_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "sas_dense_bwd": (_i, [_i, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p,
+                           _p, _sz, _p]),
+    "sas_dense_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "sas_dense_decode": (_i, [_i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _p, _sz, _p]),
+    "sas_get_device_error": (_i, [_p, ctypes.POINTER(ctypes.c_uint32)]),
+    "sas_set_wait_limit": (None, [ctypes.c_uint64]),
+    "sas_selftest_wait_timeout": (_i, [_p]),
+}
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(f"SAS CUDA library not built: {path} is missing "
+                          "(run `python -m block_sparse_attention_sas_b200.build`)")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+LIB = load_library()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise SasError(fn, status)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(dev=None):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return SAS_F32
+    if t.dtype == torch.bfloat16:
+        return SAS_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _need(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+_WS: dict = {}
+
+
+def _workspace(kind: str, nbytes: int, device, zero: bool) -> torch.Tensor:
+    """Cached device workspace (grows on demand). Decode workspaces start
+    zero-filled and the library leaves them zero-filled after every call."""
+    key = (kind, device.index if device.index is not None else torch.cuda.current_device())
+    buf = _WS.get(key)
+    if buf is None or buf.numel() < nbytes:
+        n = max(nbytes, 256)
+        buf = torch.zeros(n, dtype=torch.uint8, device=device) if zero else \
+            torch.empty(n, dtype=torch.uint8, device=device)
+        _WS[key] = buf
+    return buf
+
+
+# ---------------------------------------------------------------------------
+
+def gate_topk(scores: torch.Tensor, K: int, causal: bool = True, gates=None, idx=None):
+    """Gates [B,Hkv,R,C] fp32 and Top-K indices [B,Hkv,R,K] int32 of `scores`."""
+    _need(scores, "scores", torch.float32)
+    B, H, R, C = scores.shape
+    if gates is None:
+        gates = torch.empty_like(scores)
+    if idx is None:
+        idx = torch.empty((B, H, R, K), dtype=torch.int32, device=scores.device)
+    _check("sas_gate_topk", LIB.sas_gate_topk(_ptr(scores), B, H, R, C, int(causal), K,
+                                              _ptr(gates), _ptr(idx), _stream(scores.device)))
+    return gates, idx
+
+
+def attn_fwd(q, k, v, idx, gates, b: int, scale: float = 0.0, o=None, lse=None):
+    """Gated sparse forward. Returns (o, lse)."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, q.dtype)
+    _need(idx, "idx", torch.int32)
+    if gates is not None:
+        _need(gates, "gates", torch.float32)
+    B, Hq, T, d = q.shape
+    Hkv, K = k.shape[1], idx.shape[-1]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    _check("sas_attn_fwd", LIB.sas_attn_fwd(_dtype(q), _ptr(q), _ptr(k), _ptr(v), _ptr(idx),
+                                            _ptr(gates), B, Hq, Hkv, T, d, b, K, scale, _ptr(o),
+                                            _ptr(lse), _stream(q.device)))
+    return o, lse
+
+
+def attn_bwd(q, k, v, o, lse, dO, idx, gates, b: int, scale: float = 0.0,
+             want_dscores: bool = True):
+    """Backward. Returns (dq, dk, dv, dscores or None)."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dO", dO)):
+        _need(t, n, q.dtype)
+    _need(lse, "lse", torch.float32)
+    _need(idx, "idx", torch.int32)
+    B, Hq, T, d = q.shape
+    Hkv, K = k.shape[1], idx.shape[-1]
+    N = (T + b - 1) // b
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ds = None
+    if gates is not None and want_dscores:
+        ds = torch.empty((B, Hkv, N, N), dtype=torch.float32, device=q.device)
+    nbytes = LIB.sas_attn_bwd_workspace_size(B, Hq, Hkv, T, d, b, K)
+    ws = _workspace("bwd", nbytes, q.device, zero=False)
+    _check("sas_attn_bwd", LIB.sas_attn_bwd(_dtype(q), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                            _ptr(lse), _ptr(dO), _ptr(idx), _ptr(gates), B, Hq,
+                                            Hkv, T, d, b, K, scale, _ptr(dq), _ptr(dk), _ptr(dv),
+                                            _ptr(ds), _ptr(ws), ws.numel(), _stream(q.device)))
+    return dq, dk, dv, ds
+
+
+def decode(q, kcache, vcache, idx, gates, use_gates: bool, b: int, L: int | None = None,
+           scale: float = 0.0, o=None):
+    """One-token sparse decode. q [B,Hq,d]; caches [B,Hkv,Lcap,d]; idx [B,Hkv,K]."""
+    for n, t in (("q", q), ("kcache", kcache), ("vcache", vcache)):
+        _need(t, n, q.dtype)
+    _need(idx, "idx", torch.int32)
+    B, Hq, d = q.shape
+    Hkv, Lcap = kcache.shape[1], kcache.shape[2]
+    L = Lcap if L is None else L
+    K = idx.shape[-1]
+    if o is None:
+        o = torch.empty_like(q)
+    nbytes = LIB.sas_decode_workspace_size(B, Hq, Hkv, L, d, b, K)
+    ws = _workspace("decode", nbytes, q.device, zero=True)
+    _check("sas_decode", LIB.sas_decode(_dtype(q), _ptr(q), _ptr(kcache), _ptr(vcache), _ptr(idx),
+                                        _ptr(gates), int(use_gates), B, Hq, Hkv, L, Lcap, d, b, K,
+                                        scale, _ptr(o), _ptr(ws), ws.numel(), _stream(q.device)))
+    return o
+
+
+def dense_fwd(q, k, v, b: int = 64, scale: float = 0.0):
+    B, Hq, T, d = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    _check("sas_dense_fwd", LIB.sas_dense_fwd(_dtype(q), _ptr(q), _ptr(k), _ptr(v), B, Hq,
+                                              k.shape[1], T, d, b, scale, _ptr(o), _ptr(lse),
+                                              _stream(q.device)))
+    return o, lse
+
+
+def dense_bwd(q, k, v, o, lse, dO, b: int = 64, scale: float = 0.0):
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    nbytes = LIB.sas_dense_bwd_workspace_size(B, Hq, Hkv, T, d, b)
+    ws = _workspace("bwd", nbytes, q.device, zero=False)
+    _check("sas_dense_bwd", LIB.sas_dense_bwd(_dtype(q), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                              _ptr(lse), _ptr(dO), B, Hq, Hkv, T, d, b, scale,
+                                              _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(),
+                                              _stream(q.device)))
+    return dq, dk, dv
+
+
+def dense_decode(q, kcache, vcache, L: int | None = None, scale: float = 0.0):
+    B, Hq, d = q.shape
+    Hkv, Lcap = kcache.shape[1], kcache.shape[2]
+    L = Lcap if L is None else L
+    o = torch.empty_like(q)
+    nbytes = LIB.sas_dense_decode_workspace_size(B, Hq, Hkv, L, d)
+    ws = _workspace("dense_decode", nbytes, q.device, zero=True)
+    _check("sas_dense_decode", LIB.sas_dense_decode(_dtype(q), _ptr(q), _ptr(kcache), _ptr(vcache),
+                                                    B, Hq, Hkv, L, Lcap, d, scale, _ptr(o),
+                                                    _ptr(ws), ws.numel(), _stream(q.device)))
+    return o
+
+
+def device_error(stream=None) -> tuple[int, int]:
+    """(status, raw bits) of the current device's error word; clears it."""
+    raw = ctypes.c_uint32(0)
+    st = LIB.sas_get_device_error(stream if stream is not None else _stream(), ctypes.byref(raw))
+    return st, raw.value
+
+
+def launch_count() -> int:
+    """Kernels launched through the library so far in this process."""
+    return int(LIB.sas_launch_count())
+
+
+def set_wait_limit(iterations: int) -> None:
+    LIB.sas_set_wait_limit(iterations)
+
+
+def selftest_wait_timeout() -> None:
+    _check("sas_selftest_wait_timeout", LIB.sas_selftest_wait_timeout(_stream()))

@@ -1,0 +1,666 @@
+// Gated block-sparse causal attention on CUDA cores (fp32 FMA), forward and
+// backward, for every supported (dtype, d, b). This is the exact-fp32 path
+// (TF32 or bf16 tensor cores cannot meet an fp32 tolerance) and the path for
+// shapes the tensor-core kernels do not cover.
+//
+// Forward (picx.dev SAS summary, Methodology Eq. 9; 1/sqrt(d) scale from the
+// reproduction README, Core equations): one CTA per (query block j, row
+// chunk, q head, batch) walks the selected history blocks of its KV head
+// (bias log g_m) and then the current block (bias 0, causal), keeping an
+// online softmax (running max, running sum) per row.
+//
+// Backward (chain rule through Eq. 9; Eq. 5 inner form for the gate
+// gradient; Eq. 6 Jacobian for the scores):
+//   rowdot:  D_i = dO_i . o_i
+//   csr:     per (batch, kv head), the query blocks that selected each key block
+//   dq:      per (query block, q head): recompute P, dP = dO V^T,
+//            dS = P (dP - D), dq += scale dS K, and da(j,m) = sum of dS over
+//            the tile (one partial per q head and row chunk)
+//   dkdv:    per key block: over the diagonal and every selecting query
+//            block and head, dv += P^T dO, dk += scale dS^T Q
+//   jacobian: dscores[j,k] = [k in I_j] da_k - g_k sum_{m in I_j} da_m
+// Every sum has a fixed order, so results are deterministic.
+#include <math.h>
+
+#include "sas_common.cuh"
+#include "sas_internal.h"
+
+namespace sas {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+template <int BS> struct Tiles {
+  static constexpr int ROWS = BS < 64 ? BS : 64;  // query rows per CTA
+  static constexpr int RC = BS / ROWS;             // row chunks per block
+};
+
+__device__ __forceinline__ long long idx_row(const AttnShape& s, int bi, int kvh, int j) {
+  return ((long long)(bi * s.Hkv + kvh) * s.N + j);
+}
+
+// Block m of the iteration `it` for query block j: history slots first, then
+// the current block. Returns false when the slot is empty or invalid.
+__device__ __forceinline__ bool pick_block(const AttnShape& s, const int32_t* idx,
+                                           const float* gates, int bi, int kvh, int j, int it,
+                                           int nsel, int& m, float& bias, bool& cur,
+                                           const DevCtx& ctx) {
+  bias = 0.f;
+  if (it == nsel) {
+    m = j;
+    cur = true;
+    return true;
+  }
+  cur = false;
+  if (s.dense) {
+    m = it;
+    return true;
+  }
+  m = idx[idx_row(s, bi, kvh, j) * s.K + it];
+  if (m < 0) return false;
+  if (m >= j) {
+    if (threadIdx.x == 0) report(ctx, kDevErrBadIndex);
+    return false;
+  }
+  if (gates) bias = logf(gates[idx_row(s, bi, kvh, j) * s.N + m]);
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// Forward
+// ---------------------------------------------------------------------------
+template <typename T, int D, int BS>
+__global__ void __launch_bounds__(kThreads)
+fwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+           const int32_t* __restrict__ idx, const float* __restrict__ gates, AttnShape s,
+           T* __restrict__ o, float* __restrict__ lse, DevCtx ctx) {
+  constexpr int ROWS = Tiles<BS>::ROWS, RC = Tiles<BS>::RC;
+  constexpr int DP = D + 1, BP = BS + 1;
+  constexpr int NACC = ROWS * D / kThreads;
+  extern __shared__ float sm[];
+  float* Qs = sm;
+  float* Ks = Qs + ROWS * DP;
+  float* Vs = Ks + BS * DP;
+  float* Ps = Vs + BS * D;
+  float* row_m = Ps + ROWS * BP;
+  float* row_l = row_m + ROWS;
+  float* row_a = row_l + ROWS;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int j = blockIdx.x / RC, rc = blockIdx.x % RC;
+  const int h = blockIdx.y, bi = blockIdx.z;
+  const int G = s.Hq / s.Hkv, kvh = h / G;
+  const int r0 = j * BS + rc * ROWS;
+  if (r0 >= s.T) return;
+  const long long qbase = (long long)(bi * s.Hq + h) * s.T * D;
+  const long long kbase = (long long)(bi * s.Hkv + kvh) * s.T * D;
+
+  for (int e = tid; e < ROWS * D; e += kThreads) {
+    const int r = e / D, c = e % D, row = r0 + r;
+    Qs[r * DP + c] = row < s.T ? ld_f(q + qbase + (long long)row * D + c) : 0.f;
+  }
+  for (int r = tid; r < ROWS; r += kThreads) {
+    row_m[r] = -INFINITY;
+    row_l[r] = 0.f;
+  }
+  float acc[NACC];
+#pragma unroll
+  for (int x = 0; x < NACC; ++x) acc[x] = 0.f;
+
+  const int nsel = s.dense ? j : s.K;
+  for (int it = 0; it <= nsel; ++it) {
+    int m;
+    float bias;
+    bool cur;
+    if (!pick_block(s, idx, gates, bi, kvh, j, it, nsel, m, bias, cur, ctx)) continue;
+    __syncthreads();
+    for (int e = tid; e < BS * D; e += kThreads) {
+      const int t = e / D, c = e % D, key = m * BS + t;
+      const bool ok = key < s.T;
+      Ks[t * DP + c] = ok ? ld_f(k + kbase + (long long)key * D + c) : 0.f;
+      Vs[t * D + c] = ok ? ld_f(v + kbase + (long long)key * D + c) : 0.f;
+    }
+    __syncthreads();
+    for (int e = tid; e < ROWS * BS; e += kThreads) {
+      const int r = e / BS, c = e % BS;
+      float a = 0.f;
+#pragma unroll 8
+      for (int kk = 0; kk < D; ++kk) a = fmaf(Qs[r * DP + kk], Ks[c * DP + kk], a);
+      float x = fmaf(a, s.scale, bias);
+      const int qi = r0 + r, ki = m * BS + c;
+      if (ki >= s.T || (cur && ki > qi)) x = -INFINITY;
+      Ps[r * BP + c] = x;
+    }
+    __syncthreads();
+    for (int r = warp; r < ROWS; r += kWarps) {
+      float mx = -INFINITY;
+      for (int c = lane; c < BS; c += 32) mx = fmaxf(mx, Ps[r * BP + c]);
+      mx = warp_max(mx);
+      const float mold = row_m[r];
+      const float mnew = fmaxf(mold, mx);
+      float sum = 0.f;
+      for (int c = lane; c < BS; c += 32) {
+        const float p = (mnew == -INFINITY) ? 0.f : expf(Ps[r * BP + c] - mnew);
+        Ps[r * BP + c] = p;
+        sum += p;
+      }
+      sum = warp_sum(sum);
+      if (lane == 0) {
+        const float alpha = (mnew == -INFINITY) ? 1.f : expf(mold - mnew);
+        row_a[r] = alpha;
+        row_l[r] = row_l[r] * alpha + sum;
+        row_m[r] = mnew;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int x = 0; x < NACC; ++x) {
+      const int e = tid + x * kThreads, r = e / D, c = e % D;
+      float a = acc[x] * row_a[r];
+#pragma unroll 8
+      for (int t = 0; t < BS; ++t) a = fmaf(Ps[r * BP + t], Vs[t * D + c], a);
+      acc[x] = a;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int x = 0; x < NACC; ++x) {
+    const int e = tid + x * kThreads, r = e / D, c = e % D, row = r0 + r;
+    if (row < s.T) st_f(o + qbase + (long long)row * D + c, acc[x] / row_l[r]);
+  }
+  for (int r = tid; r < ROWS; r += kThreads) {
+    const int row = r0 + r;
+    if (row < s.T) lse[(long long)(bi * s.Hq + h) * s.T + row] = row_m[r] + logf(row_l[r]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Backward: D_i = dO_i . o_i (one warp per row)
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads)
+rowdot_kernel(const T* __restrict__ o, const T* __restrict__ dO, long long rows,
+              float* __restrict__ Dv) {
+  const long long row = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  float a = 0.f;
+  for (int c = lane; c < D; c += 32) a = fmaf(ld_f(o + row * D + c), ld_f(dO + row * D + c), a);
+  a = warp_sum(a);
+  if (lane == 0) Dv[row] = a;
+}
+
+// ---------------------------------------------------------------------------
+// Backward: reverse index. For (batch, kv head): list[off[m] .. off[m+1]) holds
+// j*K + slot for every query block j whose slot selects key block m, in
+// ascending j. One CTA per (batch, kv head).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads)
+csr_kernel(const int32_t* __restrict__ idx, AttnShape s, int32_t* __restrict__ off_all,
+           int32_t* __restrict__ list_all, DevCtx ctx) {
+  extern __shared__ int32_t cnt[];  // N counts, then N cursors
+  int32_t* cursor = cnt + s.N;
+  const int bh = blockIdx.x;
+  const int32_t* ix = idx + (long long)bh * s.N * s.K;
+  int32_t* off = off_all + (long long)bh * (s.N + 1);
+  int32_t* list = list_all + (long long)bh * s.N * s.K;
+  for (int m = threadIdx.x; m < s.N; m += kThreads) cnt[m] = 0;
+  __syncthreads();
+  const int total = s.N * s.K;
+  for (int e = threadIdx.x; e < total; e += kThreads) {
+    const int j = e / s.K, m = ix[e];
+    if (m >= 0 && m < j) atomicAdd(&cnt[m], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int m = 0; m < s.N; ++m) {
+      const int c = cnt[m];
+      off[m] = run;
+      cursor[m] = run;
+      run += c;
+    }
+    off[s.N] = run;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < total; e += kThreads) {
+    const int j = e / s.K, m = ix[e];
+    if (m >= 0 && m < j) list[atomicAdd(&cursor[m], 1)] = e;
+  }
+  __syncthreads();
+  // Sort each list ascending (e = j*K + slot, so this orders by j).
+  for (int m = threadIdx.x; m < s.N; m += kThreads) {
+    const int lo = off[m], hi = off[m + 1];
+    for (int a = lo + 1; a < hi; ++a) {
+      const int x = list[a];
+      int b = a - 1;
+      while (b >= lo && list[b] > x) {
+        list[b + 1] = list[b];
+        --b;
+      }
+      list[b + 1] = x;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Backward: dq and da (one CTA per query block row chunk and q head)
+// ---------------------------------------------------------------------------
+template <typename T, int D, int BS>
+__global__ void __launch_bounds__(kThreads)
+dq_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+          const float* __restrict__ lse, const T* __restrict__ dO, const float* __restrict__ Dv,
+          const int32_t* __restrict__ idx, const float* __restrict__ gates, AttnShape s,
+          T* __restrict__ dq, float* __restrict__ da, DevCtx ctx) {
+  constexpr int ROWS = Tiles<BS>::ROWS, RC = Tiles<BS>::RC;
+  constexpr int DP = D + 1, BP = BS + 1;
+  constexpr int NACC = ROWS * D / kThreads;
+  extern __shared__ float sm[];
+  float* Qs = sm;
+  float* dOs = Qs + ROWS * DP;
+  float* Ks = dOs + ROWS * DP;
+  float* Vs = Ks + BS * DP;
+  float* Ps = Vs + BS * DP;
+  float* dSs = Ps + ROWS * BP;
+  float* lse_s = dSs + ROWS * BP;
+  float* D_s = lse_s + ROWS;
+  float* red = D_s + ROWS;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int j = blockIdx.x / RC, rc = blockIdx.x % RC;
+  const int h = blockIdx.y, bi = blockIdx.z;
+  const int G = s.Hq / s.Hkv, kvh = h / G;
+  const int r0 = j * BS + rc * ROWS;
+  if (r0 >= s.T) return;
+  const long long qrow0 = (long long)(bi * s.Hq + h) * s.T;
+  const long long kbase = (long long)(bi * s.Hkv + kvh) * s.T * D;
+
+  for (int e = tid; e < ROWS * D; e += kThreads) {
+    const int r = e / D, c = e % D, row = r0 + r;
+    const bool ok = row < s.T;
+    Qs[r * DP + c] = ok ? ld_f(q + (qrow0 + row) * D + c) : 0.f;
+    dOs[r * DP + c] = ok ? ld_f(dO + (qrow0 + row) * D + c) : 0.f;
+  }
+  for (int r = tid; r < ROWS; r += kThreads) {
+    const int row = r0 + r;
+    lse_s[r] = row < s.T ? lse[qrow0 + row] : 0.f;
+    D_s[r] = row < s.T ? Dv[qrow0 + row] : 0.f;
+  }
+  float acc[NACC];
+#pragma unroll
+  for (int x = 0; x < NACC; ++x) acc[x] = 0.f;
+
+  const int nsel = s.dense ? j : s.K;
+  for (int it = 0; it <= nsel; ++it) {
+    int m;
+    float bias;
+    bool cur;
+    if (!pick_block(s, idx, gates, bi, kvh, j, it, nsel, m, bias, cur, ctx)) continue;
+    __syncthreads();
+    for (int e = tid; e < BS * D; e += kThreads) {
+      const int t = e / D, c = e % D, key = m * BS + t;
+      const bool ok = key < s.T;
+      Ks[t * DP + c] = ok ? ld_f(k + kbase + (long long)key * D + c) : 0.f;
+      Vs[t * DP + c] = ok ? ld_f(v + kbase + (long long)key * D + c) : 0.f;
+    }
+    __syncthreads();
+    float dsum = 0.f;
+    for (int e = tid; e < ROWS * BS; e += kThreads) {
+      const int r = e / BS, c = e % BS;
+      float a = 0.f, b = 0.f;
+#pragma unroll 8
+      for (int kk = 0; kk < D; ++kk) {
+        a = fmaf(Qs[r * DP + kk], Ks[c * DP + kk], a);
+        b = fmaf(dOs[r * DP + kk], Vs[c * DP + kk], b);
+      }
+      const int qi = r0 + r, ki = m * BS + c;
+      float p = 0.f;
+      if (qi < s.T && ki < s.T && !(cur && ki > qi)) p = expf(fmaf(a, s.scale, bias) - lse_s[r]);
+      const float ds = p * (b - D_s[r]);
+      Ps[r * BP + c] = p;
+      dSs[r * BP + c] = ds;
+      dsum += ds;
+    }
+    if (!cur && !s.dense && da != nullptr) {
+      dsum = warp_sum(dsum);
+      if (lane == 0) red[warp] = dsum;
+    }
+    __syncthreads();
+    if (!cur && !s.dense && da != nullptr && tid == 0) {
+      float t = 0.f;
+      for (int w = 0; w < kWarps; ++w) t += red[w];
+      da[((qrow0 / s.T) * (long long)s.N * RC + (long long)j * RC + rc) * s.K + it] = t;
+    }
+#pragma unroll
+    for (int x = 0; x < NACC; ++x) {
+      const int e = tid + x * kThreads, r = e / D, c = e % D;
+      float a = 0.f;
+#pragma unroll 8
+      for (int t = 0; t < BS; ++t) a = fmaf(dSs[r * BP + t], Ks[t * DP + c], a);
+      acc[x] = fmaf(a, s.scale, acc[x]);
+    }
+  }
+#pragma unroll
+  for (int x = 0; x < NACC; ++x) {
+    const int e = tid + x * kThreads, r = e / D, c = e % D, row = r0 + r;
+    if (row < s.T) st_f(dq + (qrow0 + row) * D + c, acc[x]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Backward: dk and dv (one CTA per key block, all query blocks that attend it)
+// ---------------------------------------------------------------------------
+template <typename T, int D, int BS>
+__global__ void __launch_bounds__(kThreads)
+dkdv_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+            const float* __restrict__ lse, const T* __restrict__ dO,
+            const float* __restrict__ Dv, const float* __restrict__ gates,
+            const int32_t* __restrict__ csr_off, const int32_t* __restrict__ csr_list,
+            AttnShape s, T* __restrict__ dk, T* __restrict__ dv, DevCtx ctx) {
+  constexpr int QR = Tiles<BS>::ROWS, RC = Tiles<BS>::RC;
+  constexpr int DP = D + 1, BP = BS + 1;
+  constexpr int NACC = BS * D / kThreads;
+  extern __shared__ float sm[];
+  float* Ks = sm;
+  float* Vs = Ks + BS * DP;
+  float* Qs = Vs + BS * DP;
+  float* dOs = Qs + QR * DP;
+  float* Ps = dOs + QR * DP;
+  float* dSs = Ps + QR * BP;
+  float* lse_s = dSs + QR * BP;
+  float* D_s = lse_s + QR;
+
+  const int tid = threadIdx.x;
+  const int m = blockIdx.x, kvh = blockIdx.y, bi = blockIdx.z;
+  const int G = s.Hq / s.Hkv;
+  const long long kbase = (long long)(bi * s.Hkv + kvh) * s.T * D;
+  for (int e = tid; e < BS * D; e += kThreads) {
+    const int t = e / D, c = e % D, key = m * BS + t;
+    const bool ok = key < s.T;
+    Ks[t * DP + c] = ok ? ld_f(k + kbase + (long long)key * D + c) : 0.f;
+    Vs[t * DP + c] = ok ? ld_f(v + kbase + (long long)key * D + c) : 0.f;
+  }
+  float adk[NACC], adv[NACC];
+#pragma unroll
+  for (int x = 0; x < NACC; ++x) adk[x] = adv[x] = 0.f;
+
+  const int bh = bi * s.Hkv + kvh;
+  int n_list;
+  const int32_t* lst = nullptr;
+  if (s.dense) {
+    n_list = s.N - 1 - m;
+  } else {
+    const int lo = csr_off[(long long)bh * (s.N + 1) + m];
+    n_list = csr_off[(long long)bh * (s.N + 1) + m + 1] - lo;
+    lst = csr_list + (long long)bh * s.N * s.K + lo;
+  }
+  for (int it = -1; it < n_list; ++it) {
+    int j;
+    float bias = 0.f;
+    const bool cur = it < 0;
+    if (cur) {
+      j = m;
+    } else if (s.dense) {
+      j = m + 1 + it;
+    } else {
+      j = lst[it] / s.K;
+      if (gates) bias = logf(gates[((long long)bh * s.N + j) * s.N + m]);
+    }
+    for (int g = 0; g < G; ++g) {
+      const int h = kvh * G + g;
+      const long long qrow0 = (long long)(bi * s.Hq + h) * s.T;
+      for (int qc = 0; qc < RC; ++qc) {
+        const int r0 = j * BS + qc * QR;
+        if (r0 >= s.T) break;
+        __syncthreads();
+        for (int e = tid; e < QR * D; e += kThreads) {
+          const int r = e / D, c = e % D, row = r0 + r;
+          const bool ok = row < s.T;
+          Qs[r * DP + c] = ok ? ld_f(q + (qrow0 + row) * D + c) : 0.f;
+          dOs[r * DP + c] = ok ? ld_f(dO + (qrow0 + row) * D + c) : 0.f;
+        }
+        for (int r = tid; r < QR; r += kThreads) {
+          const int row = r0 + r;
+          lse_s[r] = row < s.T ? lse[qrow0 + row] : 0.f;
+          D_s[r] = row < s.T ? Dv[qrow0 + row] : 0.f;
+        }
+        __syncthreads();
+        for (int e = tid; e < QR * BS; e += kThreads) {
+          const int r = e / BS, c = e % BS;
+          float a = 0.f, b = 0.f;
+#pragma unroll 8
+          for (int kk = 0; kk < D; ++kk) {
+            a = fmaf(Qs[r * DP + kk], Ks[c * DP + kk], a);
+            b = fmaf(dOs[r * DP + kk], Vs[c * DP + kk], b);
+          }
+          const int qi = r0 + r, ki = m * BS + c;
+          float p = 0.f;
+          if (qi < s.T && ki < s.T && !(cur && ki > qi)) p = expf(fmaf(a, s.scale, bias) - lse_s[r]);
+          Ps[r * BP + c] = p;
+          dSs[r * BP + c] = p * (b - D_s[r]);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int x = 0; x < NACC; ++x) {
+          const int e = tid + x * kThreads, t = e / D, c = e % D;
+          float a = adv[x], b = 0.f;
+#pragma unroll 8
+          for (int r = 0; r < QR; ++r) {
+            a = fmaf(Ps[r * BP + t], dOs[r * DP + c], a);
+            b = fmaf(dSs[r * BP + t], Qs[r * DP + c], b);
+          }
+          adv[x] = a;
+          adk[x] = fmaf(b, s.scale, adk[x]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int x = 0; x < NACC; ++x) {
+    const int e = tid + x * kThreads, t = e / D, c = e % D, key = m * BS + t;
+    if (key < s.T) {
+      st_f(dk + kbase + (long long)key * D + c, adk[x]);
+      st_f(dv + kbase + (long long)key * D + c, adv[x]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Backward: gate-softmax Jacobian (Eq. 6), one warp per score row
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads)
+jacobian_kernel(const float* __restrict__ da, const int32_t* __restrict__ idx,
+                const float* __restrict__ gates, AttnShape s, int RC, float* __restrict__ ds) {
+  const long long row = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const long long rows = (long long)s.B * s.Hkv * s.N;
+  if (row >= rows) return;
+  const int j = (int)(row % s.N);
+  const long long bh = row / s.N;
+  const int bi = (int)(bh / s.Hkv), kvh = (int)(bh % s.Hkv);
+  const int G = s.Hq / s.Hkv;
+  const int32_t* ix = idx + row * s.K;
+  // da of each slot: sum over the group's heads and the row chunks.
+  float tot = 0.f;
+  for (int sl = lane; sl < s.K; sl += 32) {
+    const int m = ix[sl];
+    if (m < 0 || m >= j) continue;
+    float a = 0.f;
+    for (int g = 0; g < G; ++g)
+      for (int rc = 0; rc < RC; ++rc)
+        a += da[(((long long)(bi * s.Hq + kvh * G + g) * s.N + j) * RC + rc) * s.K + sl];
+    tot += a;
+  }
+  tot = warp_sum(tot);
+  float* out = ds + row * s.N;
+  const float* g = gates + row * s.N;
+  for (int kk = lane; kk < s.N; kk += 32) out[kk] = (kk < j) ? -g[kk] * tot : 0.f;
+  __syncwarp();
+  for (int sl = lane; sl < s.K; sl += 32) {
+    const int m = ix[sl];
+    if (m < 0 || m >= j) continue;
+    float a = 0.f;
+    for (int g2 = 0; g2 < G; ++g2)
+      for (int rc = 0; rc < RC; ++rc)
+        a += da[(((long long)(bi * s.Hq + kvh * G + g2) * s.N + j) * RC + rc) * s.K + sl];
+    out[m] += a;
+  }
+}
+
+size_t fwd_smem(int D, int BS) {
+  const int ROWS = BS < 64 ? BS : 64;
+  return sizeof(float) *
+         ((size_t)ROWS * (D + 1) + (size_t)BS * (D + 1) + (size_t)BS * D + (size_t)ROWS * (BS + 1) +
+          3 * ROWS);
+}
+size_t dq_smem(int D, int BS) {
+  const int ROWS = BS < 64 ? BS : 64;
+  return sizeof(float) * (2 * (size_t)ROWS * (D + 1) + 2 * (size_t)BS * (D + 1) +
+                          2 * (size_t)ROWS * (BS + 1) + 2 * ROWS + kWarps);
+}
+size_t dkdv_smem(int D, int BS) {
+  const int QR = BS < 64 ? BS : 64;
+  return sizeof(float) * (2 * (size_t)BS * (D + 1) + 2 * (size_t)QR * (D + 1) +
+                          2 * (size_t)QR * (BS + 1) + 2 * QR);
+}
+
+template <typename T, int D, int BS>
+cudaError_t fwd_t(const AttnShape& s, const void* q, const void* k, const void* v,
+                  const int32_t* idx, const float* gates, void* o, float* lse, const DevCtx& ctx,
+                  cudaStream_t st) {
+  const size_t smem = fwd_smem(D, BS);
+  auto kern = fwd_kernel<T, D, BS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(s.N * Tiles<BS>::RC, s.Hq, s.B);
+  kern<<<grid, kThreads, smem, st>>>((const T*)q, (const T*)k, (const T*)v, idx, gates, s, (T*)o,
+                                     lse, ctx);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+template <typename T, int D, int BS>
+cudaError_t bwd_t(const AttnShape& s, const void* q, const void* k, const void* v, const void* o,
+                  const float* lse, const void* dO, const int32_t* idx, const float* gates,
+                  void* dq, void* dk, void* dv, float* dscores, void* ws, const DevCtx& ctx,
+                  cudaStream_t st) {
+  const BwdWorkspace L = bwd_workspace_layout(s);
+  char* w = static_cast<char*>(ws);
+  float* Dv = reinterpret_cast<float*>(w + L.off_D);
+  float* da = reinterpret_cast<float*>(w + L.off_da);
+  int32_t* coff = reinterpret_cast<int32_t*>(w + L.off_csr_off);
+  int32_t* clist = reinterpret_cast<int32_t*>(w + L.off_csr_list);
+  cudaError_t e;
+  const long long rows = (long long)s.B * s.Hq * s.T;
+  rowdot_kernel<T, D><<<(unsigned)((rows + kWarps - 1) / kWarps), kThreads, 0, st>>>(
+      (const T*)o, (const T*)dO, rows, Dv);
+  note_launches(1);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (!s.dense) {
+    const size_t smem = 2 * sizeof(int32_t) * (size_t)s.N;
+    e = cudaFuncSetAttribute(csr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    csr_kernel<<<s.B * s.Hkv, kThreads, smem, st>>>(idx, s, coff, clist, ctx);
+    note_launches(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  {
+    const size_t smem = dq_smem(D, BS);
+    auto kern = dq_kernel<T, D, BS>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(s.N * Tiles<BS>::RC, s.Hq, s.B);
+    kern<<<grid, kThreads, smem, st>>>((const T*)q, (const T*)k, (const T*)v, lse, (const T*)dO,
+                                       Dv, idx, gates, s, (T*)dq, dscores ? da : nullptr, ctx);
+    note_launches(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  {
+    const size_t smem = dkdv_smem(D, BS);
+    auto kern = dkdv_kernel<T, D, BS>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(s.N, s.Hkv, s.B);
+    kern<<<grid, kThreads, smem, st>>>((const T*)q, (const T*)k, (const T*)v, lse, (const T*)dO,
+                                       Dv, gates, coff, clist, s, (T*)dk, (T*)dv, ctx);
+    note_launches(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (dscores) {
+    const long long srows = (long long)s.B * s.Hkv * s.N;
+    jacobian_kernel<<<(unsigned)((srows + kWarps - 1) / kWarps), kThreads, 0, st>>>(
+        da, idx, gates, s, Tiles<BS>::RC, dscores);
+    note_launches(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+template <typename T>
+cudaError_t fwd_dispatch(const AttnShape& s, const void* q, const void* k, const void* v,
+                         const int32_t* idx, const float* gates, void* o, float* lse,
+                         const DevCtx& ctx, cudaStream_t st) {
+#define SAS_FWD_CASE(DD, BB) \
+  if (s.d == DD && s.b == BB) return fwd_t<T, DD, BB>(s, q, k, v, idx, gates, o, lse, ctx, st);
+  SAS_FWD_CASE(64, 16) SAS_FWD_CASE(64, 32) SAS_FWD_CASE(64, 64)
+  SAS_FWD_CASE(128, 16) SAS_FWD_CASE(128, 32) SAS_FWD_CASE(128, 64)
+#undef SAS_FWD_CASE
+  return cudaErrorInvalidValue;
+}
+
+template <typename T>
+cudaError_t bwd_dispatch(const AttnShape& s, const void* q, const void* k, const void* v,
+                         const void* o, const float* lse, const void* dO, const int32_t* idx,
+                         const float* gates, void* dq, void* dk, void* dv, float* dscores,
+                         void* ws, const DevCtx& ctx, cudaStream_t st) {
+#define SAS_BWD_CASE(DD, BB)                                                                    \
+  if (s.d == DD && s.b == BB)                                                                   \
+    return bwd_t<T, DD, BB>(s, q, k, v, o, lse, dO, idx, gates, dq, dk, dv, dscores, ws, ctx, \
+                            st);
+  SAS_BWD_CASE(64, 16) SAS_BWD_CASE(64, 32) SAS_BWD_CASE(64, 64)
+  SAS_BWD_CASE(128, 16) SAS_BWD_CASE(128, 32) SAS_BWD_CASE(128, 64)
+#undef SAS_BWD_CASE
+  return cudaErrorInvalidValue;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace
+
+BwdWorkspace bwd_workspace_layout(const AttnShape& s) {
+  BwdWorkspace L;
+  const int RC = s.b < 64 ? 1 : s.b / 64;
+  size_t off = 0;
+  L.off_D = off;
+  off = align256(off + sizeof(float) * (size_t)s.B * s.Hq * s.T);
+  L.off_da = off;
+  off = align256(off + sizeof(float) * (size_t)s.B * s.Hq * s.N * RC * (s.dense ? 0 : s.K));
+  L.off_csr_off = off;
+  off = align256(off + sizeof(int32_t) * (size_t)s.B * s.Hkv * (s.N + 1));
+  L.off_csr_list = off;
+  off = align256(off + sizeof(int32_t) * (size_t)s.B * s.Hkv * s.N * (s.dense ? 0 : s.K));
+  L.total = off;
+  return L;
+}
+
+cudaError_t launch_attn_fwd_simt(sas_dtype_t dt, const AttnShape& s, const void* q, const void* k,
+                                 const void* v, const int32_t* idx, const float* gates, void* o,
+                                 float* lse, const DevCtx& ctx, cudaStream_t st) {
+  if (dt == SAS_F32) return fwd_dispatch<float>(s, q, k, v, idx, gates, o, lse, ctx, st);
+  return fwd_dispatch<__nv_bfloat16>(s, q, k, v, idx, gates, o, lse, ctx, st);
+}
+
+cudaError_t launch_attn_bwd_simt(sas_dtype_t dt, const AttnShape& s, const void* q, const void* k,
+                                 const void* v, const void* o, const float* lse, const void* dO,
+                                 const int32_t* idx, const float* gates, void* dq, void* dk,
+                                 void* dv, float* dscores, void* ws, const DevCtx& ctx,
+                                 cudaStream_t st) {
+  if (dt == SAS_F32)
+    return bwd_dispatch<float>(s, q, k, v, o, lse, dO, idx, gates, dq, dk, dv, dscores, ws, ctx,
+                               st);
+  return bwd_dispatch<__nv_bfloat16>(s, q, k, v, o, lse, dO, idx, gates, dq, dk, dv, dscores, ws,
+                                     ctx, st);
+}
+
+}  // namespace sas

@@ -1,0 +1,351 @@
+// One-token decode over a KV cache: the selected history blocks plus the
+// current block (picx.dev SAS summary, Theoretical Foundation Eq. 2 with the
+// gates dropped, Methodology Eq. 9 with them; evolve.pub review, Summary:
+// hard selection kept at inference, gates dropped). Also the dense decode
+// used as the comparison (every block).
+//
+// The work is a stream over the selected K/V rows (G query heads share each
+// KV head), so it is bound by HBM bandwidth: per (batch, kv head) the
+// (K+1)*b*d*2 elements of K and V are read once, with 16-byte loads.
+//
+// Layout of the work: the block list of a (batch, kv head) is cut into
+// `splits` ranges of `bps` blocks, one CTA each. A CTA's four warps take
+// 16-token chunks of its range round-robin and keep an online softmax per
+// query head; the warps are merged in shared memory, and each CTA stores a
+// partial (max, sum, unnormalised o) to the workspace. The last CTA of a
+// (batch, kv head) to finish (counted with an atomic ticket) merges the
+// partials by log-sum-exp, writes o, and resets the ticket to zero.
+#include <math.h>
+
+#include "sas_common.cuh"
+#include "sas_internal.h"
+
+namespace sas {
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kChunk = 16;  // tokens per warp work item
+constexpr int kLPT = 8;     // lanes per token in the q.k phase
+constexpr int kMaxSplits = 256;
+
+template <typename T> struct Vec;
+// Loads `n` consecutive elements (n*sizeof(T) a multiple of 4 bytes) as floats.
+template <typename T, int n>
+__device__ __forceinline__ void load_f(const T* p, float (&out)[n]);
+
+template <>
+__device__ __forceinline__ void load_f<__nv_bfloat16, 16>(const __nv_bfloat16* p, float (&out)[16]) {
+  const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint4 b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    out[2 * i] = bf16lo(w[i]);
+    out[2 * i + 1] = bf16hi(w[i]);
+  }
+}
+template <>
+__device__ __forceinline__ void load_f<__nv_bfloat16, 8>(const __nv_bfloat16* p, float (&out)[8]) {
+  const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    out[2 * i] = bf16lo(w[i]);
+    out[2 * i + 1] = bf16hi(w[i]);
+  }
+}
+template <>
+__device__ __forceinline__ void load_f<__nv_bfloat16, 4>(const __nv_bfloat16* p, float (&out)[4]) {
+  const uint2 a = __ldg(reinterpret_cast<const uint2*>(p));
+  out[0] = bf16lo(a.x);
+  out[1] = bf16hi(a.x);
+  out[2] = bf16lo(a.y);
+  out[3] = bf16hi(a.y);
+}
+template <>
+__device__ __forceinline__ void load_f<__nv_bfloat16, 2>(const __nv_bfloat16* p, float (&out)[2]) {
+  const uint32_t a = __ldg(reinterpret_cast<const unsigned int*>(p));
+  out[0] = bf16lo(a);
+  out[1] = bf16hi(a);
+}
+template <int n>
+__device__ __forceinline__ void load_f_f32(const float* p, float (&out)[n]) {
+  static_assert(n % 2 == 0, "");
+  if constexpr (n % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < n / 4; ++i) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(p) + i);
+      out[4 * i] = a.x;
+      out[4 * i + 1] = a.y;
+      out[4 * i + 2] = a.z;
+      out[4 * i + 3] = a.w;
+    }
+  } else {
+    const float2 a = __ldg(reinterpret_cast<const float2*>(p));
+    out[0] = a.x;
+    out[1] = a.y;
+  }
+}
+template <> __device__ __forceinline__ void load_f<float, 16>(const float* p, float (&o)[16]) { load_f_f32<16>(p, o); }
+template <> __device__ __forceinline__ void load_f<float, 8>(const float* p, float (&o)[8]) { load_f_f32<8>(p, o); }
+template <> __device__ __forceinline__ void load_f<float, 4>(const float* p, float (&o)[4]) { load_f_f32<4>(p, o); }
+template <> __device__ __forceinline__ void load_f<float, 2>(const float* p, float (&o)[2]) { load_f_f32<2>(p, o); }
+
+// Block held by slot `sl` of a (batch, kv head): sparse -> idx entries then the
+// current block; dense -> blocks 0..C in order. Returns -1 for an empty slot.
+__device__ __forceinline__ int slot_block(const DecodeShape& s, const int32_t* ix, int sl,
+                                          const DevCtx& ctx) {
+  if (s.dense) return sl;
+  if (sl == s.K) return s.C;
+  const int m = ix[sl];
+  if (m < 0) return -1;
+  if (m >= s.C) {
+    report(ctx, kDevErrBadIndex);
+    return -1;
+  }
+  return m;
+}
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kThreads)
+decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
+              const int32_t* __restrict__ idx, const float* __restrict__ gates, DecodeShape s,
+              T* __restrict__ o, float* __restrict__ ws_ml, float* __restrict__ ws_o,
+              uint32_t* __restrict__ ws_cnt, DevCtx ctx) {
+  constexpr int VPL = D / kLPT;   // q.k dims per lane
+  constexpr int TPP = 32 / kLPT;  // tokens per pass
+  constexpr int DPL = D / 32;     // output dims per lane
+  __shared__ float s_x[kWarps][G][kChunk];
+  __shared__ float s_p[kWarps][kChunk][G];
+  __shared__ float s_m[kWarps][G], s_l[kWarps][G];
+  __shared__ float s_o[kWarps][G][D];
+  __shared__ int s_last;
+
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int split = blockIdx.x, kvh = blockIdx.y, bi = blockIdx.z;
+  const int unit = bi * s.Hkv + kvh;
+  const int nslots = s.dense ? s.C + 1 : s.K + 1;
+  const int sl0 = split * s.bps, sl1 = min(nslots, sl0 + s.bps);
+  const int cpb = s.b / kChunk;  // chunks per block
+  const long long cache0 = (long long)unit * s.Lcap * D;
+  const int32_t* ix = s.dense ? nullptr : idx + (long long)unit * s.K;
+
+  // q for this lane's q.k dims, all G heads.
+  float qr[G][VPL];
+  const int dseg = (lane % kLPT) * VPL;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const T* qp = q + ((long long)bi * s.Hq + kvh * G + g) * D + dseg;
+    load_f<T, VPL>(qp, qr[g]);
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) qr[g][i] *= s.scale;
+  }
+  float m_run[G], l_run[G], acc[G][DPL];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    m_run[g] = -INFINITY;
+    l_run[g] = 0.f;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) acc[g][i] = 0.f;
+  }
+
+  const int nchunks = (sl1 - sl0) * cpb;
+  for (int c = w; c < nchunks; c += kWarps) {
+    const int sl = sl0 + c / cpb;
+    const int m = slot_block(s, ix, sl, ctx);
+    if (m < 0) continue;
+    const float bias = (!s.dense && s.use_gates && sl < s.K)
+                           ? logf(gates[(long long)unit * s.C + m]) : 0.f;
+    const int t0 = m * s.b + (c % cpb) * kChunk;  // first token of the chunk
+    if (t0 >= s.L) continue;
+    const int nt = min(kChunk, s.L - t0);
+
+    // ---- logits: kLPT lanes per token, TPP tokens per pass
+#pragma unroll
+    for (int pass = 0; pass < kChunk / TPP; ++pass) {
+      const int tt = pass * TPP + lane / kLPT;
+      float dot[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) dot[g] = 0.f;
+      if (tt < nt) {
+        float kf[VPL];
+        load_f<T, VPL>(kc + cache0 + (long long)(t0 + tt) * D + dseg, kf);
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+          for (int i = 0; i < VPL; ++i) dot[g] = fmaf(qr[g][i], kf[i], dot[g]);
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+#pragma unroll
+        for (int off = kLPT / 2; off > 0; off >>= 1)
+          dot[g] += __shfl_xor_sync(0xffffffffu, dot[g], off);
+      }
+      if ((lane % kLPT) == 0) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) s_x[w][g][tt] = (tt < nt) ? dot[g] + bias : -INFINITY;
+      }
+    }
+    __syncwarp();
+    // ---- online softmax: lane t < kChunk owns token t
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float x = (lane < kChunk) ? s_x[w][g][lane] : -INFINITY;
+      const float mx = warp_max(x);
+      const float mnew = fmaxf(m_run[g], mx);
+      const float p = (mnew == -INFINITY) ? 0.f : expf(x - mnew);
+      const float alpha = (mnew == -INFINITY) ? 1.f : expf(m_run[g] - mnew);
+      l_run[g] = l_run[g] * alpha + warp_sum(p);
+      m_run[g] = mnew;
+      if (lane < kChunk) s_p[w][lane][g] = p;
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) acc[g][i] *= alpha;
+    }
+    __syncwarp();
+    // ---- o += p v: lane owns DPL consecutive dims
+    for (int t = 0; t < nt; ++t) {
+      float vf[DPL];
+      load_f<T, DPL>(vc + cache0 + (long long)(t0 + t) * D + lane * DPL, vf);
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float p = s_p[w][t][g];
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) acc[g][i] = fmaf(p, vf[i], acc[g][i]);
+      }
+    }
+    __syncwarp();
+  }
+
+  // ---- merge the warps of this CTA
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    if (lane == 0) {
+      s_m[w][g] = m_run[g];
+      s_l[w][g] = l_run[g];
+    }
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) s_o[w][g][lane * DPL + i] = acc[g][i];
+  }
+  __syncthreads();
+  const long long hbase = (long long)bi * s.Hq + kvh * G;  // first q head of the unit
+  for (int e = tid; e < G * D; e += kThreads) {
+    const int g = e / D, dd = e % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int x = 0; x < kWarps; ++x) M = fmaxf(M, s_m[x][g]);
+    float L = 0.f, A = 0.f;
+#pragma unroll
+    for (int x = 0; x < kWarps; ++x) {
+      const float f = (s_m[x][g] == -INFINITY) ? 0.f : expf(s_m[x][g] - M);
+      L += f * s_l[x][g];
+      A += f * s_o[x][g][dd];
+    }
+    if (s.splits == 1) {
+      st_f(o + (hbase + g) * D + dd, A / L);
+    } else {
+      const long long pidx = (hbase + g) * s.splits + split;
+      ws_o[pidx * D + dd] = A;
+      if (dd == 0) {
+        ws_ml[2 * pidx] = M;
+        ws_ml[2 * pidx + 1] = L;
+      }
+    }
+  }
+  if (s.splits == 1) return;
+
+  // ---- last CTA of the unit merges the partials
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const uint32_t ticket = atomicAdd(&ws_cnt[unit], 1u);
+    s_last = (ticket == (uint32_t)(s.splits - 1));
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int e = tid; e < G * D; e += kThreads) {
+    const int g = e / D, dd = e % D;
+    const long long p0 = (hbase + g) * s.splits;
+    float M = -INFINITY;
+    for (int x = 0; x < s.splits; ++x) M = fmaxf(M, __ldcg(&ws_ml[2 * (p0 + x)]));
+    float L = 0.f, A = 0.f;
+    for (int x = 0; x < s.splits; ++x) {
+      const float mx = __ldcg(&ws_ml[2 * (p0 + x)]);
+      const float f = (mx == -INFINITY) ? 0.f : expf(mx - M);
+      L += f * __ldcg(&ws_ml[2 * (p0 + x) + 1]);
+      A += f * __ldcg(&ws_o[(p0 + x) * D + dd]);
+    }
+    st_f(o + (hbase + g) * D + dd, A / L);
+  }
+  if (tid == 0) ws_cnt[unit] = 0u;
+}
+
+template <typename T, int D, int G>
+cudaError_t decode_t(const DecodeShape& s, const void* q, const void* kc, const void* vc,
+                     const int32_t* idx, const float* gates, void* o, void* ws, const DevCtx& ctx,
+                     cudaStream_t st) {
+  char* w = static_cast<char*>(ws);
+  const size_t parts = (size_t)s.B * s.Hq * s.splits;
+  float* ws_ml = reinterpret_cast<float*>(w);
+  float* ws_o = reinterpret_cast<float*>(w + ((2 * parts * sizeof(float) + 255) & ~(size_t)255));
+  uint32_t* ws_cnt = reinterpret_cast<uint32_t*>(
+      reinterpret_cast<char*>(ws_o) + ((parts * D * sizeof(float) + 255) & ~(size_t)255));
+  dim3 grid(s.splits, s.Hkv, s.B);
+  decode_kernel<T, D, G><<<grid, kThreads, 0, st>>>((const T*)q, (const T*)kc, (const T*)vc, idx,
+                                                    gates, s, (T*)o, ws_ml, ws_o, ws_cnt, ctx);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t decode_g(const DecodeShape& s, const void* q, const void* kc, const void* vc,
+                     const int32_t* idx, const float* gates, void* o, void* ws, const DevCtx& ctx,
+                     cudaStream_t st) {
+  switch (s.Hq / s.Hkv) {
+    case 1: return decode_t<T, D, 1>(s, q, kc, vc, idx, gates, o, ws, ctx, st);
+    case 2: return decode_t<T, D, 2>(s, q, kc, vc, idx, gates, o, ws, ctx, st);
+    case 3: return decode_t<T, D, 3>(s, q, kc, vc, idx, gates, o, ws, ctx, st);
+    case 4: return decode_t<T, D, 4>(s, q, kc, vc, idx, gates, o, ws, ctx, st);
+    case 5: return decode_t<T, D, 5>(s, q, kc, vc, idx, gates, o, ws, ctx, st);
+    case 6: return decode_t<T, D, 6>(s, q, kc, vc, idx, gates, o, ws, ctx, st);
+    case 7: return decode_t<T, D, 7>(s, q, kc, vc, idx, gates, o, ws, ctx, st);
+    case 8: return decode_t<T, D, 8>(s, q, kc, vc, idx, gates, o, ws, ctx, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+void decode_plan(DecodeShape& s) {
+  const int nslots = s.dense ? s.C + 1 : s.K + 1;
+  const int units = s.B * s.Hkv;
+  const int target = 148 * 4;
+  int splits = (target + units - 1) / units;
+  splits = max(1, min(splits, min(nslots, kMaxSplits)));
+  int bps = (nslots + splits - 1) / splits;
+  splits = (nslots + bps - 1) / bps;
+  s.splits = splits;
+  s.bps = bps;
+}
+
+size_t decode_workspace_bytes(const DecodeShape& s) {
+  const size_t parts = (size_t)s.B * s.Hq * s.splits;
+  const size_t a = (2 * parts * sizeof(float) + 255) & ~(size_t)255;
+  const size_t b = (parts * s.d * sizeof(float) + 255) & ~(size_t)255;
+  const size_t c = ((size_t)s.B * s.Hkv * sizeof(uint32_t) + 255) & ~(size_t)255;
+  return a + b + c;
+}
+
+cudaError_t launch_decode(sas_dtype_t dt, const DecodeShape& s, const void* q, const void* kc,
+                          const void* vc, const int32_t* idx, const float* gates, void* o,
+                          void* ws, const DevCtx& ctx, cudaStream_t st) {
+  if (dt == SAS_F32) {
+    if (s.d == 64) return decode_g<float, 64>(s, q, kc, vc, idx, gates, o, ws, ctx, st);
+    return decode_g<float, 128>(s, q, kc, vc, idx, gates, o, ws, ctx, st);
+  }
+  if (s.d == 64) return decode_g<__nv_bfloat16, 64>(s, q, kc, vc, idx, gates, o, ws, ctx, st);
+  return decode_g<__nv_bfloat16, 128>(s, q, kc, vc, idx, gates, o, ws, ctx, st);
+}
+
+}  // namespace sas

@@ -1,0 +1,344 @@
+// C ABI of the SAS library: argument validation on the host, dispatch to the
+// kernels, device-side error reporting. Every check here runs before any
+// launch, so a rejected call leaves the device untouched.
+#include <math.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "sas_common.cuh"
+#include "sas_internal.h"
+
+namespace sas {
+
+// Per-device error word (one instance per device that loads the library).
+static __device__ uint32_t g_dev_error;
+
+namespace {
+
+constexpr unsigned long long kDefaultWaitLimit = 1ull << 22;
+std::atomic<unsigned long long> g_wait_limit{kDefaultWaitLimit};
+std::atomic<unsigned long long> g_launches{0};
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+uint32_t* g_err_ptr[kMaxDevices] = {nullptr};
+
+// Device address of g_dev_error for the current device (looked up once per
+// device; in host code the symbol itself is only a host-side handle).
+cudaError_t device_ctx(DevCtx& ctx) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_dev_error);
+    if (e != cudaSuccess) return e;
+    g_err_ptr[dev] = static_cast<uint32_t*>(p);
+  }
+  ctx.err = g_err_ptr[dev];
+  ctx.wait_limit = g_wait_limit.load(std::memory_order_relaxed);
+  return cudaSuccess;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+sas_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? SAS_OK : SAS_ERR_CUDA; }
+
+float resolve_scale(float scale, int d) {
+  return scale > 0.f ? scale : 1.0f / sqrtf((float)d);
+}
+
+bool valid_dtype(sas_dtype_t dt) { return dt == SAS_F32 || dt == SAS_BF16; }
+
+// Shared checks of the attention calls (forward, backward, dense).
+sas_status_t check_attn(sas_dtype_t dt, int B, int Hq, int Hkv, int T, int d, int b, int K,
+                        bool dense, float scale) {
+  if (!valid_dtype(dt)) return SAS_ERR_INVALID_ARG;
+  if (B < 0 || Hq < 1 || Hkv < 1 || T < 1 || d < 1 || b < 1) return SAS_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return SAS_ERR_INVALID_ARG;
+  if (!dense && K < 1) return SAS_ERR_INVALID_ARG;
+  if (!isfinite(scale)) return SAS_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SAS_ERR_UNSUPPORTED;
+  if (b != 16 && b != 32 && b != 64) return SAS_ERR_UNSUPPORTED;
+  if (!dense && K > 256) return SAS_ERR_UNSUPPORTED;
+  if ((long long)B * Hq * T * d >= (1ll << 40)) return SAS_ERR_UNSUPPORTED;
+  const long long N = (T + (long long)b - 1) / b;
+  // N <= 16384 bounds the reverse-index kernel's shared memory (8 bytes per block).
+  if (N > 16384 || B > 65535 || Hq > 65535) return SAS_ERR_UNSUPPORTED;
+  return SAS_OK;
+}
+
+AttnShape make_shape(int B, int Hq, int Hkv, int T, int d, int b, int K, float scale, bool dense) {
+  AttnShape s;
+  s.B = B;
+  s.Hq = Hq;
+  s.Hkv = Hkv;
+  s.T = T;
+  s.d = d;
+  s.b = b;
+  s.N = (T + b - 1) / b;
+  s.K = dense ? 0 : K;
+  s.scale = resolve_scale(scale, d);
+  s.dense = dense;
+  return s;
+}
+
+sas_status_t check_decode(sas_dtype_t dt, int B, int Hq, int Hkv, int L, int Lcap, int d, int b,
+                          int K, bool dense, float scale) {
+  if (!valid_dtype(dt)) return SAS_ERR_INVALID_ARG;
+  if (B < 0 || Hq < 1 || Hkv < 1 || L < 1 || Lcap < L || d < 1 || b < 1)
+    return SAS_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return SAS_ERR_INVALID_ARG;
+  if (!dense && K < 1) return SAS_ERR_INVALID_ARG;
+  if (!isfinite(scale)) return SAS_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SAS_ERR_UNSUPPORTED;
+  if (b != 16 && b != 32 && b != 64) return SAS_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 8) return SAS_ERR_UNSUPPORTED;
+  if (!dense && K > 256) return SAS_ERR_UNSUPPORTED;
+  if (B > 65535 || Hkv > 65535) return SAS_ERR_UNSUPPORTED;
+  return SAS_OK;
+}
+
+DecodeShape make_decode(int B, int Hq, int Hkv, int L, int Lcap, int d, int b, int K, float scale,
+                        bool dense, int use_gates) {
+  DecodeShape s;
+  s.B = B;
+  s.Hq = Hq;
+  s.Hkv = Hkv;
+  s.L = L;
+  s.Lcap = Lcap;
+  s.d = d;
+  s.b = b;
+  s.K = dense ? 0 : K;
+  s.scale = resolve_scale(scale, d);
+  s.C = (L - 1) / b;
+  s.dense = dense;
+  s.use_gates = dense ? 0 : (use_gates != 0);
+  decode_plan(s);
+  return s;
+}
+
+__global__ void wait_selftest_kernel(DevCtx ctx) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) (void)mbar_wait(ctx, &bar, 0);  // nothing ever arrives
+}
+
+}  // namespace
+
+void note_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+
+cudaError_t launch_wait_selftest(const DevCtx& ctx, cudaStream_t stream) {
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(ctx);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace sas
+
+using namespace sas;
+
+extern "C" {
+
+const char* sas_status_string(sas_status_t s) {
+  switch (s) {
+    case SAS_OK: return "SAS_OK";
+    case SAS_ERR_INVALID_ARG: return "SAS_ERR_INVALID_ARG";
+    case SAS_ERR_UNSUPPORTED: return "SAS_ERR_UNSUPPORTED";
+    case SAS_ERR_CUDA: return "SAS_ERR_CUDA";
+    case SAS_ERR_TIMEOUT: return "SAS_ERR_TIMEOUT";
+    case SAS_ERR_WORKSPACE: return "SAS_ERR_WORKSPACE";
+    case SAS_ERR_DEVICE: return "SAS_ERR_DEVICE";
+  }
+  return "SAS_ERR_UNKNOWN";
+}
+
+int sas_version(void) { return 100; }
+
+uint64_t sas_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+void sas_set_wait_limit(uint64_t iterations) {
+  g_wait_limit.store(iterations ? iterations : kDefaultWaitLimit, std::memory_order_relaxed);
+}
+
+sas_status_t sas_get_device_error(sas_stream_t stream, uint32_t* raw) {
+  DevCtx ctx;
+  if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return SAS_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, ctx.err, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return SAS_ERR_CUDA;
+  const uint32_t zero = 0;
+  if (cudaMemcpy(ctx.err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+    return SAS_ERR_CUDA;
+  if (raw) *raw = v;
+  if (v & kDevErrTimeout) return SAS_ERR_TIMEOUT;
+  if (v) return SAS_ERR_DEVICE;
+  return SAS_OK;
+}
+
+sas_status_t sas_selftest_wait_timeout(sas_stream_t stream) {
+  DevCtx ctx;
+  if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
+  return cuda_status(launch_wait_selftest(ctx, stream));
+}
+
+sas_status_t sas_gate_topk(const float* scores, int B, int Hkv, int rows, int C, int causal,
+                           int K, float* gates, int32_t* idx, sas_stream_t stream) {
+  if (B < 0 || Hkv < 0 || rows < 0) return SAS_ERR_INVALID_ARG;
+  if (C < 1 || K < 1 || (causal != 0 && causal != 1)) return SAS_ERR_INVALID_ARG;
+  if (causal && rows != C) return SAS_ERR_INVALID_ARG;
+  if (C > 262144 || K > 256) return SAS_ERR_UNSUPPORTED;
+  if ((long long)B * Hkv * rows == 0) return SAS_OK;
+  if (!scores || !gates || !idx) return SAS_ERR_INVALID_ARG;
+  if (!aligned(scores, 4) || !aligned(gates, 4) || !aligned(idx, 4)) return SAS_ERR_INVALID_ARG;
+  if ((long long)B * Hkv * rows > (1ll << 31) - 1) return SAS_ERR_UNSUPPORTED;
+  return cuda_status(launch_gate_topk(scores, B, Hkv, rows, C, causal, K, gates, idx, stream));
+}
+
+sas_status_t sas_attn_fwd(sas_dtype_t dtype, const void* q, const void* k, const void* v,
+                          const int32_t* idx, const float* gates, int B, int Hq, int Hkv, int T,
+                          int d, int b, int K, float scale, void* o, float* lse,
+                          sas_stream_t stream) {
+  sas_status_t st = check_attn(dtype, B, Hq, Hkv, T, d, b, K, false, scale);
+  if (st != SAS_OK) return st;
+  if (B == 0) return SAS_OK;
+  if (!q || !k || !v || !idx || !o || !lse) return SAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4) || !aligned(idx, 4) || (gates && !aligned(gates, 4)))
+    return SAS_ERR_INVALID_ARG;
+  DevCtx ctx;
+  if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
+  const AttnShape s = make_shape(B, Hq, Hkv, T, d, b, K, scale, false);
+  return cuda_status(launch_attn_fwd_simt(dtype, s, q, k, v, idx, gates, o, lse, ctx, stream));
+}
+
+size_t sas_attn_bwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int b, int K) {
+  if (check_attn(SAS_BF16, B, Hq, Hkv, T, d, b, K, false, 1.f) != SAS_OK) return 0;
+  return bwd_workspace_layout(make_shape(B, Hq, Hkv, T, d, b, K, 1.f, false)).total;
+}
+
+sas_status_t sas_attn_bwd(sas_dtype_t dtype, const void* q, const void* k, const void* v,
+                          const void* o, const float* lse, const void* dO, const int32_t* idx,
+                          const float* gates, int B, int Hq, int Hkv, int T, int d, int b, int K,
+                          float scale, void* dq, void* dk, void* dv, float* dscores, void* ws,
+                          size_t ws_bytes, sas_stream_t stream) {
+  sas_status_t st = check_attn(dtype, B, Hq, Hkv, T, d, b, K, false, scale);
+  if (st != SAS_OK) return st;
+  if (B == 0) return SAS_OK;
+  if (!q || !k || !v || !o || !lse || !dO || !idx || !dq || !dk || !dv)
+    return SAS_ERR_INVALID_ARG;
+  if (!gates && dscores) return SAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(dO, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+      !aligned(lse, 4) || !aligned(idx, 4) || (gates && !aligned(gates, 4)) ||
+      (dscores && !aligned(dscores, 4)))
+    return SAS_ERR_INVALID_ARG;
+  const AttnShape s = make_shape(B, Hq, Hkv, T, d, b, K, scale, false);
+  const size_t need = bwd_workspace_layout(s).total;
+  if (!ws || ws_bytes < need || !aligned(ws, 256)) return SAS_ERR_WORKSPACE;
+  DevCtx ctx;
+  if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
+  return cuda_status(launch_attn_bwd_simt(dtype, s, q, k, v, o, lse, dO, idx, gates, dq, dk, dv,
+                                          dscores, ws, ctx, stream));
+}
+
+size_t sas_decode_workspace_size(int B, int Hq, int Hkv, int L, int d, int b, int K) {
+  if (check_decode(SAS_BF16, B, Hq, Hkv, L, L, d, b, K, false, 1.f) != SAS_OK) return 0;
+  return decode_workspace_bytes(make_decode(B, Hq, Hkv, L, L, d, b, K, 1.f, false, 0));
+}
+
+sas_status_t sas_decode(sas_dtype_t dtype, const void* q, const void* kcache, const void* vcache,
+                        const int32_t* idx, const float* gates, int use_gates, int B, int Hq,
+                        int Hkv, int L, int Lcap, int d, int b, int K, float scale, void* o,
+                        void* ws, size_t ws_bytes, sas_stream_t stream) {
+  sas_status_t st = check_decode(dtype, B, Hq, Hkv, L, Lcap, d, b, K, false, scale);
+  if (st != SAS_OK) return st;
+  if (B == 0) return SAS_OK;
+  if (!q || !kcache || !vcache || !idx || !o) return SAS_ERR_INVALID_ARG;
+  if (use_gates && !gates) return SAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(kcache, 16) || !aligned(vcache, 16) || !aligned(o, 16) ||
+      !aligned(idx, 4) || (gates && !aligned(gates, 4)))
+    return SAS_ERR_INVALID_ARG;
+  const DecodeShape s = make_decode(B, Hq, Hkv, L, Lcap, d, b, K, scale, false, use_gates);
+  if (s.splits > 1 && (!ws || ws_bytes < decode_workspace_bytes(s) || !aligned(ws, 256)))
+    return SAS_ERR_WORKSPACE;
+  DevCtx ctx;
+  if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
+  return cuda_status(launch_decode(dtype, s, q, kcache, vcache, idx, gates, o, ws, ctx, stream));
+}
+
+sas_status_t sas_dense_fwd(sas_dtype_t dtype, const void* q, const void* k, const void* v, int B,
+                           int Hq, int Hkv, int T, int d, int b, float scale, void* o, float* lse,
+                           sas_stream_t stream) {
+  sas_status_t st = check_attn(dtype, B, Hq, Hkv, T, d, b, 0, true, scale);
+  if (st != SAS_OK) return st;
+  if (B == 0) return SAS_OK;
+  if (!q || !k || !v || !o || !lse) return SAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return SAS_ERR_INVALID_ARG;
+  DevCtx ctx;
+  if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
+  const AttnShape s = make_shape(B, Hq, Hkv, T, d, b, 0, scale, true);
+  return cuda_status(launch_attn_fwd_simt(dtype, s, q, k, v, nullptr, nullptr, o, lse, ctx, stream));
+}
+
+size_t sas_dense_bwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int b) {
+  if (check_attn(SAS_BF16, B, Hq, Hkv, T, d, b, 0, true, 1.f) != SAS_OK) return 0;
+  return bwd_workspace_layout(make_shape(B, Hq, Hkv, T, d, b, 0, 1.f, true)).total;
+}
+
+sas_status_t sas_dense_bwd(sas_dtype_t dtype, const void* q, const void* k, const void* v,
+                           const void* o, const float* lse, const void* dO, int B, int Hq, int Hkv,
+                           int T, int d, int b, float scale, void* dq, void* dk, void* dv,
+                           void* ws, size_t ws_bytes, sas_stream_t stream) {
+  sas_status_t st = check_attn(dtype, B, Hq, Hkv, T, d, b, 0, true, scale);
+  if (st != SAS_OK) return st;
+  if (B == 0) return SAS_OK;
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return SAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(dO, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+      !aligned(lse, 4))
+    return SAS_ERR_INVALID_ARG;
+  const AttnShape s = make_shape(B, Hq, Hkv, T, d, b, 0, scale, true);
+  const size_t need = bwd_workspace_layout(s).total;
+  if (!ws || ws_bytes < need || !aligned(ws, 256)) return SAS_ERR_WORKSPACE;
+  DevCtx ctx;
+  if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
+  return cuda_status(launch_attn_bwd_simt(dtype, s, q, k, v, o, lse, dO, nullptr, nullptr, dq, dk,
+                                          dv, nullptr, ws, ctx, stream));
+}
+
+size_t sas_dense_decode_workspace_size(int B, int Hq, int Hkv, int L, int d) {
+  if (check_decode(SAS_BF16, B, Hq, Hkv, L, L, d, 64, 0, true, 1.f) != SAS_OK) return 0;
+  return decode_workspace_bytes(make_decode(B, Hq, Hkv, L, L, d, 64, 0, 1.f, true, 0));
+}
+
+sas_status_t sas_dense_decode(sas_dtype_t dtype, const void* q, const void* kcache,
+                              const void* vcache, int B, int Hq, int Hkv, int L, int Lcap, int d,
+                              float scale, void* o, void* ws, size_t ws_bytes,
+                              sas_stream_t stream) {
+  sas_status_t st = check_decode(dtype, B, Hq, Hkv, L, Lcap, d, 64, 0, true, scale);
+  if (st != SAS_OK) return st;
+  if (B == 0) return SAS_OK;
+  if (!q || !kcache || !vcache || !o) return SAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(kcache, 16) || !aligned(vcache, 16) || !aligned(o, 16))
+    return SAS_ERR_INVALID_ARG;
+  const DecodeShape s = make_decode(B, Hq, Hkv, L, Lcap, d, 64, 0, scale, true, 0);
+  if (s.splits > 1 && (!ws || ws_bytes < decode_workspace_bytes(s) || !aligned(ws, 256)))
+    return SAS_ERR_WORKSPACE;
+  DevCtx ctx;
+  if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
+  return cuda_status(
+      launch_decode(dtype, s, q, kcache, vcache, nullptr, nullptr, o, ws, ctx, stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,63 @@
+// Internal launchers of the SAS library. Each returns the CUDA error of its
+// launches (cudaSuccess when everything was enqueued). Arguments are already
+// validated by the C-ABI layer (sas_api.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/sas.h"
+
+namespace sas {
+
+struct DevCtx;
+
+// Adds n to the library's launch counter (sas_launch_count).
+void note_launches(int n);
+
+cudaError_t launch_gate_topk(const float* scores, int B, int Hkv, int rows, int C, int causal,
+                             int K, float* gates, int32_t* idx, cudaStream_t stream);
+
+// Problem description shared by the attention launchers.
+struct AttnShape {
+  int B, Hq, Hkv, T, d, b, K;
+  float scale;   // already resolved (> 0)
+  int N;         // ceil(T / b)
+  bool dense;    // every history block, no idx / gates
+};
+
+// Workspace carve-up of the backward pass (byte offsets, 256-aligned).
+struct BwdWorkspace {
+  size_t off_D, off_da, off_csr_off, off_csr_list, total;
+};
+BwdWorkspace bwd_workspace_layout(const AttnShape& s);
+
+cudaError_t launch_attn_fwd_simt(sas_dtype_t dt, const AttnShape& s, const void* q, const void* k,
+                                 const void* v, const int32_t* idx, const float* gates, void* o,
+                                 float* lse, const DevCtx& ctx, cudaStream_t stream);
+cudaError_t launch_attn_bwd_simt(sas_dtype_t dt, const AttnShape& s, const void* q, const void* k,
+                                 const void* v, const void* o, const float* lse, const void* dO,
+                                 const int32_t* idx, const float* gates, void* dq, void* dk,
+                                 void* dv, float* dscores, void* ws, const DevCtx& ctx,
+                                 cudaStream_t stream);
+
+// Decode (sparse and dense).
+struct DecodeShape {
+  int B, Hq, Hkv, L, Lcap, d, b, K;
+  float scale;
+  int C;        // (L - 1) / b history blocks
+  bool dense;   // all blocks 0..C, no idx / gates
+  int use_gates;
+  int splits;   // CTAs per (batch, kv head)
+  int bps;      // blocks per split
+};
+void decode_plan(DecodeShape& s);  // fills splits / bps
+size_t decode_workspace_bytes(const DecodeShape& s);
+cudaError_t launch_decode(sas_dtype_t dt, const DecodeShape& s, const void* q, const void* kc,
+                          const void* vc, const int32_t* idx, const float* gates, void* o,
+                          void* ws, const DevCtx& ctx, cudaStream_t stream);
+
+cudaError_t launch_wait_selftest(const DevCtx& ctx, cudaStream_t stream);
+
+}  // namespace sas

@@ -166,7 +166,7 @@ def make_train_inputs(cfg: TrainConfig, seed: int | None = None) -> TrainInputs:
     k = normal(s_k, (B, Hkv, T, d), bf16=False)
     v = normal(s_v, (B, Hkv, T, d), bf16=bf)
     dO = normal(s_do, (B, Hq, T, d), bf16=bf)
-    scores = normal(s_s, (B, Hkv, N, N), std=cfg.score_std)
+    scores = _train_scores(cfg, s_s)
     hot = []
     if cfg.hot_key_frac > 0:
         g = np.random.Generator(np.random.PCG64(s_hot))
@@ -179,13 +179,32 @@ def make_train_inputs(cfg: TrainConfig, seed: int | None = None) -> TrainInputs:
                     k[bi, h, m * b:min(T, (m + 1) * b)] *= np.float32(cfg.hot_key_scale)
     if bf:
         _round_bf16_inplace(k)
+    return TrainInputs(q, k, v, dO, scores, meta={"hot_blocks": hot, "seed": seed})
+
+
+def _train_scores(cfg: TrainConfig, s_s: np.random.SeedSequence) -> np.ndarray:
+    N = cfg.N
+    scores = normal(s_s, (cfg.B, cfg.Hkv, N, N), std=cfg.score_std)
     if cfg.recency:
         j = np.arange(N, dtype=np.float64)[:, None]
         m = np.arange(N, dtype=np.float64)[None, :]
         ramp = np.where(j >= 2, cfg.recency * m / np.maximum(j - 1, 1), 0.0)
         ramp = np.where(m < j, ramp, 0.0).astype(np.float32)
         scores += ramp[None, None]
-    return TrainInputs(q, k, v, dO, scores, meta={"hot_blocks": hot, "seed": seed})
+    return scores
+
+
+def make_train_scores(cfg: TrainConfig, seed: int | None = None) -> np.ndarray:
+    """Only the selector scores of make_train_inputs (the same values)."""
+    seed = cfg.seed if seed is None else seed
+    return _train_scores(cfg, np.random.SeedSequence(seed).spawn(6)[4])
+
+
+def make_decode_scores(cfg: DecodeConfig, seed: int | None = None) -> np.ndarray:
+    """Only the selector scores of make_decode_inputs (the same values)."""
+    seed = cfg.seed if seed is None else seed
+    return normal(np.random.SeedSequence(seed).spawn(4)[3], (cfg.B, cfg.Hkv, cfg.C),
+                  std=cfg.score_std)
 
 
 def make_decode_inputs(cfg: DecodeConfig, seed: int | None = None) -> DecodeInputs:

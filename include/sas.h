@@ -1,0 +1,221 @@
+/*
+ * sas.h - C ABI of a CUDA library (NVIDIA B200, sm_100a) for SAS gated
+ * block-sparse causal attention.
+ *
+ * Sources (by page and section; the pages print no code for this path):
+ *   [picx]   picx.dev summary of "SAS: Simple Attention Sparsification via
+ *            End-to-End Optimization of Context Ranking": Theoretical
+ *            Foundation (Eq. 1-3), Methodology (Eq. 4, Eq. 9), Gradient
+ *            Analysis (Eq. 5, Eq. 6), Kernel Design, Decode Efficiency (Fig. 7).
+ *   [readme] "SAS: End-to-end learning of sparse attention rankings from
+ *            language-model loss" (reproduction README): Core equations,
+ *            the only statement of the 1/sqrt(d) scale.
+ *   [review] evolve.pub review of the same paper: Summary (gates dropped at
+ *            inference, hard selection kept).
+ *
+ * Notation. B batch, Hq query heads, Hkv KV heads, G = Hq/Hkv query heads per
+ * KV head, T sequence length, d head dim, b block size (tokens per block),
+ * N = ceil(T/b) blocks, K history budget in blocks. Query block j has the
+ * history blocks 0..j-1; its "current block" is block j itself, always
+ * attended with a causal mask and gate g0 = 1 ([picx] Eq. 4). Block j selects
+ * n_j = min(K, j) history blocks.
+ *
+ * Conventions shared by every call:
+ *   - Every tensor argument is a DEVICE pointer owned by the caller, dense
+ *     row-major in the layout stated, 16-byte aligned. The library never
+ *     allocates memory the caller can see; scratch comes from the caller's
+ *     workspace (see the *_workspace_size calls).
+ *   - Every call is asynchronous on `stream` (NULL = the legacy default
+ *     stream) and returns after enqueueing its kernels.
+ *   - Argument errors are detected on the host before any launch and return
+ *     SAS_ERR_INVALID_ARG / SAS_ERR_UNSUPPORTED / SAS_ERR_WORKSPACE; nothing is
+ *     launched in that case. A failed launch returns SAS_ERR_CUDA. Errors
+ *     found on the device (a bounded wait that ran out, an index out of
+ *     range) set a per-device error word that sas_get_device_error reports;
+ *     the kernel that found them stops early and leaves its outputs undefined.
+ *   - dtype: q, k, v, o, dO, dq, dk, dv, kcache, vcache share one dtype
+ *     (SAS_F32 or SAS_BF16). scores, gates, lse, dscores are always fp32;
+ *     idx is int32. bf16 paths accumulate in fp32.
+ *   - scale <= 0 selects 1/sqrt(d) ([readme] Core equations). The scale
+ *     multiplies q.k only; log g is added unscaled.
+ *   - Limits: d in {64, 128}; b in {16, 32, 64}; 1 <= K <= 256;
+ *     Hq % Hkv == 0; G = Hq/Hkv <= 8 for decode; N <= 16384; T, L >= 1.
+ *     The entries of one idx
+ *     row must be distinct (sas_gate_topk writes them so).
+ */
+#ifndef SAS_H_
+#define SAS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* sas_stream_t; /* the same type as cudaStream_t */
+
+typedef enum {
+  SAS_F32 = 0,
+  SAS_BF16 = 1
+} sas_dtype_t;
+
+typedef enum {
+  SAS_OK = 0,
+  SAS_ERR_INVALID_ARG = 1, /* null pointer, negative or inconsistent size, misaligned pointer */
+  SAS_ERR_UNSUPPORTED = 2, /* well-formed but outside the limits above */
+  SAS_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+  SAS_ERR_TIMEOUT = 4,     /* (device) a bounded wait ran out of iterations */
+  SAS_ERR_WORKSPACE = 5,   /* workspace missing, too small or misaligned */
+  SAS_ERR_DEVICE = 6       /* (device) a device-side check failed, e.g. idx out of range */
+} sas_status_t;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* sas_status_string(sas_status_t status);
+
+/* Library version as an integer MAJOR*10000 + MINOR*100 + PATCH. */
+int sas_version(void);
+
+/* Number of kernels this process has launched through the library so far
+ * (all devices, all threads). Lets a caller count the launches of a region. */
+uint64_t sas_launch_count(void);
+
+/*
+ * sas_gate_topk - history gates and Top-K block selection.
+ *   [picx] Eq. 4 with phi = softmax and Eq. 6: log g_m = s_m - LSE(s) over the
+ *   valid history entries of a row, g_m = exp(log g_m) (so they sum to 1);
+ *   [picx] Eq. 3 / [readme] Core equations: I = Top-K(s, K).
+ *
+ *   scores [B, Hkv, rows, C] fp32 (device, read). Must be finite.
+ *   causal = 1 (training): rows == C == N and row j has j valid entries
+ *            (the history of query block j; entries m >= j are ignored).
+ *   causal = 0 (decode):   every row has C valid entries.
+ *   gates  [B, Hkv, rows, C] fp32 (device, written): g_m for valid m, 0 past
+ *            the valid length (row 0 of a causal call is all zero).
+ *   idx    [B, Hkv, rows, K] int32 (device, written): the min(K, valid)
+ *            largest scores' block indices in rank order (descending score,
+ *            equal scores ordered by lower index; -0.0 equals +0.0), padded
+ *            with -1.
+ *   Limits: 1 <= C <= 262144, 1 <= K <= 256.
+ */
+sas_status_t sas_gate_topk(const float* scores, int B, int Hkv, int rows, int C, int causal,
+                           int K, float* gates, int32_t* idx, sas_stream_t stream);
+
+/*
+ * sas_attn_fwd - gated block-sparse causal attention, forward.
+ *   [picx] Eq. 9 with the [readme] scale: for query row i of block j,
+ *   o_i = softmax(q_i K_S^T * scale + log g_S) V_S over the keys of the
+ *   selected blocks S = idx[.., j, :] (bias log g_m) and the keys t <= i of
+ *   block j (bias 0). With gates == NULL the bias of selected blocks is 0
+ *   ([picx] Eq. 2, gates dropped).
+ *
+ *   q [B, Hq, T, d]; k, v [B, Hkv, T, d] (dtype; read).
+ *   idx [B, Hkv, N, K] int32: entries -1 are skipped; every other entry of
+ *     row j must satisfy 0 <= m < j (checked on the device: SAS_ERR_DEVICE).
+ *   gates [B, Hkv, N, N] fp32 or NULL: row j holds g_{j,m} (as written by
+ *     sas_gate_topk with causal = 1). A zero gate masks its block.
+ *   o [B, Hq, T, d] (dtype; written); lse [B, Hq, T] fp32 (written): the
+ *     natural-log normaliser of each row's softmax, needed by the backward.
+ */
+sas_status_t sas_attn_fwd(sas_dtype_t dtype, const void* q, const void* k, const void* v,
+                          const int32_t* idx, const float* gates, int B, int Hq, int Hkv, int T,
+                          int d, int b, int K, float scale, void* o, float* lse,
+                          sas_stream_t stream);
+
+/*
+ * sas_attn_bwd - backward of sas_attn_fwd for L = any loss with dL/do = dO.
+ *   Recomputes the probabilities from lse and returns
+ *     dq [B, Hq, T, d], dk, dv [B, Hkv, T, d]   (dtype; written);
+ *     dscores [B, Hkv, N, N] fp32 (written; may be NULL): the gradient into
+ *       the selector scores through the gate softmax. With da_{j,m} = the sum
+ *       of dL/dlogit over the tile (all G heads, rows of block j, keys of
+ *       block m) -- equal to g_m * dg_m of [picx] Eq. 5, inner form -- and the
+ *       Jacobian of [picx] Eq. 6 (d log g_m / d s_k = delta_mk - g_k):
+ *         dscores[j, k] = [k in I_j] da_{j,k} - g_{j,k} * sum_{m in I_j} da_{j,m}
+ *       for k < j, and 0 for k >= j. No gradient flows through idx.
+ *   q, k, v, idx, gates, scale as passed to sas_attn_fwd; o, lse its outputs;
+ *   dO [B, Hq, T, d] (dtype). gates == NULL requires dscores == NULL.
+ *   ws / ws_bytes: caller workspace of at least sas_attn_bwd_workspace_size()
+ *   bytes, 256-byte aligned; its contents on entry do not matter.
+ */
+size_t sas_attn_bwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int b, int K);
+sas_status_t sas_attn_bwd(sas_dtype_t dtype, const void* q, const void* k, const void* v,
+                          const void* o, const float* lse, const void* dO, const int32_t* idx,
+                          const float* gates, int B, int Hq, int Hkv, int T, int d, int b, int K,
+                          float scale, void* dq, void* dk, void* dv, float* dscores, void* ws,
+                          size_t ws_bytes, sas_stream_t stream);
+
+/*
+ * sas_decode - one query token per sequence over a KV cache, selected blocks
+ * plus the current block ([picx] Eq. 2 with use_gates = 0, Eq. 9 with
+ * use_gates = 1; [review] Summary: gates are dropped at inference while the
+ * hard selection stays).
+ *   The query of sequence bi sits at position L-1 and its key is already in
+ *   the cache. The current block cb = floor((L-1)/b) covers positions
+ *   cb*b .. L-1 (all visible, bias 0); the C = cb blocks before it are the
+ *   history that idx selects from.
+ *   q [B, Hq, d] (dtype). kcache, vcache [B, Hkv, Lcap, d] (dtype), positions
+ *     0..L-1 valid, L <= Lcap.
+ *   idx [B, Hkv, K] int32 over 0..C-1, -1 skipped (as written by
+ *     sas_gate_topk with causal = 0, rows = 1).
+ *   gates [B, Hkv, C] fp32; read only when use_gates != 0 (may be NULL otherwise).
+ *   o [B, Hq, d] (dtype; written).
+ *   ws / ws_bytes: at least sas_decode_workspace_size() bytes, 256-byte
+ *   aligned. The workspace must be ZERO-FILLED before its first use; every
+ *   call leaves it zero-filled again, so it can be reused without clearing.
+ *   Calls that share a workspace must not overlap on the device.
+ */
+size_t sas_decode_workspace_size(int B, int Hq, int Hkv, int L, int d, int b, int K);
+sas_status_t sas_decode(sas_dtype_t dtype, const void* q, const void* kcache, const void* vcache,
+                        const int32_t* idx, const float* gates, int use_gates, int B, int Hq,
+                        int Hkv, int L, int Lcap, int d, int b, int K, float scale, void* o,
+                        void* ws, size_t ws_bytes, sas_stream_t stream);
+
+/*
+ * Dense comparison kernels ([picx] Eq. 1 with a causal mask): every block is
+ * attended, no gates. Same layouts and conventions as the sparse calls; the
+ * block size b only sets the kernels' tiling (use 64 unless d or T call for
+ * less) and does not change the result.
+ */
+sas_status_t sas_dense_fwd(sas_dtype_t dtype, const void* q, const void* k, const void* v, int B,
+                           int Hq, int Hkv, int T, int d, int b, float scale, void* o, float* lse,
+                           sas_stream_t stream);
+size_t sas_dense_bwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int b);
+sas_status_t sas_dense_bwd(sas_dtype_t dtype, const void* q, const void* k, const void* v,
+                           const void* o, const float* lse, const void* dO, int B, int Hq, int Hkv,
+                           int T, int d, int b, float scale, void* dq, void* dk, void* dv,
+                           void* ws, size_t ws_bytes, sas_stream_t stream);
+size_t sas_dense_decode_workspace_size(int B, int Hq, int Hkv, int L, int d);
+sas_status_t sas_dense_decode(sas_dtype_t dtype, const void* q, const void* kcache,
+                              const void* vcache, int B, int Hq, int Hkv, int L, int Lcap, int d,
+                              float scale, void* o, void* ws, size_t ws_bytes,
+                              sas_stream_t stream);
+
+/*
+ * Device-side error reporting. sas_get_device_error synchronises `stream`,
+ * reads the current device's error word, clears it and returns SAS_OK,
+ * SAS_ERR_TIMEOUT or SAS_ERR_DEVICE (SAS_ERR_CUDA if the read itself fails).
+ * *raw (may be NULL) receives the raw bit mask.
+ */
+sas_status_t sas_get_device_error(sas_stream_t stream, uint32_t* raw);
+
+/*
+ * Iteration limit of every bounded device wait (mbarrier and flag spins);
+ * 0 restores the default (about a second of spinning). Applies to calls
+ * enqueued afterwards from any thread.
+ */
+void sas_set_wait_limit(uint64_t iterations);
+
+/*
+ * Failure-detection self test: launches one kernel that waits, with the
+ * current wait limit, on a barrier that nothing ever completes; the wait
+ * runs out, the kernel records SAS_ERR_TIMEOUT in the error word and
+ * returns. Nothing hangs or faults. Use with a small limit.
+ */
+sas_status_t sas_selftest_wait_timeout(sas_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SAS_H_ */

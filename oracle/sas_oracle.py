@@ -395,11 +395,14 @@ def dense_decode(q, kcache, vcache, scale=0.0):
     scale = _default_scale(d, scale)
     o = np.empty((B, Hq, d))
     for bi in range(B):
-        for h in range(Hq):
-            Kc = _f64(kc[bi, h // G])
-            x = scale * (Kc @ _f64(q[bi, h]))
-            p = np.exp(x - x.max())
-            o[bi, h] = (p @ _f64(vc[bi, h // G])) / p.sum()
+        for kvh in range(kc.shape[1]):
+            Kc = _f64(kc[bi, kvh])
+            Vc = _f64(vc[bi, kvh])
+            for g in range(G):
+                h = kvh * G + g
+                x = scale * (Kc @ _f64(q[bi, h]))
+                p = np.exp(x - x.max())
+                o[bi, h] = (p @ Vc) / p.sum()
     return o
 
 

@@ -1,0 +1,99 @@
+"""Shared helpers of the GPU parity tests: tolerances and oracle sampling.
+
+Tolerances (stated by the workload definitions, read as follows):
+  * fp32 tensors of an fp32 workload: max|x - y| / max|y| <= 1e-4 (normwise).
+  * tensors of a bf16 workload: every element |x - y| <= 2e-2 + 2^-8 |y|
+    (the absolute bound on top of half an ulp of the stored bf16 value,
+    which alone exceeds 2e-2 once |y| >= 8), and ||x - y||_2 / ||y||_2 <= 1e-2.
+  * indices: bit-exact.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from oracle import sas_oracle as O
+
+BF16_ATOL = 2e-2
+BF16_RTOL_ULP = 2.0 ** -8
+BF16_REL_L2 = 1e-2
+F32_NORMWISE = 1e-4
+
+
+def dev(a: np.ndarray, dtype: str, device="cuda") -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if dtype == "bf16" and t.dtype == torch.float32:
+        t = t.to(torch.bfloat16)
+    return t.to(device)
+
+
+def host(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def check(name: str, got, want, dtype: str):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    assert got.shape == want.shape, (name, got.shape, want.shape)
+    assert np.isfinite(got).all(), f"{name}: non-finite values"
+    err = np.abs(got - want)
+    scale = np.abs(want).max() if want.size else 0.0
+    if dtype == "f32":
+        rel = err.max() / max(scale, 1e-30) if want.size else 0.0
+        assert rel <= F32_NORMWISE, f"{name}: normwise rel err {rel:.3e} > {F32_NORMWISE}"
+        return rel
+    excess = (err - BF16_RTOL_ULP * np.abs(want)).max() if want.size else 0.0
+    l2 = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
+    assert excess <= BF16_ATOL, f"{name}: max abs err beyond bf16 rounding {excess:.3e} > {BF16_ATOL}"
+    assert l2 <= BF16_REL_L2, f"{name}: rel L2 err {l2:.3e} > {BF16_REL_L2}"
+    return l2
+
+
+def oracle_gates_slice(scores, bi, kvh, K, causal=True):
+    """Oracle gates / log-gates / idx for one (batch, kv head)."""
+    g, lg, ix = O.gate_topk(scores[bi:bi + 1, kvh:kvh + 1], K, causal=causal)
+    return g[0, 0], lg[0, 0], ix[0, 0]
+
+
+def oracle_fwd_rows(x, b, K, bi, kvh, j, use_gates=True, cache=None):
+    """Oracle o [G, rows, d] and lse [G, rows] for query block j of (bi, kvh)."""
+    g, lg, ix = cache if cache is not None else oracle_gates_slice(x.scores, bi, kvh, K)
+    idx = np.zeros((bi + 1, kvh + 1) + ix.shape, np.int32)
+    idx[bi, kvh] = ix
+    logg = np.zeros((bi + 1, kvh + 1) + lg.shape)
+    logg[bi, kvh] = lg
+    return O.attn_fwd_block(x.q, x.k, x.v, idx, logg, bi, kvh, j, b, use_gates=use_gates)
+
+
+def oracle_bwd_sample(x, b, K, bi, kvh, js, ms, use_gates=True, cache=None):
+    """Oracle gradients for sampled query blocks js (dq rows, dscores rows) and
+    sampled key blocks ms (dk, dv rows; summed over every query block whose
+    key set contains block m)."""
+    g, lg, ix = cache if cache is not None else oracle_gates_slice(x.scores, bi, kvh, K)
+    idx = np.zeros((bi + 1, kvh + 1) + ix.shape, np.int32)
+    idx[bi, kvh] = ix
+    logg = np.zeros((bi + 1, kvh + 1) + lg.shape)
+    logg[bi, kvh] = lg
+    T = x.q.shape[2]
+    N = ix.shape[0]
+    out = {"dq": {}, "ds": {}, "dk": {}, "dv": {}}
+    for j in js:
+        r = O.attn_bwd_block(x.q, x.k, x.v, x.dO, idx, logg, bi, kvh, j, b, use_gates=use_gates)
+        out["dq"][j] = r["dq"]
+        if use_gates:
+            out["ds"][j] = np.concatenate([O.dscores_row(r["da"], g[j], j), np.zeros(N - j)])
+    for m in ms:
+        rows = min(T, (m + 1) * b) - m * b
+        dk = np.zeros((rows, x.q.shape[3]))
+        dv = np.zeros_like(dk)
+        for j in range(m, N):
+            if j != m and m not in set(int(t) for t in ix[j]):
+                continue
+            r = O.attn_bwd_block(x.q, x.k, x.v, x.dO, idx, logg, bi, kvh, j, b,
+                                 use_gates=use_gates)
+            sel = (r["cols"] >= m * b) & (r["cols"] < m * b + rows)
+            dk += r["dk_c"][sel]
+            dv += r["dv_c"][sel]
+        out["dk"][m] = dk
+        out["dv"][m] = dv
+    return out

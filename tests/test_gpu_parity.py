@@ -1,0 +1,222 @@
+"""GPU parity: every call of the C-ABI library against the float64 oracle on
+the same seeded inputs.
+
+Small cases compare every element and span several tiles and a ragged tail;
+the full-size training layers compare sampled query blocks and key blocks
+(the oracle computes those one by one); decode compares every output.
+"""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_sas_b200 import workloads as W
+from oracle import sas_oracle as O
+from tests.parity_util import check, dev, host, oracle_bwd_sample, oracle_fwd_rows, \
+    oracle_gates_slice
+
+pytestmark = pytest.mark.gpu
+
+
+# --------------------------------------------------------------------- gates
+
+def _gate_case(lib, scores, K, causal):
+    g, ix = lib.gate_topk(dev(scores, "f32"), K, causal=causal)
+    og, _, oi = O.gate_topk(scores, K, causal=causal)
+    np.testing.assert_array_equal(ix.cpu().numpy(), oi)
+    check("gates", host(g), og, "f32")
+
+
+@pytest.mark.parametrize("name", ["tiny", "qwen3-4b-train", "qwen3-8b-train"])
+def test_gate_topk_training_configs(cuda_lib, name):
+    cfg = W.PRESETS[name]
+    _gate_case(cuda_lib, W.make_train_scores(cfg), cfg.K, True)
+
+
+@pytest.mark.parametrize("name", ["qwen3-4b-decode", "qwen3-14b-decode"])
+def test_gate_topk_decode_configs(cuda_lib, name):
+    cfg = W.PRESETS[name]
+    _gate_case(cuda_lib, W.make_decode_scores(cfg)[:, :, None, :], cfg.K, False)
+
+
+@pytest.mark.parametrize("C,K,causal,levels", [
+    (16, 4, True, 0), (64, 64, True, 0), (200, 5, True, 2), (33, 1, True, 1),
+    (1500, 16, True, 0), (5000, 64, False, 0), (70000, 256, False, 0), (3000, 100, False, 3),
+    (1, 3, False, 0), (40, 256, False, 0),
+])
+def test_gate_topk_edges(cuda_lib, C, K, causal, levels):
+    rng = np.random.default_rng(C * 7 + K)
+    rows = C if causal else 3
+    s = rng.standard_normal((2, 1, rows, C)).astype(np.float32) * 2
+    if levels:
+        s = rng.integers(0, levels, s.shape).astype(np.float32)
+        s[s == 0] = -0.0 if levels > 1 else 0.0  # -0.0 must tie with +0.0
+        if levels > 1:
+            s[..., ::7] = 0.0
+    _gate_case(cuda_lib, s, K, causal)
+
+
+# ------------------------------------------------------------- fwd + bwd
+
+def _run_train(lib, x, cfg, use_gates=True):
+    dt = cfg.dtype
+    q, k, v, dO = (dev(a, dt) for a in (x.q, x.k, x.v, x.dO))
+    gates, idx = lib.gate_topk(dev(x.scores, "f32"), cfg.K, causal=True)
+    gg = gates if use_gates else None
+    o, lse = lib.attn_fwd(q, k, v, idx, gg, cfg.b)
+    dq, dk, dv, ds = lib.attn_bwd(q, k, v, o, lse, dO, idx, gg, cfg.b)
+    torch.cuda.synchronize()
+    st, raw = lib.device_error()
+    assert st == 0, f"device error bits {raw:#x}"
+    return dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv, ds=ds, idx=idx, gates=gates)
+
+
+def _full_compare(lib, cfg, use_gates=True):
+    x = W.make_train_inputs(cfg)
+    r = _run_train(lib, x, cfg, use_gates)
+    g, lg, ix = O.gate_topk(x.scores, cfg.K)
+    np.testing.assert_array_equal(r["idx"].cpu().numpy(), ix)
+    o, lse = O.attn_fwd(x.q, x.k, x.v, ix, lg, cfg.b, use_gates=use_gates)
+    dq, dk, dv, ds = O.attn_bwd(x.q, x.k, x.v, x.dO, ix, g, lg, cfg.b, use_gates=use_gates)
+    dt = cfg.dtype
+    check("o", host(r["o"]), o, dt)
+    check("lse", host(r["lse"]), lse, dt)
+    check("dq", host(r["dq"]), dq, dt)
+    check("dk", host(r["dk"]), dk, dt)
+    check("dv", host(r["dv"]), dv, dt)
+    if use_gates:
+        check("dscores", host(r["ds"]), ds, dt)
+    else:
+        assert r["ds"] is None
+
+
+def test_tiny_f32_config_full(cuda_lib):
+    _full_compare(cuda_lib, W.TINY_F32)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(B=1, Hq=4, Hkv=2, T=200, d=64, b=16, K=3, dtype="f32"),
+    dict(B=2, Hq=2, Hkv=1, T=130, d=128, b=32, K=2, dtype="f32"),
+    dict(B=1, Hq=8, Hkv=2, T=1000, d=128, b=64, K=3, dtype="bf16", hot_key_frac=0.1,
+         hot_key_scale=3.0),
+    dict(B=2, Hq=4, Hkv=1, T=512, d=128, b=64, K=16, dtype="bf16"),
+    dict(B=1, Hq=5, Hkv=1, T=320, d=64, b=64, K=2, dtype="bf16"),
+    dict(B=1, Hq=3, Hkv=3, T=64, d=128, b=64, K=4, dtype="bf16"),   # single block, j = 0 only
+    dict(B=1, Hq=2, Hkv=1, T=77, d=64, b=16, K=1, dtype="f32"),
+])
+@pytest.mark.parametrize("use_gates", [True, False])
+def test_train_small_full(cuda_lib, kw, use_gates):
+    _full_compare(cuda_lib, W.small_train_config(**kw), use_gates)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["qwen3-4b-train", "qwen3-8b-train"])
+def test_train_full_size_sampled(cuda_lib, name):
+    cfg = W.PRESETS[name]
+    x = W.make_train_inputs(cfg)
+    r = _run_train(cuda_lib, x, cfg)
+    N, G, b = cfg.N, cfg.G, cfg.b
+    js = [0, 1, 2, cfg.K - 1, cfg.K, cfg.K + 1, N // 2, N - 2, N - 1]
+    ms = [0, 1, N // 3, N - 2, N - 1]
+    for bi, kvh in ((0, 0), (cfg.B - 1, cfg.Hkv - 1)):
+        cache = oracle_gates_slice(x.scores, bi, kvh, cfg.K)
+        np.testing.assert_array_equal(r["idx"][bi, kvh].cpu().numpy(), cache[2])
+        check("gates", host(r["gates"][bi, kvh]), cache[0], "f32")
+        for j in js:
+            o, lse = oracle_fwd_rows(x, b, cfg.K, bi, kvh, j, cache=cache)
+            sl = slice(j * b, (j + 1) * b)
+            check(f"o[{j}]", host(r["o"][bi, kvh * G:(kvh + 1) * G, sl]), o, cfg.dtype)
+            check(f"lse[{j}]", host(r["lse"][bi, kvh * G:(kvh + 1) * G, sl]), lse, cfg.dtype)
+        ob = oracle_bwd_sample(x, b, cfg.K, bi, kvh, js, ms, cache=cache)
+        for j in js:
+            sl = slice(j * b, (j + 1) * b)
+            check(f"dq[{j}]", host(r["dq"][bi, kvh * G:(kvh + 1) * G, sl]), ob["dq"][j], cfg.dtype)
+            check(f"ds[{j}]", host(r["ds"][bi, kvh, j]), ob["ds"][j], cfg.dtype)
+        for m in ms:
+            sl = slice(m * b, (m + 1) * b)
+            check(f"dk[{m}]", host(r["dk"][bi, kvh, sl]), ob["dk"][m], cfg.dtype)
+            check(f"dv[{m}]", host(r["dv"][bi, kvh, sl]), ob["dv"][m], cfg.dtype)
+
+
+def test_dense_matches_all_blocks_selected(cuda_lib):
+    cfg = W.small_train_config(B=1, Hq=4, Hkv=2, T=300, d=128, b=64, K=8, dtype="bf16")
+    x = W.make_train_inputs(cfg)
+    q, k, v, dO = (dev(a, "bf16") for a in (x.q, x.k, x.v, x.dO))
+    o, lse = cuda_lib.dense_fwd(q, k, v, b=64)
+    dq, dk, dv = cuda_lib.dense_bwd(q, k, v, o, lse, dO, b=64)
+    oo, ol = O.dense_fwd(x.q, x.k, x.v, 64)
+    idx = O.all_blocks_idx(1, 2, cfg.N)
+    odq, odk, odv, _ = O.attn_bwd(x.q, x.k, x.v, x.dO, idx, None, None, 64, use_gates=False)
+    check("dense o", host(o), oo, "bf16")
+    check("dense lse", host(lse), ol, "bf16")
+    check("dense dq", host(dq), odq, "bf16")
+    check("dense dk", host(dk), odk, "bf16")
+    check("dense dv", host(dv), odv, "bf16")
+
+
+# ------------------------------------------------------------------ decode
+
+def _decode_case(lib, dc, use_gates, dense_too=False):
+    x = W.make_decode_inputs(dc)
+    s = x.scores[:, :, None, :]
+    gates, idx = lib.gate_topk(dev(s, "f32"), dc.K, causal=False)
+    og, olg, oi = O.gate_topk(s, dc.K, causal=False)
+    np.testing.assert_array_equal(idx.cpu().numpy(), oi)
+    q, kc, vc = (dev(a, dc.dtype) for a in (x.q, x.kcache, x.vcache))
+    o = lib.decode(q, kc, vc, idx[:, :, 0].contiguous(), gates[:, :, 0].contiguous(), use_gates,
+                   dc.b, L=dc.L)
+    torch.cuda.synchronize()
+    assert lib.device_error()[0] == 0
+    want = O.decode(x.q, x.kcache, x.vcache, oi[:, :, 0], olg[:, :, 0], dc.b, use_gates=use_gates)
+    check("decode o", host(o), want, dc.dtype)
+    if dense_too:
+        od = lib.dense_decode(q, kc, vc, L=dc.L)
+        torch.cuda.synchronize()
+        check("dense decode o", host(od), O.dense_decode(x.q, x.kcache, x.vcache), dc.dtype)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(B=2, Hq=4, Hkv=2, L=1000, d=128, b=64, K=4, dtype="f32"),
+    dict(B=3, Hq=5, Hkv=1, L=777, d=64, b=16, K=9, dtype="bf16"),
+    dict(B=1, Hq=8, Hkv=1, L=64, d=128, b=64, K=2, dtype="bf16"),     # no history
+    dict(B=1, Hq=2, Hkv=2, L=65, d=128, b=64, K=2, dtype="bf16"),     # 1 token current block
+    dict(B=2, Hq=12, Hkv=4, L=4099, d=128, b=32, K=200, dtype="bf16"),
+    dict(B=1, Hq=1, Hkv=1, L=50000, d=64, b=64, K=7, dtype="f32"),
+])
+@pytest.mark.parametrize("use_gates", [False, True])
+def test_decode_small(cuda_lib, kw, use_gates):
+    _decode_case(cuda_lib, W.small_decode_config(**kw), use_gates, dense_too=True)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,use_gates", [("qwen3-4b-decode", 0), ("qwen3-4b-decode", 1),
+                                            ("qwen3-14b-decode", 0)])
+def test_decode_full_size(cuda_lib, name, use_gates):
+    _decode_case(cuda_lib, W.PRESETS[name], bool(use_gates), dense_too=(use_gates == 0))
+
+
+# ------------------------------------------------------------ device errors
+
+def test_bad_index_is_reported_not_faulted(cuda_lib):
+    cfg = W.small_train_config(B=1, Hq=2, Hkv=1, T=128, d=64, b=32, K=2, dtype="f32")
+    x = W.make_train_inputs(cfg)
+    q, k, v = (dev(a, "f32") for a in (x.q, x.k, x.v))
+    idx = torch.full((1, 1, cfg.N, 2), -1, dtype=torch.int32, device="cuda")
+    idx[0, 0, 1, 0] = 3   # block 3 is not in the history of block 1
+    cuda_lib.device_error()
+    cuda_lib.attn_fwd(q, k, v, idx, None, cfg.b)
+    st, raw = cuda_lib.device_error()
+    assert st == 6 and raw & 2
+
+
+def test_wait_timeout_is_reported(cuda_lib):
+    cuda_lib.device_error()
+    cuda_lib.set_wait_limit(2000)
+    try:
+        cuda_lib.selftest_wait_timeout()
+        st, raw = cuda_lib.device_error()
+    finally:
+        cuda_lib.set_wait_limit(0)
+    assert st == 4 and raw & 1
+    # the context stays usable
+    x = torch.ones(4, device="cuda")
+    assert float((x * 2).sum()) == 8.0
