@@ -103,8 +103,7 @@ _WS: dict = {}
 
 
 def _workspace(kind: str, nbytes: int, device, zero: bool) -> torch.Tensor:
-    """Cached device workspace (grows on demand). Decode workspaces start
-    zero-filled and the library leaves them zero-filled after every call."""
+    """Cached device workspace (grows on demand; contents never matter)."""
     key = (kind, device.index if device.index is not None else torch.cuda.current_device())
     buf = _WS.get(key)
     if buf is None or buf.numel() < nbytes:
@@ -185,7 +184,7 @@ def decode(q, kcache, vcache, idx, gates, use_gates: bool, b: int, L: int | None
     if o is None:
         o = torch.empty_like(q)
     nbytes = LIB.sas_decode_workspace_size(B, Hq, Hkv, L, d, b, K)
-    ws = _workspace("decode", nbytes, q.device, zero=True)
+    ws = _workspace("decode", nbytes, q.device, zero=False)
     _check("sas_decode", LIB.sas_decode(_dtype(q), _ptr(q), _ptr(kcache), _ptr(vcache), _ptr(idx),
                                         _ptr(gates), int(use_gates), B, Hq, Hkv, L, Lcap, d, b, K,
                                         scale, _ptr(o), _ptr(ws), ws.numel(), _stream(q.device)))
@@ -221,7 +220,7 @@ def dense_decode(q, kcache, vcache, L: int | None = None, scale: float = 0.0):
     L = Lcap if L is None else L
     o = torch.empty_like(q)
     nbytes = LIB.sas_dense_decode_workspace_size(B, Hq, Hkv, L, d)
-    ws = _workspace("dense_decode", nbytes, q.device, zero=True)
+    ws = _workspace("dense_decode", nbytes, q.device, zero=False)
     _check("sas_dense_decode", LIB.sas_dense_decode(_dtype(q), _ptr(q), _ptr(kcache), _ptr(vcache),
                                                     B, Hq, Hkv, L, Lcap, d, scale, _ptr(o),
                                                     _ptr(ws), ws.numel(), _stream(q.device)))

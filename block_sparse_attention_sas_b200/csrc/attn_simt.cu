@@ -11,11 +11,13 @@
 //
 // Backward (chain rule through Eq. 9; Eq. 5 inner form for the gate
 // gradient; Eq. 6 Jacobian for the scores):
-//   rowdot:  D_i = dO_i . o_i
 //   csr:     per (batch, kv head), the query blocks that selected each key block
-//   dq:      per (query block, q head): recompute P, dP = dO V^T,
-//            dS = P (dP - D), dq += scale dS K, and da(j,m) = sum of dS over
-//            the tile (one partial per q head and row chunk)
+//   dq:      per (query block, q head): recompute P and dP = dO V^T; a
+//            first sweep sums D_i = sum_t P_it dP_it exactly (using the
+//            stored bf16 o for dO . o would carry its rounding into every
+//            gradient), a second forms dS = P (dP - D), dq += scale dS K and
+//            da(j,m) = sum of dS over the tile (one partial per q head and
+//            row chunk); D goes to the workspace for the dk/dv pass
 //   dkdv:    per key block: over the diagonal and every selecting query
 //            block and head, dv += P^T dO, dk += scale dS^T Q
 //   jacobian: dscores[j,k] = [k in I_j] da_k - g_k sum_{m in I_j} da_m
@@ -176,22 +178,6 @@ fwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict
 }
 
 // ---------------------------------------------------------------------------
-// Backward: D_i = dO_i . o_i (one warp per row)
-// ---------------------------------------------------------------------------
-template <typename T, int D>
-__global__ void __launch_bounds__(kThreads)
-rowdot_kernel(const T* __restrict__ o, const T* __restrict__ dO, long long rows,
-              float* __restrict__ Dv) {
-  const long long row = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  float a = 0.f;
-  for (int c = lane; c < D; c += 32) a = fmaf(ld_f(o + row * D + c), ld_f(dO + row * D + c), a);
-  a = warp_sum(a);
-  if (lane == 0) Dv[row] = a;
-}
-
-// ---------------------------------------------------------------------------
 // Backward: reverse index. For (batch, kv head): list[off[m] .. off[m+1]) holds
 // j*K + slot for every query block j whose slot selects key block m, in
 // ascending j. One CTA per (batch, kv head).
@@ -250,7 +236,7 @@ csr_kernel(const int32_t* __restrict__ idx, AttnShape s, int32_t* __restrict__ o
 template <typename T, int D, int BS>
 __global__ void __launch_bounds__(kThreads)
 dq_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-          const float* __restrict__ lse, const T* __restrict__ dO, const float* __restrict__ Dv,
+          const float* __restrict__ lse, const T* __restrict__ dO, float* __restrict__ Dv,
           const int32_t* __restrict__ idx, const float* __restrict__ gates, AttnShape s,
           T* __restrict__ dq, float* __restrict__ da, DevCtx ctx) {
   constexpr int ROWS = Tiles<BS>::ROWS, RC = Tiles<BS>::RC;
@@ -285,13 +271,16 @@ dq_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict_
   for (int r = tid; r < ROWS; r += kThreads) {
     const int row = r0 + r;
     lse_s[r] = row < s.T ? lse[qrow0 + row] : 0.f;
-    D_s[r] = row < s.T ? Dv[qrow0 + row] : 0.f;
+    D_s[r] = 0.f;
   }
   float acc[NACC];
 #pragma unroll
   for (int x = 0; x < NACC; ++x) acc[x] = 0.f;
 
+  // Sweep 0 computes D_i = sum_t P_it dP_it exactly (the softmax Jacobian's
+  // row term; equal to dO_i . o_i for the unrounded o). Sweep 1 forms dS.
   const int nsel = s.dense ? j : s.K;
+  for (int sweep = 0; sweep < 2; ++sweep)
   for (int it = 0; it <= nsel; ++it) {
     int m;
     float bias;
@@ -305,6 +294,29 @@ dq_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict_
       Vs[t * DP + c] = ok ? ld_f(v + kbase + (long long)key * D + c) : 0.f;
     }
     __syncthreads();
+    if (sweep == 0) {
+      for (int e = tid; e < ROWS * BS; e += kThreads) {
+        const int r = e / BS, c = e % BS;
+        float a = 0.f, b = 0.f;
+#pragma unroll 8
+        for (int kk = 0; kk < D; ++kk) {
+          a = fmaf(Qs[r * DP + kk], Ks[c * DP + kk], a);
+          b = fmaf(dOs[r * DP + kk], Vs[c * DP + kk], b);
+        }
+        const int qi = r0 + r, ki = m * BS + c;
+        float p = 0.f;
+        if (qi < s.T && ki < s.T && !(cur && ki > qi)) p = expf(fmaf(a, s.scale, bias) - lse_s[r]);
+        Ps[r * BP + c] = p * b;
+      }
+      __syncthreads();
+      for (int r = warp; r < ROWS; r += kWarps) {
+        float t = 0.f;
+        for (int c = lane; c < BS; c += 32) t += Ps[r * BP + c];
+        t = warp_sum(t);
+        if (lane == 0) D_s[r] += t;
+      }
+      continue;
+    }
     float dsum = 0.f;
     for (int e = tid; e < ROWS * BS; e += kThreads) {
       const int r = e / BS, c = e % BS;
@@ -345,6 +357,10 @@ dq_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict_
   for (int x = 0; x < NACC; ++x) {
     const int e = tid + x * kThreads, r = e / D, c = e % D, row = r0 + r;
     if (row < s.T) st_f(dq + (qrow0 + row) * D + c, acc[x]);
+  }
+  for (int r = tid; r < ROWS; r += kThreads) {
+    const int row = r0 + r;
+    if (row < s.T) Dv[qrow0 + row] = D_s[r];
   }
 }
 
@@ -552,11 +568,6 @@ cudaError_t bwd_t(const AttnShape& s, const void* q, const void* k, const void* 
   int32_t* coff = reinterpret_cast<int32_t*>(w + L.off_csr_off);
   int32_t* clist = reinterpret_cast<int32_t*>(w + L.off_csr_list);
   cudaError_t e;
-  const long long rows = (long long)s.B * s.Hq * s.T;
-  rowdot_kernel<T, D><<<(unsigned)((rows + kWarps - 1) / kWarps), kThreads, 0, st>>>(
-      (const T*)o, (const T*)dO, rows, Dv);
-  note_launches(1);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (!s.dense) {
     const size_t smem = 2 * sizeof(int32_t) * (size_t)s.N;
     e = cudaFuncSetAttribute(csr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

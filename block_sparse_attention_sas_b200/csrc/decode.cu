@@ -27,9 +27,8 @@ constexpr int kWarps = 4;
 constexpr int kThreads = 32 * kWarps;
 constexpr int kChunk = 16;  // tokens per warp work item
 constexpr int kLPT = 8;     // lanes per token in the q.k phase
-constexpr int kMaxSplits = 256;
+constexpr int kMaxSplits = 64;    // bounds the last CTA's merge
 
-template <typename T> struct Vec;
 // Loads `n` consecutive elements (n*sizeof(T) a multiple of 4 bytes) as floats.
 template <typename T, int n>
 __device__ __forceinline__ void load_f(const T* p, float (&out)[n]);
@@ -55,20 +54,6 @@ __device__ __forceinline__ void load_f<__nv_bfloat16, 8>(const __nv_bfloat16* p,
     out[2 * i + 1] = bf16hi(w[i]);
   }
 }
-template <>
-__device__ __forceinline__ void load_f<__nv_bfloat16, 4>(const __nv_bfloat16* p, float (&out)[4]) {
-  const uint2 a = __ldg(reinterpret_cast<const uint2*>(p));
-  out[0] = bf16lo(a.x);
-  out[1] = bf16hi(a.x);
-  out[2] = bf16lo(a.y);
-  out[3] = bf16hi(a.y);
-}
-template <>
-__device__ __forceinline__ void load_f<__nv_bfloat16, 2>(const __nv_bfloat16* p, float (&out)[2]) {
-  const uint32_t a = __ldg(reinterpret_cast<const unsigned int*>(p));
-  out[0] = bf16lo(a);
-  out[1] = bf16hi(a);
-}
 template <int n>
 __device__ __forceinline__ void load_f_f32(const float* p, float (&out)[n]) {
   static_assert(n % 2 == 0, "");
@@ -89,8 +74,6 @@ __device__ __forceinline__ void load_f_f32(const float* p, float (&out)[n]) {
 }
 template <> __device__ __forceinline__ void load_f<float, 16>(const float* p, float (&o)[16]) { load_f_f32<16>(p, o); }
 template <> __device__ __forceinline__ void load_f<float, 8>(const float* p, float (&o)[8]) { load_f_f32<8>(p, o); }
-template <> __device__ __forceinline__ void load_f<float, 4>(const float* p, float (&o)[4]) { load_f_f32<4>(p, o); }
-template <> __device__ __forceinline__ void load_f<float, 2>(const float* p, float (&o)[2]) { load_f_f32<2>(p, o); }
 
 // Block held by slot `sl` of a (batch, kv head): sparse -> idx entries then the
 // current block; dense -> blocks 0..C in order. Returns -1 for an empty slot.
@@ -107,19 +90,67 @@ __device__ __forceinline__ int slot_block(const DecodeShape& s, const int32_t* i
   return m;
 }
 
+// Shared-memory element loads (vectorised; the stage buffers are 16-byte aligned).
+template <typename T, int n>
+__device__ __forceinline__ void lds_f(const T* p, float (&out)[n]) {
+  if constexpr (sizeof(T) == 2) {
+    static_assert(n % 2 == 0, "");
+    if constexpr (n % 8 == 0) {
+#pragma unroll
+      for (int i = 0; i < n / 8; ++i) {
+        const uint4 a = reinterpret_cast<const uint4*>(p)[i];
+        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          out[8 * i + 2 * j] = bf16lo(w[j]);
+          out[8 * i + 2 * j + 1] = bf16hi(w[j]);
+        }
+      }
+    } else if constexpr (n == 4) {
+      const uint2 a = *reinterpret_cast<const uint2*>(p);
+      out[0] = bf16lo(a.x); out[1] = bf16hi(a.x); out[2] = bf16lo(a.y); out[3] = bf16hi(a.y);
+    } else {
+      const uint32_t a = *reinterpret_cast<const uint32_t*>(p);
+      out[0] = bf16lo(a); out[1] = bf16hi(a);
+    }
+  } else {
+    if constexpr (n % 4 == 0) {
+#pragma unroll
+      for (int i = 0; i < n / 4; ++i) {
+        const float4 a = reinterpret_cast<const float4*>(p)[i];
+        out[4 * i] = a.x; out[4 * i + 1] = a.y; out[4 * i + 2] = a.z; out[4 * i + 3] = a.w;
+      }
+    } else {
+      const float2 a = *reinterpret_cast<const float2*>(p);
+      out[0] = a.x; out[1] = a.y;
+    }
+  }
+}
+
+constexpr int kMaxStages = 4;
+
+// One CTA per (split, kv head, batch). Thread 0 streams the split's K/V blocks
+// into a ring of shared-memory stages with bulk async copies (one mbarrier per
+// stage, waits bounded by the context's limit); the four warps compute each
+// staged block from shared memory (warp w takes the block's 16-token chunks
+// w, w+4, ...) while later blocks are in flight.
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads)
 decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
               const int32_t* __restrict__ idx, const float* __restrict__ gates, DecodeShape s,
-              T* __restrict__ o, float* __restrict__ ws_ml, float* __restrict__ ws_o,
+              int nst, T* __restrict__ o, float* __restrict__ ws_ml, float* __restrict__ ws_o,
               uint32_t* __restrict__ ws_cnt, DevCtx ctx) {
   constexpr int VPL = D / kLPT;   // q.k dims per lane
   constexpr int TPP = 32 / kLPT;  // tokens per pass
   constexpr int DPL = D / 32;     // output dims per lane
+  extern __shared__ __align__(128) unsigned char stage_mem[];
+  __shared__ uint64_t full_bar[kMaxStages];
   __shared__ float s_x[kWarps][G][kChunk];
   __shared__ float s_p[kWarps][kChunk][G];
   __shared__ float s_m[kWarps][G], s_l[kWarps][G];
   __shared__ float s_o[kWarps][G][D];
+  __shared__ float s_w[G * kMaxSplits];
+  __shared__ float s_L[G];
   __shared__ int s_last;
 
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
@@ -127,17 +158,44 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __rest
   const int unit = bi * s.Hkv + kvh;
   const int nslots = s.dense ? s.C + 1 : s.K + 1;
   const int sl0 = split * s.bps, sl1 = min(nslots, sl0 + s.bps);
+  const int ns = sl1 - sl0;
   const int cpb = s.b / kChunk;  // chunks per block
   const long long cache0 = (long long)unit * s.Lcap * D;
   const int32_t* ix = s.dense ? nullptr : idx + (long long)unit * s.K;
+  const size_t stage_elems = (size_t)2 * s.b * D;  // K block then V block
 
-  // q for this lane's q.k dims, all G heads.
+  // Block of slot i of this split and its number of valid rows (0: skip).
+  auto slot_rows = [&](int i, int& m) -> int {
+    m = slot_block(s, ix, sl0 + i, ctx);
+    if (m < 0) return 0;
+    return min(s.b, s.L - m * s.b);
+  };
+  auto issue = [&](int i) {
+    int m;
+    const int rows = slot_rows(i, m);
+    if (rows <= 0) return;
+    const int st = i % nst;
+    T* kst = reinterpret_cast<T*>(stage_mem) + st * stage_elems;
+    const uint32_t bytes = (uint32_t)(rows * D * sizeof(T));
+    mbar_arrive_expect_tx(&full_bar[st], 2 * bytes);
+    bulk_g2s(kst, kc + cache0 + (long long)m * s.b * D, bytes, &full_bar[st]);
+    bulk_g2s(kst + (size_t)s.b * D, vc + cache0 + (long long)m * s.b * D, bytes, &full_bar[st]);
+  };
+
+  if (tid == 0) {
+    for (int st = 0; st < nst; ++st) mbar_init(&full_bar[st], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0)
+    for (int i = 0; i < min(nst, ns); ++i) issue(i);
+
+  // q for this lane's q.k dims, all G heads (scaled once).
   float qr[G][VPL];
   const int dseg = (lane % kLPT) * VPL;
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    const T* qp = q + ((long long)bi * s.Hq + kvh * G + g) * D + dseg;
-    load_f<T, VPL>(qp, qr[g]);
+    load_f<T, VPL>(q + ((long long)bi * s.Hq + kvh * G + g) * D + dseg, qr[g]);
 #pragma unroll
     for (int i = 0; i < VPL; ++i) qr[g][i] *= s.scale;
   }
@@ -150,71 +208,79 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __rest
     for (int i = 0; i < DPL; ++i) acc[g][i] = 0.f;
   }
 
-  const int nchunks = (sl1 - sl0) * cpb;
-  for (int c = w; c < nchunks; c += kWarps) {
-    const int sl = sl0 + c / cpb;
-    const int m = slot_block(s, ix, sl, ctx);
-    if (m < 0) continue;
-    const float bias = (!s.dense && s.use_gates && sl < s.K)
+  bool ok = true;
+  for (int i = 0; i < ns; ++i) {
+    int m;
+    const int rows = slot_rows(i, m);
+    if (rows <= 0) continue;  // uniform: every thread reads the same slot
+    const int st = i % nst;
+    if (!mbar_wait(ctx, &full_bar[st], (uint32_t)((i / nst) & 1))) ok = false;
+    const T* ks = reinterpret_cast<const T*>(stage_mem) + st * stage_elems;
+    const T* vs = ks + (size_t)s.b * D;
+    const float bias = (!s.dense && s.use_gates && sl0 + i < s.K)
                            ? logf(gates[(long long)unit * s.C + m]) : 0.f;
-    const int t0 = m * s.b + (c % cpb) * kChunk;  // first token of the chunk
-    if (t0 >= s.L) continue;
-    const int nt = min(kChunk, s.L - t0);
-
-    // ---- logits: kLPT lanes per token, TPP tokens per pass
+    for (int c = w; c < cpb && ok; c += kWarps) {
+      const int t0 = c * kChunk;
+      if (t0 >= rows) break;
+      const int nt = min(kChunk, rows - t0);
+      // ---- logits: kLPT lanes per token, TPP tokens per pass
 #pragma unroll
-    for (int pass = 0; pass < kChunk / TPP; ++pass) {
-      const int tt = pass * TPP + lane / kLPT;
-      float dot[G];
+      for (int pass = 0; pass < kChunk / TPP; ++pass) {
+        const int tt = pass * TPP + lane / kLPT;
+        float dot[G];
 #pragma unroll
-      for (int g = 0; g < G; ++g) dot[g] = 0.f;
-      if (tt < nt) {
-        float kf[VPL];
-        load_f<T, VPL>(kc + cache0 + (long long)(t0 + tt) * D + dseg, kf);
+        for (int g = 0; g < G; ++g) dot[g] = 0.f;
+        if (tt < nt) {
+          float kf[VPL];
+          lds_f<T, VPL>(ks + (size_t)(t0 + tt) * D + dseg, kf);
 #pragma unroll
-        for (int g = 0; g < G; ++g)
+          for (int g = 0; g < G; ++g)
 #pragma unroll
-          for (int i = 0; i < VPL; ++i) dot[g] = fmaf(qr[g][i], kf[i], dot[g]);
+            for (int x = 0; x < VPL; ++x) dot[g] = fmaf(qr[g][x], kf[x], dot[g]);
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+#pragma unroll
+          for (int off = kLPT / 2; off > 0; off >>= 1)
+            dot[g] += __shfl_xor_sync(0xffffffffu, dot[g], off);
+        }
+        if ((lane % kLPT) == 0) {
+#pragma unroll
+          for (int g = 0; g < G; ++g) s_x[w][g][tt] = (tt < nt) ? dot[g] + bias : -INFINITY;
+        }
       }
+      __syncwarp();
+      // ---- online softmax: lane t < kChunk owns token t
 #pragma unroll
       for (int g = 0; g < G; ++g) {
+        const float x = (lane < kChunk) ? s_x[w][g][lane] : -INFINITY;
+        const float mx = warp_max(x);
+        const float mnew = fmaxf(m_run[g], mx);
+        const float p = (mnew == -INFINITY) ? 0.f : expf(x - mnew);
+        const float alpha = (mnew == -INFINITY) ? 1.f : expf(m_run[g] - mnew);
+        l_run[g] = l_run[g] * alpha + warp_sum(p);
+        m_run[g] = mnew;
+        if (lane < kChunk) s_p[w][lane][g] = p;
 #pragma unroll
-        for (int off = kLPT / 2; off > 0; off >>= 1)
-          dot[g] += __shfl_xor_sync(0xffffffffu, dot[g], off);
+        for (int x2 = 0; x2 < DPL; ++x2) acc[g][x2] *= alpha;
       }
-      if ((lane % kLPT) == 0) {
+      __syncwarp();
+      // ---- o += p v: lane owns DPL consecutive dims
+#pragma unroll 4
+      for (int t = 0; t < nt; ++t) {
+        float vf[DPL];
+        lds_f<T, DPL>(vs + (size_t)(t0 + t) * D + lane * DPL, vf);
 #pragma unroll
-        for (int g = 0; g < G; ++g) s_x[w][g][tt] = (tt < nt) ? dot[g] + bias : -INFINITY;
+        for (int g = 0; g < G; ++g) {
+          const float p = s_p[w][t][g];
+#pragma unroll
+          for (int x2 = 0; x2 < DPL; ++x2) acc[g][x2] = fmaf(p, vf[x2], acc[g][x2]);
+        }
       }
+      __syncwarp();
     }
-    __syncwarp();
-    // ---- online softmax: lane t < kChunk owns token t
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float x = (lane < kChunk) ? s_x[w][g][lane] : -INFINITY;
-      const float mx = warp_max(x);
-      const float mnew = fmaxf(m_run[g], mx);
-      const float p = (mnew == -INFINITY) ? 0.f : expf(x - mnew);
-      const float alpha = (mnew == -INFINITY) ? 1.f : expf(m_run[g] - mnew);
-      l_run[g] = l_run[g] * alpha + warp_sum(p);
-      m_run[g] = mnew;
-      if (lane < kChunk) s_p[w][lane][g] = p;
-#pragma unroll
-      for (int i = 0; i < DPL; ++i) acc[g][i] *= alpha;
-    }
-    __syncwarp();
-    // ---- o += p v: lane owns DPL consecutive dims
-    for (int t = 0; t < nt; ++t) {
-      float vf[DPL];
-      load_f<T, DPL>(vc + cache0 + (long long)(t0 + t) * D + lane * DPL, vf);
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float p = s_p[w][t][g];
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) acc[g][i] = fmaf(p, vf[i], acc[g][i]);
-      }
-    }
-    __syncwarp();
+    __syncthreads();  // stage st is free
+    if (tid == 0 && i + nst < ns) issue(i + nst);
   }
 
   // ---- merge the warps of this CTA
@@ -254,7 +320,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __rest
   }
   if (s.splits == 1) return;
 
-  // ---- last CTA of the unit merges the partials
+  // ---- the last CTA of the unit merges the partials by log-sum-exp
   __threadfence();
   __syncthreads();
   if (tid == 0) {
@@ -264,21 +330,50 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __rest
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  for (int e = tid; e < G * D; e += kThreads) {
-    const int g = e / D, dd = e % D;
-    const long long p0 = (hbase + g) * s.splits;
+  const int P = s.splits;
+  for (int e = tid; e < G * P; e += kThreads) s_w[e] = __ldcg(&ws_ml[2 * (hbase * P + e)]);
+  __syncthreads();
+  for (int g = w; g < G; g += kWarps) {
     float M = -INFINITY;
-    for (int x = 0; x < s.splits; ++x) M = fmaxf(M, __ldcg(&ws_ml[2 * (p0 + x)]));
-    float L = 0.f, A = 0.f;
-    for (int x = 0; x < s.splits; ++x) {
-      const float mx = __ldcg(&ws_ml[2 * (p0 + x)]);
+    for (int x = lane; x < P; x += 32) M = fmaxf(M, s_w[g * P + x]);
+    M = warp_max(M);
+    float L = 0.f;
+    for (int x = lane; x < P; x += 32) {
+      const float mx = s_w[g * P + x];
       const float f = (mx == -INFINITY) ? 0.f : expf(mx - M);
-      L += f * __ldcg(&ws_ml[2 * (p0 + x) + 1]);
-      A += f * __ldcg(&ws_o[(p0 + x) * D + dd]);
+      L += f * __ldcg(&ws_ml[2 * (hbase * P + g * P + x) + 1]);
+      s_w[g * P + x] = f;
     }
-    st_f(o + (hbase + g) * D + dd, A / L);
+    L = warp_sum(L);
+    if (lane == 0) s_L[g] = L;
   }
-  if (tid == 0) ws_cnt[unit] = 0u;
+  __syncthreads();
+  for (int e = tid; e < G * (D / 4); e += kThreads) {
+    const int g = e / (D / 4), d4 = e % (D / 4);
+    const float4* src = reinterpret_cast<const float4*>(ws_o + (hbase + g) * P * D) + d4;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+    for (int x = 0; x < P; ++x) {
+      const float4 v = __ldcg(src + (size_t)x * (D / 4));
+      const float f = s_w[g * P + x];
+      a.x = fmaf(f, v.x, a.x);
+      a.y = fmaf(f, v.y, a.y);
+      a.z = fmaf(f, v.z, a.z);
+      a.w = fmaf(f, v.w, a.w);
+    }
+    const float inv = 1.f / s_L[g];
+    T* dst = o + (hbase + g) * D + d4 * 4;
+    st_f(dst + 0, a.x * inv);
+    st_f(dst + 1, a.y * inv);
+    st_f(dst + 2, a.z * inv);
+    st_f(dst + 3, a.w * inv);
+  }
+}
+
+int decode_stages(const DecodeShape& s, size_t elem) {
+  const size_t stage = (size_t)2 * s.b * s.d * elem;
+  int nst = (int)((96u << 10) / stage);
+  return max(2, min(kMaxStages, nst));
 }
 
 template <typename T, int D, int G>
@@ -291,13 +386,24 @@ cudaError_t decode_t(const DecodeShape& s, const void* q, const void* kc, const 
   float* ws_o = reinterpret_cast<float*>(w + ((2 * parts * sizeof(float) + 255) & ~(size_t)255));
   uint32_t* ws_cnt = reinterpret_cast<uint32_t*>(
       reinterpret_cast<char*>(ws_o) + ((parts * D * sizeof(float) + 255) & ~(size_t)255));
+  cudaError_t e;
+  if (s.splits > 1) {
+    // Tickets start at zero on every call, whatever the workspace held before.
+    e = cudaMemsetAsync(ws_cnt, 0, sizeof(uint32_t) * (size_t)s.B * s.Hkv, st);
+    if (e != cudaSuccess) return e;
+    note_launches(1);
+  }
+  const int nst = decode_stages(s, sizeof(T));
+  const size_t smem = (size_t)nst * 2 * s.b * D * sizeof(T);
+  auto kern = decode_kernel<T, D, G>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   dim3 grid(s.splits, s.Hkv, s.B);
-  decode_kernel<T, D, G><<<grid, kThreads, 0, st>>>((const T*)q, (const T*)kc, (const T*)vc, idx,
-                                                    gates, s, (T*)o, ws_ml, ws_o, ws_cnt, ctx);
+  kern<<<grid, kThreads, smem, st>>>((const T*)q, (const T*)kc, (const T*)vc, idx, gates, s, nst,
+                                     (T*)o, ws_ml, ws_o, ws_cnt, ctx);
   note_launches(1);
   return cudaGetLastError();
 }
-
 template <typename T, int D>
 cudaError_t decode_g(const DecodeShape& s, const void* q, const void* kc, const void* vc,
                      const int32_t* idx, const float* gates, void* o, void* ws, const DevCtx& ctx,
@@ -318,9 +424,10 @@ cudaError_t decode_g(const DecodeShape& s, const void* q, const void* kc, const 
 }  // namespace
 
 void decode_plan(DecodeShape& s) {
+  // About two CTAs per SM (148 SMs), at most kMaxSplits per (batch, kv head).
   const int nslots = s.dense ? s.C + 1 : s.K + 1;
   const int units = s.B * s.Hkv;
-  const int target = 148 * 4;
+  const int target = 2 * 148;
   int splits = (target + units - 1) / units;
   splits = max(1, min(splits, min(nslots, kMaxSplits)));
   int bps = (nslots + splits - 1) / splits;

@@ -7,11 +7,12 @@
 // Eq. 6; reproduction README, Core equations).
 //
 // Selection without sorting the row: scores map to order-preserving 32-bit
-// keys; a 32-step bisection on the key bits finds tau, the k-th largest key
-// (the largest value with at least k keys >= it). Every key > tau is taken,
-// plus the lowest-indexed (k - #{key > tau}) keys equal to tau, found by an
-// ordered ballot scan. The k survivors are placed by rank (a survivor's rank
-// is the number of survivors that beat it), which sorts them exactly.
+// keys; a most-significant-digit radix select (four passes over 8-bit
+// digits, each a 256-bin histogram of the keys that share the prefix found
+// so far) finds tau, the k-th largest key. Every key > tau is taken, plus the
+// lowest-indexed (k - #{key > tau}) keys equal to tau, found by an ordered
+// ballot scan. The k survivors are placed by rank (a survivor's rank is the
+// number of survivors that beat it), which sorts them exactly.
 //
 // Two layouts of the same algorithm: one warp per row for short rows (the
 // training case, one row per query block), one CTA per row for long rows
@@ -36,8 +37,50 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
+// Adds one per element to hist[bin] for the lanes with `valid`; lanes that
+// hold the same bin are combined first, so each bin takes one atomic per warp.
+__device__ __forceinline__ void warp_hist_add(int* hist, uint32_t bin, bool valid) {
+  const uint32_t lane = threadIdx.x & 31;
+  const uint32_t key = valid ? bin : (0x10000u + lane);
+  const uint32_t peers = __match_any_sync(0xffffffffu, key);
+  if (valid && (__ffs(peers) - 1) == (int)lane) atomicAdd(&hist[bin], __popc(peers));
+}
+
+// Given a 256-bin histogram (the warp reads it), finds the digit holding the
+// k-th largest element: returns the digit and sets `above` to the count of
+// elements in bins above it. Every lane returns the same values.
+__device__ __forceinline__ uint32_t warp_pick_digit(const int* hist, int k, int& above) {
+  const int lane = threadIdx.x & 31;
+  int h[8], sum = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    h[i] = hist[lane * 8 + i];
+    sum += h[i];
+  }
+  int suf = sum;  // inclusive suffix sum over lanes >= lane
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_down_sync(0xffffffffu, suf, off);
+    if (lane + off < 32) suf += v;
+  }
+  const uint32_t hit = __ballot_sync(0xffffffffu, suf >= k);
+  const int L = 31 - __clz(hit);  // highest lane whose suffix reaches k
+  int ab = suf - sum, dig = 0;    // elements in lanes above L
+  if (lane == L) {
+    for (int i = 7; i >= 0; --i) {
+      if (ab + h[i] >= k) {
+        dig = L * 8 + i;
+        break;
+      }
+      ab += h[i];
+    }
+  }
+  above = __shfl_sync(0xffffffffu, ab, L);
+  return (uint32_t)__shfl_sync(0xffffffffu, dig, L);
+}
+
 constexpr int kWarpRowsPerCta = 8;
-constexpr int kWarpCap = 1024;  // longest row handled by one warp
+constexpr int kWarpCap = 512;   // longest row handled by one warp
 constexpr int kMaxK = 256;
 
 // ---------------------------------------------------------------------------
@@ -49,6 +92,7 @@ gate_topk_warp_kernel(const float* __restrict__ scores, int total_rows, int rows
   __shared__ float s_val[kWarpRowsPerCta][kWarpCap];
   __shared__ uint32_t s_selkey[kWarpRowsPerCta][kMaxK];
   __shared__ int32_t s_selidx[kWarpRowsPerCta][kMaxK];
+  __shared__ int s_hist[kWarpRowsPerCta][256];
 
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long row = (long long)blockIdx.x * kWarpRowsPerCta + w;
@@ -76,19 +120,28 @@ gate_topk_warp_kernel(const float* __restrict__ scores, int total_rows, int rows
 
   const int k = min(K, n);
   if (k > 0) {
-    // ---- tau = k-th largest key, by bisection on the key bits
-    uint32_t tau = 0;
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = tau | (1u << bit);
-      int cnt = 0;
-      for (int i = lane; i < n; i += 32) cnt += fkey(v[i]) >= cand;
-      cnt = __reduce_add_sync(0xffffffffu, cnt);
-      if (cnt >= k) tau = cand;
+    // ---- tau = k-th largest key: radix select, four 8-bit digits
+    int* hist = s_hist[w];
+    uint32_t tau = 0, mask = 0;
+    int krem = k;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) hist[lane * 8 + i] = 0;
+      __syncwarp();
+      for (int base = 0; base < n; base += 32) {
+        const int i = base + lane;
+        const uint32_t key = (i < n) ? fkey(v[i]) : 0u;
+        warp_hist_add(hist, (key >> shift) & 255u, i < n && (key & mask) == tau);
+      }
+      __syncwarp();
+      int above;
+      const uint32_t dig = warp_pick_digit(hist, krem, above);
+      krem -= above;
+      tau |= dig << shift;
+      mask |= 255u << shift;
+      __syncwarp();
     }
-    int gt = 0;
-    for (int i = lane; i < n; i += 32) gt += fkey(v[i]) > tau;
-    gt = __reduce_add_sync(0xffffffffu, gt);
-    const int need_eq = k - gt;
+    const int need_eq = krem;
 
     // ---- ordered compaction of the survivors (index order)
     int run_eq = 0, run_sel = 0;
@@ -148,16 +201,6 @@ __device__ __forceinline__ float block_reduce_sum(float x, float* red) {
   float y = (lane < kCtaWarps) ? red[lane] : 0.f;
   return warp_sum(y);
 }
-__device__ __forceinline__ int block_reduce_add(int x, int* red) {
-  x = __reduce_add_sync(0xffffffffu, x);
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  __syncthreads();
-  if (lane == 0) red[w] = x;
-  __syncthreads();
-  int y = (lane < kCtaWarps) ? red[lane] : 0;
-  return __reduce_add_sync(0xffffffffu, y);
-}
-
 // Dynamic shared memory: the row's values when n <= cap (else they are
 // re-read from global memory, where the row stays L2-resident).
 __global__ void __launch_bounds__(kCtaThreads)
@@ -165,10 +208,12 @@ gate_topk_cta_kernel(const float* __restrict__ scores, int rows, int C, int caus
                      int cap, float* __restrict__ gates, int32_t* __restrict__ idx) {
   extern __shared__ float s_dyn[];
   __shared__ float red_f[kCtaWarps];
-  __shared__ int red_i[kCtaWarps];
   __shared__ int warp_cnt[kCtaWarps];
   __shared__ uint32_t s_selkey[kMaxK];
   __shared__ int32_t s_selidx[kMaxK];
+  __shared__ int s_whist[kCtaWarps][256];
+  __shared__ int s_hist[256];
+  __shared__ int s_pick[2];
 
   const long long row = blockIdx.x;
   const int r = (int)(row % rows);
@@ -195,18 +240,40 @@ gate_topk_cta_kernel(const float* __restrict__ scores, int rows, int C, int caus
 
   const int k = min(K, n);
   if (k > 0) {
-    uint32_t tau = 0;
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = tau | (1u << bit);
-      int cnt = 0;
-      for (int i = tid; i < n; i += kCtaThreads) cnt += fkey(v[i]) >= cand;
-      cnt = block_reduce_add(cnt, red_i);
-      if (cnt >= k) tau = cand;
+    // Radix select over four 8-bit digits: per-warp histograms, summed into
+    // one, and warp 0 picks the digit.
+    uint32_t tau = 0, mask = 0;
+    int krem = k;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = tid; i < kCtaWarps * 256; i += kCtaThreads) (&s_whist[0][0])[i] = 0;
+      __syncthreads();
+      for (int base = 0; base < n; base += kCtaThreads) {
+        const int i = base + tid;
+        const uint32_t key = (i < n) ? fkey(v[i]) : 0u;
+        warp_hist_add(s_whist[w], (key >> shift) & 255u, i < n && (key & mask) == tau);
+      }
+      __syncthreads();
+      for (int bin = tid; bin < 256; bin += kCtaThreads) {
+        int t = 0;
+#pragma unroll
+        for (int x = 0; x < kCtaWarps; ++x) t += s_whist[x][bin];
+        s_hist[bin] = t;
+      }
+      __syncthreads();
+      if (w == 0) {
+        int above;
+        const uint32_t dig = warp_pick_digit(s_hist, krem, above);
+        if (lane == 0) {
+          s_pick[0] = (int)dig;
+          s_pick[1] = above;
+        }
+      }
+      __syncthreads();
+      krem -= s_pick[1];
+      tau |= (uint32_t)s_pick[0] << shift;
+      mask |= 255u << shift;
     }
-    int gt = 0;
-    for (int i = tid; i < n; i += kCtaThreads) gt += fkey(v[i]) > tau;
-    gt = block_reduce_add(gt, red_i);
-    const int need_eq = k - gt;
+    const int need_eq = krem;
 
     // Each warp owns a contiguous, 32-aligned range of the row. Pass 1
     // counts its keys equal to tau; an exclusive scan over warps gives each

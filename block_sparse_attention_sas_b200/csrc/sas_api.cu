@@ -194,11 +194,11 @@ sas_status_t sas_selftest_wait_timeout(sas_stream_t stream) {
 sas_status_t sas_gate_topk(const float* scores, int B, int Hkv, int rows, int C, int causal,
                            int K, float* gates, int32_t* idx, sas_stream_t stream) {
   if (B < 0 || Hkv < 0 || rows < 0) return SAS_ERR_INVALID_ARG;
-  if (C < 1 || K < 1 || (causal != 0 && causal != 1)) return SAS_ERR_INVALID_ARG;
+  if (C < 0 || K < 1 || (causal != 0 && causal != 1)) return SAS_ERR_INVALID_ARG;
   if (causal && rows != C) return SAS_ERR_INVALID_ARG;
   if (C > 262144 || K > 256) return SAS_ERR_UNSUPPORTED;
   if ((long long)B * Hkv * rows == 0) return SAS_OK;
-  if (!scores || !gates || !idx) return SAS_ERR_INVALID_ARG;
+  if (!idx || (C > 0 && (!scores || !gates))) return SAS_ERR_INVALID_ARG;
   if (!aligned(scores, 4) || !aligned(gates, 4) || !aligned(idx, 4)) return SAS_ERR_INVALID_ARG;
   if ((long long)B * Hkv * rows > (1ll << 31) - 1) return SAS_ERR_UNSUPPORTED;
   return cuda_status(launch_gate_topk(scores, B, Hkv, rows, C, causal, K, gates, idx, stream));
@@ -264,7 +264,7 @@ sas_status_t sas_decode(sas_dtype_t dtype, const void* q, const void* kcache, co
   if (st != SAS_OK) return st;
   if (B == 0) return SAS_OK;
   if (!q || !kcache || !vcache || !idx || !o) return SAS_ERR_INVALID_ARG;
-  if (use_gates && !gates) return SAS_ERR_INVALID_ARG;
+  if (use_gates && !gates && (L - 1) / b > 0) return SAS_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(kcache, 16) || !aligned(vcache, 16) || !aligned(o, 16) ||
       !aligned(idx, 4) || (gates && !aligned(gates, 4)))
     return SAS_ERR_INVALID_ARG;

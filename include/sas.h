@@ -97,7 +97,8 @@ uint64_t sas_launch_count(void);
  *            largest scores' block indices in rank order (descending score,
  *            equal scores ordered by lower index; -0.0 equals +0.0), padded
  *            with -1.
- *   Limits: 1 <= C <= 262144, 1 <= K <= 256.
+ *   Limits: 0 <= C <= 262144 (C = 0: no history, idx all -1; scores and
+ *   gates may then be NULL), 1 <= K <= 256.
  */
 sas_status_t sas_gate_topk(const float* scores, int B, int Hkv, int rows, int C, int causal,
                            int K, float* gates, int32_t* idx, sas_stream_t stream);
@@ -162,9 +163,9 @@ sas_status_t sas_attn_bwd(sas_dtype_t dtype, const void* q, const void* k, const
  *   gates [B, Hkv, C] fp32; read only when use_gates != 0 (may be NULL otherwise).
  *   o [B, Hq, d] (dtype; written).
  *   ws / ws_bytes: at least sas_decode_workspace_size() bytes, 256-byte
- *   aligned. The workspace must be ZERO-FILLED before its first use; every
- *   call leaves it zero-filled again, so it can be reused without clearing.
- *   Calls that share a workspace must not overlap on the device.
+ *   aligned; its contents on entry do not matter (the call clears the part
+ *   that must start at zero). Calls that share a workspace must not overlap
+ *   on the device.
  */
 size_t sas_decode_workspace_size(int B, int Hq, int Hkv, int L, int d, int b, int K);
 sas_status_t sas_decode(sas_dtype_t dtype, const void* q, const void* kcache, const void* vcache,
