@@ -395,6 +395,21 @@ def bench_decode(S, torch, dev, stream, flush, peaks, args, rank):
     return out
 
 
+def run_decode_only(args):
+    """Only the decode lines of one preset (both gate modes it lists)."""
+    import torch
+    from block_sparse_attention_sas_b200 import _lib as S
+    global DECODES
+    cfg = W.PRESETS[args.decode_only]
+    DECODES = [(cfg, g) for g in cfg.gate_modes]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    lines = bench_decode(S, torch, dev, torch.cuda.current_stream(dev), flush, load_peaks(), args,
+                         0)
+    print(json.dumps({"decode": lines}), flush=True)
+
+
 # ----------------------------------------------------------- reference arm
 
 def run_reference(args):
@@ -436,11 +451,15 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-heads", type=int, default=2)
+    ap.add_argument("--decode-only", default=None, metavar="PRESET",
+                    help="time only the decode path of one preset (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.decode_only:
+        run_decode_only(args)
     else:
         run_ours(args)
 

@@ -151,7 +151,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __rest
   __shared__ float s_o[kWarps][G][D];
   __shared__ float s_w[G * kMaxSplits];
   __shared__ float s_L[G];
-  __shared__ int s_last;
+  __shared__ int s_last, s_abort;
 
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, kvh = blockIdx.y, bi = blockIdx.z;
@@ -170,25 +170,31 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __rest
     if (m < 0) return 0;
     return min(s.b, s.L - m * s.b);
   };
-  auto issue = [&](int i) {
+  auto issue = [&](int i) -> bool {
     int m;
     const int rows = slot_rows(i, m);
-    if (rows <= 0) return;
+    if (rows <= 0) return false;
     const int st = i % nst;
     T* kst = reinterpret_cast<T*>(stage_mem) + st * stage_elems;
     const uint32_t bytes = (uint32_t)(rows * D * sizeof(T));
     mbar_arrive_expect_tx(&full_bar[st], 2 * bytes);
     bulk_g2s(kst, kc + cache0 + (long long)m * s.b * D, bytes, &full_bar[st]);
     bulk_g2s(kst + (size_t)s.b * D, vc + cache0 + (long long)m * s.b * D, bytes, &full_bar[st]);
+    return true;
   };
 
   if (tid == 0) {
     for (int st = 0; st < nst; ++st) mbar_init(&full_bar[st], 1);
     fence_mbar_init();
+    s_abort = 0;
   }
   __syncthreads();
+  // Stage bookkeeping, identical in every thread: the parity each stage's
+  // next completion will have, and (thread 0) which stages hold a copy in flight.
+  uint32_t phase_bits = 0, pending = 0;
   if (tid == 0)
-    for (int i = 0; i < min(nst, ns); ++i) issue(i);
+    for (int i = 0; i < min(nst, ns); ++i)
+      if (issue(i)) pending |= 1u << (i % nst);
 
   // q for this lane's q.k dims, all G heads (scaled once).
   float qr[G][VPL];
@@ -208,79 +214,94 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __rest
     for (int i = 0; i < DPL; ++i) acc[g][i] = 0.f;
   }
 
-  bool ok = true;
   for (int i = 0; i < ns; ++i) {
     int m;
-    const int rows = slot_rows(i, m);
-    if (rows <= 0) continue;  // uniform: every thread reads the same slot
+    const int rows = slot_rows(i, m);  // the same in every thread
     const int st = i % nst;
-    if (!mbar_wait(ctx, &full_bar[st], (uint32_t)((i / nst) & 1))) ok = false;
-    const T* ks = reinterpret_cast<const T*>(stage_mem) + st * stage_elems;
-    const T* vs = ks + (size_t)s.b * D;
-    const float bias = (!s.dense && s.use_gates && sl0 + i < s.K)
-                           ? logf(gates[(long long)unit * s.C + m]) : 0.f;
-    for (int c = w; c < cpb && ok; c += kWarps) {
-      const int t0 = c * kChunk;
-      if (t0 >= rows) break;
-      const int nt = min(kChunk, rows - t0);
-      // ---- logits: kLPT lanes per token, TPP tokens per pass
+    if (rows > 0) {
+      const bool ready = mbar_wait(ctx, &full_bar[st], (phase_bits >> st) & 1u);
+      phase_bits ^= 1u << st;
+      if (tid == 0) pending &= ~(1u << st);
+      if (!__all_sync(0xffffffffu, ready)) {
+        if (lane == 0) s_abort = 1;
+      } else {
+        const T* ks = reinterpret_cast<const T*>(stage_mem) + st * stage_elems;
+        const T* vs = ks + (size_t)s.b * D;
+        const float bias = (!s.dense && s.use_gates && sl0 + i < s.K)
+                               ? logf(gates[(long long)unit * s.C + m]) : 0.f;
+        for (int c = w; c < cpb; c += kWarps) {
+          const int t0 = c * kChunk;
+          if (t0 >= rows) break;
+          const int nt = min(kChunk, rows - t0);
+          // ---- logits: kLPT lanes per token, TPP tokens per pass
 #pragma unroll
-      for (int pass = 0; pass < kChunk / TPP; ++pass) {
-        const int tt = pass * TPP + lane / kLPT;
-        float dot[G];
+          for (int pass = 0; pass < kChunk / TPP; ++pass) {
+            const int tt = pass * TPP + lane / kLPT;
+            float dot[G];
 #pragma unroll
-        for (int g = 0; g < G; ++g) dot[g] = 0.f;
-        if (tt < nt) {
-          float kf[VPL];
-          lds_f<T, VPL>(ks + (size_t)(t0 + tt) * D + dseg, kf);
+            for (int g = 0; g < G; ++g) dot[g] = 0.f;
+            if (tt < nt) {
+              float kf[VPL];
+              lds_f<T, VPL>(ks + (size_t)(t0 + tt) * D + dseg, kf);
 #pragma unroll
-          for (int g = 0; g < G; ++g)
+              for (int g = 0; g < G; ++g)
 #pragma unroll
-            for (int x = 0; x < VPL; ++x) dot[g] = fmaf(qr[g][x], kf[x], dot[g]);
-        }
+                for (int x = 0; x < VPL; ++x) dot[g] = fmaf(qr[g][x], kf[x], dot[g]);
+            }
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
+            for (int g = 0; g < G; ++g) {
 #pragma unroll
-          for (int off = kLPT / 2; off > 0; off >>= 1)
-            dot[g] += __shfl_xor_sync(0xffffffffu, dot[g], off);
-        }
-        if ((lane % kLPT) == 0) {
+              for (int off = kLPT / 2; off > 0; off >>= 1)
+                dot[g] += __shfl_xor_sync(0xffffffffu, dot[g], off);
+            }
+            if ((lane % kLPT) == 0) {
 #pragma unroll
-          for (int g = 0; g < G; ++g) s_x[w][g][tt] = (tt < nt) ? dot[g] + bias : -INFINITY;
-        }
-      }
-      __syncwarp();
-      // ---- online softmax: lane t < kChunk owns token t
+              for (int g = 0; g < G; ++g) s_x[w][g][tt] = (tt < nt) ? dot[g] + bias : -INFINITY;
+            }
+          }
+          __syncwarp();
+          // ---- online softmax: lane t < kChunk owns token t
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float x = (lane < kChunk) ? s_x[w][g][lane] : -INFINITY;
-        const float mx = warp_max(x);
-        const float mnew = fmaxf(m_run[g], mx);
-        const float p = (mnew == -INFINITY) ? 0.f : expf(x - mnew);
-        const float alpha = (mnew == -INFINITY) ? 1.f : expf(m_run[g] - mnew);
-        l_run[g] = l_run[g] * alpha + warp_sum(p);
-        m_run[g] = mnew;
-        if (lane < kChunk) s_p[w][lane][g] = p;
+          for (int g = 0; g < G; ++g) {
+            const float x = (lane < kChunk) ? s_x[w][g][lane] : -INFINITY;
+            const float mx = warp_max(x);
+            const float mnew = fmaxf(m_run[g], mx);
+            const float p = (mnew == -INFINITY) ? 0.f : expf(x - mnew);
+            const float alpha = (mnew == -INFINITY) ? 1.f : expf(m_run[g] - mnew);
+            l_run[g] = l_run[g] * alpha + warp_sum(p);
+            m_run[g] = mnew;
+            if (lane < kChunk) s_p[w][lane][g] = p;
 #pragma unroll
-        for (int x2 = 0; x2 < DPL; ++x2) acc[g][x2] *= alpha;
-      }
-      __syncwarp();
-      // ---- o += p v: lane owns DPL consecutive dims
+            for (int x2 = 0; x2 < DPL; ++x2) acc[g][x2] *= alpha;
+          }
+          __syncwarp();
+          // ---- o += p v: lane owns DPL consecutive dims
 #pragma unroll 4
-      for (int t = 0; t < nt; ++t) {
-        float vf[DPL];
-        lds_f<T, DPL>(vs + (size_t)(t0 + t) * D + lane * DPL, vf);
+          for (int t = 0; t < nt; ++t) {
+            float vf[DPL];
+            lds_f<T, DPL>(vs + (size_t)(t0 + t) * D + lane * DPL, vf);
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float p = s_p[w][t][g];
+            for (int g = 0; g < G; ++g) {
+              const float p = s_p[w][t][g];
 #pragma unroll
-          for (int x2 = 0; x2 < DPL; ++x2) acc[g][x2] = fmaf(p, vf[x2], acc[g][x2]);
+              for (int x2 = 0; x2 < DPL; ++x2) acc[g][x2] = fmaf(p, vf[x2], acc[g][x2]);
+            }
+          }
+          __syncwarp();
         }
       }
-      __syncwarp();
     }
-    __syncthreads();  // stage st is free
-    if (tid == 0 && i + nst < ns) issue(i + nst);
+    __syncthreads();  // stage st is free; s_abort is visible
+    if (s_abort) break;
+    if (tid == 0 && i + nst < ns && issue(i + nst)) pending |= 1u << st;
+  }
+  if (s_abort) {
+    // A copy never arrived: stop, let the copies still in flight land (bounded
+    // waits), and leave without a partial; the error word reports it.
+    if (tid == 0)
+      for (int st = 0; st < nst; ++st)
+        if (pending & (1u << st)) (void)mbar_wait(ctx, &full_bar[st], (phase_bits >> st) & 1u);
+    return;
   }
 
   // ---- merge the warps of this CTA

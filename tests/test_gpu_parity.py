@@ -220,3 +220,25 @@ def test_wait_timeout_is_reported(cuda_lib):
     # the context stays usable
     x = torch.ones(4, device="cuda")
     assert float((x * 2).sum()) == 8.0
+
+
+def test_decode_idx_with_holes(cuda_lib):
+    """-1 entries anywhere in an idx row are skipped (decode and oracle alike)."""
+    dc = W.small_decode_config(B=2, Hq=8, Hkv=2, L=3000, d=128, b=64, K=12, dtype="bf16")
+    x = W.make_decode_inputs(dc)
+    s = x.scores[:, :, None, :]
+    og, olg, oi = O.gate_topk(s, dc.K, causal=False)
+    oi = oi.copy()
+    oi[0, 0, 0, 3] = -1
+    oi[1, 1, 0, 0] = -1
+    oi[1, 0, 0, 5:9] = -1
+    q, kc, vc = (dev(a, "bf16") for a in (x.q, x.kcache, x.vcache))
+    idx = torch.from_numpy(oi[:, :, 0].copy()).cuda()
+    gates = dev(og[:, :, 0].astype(np.float32), "f32")
+    for use_gates in (False, True):
+        o = cuda_lib.decode(q, kc, vc, idx, gates, use_gates, dc.b, L=dc.L)
+        torch.cuda.synchronize()
+        assert cuda_lib.device_error()[0] == 0
+        lg = np.log(og[:, :, 0].astype(np.float32).astype(np.float64))
+        want = O.decode(x.q, x.kcache, x.vcache, oi[:, :, 0], lg, dc.b, use_gates=use_gates)
+        check("decode o (holes)", host(o), want, "bf16")
