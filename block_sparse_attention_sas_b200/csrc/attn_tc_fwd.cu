@@ -1,0 +1,414 @@
+// Gated block-sparse causal attention, forward, on the sm_100a tensor cores
+// (bf16 inputs, fp32 accumulation; head dim 128, block size 64, G = 2 or 4
+// query heads per KV head).
+//
+// What it computes (picx.dev SAS summary, Methodology Eq. 9 and Kernel
+// Design; reproduction README, Core equations for the 1/sqrt(d) scale): for
+// query block j of KV head kvh, o = softmax(q K_S^T / sqrt(d) + log g_S) V_S
+// over the selected history blocks (bias log g_m) and the current block
+// (bias 0, causal), with an online softmax so the attention matrix is never
+// stored.
+//
+// One CTA per (query block j, KV head, batch). The G heads' 64 rows stack
+// into G*64/128 M-tiles of 128 rows that share every K/V block:
+//   warp 0      TMA producer: Q once, then each attended K/V block (64 keys x
+//               128 dims, 32 KB) into a two-stage ring
+//   warp 1      MMA issuer: S_t = Q_t K^T into TMEM (double-buffered, 64
+//               columns per tile), then O_t += P_t V (128 columns per tile)
+//   warps 4-11  softmax, one warpgroup per M-tile, one thread per query row:
+//               S from TMEM, scale + log-gate bias + causal mask, running max
+//               (O rescaled in TMEM only when the max grows by more than 2^8),
+//               P as bf16 into swizzled shared memory for the PV MMA; at the
+//               end O / l and the log-sum-exp go to global memory.
+// Every wait is bounded; a wait that runs out sets the error word and a
+// CTA-wide abort flag, the roles drain their in-flight work and the CTA exits.
+#include <math.h>
+
+#include "sas_internal.h"
+#include "tc_common.cuh"
+
+namespace sas {
+namespace {
+
+using namespace tc;
+
+constexpr int kD = 128;          // head dim
+constexpr int kB = 64;           // block size (keys per K/V block, rows per head)
+constexpr int kThreads = 384;    // 12 warps
+constexpr int kFirstSoftmaxWarp = 4;
+constexpr int kStages = 2;
+constexpr uint32_t kTmemCols = 512;
+
+// Shared-memory carve-up (offsets from a 1024-byte aligned base).
+constexpr uint32_t kQBytes = 2 * 2 * 128 * 128;     // [tile][k half][128 rows][128 B]
+constexpr uint32_t kKVStageBytes = 4 * 64 * 128;    // K halves then V halves
+constexpr uint32_t kPBytes = 2 * 2 * 128 * 128;     // [tile][buffer][128 rows][128 B]
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffKV = kOffQ + kQBytes;
+constexpr uint32_t kOffP = kOffKV + kStages * kKVStageBytes;
+constexpr uint32_t kOffCtl = kOffP + kPBytes;       // barriers and the block list
+constexpr int kMaxList = 257;                        // K <= 256 selected + current
+
+struct Ctl {
+  uint64_t q_full;
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t s_full[2][2], s_free[2][2], p_full[2][2], pv_done[2][2];
+  uint64_t drain;  // abort path only: the MMA thread's last commit
+  uint32_t tmem_base;
+  int abort;
+  int nblk;
+  int blocks[kMaxList];
+  float bias[kMaxList];  // log2-domain gate bias of each attended block
+};
+constexpr size_t kSmemBytes = kOffCtl + sizeof(Ctl) + 1024;  // + alignment slack
+
+// TMEM columns: S[tile][buffer] at tile*128 + buffer*64; O[tile] at 256 + tile*128.
+__device__ __forceinline__ uint32_t s_col(int t, int b) { return t * 128 + b * 64; }
+__device__ __forceinline__ uint32_t o_col(int t) { return 256 + t * 128; }
+
+template <int TILES>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ idx,
+              const float* __restrict__ gates, AttnShape s, __nv_bfloat16* __restrict__ o,
+              float* __restrict__ lse, DevCtx ctx) {
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  unsigned char* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const uint32_t sbase = smem_u32(base);
+  Ctl& c = *reinterpret_cast<Ctl*>(base + kOffCtl);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int j = blockIdx.x, kvh = blockIdx.y, bi = blockIdx.z;
+  const int G = 2 * TILES;
+  const long long irow = ((long long)(bi * s.Hkv + kvh) * s.N + j);
+
+  if (tid == 0) {
+    mbar_init(&c.q_full, 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&c.kv_full[i], 1);
+      mbar_init(&c.kv_empty[i], 1);
+    }
+    for (int t = 0; t < 2; ++t)
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&c.s_full[t][b], 1);
+        mbar_init(&c.s_free[t][b], 128);
+        mbar_init(&c.p_full[t][b], 128);
+        mbar_init(&c.pv_done[t][b], 1);
+      }
+    mbar_init(&c.drain, 1);
+    fence_mbar_init();
+    c.abort = 0;
+    // Attended blocks in order: the selected history blocks, then block j.
+    int n = 0;
+    for (int sl = 0; sl < s.K; ++sl) {
+      const int m = idx[irow * s.K + sl];
+      if (m < 0) continue;
+      if (m >= j) {
+        report(ctx, kDevErrBadIndex);
+        continue;
+      }
+      c.blocks[n] = m;
+      c.bias[n] = gates ? logf(gates[irow * s.N + m]) * kLog2e : 0.f;
+      ++n;
+    }
+    c.blocks[n] = j;
+    c.bias[n] = 0.f;
+    c.nblk = n + 1;
+  }
+  if (warp == 1) {
+    tmem_alloc(&c.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = c.tmem_base;
+  const int nblk = c.nblk;
+  volatile int* abort = &c.abort;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(&c.q_full, TILES * 4 * 64 * 128);
+      for (int t = 0; t < TILES; ++t)
+        for (int hh = 0; hh < 2; ++hh)
+          for (int kb = 0; kb < 2; ++kb)
+            tma_load_3d(base + kOffQ + t * 32768 + kb * 16384 + hh * 8192, &tm_q, kb * 64, j * kB,
+                        bi * s.Hq + kvh * G + 2 * t + hh, &c.q_full);
+      int issued = 0;
+      for (int n = 0; n < nblk; ++n) {
+        const int st = n & 1;
+        if (n >= kStages && !wait_or_abort(ctx, &c.kv_empty[st], ((n - kStages) >> 1) & 1, abort))
+          break;
+        const int m = c.blocks[n];
+        unsigned char* kv = base + kOffKV + st * kKVStageBytes;
+        mbar_arrive_expect_tx(&c.kv_full[st], kKVStageBytes);
+        for (int h2 = 0; h2 < 2; ++h2)
+          tma_load_3d(kv + h2 * 8192, &tm_k, h2 * 64, m * kB, bi * s.Hkv + kvh, &c.kv_full[st]);
+        for (int h2 = 0; h2 < 2; ++h2)
+          tma_load_3d(kv + 16384 + h2 * 8192, &tm_v, h2 * 64, m * kB, bi * s.Hkv + kvh,
+                      &c.kv_full[st]);
+        issued = n + 1;
+      }
+      if (*abort) {
+        // Let the loads still in flight land before the CTA's memory is released.
+        (void)mbar_wait(ctx, &c.q_full, 0);
+        for (int n = max(0, issued - kStages); n < issued; ++n)
+          (void)mbar_wait(ctx, &c.kv_full[n & 1], (n >> 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16(128, 64, false, false);
+      const uint32_t id_o = idesc_bf16(128, 128, false, true);
+      bool ok = wait_or_abort(ctx, &c.q_full, 0, abort);
+      fence_after_sync();
+      auto issue_s = [&](int n) -> bool {
+        const int st = n & 1, b = n & 1;
+        if (!wait_or_abort(ctx, &c.kv_full[st], (n >> 1) & 1, abort)) return false;
+        for (int t = 0; t < TILES; ++t) {
+          if (n >= 2 && !wait_or_abort(ctx, &c.s_free[t][b], ((n - 2) >> 1) & 1, abort))
+            return false;
+          fence_after_sync();
+          const uint32_t qa = sbase + kOffQ + t * 32768;
+          const uint32_t ka = sbase + kOffKV + st * kKVStageBytes;
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+            const uint32_t koff = (ks >> 2) * 8192 + (ks & 3) * 32;
+            mma_bf16_ss(tmem + s_col(t, b), sdesc_sw128(qa + off, 16, 1024),
+                        sdesc_sw128(ka + koff, 16, 1024), id_s, ks > 0);
+          }
+          mma_commit(&c.s_full[t][b]);
+        }
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int n = 0; ok && n < nblk; ++n) {
+        if (n + 1 < nblk && !issue_s(n + 1)) break;
+        const int st = n & 1, b = n & 1;
+        for (int t = 0; t < TILES; ++t) {
+          if (!wait_or_abort(ctx, &c.p_full[t][b], (n >> 1) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          fence_after_sync();
+          const uint32_t pa = sbase + kOffP + (t * 2 + b) * 16384;
+          const uint32_t va = sbase + kOffKV + st * kKVStageBytes + 16384;
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_bf16_ss(tmem + o_col(t), sdesc_sw128(pa + ks * 32, 16, 1024),
+                        sdesc_sw128(va + ks * 2048, 8192, 1024), id_o, (n > 0 || ks > 0));
+          mma_commit(&c.pv_done[t][b]);
+        }
+        if (!ok) break;
+        mma_commit(&c.kv_empty[st]);
+      }
+      if (*abort) {
+        // MMAs already issued must finish before TMEM is released.
+        mma_commit(&c.drain);
+        (void)mbar_wait(ctx, &c.drain, 0);
+      }
+    }
+  } else if (warp >= kFirstSoftmaxWarp) {
+    // ------------------------------------------------------------ softmax
+    const int t = (warp - kFirstSoftmaxWarp) >> 2;
+    const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
+    const int rowi = quarter * 32 + lane;         // row of the M-tile (TMEM lane)
+    const int hh = rowi >> 6, r = rowi & 63;
+    const int head = kvh * G + 2 * t + hh;
+    const int qrow = j * kB + r;
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    const float sc = s.scale * kLog2e;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = t < TILES;
+    for (int n = 0; ok && n < nblk; ++n) {
+      const int b = n & 1;
+      if (!__all_sync(0xffffffffu, wait_or_abort(ctx, &c.s_full[t][b], (n >> 1) & 1, abort))) {
+        ok = false;
+        break;
+      }
+      fence_after_sync();
+      uint32_t sr[64];
+      tmem_ld32(tl + s_col(t, b), *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tl + s_col(t, b) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld_wait();
+      fence_before_sync();
+      mbar_arrive(&c.s_free[t][b]);
+
+      const int m = c.blocks[n];
+      const float bias = c.bias[n];
+      const bool cur = (n == nblk - 1);
+      const int kvalid = min(kB, s.T - m * kB);   // keys of the block inside the sequence
+      float x[64];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        float v = fmaf(__uint_as_float(sr[i]), sc, bias);
+        if (i >= kvalid || (cur && i > r)) v = -INFINITY;
+        x[i] = v;
+        mx = fmaxf(mx, v);
+      }
+      const float m_new = fmaxf(m_used, mx);
+      // Rows whose max grew by more than 2^8 rescale O (and l); the TMEM
+      // load/store is warp-wide, so the warp does it if any of its rows must.
+      const bool grow = m_new > m_used + 8.f;
+      const bool need = grow && n > 0 && m_used != -INFINITY;
+      if (__any_sync(0xffffffffu, need)) {
+        const float alpha = need ? ex2(m_used - m_new) : 1.f;
+        if (!__all_sync(0xffffffffu, wait_or_abort(ctx, &c.pv_done[t][(n - 1) & 1],
+                                                   ((n - 1) >> 1) & 1, abort))) {
+          ok = false;
+          break;
+        }
+        fence_after_sync();
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t ov[32];
+          tmem_ld32(tl + o_col(t) + ch * 32, ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          tmem_st32(tl + o_col(t) + ch * 32, ov);
+        }
+        tmem_st_wait();
+        l *= alpha;
+      }
+      if (grow) m_used = m_new;
+      float rs = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float p0 = (m_used == -INFINITY) ? 0.f : ex2(x[2 * i] - m_used);
+        const float p1 = (m_used == -INFINITY) ? 0.f : ex2(x[2 * i + 1] - m_used);
+        rs += p0 + p1;
+        pk[i] = pack_bf16(p0, p1);
+      }
+      l += rs;
+      // P buffer b is free once PV(n-2) has completed.
+      if (n >= 2 &&
+          !__all_sync(0xffffffffu, wait_or_abort(ctx, &c.pv_done[t][b], ((n - 2) >> 1) & 1, abort))) {
+        ok = false;
+        break;
+      }
+      unsigned char* prow = base + kOffP + (t * 2 + b) * 16384 + rowi * 128;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        uint4 v = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        *reinterpret_cast<uint4*>(prow + ((ch ^ (rowi & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      fence_before_sync();
+      mbar_arrive(&c.p_full[t][b]);
+    }
+    if (ok && t < TILES) {
+      // ---- epilogue: O / l and the log-sum-exp
+      const int nl = nblk - 1;
+      if (__all_sync(0xffffffffu, wait_or_abort(ctx, &c.pv_done[t][nl & 1], (nl >> 1) & 1, abort))) {
+        fence_after_sync();
+        const float inv = 1.f / l;
+        const bool write = qrow < s.T;
+        __nv_bfloat16* orow = o + ((long long)(bi * s.Hq + head) * s.T + qrow) * kD;
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t ov[32];
+          tmem_ld32(tl + o_col(t) + ch * 32, ov);
+          tmem_ld_wait();
+          if (write) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              uint4 v;
+              v.x = pack_bf16(__uint_as_float(ov[8 * q4 + 0]) * inv, __uint_as_float(ov[8 * q4 + 1]) * inv);
+              v.y = pack_bf16(__uint_as_float(ov[8 * q4 + 2]) * inv, __uint_as_float(ov[8 * q4 + 3]) * inv);
+              v.z = pack_bf16(__uint_as_float(ov[8 * q4 + 4]) * inv, __uint_as_float(ov[8 * q4 + 5]) * inv);
+              v.w = pack_bf16(__uint_as_float(ov[8 * q4 + 6]) * inv, __uint_as_float(ov[8 * q4 + 7]) * inv);
+              *reinterpret_cast<uint4*>(orow + ch * 32 + q4 * 8) = v;
+            }
+          }
+        }
+        if (write) lse[(long long)(bi * s.Hq + head) * s.T + qrow] = (m_used + log2f(l)) * kLn2;
+      }
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after_sync();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+}  // namespace
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (the library
+// does not link libcuda).
+static EncodeTiled encode_fn() {
+  static EncodeTiled fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(p);
+  }
+  return fn;
+}
+
+// 3-D map over a [planes][rows][128] bf16 tensor, 64x64 boxes, 128-byte swizzle.
+cudaError_t make_tmap_bf16(CUtensorMap* map, const void* ptr, int rows, int planes) {
+  EncodeTiled enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)rows, (cuuint64_t)planes};
+  const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)rows * kD * 2};
+  const cuuint32_t box[3] = {64, 64, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+bool tc_fwd_supported(sas_dtype_t dt, const AttnShape& s) {
+  const int G = s.Hq / s.Hkv;
+  return dt == SAS_BF16 && s.d == kD && s.b == kB && (G == 2 || G == 4) && !s.dense;
+}
+
+cudaError_t launch_attn_fwd_tc(const AttnShape& s, const void* q, const void* k, const void* v,
+                               const int32_t* idx, const float* gates, void* o, float* lse,
+                               const DevCtx& ctx, cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  cudaError_t e;
+  if ((e = make_tmap_bf16(&tq, q, s.T, s.B * s.Hq)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&tk, k, s.T, s.B * s.Hkv)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&tv, v, s.T, s.B * s.Hkv)) != cudaSuccess) return e;
+  const int G = s.Hq / s.Hkv;
+  dim3 grid(s.N, s.Hkv, s.B);
+  if (G == 4) {
+    auto kern = tc_fwd_kernel<2>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, idx, gates, s, (__nv_bfloat16*)o, lse,
+                                             ctx);
+  } else {
+    auto kern = tc_fwd_kernel<1>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, idx, gates, s, (__nv_bfloat16*)o, lse,
+                                             ctx);
+  }
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace sas

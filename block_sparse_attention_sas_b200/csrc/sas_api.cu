@@ -218,6 +218,8 @@ sas_status_t sas_attn_fwd(sas_dtype_t dtype, const void* q, const void* k, const
   DevCtx ctx;
   if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
   const AttnShape s = make_shape(B, Hq, Hkv, T, d, b, K, scale, false);
+  if (tc_fwd_supported(dtype, s))
+    return cuda_status(launch_attn_fwd_tc(s, q, k, v, idx, gates, o, lse, ctx, stream));
   return cuda_status(launch_attn_fwd_simt(dtype, s, q, k, v, idx, gates, o, lse, ctx, stream));
 }
 

@@ -36,6 +36,12 @@ BwdWorkspace bwd_workspace_layout(const AttnShape& s);
 cudaError_t launch_attn_fwd_simt(sas_dtype_t dt, const AttnShape& s, const void* q, const void* k,
                                  const void* v, const int32_t* idx, const float* gates, void* o,
                                  float* lse, const DevCtx& ctx, cudaStream_t stream);
+// Tensor-core (tcgen05) forward: bf16, d = 128, b = 64, G in {2, 4}.
+bool tc_fwd_supported(sas_dtype_t dt, const AttnShape& s);
+cudaError_t launch_attn_fwd_tc(const AttnShape& s, const void* q, const void* k, const void* v,
+                               const int32_t* idx, const float* gates, void* o, float* lse,
+                               const DevCtx& ctx, cudaStream_t stream);
+
 cudaError_t launch_attn_bwd_simt(sas_dtype_t dt, const AttnShape& s, const void* q, const void* k,
                                  const void* v, const void* o, const float* lse, const void* dO,
                                  const int32_t* idx, const float* gates, void* dq, void* dk,
