@@ -639,6 +639,26 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 }  // namespace
 
+cudaError_t launch_bwd_csr(const AttnShape& s, const int32_t* idx, int32_t* off, int32_t* list,
+                           const DevCtx& ctx, cudaStream_t st) {
+  const size_t smem = 2 * sizeof(int32_t) * (size_t)s.N;
+  cudaError_t e =
+      cudaFuncSetAttribute(csr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  csr_kernel<<<s.B * s.Hkv, kThreads, smem, st>>>(idx, s, off, list, ctx);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_jacobian(const AttnShape& s, const float* da, const int32_t* idx,
+                                const float* gates, float* dscores, cudaStream_t st) {
+  const long long srows = (long long)s.B * s.Hkv * s.N;
+  jacobian_kernel<<<(unsigned)((srows + kWarps - 1) / kWarps), kThreads, 0, st>>>(
+      da, idx, gates, s, 1, dscores);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
 BwdWorkspace bwd_workspace_layout(const AttnShape& s) {
   BwdWorkspace L;
   const int RC = s.b < 64 ? 1 : s.b / 64;

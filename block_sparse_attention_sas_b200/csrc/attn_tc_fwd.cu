@@ -366,7 +366,8 @@ static EncodeTiled encode_fn() {
 }
 
 // 3-D map over a [planes][rows][128] bf16 tensor, 64x64 boxes, 128-byte swizzle.
-cudaError_t make_tmap_bf16(CUtensorMap* map, const void* ptr, int rows, int planes) {
+cudaError_t make_tmap_bf16(void* map_out, const void* ptr, int rows, int planes) {
+  CUtensorMap* map = static_cast<CUtensorMap*>(map_out);
   EncodeTiled enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)rows, (cuuint64_t)planes};

@@ -249,6 +249,9 @@ sas_status_t sas_attn_bwd(sas_dtype_t dtype, const void* q, const void* k, const
   if (!ws || ws_bytes < need || !aligned(ws, 256)) return SAS_ERR_WORKSPACE;
   DevCtx ctx;
   if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
+  if (tc_bwd_supported(dtype, s))
+    return cuda_status(launch_attn_bwd_tc(s, q, k, v, lse, dO, idx, gates, dq, dk, dv, dscores,
+                                          ws, ctx, stream));
   return cuda_status(launch_attn_bwd_simt(dtype, s, q, k, v, o, lse, dO, idx, gates, dq, dk, dv,
                                           dscores, ws, ctx, stream));
 }

@@ -42,6 +42,20 @@ cudaError_t launch_attn_fwd_tc(const AttnShape& s, const void* q, const void* k,
                                const int32_t* idx, const float* gates, void* o, float* lse,
                                const DevCtx& ctx, cudaStream_t stream);
 
+// Tensor-core (tcgen05) backward for the same shapes as the forward.
+bool tc_bwd_supported(sas_dtype_t dt, const AttnShape& s);
+cudaError_t launch_attn_bwd_tc(const AttnShape& s, const void* q, const void* k, const void* v,
+                               const float* lse, const void* dO, const int32_t* idx,
+                               const float* gates, void* dq, void* dk, void* dv, float* dscores,
+                               void* ws, const DevCtx& ctx, cudaStream_t stream);
+// Shared pieces of the backward (defined with the SIMT kernels).
+cudaError_t launch_bwd_csr(const AttnShape& s, const int32_t* idx, int32_t* off, int32_t* list,
+                           const DevCtx& ctx, cudaStream_t stream);
+cudaError_t launch_bwd_jacobian(const AttnShape& s, const float* da, const int32_t* idx,
+                                const float* gates, float* dscores, cudaStream_t stream);
+// 3-D TMA map over a [planes][rows][128] bf16 tensor, 64x64 boxes, 128-byte swizzle.
+cudaError_t make_tmap_bf16(void* map, const void* ptr, int rows, int planes);
+
 cudaError_t launch_attn_bwd_simt(sas_dtype_t dt, const AttnShape& s, const void* q, const void* k,
                                  const void* v, const void* o, const float* lse, const void* dO,
                                  const int32_t* idx, const float* gates, void* dq, void* dk,
