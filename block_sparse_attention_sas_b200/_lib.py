@@ -42,6 +42,9 @@ SIGNATURES = {
     "sas_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "sas_decode": (_i, [_i, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p,
                         _sz, _p]),
+    "sas_decode_noalloc": (_i, [_i, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f,
+                                _p, _p]),
+    "sas_decode_noalloc_max_scratch": (_sz, []),
     "sas_dense_fwd": (_i, [_i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p]),
     "sas_dense_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "sas_dense_bwd": (_i, [_i, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p,
@@ -188,6 +191,25 @@ def decode(q, kcache, vcache, idx, gates, use_gates: bool, b: int, L: int | None
     _check("sas_decode", LIB.sas_decode(_dtype(q), _ptr(q), _ptr(kcache), _ptr(vcache), _ptr(idx),
                                         _ptr(gates), int(use_gates), B, Hq, Hkv, L, Lcap, d, b, K,
                                         scale, _ptr(o), _ptr(ws), ws.numel(), _stream(q.device)))
+    return o
+
+
+def decode_noalloc(q, kcache, vcache, idx, gates, use_gates: bool, b: int,
+                   L: int | None = None, scale: float = 0.0, o=None):
+    """sas_decode without a workspace: the library's fixed device scratch is
+    used instead (see include/sas.h for who needs this and its limits)."""
+    for n, t in (("q", q), ("kcache", kcache), ("vcache", vcache)):
+        _need(t, n, q.dtype)
+    _need(idx, "idx", torch.int32)
+    B, Hq, d = q.shape
+    Hkv, Lcap = kcache.shape[1], kcache.shape[2]
+    L = Lcap if L is None else L
+    if o is None:
+        o = torch.empty_like(q)
+    _check("sas_decode_noalloc",
+           LIB.sas_decode_noalloc(_dtype(q), _ptr(q), _ptr(kcache), _ptr(vcache), _ptr(idx),
+                                  _ptr(gates), int(use_gates), B, Hq, Hkv, L, Lcap, d, b,
+                                  idx.shape[-1], scale, _ptr(o), _stream(q.device)))
     return o
 
 

@@ -17,6 +17,8 @@
 // partials by log-sum-exp, writes o, and resets the ticket to zero.
 #include <math.h>
 
+#include <mutex>
+
 #include "sas_common.cuh"
 #include "sas_internal.h"
 
@@ -463,6 +465,39 @@ size_t decode_workspace_bytes(const DecodeShape& s) {
   const size_t b = (parts * s.d * sizeof(float) + 255) & ~(size_t)255;
   const size_t c = ((size_t)s.B * s.Hkv * sizeof(uint32_t) + 255) & ~(size_t)255;
   return a + b + c;
+}
+
+// ---------------------------------------------------------------------------
+// Scratch for decode calls that must not allocate: a fixed array in device
+// memory, present on every device that loads the library until the process
+// exits. Its address is looked up once per device (with that device current);
+// in host code the array's name is only a host-side handle, never a pointer
+// the GPU can use.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(2) << 20;  // 2 MiB
+static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
+std::mutex g_scratch_mu;
+constexpr int kMaxScratchDevices = 64;
+void* g_scratch_ptr[kMaxScratchDevices] = {nullptr};
+}  // namespace
+
+size_t decode_noalloc_capacity() { return kNoAllocScratchBytes; }
+
+cudaError_t decode_noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxScratchDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
 }
 
 cudaError_t launch_decode(sas_dtype_t dt, const DecodeShape& s, const void* q, const void* kc,

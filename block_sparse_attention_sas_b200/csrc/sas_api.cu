@@ -281,6 +281,32 @@ sas_status_t sas_decode(sas_dtype_t dtype, const void* q, const void* kcache, co
   return cuda_status(launch_decode(dtype, s, q, kcache, vcache, idx, gates, o, ws, ctx, stream));
 }
 
+sas_status_t sas_decode_noalloc(sas_dtype_t dtype, const void* q, const void* kcache,
+                                const void* vcache, const int32_t* idx, const float* gates,
+                                int use_gates, int B, int Hq, int Hkv, int L, int Lcap, int d,
+                                int b, int K, float scale, void* o, sas_stream_t stream) {
+  sas_status_t st = check_decode(dtype, B, Hq, Hkv, L, Lcap, d, b, K, false, scale);
+  if (st != SAS_OK) return st;
+  if (B == 0) return SAS_OK;
+  if (!q || !kcache || !vcache || !idx || !o) return SAS_ERR_INVALID_ARG;
+  if (use_gates && !gates && (L - 1) / b > 0) return SAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(kcache, 16) || !aligned(vcache, 16) || !aligned(o, 16) ||
+      !aligned(idx, 4) || (gates && !aligned(gates, 4)))
+    return SAS_ERR_INVALID_ARG;
+  const DecodeShape s = make_decode(B, Hq, Hkv, L, Lcap, d, b, K, scale, false, use_gates);
+  void* scratch = nullptr;
+  if (s.splits > 1) {
+    if (decode_workspace_bytes(s) > decode_noalloc_capacity()) return SAS_ERR_WORKSPACE;
+    if (decode_noalloc_scratch(&scratch) != cudaSuccess) return SAS_ERR_CUDA;
+  }
+  DevCtx ctx;
+  if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
+  return cuda_status(
+      launch_decode(dtype, s, q, kcache, vcache, idx, gates, o, scratch, ctx, stream));
+}
+
+size_t sas_decode_noalloc_max_scratch(void) { return decode_noalloc_capacity(); }
+
 sas_status_t sas_dense_fwd(sas_dtype_t dtype, const void* q, const void* k, const void* v, int B,
                            int Hq, int Hkv, int T, int d, int b, float scale, void* o, float* lse,
                            sas_stream_t stream) {

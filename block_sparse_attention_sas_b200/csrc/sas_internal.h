@@ -78,6 +78,10 @@ cudaError_t launch_decode(sas_dtype_t dt, const DecodeShape& s, const void* q, c
                           const void* vc, const int32_t* idx, const float* gates, void* o,
                           void* ws, const DevCtx& ctx, cudaStream_t stream);
 
+// Fixed-size device scratch for sas_decode_noalloc (no allocation involved).
+size_t decode_noalloc_capacity();
+cudaError_t decode_noalloc_scratch(void** out);
+
 cudaError_t launch_wait_selftest(const DevCtx& ctx, cudaStream_t stream);
 
 }  // namespace sas

@@ -174,6 +174,36 @@ sas_status_t sas_decode(sas_dtype_t dtype, const void* q, const void* kcache, co
                         void* ws, size_t ws_bytes, sas_stream_t stream);
 
 /*
+ * sas_decode_noalloc - sas_decode for callers that cannot allocate device
+ * memory. Some callers cannot call cudaMalloc or take a workspace from their
+ * framework at the point where they decode: an inference server or plugin
+ * whose host framework owns every device allocation and forbids new ones once
+ * serving starts, or a latency-critical loop that cannot afford cudaMalloc's
+ * implicit device synchronisation. This entry point takes the same inputs and
+ * outputs as sas_decode but no workspace: its scratch (the split partials and
+ * merge tickets) lives in a fixed 2 MiB array in device memory, which every
+ * GPU that loads the library holds until the process exits. The paper has no
+ * counterpart; it is a deployment convenience of this library.
+ *   - The call itself allocates nothing: no cudaMalloc, cudaFree or
+ *     allocating library routine. Its first call on a device looks up the
+ *     array's device address (once per device, with that device current);
+ *     make that first call before any stream capture.
+ *   - Every call on a device shares the one array and it keeps the last
+ *     call's contents; the call clears the part that must start at zero.
+ *     Calls that overlap on the GPU (other streams, other host threads) race
+ *     on it: issue them one after another.
+ *   - A problem whose scratch would exceed the array
+ *     (sas_decode_noalloc_max_scratch() bytes; compare with
+ *     sas_decode_workspace_size()) returns SAS_ERR_WORKSPACE before any launch.
+ *   Arguments, layouts and results are those of sas_decode.
+ */
+sas_status_t sas_decode_noalloc(sas_dtype_t dtype, const void* q, const void* kcache,
+                                const void* vcache, const int32_t* idx, const float* gates,
+                                int use_gates, int B, int Hq, int Hkv, int L, int Lcap, int d,
+                                int b, int K, float scale, void* o, sas_stream_t stream);
+size_t sas_decode_noalloc_max_scratch(void);
+
+/*
  * Dense comparison kernels ([picx] Eq. 1 with a causal mask): every block is
  * attended, no gates. Same layouts and conventions as the sparse calls; the
  * block size b only sets the kernels' tiling (use 64 unless d or T call for
