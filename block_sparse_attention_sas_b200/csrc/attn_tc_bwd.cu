@@ -42,13 +42,15 @@ constexpr int kMaxList = 257;
 // Kernel A: dq, D, da
 // ============================================================================
 namespace ka {
+constexpr int kStages = 3;              // K/V ring depth
 constexpr uint32_t kOffQ = 0;            // [k half][128 rows][128 B]
 constexpr uint32_t kOffDO = 32768;       // same layout
-constexpr uint32_t kOffKV = 65536;       // 2 stages x (K halves, V halves) 32 KB
-constexpr uint32_t kOffDS = 131072;      // 2 buffers x [128 rows][128 B]
-constexpr uint32_t kOffCtl = 163840;
+constexpr uint32_t kOffKV = 65536;       // kStages x (K halves, V halves) 32 KB
+constexpr uint32_t kOffDS = kOffKV + kStages * 32768;  // 2 buffers x [128 rows][128 B]
+constexpr uint32_t kOffCtl = kOffDS + 32768;
 struct Ctl {
-  uint64_t qdo_full, kv_full[2], kv_empty[2], s_full[2], s_free[2], ds_full[2], dq_done[2], drain;
+  uint64_t qdo_full, kv_full[kStages], kv_empty[kStages], s_full[2], s_free[2], ds_full[2],
+      dq_done[2], drain;
   uint32_t tmem_base;
   int abort, nblk;
   int blocks[kMaxList], slots[kMaxList];
@@ -81,9 +83,11 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
   if (tid == 0) {
     mbar_init(&c.qdo_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(&c.kv_full[i], 1);
       mbar_init(&c.kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&c.s_full[i], 1);
       mbar_init(&c.s_free[i], 128);
       mbar_init(&c.ds_full[i], 128);
@@ -138,8 +142,10 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
       int issued = 0;
       for (int it = 0; it < nit; ++it) {
-        const int st = it & 1;
-        if (it >= 2 && !wait_or_abort(ctx, &c.kv_empty[st], ((it - 2) >> 1) & 1, abort)) break;
+        const int st = it % kStages;
+        if (it >= kStages &&
+            !wait_or_abort(ctx, &c.kv_empty[st], ((it - kStages) / kStages) & 1, abort))
+          break;
         const int m = c.blocks[it % nblk];
         unsigned char* kv = base + kOffKV + st * 32768;
         mbar_arrive_expect_tx(&c.kv_full[st], 32768);
@@ -152,8 +158,8 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       if (*abort) {
         (void)mbar_wait(ctx, &c.qdo_full, 0);
-        for (int it = max(0, issued - 2); it < issued; ++it)
-          (void)mbar_wait(ctx, &c.kv_full[it & 1], (it >> 1) & 1);
+        for (int it = max(0, issued - kStages); it < issued; ++it)
+          (void)mbar_wait(ctx, &c.kv_full[it % kStages], (it / kStages) & 1);
       }
     }
   } else if (warp == 1) {
@@ -163,8 +169,8 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       bool ok = wait_or_abort(ctx, &c.qdo_full, 0, abort);
       fence_after_sync();
       auto issue_s = [&](int it) -> bool {
-        const int st = it & 1, b = it & 1;
-        if (!wait_or_abort(ctx, &c.kv_full[st], (it >> 1) & 1, abort)) return false;
+        const int st = it % kStages, b = it & 1;
+        if (!wait_or_abort(ctx, &c.kv_full[st], (it / kStages) & 1, abort)) return false;
         if (it >= 2 && !wait_or_abort(ctx, &c.s_free[b], ((it - 2) >> 1) & 1, abort)) return false;
         fence_after_sync();
         const uint32_t kva = sbase + kOffKV + st * 32768;
@@ -190,7 +196,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       for (int it = 0; ok && it < nit; ++it) {
         if (it + 1 < nit && !issue_s(it + 1)) break;
         if (it < nblk) continue;
-        const int i2 = it - nblk, st = it & 1;
+        const int i2 = it - nblk, st = it % kStages;
         if (!wait_or_abort(ctx, &c.ds_full[i2 & 1], (i2 >> 1) & 1, abort)) break;
         fence_after_sync();
         const uint32_t dsa = sbase + kOffDS + (i2 & 1) * 16384;
@@ -227,45 +233,54 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         break;
       }
       fence_after_sync();
-      uint32_t sr[32], pr[32];
       const int n = it % nblk;
       const int m = c.blocks[n];
       const float bias = c.bias[n];
       const bool cur = (n == nblk - 1);
       const int kvalid = min(kB, s.T - m * kB);
       const bool sweep2 = it >= nblk;
-      float rowsum = 0.f;
-      uint32_t pk[32];
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        tmem_ld32(tl + b * 64 + half * 32, sr);
-        tmem_ld32(tl + 128 + b * 64 + half * 32, pr);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float p2[2], d2[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = half * 32 + i + e;
-            float p = ex2(fmaf(__uint_as_float(sr[i + e]), sc, bias) - lse2);
-            if (!live || col >= kvalid || (cur && col > r)) p = 0.f;
-            const float dp = __uint_as_float(pr[i + e]);
-            p2[e] = p;
-            d2[e] = dp;
-          }
-          if (!sweep2) {
-            Dsum = fmaf(p2[0], d2[0], Dsum);
-            Dsum = fmaf(p2[1], d2[1], Dsum);
-          } else {
-            const float ds0 = p2[0] * (d2[0] - Dsum), ds1 = p2[1] * (d2[1] - Dsum);
-            rowsum += ds0 + ds1;
-            pk[half * 16 + i / 2] = pack_bf16(ds0, ds1);
-          }
-        }
-      }
+      uint32_t sr[64], pr[64];
+      tmem_ld32(tl + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tl + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(tl + 128 + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&pr[0]));
+      tmem_ld32(tl + 128 + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&pr[32]));
+      tmem_ld_wait();
       fence_before_sync();
       mbar_arrive(&c.s_free[b]);
-      if (!sweep2) continue;
+      if (cur || kvalid < kB) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (i >= kvalid || (cur && i > r)) sr[i] = __float_as_uint(-INFINITY);
+      }
+      // p = 2^(s*scale + bias - lse2); rows past the sequence contribute nothing.
+      const uint64_t sc2 = f2u(sc, sc);
+      const float off = live ? bias - lse2 : -INFINITY;
+      const uint64_t off2 = f2u(off, off);
+      uint32_t pk[32];
+      uint64_t acc0 = 0, acc1 = 0;
+      const uint64_t negD = f2u(-Dsum, -Dsum);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const uint64_t a2 = ffma2(f2u(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
+                                  sc2, off2);
+        const uint64_t p2 = f2u(ex2(lo_f(a2)), ex2(hi_f(a2)));
+        const uint64_t dp2 = f2u(__uint_as_float(pr[2 * i]), __uint_as_float(pr[2 * i + 1]));
+        if (!sweep2) {
+          if (i & 1) acc1 = ffma2(p2, dp2, acc1);
+          else acc0 = ffma2(p2, dp2, acc0);
+        } else {
+          const uint64_t ds2 = fmul2(p2, fadd2(dp2, negD));
+          if (i & 1) acc1 = fadd2(acc1, ds2);
+          else acc0 = fadd2(acc0, ds2);
+          pk[i] = pack_bf16(lo_f(ds2), hi_f(ds2));
+        }
+      }
+      const uint64_t accs = fadd2(acc0, acc1);
+      if (!sweep2) {
+        Dsum += lo_f(accs) + hi_f(accs);
+        continue;
+      }
+      const float rowsum = lo_f(accs) + hi_f(accs);
       const int i2 = it - nblk;
       // dS buffer (i2 & 1) is free once dQ(i2 - 2) has completed.
       if (i2 >= 2 && !__all_sync(0xffffffffu, wait_or_abort(ctx, &c.dq_done[i2 & 1],
@@ -474,14 +489,10 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
         mma_commit(&c.s_full[b]);
         return true;
       };
-      if (ok) ok = issue_s(0);
-      for (int st_i = 0; ok && st_i < nsteps; ++st_i) {
-        if (st_i + 1 < nsteps && !issue_s(st_i + 1)) break;
-        const int stg = st_i & 1;
-        if (!wait_or_abort(ctx, &c.pds_full, st_i & 1, abort)) break;
+      // dV^T[d][key] += sum_q dO[q][d] P[q][key]; dK^T[d][key] += sum_q Q[q][d] dS[q][key]
+      auto retire = [&](int st_i) {
         fence_after_sync();
-        const uint32_t qa = sbase + kOffQD + stg * 65536;
-        // dV^T[d][key] += sum_q dO[q][d] P[q][key]; dK^T[d][key] += sum_q Q[q][d] dS[q][key]
+        const uint32_t qa = sbase + kOffQD + (st_i & 1) * 65536;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
           mma_bf16_ss(tmem + 256, sdesc_sw128(qa + 32768 + ks * 2048, 16384, 1024),
@@ -493,7 +504,34 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                       sdesc_sw128(sbase + kOffDS + ks * 2048, 8192, 1024), id_t,
                       (st_i > 0 || ks > 0));
         mma_commit(&c.pds_free);
-        mma_commit(&c.qdo_empty[stg]);
+        mma_commit(&c.qdo_empty[st_i & 1]);
+      };
+      if (ok) ok = issue_s(0);
+      // Order by readiness: the next step's S/dP go first when its Q/dO tile
+      // has landed (they then overlap this step's softmax); otherwise this
+      // step's dV/dK go first, which frees the stage that the load after the
+      // next one is waiting for.
+      for (int st_i = 0; ok && st_i < nsteps; ++st_i) {
+        const int nxt = st_i + 1;
+        bool next_issued = nxt >= nsteps;
+        bool retired = false;
+        for (unsigned long long polls = 0; ok && !retired; ++polls) {
+          if (!next_issued && mbar_try_wait(&c.qdo_full[nxt & 1], (nxt >> 1) & 1)) {
+            if (!issue_s(nxt)) ok = false;
+            next_issued = true;
+          }
+          if (ok && mbar_try_wait(&c.pds_full, st_i & 1)) {
+            retire(st_i);
+            retired = true;
+          } else if (polls >= ctx.wait_limit) {
+            report(ctx, kDevErrTimeout);
+            *abort = 1;
+            ok = false;
+          } else if ((polls & 63) == 63 && *abort) {
+            ok = false;
+          }
+        }
+        if (ok && !next_issued && !issue_s(nxt)) ok = false;
       }
       mma_commit(&c.acc_done);
       if (*abort) {
@@ -527,29 +565,32 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       const float bias =
           (cur || gates == nullptr) ? 0.f
                                     : logf(gates[((long long)bh * s.N + j) * s.N + m]) * kLog2e;
-      uint32_t sr[32], pr[32], pp[32], dd[32];
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        tmem_ld32(tl + b * 64 + half * 32, sr);
-        tmem_ld32(tl + 128 + b * 64 + half * 32, pr);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float p2[2], ds2[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = half * 32 + i + e;
-            float p = ex2(fmaf(__uint_as_float(sr[i + e]), sc, bias) - lse2);
-            if (!live || col >= kvalid || (cur && col > r)) p = 0.f;
-            p2[e] = p;
-            ds2[e] = p * (__uint_as_float(pr[i + e]) - Di);
-          }
-          pp[half * 16 + i / 2] = pack_bf16(p2[0], p2[1]);
-          dd[half * 16 + i / 2] = pack_bf16(ds2[0], ds2[1]);
-        }
-      }
+      uint32_t sr[64], pr[64], pp[32], dd[32];
+      tmem_ld32(tl + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tl + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(tl + 128 + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&pr[0]));
+      tmem_ld32(tl + 128 + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&pr[32]));
+      tmem_ld_wait();
       fence_before_sync();
       mbar_arrive(&c.s_free[b]);
+      if (cur || kvalid < kB) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (i >= kvalid || (cur && i > r)) sr[i] = __float_as_uint(-INFINITY);
+      }
+      const uint64_t sc2 = f2u(sc, sc);
+      const float off = live ? bias - lse2 : -INFINITY;
+      const uint64_t off2 = f2u(off, off), negD = f2u(-Di, -Di);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const uint64_t a2 = ffma2(f2u(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
+                                  sc2, off2);
+        const float p0 = ex2(lo_f(a2)), p1 = ex2(hi_f(a2));
+        const uint64_t dp2 = f2u(__uint_as_float(pr[2 * i]), __uint_as_float(pr[2 * i + 1]));
+        const uint64_t ds2 = fmul2(f2u(p0, p1), fadd2(dp2, negD));
+        pp[i] = pack_bf16(p0, p1);
+        dd[i] = pack_bf16(lo_f(ds2), hi_f(ds2));
+      }
       // The P / dS buffers are free once step st_i - 1's dV/dK MMAs completed.
       if (st_i >= 1 && !__all_sync(0xffffffffu,
                                    wait_or_abort(ctx, &c.pds_free, (st_i - 1) & 1, abort))) {

@@ -11,15 +11,17 @@
 //
 // One CTA per (query block j, KV head, batch). The G heads' 64 rows stack
 // into G*64/128 M-tiles of 128 rows that share every K/V block:
-//   warp 0      TMA producer: Q once, then each attended K/V block (64 keys x
-//               128 dims, 32 KB) into a two-stage ring
+//   warps 0, 2  TMA producers: Q once, then the attended blocks' K (warp 0)
+//               and V (warp 2), 16 KB each, into separate three-stage rings
+//               (a K stage frees once S is computed, a V stage once PV is)
 //   warp 1      MMA issuer: S_t = Q_t K^T into TMEM (double-buffered, 64
 //               columns per tile), then O_t += P_t V (128 columns per tile)
 //   warps 4-11  softmax, one warpgroup per M-tile, one thread per query row:
 //               S from TMEM, scale + log-gate bias + causal mask, running max
-//               (O rescaled in TMEM only when the max grows by more than 2^8),
-//               P as bf16 into swizzled shared memory for the PV MMA; at the
-//               end O / l and the log-sum-exp go to global memory.
+//               (O rescaled in TMEM only when the max grows by more than 2^8;
+//               the current block goes first so the max starts high), P as
+//               bf16 into swizzled shared memory for the PV MMA; at the end
+//               O / l and the log-sum-exp go to global memory.
 // Every wait is bounded; a wait that runs out sets the error word and a
 // CTA-wide abort flag, the roles drain their in-flight work and the CTA exits.
 #include <math.h>
@@ -36,23 +38,24 @@ constexpr int kD = 128;          // head dim
 constexpr int kB = 64;           // block size (keys per K/V block, rows per head)
 constexpr int kThreads = 384;    // 12 warps
 constexpr int kFirstSoftmaxWarp = 4;
-constexpr int kStages = 2;
+constexpr int kStages = 3;        // K ring and V ring depth
 constexpr uint32_t kTmemCols = 512;
 
 // Shared-memory carve-up (offsets from a 1024-byte aligned base).
 constexpr uint32_t kQBytes = 2 * 2 * 128 * 128;     // [tile][k half][128 rows][128 B]
-constexpr uint32_t kKVStageBytes = 4 * 64 * 128;    // K halves then V halves
-constexpr uint32_t kPBytes = 2 * 2 * 128 * 128;     // [tile][buffer][128 rows][128 B]
+constexpr uint32_t kKVBytes = 2 * 64 * 128;         // one K or V block: [d half][64 rows][128 B]
+constexpr uint32_t kPBytes = 2 * 128 * 128;         // [tile][128 rows][128 B]
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffKV = kOffQ + kQBytes;
-constexpr uint32_t kOffP = kOffKV + kStages * kKVStageBytes;
+constexpr uint32_t kOffK = kOffQ + kQBytes;
+constexpr uint32_t kOffV = kOffK + kStages * kKVBytes;
+constexpr uint32_t kOffP = kOffV + kStages * kKVBytes;
 constexpr uint32_t kOffCtl = kOffP + kPBytes;       // barriers and the block list
 constexpr int kMaxList = 257;                        // K <= 256 selected + current
 
 struct Ctl {
   uint64_t q_full;
-  uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2][2], s_free[2][2], p_full[2][2], pv_done[2][2];
+  uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
+  uint64_t s_full[2][2], s_free[2][2], p_full[2], pv_done[2];
   uint64_t drain;  // abort path only: the MMA thread's last commit
   uint32_t tmem_base;
   int abort;
@@ -86,21 +89,27 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   if (tid == 0) {
     mbar_init(&c.q_full, 1);
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&c.kv_full[i], 1);
-      mbar_init(&c.kv_empty[i], 1);
+      mbar_init(&c.k_full[i], 1);
+      mbar_init(&c.k_empty[i], 1);
+      mbar_init(&c.v_full[i], 1);
+      mbar_init(&c.v_empty[i], 1);
     }
-    for (int t = 0; t < 2; ++t)
+    for (int t = 0; t < 2; ++t) {
       for (int b = 0; b < 2; ++b) {
         mbar_init(&c.s_full[t][b], 1);
         mbar_init(&c.s_free[t][b], 128);
-        mbar_init(&c.p_full[t][b], 128);
-        mbar_init(&c.pv_done[t][b], 1);
       }
+      mbar_init(&c.p_full[t], 128);
+      mbar_init(&c.pv_done[t], 1);
+    }
     mbar_init(&c.drain, 1);
     fence_mbar_init();
     c.abort = 0;
-    // Attended blocks in order: the selected history blocks, then block j.
-    int n = 0;
+    // Attended blocks in order: block j (bias 0, the largest logits in
+    // expectation), then the selected history blocks.
+    c.blocks[0] = j;
+    c.bias[0] = 0.f;
+    int n = 1;
     for (int sl = 0; sl < s.K; ++sl) {
       const int m = idx[irow * s.K + sl];
       if (m < 0) continue;
@@ -112,9 +121,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       c.bias[n] = gates ? logf(gates[irow * s.N + m]) * kLog2e : 0.f;
       ++n;
     }
-    c.blocks[n] = j;
-    c.bias[n] = 0.f;
-    c.nblk = n + 1;
+    c.nblk = n;
   }
   if (warp == 1) {
     tmem_alloc(&c.tmem_base, kTmemCols);
@@ -127,38 +134,42 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const int nblk = c.nblk;
   volatile int* abort = &c.abort;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || warp == 2) {
+    // ------------------------------------------------------------ producers
     if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(&c.q_full, TILES * 4 * 64 * 128);
-      for (int t = 0; t < TILES; ++t)
-        for (int hh = 0; hh < 2; ++hh)
-          for (int kb = 0; kb < 2; ++kb)
-            tma_load_3d(base + kOffQ + t * 32768 + kb * 16384 + hh * 8192, &tm_q, kb * 64, j * kB,
-                        bi * s.Hq + kvh * G + 2 * t + hh, &c.q_full);
+      const bool kside = (warp == 0);
+      const CUtensorMap* map = kside ? &tm_k : &tm_v;
+      uint64_t* full = kside ? c.k_full : c.v_full;
+      uint64_t* empty = kside ? c.k_empty : c.v_empty;
+      const uint32_t off = kside ? kOffK : kOffV;
+      tma_prefetch_desc(map);
+      if (kside) {
+        tma_prefetch_desc(&tm_q);
+        mbar_arrive_expect_tx(&c.q_full, TILES * 4 * 64 * 128);
+        for (int t = 0; t < TILES; ++t)
+          for (int hh = 0; hh < 2; ++hh)
+            for (int kb = 0; kb < 2; ++kb)
+              tma_load_3d(base + kOffQ + t * 32768 + kb * 16384 + hh * 8192, &tm_q, kb * 64,
+                          j * kB, bi * s.Hq + kvh * G + 2 * t + hh, &c.q_full);
+      }
       int issued = 0;
       for (int n = 0; n < nblk; ++n) {
-        const int st = n & 1;
-        if (n >= kStages && !wait_or_abort(ctx, &c.kv_empty[st], ((n - kStages) >> 1) & 1, abort))
+        const int st = n % kStages;
+        if (n >= kStages &&
+            !wait_or_abort(ctx, &empty[st], ((n - kStages) / kStages) & 1, abort))
           break;
         const int m = c.blocks[n];
-        unsigned char* kv = base + kOffKV + st * kKVStageBytes;
-        mbar_arrive_expect_tx(&c.kv_full[st], kKVStageBytes);
+        unsigned char* dst = base + off + st * kKVBytes;
+        mbar_arrive_expect_tx(&full[st], kKVBytes);
         for (int h2 = 0; h2 < 2; ++h2)
-          tma_load_3d(kv + h2 * 8192, &tm_k, h2 * 64, m * kB, bi * s.Hkv + kvh, &c.kv_full[st]);
-        for (int h2 = 0; h2 < 2; ++h2)
-          tma_load_3d(kv + 16384 + h2 * 8192, &tm_v, h2 * 64, m * kB, bi * s.Hkv + kvh,
-                      &c.kv_full[st]);
+          tma_load_3d(dst + h2 * 8192, map, h2 * 64, m * kB, bi * s.Hkv + kvh, &full[st]);
         issued = n + 1;
       }
       if (*abort) {
         // Let the loads still in flight land before the CTA's memory is released.
-        (void)mbar_wait(ctx, &c.q_full, 0);
+        if (kside) (void)mbar_wait(ctx, &c.q_full, 0);
         for (int n = max(0, issued - kStages); n < issued; ++n)
-          (void)mbar_wait(ctx, &c.kv_full[n & 1], (n >> 1) & 1);
+          (void)mbar_wait(ctx, &full[n % kStages], (n / kStages) & 1);
       }
     }
   } else if (warp == 1) {
@@ -169,14 +180,14 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       bool ok = wait_or_abort(ctx, &c.q_full, 0, abort);
       fence_after_sync();
       auto issue_s = [&](int n) -> bool {
-        const int st = n & 1, b = n & 1;
-        if (!wait_or_abort(ctx, &c.kv_full[st], (n >> 1) & 1, abort)) return false;
+        const int st = n % kStages, b = n & 1;
+        if (!wait_or_abort(ctx, &c.k_full[st], (n / kStages) & 1, abort)) return false;
         for (int t = 0; t < TILES; ++t) {
           if (n >= 2 && !wait_or_abort(ctx, &c.s_free[t][b], ((n - 2) >> 1) & 1, abort))
             return false;
           fence_after_sync();
           const uint32_t qa = sbase + kOffQ + t * 32768;
-          const uint32_t ka = sbase + kOffKV + st * kKVStageBytes;
+          const uint32_t ka = sbase + kOffK + st * kKVBytes;
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
             const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
@@ -186,28 +197,30 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           }
           mma_commit(&c.s_full[t][b]);
         }
+        mma_commit(&c.k_empty[st]);  // K block n is no longer needed once S is done
         return true;
       };
       if (ok) ok = issue_s(0);
       for (int n = 0; ok && n < nblk; ++n) {
         if (n + 1 < nblk && !issue_s(n + 1)) break;
-        const int st = n & 1, b = n & 1;
+        const int st = n % kStages;
+        if (!wait_or_abort(ctx, &c.v_full[st], (n / kStages) & 1, abort)) break;
         for (int t = 0; t < TILES; ++t) {
-          if (!wait_or_abort(ctx, &c.p_full[t][b], (n >> 1) & 1, abort)) {
+          if (!wait_or_abort(ctx, &c.p_full[t], n & 1, abort)) {
             ok = false;
             break;
           }
           fence_after_sync();
-          const uint32_t pa = sbase + kOffP + (t * 2 + b) * 16384;
-          const uint32_t va = sbase + kOffKV + st * kKVStageBytes + 16384;
+          const uint32_t pa = sbase + kOffP + t * 16384;
+          const uint32_t va = sbase + kOffV + st * kKVBytes;
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
             mma_bf16_ss(tmem + o_col(t), sdesc_sw128(pa + ks * 32, 16, 1024),
                         sdesc_sw128(va + ks * 2048, 8192, 1024), id_o, (n > 0 || ks > 0));
-          mma_commit(&c.pv_done[t][b]);
+          mma_commit(&c.pv_done[t]);
         }
         if (!ok) break;
-        mma_commit(&c.kv_empty[st]);
+        mma_commit(&c.v_empty[st]);
       }
       if (*abort) {
         // MMAs already issued must finish before TMEM is released.
@@ -243,17 +256,24 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
       const int m = c.blocks[n];
       const float bias = c.bias[n];
-      const bool cur = (n == nblk - 1);
+      const bool cur = (n == 0);
       const int kvalid = min(kB, s.T - m * kB);   // keys of the block inside the sequence
-      float x[64];
-      float mx = -INFINITY;
+      // Full history blocks need no mask; the current block (causal) and a
+      // block cut by the end of the sequence set their masked scores to -inf.
+      if (cur || kvalid < kB) {
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        float v = fmaf(__uint_as_float(sr[i]), sc, bias);
-        if (i >= kvalid || (cur && i > r)) v = -INFINITY;
-        x[i] = v;
-        mx = fmaxf(mx, v);
+        for (int i = 0; i < 64; ++i)
+          if (i >= kvalid || (cur && i > r)) sr[i] = __float_as_uint(-INFINITY);
       }
+      float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 64; i += 4) {
+        m0 = fmax3(m0, __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]));
+        m1 = fmax3(m1, __uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3]));
+      }
+      const float smax = fmaxf(m0, m1);
+      // Row max of the block's logits s*scale + bias (scale > 0).
+      const float mx = (smax == -INFINITY) ? -INFINITY : fmaf(smax, sc, bias);
       const float m_new = fmaxf(m_used, mx);
       // Rows whose max grew by more than 2^8 rescale O (and l); the TMEM
       // load/store is warp-wide, so the warp does it if any of its rows must.
@@ -261,8 +281,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const bool need = grow && n > 0 && m_used != -INFINITY;
       if (__any_sync(0xffffffffu, need)) {
         const float alpha = need ? ex2(m_used - m_new) : 1.f;
-        if (!__all_sync(0xffffffffu, wait_or_abort(ctx, &c.pv_done[t][(n - 1) & 1],
-                                                   ((n - 1) >> 1) & 1, abort))) {
+        if (!__all_sync(0xffffffffu, wait_or_abort(ctx, &c.pv_done[t], (n - 1) & 1, abort))) {
           ok = false;
           break;
         }
@@ -280,23 +299,33 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         l *= alpha;
       }
       if (grow) m_used = m_new;
-      float rs = 0.f;
+      // p = 2^(s*scale + bias - m_used): one packed FMA per pair, then ex2.
+      const float off = (m_used == -INFINITY) ? -INFINITY : bias - m_used;
+      const uint64_t sc2 = f2u(sc, sc), off2 = f2u(off, off);
+      uint64_t acc0 = 0, acc1 = 0;
       uint32_t pk[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float p0 = (m_used == -INFINITY) ? 0.f : ex2(x[2 * i] - m_used);
-        const float p1 = (m_used == -INFINITY) ? 0.f : ex2(x[2 * i + 1] - m_used);
-        rs += p0 + p1;
+      for (int i = 0; i < 32; i += 2) {
+        const uint64_t a0 = ffma2(f2u(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
+                                  sc2, off2);
+        const uint64_t a1 = ffma2(f2u(__uint_as_float(sr[2 * i + 2]), __uint_as_float(sr[2 * i + 3])),
+                                  sc2, off2);
+        const float p0 = ex2(lo_f(a0)), p1 = ex2(hi_f(a0));
+        const float p2 = ex2(lo_f(a1)), p3 = ex2(hi_f(a1));
+        acc0 = fadd2(acc0, f2u(p0, p1));
+        acc1 = fadd2(acc1, f2u(p2, p3));
         pk[i] = pack_bf16(p0, p1);
+        pk[i + 1] = pack_bf16(p2, p3);
       }
-      l += rs;
-      // P buffer b is free once PV(n-2) has completed.
-      if (n >= 2 &&
-          !__all_sync(0xffffffffu, wait_or_abort(ctx, &c.pv_done[t][b], ((n - 2) >> 1) & 1, abort))) {
+      const uint64_t accs = fadd2(acc0, acc1);
+      l += lo_f(accs) + hi_f(accs);
+      // The tile's P buffer is free once PV(n-1) has completed.
+      if (n >= 1 &&
+          !__all_sync(0xffffffffu, wait_or_abort(ctx, &c.pv_done[t], (n - 1) & 1, abort))) {
         ok = false;
         break;
       }
-      unsigned char* prow = base + kOffP + (t * 2 + b) * 16384 + rowi * 128;
+      unsigned char* prow = base + kOffP + t * 16384 + rowi * 128;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
         uint4 v = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
@@ -304,12 +333,12 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       }
       fence_proxy_async_smem();
       fence_before_sync();
-      mbar_arrive(&c.p_full[t][b]);
+      mbar_arrive(&c.p_full[t]);
     }
     if (ok && t < TILES) {
       // ---- epilogue: O / l and the log-sum-exp
       const int nl = nblk - 1;
-      if (__all_sync(0xffffffffu, wait_or_abort(ctx, &c.pv_done[t][nl & 1], (nl >> 1) & 1, abort))) {
+      if (__all_sync(0xffffffffu, wait_or_abort(ctx, &c.pv_done[t], nl & 1, abort))) {
         fence_after_sync();
         const float inv = 1.f / l;
         const bool write = qrow < s.T;
