@@ -96,23 +96,29 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     mbar_init(&c.drain, 1);
     fence_mbar_init();
     c.abort = 0;
-    int n = 0;
-    for (int sl = 0; sl < s.K; ++sl) {
-      const int m = idx[irow * s.K + sl];
-      if (m < 0) continue;
-      if (m >= j) {
-        report(ctx, kDevErrBadIndex);
-        continue;
+    // Q and dO do not depend on the selection: start their loads first.
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_do);
+    mbar_arrive_expect_tx(&c.qdo_full, 2 * 4 * 8192);
+    for (int hh = 0; hh < 2; ++hh)
+      for (int kb = 0; kb < 2; ++kb) {
+        tma_load_3d(base + kOffQ + kb * 16384 + hh * 8192, &tm_q, kb * 64, j * kB,
+                    bi * s.Hq + h0 + hh, &c.qdo_full);
+        tma_load_3d(base + kOffDO + kb * 16384 + hh * 8192, &tm_do, kb * 64, j * kB,
+                    bi * s.Hq + h0 + hh, &c.qdo_full);
       }
-      c.blocks[n] = m;
-      c.slots[n] = sl;
-      c.bias[n] = gates ? logf(gates[irow * s.N + m]) * kLog2e : 0.f;
-      ++n;
+  }
+  if (warp == 0) {
+    // Attended blocks: the selected history blocks in slot order, then block j.
+    __syncwarp();
+    const int n = warp_build_list(idx + irow * s.K, gates ? gates + irow * s.N : nullptr, s.K, j,
+                                  0, c.blocks, c.slots, c.bias, ctx);
+    if (lane == 0) {
+      c.blocks[n] = j;
+      c.slots[n] = -1;
+      c.bias[n] = 0.f;
+      c.nblk = n + 1;
     }
-    c.blocks[n] = j;
-    c.slots[n] = -1;
-    c.bias[n] = 0.f;
-    c.nblk = n + 1;
   }
   if (warp == 1) {
     tmem_alloc(&c.tmem_base, kTmemCols);
@@ -128,18 +134,8 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
   if (warp == 0) {
     if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_do);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(&c.qdo_full, 2 * 4 * 8192);
-      for (int hh = 0; hh < 2; ++hh)
-        for (int kb = 0; kb < 2; ++kb) {
-          tma_load_3d(base + kOffQ + kb * 16384 + hh * 8192, &tm_q, kb * 64, j * kB,
-                      bi * s.Hq + h0 + hh, &c.qdo_full);
-          tma_load_3d(base + kOffDO + kb * 16384 + hh * 8192, &tm_do, kb * 64, j * kB,
-                      bi * s.Hq + h0 + hh, &c.qdo_full);
-        }
       int issued = 0;
       for (int it = 0; it < nit; ++it) {
         const int st = it % kStages;
@@ -363,6 +359,11 @@ struct Ctl {
       drain;
   uint32_t tmem_base;
   int abort;
+  // Per stage, staged by the producer warp with the Q/dO tiles: the step's
+  // query block, its log2-domain gate bias, and lse / D of the tile's rows.
+  int step_j[2];
+  float step_bias[2];
+  float lse2[2][128], D[2][128];
 };
 constexpr size_t kSmem = kOffCtl + sizeof(Ctl) + 1024;
 // TMEM columns: S[b] at 64 b, dP[b] at 128 + 64 b, dV^T at 256, dK^T at 320.
@@ -403,7 +404,7 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
   if (tid == 0) {
     mbar_init(&c.kv_full, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&c.qdo_full[i], 1);
+      mbar_init(&c.qdo_full[i], 2);  // tiles (expect_tx) + staged scalars
       mbar_init(&c.qdo_empty[i], 1);
       mbar_init(&c.s_full[i], 1);
       mbar_init(&c.s_free[i], 128);
@@ -434,13 +435,16 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
         tma_load_3d(base + kOffK + h2 * 8192, &tm_k, h2 * 64, m * kB, bh, &c.kv_full);
         tma_load_3d(base + kOffV + h2 * 8192, &tm_v, h2 * 64, m * kB, bh, &c.kv_full);
       }
-      int issued = 0;
-      for (int st_i = 0; st_i < nsteps; ++st_i) {
-        const int stg = st_i & 1;
-        if (st_i >= 2 &&
-            !wait_or_abort(ctx, &c.qdo_empty[stg], ((st_i - 2) >> 1) & 1, abort))
-          break;
-        const int j = qblock(st_i), u = st_i % TILES;
+    }
+    int issued = 0;
+    for (int st_i = 0; st_i < nsteps; ++st_i) {
+      const int stg = st_i & 1;
+      bool go = true;
+      if (lane == 0 && st_i >= 2)
+        go = wait_or_abort(ctx, &c.qdo_empty[stg], ((st_i - 2) >> 1) & 1, abort);
+      if (!__shfl_sync(0xffffffffu, go, 0)) break;
+      const int j = qblock(st_i), u = st_i % TILES;
+      if (lane == 0) {
         unsigned char* qd = base + kOffQD + stg * 65536;
         mbar_arrive_expect_tx(&c.qdo_full[stg], 65536);
         for (int hh = 0; hh < 2; ++hh)
@@ -451,13 +455,32 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
             tma_load_3d(qd + 32768 + kb * 16384 + hh * 8192, &tm_do, kb * 64, j * kB, plane,
                         &c.qdo_full[stg]);
           }
-        issued = st_i + 1;
       }
-      if (*abort) {
-        (void)mbar_wait(ctx, &c.kv_full, 0);
-        for (int st_i = max(0, issued - 2); st_i < issued; ++st_i)
-          (void)mbar_wait(ctx, &c.qdo_full[st_i & 1], (st_i >> 1) & 1);
+      // Scalars of the step: every lane stages 4 rows of lse (log2 domain) and D.
+      for (int rr = lane; rr < 128; rr += 32) {
+        const int head = kvh * G + 2 * u + (rr >> 6), qrow = j * kB + (rr & 63);
+        const bool live = qrow < s.T;
+        const long long hrow = (long long)(bi * s.Hq + head) * s.T + qrow;
+        c.lse2[stg][rr] = live ? lse[hrow] * kLog2e : 0.f;
+        c.D[stg][rr] = live ? Dv[hrow] : 0.f;
       }
+      if (lane == 0) {
+        c.step_j[stg] = j;
+        c.step_bias[stg] = (j == m || gates == nullptr)
+                               ? 0.f
+                               : logf(gates[((long long)bh * s.N + j) * s.N + m]) * kLog2e;
+      }
+      __threadfence_block();
+      __syncwarp();
+      // The consumers see the staged scalars once this stage's Q/dO tiles
+      // have landed: the arrival below is part of the same barrier phase.
+      if (lane == 0) mbar_arrive(&c.qdo_full[stg]);
+      issued = st_i + 1;
+    }
+    if (lane == 0 && *abort) {
+      (void)mbar_wait(ctx, &c.kv_full, 0);
+      for (int st_i = max(0, issued - 2); st_i < issued; ++st_i)
+        (void)mbar_wait(ctx, &c.qdo_full[st_i & 1], (st_i >> 1) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -542,7 +565,7 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
   } else if (warp >= 4) {
     const int quarter = warp & 3;
     const int rowi = quarter * 32 + lane;  // tile row (query) / d index in the epilogue
-    const int hh = rowi >> 6, r = rowi & 63;
+    const int r = rowi & 63;
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
     const float sc = s.scale * kLog2e;
     const int kvalid = min(kB, s.T - m * kB);
@@ -554,17 +577,14 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
         break;
       }
       fence_after_sync();
-      const int j = qblock(st_i), u = st_i % TILES;
-      const int head = kvh * G + 2 * u + hh;
+      const int stg = st_i & 1;
+      const int j = c.step_j[stg];
       const int qrow = j * kB + r;
       const bool live = qrow < s.T;
-      const long long hrow = (long long)(bi * s.Hq + head) * s.T + qrow;
-      const float lse2 = live ? lse[hrow] * kLog2e : 0.f;
-      const float Di = live ? Dv[hrow] : 0.f;
+      const float lse2 = c.lse2[stg][rowi];
+      const float Di = c.D[stg][rowi];
       const bool cur = (j == m);
-      const float bias =
-          (cur || gates == nullptr) ? 0.f
-                                    : logf(gates[((long long)bh * s.N + j) * s.N + m]) * kLog2e;
+      const float bias = c.step_bias[stg];
       uint32_t sr[64], pr[64], pp[32], dd[32];
       tmem_ld32(tl + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
       tmem_ld32(tl + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));

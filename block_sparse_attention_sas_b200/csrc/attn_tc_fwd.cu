@@ -105,23 +105,26 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     mbar_init(&c.drain, 1);
     fence_mbar_init();
     c.abort = 0;
+    // Q does not depend on the selection: start its load first.
+    tma_prefetch_desc(&tm_q);
+    mbar_arrive_expect_tx(&c.q_full, TILES * 4 * 64 * 128);
+    for (int t = 0; t < TILES; ++t)
+      for (int hh = 0; hh < 2; ++hh)
+        for (int kb = 0; kb < 2; ++kb)
+          tma_load_3d(base + kOffQ + t * 32768 + kb * 16384 + hh * 8192, &tm_q, kb * 64, j * kB,
+                      bi * s.Hq + kvh * G + 2 * t + hh, &c.q_full);
+  }
+  if (warp == 0) {
     // Attended blocks in order: block j (bias 0, the largest logits in
-    // expectation), then the selected history blocks.
-    c.blocks[0] = j;
-    c.bias[0] = 0.f;
-    int n = 1;
-    for (int sl = 0; sl < s.K; ++sl) {
-      const int m = idx[irow * s.K + sl];
-      if (m < 0) continue;
-      if (m >= j) {
-        report(ctx, kDevErrBadIndex);
-        continue;
-      }
-      c.blocks[n] = m;
-      c.bias[n] = gates ? logf(gates[irow * s.N + m]) * kLog2e : 0.f;
-      ++n;
+    // expectation), then the selected history blocks in slot order.
+    __syncwarp();
+    if (lane == 0) {
+      c.blocks[0] = j;
+      c.bias[0] = 0.f;
     }
-    c.nblk = n;
+    const int n = warp_build_list(idx + irow * s.K, gates ? gates + irow * s.N : nullptr, s.K, j,
+                                  1, c.blocks, nullptr, c.bias, ctx);
+    if (lane == 0) c.nblk = n;
   }
   if (warp == 1) {
     tmem_alloc(&c.tmem_base, kTmemCols);
@@ -143,15 +146,6 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       uint64_t* empty = kside ? c.k_empty : c.v_empty;
       const uint32_t off = kside ? kOffK : kOffV;
       tma_prefetch_desc(map);
-      if (kside) {
-        tma_prefetch_desc(&tm_q);
-        mbar_arrive_expect_tx(&c.q_full, TILES * 4 * 64 * 128);
-        for (int t = 0; t < TILES; ++t)
-          for (int hh = 0; hh < 2; ++hh)
-            for (int kb = 0; kb < 2; ++kb)
-              tma_load_3d(base + kOffQ + t * 32768 + kb * 16384 + hh * 8192, &tm_q, kb * 64,
-                          j * kB, bi * s.Hq + kvh * G + 2 * t + hh, &c.q_full);
-      }
       int issued = 0;
       for (int n = 0; n < nblk; ++n) {
         const int st = n % kStages;

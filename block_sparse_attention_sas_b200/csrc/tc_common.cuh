@@ -178,6 +178,34 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// The attended-block list of one query block, built by one full warp: lane
+// l reads idx slot base + l, valid entries (0 <= m < j) are compacted in slot
+// order after `first` already-placed entries, with their log2-domain gate
+// bias (0 without gates); entries >= j are reported. Returns the list length.
+__device__ __forceinline__ int warp_build_list(const int32_t* idx_row, const float* gate_row,
+                                               int K, int j, int first, int* blocks, int* slots,
+                                               float* bias, const DevCtx& ctx) {
+  const int lane = threadIdx.x & 31;
+  int n = first;
+  for (int base = 0; base < K; base += 32) {
+    const int sl = base + lane;
+    const int m = sl < K ? idx_row[sl] : -1;
+    const bool bad = m >= j;
+    if (bad) report(ctx, kDevErrBadIndex);
+    const bool ok = m >= 0 && !bad;
+    const float g = (ok && gate_row) ? gate_row[m] : 1.f;
+    const uint32_t mask = __ballot_sync(0xffffffffu, ok);
+    if (ok) {
+      const int pos = n + __popc(mask & ((1u << lane) - 1u));
+      blocks[pos] = m;
+      if (slots) slots[pos] = sl;
+      bias[pos] = gate_row ? logf(g) * 1.4426950408889634f : 0.f;
+    }
+    n += __popc(mask);
+  }
+  return n;
+}
+
 // Bounded mbarrier wait that also gives up when another thread of the CTA has
 // set *abort (checked every 64 polls). On running out of polls it records a
 // timeout, sets *abort and returns false.
