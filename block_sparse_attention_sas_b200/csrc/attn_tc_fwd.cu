@@ -14,8 +14,9 @@
 //   warps 0, 2  TMA producers: Q once, then the attended blocks' K (warp 0)
 //               and V (warp 2), 16 KB each, into separate three-stage rings
 //               (a K stage frees once S is computed, a V stage once PV is)
-//   warp 1      MMA issuer: S_t = Q_t K^T into TMEM (double-buffered, 64
-//               columns per tile), then O_t += P_t V (128 columns per tile)
+//   warp 1      MMA issuer: S_t = Q_t K^T with Q_t read from TMEM (so only K
+//               crosses shared memory), then O_t += P_t V (128 columns per
+//               tile); each softmax thread first copies its Q row into TMEM
 //   warps 4-11  softmax, one warpgroup per M-tile, one thread per query row:
 //               S from TMEM, scale + log-gate bias + causal mask, running max
 //               (O rescaled in TMEM only when the max grows by more than 2^8;
@@ -55,7 +56,9 @@ constexpr int kMaxList = 257;                        // K <= 256 selected + curr
 struct Ctl {
   uint64_t q_full;
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2][2], s_free[2][2], p_full[2], pv_done[2];
+  // One barrier for both tiles where they move in step (fewer waits and
+  // commits on the MMA thread, whose overhead sits on the critical path).
+  uint64_t q_tmem, s_full, s_free, p_full, pv_done;
   uint64_t drain;  // abort path only: the MMA thread's last commit
   uint32_t tmem_base;
   int abort;
@@ -65,8 +68,10 @@ struct Ctl {
 };
 constexpr size_t kSmemBytes = kOffCtl + sizeof(Ctl) + 1024;  // + alignment slack
 
-// TMEM columns: S[tile][buffer] at tile*128 + buffer*64; O[tile] at 256 + tile*128.
-__device__ __forceinline__ uint32_t s_col(int t, int b) { return t * 128 + b * 64; }
+// TMEM columns: Q[tile] (A operand, bf16 pairs) at tile*64, S[tile] at
+// 128 + tile*64, O[tile] at 256 + tile*128.
+__device__ __forceinline__ uint32_t q_col(int t) { return t * 64; }
+__device__ __forceinline__ uint32_t s_col(int t) { return 128 + t * 64; }
 __device__ __forceinline__ uint32_t o_col(int t) { return 256 + t * 128; }
 
 template <int TILES>
@@ -94,14 +99,11 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       mbar_init(&c.v_full[i], 1);
       mbar_init(&c.v_empty[i], 1);
     }
-    for (int t = 0; t < 2; ++t) {
-      for (int b = 0; b < 2; ++b) {
-        mbar_init(&c.s_full[t][b], 1);
-        mbar_init(&c.s_free[t][b], 128);
-      }
-      mbar_init(&c.p_full[t], 128);
-      mbar_init(&c.pv_done[t], 1);
-    }
+    mbar_init(&c.q_tmem, 128 * TILES);
+    mbar_init(&c.s_full, 1);
+    mbar_init(&c.s_free, 128 * TILES);
+    mbar_init(&c.p_full, 128 * TILES);
+    mbar_init(&c.pv_done, 1);
     mbar_init(&c.drain, 1);
     fence_mbar_init();
     c.abort = 0;
@@ -173,24 +175,28 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const uint32_t id_o = idesc_bf16(128, 128, false, true);
       bool ok = wait_or_abort(ctx, &c.q_full, 0, abort);
       fence_after_sync();
+      // Descriptors are built once; a K-step or stage only moves the start
+      // address field (addresses stay below 256 KB, so no carry leaves it).
+      const uint64_t kdesc0 = sdesc_sw128(sbase + kOffK, 16, 1024);
+      const uint64_t pdesc0 = sdesc_sw128(sbase + kOffP, 16, 1024);
+      const uint64_t vdesc0 = sdesc_sw128(sbase + kOffV, 8192, 1024);
+      auto adv = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
       auto issue_s = [&](int n) -> bool {
-        const int st = n % kStages, b = n & 1;
+        const int st = n % kStages;
         if (!wait_or_abort(ctx, &c.k_full[st], (n / kStages) & 1, abort)) return false;
+        // S is single-buffered: the softmax copies S(n-1) to registers first.
+        if (!wait_or_abort(ctx, n == 0 ? &c.q_tmem : &c.s_free, n == 0 ? 0 : ((n - 1) & 1),
+                           abort))
+          return false;
+        fence_after_sync();
+        const uint64_t kd = adv(kdesc0, st * kKVBytes);
         for (int t = 0; t < TILES; ++t) {
-          if (n >= 2 && !wait_or_abort(ctx, &c.s_free[t][b], ((n - 2) >> 1) & 1, abort))
-            return false;
-          fence_after_sync();
-          const uint32_t qa = sbase + kOffQ + t * 32768;
-          const uint32_t ka = sbase + kOffK + st * kKVBytes;
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-            const uint32_t koff = (ks >> 2) * 8192 + (ks & 3) * 32;
-            mma_bf16_ss(tmem + s_col(t, b), sdesc_sw128(qa + off, 16, 1024),
-                        sdesc_sw128(ka + koff, 16, 1024), id_s, ks > 0);
-          }
-          mma_commit(&c.s_full[t][b]);
+          for (int ks = 0; ks < 8; ++ks)
+            mma_bf16_ts(tmem + s_col(t), tmem + q_col(t) + ks * 8,
+                        adv(kd, (ks >> 2) * 8192 + (ks & 3) * 32), id_s, ks > 0);
         }
+        mma_commit(&c.s_full);
         mma_commit(&c.k_empty[st]);  // K block n is no longer needed once S is done
         return true;
       };
@@ -199,21 +205,17 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (n + 1 < nblk && !issue_s(n + 1)) break;
         const int st = n % kStages;
         if (!wait_or_abort(ctx, &c.v_full[st], (n / kStages) & 1, abort)) break;
+        if (!wait_or_abort(ctx, &c.p_full, n & 1, abort)) break;
+        fence_after_sync();
+        const uint64_t vd = adv(vdesc0, st * kKVBytes);
         for (int t = 0; t < TILES; ++t) {
-          if (!wait_or_abort(ctx, &c.p_full[t], n & 1, abort)) {
-            ok = false;
-            break;
-          }
-          fence_after_sync();
-          const uint32_t pa = sbase + kOffP + t * 16384;
-          const uint32_t va = sbase + kOffV + st * kKVBytes;
+          const uint64_t pd = adv(pdesc0, t * 16384);
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
-            mma_bf16_ss(tmem + o_col(t), sdesc_sw128(pa + ks * 32, 16, 1024),
-                        sdesc_sw128(va + ks * 2048, 8192, 1024), id_o, (n > 0 || ks > 0));
-          mma_commit(&c.pv_done[t]);
+            mma_bf16_ss(tmem + o_col(t), adv(pd, ks * 32), adv(vd, ks * 2048), id_o,
+                        (n > 0 || ks > 0));
         }
-        if (!ok) break;
+        mma_commit(&c.pv_done);
         mma_commit(&c.v_empty[st]);
       }
       if (*abort) {
@@ -234,19 +236,29 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const float sc = s.scale * kLog2e;
     float m_used = -INFINITY, l = 0.f;
     bool ok = t < TILES;
+    if (ok) {
+      // This thread's Q row moves from the swizzled shared tile into TMEM.
+      if (!__all_sync(0xffffffffu, wait_or_abort(ctx, &c.q_full, 0, abort))) {
+        ok = false;
+      } else {
+        tile_row_to_tmem(base + kOffQ + t * 32768, rowi, tl + q_col(t));
+        tmem_st_wait();
+        fence_before_sync();
+        mbar_arrive(&c.q_tmem);
+      }
+    }
     for (int n = 0; ok && n < nblk; ++n) {
-      const int b = n & 1;
-      if (!__all_sync(0xffffffffu, wait_or_abort(ctx, &c.s_full[t][b], (n >> 1) & 1, abort))) {
+      if (!__all_sync(0xffffffffu, wait_or_abort(ctx, &c.s_full, n & 1, abort))) {
         ok = false;
         break;
       }
       fence_after_sync();
       uint32_t sr[64];
-      tmem_ld32(tl + s_col(t, b), *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tl + s_col(t, b) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(tl + s_col(t), *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tl + s_col(t) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_ld_wait();
       fence_before_sync();
-      mbar_arrive(&c.s_free[t][b]);
+      mbar_arrive(&c.s_free);
 
       const int m = c.blocks[n];
       const float bias = c.bias[n];
@@ -275,7 +287,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const bool need = grow && n > 0 && m_used != -INFINITY;
       if (__any_sync(0xffffffffu, need)) {
         const float alpha = need ? ex2(m_used - m_new) : 1.f;
-        if (!__all_sync(0xffffffffu, wait_or_abort(ctx, &c.pv_done[t], (n - 1) & 1, abort))) {
+        if (!__all_sync(0xffffffffu, wait_or_abort(ctx, &c.pv_done, (n - 1) & 1, abort))) {
           ok = false;
           break;
         }
@@ -315,7 +327,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       l += lo_f(accs) + hi_f(accs);
       // The tile's P buffer is free once PV(n-1) has completed.
       if (n >= 1 &&
-          !__all_sync(0xffffffffu, wait_or_abort(ctx, &c.pv_done[t], (n - 1) & 1, abort))) {
+          !__all_sync(0xffffffffu, wait_or_abort(ctx, &c.pv_done, (n - 1) & 1, abort))) {
         ok = false;
         break;
       }
@@ -327,12 +339,12 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       }
       fence_proxy_async_smem();
       fence_before_sync();
-      mbar_arrive(&c.p_full[t]);
+      mbar_arrive(&c.p_full);
     }
     if (ok && t < TILES) {
       // ---- epilogue: O / l and the log-sum-exp
       const int nl = nblk - 1;
-      if (__all_sync(0xffffffffu, wait_or_abort(ctx, &c.pv_done[t], nl & 1, abort))) {
+      if (__all_sync(0xffffffffu, wait_or_abort(ctx, &c.pv_done, nl & 1, abort))) {
         fence_after_sync();
         const float inv = 1.f / l;
         const bool write = qrow < s.T;

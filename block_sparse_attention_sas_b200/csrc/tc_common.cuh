@@ -87,6 +87,22 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, ui
       "r"(z), "r"(z)
       : "memory");
 }
+// MMA with A in TMEM: D[tmem] (+)= A[tmem] * B[smem]. A (M rows x K, 16-bit)
+// sits with row m in lane m and consecutive K elements packed two per 32-bit
+// column (the even element in the low half), so one K-step of 16 advances the
+// A address by 8 columns.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  const uint32_t z = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(z), "r"(z),
+      "r"(z), "r"(z)
+      : "memory");
+}
+
 // Arrives once on `bar` when every MMA this thread issued before has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -125,6 +141,29 @@ __device__ __forceinline__ void tmem_ld_wait() {
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
+
+// Copies row `row` of a [128 rows x 128] bf16 tile held in shared memory in
+// the K-major 128-byte-swizzle layout (two 64-element halves, 16 KB apart)
+// into 64 TMEM columns of this thread's lane, in the A-operand packing.
+// Called by all 32 lanes of a warp (tcgen05.st is warp-wide).
+__device__ __forceinline__ void tile_row_to_tmem(const unsigned char* tile, int row,
+                                                 uint32_t taddr) {
+  uint32_t w[64];
+#pragma unroll
+  for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+      const uint4 v = *reinterpret_cast<const uint4*>(tile + kb * 16384 + row * 128 +
+                                                      ((ch ^ (row & 7)) << 4));
+      w[kb * 32 + ch * 4 + 0] = v.x;
+      w[kb * 32 + ch * 4 + 1] = v.y;
+      w[kb * 32 + ch * 4 + 2] = v.z;
+      w[kb * 32 + ch * 4 + 3] = v.w;
+    }
+  tmem_st32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&w[0]));
+  tmem_st32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&w[32]));
+}
+
 
 // ---- TMA tile load (3-D tensor map), completion counted on `bar`; no multicast
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, int c0, int c1,
