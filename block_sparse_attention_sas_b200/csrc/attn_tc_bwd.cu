@@ -34,35 +34,60 @@ using namespace tc;
 
 constexpr int kD = 128;
 constexpr int kB = 64;
-constexpr int kThreads = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxList = 257;
 
 // ============================================================================
 // Kernel A: dq, D, da
 // ============================================================================
+// Q and dO of the tile are copied into TMEM once and used as the A operand of
+// every S / dP MMA, and dS goes back into TMEM as the A operand of the dQ MMA:
+// the MMAs then read only K / V from shared memory. Two groups of four
+// elementwise warps split each block's 64 keys (group g takes keys 32g ..).
+//
+// Every mbarrier wait costs the MMA-issuing thread far more than an MMA issue
+// slot, so it waits once per iteration: the full barrier of K/V stage `it`
+// also collects one arrival from each elementwise warp, given when that warp
+// is done with the S/dP buffer of iteration it - 2 (and, in sweep 2, has
+// written that iteration's dS). The MMA stream is S/dP(0), S/dP(1), ...,
+// with dQ(it - 2) issued right before S/dP(it) in sweep 2.
 namespace ka {
-constexpr int kStages = 3;              // K/V ring depth
-constexpr uint32_t kOffQ = 0;            // [k half][128 rows][128 B]
-constexpr uint32_t kOffDO = 32768;       // same layout
-constexpr uint32_t kOffKV = 65536;       // kStages x (K halves, V halves) 32 KB
-constexpr uint32_t kOffDS = kOffKV + kStages * 32768;  // 2 buffers x [128 rows][128 B]
-constexpr uint32_t kOffCtl = kOffDS + 32768;
+constexpr int kStages = 6;                // K/V ring depth (stages 4, 5 reuse the Q/dO area)
+constexpr int kWarps = 12;
+constexpr int kThreadsA = kWarps * 32;
+constexpr uint32_t kOffQ = 0;             // [k half][128 rows][128 B]
+constexpr uint32_t kOffDO = 32768;        // same layout
+constexpr uint32_t kOffKV = 65536;        // stages 0..3; stage = (K halves, V halves) 32 KB
+// TMEM columns.
+constexpr uint32_t kColQ = 0, kColDO = 64, kColS = 128, kColDP = 256, kColDQ = 384;
 struct Ctl {
-  uint64_t qdo_full, kv_full[kStages], kv_empty[kStages], s_full[2], s_free[2], ds_full[2],
-      dq_done[2], drain;
+  // kv_full[st]: the producer's expect-tx arrival, the TMA bytes and one
+  // arrival per elementwise warp (9 arrivals per phase).
+  uint64_t qdo_full, kv_full[kStages], kv_empty[kStages], s_full[2], ds_tail[2], dq_done, drain;
   uint32_t tmem_base;
   int abort, nblk;
   int blocks[kMaxList], slots[kMaxList];
   float bias[kMaxList];
-  float red[kMaxList][4];  // per-warp partial sums of dS per block
+  float red[kMaxList][8];  // per-warp partial sums of dS per block
+  float dpart[2][128];     // per-group partial D per row
 };
+constexpr uint32_t kOffCtl = kOffKV + 4 * 32768;
 constexpr size_t kSmem = kOffCtl + sizeof(Ctl) + 1024;
-// TMEM columns: S[b] at 64 b, dP[b] at 128 + 64 b, dQ at 256.
+__device__ __forceinline__ uint32_t stage_off(int st) {
+  return st < 4 ? kOffKV + st * 32768u : kOffQ + (st - 4) * 32768u;
+}
 }  // namespace ka
 
+// One lane of the warp polls the barrier; the others wait at the shuffle.
+__device__ __forceinline__ bool warp_wait(const DevCtx& ctx, uint64_t* bar, uint32_t parity,
+                                          volatile int* abort) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = wait_or_abort(ctx, bar, parity, abort) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
 template <int TILES>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(ka::kThreadsA, 1)
 tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                  const float* __restrict__ lse, const int32_t* __restrict__ idx,
@@ -80,35 +105,48 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int G = 2 * TILES;
   const int h0 = kvh * G + 2 * u;  // the tile's two heads: h0, h0 + 1
   const long long irow = ((long long)(bi * s.Hkv + kvh) * s.N + j);
+  volatile int* abort = &c.abort;
 
-  if (tid == 0) {
-    mbar_init(&c.qdo_full, 1);
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&c.kv_full[i], 1);
-      mbar_init(&c.kv_empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&c.s_full[i], 1);
-      mbar_init(&c.s_free[i], 128);
-      mbar_init(&c.ds_full[i], 128);
-      mbar_init(&c.dq_done[i], 1);
-    }
-    mbar_init(&c.drain, 1);
-    fence_mbar_init();
-    c.abort = 0;
-    // Q and dO do not depend on the selection: start their loads first.
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_do);
-    mbar_arrive_expect_tx(&c.qdo_full, 2 * 4 * 8192);
-    for (int hh = 0; hh < 2; ++hh)
-      for (int kb = 0; kb < 2; ++kb) {
-        tma_load_3d(base + kOffQ + kb * 16384 + hh * 8192, &tm_q, kb * 64, j * kB,
-                    bi * s.Hq + h0 + hh, &c.qdo_full);
-        tma_load_3d(base + kOffDO + kb * 16384 + hh * 8192, &tm_do, kb * 64, j * kB,
-                    bi * s.Hq + h0 + hh, &c.qdo_full);
-      }
-  }
+  // Elementwise warps: tile row, its head and its lse, read before the CTA barrier.
+  const int quarter = warp & 3, grp = (warp - 4) >> 2;
+  const int rowi = quarter * 32 + lane;
+  const int hh = rowi >> 6, r = rowi & 63;
+  const int qrow = j * kB + r;
+  const bool live = qrow < s.T;
+  const long long hrow = (long long)(bi * s.Hq + h0 + hh) * s.T + qrow;
+  float lse2 = 0.f;
+  if (warp >= 4 && live) lse2 = lse[hrow] * kLog2e;
+
+  int issued = 0;
   if (warp == 0) {
+    if (lane == 0) {
+      mbar_init(&c.qdo_full, 1);
+      for (int i = 0; i < kStages; ++i) {
+        mbar_init(&c.kv_full[i], 9);
+        mbar_init(&c.kv_empty[i], 1);
+      }
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&c.s_full[i], 1);
+        mbar_init(&c.ds_tail[i], 8);
+      }
+      mbar_init(&c.dq_done, 1);
+      mbar_init(&c.drain, 1);
+      fence_mbar_init();
+      c.abort = 0;
+      // Q and dO do not depend on the selection: start their loads first.
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_do);
+      mbar_arrive_expect_tx(&c.qdo_full, 2 * 4 * 8192);
+      for (int h2 = 0; h2 < 2; ++h2)
+        for (int kb = 0; kb < 2; ++kb) {
+          tma_load_3d(base + kOffQ + kb * 16384 + h2 * 8192, &tm_q, kb * 64, j * kB,
+                      bi * s.Hq + h0 + h2, &c.qdo_full);
+          tma_load_3d(base + kOffDO + kb * 16384 + h2 * 8192, &tm_do, kb * 64, j * kB,
+                      bi * s.Hq + h0 + h2, &c.qdo_full);
+        }
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
     // Attended blocks: the selected history blocks in slot order, then block j.
     __syncwarp();
     const int n = warp_build_list(idx + irow * s.K, gates ? gates + irow * s.N : nullptr, s.K, j,
@@ -118,6 +156,21 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       c.slots[n] = -1;
       c.bias[n] = 0.f;
       c.nblk = n + 1;
+    }
+    __syncwarp();
+    // Stages 0..3 are free: start their loads before the CTA barrier.
+    if (lane == 0) {
+      const int nit0 = 2 * (n + 1);  // sweep 1 then sweep 2 over the same blocks
+      for (; issued < nit0 && issued < 4; ++issued) {
+        const int m = c.blocks[issued % (n + 1)];
+        unsigned char* kv = base + stage_off(issued);
+        mbar_arrive_expect_tx(&c.kv_full[issued], 32768);
+        for (int h2 = 0; h2 < 2; ++h2) {
+          tma_load_3d(kv + h2 * 8192, &tm_k, h2 * 64, m * kB, bi * s.Hkv + kvh, &c.kv_full[issued]);
+          tma_load_3d(kv + 16384 + h2 * 8192, &tm_v, h2 * 64, m * kB, bi * s.Hkv + kvh,
+                      &c.kv_full[issued]);
+        }
+      }
     }
   }
   if (warp == 1) {
@@ -129,21 +182,22 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   fence_after_sync();
   const uint32_t tmem = c.tmem_base;
   const int nblk = c.nblk;
-  const int nit = 2 * nblk;  // sweep 1 then sweep 2 over the same blocks
-  volatile int* abort = &c.abort;
+  const int nit = 2 * nblk;
+  const int tail_first = max(nblk, nit - 2);  // sweep-2 iterations whose dQ follows the loop
 
   if (warp == 0) {
     if (lane == 0) {
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      int issued = 0;
-      for (int it = 0; it < nit; ++it) {
+      for (int it = issued; it < nit; ++it) {
         const int st = it % kStages;
-        if (it >= kStages &&
-            !wait_or_abort(ctx, &c.kv_empty[st], ((it - kStages) / kStages) & 1, abort))
-          break;
+        bool go = true;
+        // Stages 4 and 5 reuse the Q/dO area: free once every elementwise
+        // warp has moved its rows into TMEM (their first kv_full arrivals).
+        if (it == 4) go = wait_or_abort(ctx, &c.kv_full[0], 0, abort);
+        if (go && it >= kStages)
+          go = wait_or_abort(ctx, &c.kv_empty[st], ((it - kStages) / kStages) & 1, abort);
+        if (!go) break;
         const int m = c.blocks[it % nblk];
-        unsigned char* kv = base + kOffKV + st * 32768;
+        unsigned char* kv = base + stage_off(st);
         mbar_arrive_expect_tx(&c.kv_full[st], 32768);
         for (int h2 = 0; h2 < 2; ++h2) {
           tma_load_3d(kv + h2 * 8192, &tm_k, h2 * 64, m * kB, bi * s.Hkv + kvh, &c.kv_full[st]);
@@ -162,152 +216,179 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16(128, 64, false, false);
       const uint32_t id_q = idesc_bf16(128, 128, false, true);
-      bool ok = wait_or_abort(ctx, &c.qdo_full, 0, abort);
-      fence_after_sync();
-      auto issue_s = [&](int it) -> bool {
-        const int st = it % kStages, b = it & 1;
-        if (!wait_or_abort(ctx, &c.kv_full[st], (it / kStages) & 1, abort)) return false;
-        if (it >= 2 && !wait_or_abort(ctx, &c.s_free[b], ((it - 2) >> 1) & 1, abort)) return false;
-        fence_after_sync();
-        const uint32_t kva = sbase + kOffKV + st * 32768;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t ao = (ks >> 2) * 16384 + (ks & 3) * 32;
-          const uint32_t bo = (ks >> 2) * 8192 + (ks & 3) * 32;
-          mma_bf16_ss(tmem + b * 64, sdesc_sw128(sbase + kOffQ + ao, 16, 1024),
-                      sdesc_sw128(kva + bo, 16, 1024), id_s, ks > 0);
-        }
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t ao = (ks >> 2) * 16384 + (ks & 3) * 32;
-          const uint32_t bo = (ks >> 2) * 8192 + (ks & 3) * 32;
-          mma_bf16_ss(tmem + 128 + b * 64, sdesc_sw128(sbase + kOffDO + ao, 16, 1024),
-                      sdesc_sw128(kva + 16384 + bo, 16, 1024), id_s, ks > 0);
-        }
-        mma_commit(&c.s_full[b]);
-        if (it < nblk) mma_commit(&c.kv_empty[st]);  // sweep 1 only reads S and dP
-        return true;
-      };
-      if (ok) ok = issue_s(0);
-      for (int it = 0; ok && it < nit; ++it) {
-        if (it + 1 < nit && !issue_s(it + 1)) break;
-        if (it < nblk) continue;
-        const int i2 = it - nblk, st = it % kStages;
-        if (!wait_or_abort(ctx, &c.ds_full[i2 & 1], (i2 >> 1) & 1, abort)) break;
-        fence_after_sync();
-        const uint32_t dsa = sbase + kOffDS + (i2 & 1) * 16384;
-        const uint32_t ka_ = sbase + kOffKV + st * 32768;
+      // K-major K / V tiles: k-step ks at half (ks >> 2), byte (ks & 3) * 32.
+      const uint64_t dkv0 = sdesc_sw128(sbase, 16, 1024);
+      // K as the MN-major B operand of dQ: 16 keys per k-step (2048 B).
+      const uint64_t dkq0 = sdesc_sw128(sbase, 8192, 1024);
+      // dQ += dS K for sweep-2 iteration x; dS of keys 0..31 sits in S[x & 1]
+      // columns 0..15, keys 32..63 in columns 32..47.
+      auto issue_dq = [&](int x) {
+        const uint64_t kd = dkq0 + (stage_off(x % kStages) >> 4);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_bf16_ss(tmem + 256, sdesc_sw128(dsa + ks * 32, 16, 1024),
-                      sdesc_sw128(ka_ + ks * 2048, 8192, 1024), id_q, (i2 > 0 || ks > 0));
-        mma_commit(&c.dq_done[i2 & 1]);
-        mma_commit(&c.kv_empty[st]);
+          mma_bf16_ts(tmem + kColDQ, tmem + kColS + (x & 1) * 64 + (ks >> 1) * 32 + (ks & 1) * 8,
+                      kd + ((ks * 2048) >> 4), id_q, (x > nblk || ks > 0));
+      };
+      bool ok = true;
+      for (int it = 0; it < nit; ++it) {
+        const int st = it % kStages, b = it & 1;
+        if (!wait_or_abort(ctx, &c.kv_full[st], (it / kStages) & 1, abort)) {
+          ok = false;
+          break;
+        }
+        fence_after_sync();
+        if (it >= nblk + 2) {
+          issue_dq(it - 2);
+          mma_commit(&c.kv_empty[(it - 2) % kStages]);
+        }
+        const uint64_t kd = dkv0 + (stage_off(st) >> 4);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_bf16_ts(tmem + kColS + b * 64, tmem + kColQ + ks * 8,
+                      kd + (((ks >> 2) * 8192 + (ks & 3) * 32) >> 4), id_s, ks > 0);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_bf16_ts(tmem + kColDP + b * 64, tmem + kColDO + ks * 8,
+                      kd + ((16384 + (ks >> 2) * 8192 + (ks & 3) * 32) >> 4), id_s, ks > 0);
+        mma_commit(&c.s_full[b]);
+        if (it < nblk) mma_commit(&c.kv_empty[st]);  // sweep 1 only reads S and dP
       }
+      for (int x = tail_first; ok && x < nit; ++x) {
+        if (!wait_or_abort(ctx, &c.ds_tail[x - tail_first], 0, abort)) {
+          ok = false;
+          break;
+        }
+        fence_after_sync();
+        issue_dq(x);
+      }
+      mma_commit(&c.dq_done);
       if (*abort) {
         mma_commit(&c.drain);
         (void)mbar_wait(ctx, &c.drain, 0);
       }
     }
   } else if (warp >= 4) {
-    const int quarter = warp & 3;
-    const int rowi = quarter * 32 + lane;
-    const int hh = rowi >> 6, r = rowi & 63;
-    const int head = h0 + hh;
-    const int qrow = j * kB + r;
-    const bool live = qrow < s.T;
-    const long long hrow = (long long)(bi * s.Hq + head) * s.T + qrow;
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
     const float sc = s.scale * kLog2e;
-    const float lse2 = live ? lse[hrow] * kLog2e : 0.f;
+    // Arrival on the full barrier of iteration x (when there is one).
+    auto arrive_w = [&](int x) {
+      if (lane == 0 && x < nit) mbar_arrive(&c.kv_full[x % kStages]);
+    };
+    bool ok = warp_wait(ctx, &c.qdo_full, 0, abort);
+    if (ok) {
+      // Group 0 moves the Q rows into TMEM, group 1 the dO rows.
+      tile_row_to_tmem(base + (grp == 0 ? kOffQ : kOffDO), rowi,
+                       tl + (grp == 0 ? kColQ : kColDO));
+      tmem_st_wait();
+    }
+    fence_before_sync();
+    __syncwarp();
+    arrive_w(0);
+    arrive_w(1);
     float Dsum = 0.f;
-    bool ok = true;
-    for (int it = 0; it < nit; ++it) {
+    const uint64_t sc2 = f2u(sc, sc);
+    // Sweep 1: D = sum over the attended keys of P * dP.
+    for (int it = 0; ok && it < nblk; ++it) {
       const int b = it & 1;
-      if (!__all_sync(0xffffffffu, wait_or_abort(ctx, &c.s_full[b], (it >> 1) & 1, abort))) {
+      if (!warp_wait(ctx, &c.s_full[b], (it >> 1) & 1, abort)) {
         ok = false;
         break;
       }
       fence_after_sync();
-      const int n = it % nblk;
-      const int m = c.blocks[n];
-      const float bias = c.bias[n];
-      const bool cur = (n == nblk - 1);
-      const int kvalid = min(kB, s.T - m * kB);
-      const bool sweep2 = it >= nblk;
-      uint32_t sr[64], pr[64];
-      tmem_ld32(tl + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tl + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld32(tl + 128 + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&pr[0]));
-      tmem_ld32(tl + 128 + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&pr[32]));
+      const int m = c.blocks[it];
+      const float bias = c.bias[it];
+      const bool cur = (it == nblk - 1);
+      const int kvalid = min(kB, s.T - m * kB) - 32 * grp;
+      uint32_t sr[32], pr[32];
+      tmem_ld32(tl + kColS + b * 64 + 32 * grp, sr);
+      tmem_ld32(tl + kColDP + b * 64 + 32 * grp, pr);
       tmem_ld_wait();
       fence_before_sync();
-      mbar_arrive(&c.s_free[b]);
-      if (cur || kvalid < kB) {
+      __syncwarp();
+      arrive_w(it + 2);
+      if (cur || kvalid < 32) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (i >= kvalid || (cur && i > r)) sr[i] = __float_as_uint(-INFINITY);
+        for (int i = 0; i < 32; ++i)
+          if (i >= kvalid || (cur && i + 32 * grp > r)) sr[i] = __float_as_uint(-INFINITY);
       }
-      // p = 2^(s*scale + bias - lse2); rows past the sequence contribute nothing.
-      const uint64_t sc2 = f2u(sc, sc);
       const float off = live ? bias - lse2 : -INFINITY;
       const uint64_t off2 = f2u(off, off);
-      uint32_t pk[32];
       uint64_t acc0 = 0, acc1 = 0;
-      const uint64_t negD = f2u(-Dsum, -Dsum);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
+      for (int i = 0; i < 16; ++i) {
         const uint64_t a2 = ffma2(f2u(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
                                   sc2, off2);
         const uint64_t p2 = f2u(ex2(lo_f(a2)), ex2(hi_f(a2)));
         const uint64_t dp2 = f2u(__uint_as_float(pr[2 * i]), __uint_as_float(pr[2 * i + 1]));
-        if (!sweep2) {
-          if (i & 1) acc1 = ffma2(p2, dp2, acc1);
-          else acc0 = ffma2(p2, dp2, acc0);
-        } else {
-          const uint64_t ds2 = fmul2(p2, fadd2(dp2, negD));
-          if (i & 1) acc1 = fadd2(acc1, ds2);
-          else acc0 = fadd2(acc0, ds2);
-          pk[i] = pack_bf16(lo_f(ds2), hi_f(ds2));
-        }
+        if (i & 1) acc1 = ffma2(p2, dp2, acc1);
+        else acc0 = ffma2(p2, dp2, acc0);
       }
       const uint64_t accs = fadd2(acc0, acc1);
-      if (!sweep2) {
-        Dsum += lo_f(accs) + hi_f(accs);
-        continue;
-      }
-      const float rowsum = lo_f(accs) + hi_f(accs);
-      const int i2 = it - nblk;
-      // dS buffer (i2 & 1) is free once dQ(i2 - 2) has completed.
-      if (i2 >= 2 && !__all_sync(0xffffffffu, wait_or_abort(ctx, &c.dq_done[i2 & 1],
-                                                            ((i2 - 2) >> 1) & 1, abort))) {
+      Dsum += lo_f(accs) + hi_f(accs);
+    }
+    // The two groups' halves of D meet here; every elementwise warp arrives
+    // exactly once, whichever path it took.
+    c.dpart[grp][rowi] = Dsum;
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    Dsum = c.dpart[0][rowi] + c.dpart[1][rowi];
+    ok = ok && !*abort;
+    const uint64_t negD = f2u(-Dsum, -Dsum);
+    // Sweep 2: dS = P * (dP - D) back into TMEM for the dQ MMA, and its tile sums.
+    for (int it = nblk; ok && it < nit; ++it) {
+      const int b = it & 1, n = it - nblk;
+      if (!warp_wait(ctx, &c.s_full[b], (it >> 1) & 1, abort)) {
         ok = false;
         break;
       }
-      unsigned char* drow = base + kOffDS + (i2 & 1) * 16384 + rowi * 128;
+      fence_after_sync();
+      const int m = c.blocks[n];
+      const float bias = c.bias[n];
+      const bool cur = (n == nblk - 1);
+      const int kvalid = min(kB, s.T - m * kB) - 32 * grp;
+      uint32_t sr[32], pr[32];
+      tmem_ld32(tl + kColS + b * 64 + 32 * grp, sr);
+      tmem_ld32(tl + kColDP + b * 64 + 32 * grp, pr);
+      tmem_ld_wait();
+      if (cur || kvalid < 32) {
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        uint4 v = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-        *reinterpret_cast<uint4*>(drow + ((ch ^ (rowi & 7)) << 4)) = v;
+        for (int i = 0; i < 32; ++i)
+          if (i >= kvalid || (cur && i + 32 * grp > r)) sr[i] = __float_as_uint(-INFINITY);
       }
-      fence_proxy_async_smem();
+      const float off = live ? bias - lse2 : -INFINITY;
+      const uint64_t off2 = f2u(off, off);
+      uint32_t pk[16];
+      uint64_t acc0 = 0, acc1 = 0;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const uint64_t a2 = ffma2(f2u(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
+                                  sc2, off2);
+        const uint64_t p2 = f2u(ex2(lo_f(a2)), ex2(hi_f(a2)));
+        const uint64_t dp2 = f2u(__uint_as_float(pr[2 * i]), __uint_as_float(pr[2 * i + 1]));
+        const uint64_t ds2 = fmul2(p2, fadd2(dp2, negD));
+        if (i & 1) acc1 = fadd2(acc1, ds2);
+        else acc0 = fadd2(acc0, ds2);
+        pk[i] = pack_bf16(lo_f(ds2), hi_f(ds2));
+      }
+      tmem_st16(tl + kColS + b * 64 + 32 * grp, pk);
+      tmem_st_wait();
       fence_before_sync();
-      mbar_arrive(&c.ds_full[i2 & 1]);
+      __syncwarp();
+      if (it + 2 < nit) arrive_w(it + 2);
+      else if (lane == 0) mbar_arrive(&c.ds_tail[it - tail_first]);
       if (!cur) {
-        const float t = warp_sum(rowsum);
-        if (lane == 0) c.red[n][quarter] = t;
+        const uint64_t accs = fadd2(acc0, acc1);
+        const float t = warp_sum(lo_f(accs) + hi_f(accs));
+        if (lane == 0) c.red[n][grp * 4 + quarter] = t;
       }
     }
     if (ok) {
-      const int nl = nblk - 1;
-      if (__all_sync(0xffffffffu,
-                     wait_or_abort(ctx, &c.dq_done[nl & 1], (nl >> 1) & 1, abort))) {
+      if (warp_wait(ctx, &c.dq_done, 0, abort)) {
         fence_after_sync();
-        __nv_bfloat16* drow = dq + hrow * kD;
+        __nv_bfloat16* drow = dq + hrow * kD + grp * 64;
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
+        for (int ch = 0; ch < 2; ++ch) {
           uint32_t ov[32];
-          tmem_ld32(tl + 256 + ch * 32, ov);
+          tmem_ld32(tl + kColDQ + grp * 64 + ch * 32, ov);
           tmem_ld_wait();
           if (live) {
 #pragma unroll
@@ -321,15 +402,15 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
           }
         }
-        if (live) Dv[hrow] = Dsum;
+        if (live && grp == 0) Dv[hrow] = Dsum;
       }
     }
-    // da of each selected block: the four warps' partials in a fixed order.
-    // Every softmax warp reaches this barrier, whichever path it took.
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    // da of each selected block: the eight warps' partials in a fixed order.
+    asm volatile("bar.sync 1, 256;" ::: "memory");
     if (da != nullptr && !*abort) {
-      for (int n = rowi; n < nblk - 1; n += 128) {
-        const float t = (c.red[n][0] + c.red[n][1]) + (c.red[n][2] + c.red[n][3]);
+      for (int n = tid - 128; n < nblk - 1; n += 256) {
+        const float* p = c.red[n];
+        const float t = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
         const long long o0 = (((long long)(bi * s.Hq + h0)) * s.N + j) * s.K + c.slots[n];
         da[o0] = t;
         da[o0 + (long long)s.N * s.K] = 0.f;  // head h0 + 1: the tile's sum sits on h0
@@ -347,16 +428,29 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 // ============================================================================
 // Kernel B: dk, dv
 // ============================================================================
+// One CTA per (key block m, KV head, batch) steps over 128-row query tiles
+// (the diagonal block's, then those of every query block that selected m).
+// MMA stream: per step s, dV/dK(s - 1) then S/dP(s). The MMA thread waits
+// once per step, on the Q/dO stage barrier of step s, which also collects
+// one arrival from each elementwise warp once it has written P/dS of step
+// s - 1 to shared memory (so the S/dP buffer of step s - 2 is free as well).
+// A commit after dV/dK(s - 1) lets the producer reuse that Q/dO stage.
 namespace kb_ {
+constexpr int kWarps = 12;
+constexpr int kThreadsB = kWarps * 32;
 constexpr uint32_t kOffK = 0;         // [d half][64 rows][128 B]
 constexpr uint32_t kOffV = 16384;
 constexpr uint32_t kOffQD = 32768;    // 2 stages x (Q tile 32 KB, dO tile 32 KB)
 constexpr uint32_t kOffP = 163840;    // [128 rows][128 B]
 constexpr uint32_t kOffDS = 180224;
 constexpr uint32_t kOffCtl = 196608;
+// TMEM columns: S[b] at 64 b, dP[b] at 128 + 64 b, dV^T at 256, dK^T at 320.
+constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 320;
 struct Ctl {
-  uint64_t kv_full, qdo_full[2], qdo_empty[2], s_full[2], s_free[2], pds_full, pds_free, acc_done,
-      drain;
+  // qdo_full[stg]: the producer's expect-tx arrival and tile bytes, its
+  // arrival once the step's scalars are staged, and one arrival per
+  // elementwise warp (10 arrivals per phase).
+  uint64_t kv_full, qdo_full[2], s_full[2], dvdk_done[2], pds_tail, acc_done, drain;
   uint32_t tmem_base;
   int abort;
   // Per stage, staged by the producer warp with the Q/dO tiles: the step's
@@ -366,11 +460,10 @@ struct Ctl {
   float lse2[2][128], D[2][128];
 };
 constexpr size_t kSmem = kOffCtl + sizeof(Ctl) + 1024;
-// TMEM columns: S[b] at 64 b, dP[b] at 128 + 64 b, dV^T at 256, dK^T at 320.
 }  // namespace kb_
 
 template <int TILES>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kb_::kThreadsB, 1)
 tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v,
@@ -395,26 +488,31 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int32_t* lst = csr_list + (long long)bh * s.N * s.K + lo;
   const int nsteps = (1 + nl) * TILES;
   // Step s covers tile (s % TILES) of query block j(s): first the diagonal
-  // block m, then the selecting blocks in ascending order.
-  auto qblock = [&](int st) -> int {
-    const int jj = st / TILES;
-    return jj == 0 ? m : lst[jj - 1] / s.K;
-  };
+  // block m, then the selecting blocks in ascending order (entry / K of the
+  // reverse list is the query block).
+  volatile int* abort = &c.abort;
 
   if (tid == 0) {
     mbar_init(&c.kv_full, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&c.qdo_full[i], 2);  // tiles (expect_tx) + staged scalars
-      mbar_init(&c.qdo_empty[i], 1);
+      mbar_init(&c.qdo_full[i], 10);
       mbar_init(&c.s_full[i], 1);
-      mbar_init(&c.s_free[i], 128);
+      mbar_init(&c.dvdk_done[i], 1);
     }
-    mbar_init(&c.pds_full, 128);
-    mbar_init(&c.pds_free, 1);
+    mbar_init(&c.pds_tail, 8);
     mbar_init(&c.acc_done, 1);
     mbar_init(&c.drain, 1);
     fence_mbar_init();
     c.abort = 0;
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    mbar_arrive_expect_tx(&c.kv_full, 32768);
+    for (int h2 = 0; h2 < 2; ++h2) {
+      tma_load_3d(base + kOffK + h2 * 8192, &tm_k, h2 * 64, m * kB, bh, &c.kv_full);
+      tma_load_3d(base + kOffV + h2 * 8192, &tm_v, h2 * 64, m * kB, bh, &c.kv_full);
+    }
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_do);
   }
   if (warp == 1) {
     tmem_alloc(&c.tmem_base, kTmemCols);
@@ -424,26 +522,52 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = c.tmem_base;
-  volatile int* abort = &c.abort;
 
   if (warp == 0) {
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_do);
-      mbar_arrive_expect_tx(&c.kv_full, 32768);
-      for (int h2 = 0; h2 < 2; ++h2) {
-        tma_load_3d(base + kOffK + h2 * 8192, &tm_k, h2 * 64, m * kB, bh, &c.kv_full);
-        tma_load_3d(base + kOffV + h2 * 8192, &tm_v, h2 * 64, m * kB, bh, &c.kv_full);
+    // Scalars of a step (lse in the log2 domain and D of the tile's 128 rows,
+    // four per lane, the query block and its gate bias) are loaded into
+    // registers one step ahead, so staging them costs only shared stores.
+    float pre_lse[4], pre_D[4], pre_bias = 0.f;
+    int pre_j = m;
+    // The reverse list in a register window (lane l holds entry win_lo + l),
+    // with the next window already in flight.
+    int win_lo = 0;
+    int win = lane < nl ? lst[lane] : 0;
+    int win_next = 32 + lane < nl ? lst[32 + lane] : 0;
+    auto prefetch = [&](int st_i) {
+      const int jj = st_i / TILES, u = st_i % TILES;
+      int j = m;
+      if (jj > 0) {
+        const int ix = jj - 1;
+        while (ix >= win_lo + 32) {
+          win = win_next;
+          win_lo += 32;
+          win_next = win_lo + 32 + lane < nl ? lst[win_lo + 32 + lane] : 0;
+        }
+        j = __shfl_sync(0xffffffffu, win, ix - win_lo) / s.K;
       }
-    }
+      pre_j = j;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const int rr = lane + 32 * q4;
+        const int head = kvh * G + 2 * u + (rr >> 6), qrow = j * kB + (rr & 63);
+        const bool live = qrow < s.T;
+        const long long hrow = (long long)(bi * s.Hq + head) * s.T + qrow;
+        pre_lse[q4] = live ? lse[hrow] : 0.f;
+        pre_D[q4] = live ? Dv[hrow] : 0.f;
+      }
+      pre_bias = (j == m || gates == nullptr) ? 1.f : gates[((long long)bh * s.N + j) * s.N + m];
+    };
+    prefetch(0);
     int issued = 0;
     for (int st_i = 0; st_i < nsteps; ++st_i) {
       const int stg = st_i & 1;
       bool go = true;
+      // The stage is free once dV/dK of step st_i - 2 completed.
       if (lane == 0 && st_i >= 2)
-        go = wait_or_abort(ctx, &c.qdo_empty[stg], ((st_i - 2) >> 1) & 1, abort);
+        go = wait_or_abort(ctx, &c.dvdk_done[stg], ((st_i - 2) >> 1) & 1, abort);
       if (!__shfl_sync(0xffffffffu, go, 0)) break;
-      const int j = qblock(st_i), u = st_i % TILES;
+      const int j = pre_j, u = st_i % TILES;
       if (lane == 0) {
         unsigned char* qd = base + kOffQD + stg * 65536;
         mbar_arrive_expect_tx(&c.qdo_full[stg], 65536);
@@ -456,26 +580,22 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                         &c.qdo_full[stg]);
           }
       }
-      // Scalars of the step: every lane stages 4 rows of lse (log2 domain) and D.
-      for (int rr = lane; rr < 128; rr += 32) {
-        const int head = kvh * G + 2 * u + (rr >> 6), qrow = j * kB + (rr & 63);
-        const bool live = qrow < s.T;
-        const long long hrow = (long long)(bi * s.Hq + head) * s.T + qrow;
-        c.lse2[stg][rr] = live ? lse[hrow] * kLog2e : 0.f;
-        c.D[stg][rr] = live ? Dv[hrow] : 0.f;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        c.lse2[stg][lane + 32 * q4] = pre_lse[q4] * kLog2e;
+        c.D[stg][lane + 32 * q4] = pre_D[q4];
       }
       if (lane == 0) {
         c.step_j[stg] = j;
-        c.step_bias[stg] = (j == m || gates == nullptr)
-                               ? 0.f
-                               : logf(gates[((long long)bh * s.N + j) * s.N + m]) * kLog2e;
+        c.step_bias[stg] = logf(pre_bias) * kLog2e;
       }
       __threadfence_block();
       __syncwarp();
-      // The consumers see the staged scalars once this stage's Q/dO tiles
-      // have landed: the arrival below is part of the same barrier phase.
+      // The consumers see the staged scalars once this stage's barrier phase
+      // completes: the arrival below is part of it.
       if (lane == 0) mbar_arrive(&c.qdo_full[stg]);
       issued = st_i + 1;
+      if (st_i + 1 < nsteps) prefetch(st_i + 1);
     }
     if (lane == 0 && *abort) {
       (void)mbar_wait(ctx, &c.kv_full, 0);
@@ -486,75 +606,60 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16(128, 64, false, false);
       const uint32_t id_t = idesc_bf16(128, 64, true, true);
-      bool ok = wait_or_abort(ctx, &c.kv_full, 0, abort);
-      fence_after_sync();
-      auto issue_s = [&](int st_i) -> bool {
+      const uint64_t dq0 = sdesc_sw128(sbase + kOffQD, 16, 1024);    // Q/dO stages, K-major
+      const uint64_t dk0 = sdesc_sw128(sbase + kOffK, 16, 1024);     // K (V at +16 KB)
+      const uint64_t dqt0 = sdesc_sw128(sbase + kOffQD, 16384, 1024);  // Q/dO as MN-major A
+      const uint64_t dp0 = sdesc_sw128(sbase + kOffP, 8192, 1024);   // P (dS at +16 KB)
+      auto issue_sdp = [&](int st_i) {
         const int stg = st_i & 1, b = st_i & 1;
-        if (!wait_or_abort(ctx, &c.qdo_full[stg], (st_i >> 1) & 1, abort)) return false;
-        if (st_i >= 2 && !wait_or_abort(ctx, &c.s_free[b], ((st_i - 2) >> 1) & 1, abort))
-          return false;
-        fence_after_sync();
-        const uint32_t qa = sbase + kOffQD + stg * 65536;
+        const uint64_t qa = dq0 + ((stg * 65536) >> 4);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t ao = (ks >> 2) * 16384 + (ks & 3) * 32;
           const uint32_t bo = (ks >> 2) * 8192 + (ks & 3) * 32;
-          mma_bf16_ss(tmem + b * 64, sdesc_sw128(qa + ao, 16, 1024),
-                      sdesc_sw128(sbase + kOffK + bo, 16, 1024), id_s, ks > 0);
+          mma_bf16_ss(tmem + kColS + b * 64, qa + (ao >> 4), dk0 + (bo >> 4), id_s, ks > 0);
         }
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t ao = (ks >> 2) * 16384 + (ks & 3) * 32;
-          const uint32_t bo = (ks >> 2) * 8192 + (ks & 3) * 32;
-          mma_bf16_ss(tmem + 128 + b * 64, sdesc_sw128(qa + 32768 + ao, 16, 1024),
-                      sdesc_sw128(sbase + kOffV + bo, 16, 1024), id_s, ks > 0);
+          const uint32_t ao = 32768 + (ks >> 2) * 16384 + (ks & 3) * 32;
+          const uint32_t bo = 16384 + (ks >> 2) * 8192 + (ks & 3) * 32;
+          mma_bf16_ss(tmem + kColDP + b * 64, qa + (ao >> 4), dk0 + (bo >> 4), id_s, ks > 0);
         }
         mma_commit(&c.s_full[b]);
-        return true;
       };
       // dV^T[d][key] += sum_q dO[q][d] P[q][key]; dK^T[d][key] += sum_q Q[q][d] dS[q][key]
-      auto retire = [&](int st_i) {
-        fence_after_sync();
-        const uint32_t qa = sbase + kOffQD + (st_i & 1) * 65536;
+      auto issue_dvdk = [&](int st_i) {
+        const uint64_t qa = dqt0 + (((st_i & 1) * 65536) >> 4);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          mma_bf16_ss(tmem + 256, sdesc_sw128(qa + 32768 + ks * 2048, 16384, 1024),
-                      sdesc_sw128(sbase + kOffP + ks * 2048, 8192, 1024), id_t,
-                      (st_i > 0 || ks > 0));
+          mma_bf16_ss(tmem + kColDV, qa + ((32768 + ks * 2048) >> 4), dp0 + ((ks * 2048) >> 4),
+                      id_t, (st_i > 0 || ks > 0));
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          mma_bf16_ss(tmem + 320, sdesc_sw128(qa + ks * 2048, 16384, 1024),
-                      sdesc_sw128(sbase + kOffDS + ks * 2048, 8192, 1024), id_t,
-                      (st_i > 0 || ks > 0));
-        mma_commit(&c.pds_free);
-        mma_commit(&c.qdo_empty[st_i & 1]);
+          mma_bf16_ss(tmem + kColDK, qa + ((ks * 2048) >> 4), dp0 + ((16384 + ks * 2048) >> 4),
+                      id_t, (st_i > 0 || ks > 0));
       };
-      if (ok) ok = issue_s(0);
-      // Order by readiness: the next step's S/dP go first when its Q/dO tile
-      // has landed (they then overlap this step's softmax); otherwise this
-      // step's dV/dK go first, which frees the stage that the load after the
-      // next one is waiting for.
+      bool ok = wait_or_abort(ctx, &c.kv_full, 0, abort);
+      // Per step s: one wait (the Q/dO tiles of step s have landed and P/dS
+      // of step s - 1 is in shared memory), then dV/dK(s - 1), which frees
+      // the Q/dO stage of step s - 1, then S/dP(s). The commit after S/dP(s)
+      // also covers dV/dK(s - 1): the elementwise warps, waiting for S/dP(s),
+      // then know that the P/dS buffer is free again.
       for (int st_i = 0; ok && st_i < nsteps; ++st_i) {
-        const int nxt = st_i + 1;
-        bool next_issued = nxt >= nsteps;
-        bool retired = false;
-        for (unsigned long long polls = 0; ok && !retired; ++polls) {
-          if (!next_issued && mbar_try_wait(&c.qdo_full[nxt & 1], (nxt >> 1) & 1)) {
-            if (!issue_s(nxt)) ok = false;
-            next_issued = true;
-          }
-          if (ok && mbar_try_wait(&c.pds_full, st_i & 1)) {
-            retire(st_i);
-            retired = true;
-          } else if (polls >= ctx.wait_limit) {
-            report(ctx, kDevErrTimeout);
-            *abort = 1;
-            ok = false;
-          } else if ((polls & 63) == 63 && *abort) {
-            ok = false;
-          }
+        if (!wait_or_abort(ctx, &c.qdo_full[st_i & 1], (st_i >> 1) & 1, abort)) {
+          ok = false;
+          break;
         }
-        if (ok && !next_issued && !issue_s(nxt)) ok = false;
+        fence_after_sync();
+        if (st_i > 0) {
+          issue_dvdk(st_i - 1);
+          mma_commit(&c.dvdk_done[(st_i - 1) & 1]);
+        }
+        issue_sdp(st_i);
+      }
+      if (ok && wait_or_abort(ctx, &c.pds_tail, 0, abort)) {
+        fence_after_sync();
+        issue_dvdk(nsteps - 1);
       }
       mma_commit(&c.acc_done);
       if (*abort) {
@@ -563,16 +668,19 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
     }
   } else if (warp >= 4) {
-    const int quarter = warp & 3;
+    const int quarter = warp & 3, grp = (warp - 4) >> 2;
     const int rowi = quarter * 32 + lane;  // tile row (query) / d index in the epilogue
     const int r = rowi & 63;
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
     const float sc = s.scale * kLog2e;
-    const int kvalid = min(kB, s.T - m * kB);
+    const int kvalid = min(kB, s.T - m * kB) - 32 * grp;
+    const uint64_t sc2 = f2u(sc, sc);
+    // Step 0 has no P/dS of a previous step to wait for.
+    if (lane == 0) mbar_arrive(&c.qdo_full[0]);
     bool ok = true;
     for (int st_i = 0; st_i < nsteps; ++st_i) {
       const int b = st_i & 1;
-      if (!__all_sync(0xffffffffu, wait_or_abort(ctx, &c.s_full[b], (st_i >> 1) & 1, abort))) {
+      if (!warp_wait(ctx, &c.s_full[b], (st_i >> 1) & 1, abort)) {
         ok = false;
         break;
       }
@@ -585,24 +693,19 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       const float Di = c.D[stg][rowi];
       const bool cur = (j == m);
       const float bias = c.step_bias[stg];
-      uint32_t sr[64], pr[64], pp[32], dd[32];
-      tmem_ld32(tl + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tl + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld32(tl + 128 + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&pr[0]));
-      tmem_ld32(tl + 128 + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&pr[32]));
+      uint32_t sr[32], pr[32], pp[16], dd[16];
+      tmem_ld32(tl + kColS + b * 64 + 32 * grp, sr);
+      tmem_ld32(tl + kColDP + b * 64 + 32 * grp, pr);
       tmem_ld_wait();
-      fence_before_sync();
-      mbar_arrive(&c.s_free[b]);
-      if (cur || kvalid < kB) {
+      if (cur || kvalid < 32) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (i >= kvalid || (cur && i > r)) sr[i] = __float_as_uint(-INFINITY);
+        for (int i = 0; i < 32; ++i)
+          if (i >= kvalid || (cur && i + 32 * grp > r)) sr[i] = __float_as_uint(-INFINITY);
       }
-      const uint64_t sc2 = f2u(sc, sc);
       const float off = live ? bias - lse2 : -INFINITY;
       const uint64_t off2 = f2u(off, off), negD = f2u(-Di, -Di);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
+      for (int i = 0; i < 16; ++i) {
         const uint64_t a2 = ffma2(f2u(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
                                   sc2, off2);
         const float p0 = ex2(lo_f(a2)), p1 = ex2(hi_f(a2));
@@ -611,17 +714,13 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
         pp[i] = pack_bf16(p0, p1);
         dd[i] = pack_bf16(lo_f(ds2), hi_f(ds2));
       }
-      // The P / dS buffers are free once step st_i - 1's dV/dK MMAs completed.
-      if (st_i >= 1 && !__all_sync(0xffffffffu,
-                                   wait_or_abort(ctx, &c.pds_free, (st_i - 1) & 1, abort))) {
-        ok = false;
-        break;
-      }
+      // The P / dS buffers are free: dV/dK of step st_i - 1 was issued before
+      // S/dP(st_i), whose completion this warp waited for.
       unsigned char* prow = base + kOffP + rowi * 128;
       unsigned char* drow = base + kOffDS + rowi * 128;
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const uint32_t sw = (ch ^ (rowi & 7)) << 4;
+      for (int ch = 0; ch < 4; ++ch) {
+        const uint32_t sw = ((4 * grp + ch) ^ (rowi & 7)) << 4;
         *reinterpret_cast<uint4*>(prow + sw) = make_uint4(pp[4 * ch], pp[4 * ch + 1],
                                                           pp[4 * ch + 2], pp[4 * ch + 3]);
         *reinterpret_cast<uint4*>(drow + sw) = make_uint4(dd[4 * ch], dd[4 * ch + 1],
@@ -629,10 +728,14 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       fence_proxy_async_smem();
       fence_before_sync();
-      mbar_arrive(&c.pds_full);
+      __syncwarp();
+      if (lane == 0) {
+        if (st_i + 1 < nsteps) mbar_arrive(&c.qdo_full[(st_i + 1) & 1]);
+        else mbar_arrive(&c.pds_tail);
+      }
     }
-    if (ok && __all_sync(0xffffffffu, wait_or_abort(ctx, &c.acc_done, 0, abort))) {
-      // Epilogue: thread rowi holds dimension d = rowi of all 64 keys.
+    if (ok && warp_wait(ctx, &c.acc_done, 0, abort)) {
+      // Epilogue: thread rowi holds dimension d = rowi; group g the keys 32g .. 32g + 31.
       fence_after_sync();
       const int d = rowi;
       const long long kb0 = ((long long)bh * s.T + (long long)m * kB) * kD;
@@ -640,17 +743,14 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       for (int which = 0; which < 2; ++which) {
         __nv_bfloat16* out = which == 0 ? dv : dk;
         const float mul = which == 0 ? 1.f : s.scale;
+        uint32_t v[32];
+        tmem_ld32(tl + (which == 0 ? kColDV : kColDK) + grp * 32, v);
+        tmem_ld_wait();
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t v[32];
-          tmem_ld32(tl + 256 + which * 64 + half * 32, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int key = half * 32 + i;
-            if (key < kvalid) out[kb0 + (long long)key * kD + d] =
-                __float2bfloat16_rn(__uint_as_float(v[i]) * mul);
-          }
+        for (int i = 0; i < 32; ++i) {
+          const int key = grp * 32 + i;
+          if (i < kvalid) out[kb0 + (long long)key * kD + d] =
+              __float2bfloat16_rn(__uint_as_float(v[i]) * mul);
         }
       }
     }
@@ -694,7 +794,7 @@ cudaError_t launch_attn_bwd_tc(const AttnShape& s, const void* q, const void* k,
     auto kern = tiles == 2 ? tc_bwd_dq_kernel<2> : tc_bwd_dq_kernel<1>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ka::kSmem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, ka::kSmem, st>>>(tq, tk, tv, tdo, lse, idx, gates, s,
+    kern<<<grid, ka::kThreadsA, ka::kSmem, st>>>(tq, tk, tv, tdo, lse, idx, gates, s,
                                             (__nv_bfloat16*)dq, Dv, dscores ? da : nullptr, ctx);
     note_launches(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -704,7 +804,7 @@ cudaError_t launch_attn_bwd_tc(const AttnShape& s, const void* q, const void* k,
     auto kern = tiles == 2 ? tc_bwd_dkdv_kernel<2> : tc_bwd_dkdv_kernel<1>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kb_::kSmem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, kb_::kSmem, st>>>(tq, tk, tv, tdo, lse, Dv, gates, coff, clist, s,
+    kern<<<grid, kb_::kThreadsB, kb_::kSmem, st>>>(tq, tk, tv, tdo, lse, Dv, gates, coff, clist, s,
                                              (__nv_bfloat16*)dk, (__nv_bfloat16*)dv, ctx);
     note_launches(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
