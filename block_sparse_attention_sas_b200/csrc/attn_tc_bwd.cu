@@ -78,14 +78,6 @@ __device__ __forceinline__ uint32_t stage_off(int st) {
 }
 }  // namespace ka
 
-// One lane of the warp polls the barrier; the others wait at the shuffle.
-__device__ __forceinline__ bool warp_wait(const DevCtx& ctx, uint64_t* bar, uint32_t parity,
-                                          volatile int* abort) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = wait_or_abort(ctx, bar, parity, abort) ? 1 : 0;
-  return __shfl_sync(0xffffffffu, ok, 0) != 0;
-}
-
 template <int TILES>
 __global__ void __launch_bounds__(ka::kThreadsA, 1)
 tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -430,11 +422,12 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 // ============================================================================
 // One CTA per (key block m, KV head, batch) steps over 128-row query tiles
 // (the diagonal block's, then those of every query block that selected m).
-// MMA stream: per step s, dV/dK(s - 1) then S/dP(s). The MMA thread waits
+// MMA stream: per step s, S/dP(s) then dV/dK(s - 1). The MMA thread waits
 // once per step, on the Q/dO stage barrier of step s, which also collects
 // one arrival from each elementwise warp once it has written P/dS of step
 // s - 1 to shared memory (so the S/dP buffer of step s - 2 is free as well).
-// A commit after dV/dK(s - 1) lets the producer reuse that Q/dO stage.
+// A commit after dV/dK(s - 1) lets the producer reuse that Q/dO stage and
+// the elementwise warps the P/dS buffer.
 namespace kb_ {
 constexpr int kWarps = 12;
 constexpr int kThreadsB = kWarps * 32;
@@ -641,21 +634,20 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       };
       bool ok = wait_or_abort(ctx, &c.kv_full, 0, abort);
       // Per step s: one wait (the Q/dO tiles of step s have landed and P/dS
-      // of step s - 1 is in shared memory), then dV/dK(s - 1), which frees
-      // the Q/dO stage of step s - 1, then S/dP(s). The commit after S/dP(s)
-      // also covers dV/dK(s - 1): the elementwise warps, waiting for S/dP(s),
-      // then know that the P/dS buffer is free again.
+      // of step s - 1 is in shared memory), then S/dP(s), so the elementwise
+      // warps can start on it, then dV/dK(s - 1); its commit frees the Q/dO
+      // stage of step s - 1 and the P/dS buffer.
       for (int st_i = 0; ok && st_i < nsteps; ++st_i) {
         if (!wait_or_abort(ctx, &c.qdo_full[st_i & 1], (st_i >> 1) & 1, abort)) {
           ok = false;
           break;
         }
         fence_after_sync();
+        issue_sdp(st_i);
         if (st_i > 0) {
           issue_dvdk(st_i - 1);
           mma_commit(&c.dvdk_done[(st_i - 1) & 1]);
         }
-        issue_sdp(st_i);
       }
       if (ok && wait_or_abort(ctx, &c.pds_tail, 0, abort)) {
         fence_after_sync();
@@ -714,8 +706,11 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
         pp[i] = pack_bf16(p0, p1);
         dd[i] = pack_bf16(lo_f(ds2), hi_f(ds2));
       }
-      // The P / dS buffers are free: dV/dK of step st_i - 1 was issued before
-      // S/dP(st_i), whose completion this warp waited for.
+      // The P / dS buffers are free once dV/dK of step st_i - 1 completed.
+      if (st_i >= 1 && !warp_wait(ctx, &c.dvdk_done[(st_i - 1) & 1], ((st_i - 1) >> 1) & 1, abort)) {
+        ok = false;
+        break;
+      }
       unsigned char* prow = base + kOffP + rowi * 128;
       unsigned char* drow = base + kOffDS + rowi * 128;
 #pragma unroll

@@ -447,11 +447,12 @@ cudaError_t decode_g(const DecodeShape& s, const void* q, const void* kc, const 
 }  // namespace
 
 void decode_plan(DecodeShape& s) {
-  // About two CTAs per SM (148 SMs), at most kMaxSplits per (batch, kv head).
+  // At most two CTAs per SM (148 SMs) in one wave, at most kMaxSplits per
+  // (batch, kv head).
   const int nslots = s.dense ? s.C + 1 : s.K + 1;
   const int units = s.B * s.Hkv;
   const int target = 2 * 148;
-  int splits = (target + units - 1) / units;
+  int splits = target / units;
   splits = max(1, min(splits, min(nslots, kMaxSplits)));
   int bps = (nslots + splits - 1) / splits;
   splits = (nslots + bps - 1) / bps;
@@ -503,6 +504,7 @@ cudaError_t decode_noalloc_scratch(void** out) {
 cudaError_t launch_decode(sas_dtype_t dt, const DecodeShape& s, const void* q, const void* kc,
                           const void* vc, const int32_t* idx, const float* gates, void* o,
                           void* ws, const DevCtx& ctx, cudaStream_t st) {
+  if (tc_decode_supported(dt, s)) return launch_decode_tc(s, q, kc, vc, idx, gates, o, ws, ctx, st);
   if (dt == SAS_F32) {
     if (s.d == 64) return decode_g<float, 64>(s, q, kc, vc, idx, gates, o, ws, ctx, st);
     return decode_g<float, 128>(s, q, kc, vc, idx, gates, o, ws, ctx, st);

@@ -78,6 +78,14 @@ cudaError_t launch_decode(sas_dtype_t dt, const DecodeShape& s, const void* q, c
                           const void* vc, const int32_t* idx, const float* gates, void* o,
                           void* ws, const DevCtx& ctx, cudaStream_t stream);
 
+// Tensor-core (tcgen05) decode: bf16 cache, d = 128, b = 64, G <= 8.
+bool tc_decode_supported(sas_dtype_t dt, const DecodeShape& s);
+cudaError_t launch_decode_tc(const DecodeShape& s, const void* q, const void* kc, const void* vc,
+                             const int32_t* idx, const float* gates, void* o, void* ws,
+                             const DevCtx& ctx, cudaStream_t stream);
+// 3-D TMA map over planes of `pitch_rows` rows, the first `rows` of each mapped.
+cudaError_t make_tmap_bf16_pitched(void* map, const void* ptr, int rows, int pitch_rows,
+                                   int planes);
 // Fixed-size device scratch for sas_decode_noalloc (no allocation involved).
 size_t decode_noalloc_capacity();
 cudaError_t decode_noalloc_scratch(void** out);

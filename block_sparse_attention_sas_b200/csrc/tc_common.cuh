@@ -268,5 +268,13 @@ __device__ __forceinline__ bool wait_or_abort(const DevCtx& c, uint64_t* bar, ui
   return false;
 }
 
+// One lane of the warp polls the barrier; the others wait at the shuffle.
+__device__ __forceinline__ bool warp_wait(const DevCtx& ctx, uint64_t* bar, uint32_t parity,
+                                          volatile int* abort) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = wait_or_abort(ctx, bar, parity, abort) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
 }  // namespace tc
 }  // namespace sas

@@ -222,6 +222,40 @@ def test_wait_timeout_is_reported(cuda_lib):
     assert float((x * 2).sum()) == 8.0
 
 
+@pytest.mark.parametrize("kw", [
+    dict(B=2, Hq=8, Hkv=2, L=1000, d=128, b=64, K=6, dtype="bf16"),
+    dict(B=1, Hq=5, Hkv=1, L=4033, d=128, b=64, K=9, dtype="bf16"),
+    dict(B=2, Hq=4, Hkv=2, L=1000, d=128, b=64, K=4, dtype="f32"),
+])
+def test_decode_cache_capacity_tail_is_ignored(cuda_lib, kw):
+    """Caches of capacity Lcap > L: rows L.. hold NaN and must not reach o."""
+    dc = W.small_decode_config(**kw)
+    x = W.make_decode_inputs(dc)
+    s = x.scores[:, :, None, :]
+    gates, idx = cuda_lib.gate_topk(dev(s, "f32"), dc.K, causal=False)
+    og, olg, oi = O.gate_topk(s, dc.K, causal=False)
+    q = dev(x.q, dc.dtype)
+    Lcap = dc.L + 200
+    caches = []
+    for a in (x.kcache, x.vcache):
+        full = torch.full((dc.B, dc.Hkv, Lcap, dc.d), float("nan"), device="cuda",
+                          dtype=torch.bfloat16 if dc.dtype == "bf16" else torch.float32)
+        full[:, :, :dc.L] = dev(a, dc.dtype)
+        caches.append(full)
+    for use_gates in (False, True):
+        o = cuda_lib.decode(q, caches[0], caches[1], idx[:, :, 0].contiguous(),
+                            gates[:, :, 0].contiguous(), use_gates, dc.b, L=dc.L)
+        torch.cuda.synchronize()
+        assert cuda_lib.device_error()[0] == 0
+        want = O.decode(x.q, x.kcache, x.vcache, oi[:, :, 0], olg[:, :, 0], dc.b,
+                        use_gates=use_gates)
+        check("decode o (Lcap > L)", host(o), want, dc.dtype)
+    od = cuda_lib.dense_decode(q, caches[0], caches[1], L=dc.L)
+    torch.cuda.synchronize()
+    check("dense decode o (Lcap > L)", host(od), O.dense_decode(x.q, x.kcache, x.vcache),
+          dc.dtype)
+
+
 def test_decode_idx_with_holes(cuda_lib):
     """-1 entries anywhere in an idx row are skipped (decode and oracle alike)."""
     dc = W.small_decode_config(B=2, Hq=8, Hkv=2, L=3000, d=128, b=64, K=12, dtype="bf16")
