@@ -410,6 +410,32 @@ def run_decode_only(args):
     print(json.dumps({"decode": lines}), flush=True)
 
 
+def run_profile_train(args):
+    """The training step (gate_topk, forward, backward) of the Qwen3-4B layer
+    shape at a shorter sequence length, for kernel captures: warm-up steps,
+    then `steps` more, with no timing and no decode."""
+    import torch
+    from block_sparse_attention_sas_b200 import _lib as S
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cfg = W.small_train_config(B=1, Hq=32, Hkv=8, T=args.profile_train, d=128, b=64, K=16,
+                               dtype="bf16", hot_key_frac=0.05, hot_key_scale=3.0)
+    x = W.make_train_inputs(cfg)
+    t = {n: torch.from_numpy(getattr(x, n)).to(dev).to(torch.bfloat16)
+         for n in ("q", "k", "v", "dO")}
+    scores = torch.from_numpy(x.scores).to(dev)
+    for _ in range(args.warmup + args.steps):
+        gates, idx = S.gate_topk(scores, cfg.K)
+        o, lse = S.attn_fwd(t["q"], t["k"], t["v"], idx, gates, cfg.b)
+        S.attn_bwd(t["q"], t["k"], t["v"], o, lse, t["dO"], idx, gates, cfg.b)
+    torch.cuda.synchronize(dev)
+    st, raw = S.device_error()
+    print(json.dumps({"profile_train": cfg.name, "steps": args.warmup + args.steps,
+                      "device_error": st}), flush=True)
+    if st != 0:
+        raise SystemExit(1)
+
+
 # ----------------------------------------------------------- reference arm
 
 def run_reference(args):
@@ -453,6 +479,8 @@ def main():
     ap.add_argument("--cpu-heads", type=int, default=2)
     ap.add_argument("--decode-only", default=None, metavar="PRESET",
                     help="time only the decode path of one preset (for profiling)")
+    ap.add_argument("--profile-train", type=int, default=0, metavar="T",
+                    help="run only the training step at sequence length T (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -460,6 +488,8 @@ def main():
         run_reference(args)
     elif args.decode_only:
         run_decode_only(args)
+    elif args.profile_train:
+        run_profile_train(args)
     else:
         run_ours(args)
 

@@ -36,7 +36,7 @@ SIGNATURES = {
     "sas_launch_count": (ctypes.c_uint64, []),
     "sas_gate_topk": (_i, [_p, _i, _i, _i, _i, _i, _i, _p, _p, _p]),
     "sas_attn_fwd": (_i, [_i, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p]),
-    "sas_attn_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "sas_attn_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i]),
     "sas_attn_bwd": (_i, [_i, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f,
                           _p, _p, _p, _p, _p, _sz, _p]),
     "sas_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
@@ -165,7 +165,7 @@ def attn_bwd(q, k, v, o, lse, dO, idx, gates, b: int, scale: float = 0.0,
     ds = None
     if gates is not None and want_dscores:
         ds = torch.empty((B, Hkv, N, N), dtype=torch.float32, device=q.device)
-    nbytes = LIB.sas_attn_bwd_workspace_size(B, Hq, Hkv, T, d, b, K)
+    nbytes = LIB.sas_attn_bwd_workspace_size(_dtype(q), B, Hq, Hkv, T, d, b, K)
     ws = _workspace("bwd", nbytes, q.device, zero=False)
     _check("sas_attn_bwd", LIB.sas_attn_bwd(_dtype(q), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
                                             _ptr(lse), _ptr(dO), _ptr(idx), _ptr(gates), B, Hq,

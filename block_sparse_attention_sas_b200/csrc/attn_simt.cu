@@ -182,50 +182,108 @@ fwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict
 // j*K + slot for every query block j whose slot selects key block m, in
 // ascending j. One CTA per (batch, kv head).
 // ---------------------------------------------------------------------------
+constexpr int kCsrChunk = 16384;  // idx entries staged in shared memory at a time
+
+// In-place exclusive prefix sum of a[0..n) in shared memory by the whole CTA
+// (blockDim.x a multiple of 32, at most 1024); returns the total.
+__device__ int block_exclusive_scan(int32_t* a, int n, int32_t* warp_tot) {
+  const int nt = blockDim.x, t = threadIdx.x, lane = t & 31, w = t >> 5;
+  const int per = (n + nt - 1) / nt;
+  const int lo = min(n, t * per), hi = min(n, lo + per);
+  int sum = 0;
+  for (int i = lo; i < hi; ++i) sum += a[i];
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int x = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += x;
+  }
+  if (lane == 31) warp_tot[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    int v = lane < nt / 32 ? warp_tot[lane] : 0;
+    int vi = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, vi, o);
+      if (lane >= o) vi += x;
+    }
+    if (lane < nt / 32) warp_tot[lane] = vi - v;  // exclusive warp offsets
+    if (lane == 31) warp_tot[32] = vi;            // total
+  }
+  __syncthreads();
+  int run = warp_tot[w] + incl - sum;
+  for (int i = lo; i < hi; ++i) {
+    const int x = a[i];
+    a[i] = run;
+    run += x;
+  }
+  const int total = warp_tot[32];
+  __syncthreads();
+  return total;
+}
+
+// Reverse index of one (batch, KV head): for each key block m, the entries
+// e = j*K + slot with idx[e] == m (m < j), in ascending order of e (so of j).
+// The entries pass through shared memory in chunks (all threads load, many
+// loads in flight); counts by shared-memory atomics and a block scan; then
+// one warp walks the entries in order and places each at its key block's
+// cursor (lanes holding the same block are ranked within the warp), so the
+// lists come out sorted without a sort.
 __global__ void __launch_bounds__(kThreads)
 csr_kernel(const int32_t* __restrict__ idx, AttnShape s, int32_t* __restrict__ off_all,
            int32_t* __restrict__ list_all, DevCtx ctx) {
-  extern __shared__ int32_t cnt[];  // N counts, then N cursors
-  int32_t* cursor = cnt + s.N;
+  extern __shared__ int32_t cnt[];  // N counts (then cursors), then a chunk of entries
+  int32_t* stage = cnt + s.N;
+  __shared__ int32_t warp_tot[33];
   const int bh = blockIdx.x;
   const int32_t* ix = idx + (long long)bh * s.N * s.K;
   int32_t* off = off_all + (long long)bh * (s.N + 1);
   int32_t* list = list_all + (long long)bh * s.N * s.K;
-  for (int m = threadIdx.x; m < s.N; m += kThreads) cnt[m] = 0;
-  __syncthreads();
   const int total = s.N * s.K;
-  for (int e = threadIdx.x; e < total; e += kThreads) {
-    const int j = e / s.K, m = ix[e];
-    if (m >= 0 && m < j) atomicAdd(&cnt[m], 1);
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int run = 0;
-    for (int m = 0; m < s.N; ++m) {
-      const int c = cnt[m];
-      off[m] = run;
-      cursor[m] = run;
-      run += c;
+  const bool one_chunk = total <= kCsrChunk;
+  auto load_chunk = [&](int c0, int nc) {
+#pragma unroll 8
+    for (int i = threadIdx.x; i < nc; i += blockDim.x) stage[i] = __ldg(ix + c0 + i);
+  };
+  for (int m = threadIdx.x; m < s.N; m += blockDim.x) cnt[m] = 0;
+  for (int c0 = 0; c0 < total; c0 += kCsrChunk) {
+    const int nc = min(kCsrChunk, total - c0);
+    __syncthreads();
+    load_chunk(c0, nc);
+    __syncthreads();
+    for (int i = threadIdx.x; i < nc; i += blockDim.x) {
+      const int e = c0 + i, m = stage[i];
+      if (m >= 0 && m < e / s.K) atomicAdd(&cnt[m], 1);
     }
-    off[s.N] = run;
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < total; e += kThreads) {
-    const int j = e / s.K, m = ix[e];
-    if (m >= 0 && m < j) list[atomicAdd(&cursor[m], 1)] = e;
-  }
-  __syncthreads();
-  // Sort each list ascending (e = j*K + slot, so this orders by j).
-  for (int m = threadIdx.x; m < s.N; m += kThreads) {
-    const int lo = off[m], hi = off[m + 1];
-    for (int a = lo + 1; a < hi; ++a) {
-      const int x = list[a];
-      int b = a - 1;
-      while (b >= lo && list[b] > x) {
-        list[b + 1] = list[b];
-        --b;
+  const int n_all = block_exclusive_scan(cnt, s.N, warp_tot);
+  for (int m = threadIdx.x; m < s.N; m += blockDim.x) off[m] = cnt[m];
+  if (threadIdx.x == 0) off[s.N] = n_all;
+  for (int c0 = 0; c0 < total; c0 += kCsrChunk) {
+    const int nc = min(kCsrChunk, total - c0);
+    if (!one_chunk) {
+      __syncthreads();
+      load_chunk(c0, nc);
+      __syncthreads();
+    }
+    if (threadIdx.x < 32) {
+      const int lane = threadIdx.x;
+      const uint32_t lt = (1u << lane) - 1u;
+      for (int c = 0; c < nc; c += 32) {
+        const int e = c0 + c + lane;
+        const int m = c + lane < nc ? stage[c + lane] : -1;
+        const bool valid = m >= 0 && m < e / s.K;
+        const int key = valid ? m : -1 - lane;  // invalid lanes match nobody
+        const uint32_t peers = __match_any_sync(0xffffffffu, key);
+        int pos = 0;
+        if (valid) pos = cnt[m] + __popc(peers & lt);
+        __syncwarp();
+        if (valid && (peers & lt) == 0) cnt[m] += __popc(peers);  // the group's leader
+        __syncwarp();
+        if (valid) list[pos] = e;
       }
-      list[b + 1] = x;
     }
   }
 }
@@ -561,7 +619,7 @@ cudaError_t bwd_t(const AttnShape& s, const void* q, const void* k, const void* 
                   const float* lse, const void* dO, const int32_t* idx, const float* gates,
                   void* dq, void* dk, void* dv, float* dscores, void* ws, const DevCtx& ctx,
                   cudaStream_t st) {
-  const BwdWorkspace L = bwd_workspace_layout(s);
+  const BwdWorkspace L = bwd_workspace_layout(s, false);
   char* w = static_cast<char*>(ws);
   float* Dv = reinterpret_cast<float*>(w + L.off_D);
   float* da = reinterpret_cast<float*>(w + L.off_da);
@@ -569,7 +627,7 @@ cudaError_t bwd_t(const AttnShape& s, const void* q, const void* k, const void* 
   int32_t* clist = reinterpret_cast<int32_t*>(w + L.off_csr_list);
   cudaError_t e;
   if (!s.dense) {
-    const size_t smem = 2 * sizeof(int32_t) * (size_t)s.N;
+    const size_t smem = sizeof(int32_t) * ((size_t)s.N + kCsrChunk);
     e = cudaFuncSetAttribute(csr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     csr_kernel<<<s.B * s.Hkv, kThreads, smem, st>>>(idx, s, coff, clist, ctx);
@@ -641,7 +699,7 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 cudaError_t launch_bwd_csr(const AttnShape& s, const int32_t* idx, int32_t* off, int32_t* list,
                            const DevCtx& ctx, cudaStream_t st) {
-  const size_t smem = 2 * sizeof(int32_t) * (size_t)s.N;
+  const size_t smem = sizeof(int32_t) * ((size_t)s.N + kCsrChunk);
   cudaError_t e =
       cudaFuncSetAttribute(csr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -651,17 +709,17 @@ cudaError_t launch_bwd_csr(const AttnShape& s, const int32_t* idx, int32_t* off,
 }
 
 cudaError_t launch_bwd_jacobian(const AttnShape& s, const float* da, const int32_t* idx,
-                                const float* gates, float* dscores, cudaStream_t st) {
+                                const float* gates, float* dscores, int RC, cudaStream_t st) {
   const long long srows = (long long)s.B * s.Hkv * s.N;
   jacobian_kernel<<<(unsigned)((srows + kWarps - 1) / kWarps), kThreads, 0, st>>>(
-      da, idx, gates, s, 1, dscores);
+      da, idx, gates, s, RC, dscores);
   note_launches(1);
   return cudaGetLastError();
 }
 
-BwdWorkspace bwd_workspace_layout(const AttnShape& s) {
+BwdWorkspace bwd_workspace_layout(const AttnShape& s, bool tc) {
   BwdWorkspace L;
-  const int RC = s.b < 64 ? 1 : s.b / 64;
+  const int RC = tc ? 4 : (s.b < 64 ? 1 : s.b / 64);
   size_t off = 0;
   L.off_D = off;
   off = align256(off + sizeof(float) * (size_t)s.B * s.Hq * s.T);
@@ -671,6 +729,15 @@ BwdWorkspace bwd_workspace_layout(const AttnShape& s) {
   off = align256(off + sizeof(int32_t) * (size_t)s.B * s.Hkv * (s.N + 1));
   L.off_csr_list = off;
   off = align256(off + sizeof(int32_t) * (size_t)s.B * s.Hkv * s.N * (s.dense ? 0 : s.K));
+  // Launch order of the key-outer dK/dV CTAs (most selected key blocks first).
+  L.off_order = off;
+  off = align256(off + sizeof(int32_t) * (size_t)s.B * s.Hkv * s.N);
+  // dS tiles of every (query block, 128-row tile, slot) for the dq kernel:
+  // [B][Hkv][N][G/2][K + 1][128][64] bf16 (slot K: the current block).
+  L.off_ds = off;
+  if (tc)
+    off = align256(off + sizeof(uint16_t) * (size_t)s.B * s.Hkv * s.N * (s.Hq / s.Hkv / 2) *
+                             (s.K + 1) * 128 * 64);
   L.total = off;
   return L;
 }

@@ -38,54 +38,41 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxList = 257;
 
 // ============================================================================
-// Kernel A: dq, D, da
+// Kernel D: D_i = sum over the attended keys of P_it dP_it (exact, r12 of the
+// design notes is the reading; the forward's bf16 o would round it)
 // ============================================================================
-// Q and dO of the tile are copied into TMEM once and used as the A operand of
-// every S / dP MMA, and dS goes back into TMEM as the A operand of the dQ MMA:
-// the MMAs then read only K / V from shared memory. Two groups of four
-// elementwise warps split each block's 64 keys (group g takes keys 32g ..).
-//
-// Every mbarrier wait costs the MMA-issuing thread far more than an MMA issue
-// slot, so it waits once per iteration: the full barrier of K/V stage `it`
-// also collects one arrival from each elementwise warp, given when that warp
-// is done with the S/dP buffer of iteration it - 2 (and, in sweep 2, has
-// written that iteration's dS). The MMA stream is S/dP(0), S/dP(1), ...,
-// with dQ(it - 2) issued right before S/dP(it) in sweep 2.
-namespace ka {
-constexpr int kStages = 6;                // K/V ring depth (stages 4, 5 reuse the Q/dO area)
-constexpr int kWarps = 12;
-constexpr int kThreadsA = kWarps * 32;
-constexpr uint32_t kOffQ = 0;             // [k half][128 rows][128 B]
-constexpr uint32_t kOffDO = 32768;        // same layout
-constexpr uint32_t kOffKV = 65536;        // stages 0..3; stage = (K halves, V halves) 32 KB
-// TMEM columns.
-constexpr uint32_t kColQ = 0, kColDO = 64, kColS = 128, kColDP = 256, kColDQ = 384;
+// One CTA per (query block j, 128-row tile of two heads, KV head, batch),
+// two CTAs per SM (256 TMEM columns, 97 KB of shared memory), so one CTA's
+// prologue and bubbles are filled by the other's MMAs. Q and dO pass through
+// one 32 KB staging buffer into TMEM (the A operand of every S / dP MMA);
+// K/V blocks stream through a two-stage ring. The S/dP accumulators are
+// single-buffered: the full barrier of K/V block n also takes one arrival
+// per elementwise warp once it has read S/dP(n-1), so the MMA thread waits
+// once per block.
+namespace kd {
+constexpr int kThreadsD = 256;   // warp 0 producer + list, warp 1 MMA, warps 4-7 rows
+constexpr uint32_t kTmemColsD = 256;
+constexpr uint32_t kColQ = 0, kColDO = 64, kColS = 128, kColDP = 192;
+constexpr uint32_t kOffStage = 0;       // Q, then dO: [k half][128 rows][128 B]
+constexpr uint32_t kOffKV = 32768;      // 2 stages x (K halves, V halves)
+constexpr uint32_t kOffCtl = kOffKV + 2 * 32768;
 struct Ctl {
-  // kv_full[st]: the producer's expect-tx arrival, the TMA bytes and one
-  // arrival per elementwise warp (9 arrivals per phase).
-  uint64_t qdo_full, kv_full[kStages], kv_empty[kStages], s_full[2], ds_tail[2], dq_done, drain;
+  uint64_t qd_full, qd_free, kv_full[2], kv_empty[2], s_full, drain;
   uint32_t tmem_base;
   int abort, nblk;
-  int blocks[kMaxList], slots[kMaxList];
+  int blocks[kMaxList];
   float bias[kMaxList];
-  float red[kMaxList][8];  // per-warp partial sums of dS per block
-  float dpart[2][128];     // per-group partial D per row
 };
-constexpr uint32_t kOffCtl = kOffKV + 4 * 32768;
 constexpr size_t kSmem = kOffCtl + sizeof(Ctl) + 1024;
-__device__ __forceinline__ uint32_t stage_off(int st) {
-  return st < 4 ? kOffKV + st * 32768u : kOffQ + (st - 4) * 32768u;
-}
-}  // namespace ka
+}  // namespace kd
 
 template <int TILES>
-__global__ void __launch_bounds__(ka::kThreadsA, 1)
-tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                 const float* __restrict__ lse, const int32_t* __restrict__ idx,
-                 const float* __restrict__ gates, AttnShape s, __nv_bfloat16* __restrict__ dq,
-                 float* __restrict__ Dv, float* __restrict__ da, DevCtx ctx) {
-  using namespace ka;
+__global__ void __launch_bounds__(kd::kThreadsD, 2)
+tc_bwd_d_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                const float* __restrict__ lse, const int32_t* __restrict__ idx,
+                const float* __restrict__ gates, AttnShape s, float* __restrict__ Dv, DevCtx ctx) {
+  using namespace kd;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   unsigned char* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -99,63 +86,51 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const long long irow = ((long long)(bi * s.Hkv + kvh) * s.N + j);
   volatile int* abort = &c.abort;
 
-  // Elementwise warps: tile row, its head and its lse, read before the CTA barrier.
-  const int quarter = warp & 3, grp = (warp - 4) >> 2;
+  const int quarter = warp & 3;
   const int rowi = quarter * 32 + lane;
-  const int hh = rowi >> 6, r = rowi & 63;
+  const int r = rowi & 63;
   const int qrow = j * kB + r;
   const bool live = qrow < s.T;
-  const long long hrow = (long long)(bi * s.Hq + h0 + hh) * s.T + qrow;
+  const long long hrow = (long long)(bi * s.Hq + h0 + (rowi >> 6)) * s.T + qrow;
   float lse2 = 0.f;
   if (warp >= 4 && live) lse2 = lse[hrow] * kLog2e;
 
   int issued = 0;
   if (warp == 0) {
     if (lane == 0) {
-      mbar_init(&c.qdo_full, 1);
-      for (int i = 0; i < kStages; ++i) {
-        mbar_init(&c.kv_full[i], 9);
+      mbar_init(&c.qd_full, 1);
+      mbar_init(&c.qd_free, 4);
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&c.kv_full[i], 5);  // expect-tx arrival + one per elementwise warp
         mbar_init(&c.kv_empty[i], 1);
       }
-      for (int i = 0; i < 2; ++i) {
-        mbar_init(&c.s_full[i], 1);
-        mbar_init(&c.ds_tail[i], 8);
-      }
-      mbar_init(&c.dq_done, 1);
+      mbar_init(&c.s_full, 1);
       mbar_init(&c.drain, 1);
       fence_mbar_init();
       c.abort = 0;
-      // Q and dO do not depend on the selection: start their loads first.
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_do);
-      mbar_arrive_expect_tx(&c.qdo_full, 2 * 4 * 8192);
+      mbar_arrive_expect_tx(&c.qd_full, 4 * 8192);
       for (int h2 = 0; h2 < 2; ++h2)
-        for (int kb = 0; kb < 2; ++kb) {
-          tma_load_3d(base + kOffQ + kb * 16384 + h2 * 8192, &tm_q, kb * 64, j * kB,
-                      bi * s.Hq + h0 + h2, &c.qdo_full);
-          tma_load_3d(base + kOffDO + kb * 16384 + h2 * 8192, &tm_do, kb * 64, j * kB,
-                      bi * s.Hq + h0 + h2, &c.qdo_full);
-        }
+        for (int kb = 0; kb < 2; ++kb)
+          tma_load_3d(base + kOffStage + kb * 16384 + h2 * 8192, &tm_q, kb * 64, j * kB,
+                      bi * s.Hq + h0 + h2, &c.qd_full);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
     }
-    // Attended blocks: the selected history blocks in slot order, then block j.
     __syncwarp();
     const int n = warp_build_list(idx + irow * s.K, gates ? gates + irow * s.N : nullptr, s.K, j,
-                                  0, c.blocks, c.slots, c.bias, ctx);
+                                  0, c.blocks, nullptr, c.bias, ctx);
     if (lane == 0) {
       c.blocks[n] = j;
-      c.slots[n] = -1;
       c.bias[n] = 0.f;
       c.nblk = n + 1;
     }
     __syncwarp();
-    // Stages 0..3 are free: start their loads before the CTA barrier.
     if (lane == 0) {
-      const int nit0 = 2 * (n + 1);  // sweep 1 then sweep 2 over the same blocks
-      for (; issued < nit0 && issued < 4; ++issued) {
-        const int m = c.blocks[issued % (n + 1)];
-        unsigned char* kv = base + stage_off(issued);
+      for (; issued < n + 1 && issued < 2; ++issued) {
+        const int m = c.blocks[issued];
+        unsigned char* kv = base + kOffKV + issued * 32768;
         mbar_arrive_expect_tx(&c.kv_full[issued], 32768);
         for (int h2 = 0; h2 < 2; ++h2) {
           tma_load_3d(kv + h2 * 8192, &tm_k, h2 * 64, m * kB, bi * s.Hkv + kvh, &c.kv_full[issued]);
@@ -166,7 +141,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
   }
   if (warp == 1) {
-    tmem_alloc(&c.tmem_base, kTmemCols);
+    tmem_alloc(&c.tmem_base, kTmemColsD);
     tmem_relinquish();
   }
   fence_before_sync();
@@ -174,86 +149,63 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   fence_after_sync();
   const uint32_t tmem = c.tmem_base;
   const int nblk = c.nblk;
-  const int nit = 2 * nblk;
-  const int tail_first = max(nblk, nit - 2);  // sweep-2 iterations whose dQ follows the loop
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int it = issued; it < nit; ++it) {
-        const int st = it % kStages;
-        bool go = true;
-        // Stages 4 and 5 reuse the Q/dO area: free once every elementwise
-        // warp has moved its rows into TMEM (their first kv_full arrivals).
-        if (it == 4) go = wait_or_abort(ctx, &c.kv_full[0], 0, abort);
-        if (go && it >= kStages)
-          go = wait_or_abort(ctx, &c.kv_empty[st], ((it - kStages) / kStages) & 1, abort);
-        if (!go) break;
-        const int m = c.blocks[it % nblk];
-        unsigned char* kv = base + stage_off(st);
+      // dO follows Q through the staging buffer once Q has moved into TMEM.
+      bool go = wait_or_abort(ctx, &c.qd_free, 0, abort);
+      if (go) {
+        mbar_arrive_expect_tx(&c.qd_full, 4 * 8192);
+        for (int h2 = 0; h2 < 2; ++h2)
+          for (int kb = 0; kb < 2; ++kb)
+            tma_load_3d(base + kOffStage + kb * 16384 + h2 * 8192, &tm_do, kb * 64, j * kB,
+                        bi * s.Hq + h0 + h2, &c.qd_full);
+      }
+      for (int n = issued; go && n < nblk; ++n) {
+        const int st = n & 1;
+        if (!wait_or_abort(ctx, &c.kv_empty[st], ((n - 2) >> 1) & 1, abort)) break;
+        const int m = c.blocks[n];
+        unsigned char* kv = base + kOffKV + st * 32768;
         mbar_arrive_expect_tx(&c.kv_full[st], 32768);
         for (int h2 = 0; h2 < 2; ++h2) {
           tma_load_3d(kv + h2 * 8192, &tm_k, h2 * 64, m * kB, bi * s.Hkv + kvh, &c.kv_full[st]);
           tma_load_3d(kv + 16384 + h2 * 8192, &tm_v, h2 * 64, m * kB, bi * s.Hkv + kvh,
                       &c.kv_full[st]);
         }
-        issued = it + 1;
+        issued = n + 1;
       }
-      if (*abort) {
-        (void)mbar_wait(ctx, &c.qdo_full, 0);
-        for (int it = max(0, issued - kStages); it < issued; ++it)
-          (void)mbar_wait(ctx, &c.kv_full[it % kStages], (it / kStages) & 1);
-      }
+      // The staging copies land before the CTA leaves (the dO phase, when
+      // issued, completes after the Q phase).
+      (void)mbar_wait(ctx, &c.qd_full, go ? 1 : 0);
+      if (*abort)
+        for (int n = max(0, issued - 2); n < issued; ++n)
+          (void)mbar_wait(ctx, &c.kv_full[n & 1], (n >> 1) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16(128, 64, false, false);
-      const uint32_t id_q = idesc_bf16(128, 128, false, true);
-      // K-major K / V tiles: k-step ks at half (ks >> 2), byte (ks & 3) * 32.
-      const uint64_t dkv0 = sdesc_sw128(sbase, 16, 1024);
-      // K as the MN-major B operand of dQ: 16 keys per k-step (2048 B).
-      const uint64_t dkq0 = sdesc_sw128(sbase, 8192, 1024);
-      // dQ += dS K for sweep-2 iteration x; dS of keys 0..31 sits in S[x & 1]
-      // columns 0..15, keys 32..63 in columns 32..47.
-      auto issue_dq = [&](int x) {
-        const uint64_t kd = dkq0 + (stage_off(x % kStages) >> 4);
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_bf16_ts(tmem + kColDQ, tmem + kColS + (x & 1) * 64 + (ks >> 1) * 32 + (ks & 1) * 8,
-                      kd + ((ks * 2048) >> 4), id_q, (x > nblk || ks > 0));
-      };
+      const uint64_t dkv0 = sdesc_sw128(sbase + kOffKV, 16, 1024);
       bool ok = true;
-      for (int it = 0; it < nit; ++it) {
-        const int st = it % kStages, b = it & 1;
-        if (!wait_or_abort(ctx, &c.kv_full[st], (it / kStages) & 1, abort)) {
+      for (int n = 0; n < nblk; ++n) {
+        const int st = n & 1;
+        if (!wait_or_abort(ctx, &c.kv_full[st], (n >> 1) & 1, abort)) {
           ok = false;
           break;
         }
         fence_after_sync();
-        if (it >= nblk + 2) {
-          issue_dq(it - 2);
-          mma_commit(&c.kv_empty[(it - 2) % kStages]);
-        }
-        const uint64_t kd = dkv0 + (stage_off(st) >> 4);
+        const uint64_t kd = dkv0 + ((st * 32768) >> 4);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          mma_bf16_ts(tmem + kColS + b * 64, tmem + kColQ + ks * 8,
+          mma_bf16_ts(tmem + kColS, tmem + kColQ + ks * 8,
                       kd + (((ks >> 2) * 8192 + (ks & 3) * 32) >> 4), id_s, ks > 0);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          mma_bf16_ts(tmem + kColDP + b * 64, tmem + kColDO + ks * 8,
+          mma_bf16_ts(tmem + kColDP, tmem + kColDO + ks * 8,
                       kd + ((16384 + (ks >> 2) * 8192 + (ks & 3) * 32) >> 4), id_s, ks > 0);
-        mma_commit(&c.s_full[b]);
-        if (it < nblk) mma_commit(&c.kv_empty[st]);  // sweep 1 only reads S and dP
+        mma_commit(&c.s_full);
+        mma_commit(&c.kv_empty[st]);
       }
-      for (int x = tail_first; ok && x < nit; ++x) {
-        if (!wait_or_abort(ctx, &c.ds_tail[x - tail_first], 0, abort)) {
-          ok = false;
-          break;
-        }
-        fence_after_sync();
-        issue_dq(x);
-      }
-      mma_commit(&c.dq_done);
+      (void)ok;
       if (*abort) {
         mma_commit(&c.drain);
         (void)mbar_wait(ctx, &c.drain, 0);
@@ -262,49 +214,47 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   } else if (warp >= 4) {
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
     const float sc = s.scale * kLog2e;
-    // Arrival on the full barrier of iteration x (when there is one).
-    auto arrive_w = [&](int x) {
-      if (lane == 0 && x < nit) mbar_arrive(&c.kv_full[x % kStages]);
-    };
-    bool ok = warp_wait(ctx, &c.qdo_full, 0, abort);
+    const uint64_t sc2 = f2u(sc, sc);
+    // Q, then dO, from the staging buffer into this row's TMEM lane.
+    bool ok = warp_wait(ctx, &c.qd_full, 0, abort);
     if (ok) {
-      // Group 0 moves the Q rows into TMEM, group 1 the dO rows.
-      tile_row_to_tmem(base + (grp == 0 ? kOffQ : kOffDO), rowi,
-                       tl + (grp == 0 ? kColQ : kColDO));
+      tile_row_to_tmem(base + kOffStage, rowi, tl + kColQ);
       tmem_st_wait();
     }
     fence_before_sync();
     __syncwarp();
-    arrive_w(0);
-    arrive_w(1);
+    if (lane == 0) mbar_arrive(&c.qd_free);
+    ok = ok && warp_wait(ctx, &c.qd_full, 1, abort);
+    if (ok) {
+      tile_row_to_tmem(base + kOffStage, rowi, tl + kColDO);
+      tmem_st_wait();
+    }
+    fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&c.kv_full[0]);  // Q, dO in TMEM: S/dP(0) may start
     float Dsum = 0.f;
-    const uint64_t sc2 = f2u(sc, sc);
-    // Sweep 1: D = sum over the attended keys of P * dP.
-    for (int it = 0; ok && it < nblk; ++it) {
-      const int b = it & 1;
-      if (!warp_wait(ctx, &c.s_full[b], (it >> 1) & 1, abort)) {
+    for (int n = 0; ok && n < nblk; ++n) {
+      if (!warp_wait(ctx, &c.s_full, n & 1, abort)) {
         ok = false;
         break;
       }
       fence_after_sync();
-      const int m = c.blocks[it];
-      const float bias = c.bias[it];
-      const bool cur = (it == nblk - 1);
-      const int kvalid = min(kB, s.T - m * kB) - 32 * grp;
-      uint32_t sr[32], pr[32];
-      tmem_ld32(tl + kColS + b * 64 + 32 * grp, sr);
-      tmem_ld32(tl + kColDP + b * 64 + 32 * grp, pr);
-      tmem_ld_wait();
-      fence_before_sync();
-      __syncwarp();
-      arrive_w(it + 2);
-      if (cur || kvalid < 32) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (i >= kvalid || (cur && i + 32 * grp > r)) sr[i] = __float_as_uint(-INFINITY);
-      }
+      const int m = c.blocks[n];
+      const float bias = c.bias[n];
+      const bool cur = (n == nblk - 1);
+      const int kvalid = min(kB, s.T - m * kB);
       const float off = live ? bias - lse2 : -INFINITY;
       const uint64_t off2 = f2u(off, off);
+      uint32_t sr[64], pr[32];
+      tmem_ld32(tl + kColS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tl + kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(tl + kColDP, pr);
+      tmem_ld_wait();
+      if (cur || kvalid < kB) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (i >= kvalid || (cur && i > r)) sr[i] = __float_as_uint(-INFINITY);
+      }
       uint64_t acc0 = 0, acc1 = 0;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
@@ -315,97 +265,176 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (i & 1) acc1 = ffma2(p2, dp2, acc1);
         else acc0 = ffma2(p2, dp2, acc0);
       }
-      const uint64_t accs = fadd2(acc0, acc1);
-      Dsum += lo_f(accs) + hi_f(accs);
-    }
-    // The two groups' halves of D meet here; every elementwise warp arrives
-    // exactly once, whichever path it took.
-    c.dpart[grp][rowi] = Dsum;
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    Dsum = c.dpart[0][rowi] + c.dpart[1][rowi];
-    ok = ok && !*abort;
-    const uint64_t negD = f2u(-Dsum, -Dsum);
-    // Sweep 2: dS = P * (dP - D) back into TMEM for the dQ MMA, and its tile sums.
-    for (int it = nblk; ok && it < nit; ++it) {
-      const int b = it & 1, n = it - nblk;
-      if (!warp_wait(ctx, &c.s_full[b], (it >> 1) & 1, abort)) {
-        ok = false;
-        break;
-      }
-      fence_after_sync();
-      const int m = c.blocks[n];
-      const float bias = c.bias[n];
-      const bool cur = (n == nblk - 1);
-      const int kvalid = min(kB, s.T - m * kB) - 32 * grp;
-      uint32_t sr[32], pr[32];
-      tmem_ld32(tl + kColS + b * 64 + 32 * grp, sr);
-      tmem_ld32(tl + kColDP + b * 64 + 32 * grp, pr);
+      tmem_ld32(tl + kColDP + 32, pr);
       tmem_ld_wait();
-      if (cur || kvalid < 32) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (i >= kvalid || (cur && i + 32 * grp > r)) sr[i] = __float_as_uint(-INFINITY);
-      }
-      const float off = live ? bias - lse2 : -INFINITY;
-      const uint64_t off2 = f2u(off, off);
-      uint32_t pk[16];
-      uint64_t acc0 = 0, acc1 = 0;
+      // S/dP(n) are in registers: S/dP(n + 1) may overwrite the accumulators.
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0 && n + 1 < nblk) mbar_arrive(&c.kv_full[(n + 1) & 1]);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const uint64_t a2 = ffma2(f2u(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
+        const uint64_t a2 = ffma2(f2u(__uint_as_float(sr[32 + 2 * i]), __uint_as_float(sr[32 + 2 * i + 1])),
                                   sc2, off2);
         const uint64_t p2 = f2u(ex2(lo_f(a2)), ex2(hi_f(a2)));
         const uint64_t dp2 = f2u(__uint_as_float(pr[2 * i]), __uint_as_float(pr[2 * i + 1]));
-        const uint64_t ds2 = fmul2(p2, fadd2(dp2, negD));
-        if (i & 1) acc1 = fadd2(acc1, ds2);
-        else acc0 = fadd2(acc0, ds2);
-        pk[i] = pack_bf16(lo_f(ds2), hi_f(ds2));
+        if (i & 1) acc1 = ffma2(p2, dp2, acc1);
+        else acc0 = ffma2(p2, dp2, acc0);
       }
-      tmem_st16(tl + kColS + b * 64 + 32 * grp, pk);
-      tmem_st_wait();
-      fence_before_sync();
-      __syncwarp();
-      if (it + 2 < nit) arrive_w(it + 2);
-      else if (lane == 0) mbar_arrive(&c.ds_tail[it - tail_first]);
-      if (!cur) {
-        const uint64_t accs = fadd2(acc0, acc1);
-        const float t = warp_sum(lo_f(accs) + hi_f(accs));
-        if (lane == 0) c.red[n][grp * 4 + quarter] = t;
+      const uint64_t accs = fadd2(acc0, acc1);
+      Dsum += lo_f(accs) + hi_f(accs);
+    }
+    if (ok && live) Dv[hrow] = Dsum;
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after_sync();
+    tmem_dealloc(tmem, kTmemColsD);
+  }
+}
+
+// ============================================================================
+// Kernel Q: dq = scale * sum over the attended blocks of dS K, from the dS
+// tiles the dK/dV kernel stored (no recomputation of S / dP)
+// ============================================================================
+// One CTA per (query block j, 128-row tile, KV head, batch), two CTAs per
+// SM: each attended block brings its 16 KB dS tile and 16 KB K block through
+// a three-stage TMA ring; dQ (128 x 128 fp32) accumulates in TMEM with four
+// M=128 N=128 MMAs per block, in the block list's order.
+namespace kq {
+constexpr int kThreadsQ = 256;   // warp 0 producer + list, warp 1 MMA, warps 4-7 epilogue
+constexpr uint32_t kTmemColsQ = 128;
+constexpr int kStages = 3;
+constexpr uint32_t kOffCtl = kStages * 32768;  // stage: dS tile 16 KB, then K halves
+struct Ctl {
+  uint64_t kv_full[kStages], kv_empty[kStages], dq_done, drain;
+  uint32_t tmem_base;
+  int abort, nblk;
+  int blocks[kMaxList], slots[kMaxList];
+  float bias[kMaxList];
+};
+constexpr size_t kSmem = kOffCtl + sizeof(Ctl) + 1024;
+}  // namespace kq
+
+template <int TILES>
+__global__ void __launch_bounds__(kq::kThreadsQ, 2)
+tc_bwd_dq_kernel(const __nv_bfloat16* __restrict__ ds, const __grid_constant__ CUtensorMap tm_k,
+                 const int32_t* __restrict__ idx, AttnShape s, __nv_bfloat16* __restrict__ dq,
+                 DevCtx ctx) {
+  using namespace kq;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  unsigned char* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const uint32_t sbase = smem_u32(base);
+  Ctl& c = *reinterpret_cast<Ctl*>(base + kOffCtl);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int j = blockIdx.x, kvh = blockIdx.y / TILES, u = blockIdx.y % TILES, bi = blockIdx.z;
+  const int G = 2 * TILES;
+  const int h0 = kvh * G + 2 * u;
+  const long long irow = ((long long)(bi * s.Hkv + kvh) * s.N + j);
+  // dS tiles of this (query block, tile): plane index of slot sl.
+  const long long plane0 = (irow * TILES + u) * (s.K + 1);
+  volatile int* abort = &c.abort;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int i = 0; i < kStages; ++i) {
+        mbar_init(&c.kv_full[i], 1);
+        mbar_init(&c.kv_empty[i], 1);
+      }
+      mbar_init(&c.dq_done, 1);
+      mbar_init(&c.drain, 1);
+      fence_mbar_init();
+      c.abort = 0;
+      tma_prefetch_desc(&tm_k);
+    }
+    __syncwarp();
+    const int n = warp_build_list(idx + irow * s.K, nullptr, s.K, j, 0, c.blocks, c.slots, c.bias,
+                                  ctx);
+    if (lane == 0) {
+      c.blocks[n] = j;
+      c.slots[n] = s.K;  // the current block's tile sits after the K slots
+      c.nblk = n + 1;
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(&c.tmem_base, kTmemColsQ);
+    tmem_relinquish();
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = c.tmem_base;
+  const int nblk = c.nblk;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int n = 0; n < nblk; ++n) {
+        const int st = n % kStages;
+        if (n >= kStages &&
+            !wait_or_abort(ctx, &c.kv_empty[st], ((n - kStages) / kStages) & 1, abort))
+          break;
+        unsigned char* sb = base + st * 32768;
+        mbar_arrive_expect_tx(&c.kv_full[st], 32768);
+        bulk_g2s(sb, ds + (plane0 + c.slots[n]) * (128 * 64), 16384, &c.kv_full[st]);
+        for (int h2 = 0; h2 < 2; ++h2)
+          tma_load_3d(sb + 16384 + h2 * 8192, &tm_k, h2 * 64, c.blocks[n] * kB, bi * s.Hkv + kvh,
+                      &c.kv_full[st]);
+        issued = n + 1;
+      }
+      if (*abort)
+        for (int n = max(0, issued - kStages); n < issued; ++n)
+          (void)mbar_wait(ctx, &c.kv_full[n % kStages], (n / kStages) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id_q = idesc_bf16(128, 128, false, true);
+      const uint64_t dds0 = sdesc_sw128(sbase, 16, 1024);            // dS, K-major
+      const uint64_t dk0 = sdesc_sw128(sbase + 16384, 8192, 1024);   // K as MN-major B
+      for (int n = 0; n < nblk; ++n) {
+        const int st = n % kStages;
+        if (!wait_or_abort(ctx, &c.kv_full[st], (n / kStages) & 1, abort)) break;
+        fence_after_sync();
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_bf16_ss(tmem, dds0 + ((st * 32768 + ks * 32) >> 4),
+                      dk0 + ((st * 32768 + ks * 2048) >> 4), id_q, (n > 0 || ks > 0));
+        mma_commit(&c.kv_empty[st]);
+      }
+      mma_commit(&c.dq_done);
+      if (*abort) {
+        mma_commit(&c.drain);
+        (void)mbar_wait(ctx, &c.drain, 0);
       }
     }
-    if (ok) {
-      if (warp_wait(ctx, &c.dq_done, 0, abort)) {
-        fence_after_sync();
-        __nv_bfloat16* drow = dq + hrow * kD + grp * 64;
+  } else if (warp >= 4) {
+    const int quarter = warp & 3;
+    const int rowi = quarter * 32 + lane;
+    const int r = rowi & 63;
+    const int qrow = j * kB + r;
+    const long long hrow = (long long)(bi * s.Hq + h0 + (rowi >> 6)) * s.T + qrow;
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    if (warp_wait(ctx, &c.dq_done, 0, abort)) {
+      fence_after_sync();
+      __nv_bfloat16* drow = dq + hrow * kD;
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          uint32_t ov[32];
-          tmem_ld32(tl + kColDQ + grp * 64 + ch * 32, ov);
-          tmem_ld_wait();
-          if (live) {
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t ov[32];
+        tmem_ld32(tl + ch * 32, ov);
+        tmem_ld_wait();
+        if (qrow < s.T) {
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              uint4 v;
-              v.x = pack_bf16(__uint_as_float(ov[8 * q4 + 0]) * s.scale, __uint_as_float(ov[8 * q4 + 1]) * s.scale);
-              v.y = pack_bf16(__uint_as_float(ov[8 * q4 + 2]) * s.scale, __uint_as_float(ov[8 * q4 + 3]) * s.scale);
-              v.z = pack_bf16(__uint_as_float(ov[8 * q4 + 4]) * s.scale, __uint_as_float(ov[8 * q4 + 5]) * s.scale);
-              v.w = pack_bf16(__uint_as_float(ov[8 * q4 + 6]) * s.scale, __uint_as_float(ov[8 * q4 + 7]) * s.scale);
-              *reinterpret_cast<uint4*>(drow + ch * 32 + q4 * 8) = v;
-            }
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 v;
+            v.x = pack_bf16(__uint_as_float(ov[8 * q4 + 0]) * s.scale, __uint_as_float(ov[8 * q4 + 1]) * s.scale);
+            v.y = pack_bf16(__uint_as_float(ov[8 * q4 + 2]) * s.scale, __uint_as_float(ov[8 * q4 + 3]) * s.scale);
+            v.z = pack_bf16(__uint_as_float(ov[8 * q4 + 4]) * s.scale, __uint_as_float(ov[8 * q4 + 5]) * s.scale);
+            v.w = pack_bf16(__uint_as_float(ov[8 * q4 + 6]) * s.scale, __uint_as_float(ov[8 * q4 + 7]) * s.scale);
+            *reinterpret_cast<uint4*>(drow + ch * 32 + q4 * 8) = v;
           }
         }
-        if (live && grp == 0) Dv[hrow] = Dsum;
-      }
-    }
-    // da of each selected block: the eight warps' partials in a fixed order.
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    if (da != nullptr && !*abort) {
-      for (int n = tid - 128; n < nblk - 1; n += 256) {
-        const float* p = c.red[n];
-        const float t = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
-        const long long o0 = (((long long)(bi * s.Hq + h0)) * s.N + j) * s.K + c.slots[n];
-        da[o0] = t;
-        da[o0 + (long long)s.N * s.K] = 0.f;  // head h0 + 1: the tile's sum sits on h0
       }
     }
   }
@@ -413,7 +442,43 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   __syncthreads();
   if (warp == 1) {
     fence_after_sync();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, kTmemColsQ);
+  }
+}
+
+// ============================================================================
+// Launch order of kernel B: the (batch, KV head, key block) units sorted by
+// descending reverse-list length, so the longest CTAs start first and the
+// short ones fill in behind them. Any order gives the same results (every
+// unit's outputs come from one CTA); ties are left in whatever order the
+// atomics produce.
+// ============================================================================
+__global__ void __launch_bounds__(1024)
+order_kernel(const int32_t* __restrict__ off_all, AttnShape s, int32_t* __restrict__ order) {
+  extern __shared__ int32_t hist[];  // N + 1 buckets (list length 0..N-1)
+  const int U = s.B * s.Hkv * s.N;
+  const int nb = s.N + 1;
+  for (int i = threadIdx.x; i < nb; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  for (int u = threadIdx.x; u < U; u += blockDim.x) {
+    const int bh = u / s.N, m = u % s.N;
+    const int len = off_all[(long long)bh * (s.N + 1) + m + 1] - off_all[(long long)bh * (s.N + 1) + m];
+    atomicAdd(&hist[s.N - len], 1);  // bucket 0 holds the longest lists
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int i = 0; i < nb; ++i) {
+      const int c = hist[i];
+      hist[i] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  for (int u = threadIdx.x; u < U; u += blockDim.x) {
+    const int bh = u / s.N, m = u % s.N;
+    const int len = off_all[(long long)bh * (s.N + 1) + m + 1] - off_all[(long long)bh * (s.N + 1) + m];
+    order[atomicAdd(&hist[s.N - len], 1)] = u;
   }
 }
 
@@ -448,9 +513,10 @@ struct Ctl {
   int abort;
   // Per stage, staged by the producer warp with the Q/dO tiles: the step's
   // query block, its log2-domain gate bias, and lse / D of the tile's rows.
-  int step_j[2];
+  int step_j[2], step_slot[2];
   float step_bias[2];
   float lse2[2][128], D[2][128];
+  float dapart[2][8];  // per-warp shares of the step's tile sum of dS
 };
 constexpr size_t kSmem = kOffCtl + sizeof(Ctl) + 1024;
 }  // namespace kb_
@@ -463,8 +529,9 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ lse,
                    const float* __restrict__ Dv, const float* __restrict__ gates,
                    const int32_t* __restrict__ csr_off, const int32_t* __restrict__ csr_list,
-                   AttnShape s, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
-                   DevCtx ctx) {
+                   const int32_t* __restrict__ order, AttnShape s,
+                   __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
+                   __nv_bfloat16* __restrict__ ds_out, float* __restrict__ da, DevCtx ctx) {
   using namespace kb_;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -473,9 +540,9 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
   Ctl& c = *reinterpret_cast<Ctl*>(base + kOffCtl);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int m = blockIdx.x, kvh = blockIdx.y, bi = blockIdx.z;
+  const int unit = order[blockIdx.x];
+  const int m = unit % s.N, bh = unit / s.N, kvh = bh % s.Hkv, bi = bh / s.Hkv;
   const int G = 2 * TILES;
-  const int bh = bi * s.Hkv + kvh;
   const int lo = csr_off[(long long)bh * (s.N + 1) + m];
   const int nl = csr_off[(long long)bh * (s.N + 1) + m + 1] - lo;
   const int32_t* lst = csr_list + (long long)bh * s.N * s.K + lo;
@@ -490,7 +557,7 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int i = 0; i < 2; ++i) {
       mbar_init(&c.qdo_full[i], 10);
       mbar_init(&c.s_full[i], 1);
-      mbar_init(&c.dvdk_done[i], 1);
+      mbar_init(&c.dvdk_done[i], 2);  // the MMA commit + the dS store warp
     }
     mbar_init(&c.pds_tail, 8);
     mbar_init(&c.acc_done, 1);
@@ -521,7 +588,7 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
     // four per lane, the query block and its gate bias) are loaded into
     // registers one step ahead, so staging them costs only shared stores.
     float pre_lse[4], pre_D[4], pre_bias = 0.f;
-    int pre_j = m;
+    int pre_j = m, pre_slot = s.K;
     // The reverse list in a register window (lane l holds entry win_lo + l),
     // with the next window already in flight.
     int win_lo = 0;
@@ -529,7 +596,7 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
     int win_next = 32 + lane < nl ? lst[32 + lane] : 0;
     auto prefetch = [&](int st_i) {
       const int jj = st_i / TILES, u = st_i % TILES;
-      int j = m;
+      int j = m, slot = s.K;  // the diagonal step's tile sits after the K slots
       if (jj > 0) {
         const int ix = jj - 1;
         while (ix >= win_lo + 32) {
@@ -537,9 +604,12 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
           win_lo += 32;
           win_next = win_lo + 32 + lane < nl ? lst[win_lo + 32 + lane] : 0;
         }
-        j = __shfl_sync(0xffffffffu, win, ix - win_lo) / s.K;
+        const int e = __shfl_sync(0xffffffffu, win, ix - win_lo);
+        j = e / s.K;
+        slot = e % s.K;
       }
       pre_j = j;
+      pre_slot = slot;
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         const int rr = lane + 32 * q4;
@@ -580,6 +650,7 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       if (lane == 0) {
         c.step_j[stg] = j;
+        c.step_slot[stg] = pre_slot;
         c.step_bias[stg] = logf(pre_bias) * kLog2e;
       }
       __threadfence_block();
@@ -659,6 +730,36 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
         (void)mbar_wait(ctx, &c.drain, 0);
       }
     }
+  } else if (warp == 2) {
+    // dS store warp: once P/dS of step s are in shared memory (the next
+    // stage's full barrier, or the tail barrier), copy the raw 16 KB dS tile
+    // (swizzled, as the dq kernel's MMA reads it) to the workspace with the
+    // TMA engine and write the step's da shares; its arrival on dvdk_done
+    // (with the MMA's commit) frees the P/dS buffer and the stage's scalars.
+    if (lane == 0) {
+      for (int st_i = 0; st_i < nsteps; ++st_i) {
+        const bool last = st_i + 1 == nsteps;
+        const bool ok2 = last ? wait_or_abort(ctx, &c.pds_tail, 0, abort)
+                              : wait_or_abort(ctx, &c.qdo_full[(st_i + 1) & 1],
+                                              ((st_i + 1) >> 1) & 1, abort);
+        if (!ok2) break;
+        const int stg = st_i & 1, u = st_i % TILES;
+        const int j = c.step_j[stg], slot = c.step_slot[stg];
+        const long long tile = (((long long)bh * s.N + j) * TILES + u) * (s.K + 1) + slot;
+        bulk_s2g(ds_out + tile * (128 * 64), base + kOffDS, 16384);
+        bulk_commit();
+        if (da != nullptr && slot < s.K) {
+#pragma unroll
+          for (int p = 0; p < 8; ++p) {
+            const int head = kvh * G + 2 * u + ((p & 3) >> 1), rc = (p >> 2) * 2 + (p & 1);
+            da[(((long long)(bi * s.Hq + head) * s.N + j) * 4 + rc) * s.K + slot] = c.dapart[stg][p];
+          }
+        }
+        bulk_wait_read_all();
+        if (!last) mbar_arrive(&c.dvdk_done[stg]);
+      }
+      bulk_wait_all();
+    }
   } else if (warp >= 4) {
     const int quarter = warp & 3, grp = (warp - 4) >> 2;
     const int rowi = quarter * 32 + lane;  // tile row (query) / d index in the epilogue
@@ -696,6 +797,7 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       const float off = live ? bias - lse2 : -INFINITY;
       const uint64_t off2 = f2u(off, off), negD = f2u(-Di, -Di);
+      uint64_t dsum = 0;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const uint64_t a2 = ffma2(f2u(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
@@ -703,13 +805,19 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
         const float p0 = ex2(lo_f(a2)), p1 = ex2(hi_f(a2));
         const uint64_t dp2 = f2u(__uint_as_float(pr[2 * i]), __uint_as_float(pr[2 * i + 1]));
         const uint64_t ds2 = fmul2(f2u(p0, p1), fadd2(dp2, negD));
+        dsum = fadd2(dsum, ds2);
         pp[i] = pack_bf16(p0, p1);
         dd[i] = pack_bf16(lo_f(ds2), hi_f(ds2));
       }
+
       // The P / dS buffers are free once dV/dK of step st_i - 1 completed.
       if (st_i >= 1 && !warp_wait(ctx, &c.dvdk_done[(st_i - 1) & 1], ((st_i - 1) >> 1) & 1, abort)) {
         ok = false;
         break;
+      }
+      {  // this warp's share of the tile sum of dS, for the store warp
+        const float t = warp_sum(lo_f(dsum) + hi_f(dsum));
+        if (lane == 0) c.dapart[stg][grp * 4 + quarter] = t;
       }
       unsigned char* prow = base + kOffP + rowi * 128;
       unsigned char* drow = base + kOffDS + rowi * 128;
@@ -769,12 +877,16 @@ cudaError_t launch_attn_bwd_tc(const AttnShape& s, const void* q, const void* k,
                                const float* lse, const void* dO, const int32_t* idx,
                                const float* gates, void* dq, void* dk, void* dv, float* dscores,
                                void* ws, const DevCtx& ctx, cudaStream_t st) {
-  const BwdWorkspace L = bwd_workspace_layout(s);
+  const BwdWorkspace L = bwd_workspace_layout(s, true);
   char* w = static_cast<char*>(ws);
   float* Dv = reinterpret_cast<float*>(w + L.off_D);
   float* da = reinterpret_cast<float*>(w + L.off_da);
   int32_t* coff = reinterpret_cast<int32_t*>(w + L.off_csr_off);
   int32_t* clist = reinterpret_cast<int32_t*>(w + L.off_csr_list);
+  int32_t* order = reinterpret_cast<int32_t*>(w + L.off_order);
+  __nv_bfloat16* dsbuf = reinterpret_cast<__nv_bfloat16*>(w + L.off_ds);
+  const int G = s.Hq / s.Hkv;
+  const int tiles = G / 2;
   CUtensorMap tq, tk, tv, tdo;
   cudaError_t e;
   if ((e = make_tmap_bf16(&tq, q, s.T, s.B * s.Hq)) != cudaSuccess) return e;
@@ -782,29 +894,45 @@ cudaError_t launch_attn_bwd_tc(const AttnShape& s, const void* q, const void* k,
   if ((e = make_tmap_bf16(&tk, k, s.T, s.B * s.Hkv)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16(&tv, v, s.T, s.B * s.Hkv)) != cudaSuccess) return e;
   if ((e = launch_bwd_csr(s, idx, coff, clist, ctx, st)) != cudaSuccess) return e;
-  const int G = s.Hq / s.Hkv;
-  const int tiles = G / 2;
   {
-    dim3 grid(s.N, s.Hkv * tiles, s.B);
-    auto kern = tiles == 2 ? tc_bwd_dq_kernel<2> : tc_bwd_dq_kernel<1>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ka::kSmem);
+    const size_t smem = sizeof(int32_t) * ((size_t)s.N + 1);
+    e = cudaFuncSetAttribute(order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, ka::kThreadsA, ka::kSmem, st>>>(tq, tk, tv, tdo, lse, idx, gates, s,
-                                            (__nv_bfloat16*)dq, Dv, dscores ? da : nullptr, ctx);
+    order_kernel<<<1, 1024, smem, st>>>(coff, s, order);
     note_launches(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  {
-    dim3 grid(s.N, s.Hkv, s.B);
+  {  // D
+    dim3 grid(s.N, s.Hkv * tiles, s.B);
+    auto kern = tiles == 2 ? tc_bwd_d_kernel<2> : tc_bwd_d_kernel<1>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kd::kSmem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kd::kThreadsD, kd::kSmem, st>>>(tq, tk, tv, tdo, lse, idx, gates, s, Dv, ctx);
+    note_launches(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  {  // dK, dV, dS tiles, da
+    dim3 grid(s.N * s.Hkv * s.B);
     auto kern = tiles == 2 ? tc_bwd_dkdv_kernel<2> : tc_bwd_dkdv_kernel<1>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kb_::kSmem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kb_::kThreadsB, kb_::kSmem, st>>>(tq, tk, tv, tdo, lse, Dv, gates, coff, clist, s,
-                                             (__nv_bfloat16*)dk, (__nv_bfloat16*)dv, ctx);
+    kern<<<grid, kb_::kThreadsB, kb_::kSmem, st>>>(tq, tk, tv, tdo, lse, Dv, gates, coff, clist,
+                                                   order, s, (__nv_bfloat16*)dk,
+                                                   (__nv_bfloat16*)dv, dsbuf,
+                                                   dscores ? da : nullptr, ctx);
     note_launches(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  if (dscores) return launch_bwd_jacobian(s, da, idx, gates, dscores, st);
+  {  // dq
+    dim3 grid(s.N, s.Hkv * tiles, s.B);
+    auto kern = tiles == 2 ? tc_bwd_dq_kernel<2> : tc_bwd_dq_kernel<1>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kq::kSmem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kq::kThreadsQ, kq::kSmem, st>>>(dsbuf, tk, idx, s, (__nv_bfloat16*)dq, ctx);
+    note_launches(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (dscores) return launch_bwd_jacobian(s, da, idx, gates, dscores, 4, st);
   return cudaSuccess;
 }
 

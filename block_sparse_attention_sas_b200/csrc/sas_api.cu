@@ -223,9 +223,11 @@ sas_status_t sas_attn_fwd(sas_dtype_t dtype, const void* q, const void* k, const
   return cuda_status(launch_attn_fwd_simt(dtype, s, q, k, v, idx, gates, o, lse, ctx, stream));
 }
 
-size_t sas_attn_bwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int b, int K) {
-  if (check_attn(SAS_BF16, B, Hq, Hkv, T, d, b, K, false, 1.f) != SAS_OK) return 0;
-  return bwd_workspace_layout(make_shape(B, Hq, Hkv, T, d, b, K, 1.f, false)).total;
+size_t sas_attn_bwd_workspace_size(sas_dtype_t dtype, int B, int Hq, int Hkv, int T, int d, int b,
+                                   int K) {
+  if (check_attn(dtype, B, Hq, Hkv, T, d, b, K, false, 1.f) != SAS_OK) return 0;
+  const AttnShape s = make_shape(B, Hq, Hkv, T, d, b, K, 1.f, false);
+  return bwd_workspace_layout(s, tc_bwd_supported(dtype, s)).total;
 }
 
 sas_status_t sas_attn_bwd(sas_dtype_t dtype, const void* q, const void* k, const void* v,
@@ -245,7 +247,7 @@ sas_status_t sas_attn_bwd(sas_dtype_t dtype, const void* q, const void* k, const
       (dscores && !aligned(dscores, 4)))
     return SAS_ERR_INVALID_ARG;
   const AttnShape s = make_shape(B, Hq, Hkv, T, d, b, K, scale, false);
-  const size_t need = bwd_workspace_layout(s).total;
+  const size_t need = bwd_workspace_layout(s, tc_bwd_supported(dtype, s)).total;
   if (!ws || ws_bytes < need || !aligned(ws, 256)) return SAS_ERR_WORKSPACE;
   DevCtx ctx;
   if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
@@ -324,7 +326,7 @@ sas_status_t sas_dense_fwd(sas_dtype_t dtype, const void* q, const void* k, cons
 
 size_t sas_dense_bwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int b) {
   if (check_attn(SAS_BF16, B, Hq, Hkv, T, d, b, 0, true, 1.f) != SAS_OK) return 0;
-  return bwd_workspace_layout(make_shape(B, Hq, Hkv, T, d, b, 0, 1.f, true)).total;
+  return bwd_workspace_layout(make_shape(B, Hq, Hkv, T, d, b, 0, 1.f, true), false).total;
 }
 
 sas_status_t sas_dense_bwd(sas_dtype_t dtype, const void* q, const void* k, const void* v,
@@ -340,7 +342,7 @@ sas_status_t sas_dense_bwd(sas_dtype_t dtype, const void* q, const void* k, cons
       !aligned(lse, 4))
     return SAS_ERR_INVALID_ARG;
   const AttnShape s = make_shape(B, Hq, Hkv, T, d, b, 0, scale, true);
-  const size_t need = bwd_workspace_layout(s).total;
+  const size_t need = bwd_workspace_layout(s, false).total;
   if (!ws || ws_bytes < need || !aligned(ws, 256)) return SAS_ERR_WORKSPACE;
   DevCtx ctx;
   if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;

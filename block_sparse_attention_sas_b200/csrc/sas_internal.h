@@ -29,9 +29,11 @@ struct AttnShape {
 
 // Workspace carve-up of the backward pass (byte offsets, 256-aligned).
 struct BwdWorkspace {
-  size_t off_D, off_da, off_csr_off, off_csr_list, total;
+  size_t off_D, off_da, off_csr_off, off_csr_list, off_order, off_ds, total;
 };
-BwdWorkspace bwd_workspace_layout(const AttnShape& s);
+// `tc`: the tensor-core backward runs (it adds the stored dS tiles and keeps
+// da in four row chunks per head).
+BwdWorkspace bwd_workspace_layout(const AttnShape& s, bool tc);
 
 cudaError_t launch_attn_fwd_simt(sas_dtype_t dt, const AttnShape& s, const void* q, const void* k,
                                  const void* v, const int32_t* idx, const float* gates, void* o,
@@ -51,8 +53,9 @@ cudaError_t launch_attn_bwd_tc(const AttnShape& s, const void* q, const void* k,
 // Shared pieces of the backward (defined with the SIMT kernels).
 cudaError_t launch_bwd_csr(const AttnShape& s, const int32_t* idx, int32_t* off, int32_t* list,
                            const DevCtx& ctx, cudaStream_t stream);
+// da holds RC row chunks per (head, query block, slot).
 cudaError_t launch_bwd_jacobian(const AttnShape& s, const float* da, const int32_t* idx,
-                                const float* gates, float* dscores, cudaStream_t stream);
+                                const float* gates, float* dscores, int RC, cudaStream_t stream);
 // 3-D TMA map over a [planes][rows][128] bf16 tensor, 64x64 boxes, 128-byte swizzle.
 cudaError_t make_tmap_bf16(void* map, const void* ptr, int rows, int planes);
 

@@ -138,9 +138,12 @@ sas_status_t sas_attn_fwd(sas_dtype_t dtype, const void* q, const void* k, const
  *   q, k, v, idx, gates, scale as passed to sas_attn_fwd; o, lse its outputs;
  *   dO [B, Hq, T, d] (dtype). gates == NULL requires dscores == NULL.
  *   ws / ws_bytes: caller workspace of at least sas_attn_bwd_workspace_size()
- *   bytes, 256-byte aligned; its contents on entry do not matter.
+ *   bytes for the same dtype and shape, 256-byte aligned; its contents on
+ *   entry do not matter. (For bf16 with d = 128, b = 64 and G = 2 or 4 it
+ *   holds the dS tiles of every attended block: B*Hkv*N*(G/2)*(K+1)*16 KB.)
  */
-size_t sas_attn_bwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int b, int K);
+size_t sas_attn_bwd_workspace_size(sas_dtype_t dtype, int B, int Hq, int Hkv, int T, int d, int b,
+                                   int K);
 sas_status_t sas_attn_bwd(sas_dtype_t dtype, const void* q, const void* k, const void* v,
                           const void* o, const float* lse, const void* dO, const int32_t* idx,
                           const float* gates, int B, int Hq, int Hkv, int T, int d, int b, int K,

@@ -82,9 +82,12 @@ def test_gate_topk_rejects(raw):
 
 def test_bwd_workspace_and_gate_rules(raw):
     L = raw.LIB
-    need = L.sas_attn_bwd_workspace_size(1, 32, 8, 16384, 128, 64, 16)
+    need = L.sas_attn_bwd_workspace_size(1, 1, 32, 8, 16384, 128, 64, 16)
     assert need > 4 * 32 * 16384  # at least the per-row D vector
-    assert L.sas_attn_bwd_workspace_size(1, 3, 2, 128, 128, 64, 2) == 0  # invalid shape
+    # bf16 with the tensor-core shape also holds the dS tiles: 8*256*2*17 of 16 KB
+    assert need > 8 * 256 * 2 * 17 * 16384
+    assert L.sas_attn_bwd_workspace_size(0, 1, 32, 8, 16384, 128, 64, 16) < need  # fp32: no tiles
+    assert L.sas_attn_bwd_workspace_size(1, 1, 3, 2, 128, 128, 64, 2) == 0  # invalid shape
 
     def bwd(ws, ws_bytes, gates=None, ds=None):
         return L.sas_attn_bwd(1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, gates, 1, 32, 8, 16384,
