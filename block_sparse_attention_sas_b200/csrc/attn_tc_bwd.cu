@@ -585,16 +585,20 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   if (warp == 0) {
     // Scalars of a step (lse in the log2 domain and D of the tile's 128 rows,
-    // four per lane, the query block and its gate bias) are loaded into
-    // registers one step ahead, so staging them costs only shared stores.
-    float pre_lse[4], pre_D[4], pre_bias = 0.f;
-    int pre_j = m, pre_slot = s.K;
+    // four per lane, the query block, its slot and its gate) are loaded into
+    // registers two steps ahead (global loads are slow under this kernel's
+    // traffic), so staging them costs only shared stores.
+    struct Pre {
+      float lse[4], D[4], bias;
+      int j, slot;
+    };
     // The reverse list in a register window (lane l holds entry win_lo + l),
     // with the next window already in flight.
     int win_lo = 0;
     int win = lane < nl ? lst[lane] : 0;
     int win_next = 32 + lane < nl ? lst[32 + lane] : 0;
-    auto prefetch = [&](int st_i) {
+    auto prefetch = [&](int st_i) -> Pre {
+      Pre p;
       const int jj = st_i / TILES, u = st_i % TILES;
       int j = m, slot = s.K;  // the diagonal step's tile sits after the K slots
       if (jj > 0) {
@@ -608,20 +612,22 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
         j = e / s.K;
         slot = e % s.K;
       }
-      pre_j = j;
-      pre_slot = slot;
+      p.j = j;
+      p.slot = slot;
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         const int rr = lane + 32 * q4;
         const int head = kvh * G + 2 * u + (rr >> 6), qrow = j * kB + (rr & 63);
         const bool live = qrow < s.T;
         const long long hrow = (long long)(bi * s.Hq + head) * s.T + qrow;
-        pre_lse[q4] = live ? lse[hrow] : 0.f;
-        pre_D[q4] = live ? Dv[hrow] : 0.f;
+        p.lse[q4] = live ? lse[hrow] : 0.f;
+        p.D[q4] = live ? Dv[hrow] : 0.f;
       }
-      pre_bias = (j == m || gates == nullptr) ? 1.f : gates[((long long)bh * s.N + j) * s.N + m];
+      p.bias = (j == m || gates == nullptr) ? 1.f : gates[((long long)bh * s.N + j) * s.N + m];
+      return p;
     };
-    prefetch(0);
+    Pre cur = prefetch(0);
+    Pre nxt = nsteps > 1 ? prefetch(1) : cur;
     int issued = 0;
     for (int st_i = 0; st_i < nsteps; ++st_i) {
       const int stg = st_i & 1;
@@ -630,28 +636,26 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (lane == 0 && st_i >= 2)
         go = wait_or_abort(ctx, &c.dvdk_done[stg], ((st_i - 2) >> 1) & 1, abort);
       if (!__shfl_sync(0xffffffffu, go, 0)) break;
-      const int j = pre_j, u = st_i % TILES;
+      const int j = cur.j, u = st_i % TILES;
       if (lane == 0) {
+        // One 64 x 64 x 2 box per k-half brings both heads' rows of the tile.
         unsigned char* qd = base + kOffQD + stg * 65536;
+        const int plane = bi * s.Hq + kvh * G + 2 * u;
         mbar_arrive_expect_tx(&c.qdo_full[stg], 65536);
-        for (int hh = 0; hh < 2; ++hh)
-          for (int kb = 0; kb < 2; ++kb) {
-            const int plane = bi * s.Hq + kvh * G + 2 * u + hh;
-            tma_load_3d(qd + kb * 16384 + hh * 8192, &tm_q, kb * 64, j * kB, plane,
-                        &c.qdo_full[stg]);
-            tma_load_3d(qd + 32768 + kb * 16384 + hh * 8192, &tm_do, kb * 64, j * kB, plane,
-                        &c.qdo_full[stg]);
-          }
+        for (int kb = 0; kb < 2; ++kb) {
+          tma_load_3d(qd + kb * 16384, &tm_q, kb * 64, j * kB, plane, &c.qdo_full[stg]);
+          tma_load_3d(qd + 32768 + kb * 16384, &tm_do, kb * 64, j * kB, plane, &c.qdo_full[stg]);
+        }
       }
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
-        c.lse2[stg][lane + 32 * q4] = pre_lse[q4] * kLog2e;
-        c.D[stg][lane + 32 * q4] = pre_D[q4];
+        c.lse2[stg][lane + 32 * q4] = cur.lse[q4] * kLog2e;
+        c.D[stg][lane + 32 * q4] = cur.D[q4];
       }
       if (lane == 0) {
         c.step_j[stg] = j;
-        c.step_slot[stg] = pre_slot;
-        c.step_bias[stg] = logf(pre_bias) * kLog2e;
+        c.step_slot[stg] = cur.slot;
+        c.step_bias[stg] = logf(cur.bias) * kLog2e;
       }
       __threadfence_block();
       __syncwarp();
@@ -659,7 +663,8 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       // completes: the arrival below is part of it.
       if (lane == 0) mbar_arrive(&c.qdo_full[stg]);
       issued = st_i + 1;
-      if (st_i + 1 < nsteps) prefetch(st_i + 1);
+      cur = nxt;
+      if (st_i + 2 < nsteps) nxt = prefetch(st_i + 2);
     }
     if (lane == 0 && *abort) {
       (void)mbar_wait(ctx, &c.kv_full, 0);
@@ -893,6 +898,9 @@ cudaError_t launch_attn_bwd_tc(const AttnShape& s, const void* q, const void* k,
   if ((e = make_tmap_bf16(&tdo, dO, s.T, s.B * s.Hq)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16(&tk, k, s.T, s.B * s.Hkv)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16(&tv, v, s.T, s.B * s.Hkv)) != cudaSuccess) return e;
+  CUtensorMap tq2, tdo2;  // 64 x 64 x 2 boxes for the dK/dV kernel's 128-row tiles
+  if ((e = make_tmap_bf16_2planes(&tq2, q, s.T, s.B * s.Hq)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_2planes(&tdo2, dO, s.T, s.B * s.Hq)) != cudaSuccess) return e;
   if ((e = launch_bwd_csr(s, idx, coff, clist, ctx, st)) != cudaSuccess) return e;
   {
     const size_t smem = sizeof(int32_t) * ((size_t)s.N + 1);
@@ -916,7 +924,7 @@ cudaError_t launch_attn_bwd_tc(const AttnShape& s, const void* q, const void* k,
     auto kern = tiles == 2 ? tc_bwd_dkdv_kernel<2> : tc_bwd_dkdv_kernel<1>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kb_::kSmem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kb_::kThreadsB, kb_::kSmem, st>>>(tq, tk, tv, tdo, lse, Dv, gates, coff, clist,
+    kern<<<grid, kb_::kThreadsB, kb_::kSmem, st>>>(tq2, tk, tv, tdo2, lse, Dv, gates, coff, clist,
                                                    order, s, (__nv_bfloat16*)dk,
                                                    (__nv_bfloat16*)dv, dsbuf,
                                                    dscores ? da : nullptr, ctx);

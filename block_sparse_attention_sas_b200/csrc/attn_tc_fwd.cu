@@ -415,6 +415,22 @@ cudaError_t make_tmap_bf16(void* map_out, const void* ptr, int rows, int planes)
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// Same map with 64 x 64 x 2 boxes: one box brings the same 64 rows of two
+// consecutive planes (two heads), i.e. a 128-row tile's k-half.
+cudaError_t make_tmap_bf16_2planes(void* map_out, const void* ptr, int rows, int planes) {
+  CUtensorMap* map = static_cast<CUtensorMap*>(map_out);
+  EncodeTiled enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)rows, (cuuint64_t)planes};
+  const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)rows * kD * 2};
+  const cuuint32_t box[3] = {64, 64, 2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 // Same, with planes `pitch_rows` rows apart of which the first `rows` are in
 // the map (a KV cache of capacity pitch_rows filled up to rows).
 cudaError_t make_tmap_bf16_pitched(void* map_out, const void* ptr, int rows, int pitch_rows,

@@ -86,6 +86,8 @@ bool tc_decode_supported(sas_dtype_t dt, const DecodeShape& s);
 cudaError_t launch_decode_tc(const DecodeShape& s, const void* q, const void* kc, const void* vc,
                              const int32_t* idx, const float* gates, void* o, void* ws,
                              const DevCtx& ctx, cudaStream_t stream);
+// The same map with 64 x 64 x 2 boxes (two consecutive planes per box).
+cudaError_t make_tmap_bf16_2planes(void* map, const void* ptr, int rows, int planes);
 // 3-D TMA map over planes of `pitch_rows` rows, the first `rows` of each mapped.
 cudaError_t make_tmap_bf16_pitched(void* map, const void* ptr, int rows, int pitch_rows,
                                    int planes);
