@@ -58,7 +58,11 @@ struct Ctl {
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
   // One barrier for both tiles where they move in step (fewer waits and
   // commits on the MMA thread, whose overhead sits on the critical path).
-  uint64_t q_tmem, s_full, s_free, p_full, pv_done;
+  // k_full[st] also takes one arrival per softmax warp once it is done with
+  // the previous S (or, for block 0, has moved its Q rows into TMEM); v_full[st]
+  // also takes one per softmax warp once P of that block is in shared memory.
+  // The MMA thread thus waits twice per block.
+  uint64_t s_full, pv_done;
   uint64_t drain;  // abort path only: the MMA thread's last commit
   uint32_t tmem_base;
   int abort;
@@ -94,15 +98,12 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   if (tid == 0) {
     mbar_init(&c.q_full, 1);
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&c.k_full[i], 1);
+      mbar_init(&c.k_full[i], 1 + 4 * TILES);
       mbar_init(&c.k_empty[i], 1);
-      mbar_init(&c.v_full[i], 1);
+      mbar_init(&c.v_full[i], 1 + 4 * TILES);
       mbar_init(&c.v_empty[i], 1);
     }
-    mbar_init(&c.q_tmem, 128 * TILES);
     mbar_init(&c.s_full, 1);
-    mbar_init(&c.s_free, 128 * TILES);
-    mbar_init(&c.p_full, 128 * TILES);
     mbar_init(&c.pv_done, 1);
     mbar_init(&c.drain, 1);
     fence_mbar_init();
@@ -183,11 +184,9 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       auto adv = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
       auto issue_s = [&](int n) -> bool {
         const int st = n % kStages;
+        // K(n) has landed and S is free: the softmax warps copied S(n-1) (or
+        // their Q rows, for n = 0) out of TMEM.
         if (!wait_or_abort(ctx, &c.k_full[st], (n / kStages) & 1, abort)) return false;
-        // S is single-buffered: the softmax copies S(n-1) to registers first.
-        if (!wait_or_abort(ctx, n == 0 ? &c.q_tmem : &c.s_free, n == 0 ? 0 : ((n - 1) & 1),
-                           abort))
-          return false;
         fence_after_sync();
         const uint64_t kd = adv(kdesc0, st * kKVBytes);
         for (int t = 0; t < TILES; ++t) {
@@ -204,8 +203,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       for (int n = 0; ok && n < nblk; ++n) {
         if (n + 1 < nblk && !issue_s(n + 1)) break;
         const int st = n % kStages;
+        // V(n) has landed and P(n) is in shared memory.
         if (!wait_or_abort(ctx, &c.v_full[st], (n / kStages) & 1, abort)) break;
-        if (!wait_or_abort(ctx, &c.p_full, n & 1, abort)) break;
         fence_after_sync();
         const uint64_t vd = adv(vdesc0, st * kKVBytes);
         for (int t = 0; t < TILES; ++t) {
@@ -244,7 +243,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tile_row_to_tmem(base + kOffQ + t * 32768, rowi, tl + q_col(t));
         tmem_st_wait();
         fence_before_sync();
-        mbar_arrive(&c.q_tmem);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c.k_full[0]);  // S(0) may read Q from TMEM
       }
     }
     for (int n = 0; ok && n < nblk; ++n) {
@@ -258,7 +258,9 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       tmem_ld32(tl + s_col(t) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_ld_wait();
       fence_before_sync();
-      mbar_arrive(&c.s_free);
+      __syncwarp();
+      // S(n) is in registers: S(n + 1) may overwrite the accumulator.
+      if (lane == 0 && n + 1 < nblk) mbar_arrive(&c.k_full[(n + 1) % kStages]);
 
       const int m = c.blocks[n];
       const float bias = c.bias[n];
@@ -339,7 +341,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       }
       fence_proxy_async_smem();
       fence_before_sync();
-      mbar_arrive(&c.p_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&c.v_full[n % kStages]);  // P(n) is ready for PV(n)
     }
     if (ok && t < TILES) {
       // ---- epilogue: O / l and the log-sum-exp
