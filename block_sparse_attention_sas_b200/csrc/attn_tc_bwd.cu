@@ -487,28 +487,34 @@ order_kernel(const int32_t* __restrict__ off_all, AttnShape s, int32_t* __restri
 // ============================================================================
 // One CTA per (key block m, KV head, batch) steps over 128-row query tiles
 // (the diagonal block's, then those of every query block that selected m).
-// MMA stream: per step s, S/dP(s) then dV/dK(s - 1). The MMA thread waits
-// once per step, on the Q/dO stage barrier of step s, which also collects
-// one arrival from each elementwise warp once it has written P/dS of step
-// s - 1 to shared memory (so the S/dP buffer of step s - 2 is free as well).
-// A commit after dV/dK(s - 1) lets the producer reuse that Q/dO stage and
-// the elementwise warps the P/dS buffer.
+// The MMA stream goes by pairs of steps: S/dP(s), S/dP(s + 1), dV/dK(s),
+// dV/dK(s + 1). P/dS are double-buffered in shared memory, so while the
+// elementwise warps turn S/dP(s + 1) into P/dS the tensor pipe runs dV/dK(s),
+// and a Q/dO stage freed by dV/dK(s) reloads while dV/dK(s + 1) and the next
+// S/dP run. Each hand-off has its own barrier, so a stage is refilled as
+// soon as the MMAs that read it are done, whatever the dS store warp is
+// doing.
 namespace kb_ {
 constexpr int kWarps = 12;
 constexpr int kThreadsB = kWarps * 32;
+// Tile offsets from the first 1024-byte boundary after the control block.
 constexpr uint32_t kOffK = 0;         // [d half][64 rows][128 B]
 constexpr uint32_t kOffV = 16384;
 constexpr uint32_t kOffQD = 32768;    // 2 stages x (Q tile 32 KB, dO tile 32 KB)
-constexpr uint32_t kOffP = 163840;    // [128 rows][128 B]
-constexpr uint32_t kOffDS = 180224;
-constexpr uint32_t kOffCtl = 196608;
+constexpr uint32_t kOffPD = 163840;   // 2 buffers x (P [128 rows][128 B], dS at +16 KB)
+constexpr uint32_t kTileBytes = 229376;
 // TMEM columns: S[b] at 64 b, dP[b] at 128 + 64 b, dV^T at 256, dK^T at 320.
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 320;
 struct Ctl {
-  // qdo_full[stg]: the producer's expect-tx arrival and tile bytes, its
-  // arrival once the step's scalars are staged, and one arrival per
-  // elementwise warp (10 arrivals per phase).
-  uint64_t kv_full, qdo_full[2], s_full[2], dvdk_done[2], pds_tail, acc_done, drain;
+  // qdo_full[stg]: the producer's expect-tx arrival plus tile bytes, and its
+  // arrival once the step's scalars are staged. s_full[b]: MMA commit after
+  // S/dP. pds_full[b]: one arrival per elementwise warp once P/dS of the step
+  // are in buffer b. stage_free[b]: MMA commit after dV/dK of the step (the
+  // Q/dO stage and its scalars may be refilled). buf_free[b]: the dS store
+  // warp, once dV/dK of the step are done and it has copied dS out of
+  // buffer b (the buffer and its scalars may be rewritten).
+  uint64_t kv_full, qdo_full[2], s_full[2], pds_full[2], stage_free[2], buf_free[2];
+  uint64_t acc_done, drain;
   uint32_t tmem_base;
   int abort;
   // Per stage, staged by the producer warp with the Q/dO tiles: the step's
@@ -516,9 +522,19 @@ struct Ctl {
   int step_j[2], step_slot[2];
   float step_bias[2];
   float lse2[2][128], D[2][128];
-  float dapart[2][8];  // per-warp shares of the step's tile sum of dS
+  // Per P/dS buffer, written by the elementwise warps for the store warp:
+  // the step's query block and slot, and per-warp shares of its tile sum of dS.
+  int buf_j[2], buf_slot[2];
+  float dapart[2][8];
 };
-constexpr size_t kSmem = kOffCtl + sizeof(Ctl) + 1024;
+// The control block sits at the start of dynamic shared memory and the tiles
+// at the next 1024-byte boundary. With a 1024-aligned base (the case when a
+// kernel declares no static shared memory) this is exactly the 227 KB limit;
+// the kernel checks the carve-out and reports kDevErrLayout otherwise.
+constexpr uint32_t kCtlSpan = 3072;
+static_assert(sizeof(Ctl) <= kCtlSpan, "control block outgrew its span");
+constexpr size_t kSmem = kCtlSpan + kTileBytes;
+static_assert(kSmem <= 232448, "over the per-block shared memory limit");
 }  // namespace kb_
 
 template <int TILES>
@@ -535,9 +551,14 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
   using namespace kb_;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
-  unsigned char* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const uint32_t tiles_off = ((raw + (uint32_t)sizeof(Ctl) + 1023u) & ~1023u) - raw;
+  if (tiles_off + kTileBytes > kSmem) {  // uniform over the CTA: nothing started yet
+    if (threadIdx.x == 0) report(ctx, kDevErrLayout);
+    return;
+  }
+  Ctl& c = *reinterpret_cast<Ctl*>(smem_raw);
+  unsigned char* base = smem_raw + tiles_off;
   const uint32_t sbase = smem_u32(base);
-  Ctl& c = *reinterpret_cast<Ctl*>(base + kOffCtl);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int unit = order[blockIdx.x];
@@ -555,11 +576,12 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
   if (tid == 0) {
     mbar_init(&c.kv_full, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&c.qdo_full[i], 10);
+      mbar_init(&c.qdo_full[i], 2);
       mbar_init(&c.s_full[i], 1);
-      mbar_init(&c.dvdk_done[i], 2);  // the MMA commit + the dS store warp
+      mbar_init(&c.pds_full[i], 8);
+      mbar_init(&c.stage_free[i], 1);
+      mbar_init(&c.buf_free[i], 1);
     }
-    mbar_init(&c.pds_tail, 8);
     mbar_init(&c.acc_done, 1);
     mbar_init(&c.drain, 1);
     fence_mbar_init();
@@ -634,7 +656,7 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       bool go = true;
       // The stage is free once dV/dK of step st_i - 2 completed.
       if (lane == 0 && st_i >= 2)
-        go = wait_or_abort(ctx, &c.dvdk_done[stg], ((st_i - 2) >> 1) & 1, abort);
+        go = wait_or_abort(ctx, &c.stage_free[stg], ((st_i - 2) >> 1) & 1, abort);
       if (!__shfl_sync(0xffffffffu, go, 0)) break;
       const int j = cur.j, u = st_i % TILES;
       if (lane == 0) {
@@ -657,12 +679,18 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
         c.step_slot[stg] = cur.slot;
         c.step_bias[stg] = logf(cur.bias) * kLog2e;
       }
-      __threadfence_block();
+      // The arrival that completes this stage's phase also waits until the
+      // store warp has released P/dS buffer st_i & 1 (step st_i - 2), so the
+      // elementwise warps may write it as soon as S/dP of this step are done;
+      // the wait overlaps the tile loads. The consumers see the staged
+      // scalars once the phase completes: the warp's stores are ordered
+      // before lane 0's (release) arrival by the warp barrier.
+      if (lane == 0 && st_i >= 2)
+        go = wait_or_abort(ctx, &c.buf_free[stg], ((st_i - 2) >> 1) & 1, abort);
       __syncwarp();
-      // The consumers see the staged scalars once this stage's barrier phase
-      // completes: the arrival below is part of it.
       if (lane == 0) mbar_arrive(&c.qdo_full[stg]);
       issued = st_i + 1;
+      if (!__shfl_sync(0xffffffffu, go, 0)) break;
       cur = nxt;
       if (st_i + 2 < nsteps) nxt = prefetch(st_i + 2);
     }
@@ -678,10 +706,10 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint64_t dq0 = sdesc_sw128(sbase + kOffQD, 16, 1024);    // Q/dO stages, K-major
       const uint64_t dk0 = sdesc_sw128(sbase + kOffK, 16, 1024);     // K (V at +16 KB)
       const uint64_t dqt0 = sdesc_sw128(sbase + kOffQD, 16384, 1024);  // Q/dO as MN-major A
-      const uint64_t dp0 = sdesc_sw128(sbase + kOffP, 8192, 1024);   // P (dS at +16 KB)
+      const uint64_t dp0 = sdesc_sw128(sbase + kOffPD, 8192, 1024);  // P[b] (dS[b] at +16 KB)
       auto issue_sdp = [&](int st_i) {
-        const int stg = st_i & 1, b = st_i & 1;
-        const uint64_t qa = dq0 + ((stg * 65536) >> 4);
+        const int b = st_i & 1;
+        const uint64_t qa = dq0 + ((b * 65536) >> 4);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t ao = (ks >> 2) * 16384 + (ks & 3) * 32;
@@ -698,36 +726,33 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       };
       // dV^T[d][key] += sum_q dO[q][d] P[q][key]; dK^T[d][key] += sum_q Q[q][d] dS[q][key]
       auto issue_dvdk = [&](int st_i) {
-        const uint64_t qa = dqt0 + (((st_i & 1) * 65536) >> 4);
+        const int b = st_i & 1;
+        const uint64_t qa = dqt0 + ((b * 65536) >> 4);
+        const uint64_t pa = dp0 + ((b * 32768) >> 4);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          mma_bf16_ss(tmem + kColDV, qa + ((32768 + ks * 2048) >> 4), dp0 + ((ks * 2048) >> 4),
+          mma_bf16_ss(tmem + kColDV, qa + ((32768 + ks * 2048) >> 4), pa + ((ks * 2048) >> 4),
                       id_t, (st_i > 0 || ks > 0));
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          mma_bf16_ss(tmem + kColDK, qa + ((ks * 2048) >> 4), dp0 + ((16384 + ks * 2048) >> 4),
+          mma_bf16_ss(tmem + kColDK, qa + ((ks * 2048) >> 4), pa + ((16384 + ks * 2048) >> 4),
                       id_t, (st_i > 0 || ks > 0));
+        mma_commit(&c.stage_free[b]);
       };
       bool ok = wait_or_abort(ctx, &c.kv_full, 0, abort);
-      // Per step s: one wait (the Q/dO tiles of step s have landed and P/dS
-      // of step s - 1 is in shared memory), then S/dP(s), so the elementwise
-      // warps can start on it, then dV/dK(s - 1); its commit frees the Q/dO
-      // stage of step s - 1 and the P/dS buffer.
-      for (int st_i = 0; ok && st_i < nsteps; ++st_i) {
-        if (!wait_or_abort(ctx, &c.qdo_full[st_i & 1], (st_i >> 1) & 1, abort)) {
-          ok = false;
-          break;
+      for (int s0 = 0; ok && s0 < nsteps; s0 += 2) {
+        const int npair = min(2, nsteps - s0);
+        const uint32_t ph = (s0 >> 1) & 1;
+        for (int e = 0; ok && e < npair; ++e) {
+          if (!wait_or_abort(ctx, &c.qdo_full[e], ph, abort)) { ok = false; break; }
+          fence_after_sync();
+          issue_sdp(s0 + e);
         }
-        fence_after_sync();
-        issue_sdp(st_i);
-        if (st_i > 0) {
-          issue_dvdk(st_i - 1);
-          mma_commit(&c.dvdk_done[(st_i - 1) & 1]);
+        for (int e = 0; ok && e < npair; ++e) {
+          if (!wait_or_abort(ctx, &c.pds_full[e], ph, abort)) { ok = false; break; }
+          fence_after_sync();
+          issue_dvdk(s0 + e);
         }
-      }
-      if (ok && wait_or_abort(ctx, &c.pds_tail, 0, abort)) {
-        fence_after_sync();
-        issue_dvdk(nsteps - 1);
       }
       mma_commit(&c.acc_done);
       if (*abort) {
@@ -736,32 +761,30 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
     }
   } else if (warp == 2) {
-    // dS store warp: once P/dS of step s are in shared memory (the next
-    // stage's full barrier, or the tail barrier), copy the raw 16 KB dS tile
-    // (swizzled, as the dq kernel's MMA reads it) to the workspace with the
-    // TMA engine and write the step's da shares; its arrival on dvdk_done
-    // (with the MMA's commit) frees the P/dS buffer and the stage's scalars.
+    // dS store warp: once P/dS of step s are in buffer s & 1, copy the raw
+    // 16 KB dS tile (swizzled, as the dq kernel's MMA reads it) to the
+    // workspace with the TMA engine and write the step's da shares; once the
+    // copy has read the buffer and dV/dK of the step are done, its arrival
+    // on buf_free lets the elementwise warps rewrite the buffer.
     if (lane == 0) {
       for (int st_i = 0; st_i < nsteps; ++st_i) {
-        const bool last = st_i + 1 == nsteps;
-        const bool ok2 = last ? wait_or_abort(ctx, &c.pds_tail, 0, abort)
-                              : wait_or_abort(ctx, &c.qdo_full[(st_i + 1) & 1],
-                                              ((st_i + 1) >> 1) & 1, abort);
-        if (!ok2) break;
-        const int stg = st_i & 1, u = st_i % TILES;
-        const int j = c.step_j[stg], slot = c.step_slot[stg];
+        const int b = st_i & 1, u = st_i % TILES;
+        const uint32_t ph = (st_i >> 1) & 1;
+        if (!wait_or_abort(ctx, &c.pds_full[b], ph, abort)) break;
+        const int j = c.buf_j[b], slot = c.buf_slot[b];
         const long long tile = (((long long)bh * s.N + j) * TILES + u) * (s.K + 1) + slot;
-        bulk_s2g(ds_out + tile * (128 * 64), base + kOffDS, 16384);
+        bulk_s2g(ds_out + tile * (128 * 64), base + kOffPD + b * 32768 + 16384, 16384);
         bulk_commit();
         if (da != nullptr && slot < s.K) {
 #pragma unroll
           for (int p = 0; p < 8; ++p) {
             const int head = kvh * G + 2 * u + ((p & 3) >> 1), rc = (p >> 2) * 2 + (p & 1);
-            da[(((long long)(bi * s.Hq + head) * s.N + j) * 4 + rc) * s.K + slot] = c.dapart[stg][p];
+            da[(((long long)(bi * s.Hq + head) * s.N + j) * 4 + rc) * s.K + slot] = c.dapart[b][p];
           }
         }
         bulk_wait_read_all();
-        if (!last) mbar_arrive(&c.dvdk_done[stg]);
+        if (!wait_or_abort(ctx, &c.stage_free[b], ph, abort)) break;
+        mbar_arrive(&c.buf_free[b]);
       }
       bulk_wait_all();
     }
@@ -773,8 +796,6 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
     const float sc = s.scale * kLog2e;
     const int kvalid = min(kB, s.T - m * kB) - 32 * grp;
     const uint64_t sc2 = f2u(sc, sc);
-    // Step 0 has no P/dS of a previous step to wait for.
-    if (lane == 0) mbar_arrive(&c.qdo_full[0]);
     bool ok = true;
     for (int st_i = 0; st_i < nsteps; ++st_i) {
       const int b = st_i & 1;
@@ -783,15 +804,16 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
         break;
       }
       fence_after_sync();
-      const int stg = st_i & 1;
-      const int j = c.step_j[stg];
+      const int j = c.step_j[b];
       const int qrow = j * kB + r;
       const bool live = qrow < s.T;
-      const float lse2 = c.lse2[stg][rowi];
-      const float Di = c.D[stg][rowi];
+      const float lse2 = c.lse2[b][rowi];
+      const float Di = c.D[b][rowi];
       const bool cur = (j == m);
-      const float bias = c.step_bias[stg];
+      const float bias = c.step_bias[b];
       uint32_t sr[32], pr[32], pp[16], dd[16];
+      // Buffer b is free: the producer's arrival in this step's Q/dO phase,
+      // which S/dP(st_i) waited for, came after the store warp released it.
       tmem_ld32(tl + kColS + b * 64 + 32 * grp, sr);
       tmem_ld32(tl + kColDP + b * 64 + 32 * grp, pr);
       tmem_ld_wait();
@@ -815,17 +837,16 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
         dd[i] = pack_bf16(lo_f(ds2), hi_f(ds2));
       }
 
-      // The P / dS buffers are free once dV/dK of step st_i - 1 completed.
-      if (st_i >= 1 && !warp_wait(ctx, &c.dvdk_done[(st_i - 1) & 1], ((st_i - 1) >> 1) & 1, abort)) {
-        ok = false;
-        break;
-      }
       {  // this warp's share of the tile sum of dS, for the store warp
         const float t = warp_sum(lo_f(dsum) + hi_f(dsum));
-        if (lane == 0) c.dapart[stg][grp * 4 + quarter] = t;
+        if (lane == 0) c.dapart[b][grp * 4 + quarter] = t;
+        if (lane == 0 && warp == 4) {
+          c.buf_j[b] = j;
+          c.buf_slot[b] = c.step_slot[b];
+        }
       }
-      unsigned char* prow = base + kOffP + rowi * 128;
-      unsigned char* drow = base + kOffDS + rowi * 128;
+      unsigned char* prow = base + kOffPD + b * 32768 + rowi * 128;
+      unsigned char* drow = prow + 16384;
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         const uint32_t sw = ((4 * grp + ch) ^ (rowi & 7)) << 4;
@@ -837,10 +858,7 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       fence_proxy_async_smem();
       fence_before_sync();
       __syncwarp();
-      if (lane == 0) {
-        if (st_i + 1 < nsteps) mbar_arrive(&c.qdo_full[(st_i + 1) & 1]);
-        else mbar_arrive(&c.pds_tail);
-      }
+      if (lane == 0) mbar_arrive(&c.pds_full[b]);
     }
     if (ok && warp_wait(ctx, &c.acc_done, 0, abort)) {
       // Epilogue: thread rowi holds dimension d = rowi; group g the keys 32g .. 32g + 31.

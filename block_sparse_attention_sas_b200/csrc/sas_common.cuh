@@ -13,6 +13,7 @@ namespace sas {
 enum : uint32_t {
   kDevErrTimeout = 1u,  // a bounded wait ran out of iterations
   kDevErrBadIndex = 2u, // an idx entry outside [0, j) (or [0, C) for decode)
+  kDevErrLayout = 4u,   // dynamic shared memory too misaligned for a kernel's tile layout
 };
 
 // Passed by value to every kernel: where to report device-side errors and
