@@ -507,13 +507,15 @@ constexpr uint32_t kTileBytes = 229376;
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 320;
 struct Ctl {
   // qdo_full[stg]: the producer's expect-tx arrival plus tile bytes, and its
-  // arrival once the step's scalars are staged. s_full[b]: MMA commit after
-  // S/dP. pds_full[b]: one arrival per elementwise warp once P/dS of the step
-  // are in buffer b. stage_free[b]: MMA commit after dV/dK of the step (the
+  // arrival once the step's scalars are staged. s_full[b] / dp_full[b]: MMA
+  // commits after S and after dP. pds_full[b]: one arrival per elementwise
+  // warp once P/dS of the step are in buffer b; da_full[b]: the same once its
+  // share of the tile sum of dS is in dapart. stage_free[b]: MMA commit after dV/dK of the step (the
   // Q/dO stage and its scalars may be refilled). buf_free[b]: the dS store
   // warp, once dV/dK of the step are done and it has copied dS out of
   // buffer b (the buffer and its scalars may be rewritten).
-  uint64_t kv_full, qdo_full[2], s_full[2], pds_full[2], stage_free[2], buf_free[2];
+  uint64_t kv_full, qdo_full[2], s_full[2], dp_full[2], pds_full[2], da_full[2];
+  uint64_t stage_free[2], buf_free[2];
   uint64_t acc_done, drain;
   uint32_t tmem_base;
   int abort;
@@ -578,7 +580,9 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int i = 0; i < 2; ++i) {
       mbar_init(&c.qdo_full[i], 2);
       mbar_init(&c.s_full[i], 1);
+      mbar_init(&c.dp_full[i], 1);
       mbar_init(&c.pds_full[i], 8);
+      mbar_init(&c.da_full[i], 8);
       mbar_init(&c.stage_free[i], 1);
       mbar_init(&c.buf_free[i], 1);
     }
@@ -692,7 +696,19 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       issued = st_i + 1;
       if (!__shfl_sync(0xffffffffu, go, 0)) break;
       cur = nxt;
-      if (st_i + 2 < nsteps) nxt = prefetch(st_i + 2);
+      if (st_i + 2 < nsteps) {
+        nxt = prefetch(st_i + 2);
+        // Under this kernel's load a stage's tiles take ~2000 cycles to land
+        // from HBM, more than the MMAs between a stage's release and its next
+        // use; pulling the tiles of step st_i + 2 into L2 now hides that.
+        if (lane == 0) {
+          const int plane2 = bi * s.Hq + kvh * G + 2 * ((st_i + 2) % TILES);
+          for (int kb = 0; kb < 2; ++kb) {
+            tma_prefetch_l2_3d(&tm_q, kb * 64, nxt.j * kB, plane2);
+            tma_prefetch_l2_3d(&tm_do, kb * 64, nxt.j * kB, plane2);
+          }
+        }
+      }
     }
     if (lane == 0 && *abort) {
       (void)mbar_wait(ctx, &c.kv_full, 0);
@@ -716,13 +732,14 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
           const uint32_t bo = (ks >> 2) * 8192 + (ks & 3) * 32;
           mma_bf16_ss(tmem + kColS + b * 64, qa + (ao >> 4), dk0 + (bo >> 4), id_s, ks > 0);
         }
+        mma_commit(&c.s_full[b]);  // P can be formed while dP runs
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t ao = 32768 + (ks >> 2) * 16384 + (ks & 3) * 32;
           const uint32_t bo = 16384 + (ks >> 2) * 8192 + (ks & 3) * 32;
           mma_bf16_ss(tmem + kColDP + b * 64, qa + (ao >> 4), dk0 + (bo >> 4), id_s, ks > 0);
         }
-        mma_commit(&c.s_full[b]);
+        mma_commit(&c.dp_full[b]);
       };
       // dV^T[d][key] += sum_q dO[q][d] P[q][key]; dK^T[d][key] += sum_q Q[q][d] dS[q][key]
       auto issue_dvdk = [&](int st_i) {
@@ -775,6 +792,7 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
         const long long tile = (((long long)bh * s.N + j) * TILES + u) * (s.K + 1) + slot;
         bulk_s2g(ds_out + tile * (128 * 64), base + kOffPD + b * 32768 + 16384, 16384);
         bulk_commit();
+        if (da != nullptr && !wait_or_abort(ctx, &c.da_full[b], ph, abort)) break;
         if (da != nullptr && slot < s.K) {
 #pragma unroll
           for (int p = 0; p < 8; ++p) {
@@ -811,54 +829,77 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       const float Di = c.D[b][rowi];
       const bool cur = (j == m);
       const float bias = c.step_bias[b];
-      uint32_t sr[32], pr[32], pp[16], dd[16];
       // Buffer b is free: the producer's arrival in this step's Q/dO phase,
-      // which S/dP(st_i) waited for, came after the store warp released it.
-      tmem_ld32(tl + kColS + b * 64 + 32 * grp, sr);
-      tmem_ld32(tl + kColDP + b * 64 + 32 * grp, pr);
-      tmem_ld_wait();
-      if (cur || kvalid < 32) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (i >= kvalid || (cur && i + 32 * grp > r)) sr[i] = __float_as_uint(-INFINITY);
-      }
-      const float off = live ? bias - lse2 : -INFINITY;
-      const uint64_t off2 = f2u(off, off), negD = f2u(-Di, -Di);
-      uint64_t dsum = 0;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const uint64_t a2 = ffma2(f2u(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
-                                  sc2, off2);
-        const float p0 = ex2(lo_f(a2)), p1 = ex2(hi_f(a2));
-        const uint64_t dp2 = f2u(__uint_as_float(pr[2 * i]), __uint_as_float(pr[2 * i + 1]));
-        const uint64_t ds2 = fmul2(f2u(p0, p1), fadd2(dp2, negD));
-        dsum = fadd2(dsum, ds2);
-        pp[i] = pack_bf16(p0, p1);
-        dd[i] = pack_bf16(lo_f(ds2), hi_f(ds2));
-      }
-
-      {  // this warp's share of the tile sum of dS, for the store warp
-        const float t = warp_sum(lo_f(dsum) + hi_f(dsum));
-        if (lane == 0) c.dapart[b][grp * 4 + quarter] = t;
-        if (lane == 0 && warp == 4) {
-          c.buf_j[b] = j;
-          c.buf_slot[b] = c.step_slot[b];
-        }
-      }
+      // which S(st_i) waited for, came after the store warp released it.
       unsigned char* prow = base + kOffPD + b * 32768 + rowi * 128;
       unsigned char* drow = prow + 16384;
+      float pf[32];
+      {  // P = exp2(S * scale * log2 e + log2 gate - lse * log2 e), while dP is computed
+        uint32_t sr[32], pp[16];
+        tmem_ld32(tl + kColS + b * 64 + 32 * grp, sr);
+        tmem_ld_wait();
+        if (cur || kvalid < 32) {
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        const uint32_t sw = ((4 * grp + ch) ^ (rowi & 7)) << 4;
-        *reinterpret_cast<uint4*>(prow + sw) = make_uint4(pp[4 * ch], pp[4 * ch + 1],
-                                                          pp[4 * ch + 2], pp[4 * ch + 3]);
-        *reinterpret_cast<uint4*>(drow + sw) = make_uint4(dd[4 * ch], dd[4 * ch + 1],
-                                                          dd[4 * ch + 2], dd[4 * ch + 3]);
+          for (int i = 0; i < 32; ++i)
+            if (i >= kvalid || (cur && i + 32 * grp > r)) sr[i] = __float_as_uint(-INFINITY);
+        }
+        const float off = live ? bias - lse2 : -INFINITY;
+        const uint64_t off2 = f2u(off, off);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint64_t a2 = ffma2(f2u(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
+                                    sc2, off2);
+          pf[2 * i] = ex2(lo_f(a2));
+          pf[2 * i + 1] = ex2(hi_f(a2));
+          pp[i] = pack_bf16(pf[2 * i], pf[2 * i + 1]);
+        }
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const uint32_t sw = ((4 * grp + ch) ^ (rowi & 7)) << 4;
+          *reinterpret_cast<uint4*>(prow + sw) = make_uint4(pp[4 * ch], pp[4 * ch + 1],
+                                                            pp[4 * ch + 2], pp[4 * ch + 3]);
+        }
+      }
+      if (!warp_wait(ctx, &c.dp_full[b], (st_i >> 1) & 1, abort)) {
+        ok = false;
+        break;
+      }
+      fence_after_sync();
+      uint64_t dsum = 0;
+      {  // dS = P (dP - D)
+        uint32_t pr[32], dd[16];
+        tmem_ld32(tl + kColDP + b * 64 + 32 * grp, pr);
+        tmem_ld_wait();
+        const uint64_t negD = f2u(-Di, -Di);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint64_t dp2 = f2u(__uint_as_float(pr[2 * i]), __uint_as_float(pr[2 * i + 1]));
+          const uint64_t ds2 = fmul2(f2u(pf[2 * i], pf[2 * i + 1]), fadd2(dp2, negD));
+          dsum = fadd2(dsum, ds2);
+          dd[i] = pack_bf16(lo_f(ds2), hi_f(ds2));
+        }
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const uint32_t sw = ((4 * grp + ch) ^ (rowi & 7)) << 4;
+          *reinterpret_cast<uint4*>(drow + sw) = make_uint4(dd[4 * ch], dd[4 * ch + 1],
+                                                            dd[4 * ch + 2], dd[4 * ch + 3]);
+        }
+      }
+      if (lane == 0 && warp == 4) {
+        c.buf_j[b] = j;
+        c.buf_slot[b] = c.step_slot[b];
       }
       fence_proxy_async_smem();
       fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&c.pds_full[b]);
+      {  // this warp's share of the tile sum of dS, for the store warp, off the MMA's path
+        const float t = warp_sum(lo_f(dsum) + hi_f(dsum));
+        if (lane == 0) {
+          c.dapart[b][grp * 4 + quarter] = t;
+          mbar_arrive(&c.da_full[b]);
+        }
+      }
     }
     if (ok && warp_wait(ctx, &c.acc_done, 0, abort)) {
       // Epilogue: thread rowi holds dimension d = rowi; group g the keys 32g .. 32g + 31.
