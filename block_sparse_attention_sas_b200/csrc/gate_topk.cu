@@ -178,172 +178,349 @@ gate_topk_warp_kernel(const float* __restrict__ scores, int total_rows, int rows
 }
 
 // ---------------------------------------------------------------------------
-// One CTA per row (long rows).
+// Long rows: a block per chunk of the row sorts the chunk, then a block per
+// row merges the chunks' candidates.
 // ---------------------------------------------------------------------------
-constexpr int kCtaThreads = 512;
-constexpr int kCtaWarps = kCtaThreads / 32;
+// A row's k largest scores are among the k largest of each chunk, so each
+// chunk passes on its top min(K, chunk) entries; the merge picks the row's k
+// from those. Entries are compared by a composite 64-bit key: the score's
+// order-preserving key above the complement of the block index. Larger
+// composites are higher scores and, among equal scores, lower indices, and
+// no two entries of a row share one, so a descending sort is the Top-K order
+// with its tie rule. The gate softmax combines the chunks' (max, sum of exp)
+// pairs. The chunk results travel through the row's own gates, which the
+// merge reads first and then overwrites with the final gates (no workspace).
+constexpr int kMaxChunk = 8192;       // longest chunk (64 KB of keys)
+constexpr int kMaxCandidates = 8192;  // chunks x per-chunk candidates
 
-__device__ __forceinline__ float block_reduce_max(float x, float* red) {
+__device__ __forceinline__ uint64_t ckey(float f, int i) {
+  return ((uint64_t)fkey(f) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)i);
+}
+__device__ __forceinline__ int ckey_index(uint64_t c) {
+  return (int)(0xFFFFFFFFu - (uint32_t)(c & 0xFFFFFFFFu));
+}
+
+// Block reductions for any multiple of 32 threads up to 1024 (red: 32 floats).
+__device__ __forceinline__ float block_max(float x, float* red) {
   x = warp_max(x);
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __syncthreads();
   if (lane == 0) red[w] = x;
   __syncthreads();
-  float y = (lane < kCtaWarps) ? red[lane] : -INFINITY;
-  return warp_max(y);
+  return warp_max(lane < (int)(blockDim.x >> 5) ? red[lane] : -INFINITY);
 }
-__device__ __forceinline__ float block_reduce_sum(float x, float* red) {
+__device__ __forceinline__ float block_sum(float x, float* red) {
   x = warp_sum(x);
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __syncthreads();
   if (lane == 0) red[w] = x;
   __syncthreads();
-  float y = (lane < kCtaWarps) ? red[lane] : 0.f;
-  return warp_sum(y);
+  return warp_sum(lane < (int)(blockDim.x >> 5) ? red[lane] : 0.f);
 }
-// Dynamic shared memory: the row's values when n <= cap (else they are
-// re-read from global memory, where the row stays L2-resident).
-__global__ void __launch_bounds__(kCtaThreads)
-gate_topk_cta_kernel(const float* __restrict__ scores, int rows, int C, int causal, int K,
-                     int cap, float* __restrict__ gates, int32_t* __restrict__ idx) {
-  extern __shared__ float s_dyn[];
-  __shared__ float red_f[kCtaWarps];
-  __shared__ int warp_cnt[kCtaWarps];
-  __shared__ uint32_t s_selkey[kMaxK];
-  __shared__ int32_t s_selidx[kMaxK];
-  __shared__ int s_whist[kCtaWarps][256];
-  __shared__ int s_hist[256];
-  __shared__ int s_pick[2];
 
+// Sorts the block's E * blockDim.x keys (a power of two) in descending
+// order with a bitonic network; thread t holds the keys at indices
+// e * blockDim.x + t in v[e]. Stages whose partners are less than 32 apart
+// exchange through warp shuffles (no barrier); the wider ones go through
+// sm (E * blockDim.x keys). On return the sorted keys are in sm.
+template <int E>
+__device__ void block_sort_desc(uint64_t (&v)[E], uint64_t* sm) {
+  const int bd = blockDim.x, tid = threadIdx.x, n = E * bd;
+  bool in_smem = false;
+  for (int k = 2; k <= n; k <<= 1)
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j >= 32) {
+        if (!in_smem) {
+          __syncthreads();  // every thread has read sm into registers
+#pragma unroll
+          for (int e = 0; e < E; ++e) sm[e * bd + tid] = v[e];
+          __syncthreads();
+          in_smem = true;
+        }
+        for (int i = tid; i < n; i += bd) {
+          const int p = i ^ j;
+          if (p > i) {
+            const uint64_t a = sm[i], b = sm[p];
+            if (((i & k) == 0) ? (a < b) : (a > b)) {
+              sm[i] = b;
+              sm[p] = a;
+            }
+          }
+        }
+        __syncthreads();
+      } else {
+        if (in_smem) {
+#pragma unroll
+          for (int e = 0; e < E; ++e) v[e] = sm[e * bd + tid];
+          in_smem = false;
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int i = e * bd + tid;
+          const uint64_t o = __shfl_xor_sync(0xffffffffu, v[e], j);
+          // the lower index of a pair keeps the larger key in a descending run
+          const bool keep_max = ((i & j) == 0) == ((i & k) == 0);
+          v[e] = keep_max ? (v[e] > o ? v[e] : o) : (v[e] < o ? v[e] : o);
+        }
+      }
+    }
+  if (!in_smem) {
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < E; ++e) sm[e * bd + tid] = v[e];
+  }
+  __syncthreads();
+}
+
+// Sorts one warp's 32 * EW keys in descending order in registers (lane l
+// holds indices e * 32 + l in w[e]); every lane of the warp calls it.
+template <int EW>
+__device__ __forceinline__ void warp_sort_desc(uint64_t (&w)[EW]) {
+  const int lane = threadIdx.x & 31;
+  constexpr int n = 32 * EW;
+#pragma unroll
+  for (int k = 2; k <= n; k <<= 1)
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j >= 32) {
+#pragma unroll
+        for (int e = 0; e < EW; ++e) {
+          const int pe = e ^ (j >> 5);
+          if (pe > e) {
+            const bool desc = ((e * 32 + lane) & k) == 0;
+            const uint64_t a = w[e], b = w[pe];
+            if (desc ? (a < b) : (a > b)) {
+              w[e] = b;
+              w[pe] = a;
+            }
+          }
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < EW; ++e) {
+          const int i = e * 32 + lane;
+          const uint64_t o = __shfl_xor_sync(0xffffffffu, w[e], j);
+          const bool keep_max = ((i & j) == 0) == ((i & k) == 0);
+          w[e] = keep_max ? (w[e] > o ? w[e] : o) : (w[e] < o ? w[e] : o);
+        }
+      }
+    }
+}
+
+template <int EW>
+__device__ __forceinline__ void warp_sort_cand(const uint64_t* cand, int m, uint64_t* out, int k) {
+  const int lane = threadIdx.x & 31;
+  uint64_t w[EW];
+#pragma unroll
+  for (int e = 0; e < EW; ++e) w[e] = e * 32 + lane < m ? cand[e * 32 + lane] : 0ull;
+  warp_sort_desc<EW>(w);
+#pragma unroll
+  for (int e = 0; e < EW; ++e)
+    if (e * 32 + lane < k) out[e * 32 + lane] = w[e];
+}
+
+constexpr int kBins = 4096;     // histogram over the top 12 bits of a key
+constexpr int kCandCap = 256;   // candidates sorted by one warp
+
+struct TopkScratch {
+  int hist[kBins];
+  uint64_t cand[kCandCap];
+  int warp_tot[32];
+  int ncand, bin, above;
+};
+// Static shared memory of the chunk and merge kernels (scratch + reduction),
+// counted against the 48 KB a launch gets without opting in.
+constexpr size_t kStaticSmem = sizeof(TopkScratch) + 32 * sizeof(float) + 64;
+
+// Leaves the k largest of the block's keys (v[e], E per thread; 0 = empty),
+// in descending order, in sm[0, k). Radix filter: a histogram over the top
+// 12 bits of the keys finds the bin b holding the k-th largest; every key in
+// a bin above b is in, and the rest come from bin b, so the keys in bins >= b
+// are the candidates. Up to 256 candidates are sorted by one warp; past that
+// (heavy ties) the block sorts all its keys. 1 <= k; every thread calls it.
+template <int E>
+__device__ void block_topk(uint64_t (&v)[E], int k, TopkScratch& ts, uint64_t* sm) {
+  const int tid = threadIdx.x, bd = blockDim.x, lane = tid & 31, w = tid >> 5;
+  for (int i = tid; i < kBins; i += bd) ts.hist[i] = 0;
+  if (tid == 0) {
+    ts.ncand = 0;
+    ts.bin = 0;  // always overwritten: the block holds at least k keys
+    ts.above = 0;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int e = 0; e < E; ++e)
+    if (v[e] != 0ull) atomicAdd(&ts.hist[(int)(v[e] >> 52)], 1);
+  __syncthreads();
+  // Suffix counts: thread t owns bins [t W, t W + W).
+  const int W = kBins / bd, b0 = tid * W;
+  int local = 0;
+  for (int x = 0; x < W; ++x) local += ts.hist[b0 + x];
+  int suf = local;  // over this warp's lanes >= lane
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_down_sync(0xffffffffu, suf, off);
+    if (lane + off < 32) suf += y;
+  }
+  if (lane == 0) ts.warp_tot[w] = suf;
+  __syncthreads();
+  int running = suf - local;
+  for (int x = w + 1; x < (bd >> 5); ++x) running += ts.warp_tot[x];
+  for (int x = W - 1; x >= 0; --x) {
+    const int h = ts.hist[b0 + x];
+    if (running < k && running + h >= k) {
+      ts.bin = b0 + x;
+      ts.above = running;
+    }
+    running += h;
+  }
+  __syncthreads();
+  const int b = ts.bin, m = ts.above + ts.hist[b];
+  if (m <= kCandCap) {
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+      if (v[e] != 0ull && (int)(v[e] >> 52) >= b) ts.cand[atomicAdd(&ts.ncand, 1)] = v[e];
+    __syncthreads();
+    if (w == 0) {
+      if (m <= 32) warp_sort_cand<1>(ts.cand, m, sm, k);
+      else if (m <= 64) warp_sort_cand<2>(ts.cand, m, sm, k);
+      else if (m <= 128) warp_sort_cand<4>(ts.cand, m, sm, k);
+      else warp_sort_cand<8>(ts.cand, m, sm, k);
+    }
+    __syncthreads();
+  } else {
+    block_sort_desc<E>(v, sm);
+  }
+}
+
+// Writes g = exp(s - lse) for i < n and 0 past n, over [0, C) of one row
+// (float4 accesses when both rows are 16-byte aligned).
+__device__ __forceinline__ void write_gates(const float* srow, float* grow, int C, int n, float lse) {
+  const int tid = threadIdx.x, bd = blockDim.x;
+  const bool vec = ((reinterpret_cast<uintptr_t>(srow) | reinterpret_cast<uintptr_t>(grow)) & 15) == 0;
+  int i0 = 0;
+  if (vec) {
+    const int C4 = C >> 2;
+    for (int q = tid; q < C4; q += bd) {
+      const float4 x = reinterpret_cast<const float4*>(srow)[q];
+      const int i = q * 4;
+      float4 g;
+      g.x = i < n ? expf(x.x - lse) : 0.f;
+      g.y = i + 1 < n ? expf(x.y - lse) : 0.f;
+      g.z = i + 2 < n ? expf(x.z - lse) : 0.f;
+      g.w = i + 3 < n ? expf(x.w - lse) : 0.f;
+      reinterpret_cast<float4*>(grow)[q] = g;
+    }
+    i0 = C4 * 4;
+  }
+  for (int i = i0 + tid; i < C; i += bd) grow[i] = i < n ? expf(srow[i] - lse) : 0.f;
+}
+
+// One block per (row, chunk of Lc = E * blockDim.x entries). FINAL (the row
+// is one chunk): writes the row's idx and gates. Otherwise writes the
+// chunk's max and sum of exp to gates[2c], gates[2c + 1] of its row, and its
+// kc best composites, as pairs of 32-bit words, after the 2 * chunks floats
+// of those pairs.
+template <bool FINAL, int E>
+__global__ void __launch_bounds__(1024)
+gate_topk_chunk_kernel(const float* __restrict__ scores, int rows, int C, int causal, int K,
+                       int chunks, int kc, float* __restrict__ gates, int32_t* __restrict__ idx) {
+  extern __shared__ uint64_t s_key[];  // E * blockDim.x keys
+  __shared__ float red[32];
+  __shared__ TopkScratch ts;
+  const int tid = threadIdx.x, bd = blockDim.x, Lc = E * bd;
+  const long long row = blockIdx.x / chunks;
+  const int c = (int)(blockIdx.x % chunks);
+  const int r = (int)(row % rows);
+  const int n = causal ? min(r, C) : C;
+  const int lo = c * Lc, len = max(0, min(n - lo, Lc));
+  const float* srow = scores + row * (long long)C;
+
+  uint64_t v[E];
+  float f[E];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = e * bd + tid;
+    const bool ok = i < len;
+    f[e] = ok ? srow[lo + i] : -INFINITY;
+    v[e] = ok ? ckey(f[e], lo + i) : 0ull;  // 0 is below every entry's composite
+    mx = fmaxf(mx, f[e]);
+  }
+  mx = block_max(mx, red);
+  float sum = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e)
+    if (e * bd + tid < len) sum += expf(f[e] - mx);
+  sum = block_sum(sum, red);
+  // The chunk's best min(K or kc, len) keys, sorted, in s_key.
+  const int kk = min(FINAL ? K : kc, len);
+  if (kk > 0) block_topk<E>(v, kk, ts, s_key);
+
+  float* grow = gates + row * (long long)C;
+  if (FINAL) {
+    int32_t* out = idx + row * (long long)K;
+    for (int p = tid; p < K; p += bd) out[p] = p < kk ? ckey_index(s_key[p]) : -1;
+    write_gates(srow, grow, C, n, mx + logf(sum));
+  } else {
+    if (tid == 0) {
+      grow[2 * c] = mx;
+      grow[2 * c + 1] = sum;
+    }
+    uint32_t* cand = reinterpret_cast<uint32_t*>(grow + 2 * chunks) + 2LL * c * kc;
+    for (int p = tid; p < kc; p += bd) {
+      const uint64_t key = p < kk ? s_key[p] : 0ull;
+      cand[2 * p] = (uint32_t)(key & 0xFFFFFFFFu);
+      cand[2 * p + 1] = (uint32_t)(key >> 32);
+    }
+  }
+}
+
+// One block per row: combines the chunks' softmax partials into the row's
+// LSE, sorts the chunks' candidates (E * blockDim.x >= chunks * kc keys), and
+// writes the row's idx and gates.
+template <int E>
+__global__ void __launch_bounds__(1024)
+gate_topk_merge_kernel(const float* __restrict__ scores, int rows, int C, int causal, int K,
+                       int chunks, int kc, float* __restrict__ gates, int32_t* __restrict__ idx) {
+  extern __shared__ uint64_t s_key[];  // E * blockDim.x keys
+  __shared__ float red[32];
+  __shared__ TopkScratch ts;
   const long long row = blockIdx.x;
   const int r = (int)(row % rows);
   const int n = causal ? min(r, C) : C;
-  const float* s = scores + row * (long long)C;
-  float* g = gates + row * (long long)C;
-  int32_t* out = idx + row * (long long)K;
-  const bool in_smem = n <= cap;
-  const float* v = in_smem ? s_dyn : s;
-  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  float* grow = gates + row * (long long)C;
+  const uint32_t* cand = reinterpret_cast<const uint32_t*>(grow + 2 * chunks);
+  const int tid = threadIdx.x, bd = blockDim.x, nc = chunks * kc;
 
-  float mx = -INFINITY;
-  for (int i = tid; i < n; i += kCtaThreads) {
-    const float f = s[i];
-    if (in_smem) s_dyn[i] = f;
-    mx = fmaxf(mx, f);
-  }
-  mx = block_reduce_max(mx, red_f);  // includes a __syncthreads after the smem fill
-  float sum = 0.f;
-  for (int i = tid; i < n; i += kCtaThreads) sum += expf(v[i] - mx);
-  sum = block_reduce_sum(sum, red_f);
-  const float lse = mx + logf(sum);
-  for (int i = tid; i < C; i += kCtaThreads) g[i] = (i < n) ? expf(v[i] - lse) : 0.f;
-
-  const int k = min(K, n);
-  if (k > 0) {
-    // Radix select over four 8-bit digits: per-warp histograms, summed into
-    // one, and warp 0 picks the digit.
-    uint32_t tau = 0, mask = 0;
-    int krem = k;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = tid; i < kCtaWarps * 256; i += kCtaThreads) (&s_whist[0][0])[i] = 0;
-      __syncthreads();
-      for (int base = 0; base < n; base += kCtaThreads) {
-        const int i = base + tid;
-        const uint32_t key = (i < n) ? fkey(v[i]) : 0u;
-        warp_hist_add(s_whist[w], (key >> shift) & 255u, i < n && (key & mask) == tau);
-      }
-      __syncthreads();
-      for (int bin = tid; bin < 256; bin += kCtaThreads) {
-        int t = 0;
+  uint64_t v[E];
 #pragma unroll
-        for (int x = 0; x < kCtaWarps; ++x) t += s_whist[x][bin];
-        s_hist[bin] = t;
-      }
-      __syncthreads();
-      if (w == 0) {
-        int above;
-        const uint32_t dig = warp_pick_digit(s_hist, krem, above);
-        if (lane == 0) {
-          s_pick[0] = (int)dig;
-          s_pick[1] = above;
-        }
-      }
-      __syncthreads();
-      krem -= s_pick[1];
-      tau |= (uint32_t)s_pick[0] << shift;
-      mask |= 255u << shift;
-    }
-    const int need_eq = krem;
-
-    // Each warp owns a contiguous, 32-aligned range of the row. Pass 1
-    // counts its keys equal to tau; an exclusive scan over warps gives each
-    // warp the number of equal keys before its range.
-    const int chunk = ((n + kCtaWarps - 1) / kCtaWarps + 31) & ~31;
-    const int lo = min(n, w * chunk), hi = min(n, lo + chunk);
-    const uint32_t lt = lanemask_lt();
-    int eq_here = 0;
-    for (int i = lo + lane; i < hi; i += 32) eq_here += fkey(v[i]) == tau;
-    eq_here = __reduce_add_sync(0xffffffffu, eq_here);
-    __syncthreads();
-    if (lane == 0) warp_cnt[w] = eq_here;
-    __syncthreads();
-    int eq_before = 0;
-    for (int x = 0; x < w; ++x) eq_before += warp_cnt[x];
-    // Pass 2: survivors per warp (no writes), then scan for output offsets.
-    int sel_here = 0;
-    {
-      int run_eq = eq_before;
-      for (int base = lo; base < hi; base += 32) {
-        const int i = base + lane;
-        const uint32_t key = (i < hi) ? fkey(v[i]) : 0u;
-        const bool is_gt = (i < hi) && key > tau;
-        const bool is_eq = (i < hi) && key == tau;
-        const uint32_t eqm = __ballot_sync(0xffffffffu, is_eq);
-        const bool sel = is_gt || (is_eq && run_eq + __popc(eqm & lt) < need_eq);
-        sel_here += __popc(__ballot_sync(0xffffffffu, sel));
-        run_eq += __popc(eqm);
-      }
-    }
-    __syncthreads();
-    if (lane == 0) warp_cnt[w] = sel_here;
-    __syncthreads();
-    int sel_before = 0;
-    for (int x = 0; x < w; ++x) sel_before += warp_cnt[x];
-    // Pass 3: write survivors in index order.
-    {
-      int run_eq = eq_before, run_sel = sel_before;
-      for (int base = lo; base < hi; base += 32) {
-        const int i = base + lane;
-        const uint32_t key = (i < hi) ? fkey(v[i]) : 0u;
-        const bool is_gt = (i < hi) && key > tau;
-        const bool is_eq = (i < hi) && key == tau;
-        const uint32_t eqm = __ballot_sync(0xffffffffu, is_eq);
-        const bool sel = is_gt || (is_eq && run_eq + __popc(eqm & lt) < need_eq);
-        const uint32_t selm = __ballot_sync(0xffffffffu, sel);
-        if (sel) {
-          const int p = run_sel + __popc(selm & lt);
-          s_selkey[p] = key;
-          s_selidx[p] = i;
-        }
-        run_eq += __popc(eqm);
-        run_sel += __popc(selm);
-      }
-    }
-    __syncthreads();
-    for (int p = tid; p < k; p += kCtaThreads) {
-      const uint32_t kp = s_selkey[p];
-      int rank = 0;
-      for (int q = 0; q < k; ++q) {
-        const uint32_t kq = s_selkey[q];
-        rank += (kq > kp) || (kq == kp && q < p);
-      }
-      out[rank] = s_selidx[p];
-    }
+  for (int e = 0; e < E; ++e) {
+    const int i = e * bd + tid;
+    v[e] = i < nc ? (((uint64_t)cand[2 * i + 1] << 32) | cand[2 * i]) : 0ull;
   }
-  for (int p = k + tid; p < K; p += kCtaThreads) out[p] = -1;
+  float m = -INFINITY;
+  for (int c = tid; c < chunks; c += bd) m = fmaxf(m, grow[2 * c]);
+  m = block_max(m, red);
+  float acc = 0.f;
+  for (int c = tid; c < chunks; c += bd) {
+    const float sc = grow[2 * c + 1];
+    if (sc > 0.f) acc += sc * expf(grow[2 * c] - m);  // empty chunks hold (-inf, 0)
+  }
+  acc = block_sum(acc, red);  // its barriers also order every scratch read before the writes below
+  const float lse = m + logf(acc);
+  const int k = min(K, n);
+  if (k > 0) block_topk<E>(v, k, ts, s_key);
+  int32_t* out = idx + row * (long long)K;
+  for (int p = tid; p < K; p += bd) out[p] = p < k ? ckey_index(s_key[p]) : -1;
+  write_gates(scores + row * (long long)C, grow, C, n, lse);
 }
 
-constexpr int kCtaSmemCap = 48 * 1024;  // floats kept in shared memory (192 KB)
+int pow2_at_least(int x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
 
 }  // namespace
 
@@ -357,15 +534,68 @@ cudaError_t launch_gate_topk(const float* scores, int B, int Hkv, int rows, int 
     gate_topk_warp_kernel<<<(unsigned)grid, 32 * kWarpRowsPerCta, 0, stream>>>(
         scores, (int)total, rows, C, causal, K, gates, idx);
     note_launches(1);
-  } else {
-    const int cap = min(maxlen, kCtaSmemCap);
-    const size_t smem = (size_t)cap * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(gate_topk_cta_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    gate_topk_cta_kernel<<<(unsigned)total, kCtaThreads, smem, stream>>>(scores, rows, C, causal,
-                                                                          K, cap, gates, idx);
+  } else if (C <= 2048) {
+    // One block per row sorts the whole row.
+    const int Lp = pow2_at_least(C), threads = min(1024, Lp);
+    const size_t smem = (size_t)Lp * sizeof(uint64_t);
+    if (Lp / threads == 1)
+      gate_topk_chunk_kernel<true, 1><<<(unsigned)total, threads, smem, stream>>>(
+          scores, rows, C, causal, K, 1, min(K, Lp), gates, idx);
+    else
+      gate_topk_chunk_kernel<true, 2><<<(unsigned)total, threads, smem, stream>>>(
+          scores, rows, C, causal, K, 1, min(K, Lp), gates, idx);
     note_launches(1);
+  } else {
+    // The shortest chunk (a power of two from 512) whose candidates fit the
+    // merge (chunks * kc <= 8192) and whose partials fit the row's gates
+    // (chunks * (2 + 2 kc) floats <= C). 8192 always qualifies for
+    // 2048 < C <= 262144.
+    int Lc = 512, chunks = 0, kc = 0;
+    for (;; Lc <<= 1) {
+      chunks = (C + Lc - 1) / Lc;
+      kc = min(K, Lc);
+      if (Lc == kMaxChunk ||
+          ((long long)chunks * kc <= kMaxCandidates && (long long)chunks * (2 + 2 * kc) <= C))
+        break;
+    }
+    if ((long long)chunks * kc > kMaxCandidates || (long long)chunks * (2 + 2 * kc) > C)
+      return cudaErrorInvalidValue;  // beyond the documented C limit
+    const int threads = min(1024, Lc), E = Lc / threads;
+    cudaError_t e = cudaSuccess;
+    const size_t smem = (size_t)Lc * sizeof(uint64_t);
+    const unsigned grid = (unsigned)(total * chunks);
+    auto chunk = [&](auto kern) {
+      if (smem + kStaticSmem > 48 * 1024)
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess)
+        kern<<<grid, threads, smem, stream>>>(scores, rows, C, causal, K, chunks, kc, gates, idx);
+    };
+    switch (E) {
+      case 1: chunk(gate_topk_chunk_kernel<false, 1>); break;
+      case 2: chunk(gate_topk_chunk_kernel<false, 2>); break;
+      case 4: chunk(gate_topk_chunk_kernel<false, 4>); break;
+      default: chunk(gate_topk_chunk_kernel<false, 8>); break;
+    }
+    note_launches(1);
+    if (e != cudaSuccess || (e = cudaGetLastError()) != cudaSuccess) return e;
+    const int Mp = pow2_at_least(chunks * kc);
+    const int mthreads = min(1024, max(256, Mp)), ME = max(1, Mp / mthreads);
+    const size_t msmem = (size_t)ME * mthreads * sizeof(uint64_t);
+    auto merge = [&](auto kern) {
+      if (msmem + kStaticSmem > 48 * 1024)
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
+      if (e == cudaSuccess)
+        kern<<<(unsigned)total, mthreads, msmem, stream>>>(scores, rows, C, causal, K, chunks, kc,
+                                                           gates, idx);
+    };
+    switch (ME) {
+      case 1: merge(gate_topk_merge_kernel<1>); break;
+      case 2: merge(gate_topk_merge_kernel<2>); break;
+      case 4: merge(gate_topk_merge_kernel<4>); break;
+      default: merge(gate_topk_merge_kernel<8>); break;
+    }
+    note_launches(1);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }
