@@ -16,10 +16,12 @@
 //   warp 1  MMA issuer: S(n+1) is issued before PV(n) so the softmax of block
 //           n overlaps the next QK^T
 //   warp 0  softmax, one thread per query row (TMEM lane): masks keys past
-//           the cache length, running max, P as bf16 back into the S columns
-//           of TMEM (the A operand of PV), then acc = acc * alpha + O_n in
-//           registers, so the online softmax needs no rescale of TMEM
-// TMEM: S[2] at columns 0 / 64, O_n at 128 (256 columns, so two CTAs share an
+//           the cache length, P as bf16 back into the S columns of TMEM (the
+//           A operand of PV). O accumulates in TMEM over the blocks against a
+//           per-row reference max: P = 2^(s * scale + bias - m_ref) stays
+//           below 2^8 and O is rescaled in TMEM only when a row max rises
+//           past that, so the softmax of block n + 1 never waits for PV(n)
+// TMEM: S[2] at columns 0 / 64, O at 128 (256 columns, so two CTAs share an
 // SM). Cache rows past L lie outside the tensor map and are read as zeros.
 // Partial (max, sum, o) of each split go to the workspace; the last CTA of a
 // (batch, KV head), found with an atomic ticket, merges them by log-sum-exp.
@@ -51,7 +53,7 @@ constexpr uint32_t kOffCtl = kOffKV + 2 * 32768;
 constexpr uint32_t kColS = 0, kColO = 128;
 
 struct Ctl {
-  uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], p_full[2], o_full, drain;
+  uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], p_full[2], o_full, o_final, drain;
   uint32_t tmem_base;
   int abort, nblk;
   int blocks[kMaxSlotsPerSplit];
@@ -93,6 +95,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         mbar_init(&c.p_full[i], 1);
       }
       mbar_init(&c.o_full, 1);
+      mbar_init(&c.o_final, 1);
       mbar_init(&c.drain, 1);
       fence_mbar_init();
       c.abort = 0;
@@ -198,15 +201,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (n + 1 < nblk && !issue_s(n + 1)) break;
         if (!wait_or_abort(ctx, &c.p_full[st], (n >> 1) & 1, abort)) break;
         fence_after_sync();
-        // O_n = P(n) V(n): P in S[n & 1] columns 0..31 (two bf16 per column).
+        // O += P(n) V(n): P in S[n & 1] columns 0..31 (two bf16 per column);
+        // block 0 starts O.
         const uint64_t vd = dv0 + ((st * 32768) >> 4);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
           mma_bf16_ts(tmem + kColO, tmem + kColS + st * 64 + ks * 8, vd + ((ks * 2048) >> 4), id_o,
-                      ks > 0);
+                      n > 0 || ks > 0);
         mma_commit(&c.o_full);
         mma_commit(&c.kv_empty[st]);
       }
+      mma_commit(&c.o_final);  // O complete: every PV issued above is done
       if (*abort) {
         mma_commit(&c.drain);
         (void)mbar_wait(ctx, &c.drain, 0);
@@ -214,10 +219,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
   } else if (warp == kSoftmaxWarp) {
     // Thread `lane` owns query row `lane` of the tile (head lane < G).
+    constexpr float kLazy = 8.f;  // log2 headroom of P over the reference max
     const float sc = s.scale * kLog2e;
     const uint32_t tl = tmem;  // lanes 0..31
-#pragma unroll
-    for (int i = 0; i < kD; ++i) acc[i] = 0.f;
     for (int n = 0; n < nblk; ++n) {
       const int st = n & 1;
       if (!warp_wait(ctx, &c.s_full[st], (n >> 1) & 1, abort)) {
@@ -228,9 +232,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const int m = c.blocks[n];
       const float bias = c.bias[n];
       const int kvalid = min(kB, s.L - m * kB);
-      // Two passes over the two 32-column halves of S (to keep registers for
-      // acc): the row max first, then p = 2^(s*scale + bias - max) as bf16
-      // into the S columns already read (P(n) takes columns 0..31).
+      // Two passes over the two 32-column halves of S: the row max first,
+      // then p = 2^(s*scale + bias - m_ref) as bf16 into the S columns
+      // already read (P(n) takes columns 0..31).
       float smax = -INFINITY;
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
@@ -250,9 +254,37 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         smax = fmax3(smax, m0, m1);
       }
       const float mx = (smax == -INFINITY) ? -INFINITY : fmaf(smax, sc, bias);
-      const float m_new = fmaxf(m_run, mx);
-      const float alpha = (m_run == -INFINITY) ? 0.f : ex2(m_run - m_new);
-      const float off = (m_new == -INFINITY) ? -INFINITY : bias - m_new;
+      // Reference update: the first finite max sets it (nothing accumulated
+      // for the row yet); a max more than kLazy above it rescales O.
+      const bool need = lane < G && m_run != -INFINITY && mx > m_run + kLazy;
+      if (m_run == -INFINITY) m_run = mx;
+      if (__any_sync(0xffffffffu, need)) {
+        // O must hold every PV issued so far. Seeing S(n) complete already
+        // implies PV(n - 2) completed, so waiting for the parity of PV(n - 1)
+        // is unambiguous.
+        if (n >= 1 && !warp_wait(ctx, &c.o_full, (n - 1) & 1, abort)) {
+          ok_sm = false;
+          break;
+        }
+        fence_after_sync();
+        const float alpha = need ? ex2(m_run - mx) : 1.f;
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t ov[32], lo16[16], hi16[16];
+          tmem_ld32(tl + kColO + ch * 32, ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            lo16[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            hi16[i] = __float_as_uint(__uint_as_float(ov[16 + i]) * alpha);
+          }
+          tmem_st16(tl + kColO + ch * 32, lo16);
+          tmem_st16(tl + kColO + ch * 32 + 16, hi16);
+        }
+        l_run *= alpha;
+        if (need) m_run = mx;
+      }
+      const float off = (m_run == -INFINITY) ? -INFINITY : bias - m_run;
       const uint64_t sc2 = f2u(sc, sc), off2 = f2u(off, off);
       uint64_t accp = 0;
 #pragma unroll
@@ -275,31 +307,27 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         tmem_st16(tl + kColS + st * 64 + hf * 16, pk);
       }
-      l_run = l_run * alpha + (lo_f(accp) + hi_f(accp));
-      m_run = m_new;
-      // P(n) over the S columns just read; O_{n-1} was read in the previous
-      // iteration, so PV(n) may overwrite it once P(n) is announced.
+      l_run += lo_f(accp) + hi_f(accp);
+      // P(n) (and a rescaled O) in TMEM before PV(n) is issued.
       tmem_st_wait();
       fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&c.p_full[st]);
-      if (!warp_wait(ctx, &c.o_full, n & 1, abort)) {
+    }
+#pragma unroll
+    for (int i = 0; i < kD; ++i) acc[i] = 0.f;
+    if (ok_sm && nblk > 0) {
+      if (!warp_wait(ctx, &c.o_final, 0, abort)) {
         ok_sm = false;
-        break;
-      }
-      fence_after_sync();
-      const uint64_t al2 = f2u(alpha, alpha);
+      } else {
+        fence_after_sync();
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t ov[32];
-        tmem_ld32(tl + kColO + ch * 32, ov);
-        tmem_ld_wait();
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t ov[32];
+          tmem_ld32(tl + kColO + ch * 32, ov);
+          tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const uint64_t a = ffma2(f2u(acc[ch * 32 + i], acc[ch * 32 + i + 1]), al2,
-                                   f2u(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1])));
-          acc[ch * 32 + i] = lo_f(a);
-          acc[ch * 32 + i + 1] = hi_f(a);
+          for (int i = 0; i < 32; ++i) acc[ch * 32 + i] = __uint_as_float(ov[i]);
         }
       }
     }
