@@ -434,6 +434,22 @@ cudaError_t make_tmap_bf16_2planes(void* map_out, const void* ptr, int rows, int
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// Map over a [rows][128] bf16 matrix (one plane) with 64 x 8 x 1 boxes: eight
+// rows of one k-half, 128-byte swizzle (the query rows of a decode unit).
+cudaError_t make_tmap_bf16_rows8(void* map_out, const void* ptr, int rows) {
+  CUtensorMap* map = static_cast<CUtensorMap*>(map_out);
+  EncodeTiled enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)rows, 1};
+  const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)rows * kD * 2};
+  const cuuint32_t box[3] = {64, 8, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 // Same, with planes `pitch_rows` rows apart of which the first `rows` are in
 // the map (a KV cache of capacity pitch_rows filled up to rows).
 cudaError_t make_tmap_bf16_pitched(void* map_out, const void* ptr, int rows, int pitch_rows,

@@ -5,14 +5,15 @@
 // kept at inference), and the dense decode (every block) used as comparison.
 //
 // The G query rows of a (batch, KV head) form the A operand of a 128-row MMA
-// tile (rows past G hold whatever the Q box brought in and are never read),
+// tile: an 8-row Q box (2 KB) read with a zero stride between 8-row groups,
+// so all 16 row groups see the same rows (rows past G are never read),
 // so each 64-key K/V block costs one S = Q K^T (8 MMAs, N = 64) and one
 // O_n = P V (4 MMAs, N = 128): the CUDA cores only run the softmax of G rows,
 // and the kernel streams the cache at HBM speed instead of FMA speed.
 //
 // One CTA per (split, KV head, batch); a split is a run of block slots.
 //   warp 2  list of the split's blocks, TMA producer: Q once, then K and V of
-//           each block into a two-stage ring (32 KB a stage)
+//           each block into a three-stage ring (32 KB a stage)
 //   warp 1  MMA issuer: S(n+1) is issued before PV(n) so the softmax of block
 //           n overlaps the next QK^T
 //   warp 0  softmax, one thread per query row (TMEM lane): masks keys past
@@ -47,13 +48,15 @@ constexpr int kMaxG = 8;
 constexpr int kMaxSlotsPerSplit = 512;
 
 // Shared memory (offsets from a 1024-byte aligned base).
-constexpr uint32_t kOffQ = 0;           // [k half][128 rows][128 B]; rows 0..63 loaded
-constexpr uint32_t kOffKV = 32768;      // 2 stages x (K halves 16 KB, V halves 16 KB)
-constexpr uint32_t kOffCtl = kOffKV + 2 * 32768;
+constexpr int kStages = 3;
+constexpr uint32_t kOffQ = 0;           // [k half][8 rows][128 B]
+constexpr uint32_t kOffKV = 2048;       // stages x (K halves 16 KB, V halves 16 KB)
+constexpr uint32_t kOffCtl = kOffKV + kStages * 32768;
 constexpr uint32_t kColS = 0, kColO = 128;
 
 struct Ctl {
-  uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], p_full[2], o_full, o_final, drain;
+  uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[2], p_full[2], o_full, o_final,
+      drain;
   uint32_t tmem_base;
   int abort, nblk;
   int blocks[kMaxSlotsPerSplit];
@@ -88,9 +91,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   if (warp == kProducerWarp) {
     if (lane == 0) {
       mbar_init(&c.q_full, 1);
-      for (int i = 0; i < 2; ++i) {
+      for (int i = 0; i < kStages; ++i) {
         mbar_init(&c.kv_full[i], 1);
         mbar_init(&c.kv_empty[i], 1);
+      }
+      for (int i = 0; i < 2; ++i) {
         mbar_init(&c.s_full[i], 1);
         mbar_init(&c.p_full[i], 1);
       }
@@ -101,9 +106,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       c.abort = 0;
       c.last = 0;
       tma_prefetch_desc(&tm_q);
-      mbar_arrive_expect_tx(&c.q_full, 2 * 8192);
+      mbar_arrive_expect_tx(&c.q_full, 2 * 1024);
       for (int kb = 0; kb < 2; ++kb)
-        tma_load_3d(base + kOffQ + kb * 16384, &tm_q, kb * 64, (int)hbase, 0, &c.q_full);
+        tma_load_3d(base + kOffQ + kb * 1024, &tm_q, kb * 64, (int)hbase, 0, &c.q_full);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
     }
@@ -157,8 +162,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (lane == 0) {
       int issued = 0;
       for (int n = 0; n < nblk; ++n) {
-        const int st = n & 1;
-        if (n >= 2 && !wait_or_abort(ctx, &c.kv_empty[st], ((n - 2) >> 1) & 1, abort)) break;
+        const int st = n % kStages;
+        if (n >= kStages &&
+            !wait_or_abort(ctx, &c.kv_empty[st], ((n - kStages) / kStages) & 1, abort))
+          break;
         const int m = c.blocks[n];
         unsigned char* kv = base + kOffKV + st * 32768;
         mbar_arrive_expect_tx(&c.kv_full[st], 32768);
@@ -171,42 +178,42 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       // The Q copy lands before the CTA leaves, even when the split is empty.
       (void)mbar_wait(ctx, &c.q_full, 0);
       if (*abort)
-        for (int n = max(0, issued - 2); n < issued; ++n)
-          (void)mbar_wait(ctx, &c.kv_full[n & 1], (n >> 1) & 1);
+        for (int n = max(0, issued - kStages); n < issued; ++n)
+          (void)mbar_wait(ctx, &c.kv_full[n % kStages], (n / kStages) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0 && nblk > 0) {
       const uint32_t id_s = idesc_bf16(128, 64, false, false);
       const uint32_t id_o = idesc_bf16(128, 128, false, true);
-      const uint64_t dq0 = sdesc_sw128(sbase + kOffQ, 16, 1024);
+      const uint64_t dq0 = sdesc_sw128(sbase + kOffQ, 16, 0);  // 8 rows, repeated
       const uint64_t dk0 = sdesc_sw128(sbase + kOffKV, 16, 1024);     // K, K-major
       const uint64_t dv0 = sdesc_sw128(sbase + kOffKV + 16384, 8192, 1024);  // V, MN-major
       auto issue_s = [&](int n) -> bool {
-        const int st = n & 1;
-        if (!wait_or_abort(ctx, &c.kv_full[st], (n >> 1) & 1, abort)) return false;
+        const int st = n % kStages, sb = n & 1;
+        if (!wait_or_abort(ctx, &c.kv_full[st], (n / kStages) & 1, abort)) return false;
         fence_after_sync();
         const uint64_t kd = dk0 + ((st * 32768) >> 4);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t off = ((ks >> 2) * 8192 + (ks & 3) * 32) >> 4;
-          mma_bf16_ss(tmem + kColS + st * 64, dq0 + ((((ks >> 2) * 16384 + (ks & 3) * 32)) >> 4),
+          mma_bf16_ss(tmem + kColS + sb * 64, dq0 + ((((ks >> 2) * 1024 + (ks & 3) * 32)) >> 4),
                       kd + off, id_s, ks > 0);
         }
-        mma_commit(&c.s_full[st]);
+        mma_commit(&c.s_full[sb]);
         return true;
       };
       bool ok = wait_or_abort(ctx, &c.q_full, 0, abort) && issue_s(0);
       for (int n = 0; ok && n < nblk; ++n) {
-        const int st = n & 1;
+        const int st = n % kStages, sb = n & 1;
         if (n + 1 < nblk && !issue_s(n + 1)) break;
-        if (!wait_or_abort(ctx, &c.p_full[st], (n >> 1) & 1, abort)) break;
+        if (!wait_or_abort(ctx, &c.p_full[sb], (n >> 1) & 1, abort)) break;
         fence_after_sync();
         // O += P(n) V(n): P in S[n & 1] columns 0..31 (two bf16 per column);
         // block 0 starts O.
         const uint64_t vd = dv0 + ((st * 32768) >> 4);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_bf16_ts(tmem + kColO, tmem + kColS + st * 64 + ks * 8, vd + ((ks * 2048) >> 4), id_o,
+          mma_bf16_ts(tmem + kColO, tmem + kColS + sb * 64 + ks * 8, vd + ((ks * 2048) >> 4), id_o,
                       n > 0 || ks > 0);
         mma_commit(&c.o_full);
         mma_commit(&c.kv_empty[st]);
@@ -444,7 +451,7 @@ cudaError_t launch_decode_tc(const DecodeShape& s, const void* q, const void* kc
   cudaError_t e;
   // q as [B*Hq rows][128]; the cache as [B*Hkv planes][L rows][128] with a
   // plane pitch of Lcap rows, so rows past L read as zeros.
-  if ((e = make_tmap_bf16(&tq, q, s.B * s.Hq, 1)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_rows8(&tq, q, s.B * s.Hq)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16_pitched(&tk, kc, s.L, s.Lcap, s.B * s.Hkv)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16_pitched(&tv, vc, s.L, s.Lcap, s.B * s.Hkv)) != cudaSuccess) return e;
   char* w = static_cast<char*>(ws);

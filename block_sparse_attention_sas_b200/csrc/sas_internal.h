@@ -89,6 +89,7 @@ cudaError_t launch_decode_tc(const DecodeShape& s, const void* q, const void* kc
 // The same map with 64 x 64 x 2 boxes (two consecutive planes per box).
 cudaError_t make_tmap_bf16_2planes(void* map, const void* ptr, int rows, int planes);
 // 3-D TMA map over planes of `pitch_rows` rows, the first `rows` of each mapped.
+cudaError_t make_tmap_bf16_rows8(void* map_out, const void* ptr, int rows);
 cudaError_t make_tmap_bf16_pitched(void* map, const void* ptr, int rows, int pitch_rows,
                                    int planes);
 // Fixed-size device scratch for sas_decode_noalloc (no allocation involved).
