@@ -288,6 +288,50 @@ csr_kernel(const int32_t* __restrict__ idx, AttnShape s, int32_t* __restrict__ o
   }
 }
 
+// The same reverse index for N <= 1024 from a bitmap in shared memory: bit
+// (m, j) is set when query block j selects key block m (rows of idx are
+// distinct, so once at most). The entry e = j K + slot goes to position
+// off[m] + (set bits of row m below j): the list of m in ascending j, the
+// order the kernel above produces, with no ordered scan.
+constexpr int kCsrBitmapMaxN = 1024;
+__global__ void __launch_bounds__(1024)
+csr_bitmap_kernel(const int32_t* __restrict__ idx, AttnShape s, int32_t* __restrict__ off_all,
+                  int32_t* __restrict__ list_all) {
+  extern __shared__ uint32_t bm[];  // [N][W] bit rows, then N counts
+  __shared__ int32_t warp_tot[33];
+  const int W = (s.N + 31) >> 5;
+  int32_t* cnt = reinterpret_cast<int32_t*>(bm + (size_t)s.N * W);
+  const int bh = blockIdx.x, tid = threadIdx.x, bd = blockDim.x;
+  const int32_t* ix = idx + (long long)bh * s.N * s.K;
+  int32_t* off = off_all + (long long)bh * (s.N + 1);
+  int32_t* list = list_all + (long long)bh * s.N * s.K;
+  const int total = s.N * s.K;
+  for (int i = tid; i < s.N * W; i += bd) bm[i] = 0u;
+  for (int m = tid; m < s.N; m += bd) cnt[m] = 0;
+  __syncthreads();
+  for (int e = tid; e < total; e += bd) {
+    const int m = __ldg(ix + e), j = e / s.K;
+    if (m >= 0 && m < j) {
+      atomicOr(&bm[m * W + (j >> 5)], 1u << (j & 31));
+      atomicAdd(&cnt[m], 1);
+    }
+  }
+  __syncthreads();
+  const int n_all = block_exclusive_scan(cnt, s.N, warp_tot);
+  __syncthreads();
+  for (int m = tid; m < s.N; m += bd) off[m] = cnt[m];
+  if (tid == 0) off[s.N] = n_all;
+  for (int e = tid; e < total; e += bd) {
+    const int m = __ldg(ix + e), j = e / s.K;
+    if (m >= 0 && m < j) {
+      const uint32_t* row = bm + m * W;
+      int r = __popc(row[j >> 5] & ((1u << (j & 31)) - 1u));
+      for (int x = 0; x < (j >> 5); ++x) r += __popc(row[x]);
+      list[cnt[m] + r] = e;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Backward: dq and da (one CTA per query block row chunk and q head)
 // ---------------------------------------------------------------------------
@@ -627,12 +671,7 @@ cudaError_t bwd_t(const AttnShape& s, const void* q, const void* k, const void* 
   int32_t* clist = reinterpret_cast<int32_t*>(w + L.off_csr_list);
   cudaError_t e;
   if (!s.dense) {
-    const size_t smem = sizeof(int32_t) * ((size_t)s.N + kCsrChunk);
-    e = cudaFuncSetAttribute(csr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    csr_kernel<<<s.B * s.Hkv, kThreads, smem, st>>>(idx, s, coff, clist, ctx);
-    note_launches(1);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_bwd_csr(s, idx, coff, clist, ctx, st)) != cudaSuccess) return e;
   }
   {
     const size_t smem = dq_smem(D, BS);
@@ -699,6 +738,16 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 cudaError_t launch_bwd_csr(const AttnShape& s, const int32_t* idx, int32_t* off, int32_t* list,
                            const DevCtx& ctx, cudaStream_t st) {
+  if (s.N <= kCsrBitmapMaxN) {
+    const size_t W = ((size_t)s.N + 31) / 32;
+    const size_t smem = sizeof(uint32_t) * ((size_t)s.N * W + s.N);
+    cudaError_t e = cudaFuncSetAttribute(csr_bitmap_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    csr_bitmap_kernel<<<s.B * s.Hkv, 1024, smem, st>>>(idx, s, off, list);
+    note_launches(1);
+    return cudaGetLastError();
+  }
   const size_t smem = sizeof(int32_t) * ((size_t)s.N + kCsrChunk);
   cudaError_t e =
       cudaFuncSetAttribute(csr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

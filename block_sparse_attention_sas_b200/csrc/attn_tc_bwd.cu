@@ -43,21 +43,23 @@ constexpr int kMaxList = 257;
 // ============================================================================
 // One CTA per (query block j, 128-row tile of two heads, KV head, batch),
 // two CTAs per SM (256 TMEM columns, 97 KB of shared memory), so one CTA's
-// prologue and bubbles are filled by the other's MMAs. Q and dO pass through
-// one 32 KB staging buffer into TMEM (the A operand of every S / dP MMA);
-// K/V blocks stream through a two-stage ring. The S/dP accumulators are
+// prologue and bubbles are filled by the other's MMAs. Q (through a 32 KB
+// staging buffer) and dO (through the second K/V stage, before its first
+// use) land together and are copied into TMEM (the A operand of every S / dP
+// MMA); K/V blocks stream through a two-stage ring. The S/dP accumulators are
 // single-buffered: the full barrier of K/V block n also takes one arrival
 // per elementwise warp once it has read S/dP(n-1), so the MMA thread waits
-// once per block.
+// once per block. S and dP have separate commits, so P is formed while the
+// dP MMAs run.
 namespace kd {
 constexpr int kThreadsD = 256;   // warp 0 producer + list, warp 1 MMA, warps 4-7 rows
 constexpr uint32_t kTmemColsD = 256;
 constexpr uint32_t kColQ = 0, kColDO = 64, kColS = 128, kColDP = 192;
-constexpr uint32_t kOffStage = 0;       // Q, then dO: [k half][128 rows][128 B]
+constexpr uint32_t kOffStage = 0;       // Q: [k half][128 rows][128 B]; dO in KV stage 1
 constexpr uint32_t kOffKV = 32768;      // 2 stages x (K halves, V halves)
 constexpr uint32_t kOffCtl = kOffKV + 2 * 32768;
 struct Ctl {
-  uint64_t qd_full, qd_free, kv_full[2], kv_empty[2], s_full, drain;
+  uint64_t qd_full, qd_free, kv_full[2], kv_empty[2], s_full, dp_full, drain;
   uint32_t tmem_base;
   int abort, nblk;
   int blocks[kMaxList];
@@ -105,16 +107,21 @@ tc_bwd_d_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(&c.kv_empty[i], 1);
       }
       mbar_init(&c.s_full, 1);
+      mbar_init(&c.dp_full, 1);
       mbar_init(&c.drain, 1);
       fence_mbar_init();
       c.abort = 0;
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_do);
-      mbar_arrive_expect_tx(&c.qd_full, 4 * 8192);
+      // Q into the staging buffer and dO into K/V stage 1, one phase.
+      mbar_arrive_expect_tx(&c.qd_full, 8 * 8192);
       for (int h2 = 0; h2 < 2; ++h2)
-        for (int kb = 0; kb < 2; ++kb)
+        for (int kb = 0; kb < 2; ++kb) {
           tma_load_3d(base + kOffStage + kb * 16384 + h2 * 8192, &tm_q, kb * 64, j * kB,
                       bi * s.Hq + h0 + h2, &c.qd_full);
+          tma_load_3d(base + kOffKV + 32768 + kb * 16384 + h2 * 8192, &tm_do, kb * 64, j * kB,
+                      bi * s.Hq + h0 + h2, &c.qd_full);
+        }
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
     }
@@ -128,7 +135,7 @@ tc_bwd_d_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     __syncwarp();
     if (lane == 0) {
-      for (; issued < n + 1 && issued < 2; ++issued) {
+      for (; issued < n + 1 && issued < 1; ++issued) {  // stage 1 holds dO until it is in TMEM
         const int m = c.blocks[issued];
         unsigned char* kv = base + kOffKV + issued * 32768;
         mbar_arrive_expect_tx(&c.kv_full[issued], 32768);
@@ -152,18 +159,11 @@ tc_bwd_d_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   if (warp == 0) {
     if (lane == 0) {
-      // dO follows Q through the staging buffer once Q has moved into TMEM.
+      // Block 1 goes into stage 1 once dO has moved from there into TMEM.
       bool go = wait_or_abort(ctx, &c.qd_free, 0, abort);
-      if (go) {
-        mbar_arrive_expect_tx(&c.qd_full, 4 * 8192);
-        for (int h2 = 0; h2 < 2; ++h2)
-          for (int kb = 0; kb < 2; ++kb)
-            tma_load_3d(base + kOffStage + kb * 16384 + h2 * 8192, &tm_do, kb * 64, j * kB,
-                        bi * s.Hq + h0 + h2, &c.qd_full);
-      }
       for (int n = issued; go && n < nblk; ++n) {
         const int st = n & 1;
-        if (!wait_or_abort(ctx, &c.kv_empty[st], ((n - 2) >> 1) & 1, abort)) break;
+        if (n >= 2 && !wait_or_abort(ctx, &c.kv_empty[st], ((n - 2) >> 1) & 1, abort)) break;
         const int m = c.blocks[n];
         unsigned char* kv = base + kOffKV + st * 32768;
         mbar_arrive_expect_tx(&c.kv_full[st], 32768);
@@ -174,9 +174,8 @@ tc_bwd_d_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         issued = n + 1;
       }
-      // The staging copies land before the CTA leaves (the dO phase, when
-      // issued, completes after the Q phase).
-      (void)mbar_wait(ctx, &c.qd_full, go ? 1 : 0);
+      // The Q / dO copies land before the CTA leaves.
+      (void)mbar_wait(ctx, &c.qd_full, 0);
       if (*abort)
         for (int n = max(0, issued - 2); n < issued; ++n)
           (void)mbar_wait(ctx, &c.kv_full[n & 1], (n >> 1) & 1);
@@ -198,11 +197,12 @@ tc_bwd_d_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int ks = 0; ks < 8; ++ks)
           mma_bf16_ts(tmem + kColS, tmem + kColQ + ks * 8,
                       kd + (((ks >> 2) * 8192 + (ks & 3) * 32) >> 4), id_s, ks > 0);
+        mma_commit(&c.s_full);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
           mma_bf16_ts(tmem + kColDP, tmem + kColDO + ks * 8,
                       kd + ((16384 + (ks >> 2) * 8192 + (ks & 3) * 32) >> 4), id_s, ks > 0);
-        mma_commit(&c.s_full);
+        mma_commit(&c.dp_full);
         mma_commit(&c.kv_empty[st]);
       }
       (void)ok;
@@ -215,23 +215,19 @@ tc_bwd_d_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
     const float sc = s.scale * kLog2e;
     const uint64_t sc2 = f2u(sc, sc);
-    // Q, then dO, from the staging buffer into this row's TMEM lane.
+    // Q (staging buffer) and dO (K/V stage 1) into this row's TMEM lane.
     bool ok = warp_wait(ctx, &c.qd_full, 0, abort);
     if (ok) {
       tile_row_to_tmem(base + kOffStage, rowi, tl + kColQ);
+      tile_row_to_tmem(base + kOffKV + 32768, rowi, tl + kColDO);
       tmem_st_wait();
     }
     fence_before_sync();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&c.qd_free);
-    ok = ok && warp_wait(ctx, &c.qd_full, 1, abort);
-    if (ok) {
-      tile_row_to_tmem(base + kOffStage, rowi, tl + kColDO);
-      tmem_st_wait();
+    if (lane == 0) {
+      mbar_arrive(&c.qd_free);     // stage 1 may take block 1
+      mbar_arrive(&c.kv_full[0]);  // Q, dO in TMEM: S/dP(0) may start
     }
-    fence_before_sync();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&c.kv_full[0]);  // Q, dO in TMEM: S/dP(0) may start
     float Dsum = 0.f;
     for (int n = 0; ok && n < nblk; ++n) {
       if (!warp_wait(ctx, &c.s_full, n & 1, abort)) {
@@ -245,40 +241,48 @@ tc_bwd_d_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int kvalid = min(kB, s.T - m * kB);
       const float off = live ? bias - lse2 : -INFINITY;
       const uint64_t off2 = f2u(off, off);
-      uint32_t sr[64], pr[32];
-      tmem_ld32(tl + kColS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tl + kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld32(tl + kColDP, pr);
-      tmem_ld_wait();
-      if (cur || kvalid < kB) {
+      // P from S while the dP MMAs run.
+      uint64_t p2[32];
+      {
+        uint32_t sr[64];
+        tmem_ld32(tl + kColS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(tl + kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_ld_wait();
+        if (cur || kvalid < kB) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (i >= kvalid || (cur && i > r)) sr[i] = __float_as_uint(-INFINITY);
+          for (int i = 0; i < 64; ++i)
+            if (i >= kvalid || (cur && i > r)) sr[i] = __float_as_uint(-INFINITY);
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const uint64_t a2 = ffma2(f2u(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
+                                    sc2, off2);
+          p2[i] = f2u(ex2(lo_f(a2)), ex2(hi_f(a2)));
+        }
       }
+      if (!warp_wait(ctx, &c.dp_full, n & 1, abort)) {
+        ok = false;
+        break;
+      }
+      fence_after_sync();
       uint64_t acc0 = 0, acc1 = 0;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const uint64_t a2 = ffma2(f2u(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
-                                  sc2, off2);
-        const uint64_t p2 = f2u(ex2(lo_f(a2)), ex2(hi_f(a2)));
-        const uint64_t dp2 = f2u(__uint_as_float(pr[2 * i]), __uint_as_float(pr[2 * i + 1]));
-        if (i & 1) acc1 = ffma2(p2, dp2, acc1);
-        else acc0 = ffma2(p2, dp2, acc0);
-      }
-      tmem_ld32(tl + kColDP + 32, pr);
-      tmem_ld_wait();
-      // S/dP(n) are in registers: S/dP(n + 1) may overwrite the accumulators.
-      fence_before_sync();
-      __syncwarp();
-      if (lane == 0 && n + 1 < nblk) mbar_arrive(&c.kv_full[(n + 1) & 1]);
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t pr[32];
+        tmem_ld32(tl + kColDP + hf * 32, pr);
+        tmem_ld_wait();
+        if (hf == 1) {
+          // S/dP(n) are in registers: S/dP(n + 1) may overwrite the accumulators.
+          fence_before_sync();
+          __syncwarp();
+          if (lane == 0 && n + 1 < nblk) mbar_arrive(&c.kv_full[(n + 1) & 1]);
+        }
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const uint64_t a2 = ffma2(f2u(__uint_as_float(sr[32 + 2 * i]), __uint_as_float(sr[32 + 2 * i + 1])),
-                                  sc2, off2);
-        const uint64_t p2 = f2u(ex2(lo_f(a2)), ex2(hi_f(a2)));
-        const uint64_t dp2 = f2u(__uint_as_float(pr[2 * i]), __uint_as_float(pr[2 * i + 1]));
-        if (i & 1) acc1 = ffma2(p2, dp2, acc1);
-        else acc0 = ffma2(p2, dp2, acc0);
+        for (int i = 0; i < 16; ++i) {
+          const uint64_t dp2 = f2u(__uint_as_float(pr[2 * i]), __uint_as_float(pr[2 * i + 1]));
+          if (i & 1) acc1 = ffma2(p2[hf * 16 + i], dp2, acc1);
+          else acc0 = ffma2(p2[hf * 16 + i], dp2, acc0);
+        }
       }
       const uint64_t accs = fadd2(acc0, acc1);
       Dsum += lo_f(accs) + hi_f(accs);
