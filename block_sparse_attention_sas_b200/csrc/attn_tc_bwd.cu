@@ -257,7 +257,8 @@ tc_bwd_d_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int i = 0; i < 32; ++i) {
           const uint64_t a2 = ffma2(f2u(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
                                     sc2, off2);
-          p2[i] = f2u(ex2(lo_f(a2)), ex2(hi_f(a2)));
+          // A quarter of the exponentials on the FMA pipe (MUFU-bound phase).
+          p2[i] = ((i & 3) == 3) ? ex2_poly2(a2) : f2u(ex2(lo_f(a2)), ex2(hi_f(a2)));
         }
       }
       if (!warp_wait(ctx, &c.dp_full, n & 1, abort)) {
@@ -853,8 +854,14 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int i = 0; i < 16; ++i) {
           const uint64_t a2 = ffma2(f2u(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
                                     sc2, off2);
-          pf[2 * i] = ex2(lo_f(a2));
-          pf[2 * i + 1] = ex2(hi_f(a2));
+          if ((i & 3) == 3) {  // a quarter of the exponentials on the FMA pipe
+            const uint64_t e = ex2_poly2(a2);
+            pf[2 * i] = lo_f(e);
+            pf[2 * i + 1] = hi_f(e);
+          } else {
+            pf[2 * i] = ex2(lo_f(a2));
+            pf[2 * i + 1] = ex2(hi_f(a2));
+          }
           pp[i] = pack_bf16(pf[2 * i], pf[2 * i + 1]);
         }
 #pragma unroll

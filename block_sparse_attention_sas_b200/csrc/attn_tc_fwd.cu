@@ -318,8 +318,18 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                                   sc2, off2);
         const uint64_t a1 = ffma2(f2u(__uint_as_float(sr[2 * i + 2]), __uint_as_float(sr[2 * i + 3])),
                                   sc2, off2);
+        // A quarter of the exponentials go to the FMA pipe (the softmax is
+        // bound by the MUFU unit otherwise).
         const float p0 = ex2(lo_f(a0)), p1 = ex2(hi_f(a0));
-        const float p2 = ex2(lo_f(a1)), p3 = ex2(hi_f(a1));
+        float p2, p3;
+        if ((i & 3) == 2) {
+          const uint64_t e = ex2_poly2(a1);
+          p2 = lo_f(e);
+          p3 = hi_f(e);
+        } else {
+          p2 = ex2(lo_f(a1));
+          p3 = ex2(hi_f(a1));
+        }
         acc0 = fadd2(acc0, f2u(p0, p1));
         acc1 = fadd2(acc1, f2u(p2, p3));
         pk[i] = pack_bf16(p0, p1);

@@ -14,6 +14,7 @@
 // [4,7) xor [7,10)) matches the TMA's.
 #pragma once
 
+#include "exp2_poly.h"
 #include <cuda.h>
 #include <stdint.h>
 
@@ -241,6 +242,31 @@ __device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
   asm("mul.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+
+// ---- exp2 of a pair on the FMA pipe, to take part of the ex2 work off the
+// MUFU unit where an elementwise phase is bound by it. x = n + f with
+// n = round(x) (adding 1.5 * 2^23 rounds to nearest and leaves n in the low
+// mantissa bits), f in [-1/2, 1/2]; 2^f by the degree-5 polynomial of
+// exp2_poly.h in Horner form; n is then added to the exponent field (the
+// magic constant's low 9 bits are zero, so bits(t) << 23 == n << 23). Inputs
+// are clamped to -125, so -inf gives 2^-125 (~2.4e-38) where ex2.approx.ftz
+// gives 0. Relative error ~2.5e-7 on [-125, 127].
+__device__ __forceinline__ uint64_t ex2_poly2(uint64_t x2) {
+  const float xa = fmaxf(lo_f(x2), -125.f), xb = fmaxf(hi_f(x2), -125.f);
+  const uint64_t x = f2u(xa, xb);
+  const uint64_t t = fadd2(x, f2u(12582912.f, 12582912.f));
+  const uint64_t n = fadd2(t, f2u(-12582912.f, -12582912.f));
+  const uint64_t f = ffma2(n, f2u(-1.f, -1.f), x);
+  uint64_t p = ffma2(f2u(kExp2C5, kExp2C5), f, f2u(kExp2C4, kExp2C4));
+  p = ffma2(p, f, f2u(kExp2C3, kExp2C3));
+  p = ffma2(p, f, f2u(kExp2C2, kExp2C2));
+  p = ffma2(p, f, f2u(kExp2C1, kExp2C1));
+  p = ffma2(p, f, f2u(kExp2C0, kExp2C0));
+  const uint32_t ra = (uint32_t)p + ((uint32_t)t << 23);
+  const uint32_t rb = (uint32_t)(p >> 32) + ((uint32_t)(t >> 32) << 23);
+  return ((uint64_t)rb << 32) | ra;
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
