@@ -38,8 +38,9 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxList = 257;
 
 // ============================================================================
-// Kernel D: D_i = sum over the attended keys of P_it dP_it (exact, r12 of the
-// design notes is the reading; the forward's bf16 o would round it)
+// Kernel D: D_i = sum over the attended keys of P_it dP_it, summed exactly
+// rather than taken as dO . o: the forward's o is stored in bf16, and its
+// rounding (up to 2^-9 |o|) would reach every gradient through D.
 // ============================================================================
 // One CTA per (query block j, 128-row tile of two heads, KV head, batch),
 // two CTAs per SM (256 TMEM columns, 97 KB of shared memory), so one CTA's
