@@ -42,6 +42,10 @@ def test_gate_topk_decode_configs(cuda_lib, name):
     (16, 4, True, 0), (64, 64, True, 0), (200, 5, True, 2), (33, 1, True, 1),
     (1500, 16, True, 0), (5000, 64, False, 0), (70000, 256, False, 0), (3000, 100, False, 3),
     (1, 3, False, 0), (40, 256, False, 0),
+    # long-row paths: first chunked size, one block with K = 256 (full-sort
+    # fallback), chunked rows with heavy ties, chunked causal rows, many chunks
+    (2049, 8, False, 0), (2048, 256, False, 0), (9000, 256, False, 2), (2100, 16, True, 0),
+    (20000, 64, False, 0),
 ])
 def test_gate_topk_edges(cuda_lib, C, K, causal, levels):
     rng = np.random.default_rng(C * 7 + K)
