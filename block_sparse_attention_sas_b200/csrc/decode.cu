@@ -447,11 +447,15 @@ cudaError_t decode_g(const DecodeShape& s, const void* q, const void* kc, const 
 }  // namespace
 
 void decode_plan(DecodeShape& s) {
-  // At most two CTAs per SM (148 SMs) in one wave, at most kMaxSplits per
-  // (batch, kv head).
+  // CTAs in one wave (148 SMs), at most kMaxSplits per (batch, kv head). A
+  // sparse call's lists are short (tens of blocks per (batch, KV head)), and
+  // about 1.5 CTAs per SM gave the shortest times there: fewer, longer CTAs
+  // pay less prologue and merge per block. 1 and 2 per SM were slower for the
+  // Qwen3-14B 512K or the Qwen3-4B 64K decode. The dense comparison streams
+  // long lists and keeps two per SM.
   const int nslots = s.dense ? s.C + 1 : s.K + 1;
   const int units = s.B * s.Hkv;
-  const int target = 2 * 148;
+  const int target = s.dense ? 2 * 148 : 3 * 148 / 2;
   int splits = target / units;
   splits = max(1, min(splits, min(nslots, kMaxSplits)));
   int bps = (nslots + splits - 1) / splits;
