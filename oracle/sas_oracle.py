@@ -294,6 +294,240 @@ def attn_bwd(q, k, v, dO, idx, gates, logg, b, scale=0.0, use_gates=True):
     return dq, dk, dv, ds
 
 
+# ---------------------------------------------------------------------------
+# Gate variants: the ablation axes of the pages (the functions above are the
+# method itself; these are its ablated forms, for the variant kernels)
+# ---------------------------------------------------------------------------
+# [Methodology, Eq. 4] (picx.dev) leaves the gate activation phi open, and
+# the summary's ablations (Table 1 as summarised there) compare phi =
+# softmax with sigmoid and raw-logit gates. [Gradient Analysis, Eq. 5]
+# contrasts inner gating (log g added to the logits, Eq. 9) with outer
+# gating. Readings, for lack of a formula on the pages:
+#   - sigmoid: g_m = 1 / (1 + exp(-s_m)), elementwise, no normalisation over
+#     the history, so log g_m = -log(1 + exp(-s_m));
+#   - raw logits: log g_m = s_m, the score enters the logits as it is;
+#   - outer gating: o = sum_i g_{m(i)} p_i v_i with p the ungated softmax
+#     over the selected keys plus the current block (g0 = 1): the form whose
+#     derivative in g_m is the outer form of Eq. 5.
+# Top-K is over the scores in every variant (every phi is increasing).
+
+PHIS = ("softmax", "sigmoid", "raw")
+
+
+def log_gates_row_phi(s_row, n: int, phi: str) -> np.ndarray:
+    """log g over the n history blocks for the gate activation ``phi``."""
+    s = _f64(s_row[:n])
+    if phi == "softmax":
+        return log_gates_row(s_row, n)
+    if phi == "sigmoid":
+        return -np.logaddexp(0.0, -s)
+    if phi == "raw":
+        return s.copy()
+    raise ValueError(phi)
+
+
+def gate_topk_phi(scores, K: int, phi: str, causal: bool = True):
+    """gate_topk with the activation ``phi``: (gates, log_gates, idx)."""
+    gates, logg, idx = gate_topk(scores, K, causal)
+    if phi == "softmax":
+        return gates, logg, idx
+    s = np.asarray(scores)
+    B, H, R, C = s.shape
+    for bi in range(B):
+        for h in range(H):
+            for r in range(R):
+                n = min(r, C) if causal else C
+                lg = log_gates_row_phi(s[bi, h, r], n, phi)
+                logg[bi, h, r, :n] = lg
+                gates[bi, h, r, :n] = np.exp(lg)
+    return gates, logg, idx
+
+
+def dscores_row_phi(da: dict, s_row, n: int, phi: str) -> np.ndarray:
+    """dL/ds_k for k < n from da_m = dL/d log g_m of the selected blocks.
+
+    softmax: d log g_m / d s_k = delta_mk - g_k (Eq. 6, as dscores_row);
+    sigmoid: d log g_m / d s_k = delta_mk (1 - sigmoid(s_k));
+    raw:     d log g_m / d s_k = delta_mk.
+    """
+    if phi == "softmax":
+        return dscores_row(da, np.exp(log_gates_row(s_row, n)), n)
+    out = np.zeros(n)
+    s = _f64(s_row[:n])
+    for m, a in da.items():
+        out[m] = a * (np.exp(-np.logaddexp(0.0, s[m])) if phi == "sigmoid" else 1.0)
+    return out
+
+
+def attn_bwd_phi(q, k, v, dO, idx, scores, b, phi: str, scale=0.0):
+    """Inner gating (Eq. 9) with gates from ``phi``: (dq, dk, dv, dscores)."""
+    _, logg, _ = gate_topk_phi(scores, idx.shape[-1], phi)
+    B, Hq, T, d = np.shape(q)
+    Hkv = np.shape(k)[1]
+    G = Hq // Hkv
+    N = (T + b - 1) // b
+    dq = np.zeros((B, Hq, T, d))
+    dk = np.zeros((B, Hkv, T, d))
+    dv = np.zeros((B, Hkv, T, d))
+    ds = np.zeros((B, Hkv, N, N))
+    for bi in range(B):
+        for kvh in range(Hkv):
+            for j in range(N):
+                r = attn_bwd_block(q, k, v, dO, idx, logg, bi, kvh, j, b, scale)
+                r0, r1 = j * b, min(T, (j + 1) * b)
+                dq[bi, kvh * G:(kvh + 1) * G, r0:r1] = r["dq"]
+                np.add.at(dk[bi, kvh], r["cols"], r["dk_c"])
+                np.add.at(dv[bi, kvh], r["cols"], r["dv_c"])
+                ds[bi, kvh, j, :j] = dscores_row_phi(r["da"], scores[bi, kvh, j], j, phi)
+    return dq, dk, dv, ds
+
+
+def _col_gates(j, b, T, sel_row, gates_row):
+    """Per-column gate of query block j's key set (g_m on block m, 1 on block j)."""
+    w = []
+    for m in sel_row:
+        m = int(m)
+        if m >= 0:
+            w.extend([float(gates_row[m])] * b)
+    w.extend([1.0] * (min(T, (j + 1) * b) - j * b))
+    return np.asarray(w)
+
+
+def attn_fwd_outer_block(q, k, v, idx, gates, bi, kvh, j, b, scale=0.0):
+    """Outer gating for the G heads of KV head ``kvh`` and block j's rows:
+    o = (P * w) V with P the ungated softmax and w the per-column gates.
+    Returns (o [G, rows, d], lse [G, rows]) where lse is the ungated one."""
+    q, k, v = np.asarray(q), np.asarray(k), np.asarray(v)
+    Hq, T, d = q.shape[1], q.shape[2], q.shape[3]
+    G = Hq // k.shape[1]
+    scale = _default_scale(d, scale)
+    cols, bias, nh = _key_set(j, b, T, idx[bi, kvh, j], None, False)
+    w = _col_gates(j, b, T, idx[bi, kvh, j], gates[bi, kvh, j])
+    Kc, Vc = _f64(k[bi, kvh, cols]), _f64(v[bi, kvh, cols])
+    r0, r1 = j * b, min(T, (j + 1) * b)
+    O = np.empty((G, r1 - r0, d))
+    L = np.empty((G, r1 - r0))
+    for g in range(G):
+        X = _block_logits(_f64(q[bi, kvh * G + g, r0:r1]), Kc, bias, nh, scale, r0, j * b)
+        lse = _lse_rows(X)
+        O[g] = (np.exp(X - lse[:, None]) * w[None, :]) @ Vc
+        L[g] = lse
+    return O, L
+
+
+def attn_fwd_outer(q, k, v, idx, gates, b, scale=0.0):
+    """Outer gating over every query block: (o [B,Hq,T,d], lse [B,Hq,T])."""
+    B, Hq, T, d = np.shape(q)
+    Hkv = np.shape(k)[1]
+    G = Hq // Hkv
+    N = (T + b - 1) // b
+    o = np.empty((B, Hq, T, d))
+    lse = np.empty((B, Hq, T))
+    for bi in range(B):
+        for kvh in range(Hkv):
+            for j in range(N):
+                O, L = attn_fwd_outer_block(q, k, v, idx, gates, bi, kvh, j, b, scale)
+                r0, r1 = j * b, min(T, (j + 1) * b)
+                o[bi, kvh * G:(kvh + 1) * G, r0:r1] = O
+                lse[bi, kvh * G:(kvh + 1) * G, r0:r1] = L
+    return o, lse
+
+
+def attn_bwd_outer_block(q, k, v, dO, idx, gates, bi, kvh, j, b, scale=0.0):
+    """Gradients of L = sum(o * dO) under outer gating from query block j.
+
+    With W = P * w: dv += W^T dO; dL/dP = w * dP (dP = dO V^T), so the
+    softmax Jacobian gives dX = P * (w dP - rowsum(P w dP)); dq = scale dX K,
+    dk += scale dX^T Q; dg_m = sum over block m's columns, all rows and all G
+    heads of P * dP (Eq. 5, outer form), returned as da_m = g_m dg_m
+    (= dL/d log g_m, the input of the phi Jacobians above).
+    """
+    q, k, v, dO = np.asarray(q), np.asarray(k), np.asarray(v), np.asarray(dO)
+    Hq, T, d = q.shape[1], q.shape[2], q.shape[3]
+    G = Hq // k.shape[1]
+    scale = _default_scale(d, scale)
+    cols, bias, nh = _key_set(j, b, T, idx[bi, kvh, j], None, False)
+    w = _col_gates(j, b, T, idx[bi, kvh, j], gates[bi, kvh, j])
+    Kc, Vc = _f64(k[bi, kvh, cols]), _f64(v[bi, kvh, cols])
+    r0, r1 = j * b, min(T, (j + 1) * b)
+    dq = np.zeros((G, r1 - r0, d))
+    dk_c, dv_c = np.zeros_like(Kc), np.zeros_like(Vc)
+    pdp_hist = np.zeros(nh)
+    for g in range(G):
+        Qb = _f64(q[bi, kvh * G + g, r0:r1])
+        dOb = _f64(dO[bi, kvh * G + g, r0:r1])
+        X = _block_logits(Qb, Kc, bias, nh, scale, r0, j * b)
+        P = np.exp(X - _lse_rows(X)[:, None])
+        dP = dOb @ Vc.T
+        wdP = dP * w[None, :]
+        dX = P * (wdP - (P * wdP).sum(axis=1, keepdims=True))
+        dq[g] = scale * (dX @ Kc)
+        dk_c += scale * (dX.T @ Qb)
+        dv_c += (P * w[None, :]).T @ dOb
+        pdp_hist += (P * dP)[:, :nh].sum(axis=0)
+    da, pos = {}, 0
+    for m in idx[bi, kvh, j]:
+        m = int(m)
+        if m < 0:
+            continue
+        da[m] = float(gates[bi, kvh, j, m]) * pdp_hist[pos:pos + b].sum()
+        pos += b
+    return {"dq": dq, "cols": cols, "dk_c": dk_c, "dv_c": dv_c, "da": da}
+
+
+def gate_grad_eq5_outer(q, k, v, dO, idx, gates, bi, kvh, j, b, scale=0.0):
+    """Eq. 5, outer form, literally: dg_m = sum_i p_i dO^T v_i over the keys i
+    of selected block m, for every row and every head of the group, with p
+    the ungated softmax over the block's key set. Returns {m: dg_m}."""
+    q, k, v, dO = np.asarray(q), np.asarray(k), np.asarray(v), np.asarray(dO)
+    Hq, T, d = q.shape[1], q.shape[2], q.shape[3]
+    G = Hq // k.shape[1]
+    scale = _default_scale(d, scale)
+    cols, bias, nh = _key_set(j, b, T, idx[bi, kvh, j], None, False)
+    Kc, Vc = _f64(k[bi, kvh, cols]), _f64(v[bi, kvh, cols])
+    r0, r1 = j * b, min(T, (j + 1) * b)
+    out, pos = {}, 0
+    for m in idx[bi, kvh, j]:
+        m = int(m)
+        if m < 0:
+            continue
+        tot = 0.0
+        for g in range(G):
+            Qb = _f64(q[bi, kvh * G + g, r0:r1])
+            dOb = _f64(dO[bi, kvh * G + g, r0:r1])
+            X = _block_logits(Qb, Kc, bias, nh, scale, r0, j * b)
+            P = np.exp(X - _lse_rows(X)[:, None])
+            for row in range(r1 - r0):
+                for c in range(pos, pos + b):
+                    tot += P[row, c] * float(dOb[row] @ Vc[c])
+        out[m] = tot
+        pos += b
+    return out
+
+
+def attn_bwd_outer(q, k, v, dO, idx, scores, b, phi: str = "softmax", scale=0.0):
+    """Outer gating with gates from ``phi``: (dq, dk, dv, dscores)."""
+    gates, _, _ = gate_topk_phi(scores, idx.shape[-1], phi)
+    B, Hq, T, d = np.shape(q)
+    Hkv = np.shape(k)[1]
+    G = Hq // Hkv
+    N = (T + b - 1) // b
+    dq = np.zeros((B, Hq, T, d))
+    dk = np.zeros((B, Hkv, T, d))
+    dv = np.zeros((B, Hkv, T, d))
+    ds = np.zeros((B, Hkv, N, N))
+    for bi in range(B):
+        for kvh in range(Hkv):
+            for j in range(N):
+                r = attn_bwd_outer_block(q, k, v, dO, idx, gates, bi, kvh, j, b, scale)
+                r0, r1 = j * b, min(T, (j + 1) * b)
+                dq[bi, kvh * G:(kvh + 1) * G, r0:r1] = r["dq"]
+                np.add.at(dk[bi, kvh], r["cols"], r["dk_c"])
+                np.add.at(dv[bi, kvh], r["cols"], r["dv_c"])
+                ds[bi, kvh, j, :j] = dscores_row_phi(r["da"], scores[bi, kvh, j], j, phi)
+    return dq, dk, dv, ds
+
+
 def gate_grad_eq5(q, k, v, dO, idx, gates, logg, bi, kvh, j, b, scale=0.0):
     """Eq. 5, inner form, literally: dg_m = sum_i (p~_i / g_m) dO^T (v_i - o).
 

@@ -13,6 +13,7 @@ import pytest
 
 from oracle import sas_oracle as O
 from tests import test_oracle as P
+from tests import test_oracle_variants as V
 
 
 def _no_scale(d, scale):
@@ -59,6 +60,45 @@ ORIG = {name: getattr(O, name) for name in
         ("_default_scale", "_key_set", "dscores_row", "_block_logits", "topk_row",
          "log_gates_row", "_lse_rows")}
 
+ORIG_V = {name: getattr(O, name) for name in
+          ("dscores_row_phi", "log_gates_row_phi", "attn_bwd_outer_block", "_col_gates")}
+
+
+def _sigmoid_jacobian_flipped(da, s_row, n, phi):
+    out = ORIG_V["dscores_row_phi"](da, s_row, n, phi)
+    if phi == "sigmoid":
+        s = np.asarray(s_row[:n], np.float64)
+        for m, a in da.items():
+            out[m] = a / (1.0 + np.exp(-s[m]))  # sigma(s) where 1 - sigma(s) belongs
+    return out
+
+
+def _sigmoid_log_gate_sign(s_row, n, phi):
+    if phi == "sigmoid":
+        return -np.logaddexp(0.0, np.asarray(s_row[:n], np.float64))
+    return ORIG_V["log_gates_row_phi"](s_row, n, phi)
+
+
+def _outer_da_without_gate(q, k, v, dO, idx, gates, bi, kvh, j, b, scale=0.0):
+    r = ORIG_V["attn_bwd_outer_block"](q, k, v, dO, idx, gates, bi, kvh, j, b, scale)
+    r["da"] = {m: a / float(gates[bi, kvh, j, m]) for m, a in r["da"].items()}
+    return r
+
+
+def _current_block_gated(j, b, T, sel_row, gates_row):
+    w = ORIG_V["_col_gates"](j, b, T, sel_row, gates_row)
+    ncur = min(T, (j + 1) * b) - j * b
+    w[len(w) - ncur:] = 0.5
+    return w
+
+
+def _pin(fn, *args):
+    def run():
+        fn(*args)
+    run.__name__ = fn.__name__ + "".join(f"[{a}]" for a in args)
+    return run
+
+
 MUTANTS = {
     "dropped 1/sqrt(d)": ("_default_scale", _no_scale,
                           [P.test_golden_scale, P.test_fwd_reduces_to_dense_causal]),
@@ -75,6 +115,16 @@ MUTANTS = {
                            [P.test_golden_gate_softmax, P.test_gates_sum_to_one_and_positive]),
     "lse without the sum": ("_lse_rows", _lse_max_only,
                             [P.test_fwd_reduces_to_dense_causal, P.test_golden_scale]),
+    "sigmoid Jacobian uses sigma(s)": ("dscores_row_phi", _sigmoid_jacobian_flipped,
+                                       [_pin(V.test_inner_gating_finite_differences, "sigmoid")]),
+    "sigmoid log gate of -s": ("log_gates_row_phi", _sigmoid_log_gate_sign,
+                               [V.test_sigmoid_gates_are_the_logistic_function]),
+    "outer da without g_m": ("attn_bwd_outer_block", _outer_da_without_gate,
+                             [V.test_eq5_outer_gate_gradient,
+                              _pin(V.test_outer_gating_finite_differences, "softmax")]),
+    "outer gate on the current block": ("_col_gates", _current_block_gated,
+                                        [V.test_outer_with_unit_gates_is_ungated_sparse_attention,
+                                         V.test_outer_backward_matches_autograd]),
 }
 
 
