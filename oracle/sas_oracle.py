@@ -602,6 +602,39 @@ def decode(q, kcache, vcache, idx, logg, b, scale=0.0, use_gates=False):
     return o
 
 
+def decode_paged(q, kpages, vpages, page_indptr, page_indices, seq_lens, idx, logg, b,
+                 scale=0.0, use_gates=False):
+    """Decode over a paged KV cache, one sequence per batch entry.
+
+    The pages mention that deployment decodes on a paged cache (SGLang /
+    FlashInfer) without fixing a layout. Reading: kpages / vpages are
+    [num_pages, Hkv, P, d] (P tokens per page); sequence bi owns the pages
+    page_indices[page_indptr[bi]:page_indptr[bi+1]] in logical order, token t
+    sits at offset t % P of its (t // P)-th page, and it has seq_lens[bi]
+    tokens (the last page may be partly used). Its query is at position
+    seq_lens[bi] - 1; idx[bi] selects among its floor((seq_lens[bi]-1)/b)
+    history blocks, and logg[bi] holds their log gates. The result is that of
+    ``decode`` on the sequence's gathered contiguous cache.
+    Returns o [B,Hq,d] float64.
+    """
+    q = np.asarray(q)
+    kp, vp = np.asarray(kpages), np.asarray(vpages)
+    B = q.shape[0]
+    P = kp.shape[2]
+    o = np.empty(q.shape, dtype=np.float64)
+    for bi in range(B):
+        L = int(seq_lens[bi])
+        pages = np.asarray(page_indices[page_indptr[bi]:page_indptr[bi + 1]], np.int64)
+        t = np.arange(L)
+        kc = kp[pages[t // P], :, t % P].transpose(1, 0, 2)  # [Hkv, L, d]
+        vc = vp[pages[t // P], :, t % P].transpose(1, 0, 2)
+        C = (L - 1) // b
+        lg = np.asarray(logg)[bi:bi + 1, :, :C] if logg is not None else None
+        o[bi] = decode(q[bi:bi + 1], kc[None], vc[None], np.asarray(idx)[bi:bi + 1], lg, b,
+                       scale, use_gates)[0]
+    return o
+
+
 # ---------------------------------------------------------------------------
 # Dense comparison (Eq. 1 with a causal mask): every block, gates off
 # ---------------------------------------------------------------------------

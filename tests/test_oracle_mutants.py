@@ -14,6 +14,7 @@ import pytest
 from oracle import sas_oracle as O
 from tests import test_oracle as P
 from tests import test_oracle_variants as V
+from tests import test_oracle_paged as PG
 
 
 def _no_scale(d, scale):
@@ -61,7 +62,18 @@ ORIG = {name: getattr(O, name) for name in
          "log_gates_row", "_lse_rows")}
 
 ORIG_V = {name: getattr(O, name) for name in
-          ("dscores_row_phi", "log_gates_row_phi", "attn_bwd_outer_block", "_col_gates")}
+          ("dscores_row_phi", "log_gates_row_phi", "attn_bwd_outer_block", "_col_gates",
+           "decode_paged")}
+
+
+def _paged_pages_reversed(q, kpages, vpages, page_indptr, page_indices, seq_lens, idx, logg, b,
+                          scale=0.0, use_gates=False):
+    ix = np.asarray(page_indices).copy()
+    for bi in range(len(page_indptr) - 1):
+        lo, hi = page_indptr[bi], page_indptr[bi + 1]
+        ix[lo:hi] = ix[lo:hi][::-1]
+    return ORIG_V["decode_paged"](q, kpages, vpages, page_indptr, ix, seq_lens, idx, logg, b,
+                                  scale, use_gates)
 
 
 def _sigmoid_jacobian_flipped(da, s_row, n, phi):
@@ -125,6 +137,9 @@ MUTANTS = {
     "outer gate on the current block": ("_col_gates", _current_block_gated,
                                         [V.test_outer_with_unit_gates_is_ungated_sparse_attention,
                                          V.test_outer_backward_matches_autograd]),
+    "paged: pages in reverse order": ("decode_paged", _paged_pages_reversed,
+                                      [PG.test_uniform_lengths_equal_contiguous_decode,
+                                       PG.test_full_selection_is_attention_of_the_last_token]),
 }
 
 
