@@ -14,14 +14,17 @@ CPU throughput.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Under torchrun (N > 1) every rank runs its own batch (weak scaling, no
-collective on the data path); the step time is the max over ranks.
+With N > 1 every rank runs its own batch (weak scaling, no collective on the
+data path); the step time is the max over ranks. Started without a torchrun
+environment, `--gpus N` re-launches itself under torch.distributed.run with N
+ranks on 127.0.0.1.
 """
 from __future__ import annotations
 
 import argparse
 import json
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -88,31 +91,91 @@ def load_peaks():
 # ---------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    """SM clocks and throttle reasons sampled while the timed region runs: an
+    NVML polling thread (every 5 ms, read-only queries), else nvidia-smi
+    every 50 ms. Samples taken before mark() (the idle lead-in) are dropped."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, gpu_id: str | None):
         self.proc = None
         self.path = None
         self.gpu_id = gpu_id
+        self.skip = 0
+        self.samples = []  # (sm_mhz, sm_max_mhz, reasons) from NVML
+        self.thread = None
+        self.stop = False
+
+    def _nvml_loop(self, nv, h):
+        bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+        smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self.stop:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((sm, smax, [n for n, b in bits.items() if r & b]))
+            except Exception:
+                pass
+            time.sleep(0.005)
 
     def __enter__(self):
+        try:
+            import threading
+
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByPciBusId(self.gpu_id) if self.gpu_id else \
+                nv.nvmlDeviceGetHandleByIndex(0)
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
+            self.thread.start()
+            t0 = time.time()
+            while not self.samples and time.time() - t0 < 2.0:
+                time.sleep(0.005)
+            if self.samples:
+                return self
+            self.stop = True
+        except Exception:
+            self.thread = None
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             cmd = ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                   "-lms", "200"]
+                   "-lms", "50"]
             if self.gpu_id:
                 cmd += ["-i", self.gpu_id]
             self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"),
                                          stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+        # nvidia-smi takes a moment to start: wait (up to 5 s) for its first
+        # sample so the timed region that follows is covered.
+        t0 = time.time()
+        while self.proc is not None and time.time() - t0 < 5.0:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.02)
         return self
 
+    def mark(self):
+        """Samples taken before this call (the idle lead-in) are left out."""
+        if self.thread is not None and not self.stop:
+            self.skip = len(self.samples)
+            return
+        try:
+            with open(self.path) as f:
+                self.skip = sum(1 for _ in f)
+        except (OSError, TypeError):
+            self.skip = 0
+
     def __exit__(self, *a):
+        self.stop = True
+        if self.thread is not None:
+            self.thread.join(timeout=1.0)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -121,11 +184,18 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
+        if self.samples and self.proc is None:
+            got = self.samples[self.skip:] or self.samples[-1:]
+            reasons = sorted({r for _, _, rs in got for r in rs})
+            return {"sm_mhz": statistics.median(x for x, _, _ in got),
+                    "sm_max_mhz": max(y for _, y, _ in got), "reasons": reasons,
+                    "samples": len(got), "source": "nvml 5 ms"}
         if not self.path or not os.path.exists(self.path):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
         sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
+        for n_line, line in enumerate(open(self.path)):
+            if n_line < self.skip:
+                continue
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
                 continue
@@ -134,14 +204,14 @@ class ClockSampler:
                 smax.append(float(f[2]))
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
+            for n, v in zip(self.NAMES, f[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
         os.unlink(self.path)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi 50 ms"}
 
 
 def gpu_pci_id(torch, dev):
@@ -154,6 +224,16 @@ def gpu_pci_id(torch, dev):
 
 
 # ------------------------------------------------------------------ CPU side
+
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
 
 def blas_threads():
     try:
@@ -246,6 +326,7 @@ def run_ours(args):
     with ClockSampler(gpu_pci_id(torch, dev)) as clk:
         D.barrier(dev)
         torch.cuda.synchronize(dev)
+        clk.mark()
         t_wall = time.perf_counter()
         for i in range(args.steps):
             flush.zero_()
@@ -263,31 +344,23 @@ def run_ours(args):
     step_ms_max = D.max_over_ranks(step_ms, dev)
     value = world * (f_fwd + f_bwd) / (step_ms_max * 1e-3) / 1e12
 
-    # ---- e2e: host buffers in, result (dscores, the selector gradient) out
-    out_h = torch.empty((cfg.B, cfg.Hkv, cfg.N, cfg.N), dtype=torch.float32).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in h.values())
-    d2h = out_h.numel() * out_h.element_size()
-    e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(args.steps)]
-    D.barrier(dev)
-    torch.cuda.synchronize(dev)
-    for i in range(args.steps):
-        flush.zero_()
-        torch.cuda._sleep(HEAD_START_CYCLES)
-        e_ev[i][0].record(stream)
-        for n in d:
-            d[n].copy_(h[n], non_blocking=True)
-        ds = step(d)[4]
-        out_h.copy_(ds, non_blocking=True)
-        e_ev[i][1].record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = D.max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev) / args.steps, dev)
-    e2e_val = world * (f_fwd + f_bwd) / (e2e_ms * 1e-3) / 1e12
+    # ---- e2e: host buffers in, every result out, through the same calls.
+    # Three streams (host-to-device copies, compute, device-to-host copies)
+    # and two device buffer sets, so step i's inputs cross PCIe while step
+    # i - 1 computes and its results come back; the value is K steps over the
+    # time from the first copy to the last result on the host side.
+    e2e = run_e2e(S, torch, dev, h, d, step, args, world, f_fwd + f_bwd)
 
     # ---- decode lines (one call per timing, L2 flushed before each)
     decode_lines = []
     if not args.no_decode:
         decode_lines = bench_decode(S, torch, dev, stream, flush, peaks, args, rank)
+
+    # ---- the Qwen3-8B training layer (device-timed; median of its steps)
+    other_train = []
+    if not args.no_8b:
+        other_train.append(run_train_line(S, torch, dev, W.QWEN3_8B_TRAIN, flush, peaks,
+                                          max(3, min(args.steps, 10)), 2, rank))
 
     # ---- roofline of the dominant call of the training step
     dom = max(k_ms, key=k_ms.get)
@@ -310,23 +383,137 @@ def run_ours(args):
                    "algorithmic_tflop_per_step": (f_fwd + f_bwd) / 1e12},
         "kernels_ms": k_ms,
         "roofline": roof,
-        "e2e": {"value": e2e_val, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clocks,
         "decode": decode_lines,
+        "train_other": other_train,
         "wall_s_timed": t_wall,
     }
     if rank == 0 and world == 1 and not args.no_cpu:
-        kvh = tuple(range(args.cpu_heads))
-        secs, fl = oracle_sample(cfg, kvh, x)
-        line["cpu_baseline"] = {"value": fl / secs / 1e12, "unit": "TFLOP/s",
-                                "cores": blas_threads(), "kind": "oracle",
-                                "sample": f"float64 oracle, gates+top-k+fwd+bwd of {len(kvh)} of "
-                                          f"{cfg.Hkv} KV heads of {cfg.name} ({secs:.1f} s)"}
+        line["cpu_baseline"] = cpu_baseline(cfg, x, args.cpu_heads)
     if rank == 0:
         print(json.dumps(line), flush=True)
     D.shutdown()
+
+
+def cpu_baseline(cfg, x, heads):
+    """The float64 oracle on the host: `heads` KV heads with every BLAS thread,
+    and one KV head on one thread."""
+    kvh = tuple(range(heads))
+    secs, fl = oracle_sample(cfg, kvh, x)
+    out = {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+           "kind": "oracle", "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
+           "sample": f"float64 oracle, gates+top-k+fwd+bwd of {len(kvh)} of "
+                     f"{cfg.Hkv} KV heads of {cfg.name} ({secs:.1f} s)"}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            s1, f1 = oracle_sample(cfg, (0,), x)
+        out["single_thread"] = {"value": f1 / s1 / 1e12, "unit": "TFLOP/s", "cores": 1,
+                                "sample": f"one KV head on one BLAS thread ({s1:.1f} s)"}
+    except Exception as e:  # threadpoolctl missing: report the all-thread figure only
+        out["single_thread"] = {"unavailable": str(e)}
+    return out
+
+
+def run_e2e(S, torch, dev, h, d, step, args, world, flops):
+    """End-to-end training steps from pinned host buffers: inputs copied in,
+    gate + Top-K, forward and backward through the library, and every result
+    (o, dq, dk, dv, dscores) copied back to pinned host memory."""
+    s_in = torch.cuda.Stream(dev)
+    s_comp = torch.cuda.current_stream(dev)
+    s_out = torch.cuda.Stream(dev)
+    bufs = [d, {n: torch.empty_like(t) for n, t in d.items()}]
+    outs = None
+    in_ev = [torch.cuda.Event() for _ in range(2)]
+    done_ev = [torch.cuda.Event() for _ in range(2)]
+    back_ev = [torch.cuda.Event() for _ in range(2)]
+    names = ("o", "dq", "dk", "dv", "dscores")
+    K = args.steps
+    h2d = sum(t.numel() * t.element_size() for t in h.values())
+
+    def one(i, t0=None):
+        nonlocal outs
+        b = i % 2
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(done_ev[b])  # step i - 2 has finished with this buffer set
+            if t0 is not None:
+                t0.record(s_in)
+            for n in bufs[b]:
+                bufs[b][n].copy_(h[n], non_blocking=True)
+            in_ev[b].record(s_in)
+        s_comp.wait_event(in_ev[b])
+        res = step(bufs[b])
+        done_ev[b].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(done_ev[b])
+            if outs is None:
+                outs = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in res]
+                        for _ in range(2)]
+            if i >= 2:
+                back_ev[b].synchronize()  # the host has the results of step i - 2
+            for dst, src in zip(outs[b], res):
+                dst.copy_(src, non_blocking=True)
+                src.record_stream(s_out)
+            back_ev[b].record(s_out)
+
+    for i in range(2):
+        one(i)
+    torch.cuda.synchronize(dev)
+    D.barrier(dev)
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(K):
+        one(i, t0 if i == 0 else None)
+    t1.record(s_out)
+    torch.cuda.synchronize(dev)
+    ms = D.max_over_ranks(t0.elapsed_time(t1) / K, dev)
+    d2h = sum(t.numel() * t.element_size() for t in outs[0])
+    return {"value": world * flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "results_copied": list(names),
+            "overlap": "copy-in, compute and copy-out on three streams, two buffer sets"}
+
+
+def run_train_line(S, torch, dev, cfg, flush, peaks, steps, warmup, rank):
+    """Device-timed training steps of another layer shape (L2 flushed before each)."""
+    x = W.make_train_inputs(cfg, seed=D.rank_seed(cfg.seed, rank))
+    bf = torch.bfloat16
+    t = {n: torch.from_numpy(getattr(x, n)).to(bf).to(dev) for n in ("q", "k", "v", "dO")}
+    t["scores"] = torch.from_numpy(x.scores).to(dev)
+    del x
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        gates, idx = S.gate_topk(t["scores"], cfg.K, causal=True)
+        o, lse = S.attn_fwd(t["q"], t["k"], t["v"], idx, gates, cfg.b)
+        if ev:
+            ev[1].record(stream)
+        S.attn_bwd(t["q"], t["k"], t["v"], o, lse, t["dO"], idx, gates, cfg.b)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(warmup):
+        step()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        torch.cuda._sleep(HEAD_START_CYCLES)
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    f_fwd, f_bwd = train_flops(cfg)
+    fwd_ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
+    ms = fwd_ms + bwd_ms
+    tf = (f_fwd + f_bwd) / (ms * 1e-3) / 1e12
+    del t
+    torch.cuda.empty_cache()
+    return {"workload": cfg.name, "ms_per_step": ms, "gate_fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+            "TFLOP/s": tf, "frac": tf / peaks["bf16_tflops"],
+            "algorithmic_tflop_per_step": (f_fwd + f_bwd) / 1e12}
 
 
 def bench_decode(S, torch, dev, stream, flush, peaks, args, rank):
@@ -468,6 +655,41 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def _free_port() -> int:
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def relaunch(n: int) -> int:
+    """Runs this script again under torch.distributed.run with n ranks (one
+    per GPU) on 127.0.0.1 and returns its exit code."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()),
+           os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
+def run_dry(args):
+    """The launch and timing plumbing without a GPU: gloo ranks time a small
+    host-side step, reduce the max over ranks, and rank 0 prints a JSON line."""
+    rank, _, world = D.env_rank()
+    D.init("gloo", timeout_s=60)
+    a = np.random.default_rng(D.rank_seed(0, rank)).standard_normal((256, 256))
+    for _ in range(args.warmup):
+        a @ a
+    D.barrier()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        a @ a
+    ms = D.max_over_ranks(1e3 * (time.perf_counter() - t) / max(1, args.steps))
+    if rank == 0:
+        print(json.dumps({"dry_run": True, "n_gpus": world, "steps": args.steps,
+                          "warmup": args.warmup, "ms_per_step": ms, "scaling": "weak"}),
+              flush=True)
+    D.shutdown()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -481,10 +703,17 @@ def main():
                     help="time only the decode path of one preset (for profiling)")
     ap.add_argument("--profile-train", type=int, default=0, metavar="T",
                     help="run only the training step at sequence length T (for profiling)")
+    ap.add_argument("--no-8b", action="store_true", help="skip the Qwen3-8B training line")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="CPU only: exercise the rank launch and timing reduction on gloo")
     args = ap.parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        raise SystemExit(relaunch(args.gpus))
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
-    if args.impl == "reference":
+    if args.dry_run:
+        run_dry(args)
+    elif args.impl == "reference":
         run_reference(args)
     elif args.decode_only:
         run_decode_only(args)

@@ -60,8 +60,8 @@ __device__ __forceinline__ bool pick_block(const AttnShape& s, const int32_t* id
     return true;
   }
   m = idx[idx_row(s, bi, kvh, j) * s.K + it];
-  if (m < 0) return false;
-  if (m >= j) {
+  if (m == -1) return false;
+  if (m < -1 || m >= j) {
     if (threadIdx.x == 0) report(ctx, kDevErrBadIndex);
     return false;
   }

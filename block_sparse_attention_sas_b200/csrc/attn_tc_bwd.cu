@@ -8,20 +8,29 @@
 //   da(j,m) = sum of dS over the (query block j, key block m) tile, all G
 //   heads -- equal to g_m * dg_m of Eq. 5 (Gradient Analysis, inner form) --
 //   which the gate Jacobian of Eq. 6 then turns into d scores.
-// D is summed exactly from P and dP (a first sweep of kernel A) instead of
-// dO . o from the stored bf16 o, whose rounding would reach every gradient.
+// D is summed exactly from P and dP instead of taken as dO . o from the
+// stored bf16 o, whose rounding would reach every gradient.
 //
-// Kernel A (query-outer), one CTA per (query block j, 128-row tile of two
-//   heads, KV head, batch): sweep 1 over the attended blocks sums D; sweep 2
-//   forms dS, accumulates dQ += dS K in TMEM (K read as an MN-major operand)
-//   and the tile's sum of dS per selected block; writes dq, D and da.
-// Kernel B (key-outer), one CTA per (key block m, KV head, batch): over the
-//   diagonal block and every query block whose selection holds m (a reverse
-//   index), per 128-row tile: S = Q K^T and dP = dO V^T into TMEM, P and dS
-//   into swizzled shared memory, then dV^T += dO^T P and dK^T += Q^T dS with
-//   the Q / dO tiles read again as MN-major operands (no transposes).
-// Warp roles as in the forward: warp 0 TMA producer, warp 1 MMA issuer,
-// warps 4-7 the elementwise work, one thread per tile row. Waits are bounded.
+// Three kernels, run in this order after the reverse index (for each key
+// block, the query blocks that selected it) and a launch order:
+//   tc_bwd_d_kernel (query-outer), one CTA per (query block j, 128-row tile
+//     of two heads, KV head, batch): S = Q K^T and dP = dO V^T per attended
+//     block, D_i = sum_t P_it dP_it; writes D.
+//   tc_bwd_dkdv_kernel (key-outer), one CTA per (key block m, KV head,
+//     batch): over the diagonal block and every query block whose selection
+//     holds m, per 128-row tile: S and dP into TMEM, P and dS into swizzled
+//     shared memory, then dV^T += dO^T P and dK^T += Q^T dS with the Q / dO
+//     tiles read again as MN-major operands (no transposes). It writes dk,
+//     dv, every dS tile (bf16, 16 KB) to the workspace, and the tile's sum of
+//     dS per selected block (da) in eight fixed shares.
+//   tc_bwd_dq_kernel (query-outer), one CTA per (query block, 128-row tile,
+//     KV head, batch): dq = scale * sum over the attended blocks of dS K from
+//     the stored tiles; no recomputation.
+// The gate Jacobian (a separate small kernel) turns da into d scores.
+// Every result comes from one CTA in a fixed order: no atomics, so the
+// gradients are deterministic. Warp roles: a TMA producer warp, one MMA
+// issuing thread, elementwise warps with one thread per tile row (TMEM
+// lane). Every wait is bounded.
 #include <math.h>
 
 #include "sas_internal.h"

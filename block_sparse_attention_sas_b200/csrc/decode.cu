@@ -84,8 +84,8 @@ __device__ __forceinline__ int slot_block(const DecodeShape& s, const int32_t* i
   if (s.dense) return sl;
   if (sl == s.K) return s.C;
   const int m = ix[sl];
-  if (m < 0) return -1;
-  if (m >= s.C) {
+  if (m == -1) return -1;
+  if (m < -1 || m >= s.C) {
     report(ctx, kDevErrBadIndex);
     return -1;
   }

@@ -125,7 +125,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           m = s.dense ? sl : s.C;
         } else {
           m = ix[sl];
-          if (m >= s.C) {
+          if (m >= s.C || m < -1) {
             report(ctx, kDevErrBadIndex);
             m = -1;
           } else if (m >= 0 && s.use_gates) {

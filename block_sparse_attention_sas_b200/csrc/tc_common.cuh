@@ -281,7 +281,8 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // The attended-block list of one query block, built by one full warp: lane
 // l reads idx slot base + l, valid entries (0 <= m < j) are compacted in slot
 // order after `first` already-placed entries, with their log2-domain gate
-// bias (0 without gates); entries >= j are reported. Returns the list length.
+// bias (0 without gates); entries >= j or below -1 (-1 marks an empty slot)
+// are reported and skipped. Returns the list length.
 __device__ __forceinline__ int warp_build_list(const int32_t* idx_row, const float* gate_row,
                                                int K, int j, int first, int* blocks, int* slots,
                                                float* bias, const DevCtx& ctx) {
@@ -290,7 +291,7 @@ __device__ __forceinline__ int warp_build_list(const int32_t* idx_row, const flo
   for (int base = 0; base < K; base += 32) {
     const int sl = base + lane;
     const int m = sl < K ? idx_row[sl] : -1;
-    const bool bad = m >= j;
+    const bool bad = m >= j || m < -1;
     if (bad) report(ctx, kDevErrBadIndex);
     const bool ok = m >= 0 && !bad;
     const float g = (ok && gate_row) ? gate_row[m] : 1.f;

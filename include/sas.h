@@ -113,7 +113,8 @@ sas_status_t sas_gate_topk(const float* scores, int B, int Hkv, int rows, int C,
  *
  *   q [B, Hq, T, d]; k, v [B, Hkv, T, d] (dtype; read).
  *   idx [B, Hkv, N, K] int32: entries -1 are skipped; every other entry of
- *     row j must satisfy 0 <= m < j (checked on the device: SAS_ERR_DEVICE).
+ *     row j must satisfy 0 <= m < j (checked on the device: an entry >= j or
+ *     below -1 is skipped and reported as SAS_ERR_DEVICE).
  *   gates [B, Hkv, N, N] fp32 or NULL: row j holds g_{j,m} (as written by
  *     sas_gate_topk with causal = 1). A zero gate masks its block.
  *   o [B, Hq, T, d] (dtype; written); lse [B, Hq, T] fp32 (written): the
@@ -162,7 +163,8 @@ sas_status_t sas_attn_bwd(sas_dtype_t dtype, const void* q, const void* k, const
  *   q [B, Hq, d] (dtype). kcache, vcache [B, Hkv, Lcap, d] (dtype), positions
  *     0..L-1 valid, L <= Lcap.
  *   idx [B, Hkv, K] int32 over 0..C-1, -1 skipped (as written by
- *     sas_gate_topk with causal = 0, rows = 1).
+ *     sas_gate_topk with causal = 0, rows = 1); an entry >= C or below -1 is
+ *     skipped and reported as SAS_ERR_DEVICE.
  *   gates [B, Hkv, C] fp32; read only when use_gates != 0 (may be NULL otherwise).
  *   o [B, Hq, d] (dtype; written).
  *   ws / ws_bytes: at least sas_decode_workspace_size() bytes, 256-byte
@@ -189,8 +191,13 @@ sas_status_t sas_decode(sas_dtype_t dtype, const void* q, const void* kcache, co
  * counterpart; it is a deployment convenience of this library.
  *   - The call itself allocates nothing: no cudaMalloc, cudaFree or
  *     allocating library routine. Its first call on a device looks up the
- *     array's device address (once per device, with that device current);
- *     make that first call before any stream capture.
+ *     array's device address (once per device, with that device current).
+ *     That first call (like the first call of any entry point on a device)
+ *     is also when the CUDA runtime loads the library's device code onto the
+ *     device: the loader reserves the array and the code in device memory,
+ *     an allocation the runtime makes, and may synchronise the device. Make
+ *     one warm-up call per device at initialisation, before serving starts
+ *     and before any stream capture, so that later calls do none of this.
  *   - Every call on a device shares the one array and it keeps the last
  *     call's contents; the call clears the part that must start at zero.
  *     Calls that overlap on the GPU (other streams, other host threads) race

@@ -2,9 +2,11 @@
 
 Tolerances (stated by the workload definitions, read as follows):
   * fp32 tensors of an fp32 workload: max|x - y| / max|y| <= 1e-4 (normwise).
-  * tensors of a bf16 workload: every element |x - y| <= 2e-2 + 2^-8 |y|
-    (the absolute bound on top of half an ulp of the stored bf16 value,
-    which alone exceeds 2e-2 once |y| >= 8), and ||x - y||_2 / ||y||_2 <= 1e-2.
+  * tensors of a bf16 workload: every element |x - y| <= 2e-2, and
+    ||x - y||_2 / ||y||_2 <= 1e-2. A tensor the library stores in bf16 (o,
+    dq, dk, dv) may in addition be off by half an ulp of its stored value,
+    2^-8 |y|, which alone exceeds 2e-2 once |y| >= 8. fp32-stored outputs of
+    a bf16 workload (lse, dscores) get the plain 2e-2 bound.
   * indices: bit-exact.
 """
 from __future__ import annotations
@@ -31,7 +33,11 @@ def host(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def check(name: str, got, want, dtype: str):
+def check(name: str, got, want, dtype: str, stored: str | None = None):
+    """Compare at the workload's tolerance. `stored` is the dtype the library
+    writes the tensor in (defaults to the workload dtype); the half-ulp
+    allowance applies only to bf16-stored tensors."""
+    stored = dtype if stored is None else stored
     got = np.asarray(got, np.float64)
     want = np.asarray(want, np.float64)
     assert got.shape == want.shape, (name, got.shape, want.shape)
@@ -42,9 +48,10 @@ def check(name: str, got, want, dtype: str):
         rel = err.max() / max(scale, 1e-30) if want.size else 0.0
         assert rel <= F32_NORMWISE, f"{name}: normwise rel err {rel:.3e} > {F32_NORMWISE}"
         return rel
-    excess = (err - BF16_RTOL_ULP * np.abs(want)).max() if want.size else 0.0
+    ulp = BF16_RTOL_ULP if stored == "bf16" else 0.0
+    excess = (err - ulp * np.abs(want)).max() if want.size else 0.0
     l2 = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
-    assert excess <= BF16_ATOL, f"{name}: max abs err beyond bf16 rounding {excess:.3e} > {BF16_ATOL}"
+    assert excess <= BF16_ATOL, f"{name}: max abs err {excess:.3e} > {BF16_ATOL} (stored {stored})"
     assert l2 <= BF16_REL_L2, f"{name}: rel L2 err {l2:.3e} > {BF16_REL_L2}"
     return l2
 

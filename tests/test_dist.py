@@ -105,3 +105,22 @@ def test_gloo_two_ranks_sharded_units(tmp_path):
         np.testing.assert_array_equal(udk[0, 0], dk[bi, h])
         np.testing.assert_array_equal(udv[0, 0], dv[bi, h])
         np.testing.assert_array_equal(uds[0, 0], ds[bi, h])
+
+
+def test_bench_gpus_flag_launches_ranks_itself():
+    """`bench.py --gpus 2` without a torchrun environment re-launches itself
+    with two ranks; the dry run does the rank plumbing on gloo/CPU."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2",
+                        "--dry-run", "--steps", "2", "--warmup", "1"],
+                       capture_output=True, text=True, timeout=300, env=env, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    out = json.loads(lines[0])
+    assert out["n_gpus"] == 2 and out["dry_run"] is True

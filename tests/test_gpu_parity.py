@@ -83,12 +83,12 @@ def _full_compare(lib, cfg, use_gates=True):
     dq, dk, dv, ds = O.attn_bwd(x.q, x.k, x.v, x.dO, ix, g, lg, cfg.b, use_gates=use_gates)
     dt = cfg.dtype
     check("o", host(r["o"]), o, dt)
-    check("lse", host(r["lse"]), lse, dt)
+    check("lse", host(r["lse"]), lse, dt, stored="f32")
     check("dq", host(r["dq"]), dq, dt)
     check("dk", host(r["dk"]), dk, dt)
     check("dv", host(r["dv"]), dv, dt)
     if use_gates:
-        check("dscores", host(r["ds"]), ds, dt)
+        check("dscores", host(r["ds"]), ds, dt, stored="f32")
     else:
         assert r["ds"] is None
 
@@ -106,6 +106,11 @@ def test_tiny_f32_config_full(cuda_lib):
     dict(B=1, Hq=5, Hkv=1, T=320, d=64, b=64, K=2, dtype="bf16"),
     dict(B=1, Hq=3, Hkv=3, T=64, d=128, b=64, K=4, dtype="bf16"),   # single block, j = 0 only
     dict(B=1, Hq=2, Hkv=1, T=77, d=64, b=16, K=1, dtype="f32"),
+    # G = 2 on the tensor-core kernels (one 128-row tile per query block):
+    # ragged T, 10% hot key blocks
+    dict(B=1, Hq=8, Hkv=4, T=1000, d=128, b=64, K=3, dtype="bf16", hot_key_frac=0.1,
+         hot_key_scale=3.0),
+    dict(B=2, Hq=4, Hkv=2, T=700, d=128, b=64, K=5, dtype="bf16"),
 ])
 @pytest.mark.parametrize("use_gates", [True, False])
 def test_train_small_full(cuda_lib, kw, use_gates):
@@ -129,16 +134,26 @@ def test_train_full_size_sampled(cuda_lib, name):
             o, lse = oracle_fwd_rows(x, b, cfg.K, bi, kvh, j, cache=cache)
             sl = slice(j * b, (j + 1) * b)
             check(f"o[{j}]", host(r["o"][bi, kvh * G:(kvh + 1) * G, sl]), o, cfg.dtype)
-            check(f"lse[{j}]", host(r["lse"][bi, kvh * G:(kvh + 1) * G, sl]), lse, cfg.dtype)
+            check(f"lse[{j}]", host(r["lse"][bi, kvh * G:(kvh + 1) * G, sl]), lse, cfg.dtype,
+                  stored="f32")
         ob = oracle_bwd_sample(x, b, cfg.K, bi, kvh, js, ms, cache=cache)
         for j in js:
             sl = slice(j * b, (j + 1) * b)
             check(f"dq[{j}]", host(r["dq"][bi, kvh * G:(kvh + 1) * G, sl]), ob["dq"][j], cfg.dtype)
-            check(f"ds[{j}]", host(r["ds"][bi, kvh, j]), ob["ds"][j], cfg.dtype)
+            check(f"ds[{j}]", host(r["ds"][bi, kvh, j]), ob["ds"][j], cfg.dtype, stored="f32")
         for m in ms:
             sl = slice(m * b, (m + 1) * b)
             check(f"dk[{m}]", host(r["dk"][bi, kvh, sl]), ob["dk"][m], cfg.dtype)
             check(f"dv[{m}]", host(r["dv"][bi, kvh, sl]), ob["dv"][m], cfg.dtype)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_train_reverse_index_past_1024_blocks(cuda_lib, dtype):
+    """N = 1025 query blocks: the backward builds its reverse index with the
+    warp-ranked list kernel (the bitmap one covers N <= 1024)."""
+    cfg = W.small_train_config(B=1, Hq=2, Hkv=1, T=16400, d=64, b=16, K=2, dtype=dtype)
+    assert cfg.N > 1024
+    _full_compare(cuda_lib, cfg, True)
 
 
 def test_dense_matches_all_blocks_selected(cuda_lib):
@@ -151,7 +166,7 @@ def test_dense_matches_all_blocks_selected(cuda_lib):
     idx = O.all_blocks_idx(1, 2, cfg.N)
     odq, odk, odv, _ = O.attn_bwd(x.q, x.k, x.v, x.dO, idx, None, None, 64, use_gates=False)
     check("dense o", host(o), oo, "bf16")
-    check("dense lse", host(lse), ol, "bf16")
+    check("dense lse", host(lse), ol, "bf16", stored="f32")
     check("dense dq", host(dq), odq, "bf16")
     check("dense dk", host(dk), odk, "bf16")
     check("dense dv", host(dv), odv, "bf16")
@@ -184,6 +199,7 @@ def _decode_case(lib, dc, use_gates, dense_too=False):
     dict(B=1, Hq=8, Hkv=1, L=64, d=128, b=64, K=2, dtype="bf16"),     # no history
     dict(B=1, Hq=2, Hkv=2, L=65, d=128, b=64, K=2, dtype="bf16"),     # 1 token current block
     dict(B=2, Hq=12, Hkv=4, L=4099, d=128, b=32, K=200, dtype="bf16"),
+    dict(B=2, Hq=16, Hkv=2, L=5000, d=128, b=64, K=16, dtype="bf16"),  # G = 8 with history
     dict(B=1, Hq=1, Hkv=1, L=50000, d=64, b=64, K=7, dtype="f32"),
 ])
 @pytest.mark.parametrize("use_gates", [False, True])
@@ -208,6 +224,31 @@ def test_bad_index_is_reported_not_faulted(cuda_lib):
     idx[0, 0, 1, 0] = 3   # block 3 is not in the history of block 1
     cuda_lib.device_error()
     cuda_lib.attn_fwd(q, k, v, idx, None, cfg.b)
+    st, raw = cuda_lib.device_error()
+    assert st == 6 and raw & 2
+
+
+@pytest.mark.parametrize("path", ["simt", "tc"])
+def test_negative_index_other_than_minus_one_is_reported(cuda_lib, path):
+    """-1 marks an empty slot; any other negative entry is a bad index."""
+    if path == "simt":
+        cfg = W.small_train_config(B=1, Hq=2, Hkv=1, T=128, d=64, b=32, K=2, dtype="f32")
+    else:
+        cfg = W.small_train_config(B=1, Hq=4, Hkv=1, T=256, d=128, b=64, K=2, dtype="bf16")
+    x = W.make_train_inputs(cfg)
+    q, k, v = (dev(a, cfg.dtype) for a in (x.q, x.k, x.v))
+    idx = torch.full((1, 1, cfg.N, 2), -1, dtype=torch.int32, device="cuda")
+    idx[0, 0, 2, 1] = -5
+    cuda_lib.device_error()
+    cuda_lib.attn_fwd(q, k, v, idx, None, cfg.b)
+    st, raw = cuda_lib.device_error()
+    assert st == 6 and raw & 2
+    dc = W.small_decode_config(B=1, Hq=4, Hkv=1, L=1000, d=128, b=64, K=4,
+                               dtype=cfg.dtype if path == "tc" else "f32")
+    xd = W.make_decode_inputs(dc)
+    qd, kc, vc = (dev(a, dc.dtype) for a in (xd.q, xd.kcache, xd.vcache))
+    ix = torch.tensor([[[0, -7, 3, -1]]], dtype=torch.int32, device="cuda")
+    cuda_lib.decode(qd, kc, vc, ix, None, False, dc.b, L=dc.L)
     st, raw = cuda_lib.device_error()
     assert st == 6 and raw & 2
 
