@@ -17,6 +17,8 @@ import torch
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsas_b200.so")
 
 SAS_F32, SAS_BF16 = 0, 1
+PHI = {"softmax": 0, "sigmoid": 1, "raw": 2}
+GATING = {"inner": 0, "outer": 1}
 STATUS = {0: "SAS_OK", 1: "SAS_ERR_INVALID_ARG", 2: "SAS_ERR_UNSUPPORTED", 3: "SAS_ERR_CUDA",
           4: "SAS_ERR_TIMEOUT", 5: "SAS_ERR_WORKSPACE", 6: "SAS_ERR_DEVICE"}
 
@@ -35,6 +37,11 @@ SIGNATURES = {
     "sas_version": (_i, []),
     "sas_launch_count": (ctypes.c_uint64, []),
     "sas_gate_topk": (_i, [_p, _i, _i, _i, _i, _i, _i, _p, _p, _p]),
+    "sas_gate_topk_phi": (_i, [_p, _i, _i, _i, _i, _i, _i, _i, _p, _p, _p]),
+    "sas_attn_fwd_gated": (_i, [_i, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _i, _p,
+                                _p, _p]),
+    "sas_attn_bwd_gated": (_i, [_i, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i,
+                                _f, _i, _i, _p, _p, _p, _p, _p, _sz, _p]),
     "sas_attn_fwd": (_i, [_i, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p]),
     "sas_attn_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i]),
     "sas_attn_bwd": (_i, [_i, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f,
@@ -45,6 +52,9 @@ SIGNATURES = {
     "sas_decode_noalloc": (_i, [_i, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                                 _p, _p]),
     "sas_decode_noalloc_max_scratch": (_sz, []),
+    "sas_decode_paged_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "sas_decode_paged": (_i, [_i, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i,
+                              _i, _i, _i, _f, _p, _p, _sz, _p]),
     "sas_dense_fwd": (_i, [_i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p]),
     "sas_dense_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "sas_dense_bwd": (_i, [_i, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p,
@@ -119,21 +129,31 @@ def _workspace(kind: str, nbytes: int, device, zero: bool) -> torch.Tensor:
 
 # ---------------------------------------------------------------------------
 
-def gate_topk(scores: torch.Tensor, K: int, causal: bool = True, gates=None, idx=None):
-    """Gates [B,Hkv,R,C] fp32 and Top-K indices [B,Hkv,R,K] int32 of `scores`."""
+def gate_topk(scores: torch.Tensor, K: int, causal: bool = True, gates=None, idx=None,
+              phi: str = "softmax"):
+    """Gates [B,Hkv,R,C] fp32 and Top-K indices [B,Hkv,R,K] int32 of `scores`
+    (phi: the gate activation, "softmax" for the method, "sigmoid" / "raw"
+    for the ablation variants)."""
     _need(scores, "scores", torch.float32)
     B, H, R, C = scores.shape
     if gates is None:
         gates = torch.empty_like(scores)
     if idx is None:
         idx = torch.empty((B, H, R, K), dtype=torch.int32, device=scores.device)
-    _check("sas_gate_topk", LIB.sas_gate_topk(_ptr(scores), B, H, R, C, int(causal), K,
-                                              _ptr(gates), _ptr(idx), _stream(scores.device)))
+    if phi == "softmax":
+        _check("sas_gate_topk", LIB.sas_gate_topk(_ptr(scores), B, H, R, C, int(causal), K,
+                                                  _ptr(gates), _ptr(idx), _stream(scores.device)))
+    else:
+        _check("sas_gate_topk_phi",
+               LIB.sas_gate_topk_phi(_ptr(scores), B, H, R, C, int(causal), K, PHI[phi],
+                                     _ptr(gates), _ptr(idx), _stream(scores.device)))
     return gates, idx
 
 
-def attn_fwd(q, k, v, idx, gates, b: int, scale: float = 0.0, o=None, lse=None):
-    """Gated sparse forward. Returns (o, lse)."""
+def attn_fwd(q, k, v, idx, gates, b: int, scale: float = 0.0, o=None, lse=None,
+             gating: str = "inner"):
+    """Gated sparse forward (gating "inner" is the method's Eq. 9; "outer"
+    the ablation variant). Returns (o, lse)."""
     for n, t in (("q", q), ("k", k), ("v", v)):
         _need(t, n, q.dtype)
     _need(idx, "idx", torch.int32)
@@ -145,15 +165,22 @@ def attn_fwd(q, k, v, idx, gates, b: int, scale: float = 0.0, o=None, lse=None):
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
-    _check("sas_attn_fwd", LIB.sas_attn_fwd(_dtype(q), _ptr(q), _ptr(k), _ptr(v), _ptr(idx),
-                                            _ptr(gates), B, Hq, Hkv, T, d, b, K, scale, _ptr(o),
-                                            _ptr(lse), _stream(q.device)))
+    if gating == "inner":
+        _check("sas_attn_fwd", LIB.sas_attn_fwd(_dtype(q), _ptr(q), _ptr(k), _ptr(v), _ptr(idx),
+                                                _ptr(gates), B, Hq, Hkv, T, d, b, K, scale,
+                                                _ptr(o), _ptr(lse), _stream(q.device)))
+    else:
+        _check("sas_attn_fwd_gated",
+               LIB.sas_attn_fwd_gated(_dtype(q), _ptr(q), _ptr(k), _ptr(v), _ptr(idx),
+                                      _ptr(gates), B, Hq, Hkv, T, d, b, K, scale, GATING[gating],
+                                      _ptr(o), _ptr(lse), _stream(q.device)))
     return o, lse
 
 
 def attn_bwd(q, k, v, o, lse, dO, idx, gates, b: int, scale: float = 0.0,
-             want_dscores: bool = True):
-    """Backward. Returns (dq, dk, dv, dscores or None)."""
+             want_dscores: bool = True, phi: str = "softmax", gating: str = "inner"):
+    """Backward (phi and gating as passed to gate_topk and attn_fwd).
+    Returns (dq, dk, dv, dscores or None)."""
     for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dO", dO)):
         _need(t, n, q.dtype)
     _need(lse, "lse", torch.float32)
@@ -167,10 +194,19 @@ def attn_bwd(q, k, v, o, lse, dO, idx, gates, b: int, scale: float = 0.0,
         ds = torch.empty((B, Hkv, N, N), dtype=torch.float32, device=q.device)
     nbytes = LIB.sas_attn_bwd_workspace_size(_dtype(q), B, Hq, Hkv, T, d, b, K)
     ws = _workspace("bwd", nbytes, q.device, zero=False)
-    _check("sas_attn_bwd", LIB.sas_attn_bwd(_dtype(q), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
-                                            _ptr(lse), _ptr(dO), _ptr(idx), _ptr(gates), B, Hq,
-                                            Hkv, T, d, b, K, scale, _ptr(dq), _ptr(dk), _ptr(dv),
-                                            _ptr(ds), _ptr(ws), ws.numel(), _stream(q.device)))
+    if phi == "softmax" and gating == "inner":
+        _check("sas_attn_bwd", LIB.sas_attn_bwd(_dtype(q), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                                _ptr(lse), _ptr(dO), _ptr(idx), _ptr(gates), B,
+                                                Hq, Hkv, T, d, b, K, scale, _ptr(dq), _ptr(dk),
+                                                _ptr(dv), _ptr(ds), _ptr(ws), ws.numel(),
+                                                _stream(q.device)))
+    else:
+        _check("sas_attn_bwd_gated",
+               LIB.sas_attn_bwd_gated(_dtype(q), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                      _ptr(dO), _ptr(idx), _ptr(gates), B, Hq, Hkv, T, d, b, K,
+                                      scale, PHI[phi], GATING[gating], _ptr(dq), _ptr(dk),
+                                      _ptr(dv), _ptr(ds), _ptr(ws), ws.numel(),
+                                      _stream(q.device)))
     return dq, dk, dv, ds
 
 
@@ -210,6 +246,31 @@ def decode_noalloc(q, kcache, vcache, idx, gates, use_gates: bool, b: int,
            LIB.sas_decode_noalloc(_dtype(q), _ptr(q), _ptr(kcache), _ptr(vcache), _ptr(idx),
                                   _ptr(gates), int(use_gates), B, Hq, Hkv, L, Lcap, d, b,
                                   idx.shape[-1], scale, _ptr(o), _stream(q.device)))
+    return o
+
+
+def decode_paged(q, kpages, vpages, page_indptr, page_indices, seq_lens, idx, gates,
+                 use_gates: bool, b: int, max_len: int, scale: float = 0.0, o=None):
+    """Sparse decode over a paged cache: q [B,Hq,d]; pages [num_pages,Hkv,P,d];
+    page_indptr [B+1], page_indices, seq_lens [B], idx [B,Hkv,K] int32;
+    gates [B,Hkv,(max_len-1)//b] fp32 or None."""
+    for n, t in (("q", q), ("kpages", kpages), ("vpages", vpages)):
+        _need(t, n, q.dtype)
+    for n, t in (("page_indptr", page_indptr), ("page_indices", page_indices),
+                 ("seq_lens", seq_lens), ("idx", idx)):
+        _need(t, n, torch.int32)
+    B, Hq, d = q.shape
+    num_pages, Hkv, P = kpages.shape[0], kpages.shape[1], kpages.shape[2]
+    K = idx.shape[-1]
+    if o is None:
+        o = torch.empty_like(q)
+    nbytes = LIB.sas_decode_paged_workspace_size(B, Hq, Hkv, max_len, d, b, K)
+    ws = _workspace("decode", nbytes, q.device, zero=False)
+    _check("sas_decode_paged",
+           LIB.sas_decode_paged(_dtype(q), _ptr(q), _ptr(kpages), _ptr(vpages), _ptr(page_indptr),
+                                _ptr(page_indices), _ptr(seq_lens), _ptr(idx), _ptr(gates),
+                                int(use_gates), B, Hq, Hkv, num_pages, P, max_len, d, b, K, scale,
+                                _ptr(o), _ptr(ws), ws.numel(), _stream(q.device)))
     return o
 
 

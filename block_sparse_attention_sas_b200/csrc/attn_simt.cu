@@ -116,6 +116,10 @@ fwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict
     float bias;
     bool cur;
     if (!pick_block(s, idx, gates, bi, kvh, j, it, nsel, m, bias, cur, ctx)) continue;
+    // Outer gating: the logits carry no bias and the block's weights are
+    // scaled by its gate w after the softmax.
+    const float w = s.outer ? expf(bias) : 1.f;
+    if (s.outer) bias = 0.f;
     __syncthreads();
     for (int e = tid; e < BS * D; e += kThreads) {
       const int t = e / D, c = e % D, key = m * BS + t;
@@ -144,7 +148,7 @@ fwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict
       float sum = 0.f;
       for (int c = lane; c < BS; c += 32) {
         const float p = (mnew == -INFINITY) ? 0.f : expf(Ps[r * BP + c] - mnew);
-        Ps[r * BP + c] = p;
+        Ps[r * BP + c] = p * w;
         sum += p;
       }
       sum = warp_sum(sum);
@@ -420,6 +424,7 @@ dq_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict_
       continue;
     }
     float dsum = 0.f;
+    const float dinv = s.outer ? fminf(expf(-bias), 3.0e38f) : 1.f;
     for (int e = tid; e < ROWS * BS; e += kThreads) {
       const int r = e / BS, c = e % BS;
       float a = 0.f, b = 0.f;
@@ -431,10 +436,12 @@ dq_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict_
       const int qi = r0 + r, ki = m * BS + c;
       float p = 0.f;
       if (qi < s.T && ki < s.T && !(cur && ki > qi)) p = expf(fmaf(a, s.scale, bias) - lse_s[r]);
-      const float ds = p * (b - D_s[r]);
+      // p is the gated weight (g p under outer gating). Inner: dS = p (dP - D);
+      // outer: dS = p (dP - D / g) and da sums p dP (Eq. 5, outer form, times g).
+      const float ds = p * (b - D_s[r] * dinv);
       Ps[r * BP + c] = p;
       dSs[r * BP + c] = ds;
-      dsum += ds;
+      dsum += s.outer ? p * b : ds;
     }
     if (!cur && !s.dense && da != nullptr) {
       dsum = warp_sum(dsum);
@@ -525,6 +532,7 @@ dkdv_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
       j = lst[it] / s.K;
       if (gates) bias = logf(gates[((long long)bh * s.N + j) * s.N + m]);
     }
+    const float dinv = s.outer ? fminf(expf(-bias), 3.0e38f) : 1.f;  // outer gating: dS = p (dP - D / g)
     for (int g = 0; g < G; ++g) {
       const int h = kvh * G + g;
       const long long qrow0 = (long long)(bi * s.Hq + h) * s.T;
@@ -556,7 +564,7 @@ dkdv_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
           float p = 0.f;
           if (qi < s.T && ki < s.T && !(cur && ki > qi)) p = expf(fmaf(a, s.scale, bias) - lse_s[r]);
           Ps[r * BP + c] = p;
-          dSs[r * BP + c] = p * (b - D_s[r]);
+          dSs[r * BP + c] = p * (b - D_s[r] * dinv);
         }
         __syncthreads();
 #pragma unroll
@@ -585,7 +593,8 @@ dkdv_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
 }
 
 // ---------------------------------------------------------------------------
-// Backward: gate-softmax Jacobian (Eq. 6), one warp per score row
+// Backward: gate Jacobian (Eq. 6 for the softmax gates; the sigmoid and
+// raw-logit variants have diagonal Jacobians), one warp per score row
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads)
 jacobian_kernel(const float* __restrict__ da, const int32_t* __restrict__ idx,
@@ -613,7 +622,10 @@ jacobian_kernel(const float* __restrict__ da, const int32_t* __restrict__ idx,
   tot = warp_sum(tot);
   float* out = ds + row * s.N;
   const float* g = gates + row * s.N;
-  for (int kk = lane; kk < s.N; kk += 32) out[kk] = (kk < j) ? -g[kk] * tot : 0.f;
+  // softmax: d log g_m / d s_k = delta_mk - g_k (Eq. 6); sigmoid: delta_mk
+  // (1 - g_k); raw logits: delta_mk. Only the softmax has the -g_k sum term.
+  const bool softmax = s.phi == SAS_PHI_SOFTMAX;
+  for (int kk = lane; kk < s.N; kk += 32) out[kk] = (kk < j && softmax) ? -g[kk] * tot : 0.f;
   __syncwarp();
   for (int sl = lane; sl < s.K; sl += 32) {
     const int m = ix[sl];
@@ -622,6 +634,7 @@ jacobian_kernel(const float* __restrict__ da, const int32_t* __restrict__ idx,
     for (int g2 = 0; g2 < G; ++g2)
       for (int rc = 0; rc < RC; ++rc)
         a += da[(((long long)(bi * s.Hq + kvh * G + g2) * s.N + j) * RC + rc) * s.K + sl];
+    if (s.phi == SAS_PHI_SIGMOID) a *= 1.f - g[m];
     out[m] += a;
   }
 }

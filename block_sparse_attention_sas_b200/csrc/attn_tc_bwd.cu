@@ -27,6 +27,9 @@
 //     KV head, batch): dq = scale * sum over the attended blocks of dS K from
 //     the stored tiles; no recomputation.
 // The gate Jacobian (a separate small kernel) turns da into d scores.
+// OUTER (outer gating, the ablation variant): P recomputed from the
+// ungated lse is the gated weight g p, so D and dV need no change; dS =
+// g p (dP - D / g) and da sums g p dP (Eq. 5, outer form, times g).
 // Every result comes from one CTA in a fixed order: no atomics, so the
 // gradients are deterministic. Warp roles: a TMA producer warp, one MMA
 // issuing thread, elementwise warps with one thread per tile row (TMEM
@@ -554,7 +557,7 @@ constexpr size_t kSmem = kCtlSpan + kTileBytes;
 static_assert(kSmem <= 232448, "over the per-block shared memory limit");
 }  // namespace kb_
 
-template <int TILES>
+template <int TILES, bool OUTER>
 __global__ void __launch_bounds__(kb_::kThreadsB, 1)
 tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k,
@@ -887,16 +890,18 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       fence_after_sync();
       uint64_t dsum = 0;
-      {  // dS = P (dP - D)
+      {  // dS = P (dP - D); outer gating: P (dP - D / g)
         uint32_t pr[32], dd[16];
         tmem_ld32(tl + kColDP + b * 64 + 32 * grp, pr);
         tmem_ld_wait();
-        const uint64_t negD = f2u(-Di, -Di);
+        const float dinv = OUTER ? fminf(ex2(-bias), 3.0e38f) : 1.f;
+        const uint64_t negD = f2u(-Di * dinv, -Di * dinv);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const uint64_t dp2 = f2u(__uint_as_float(pr[2 * i]), __uint_as_float(pr[2 * i + 1]));
-          const uint64_t ds2 = fmul2(f2u(pf[2 * i], pf[2 * i + 1]), fadd2(dp2, negD));
-          dsum = fadd2(dsum, ds2);
+          const uint64_t p2 = f2u(pf[2 * i], pf[2 * i + 1]);
+          const uint64_t ds2 = fmul2(p2, fadd2(dp2, negD));
+          dsum = OUTER ? ffma2(p2, dp2, dsum) : fadd2(dsum, ds2);
           dd[i] = pack_bf16(lo_f(ds2), hi_f(ds2));
         }
 #pragma unroll
@@ -1001,7 +1006,9 @@ cudaError_t launch_attn_bwd_tc(const AttnShape& s, const void* q, const void* k,
   }
   {  // dK, dV, dS tiles, da
     dim3 grid(s.N * s.Hkv * s.B);
-    auto kern = tiles == 2 ? tc_bwd_dkdv_kernel<2> : tc_bwd_dkdv_kernel<1>;
+    const bool outer = s.outer && gates != nullptr;
+    auto kern = tiles == 2 ? (outer ? tc_bwd_dkdv_kernel<2, true> : tc_bwd_dkdv_kernel<2, false>)
+                           : (outer ? tc_bwd_dkdv_kernel<1, true> : tc_bwd_dkdv_kernel<1, false>);
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kb_::kSmem);
     if (e != cudaSuccess) return e;
     kern<<<grid, kb_::kThreadsB, kb_::kSmem, st>>>(tq2, tk, tv, tdo2, lse, Dv, gates, coff, clist,

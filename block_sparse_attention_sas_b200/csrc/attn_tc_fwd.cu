@@ -23,6 +23,10 @@
 //               the current block goes first so the max starts high), P as
 //               bf16 into swizzled shared memory for the PV MMA; at the end
 //               O / l and the log-sum-exp go to global memory.
+// OUTER (the outer-gating ablation variant, evolve.pub review, Summary;
+// Eq. 5 outer form): the logits carry no gate bias, so the max, the sum and
+// lse are those of the ungated softmax, and P of a selected block is scaled
+// by its gate before the PV MMA.
 // Every wait is bounded; a wait that runs out sets the error word and a
 // CTA-wide abort flag, the roles drain their in-flight work and the CTA exits.
 #include <math.h>
@@ -78,7 +82,7 @@ __device__ __forceinline__ uint32_t q_col(int t) { return t * 64; }
 __device__ __forceinline__ uint32_t s_col(int t) { return 128 + t * 64; }
 __device__ __forceinline__ uint32_t o_col(int t) { return 256 + t * 128; }
 
-template <int TILES>
+template <int TILES, bool OUTER>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ idx,
@@ -263,7 +267,9 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       if (lane == 0 && n + 1 < nblk) mbar_arrive(&c.k_full[(n + 1) % kStages]);
 
       const int m = c.blocks[n];
-      const float bias = c.bias[n];
+      // Inner gating: log2 g joins the logits. Outer: P is scaled by g.
+      const float bias = OUTER ? 0.f : c.bias[n];
+      const float wgt = OUTER ? ex2(c.bias[n]) : 1.f;
       const bool cur = (n == 0);
       const int kvalid = min(kB, s.T - m * kB);   // keys of the block inside the sequence
       // Full history blocks need no mask; the current block (causal) and a
@@ -332,8 +338,13 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         acc0 = fadd2(acc0, f2u(p0, p1));
         acc1 = fadd2(acc1, f2u(p2, p3));
-        pk[i] = pack_bf16(p0, p1);
-        pk[i + 1] = pack_bf16(p2, p3);
+        if (OUTER) {
+          pk[i] = pack_bf16(p0 * wgt, p1 * wgt);
+          pk[i + 1] = pack_bf16(p2 * wgt, p3 * wgt);
+        } else {
+          pk[i] = pack_bf16(p0, p1);
+          pk[i + 1] = pack_bf16(p2, p3);
+        }
       }
       const uint64_t accs = fadd2(acc0, acc1);
       l += lo_f(accs) + hi_f(accs);
@@ -477,6 +488,23 @@ cudaError_t make_tmap_bf16_pitched(void* map_out, const void* ptr, int rows, int
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// Map over [planes][rows][128] bf16 with 64 x box_rows x 1 boxes, 128-byte
+// swizzle: the pages of a paged KV cache (rows = tokens per page).
+cudaError_t make_tmap_bf16_box(void* map_out, const void* ptr, int rows, int planes,
+                               int box_rows) {
+  CUtensorMap* map = static_cast<CUtensorMap*>(map_out);
+  EncodeTiled enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)rows, (cuuint64_t)planes};
+  const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)rows * kD * 2};
+  const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 bool tc_fwd_supported(sas_dtype_t dt, const AttnShape& s) {
   const int G = s.Hq / s.Hkv;
   return dt == SAS_BF16 && s.d == kD && s.b == kB && (G == 2 || G == 4) && !s.dense;
@@ -492,19 +520,12 @@ cudaError_t launch_attn_fwd_tc(const AttnShape& s, const void* q, const void* k,
   if ((e = make_tmap_bf16(&tv, v, s.T, s.B * s.Hkv)) != cudaSuccess) return e;
   const int G = s.Hq / s.Hkv;
   dim3 grid(s.N, s.Hkv, s.B);
-  if (G == 4) {
-    auto kern = tc_fwd_kernel<2>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, idx, gates, s, (__nv_bfloat16*)o, lse,
-                                             ctx);
-  } else {
-    auto kern = tc_fwd_kernel<1>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, idx, gates, s, (__nv_bfloat16*)o, lse,
-                                             ctx);
-  }
+  const bool outer = s.outer && gates != nullptr;  // no gates: both gatings coincide
+  auto kern = G == 4 ? (outer ? tc_fwd_kernel<2, true> : tc_fwd_kernel<2, false>)
+                     : (outer ? tc_fwd_kernel<1, true> : tc_fwd_kernel<1, false>);
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, idx, gates, s, (__nv_bfloat16*)o, lse, ctx);
   note_launches(1);
   return cudaGetLastError();
 }

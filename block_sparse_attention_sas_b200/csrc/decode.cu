@@ -453,15 +453,18 @@ void decode_plan(DecodeShape& s) {
   // pay less prologue and merge per block. 1 and 2 per SM were slower for the
   // Qwen3-14B 512K or the Qwen3-4B 64K decode. The dense comparison streams
   // long lists and keeps two per SM.
+  // A sparse call keeps at most 16 splits per unit, so the tensor-core
+  // decode can merge them inside one cluster.
   const int nslots = s.dense ? s.C + 1 : s.K + 1;
   const int units = s.B * s.Hkv;
   const int target = s.dense ? 2 * 148 : 3 * 148 / 2;
   int splits = target / units;
-  splits = max(1, min(splits, min(nslots, kMaxSplits)));
+  splits = max(1, min(splits, min(nslots, s.dense ? kMaxSplits : 16)));
   int bps = (nslots + splits - 1) / splits;
   splits = (nslots + bps - 1) / bps;
   s.splits = splits;
   s.bps = bps;
+  s.cluster = false;
 }
 
 size_t decode_workspace_bytes(const DecodeShape& s) {

@@ -24,10 +24,20 @@
 //           past that, so the softmax of block n + 1 never waits for PV(n)
 // TMEM: S[2] at columns 0 / 64, O at 128 (256 columns, so two CTAs share an
 // SM). Cache rows past L lie outside the tensor map and are read as zeros.
-// Partial (max, sum, o) of each split go to the workspace; the last CTA of a
-// (batch, KV head), found with an atomic ticket, merges them by log-sum-exp.
+// The splits of one (batch, KV head) merge their partial (max, sum, o) by
+// log-sum-exp. Up to 16 splits run as one thread-block cluster: each CTA
+// leaves its partial in its shared memory and, after a cluster barrier, CTA
+// r merges the heads g = r, r + splits, ... by reading the others' partials
+// through distributed shared memory (no workspace, no extra launch). More
+// splits (the long dense comparison) go through the workspace, where the last
+// CTA of the unit, found with an atomic ticket, merges them.
+// The kernel waits for the previous grid of the stream (programmatic
+// dependent launch) only once its prologue (barriers, TMEM, tensor-map
+// prefetch) is done, so that prologue overlaps the tail of the Top-K.
 // Every wait is bounded.
 #include <math.h>
+
+#include <mutex>
 
 #include "sas_internal.h"
 #include "tc_common.cuh"
@@ -46,6 +56,7 @@ constexpr int kProducerWarp = 2;
 constexpr uint32_t kTmemCols = 256;
 constexpr int kMaxG = 8;
 constexpr int kMaxSlotsPerSplit = 512;
+constexpr int kMaxClusterSplits = 16;  // largest (non-portable) cluster
 
 // Shared memory (offsets from a 1024-byte aligned base).
 constexpr int kStages = 3;
@@ -53,6 +64,7 @@ constexpr uint32_t kOffQ = 0;           // [k half][8 rows][128 B]
 constexpr uint32_t kOffKV = 2048;       // stages x (K halves 16 KB, V halves 16 KB)
 constexpr uint32_t kOffCtl = kOffKV + kStages * 32768;
 constexpr uint32_t kColS = 0, kColO = 128;
+constexpr int kSub = 4;  // most page boxes per 64-token block (pages of 16 tokens)
 
 struct Ctl {
   uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[2], p_full[2], o_full, o_final,
@@ -61,9 +73,22 @@ struct Ctl {
   int abort, nblk;
   int blocks[kMaxSlotsPerSplit];
   float bias[kMaxSlotsPerSplit];  // log2-domain gate bias
-  float wgt[kMaxG * 64];          // merge weights of the last CTA
+  union {
+    struct {
+      float wgt[kMaxG * 64];  // merge weights of the last CTA
+      // This split's partial for the cluster merge: unnormalised o per head.
+      float part_o[kMaxG][kD];
+    };
+    // Paged cache, while the blocks stream: the page of each of a block's
+    // sub-boxes (-1: nothing to load), kSub entries per block.
+    int pg[kMaxG * 64 + kMaxG * kD];
+  };
   float lsum[kMaxG];
   int last;
+  int Lseq;  // tokens of this unit's sequence
+  // Running max (log2 domain) and sum of this split's partial per head.
+  float part_m[kMaxG], part_l[kMaxG];
+  float mw[16], ml[16];  // the cluster's (max, sum) of the head being merged
 };
 constexpr size_t kSmem = kOffCtl + sizeof(Ctl) + 1024;
 
@@ -73,7 +98,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                  const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ idx,
                  const float* __restrict__ gates, DecodeShape s, __nv_bfloat16* __restrict__ o,
                  float* __restrict__ ws_ml, float* __restrict__ ws_o, uint32_t* __restrict__ ws_cnt,
-                 DevCtx ctx) {
+                 PagedArgs pa, DevCtx ctx) {
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   unsigned char* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -90,6 +115,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
       mbar_init(&c.q_full, 1);
       for (int i = 0; i < kStages; ++i) {
         mbar_init(&c.kv_full[i], 1);
@@ -105,27 +133,38 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       fence_mbar_init();
       c.abort = 0;
       c.last = 0;
-      tma_prefetch_desc(&tm_q);
+    }
+    // The inputs may come from the previous grid of the stream: nothing of
+    // them is read before it has completed.
+    grid_dependency_wait();
+    if (lane == 0) {
       mbar_arrive_expect_tx(&c.q_full, 2 * 1024);
       for (int kb = 0; kb < 2; ++kb)
         tma_load_3d(base + kOffQ + kb * 1024, &tm_q, kb * 64, (int)hbase, 0, &c.q_full);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
     }
     // The split's blocks in slot order: selected history blocks (bias log g
     // when gates are on), then the current block C; empty slots are skipped.
+    // A paged cache has its own length per sequence, so its own C.
     const int32_t* ix = s.dense ? nullptr : idx + (long long)unit * s.K;
+    int Lq = s.L, Cq = s.C;
+    bool seq_ok = true;
+    if (s.paged) {
+      Lq = pa.lens[bi];
+      seq_ok = Lq >= 1 && Lq <= s.L;
+      if (!seq_ok && lane == 0) report(ctx, kDevErrBadIndex);
+      Cq = seq_ok ? (Lq - 1) / kB : 0;
+    }
     int n = 0;
-    for (int sb = sl0; sb < sl1; sb += 32) {
+    for (int sb = sl0; seq_ok && sb < sl1; sb += 32) {
       const int sl = sb + lane;
       int m = -1;
       float bias = 0.f;
       if (sl < sl1) {
         if (s.dense || sl == s.K) {
-          m = s.dense ? sl : s.C;
+          m = s.dense ? sl : Cq;
         } else {
           m = ix[sl];
-          if (m >= s.C || m < -1) {
+          if (m >= Cq || m < -1) {
             report(ctx, kDevErrBadIndex);
             m = -1;
           } else if (m >= 0 && s.use_gates) {
@@ -138,10 +177,32 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int pos = n + __popc(mask & ((1u << lane) - 1u));
         c.blocks[pos] = m;
         c.bias[pos] = bias;
+        if (s.paged) {
+          // Pages of the block's sub-boxes of min(P, 64) tokens; boxes that
+          // start past the sequence, or whose page is missing, load nothing.
+          const int rows = min(pa.P, kB), nsub = kB / rows;
+          const long long p0 = pa.indptr[bi], np = pa.indptr[bi + 1] - p0;
+          for (int i = 0; i < kSub; ++i) {
+            int page = -1;
+            const int t0 = m * kB + i * rows;
+            if (i < nsub && t0 < Lq) {
+              const long long lp = t0 / pa.P;
+              if (lp < np) page = pa.indices[p0 + lp];
+              if (lp >= np || page < 0 || page >= pa.num_pages) {
+                report(ctx, kDevErrBadIndex);
+                page = -1;
+              }
+            }
+            c.pg[pos * kSub + i] = page;
+          }
+        }
       }
       n += __popc(mask);
     }
-    if (lane == 0) c.nblk = n;
+    if (lane == 0) {
+      c.nblk = n;
+      c.Lseq = Lq;
+    }
   }
   if (warp == 1) {
     tmem_alloc(&c.tmem_base, kTmemCols);
@@ -168,10 +229,32 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           break;
         const int m = c.blocks[n];
         unsigned char* kv = base + kOffKV + st * 32768;
-        mbar_arrive_expect_tx(&c.kv_full[st], 32768);
-        for (int h2 = 0; h2 < 2; ++h2) {
-          tma_load_3d(kv + h2 * 8192, &tm_k, h2 * 64, m * kB, (int)plane, &c.kv_full[st]);
-          tma_load_3d(kv + 16384 + h2 * 8192, &tm_v, h2 * 64, m * kB, (int)plane, &c.kv_full[st]);
+        if (!s.paged) {
+          mbar_arrive_expect_tx(&c.kv_full[st], 32768);
+          for (int h2 = 0; h2 < 2; ++h2) {
+            tma_load_3d(kv + h2 * 8192, &tm_k, h2 * 64, m * kB, (int)plane, &c.kv_full[st]);
+            tma_load_3d(kv + 16384 + h2 * 8192, &tm_v, h2 * 64, m * kB, (int)plane,
+                        &c.kv_full[st]);
+          }
+        } else {
+          // Sub-box i (rows rows, 8-row aligned, so the 128-byte swizzle
+          // phase is that of a whole-block load) from page pg[i].
+          const int rows = min(pa.P, kB), nsub = kB / rows;
+          const int row0 = pa.P > kB ? (m * kB) % pa.P : 0;
+          uint32_t bytes = 0;
+          for (int i = 0; i < nsub; ++i) bytes += c.pg[n * kSub + i] >= 0 ? 512u * rows : 0u;
+          mbar_arrive_expect_tx(&c.kv_full[st], bytes);
+          for (int i = 0; i < nsub; ++i) {
+            const int page = c.pg[n * kSub + i];
+            if (page < 0) continue;
+            const int pl = page * s.Hkv + kvh;
+            for (int h2 = 0; h2 < 2; ++h2) {
+              tma_load_3d(kv + h2 * 8192 + i * rows * 128, &tm_k, h2 * 64, row0, pl,
+                          &c.kv_full[st]);
+              tma_load_3d(kv + 16384 + h2 * 8192 + i * rows * 128, &tm_v, h2 * 64, row0, pl,
+                          &c.kv_full[st]);
+            }
+          }
         }
         issued = n + 1;
       }
@@ -238,7 +321,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       fence_after_sync();
       const int m = c.blocks[n];
       const float bias = c.bias[n];
-      const int kvalid = min(kB, s.L - m * kB);
+      const int kvalid = min(kB, c.Lseq - m * kB);
       // Two passes over the two 32-column halves of S: the row max first,
       // then p = 2^(s*scale + bias - m_ref) as bf16 into the S columns
       // already read (P(n) takes columns 0..31).
@@ -315,6 +398,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tmem_st16(tl + kColS + st * 64 + hf * 16, pk);
       }
       l_run += lo_f(accp) + hi_f(accp);
+      if (s.paged && kvalid < kB) {
+        // Rows past the sequence in a page hold other tokens or stale data:
+        // zero them (whole 128-byte rows, so the swizzle does not matter) so
+        // that PV reads 0 there; their P is 0 already.
+        unsigned char* vst = base + kOffKV + (n % kStages) * 32768 + 16384;
+        const int nz = (kB - kvalid) * 8;  // 16-byte chunks per d-half
+        for (int e = lane; e < 2 * nz; e += 32) {
+          const int h2 = e / nz, x = e - h2 * nz;
+          *reinterpret_cast<uint4*>(vst + h2 * 8192 + kvalid * 128 + x * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+      }
       // P(n) (and a rescaled O) in TMEM before PV(n) is issued.
       tmem_st_wait();
       fence_before_sync();
@@ -345,7 +441,58 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     fence_after_sync();
     tmem_dealloc(tmem, kTmemCols);
   }
-  if (*abort) return;
+  const bool ok_cta = !*abort;  // uniform: read after the barrier above
+
+  if (s.cluster) {
+    // ---- cluster merge: partials in shared memory, read by rank
+    if (warp == kSoftmaxWarp && lane < G) {
+      const bool good = ok_cta && ok_sm;
+      float4* dst = reinterpret_cast<float4*>(c.part_o[lane]);
+#pragma unroll
+      for (int q4 = 0; q4 < kD / 4; ++q4)
+        dst[q4] = make_float4(acc[4 * q4], acc[4 * q4 + 1], acc[4 * q4 + 2], acc[4 * q4 + 3]);
+      c.part_m[lane] = good ? m_run : -INFINITY;
+      c.part_l[lane] = good ? l_run : 0.f;
+    }
+    cluster_sync_all();
+    const int P = s.splits;
+    for (int g = split; g < G; g += P) {
+      // (max, sum) of every split for head g, then the weighted sum of the
+      // partial o rows; thread t owns columns 4t .. 4t + 3 (t < 32).
+      if (tid < P) {
+        c.mw[tid] = dsmem_ld_f32(dsmem_addr(&c.part_m[g], (uint32_t)tid));
+        c.ml[tid] = dsmem_ld_f32(dsmem_addr(&c.part_l[g], (uint32_t)tid));
+      }
+      __syncthreads();
+      float M = -INFINITY;
+      for (int x = 0; x < P; ++x) M = fmaxf(M, c.mw[x]);
+      float Lsum = 0.f;
+      for (int x = 0; x < P; ++x)
+        if (c.mw[x] != -INFINITY) Lsum += ex2(c.mw[x] - M) * c.ml[x];
+      if (tid < kD / 4) {
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int x = 0; x < P; ++x) {
+          if (c.mw[x] == -INFINITY) continue;
+          const float f = ex2(c.mw[x] - M);
+          const float4 v = dsmem_ld_f32x4(dsmem_addr(&c.part_o[g][4 * tid], (uint32_t)x));
+          a.x = fmaf(f, v.x, a.x);
+          a.y = fmaf(f, v.y, a.y);
+          a.z = fmaf(f, v.z, a.z);
+          a.w = fmaf(f, v.w, a.w);
+        }
+        const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+        uint2 pk;
+        pk.x = pack_bf16(a.x * inv, a.y * inv);
+        pk.y = pack_bf16(a.z * inv, a.w * inv);
+        *reinterpret_cast<uint2*>(o + (hbase + g) * kD + 4 * tid) = pk;
+      }
+      __syncthreads();
+    }
+    // Every rank's shared memory stays alive until all reads above are done.
+    cluster_sync_all();
+    return;
+  }
+  if (!ok_cta) return;
 
   // ---- this split's partial: row `lane` of the softmax warp is head lane < G
   if (warp == kSoftmaxWarp && ok_sm && lane < G) {
@@ -421,19 +568,97 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   }
 }
 
+// Launch through cudaLaunchKernelEx: as a programmatic dependent of the
+// previous grid (its prologue overlaps that grid's tail), and with the
+// unit's splits as one cluster when s.cluster is set.
 template <int G>
 cudaError_t launch_g(const DecodeShape& s, const CUtensorMap& tq, const CUtensorMap& tk,
                      const CUtensorMap& tv, const int32_t* idx, const float* gates, void* o,
-                     float* ws_ml, float* ws_o, uint32_t* ws_cnt, const DevCtx& ctx,
-                     cudaStream_t st) {
+                     float* ws_ml, float* ws_o, uint32_t* ws_cnt, const PagedArgs& pa,
+                     const DevCtx& ctx, cudaStream_t st, bool pdl) {
   auto kern = decode_tc_kernel<G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
   if (e != cudaSuccess) return e;
-  dim3 grid(s.splits, s.Hkv, s.B);
-  kern<<<grid, kThreads, kSmem, st>>>(tq, tk, tv, idx, gates, s, (__nv_bfloat16*)o, ws_ml, ws_o,
-                                      ws_cnt, ctx);
-  note_launches(1);
-  return cudaGetLastError();
+  if (s.cluster && s.splits > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(s.splits, s.Hkv, s.B);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (s.cluster) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = (unsigned)s.splits;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, idx, gates, s, (__nv_bfloat16*)o, ws_ml, ws_o,
+                         ws_cnt, pa, ctx);
+  if (e == cudaSuccess) note_launches(1);
+  return e;
+}
+
+// Whether a cluster of `splits` decode CTAs (G heads) fits on the device,
+// asked once per (G, splits) and process.
+template <int G>
+bool cluster_fits(int splits) {
+  static std::mutex mu;
+  static signed char fits[17] = {};
+  std::lock_guard<std::mutex> lk(mu);
+  if (fits[splits] == 0) {
+    auto kern = decode_tc_kernel<G>;
+    bool ok = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem) ==
+              cudaSuccess;
+    if (ok && splits > 8)
+      ok = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+           cudaSuccess;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(splits, 1, 1);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (ok) ok = cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess;
+    (void)cudaGetLastError();
+    fits[splits] = (ok && n > 0) ? 1 : -1;
+  }
+  return fits[splits] > 0;
+}
+
+template <int G>
+cudaError_t launch_any(DecodeShape s, const CUtensorMap& tq, const CUtensorMap& tk,
+                       const CUtensorMap& tv, const int32_t* idx, const float* gates, void* o,
+                       float* ws_ml, float* ws_o, uint32_t* ws_cnt, const PagedArgs& pa,
+                       const DevCtx& ctx, cudaStream_t st) {
+  s.cluster = s.splits >= 2 && s.splits <= kMaxClusterSplits && cluster_fits<G>(s.splits);
+  if (!s.cluster && s.splits > 1) {
+    // Tickets start at zero on every call, whatever the workspace held before.
+    cudaError_t e = cudaMemsetAsync(ws_cnt, 0, sizeof(uint32_t) * (size_t)s.B * s.Hkv, st);
+    if (e != cudaSuccess) return e;
+    note_launches(1);
+  }
+  // Only a kernel may precede a programmatic dependent: after the memset the
+  // launch is an ordinary one.
+  const bool pdl = s.cluster || s.splits == 1;
+  return launch_g<G>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, ctx, st, pdl);
 }
 
 }  // namespace
@@ -443,6 +668,31 @@ bool tc_decode_supported(sas_dtype_t dt, const DecodeShape& s) {
   return dt == SAS_BF16 && s.d == kD && s.b == kB && G >= 1 && G <= kMaxG && s.splits <= 64 &&
          s.bps <= kMaxSlotsPerSplit;
 }
+
+namespace {
+cudaError_t launch_tc_maps(const DecodeShape& s, const CUtensorMap& tq, const CUtensorMap& tk,
+                           const CUtensorMap& tv, const PagedArgs& pa, const int32_t* idx,
+                           const float* gates, void* o, void* ws, const DevCtx& ctx,
+                           cudaStream_t st) {
+  char* w = static_cast<char*>(ws);
+  const size_t parts = (size_t)s.B * s.Hq * s.splits;
+  float* ws_ml = reinterpret_cast<float*>(w);
+  float* ws_o = reinterpret_cast<float*>(w + ((2 * parts * sizeof(float) + 255) & ~(size_t)255));
+  uint32_t* ws_cnt = reinterpret_cast<uint32_t*>(
+      reinterpret_cast<char*>(ws_o) + ((parts * s.d * sizeof(float) + 255) & ~(size_t)255));
+  switch (s.Hq / s.Hkv) {
+    case 1: return launch_any<1>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, ctx, st);
+    case 2: return launch_any<2>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, ctx, st);
+    case 3: return launch_any<3>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, ctx, st);
+    case 4: return launch_any<4>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, ctx, st);
+    case 5: return launch_any<5>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, ctx, st);
+    case 6: return launch_any<6>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, ctx, st);
+    case 7: return launch_any<7>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, ctx, st);
+    case 8: return launch_any<8>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, ctx, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+}  // namespace
 
 cudaError_t launch_decode_tc(const DecodeShape& s, const void* q, const void* kc, const void* vc,
                              const int32_t* idx, const float* gates, void* o, void* ws,
@@ -454,29 +704,24 @@ cudaError_t launch_decode_tc(const DecodeShape& s, const void* q, const void* kc
   if ((e = make_tmap_bf16_rows8(&tq, q, s.B * s.Hq)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16_pitched(&tk, kc, s.L, s.Lcap, s.B * s.Hkv)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16_pitched(&tv, vc, s.L, s.Lcap, s.B * s.Hkv)) != cudaSuccess) return e;
-  char* w = static_cast<char*>(ws);
-  const size_t parts = (size_t)s.B * s.Hq * s.splits;
-  float* ws_ml = reinterpret_cast<float*>(w);
-  float* ws_o = reinterpret_cast<float*>(w + ((2 * parts * sizeof(float) + 255) & ~(size_t)255));
-  uint32_t* ws_cnt = reinterpret_cast<uint32_t*>(
-      reinterpret_cast<char*>(ws_o) + ((parts * s.d * sizeof(float) + 255) & ~(size_t)255));
-  if (s.splits > 1) {
-    // Tickets start at zero on every call, whatever the workspace held before.
-    e = cudaMemsetAsync(ws_cnt, 0, sizeof(uint32_t) * (size_t)s.B * s.Hkv, st);
-    if (e != cudaSuccess) return e;
-    note_launches(1);
-  }
-  switch (s.Hq / s.Hkv) {
-    case 1: return launch_g<1>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, ctx, st);
-    case 2: return launch_g<2>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, ctx, st);
-    case 3: return launch_g<3>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, ctx, st);
-    case 4: return launch_g<4>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, ctx, st);
-    case 5: return launch_g<5>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, ctx, st);
-    case 6: return launch_g<6>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, ctx, st);
-    case 7: return launch_g<7>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, ctx, st);
-    case 8: return launch_g<8>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, ctx, st);
-    default: return cudaErrorInvalidValue;
-  }
+  const PagedArgs none = {nullptr, nullptr, nullptr, 0, 0};
+  return launch_tc_maps(s, tq, tk, tv, none, idx, gates, o, ws, ctx, st);
+}
+
+cudaError_t launch_decode_paged_tc(const DecodeShape& s, const PagedArgs& pa, const void* q,
+                                   const void* kpages, const void* vpages, const int32_t* idx,
+                                   const float* gates, void* o, void* ws, const DevCtx& ctx,
+                                   cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  cudaError_t e;
+  // Pages as [num_pages * Hkv planes][P rows][128], boxes of min(P, 64) rows.
+  const int rows = pa.P < kB ? pa.P : kB;
+  if ((e = make_tmap_bf16_rows8(&tq, q, s.B * s.Hq)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_box(&tk, kpages, pa.P, pa.num_pages * s.Hkv, rows)) != cudaSuccess)
+    return e;
+  if ((e = make_tmap_bf16_box(&tv, vpages, pa.P, pa.num_pages * s.Hkv, rows)) != cudaSuccess)
+    return e;
+  return launch_tc_maps(s, tq, tk, tv, pa, idx, gates, o, ws, ctx, st);
 }
 
 }  // namespace sas

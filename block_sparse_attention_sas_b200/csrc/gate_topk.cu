@@ -17,6 +17,14 @@
 // Two layouts of the same algorithm: one warp per row for short rows (the
 // training case, one row per query block), one CTA per row for long rows
 // (decode over thousands of history blocks).
+//
+// Gate activations (phi of Eq. 4): softmax over the valid history (Eq. 6,
+// the method's own), and the two ablation variants the evolve.pub review
+// (Summary) names: an elementwise sigmoid g = 1 / (1 + e^-s) and raw logits
+// (log g = s, stored as g = e^s). Top-K is over the scores for every phi:
+// each is increasing, so the selection is the same.
+#include <mutex>
+
 #include "sas_common.cuh"
 #include "sas_internal.h"
 
@@ -79,6 +87,14 @@ __device__ __forceinline__ uint32_t warp_pick_digit(const int* hist, int k, int&
   return (uint32_t)__shfl_sync(0xffffffffu, dig, L);
 }
 
+// Gate of one valid entry from its score (lse: the row's log-sum-exp, used by
+// the softmax only).
+__device__ __forceinline__ float gate_of(float sc, float lse, int phi) {
+  if (phi == SAS_PHI_SIGMOID) return 1.f / (1.f + expf(-sc));
+  if (phi == SAS_PHI_RAW) return expf(sc);
+  return expf(sc - lse);
+}
+
 constexpr int kWarpRowsPerCta = 8;
 constexpr int kWarpCap = 512;   // longest row handled by one warp
 constexpr int kMaxK = 256;
@@ -88,12 +104,14 @@ constexpr int kMaxK = 256;
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(32 * kWarpRowsPerCta)
 gate_topk_warp_kernel(const float* __restrict__ scores, int total_rows, int rows, int C,
-                      int causal, int K, float* __restrict__ gates, int32_t* __restrict__ idx) {
+                      int causal, int K, int phi, float* __restrict__ gates,
+                      int32_t* __restrict__ idx) {
   __shared__ float s_val[kWarpRowsPerCta][kWarpCap];
   __shared__ uint32_t s_selkey[kWarpRowsPerCta][kMaxK];
   __shared__ int32_t s_selidx[kWarpRowsPerCta][kMaxK];
   __shared__ int s_hist[kWarpRowsPerCta][256];
 
+  grid_launch_dependents();  // a dependent decode may start its prologue
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long row = (long long)blockIdx.x * kWarpRowsPerCta + w;
   if (row >= total_rows) return;
@@ -116,7 +134,7 @@ gate_topk_warp_kernel(const float* __restrict__ scores, int total_rows, int rows
   for (int i = lane; i < n; i += 32) sum += expf(v[i] - mx);
   sum = warp_sum(sum);
   const float lse = mx + logf(sum);
-  for (int i = lane; i < C; i += 32) g[i] = (i < n) ? expf(v[i] - lse) : 0.f;
+  for (int i = lane; i < C; i += 32) g[i] = (i < n) ? gate_of(v[i], lse, phi) : 0.f;
 
   const int k = min(K, n);
   if (k > 0) {
@@ -395,7 +413,8 @@ __device__ void block_topk(uint64_t (&v)[E], int k, TopkScratch& ts, uint64_t* s
 
 // Writes g = exp(s - lse) for i < n and 0 past n, over [0, C) of one row
 // (float4 accesses when both rows are 16-byte aligned).
-__device__ __forceinline__ void write_gates(const float* srow, float* grow, int C, int n, float lse) {
+__device__ __forceinline__ void write_gates(const float* srow, float* grow, int C, int n, float lse,
+                                            int phi) {
   const int tid = threadIdx.x, bd = blockDim.x;
   const bool vec = ((reinterpret_cast<uintptr_t>(srow) | reinterpret_cast<uintptr_t>(grow)) & 15) == 0;
   int i0 = 0;
@@ -405,15 +424,15 @@ __device__ __forceinline__ void write_gates(const float* srow, float* grow, int 
       const float4 x = reinterpret_cast<const float4*>(srow)[q];
       const int i = q * 4;
       float4 g;
-      g.x = i < n ? expf(x.x - lse) : 0.f;
-      g.y = i + 1 < n ? expf(x.y - lse) : 0.f;
-      g.z = i + 2 < n ? expf(x.z - lse) : 0.f;
-      g.w = i + 3 < n ? expf(x.w - lse) : 0.f;
+      g.x = i < n ? gate_of(x.x, lse, phi) : 0.f;
+      g.y = i + 1 < n ? gate_of(x.y, lse, phi) : 0.f;
+      g.z = i + 2 < n ? gate_of(x.z, lse, phi) : 0.f;
+      g.w = i + 3 < n ? gate_of(x.w, lse, phi) : 0.f;
       reinterpret_cast<float4*>(grow)[q] = g;
     }
     i0 = C4 * 4;
   }
-  for (int i = i0 + tid; i < C; i += bd) grow[i] = i < n ? expf(srow[i] - lse) : 0.f;
+  for (int i = i0 + tid; i < C; i += bd) grow[i] = i < n ? gate_of(srow[i], lse, phi) : 0.f;
 }
 
 // One block per (row, chunk of Lc = E * blockDim.x entries). FINAL (the row
@@ -424,7 +443,8 @@ __device__ __forceinline__ void write_gates(const float* srow, float* grow, int 
 template <bool FINAL, int E>
 __global__ void __launch_bounds__(1024)
 gate_topk_chunk_kernel(const float* __restrict__ scores, int rows, int C, int causal, int K,
-                       int chunks, int kc, float* __restrict__ gates, int32_t* __restrict__ idx) {
+                       int chunks, int kc, int phi, float* __restrict__ gates,
+                       int32_t* __restrict__ idx) {
   extern __shared__ uint64_t s_key[];  // E * blockDim.x keys
   __shared__ float red[32];
   __shared__ TopkScratch ts;
@@ -461,7 +481,7 @@ gate_topk_chunk_kernel(const float* __restrict__ scores, int rows, int C, int ca
   if (FINAL) {
     int32_t* out = idx + row * (long long)K;
     for (int p = tid; p < K; p += bd) out[p] = p < kk ? ckey_index(s_key[p]) : -1;
-    write_gates(srow, grow, C, n, mx + logf(sum));
+    write_gates(srow, grow, C, n, mx + logf(sum), phi);
   } else {
     if (tid == 0) {
       grow[2 * c] = mx;
@@ -482,7 +502,8 @@ gate_topk_chunk_kernel(const float* __restrict__ scores, int rows, int C, int ca
 template <int E>
 __global__ void __launch_bounds__(1024)
 gate_topk_merge_kernel(const float* __restrict__ scores, int rows, int C, int causal, int K,
-                       int chunks, int kc, float* __restrict__ gates, int32_t* __restrict__ idx) {
+                       int chunks, int kc, int phi, float* __restrict__ gates,
+                       int32_t* __restrict__ idx) {
   extern __shared__ uint64_t s_key[];  // E * blockDim.x keys
   __shared__ float red[32];
   __shared__ TopkScratch ts;
@@ -513,7 +534,124 @@ gate_topk_merge_kernel(const float* __restrict__ scores, int rows, int C, int ca
   if (k > 0) block_topk<E>(v, k, ts, s_key);
   int32_t* out = idx + row * (long long)K;
   for (int p = tid; p < K; p += bd) out[p] = p < k ? ckey_index(s_key[p]) : -1;
-  write_gates(scores + row * (long long)C, grow, C, n, lse);
+  write_gates(scores + row * (long long)C, grow, C, n, lse, phi);
+}
+
+// ---------------------------------------------------------------------------
+// Long rows in one launch: a thread-block cluster of CS CTAs per row, CTA r
+// taking the chunk [r Lc, (r + 1) Lc). Each chunk forms its softmax partial
+// (max, sum of exp) and its best min(K, Lc) composites in shared memory; after
+// a cluster barrier every CTA reads the CS partials through distributed shared
+// memory (in rank order, so all form the same LSE) and writes its chunk's
+// gates from the scores it still holds, while rank 0 gathers the candidates
+// and selects the row's Top-K. A second barrier keeps every chunk's shared
+// memory alive until those reads are done. No workspace, no second launch.
+// ---------------------------------------------------------------------------
+constexpr int kClThreads = 512;
+constexpr int kClMaxCta = 16;
+
+template <int EM>
+__device__ void cluster_merge_topk(const uint64_t* cand_local, const int* cnt_local, int CS, int kc,
+                                   int k, TopkScratch& ts, uint64_t* sm, int32_t* out, int K) {
+  const int tid = threadIdx.x, bd = blockDim.x;
+  uint64_t v[EM];
+#pragma unroll
+  for (int e = 0; e < EM; ++e) {
+    const int i = e * bd + tid;
+    const int r = i / kc, p = i - r * kc;
+    uint64_t key = 0ull;
+    if (r < CS) {
+      const int cnt = (int)dsmem_ld_u32(dsmem_addr(cnt_local, (uint32_t)r));
+      if (p < cnt) key = dsmem_ld_u64(dsmem_addr(cand_local + p, (uint32_t)r));
+    }
+    v[e] = key;
+  }
+  // Every CTA of the cluster may now leave once it is done with its gates:
+  // this barrier pairs with the one the other ranks pass after their reads.
+  cluster_sync_all();
+  block_topk<EM>(v, k, ts, sm);
+  for (int p = tid; p < K; p += bd) out[p] = p < k ? ckey_index(sm[p]) : -1;
+}
+
+template <int E>
+__global__ void __launch_bounds__(kClThreads)
+gate_topk_cluster_kernel(const float* __restrict__ scores, int rows, int C, int causal, int K,
+                         int CS, int phi, float* __restrict__ gates, int32_t* __restrict__ idx) {
+  extern __shared__ uint64_t s_key[];  // max(E, merge width) * blockDim.x keys
+  __shared__ float red[32];
+  __shared__ TopkScratch ts;
+  __shared__ float s_part[2];  // this chunk's (max, sum of exp)
+  __shared__ int s_cnt;        // its candidate count
+  __shared__ float s_lse;
+  grid_launch_dependents();  // a dependent decode may start its prologue
+  const int tid = threadIdx.x, bd = blockDim.x, Lc = E * bd;
+  const uint32_t rank = cluster_rank();
+  const long long row = blockIdx.x / CS;
+  const int r = (int)(row % rows);
+  const int n = causal ? min(r, C) : C;
+  const int lo = (int)rank * Lc, len = max(0, min(n - lo, Lc));
+  const int kc = min(K, Lc);
+  const float* srow = scores + row * (long long)C;
+
+  uint64_t v[E];
+  float f[E];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = e * bd + tid;
+    const bool ok = i < len;
+    f[e] = ok ? srow[lo + i] : -INFINITY;
+    v[e] = ok ? ckey(f[e], lo + i) : 0ull;
+    mx = fmaxf(mx, f[e]);
+  }
+  mx = block_max(mx, red);
+  float sum = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e)
+    if (e * bd + tid < len) sum += expf(f[e] - mx);
+  sum = block_sum(sum, red);
+  const int kk = min(kc, len);
+  if (kk > 0) block_topk<E>(v, kk, ts, s_key);
+  if (tid == 0) {
+    s_part[0] = mx;
+    s_part[1] = sum;
+    s_cnt = kk;
+  }
+  cluster_sync_all();
+
+  // The row's LSE from the CS partials, combined in rank order by warp 0.
+  if (tid < 32) {
+    float pm = -INFINITY, ps = 0.f;
+    if (tid < CS) {
+      pm = dsmem_ld_f32(dsmem_addr(&s_part[0], (uint32_t)tid));
+      ps = dsmem_ld_f32(dsmem_addr(&s_part[1], (uint32_t)tid));
+    }
+    const float M = warp_max(pm);
+    const float t = warp_sum(ps > 0.f ? ps * expf(pm - M) : 0.f);
+    if (tid == 0) s_lse = M + logf(t);
+  }
+  const int k = min(K, n);
+  if (rank == 0) {
+    // Gathers the candidates (registers), passes the second barrier, selects.
+    const int nc = CS * kc;
+    int32_t* out = idx + row * (long long)K;
+    if (nc <= bd) cluster_merge_topk<1>(s_key, &s_cnt, CS, kc, max(k, 1), ts, s_key, out, k > 0 ? K : 0);
+    else if (nc <= 2 * bd) cluster_merge_topk<2>(s_key, &s_cnt, CS, kc, max(k, 1), ts, s_key, out, k > 0 ? K : 0);
+    else if (nc <= 4 * bd) cluster_merge_topk<4>(s_key, &s_cnt, CS, kc, max(k, 1), ts, s_key, out, k > 0 ? K : 0);
+    else cluster_merge_topk<8>(s_key, &s_cnt, CS, kc, max(k, 1), ts, s_key, out, k > 0 ? K : 0);
+    if (k == 0)
+      for (int p = tid; p < K; p += bd) out[p] = -1;
+  } else {
+    cluster_sync_all();
+  }
+  __syncthreads();
+  const float lse = s_lse;
+  float* grow = gates + row * (long long)C;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int gi = lo + e * bd + tid;
+    if (gi < C) grow[gi] = gi < n ? gate_of(f[e], lse, phi) : 0.f;
+  }
 }
 
 int pow2_at_least(int x) {
@@ -522,28 +660,84 @@ int pow2_at_least(int x) {
   return p;
 }
 
+// Launches the cluster kernel when the row fits (C <= 16 chunks of 4096) and
+// the device can hold such a cluster; returns false (nothing launched) to
+// leave the row to the two-launch path.
+bool launch_cluster_topk(const float* scores, long long total, int rows, int C, int causal, int K,
+                         int phi, float* gates, int32_t* idx, cudaStream_t stream) {
+  if (C > kClMaxCta * 4096 || total * kClMaxCta > 0x7fffffffLL) return false;
+  int Lc = kClThreads;
+  while ((C + Lc - 1) / Lc > kClMaxCta) Lc <<= 1;
+  const int CS = (C + Lc - 1) / Lc, E = Lc / kClThreads, kc = min(K, Lc);
+  const int EM = pow2_at_least((CS * kc + kClThreads - 1) / kClThreads);
+  const size_t smem = (size_t)max(E, EM) * kClThreads * sizeof(uint64_t);
+  void (*kern)(const float*, int, int, int, int, int, int, float*, int32_t*) =
+      E == 1 ? gate_topk_cluster_kernel<1> : E == 2 ? gate_topk_cluster_kernel<2>
+             : E == 4 ? gate_topk_cluster_kernel<4> : gate_topk_cluster_kernel<8>;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(total * CS));
+  cfg.blockDim = dim3(kClThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // Whether this (E, CS) fits on the device, asked once per process.
+  static std::mutex mu;
+  static signed char fits[4][kClMaxCta + 1] = {};
+  const int ei = E == 1 ? 0 : E == 2 ? 1 : E == 4 ? 2 : 3;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (fits[ei][CS] == 0) {
+      bool ok = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)smem) == cudaSuccess;
+      if (ok && CS > 8)
+        ok = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+             cudaSuccess;
+      int nclusters = 0;
+      if (ok) ok = cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) == cudaSuccess;
+      fits[ei][CS] = (ok && nclusters > 0) ? 1 : -1;
+      (void)cudaGetLastError();  // a refused query leaves no sticky error behind
+    }
+    if (fits[ei][CS] < 0) return false;
+  }
+  if (cudaLaunchKernelEx(&cfg, kern, scores, rows, C, causal, K, CS, phi, gates, idx) !=
+      cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  note_launches(1);
+  return true;
+}
+
 }  // namespace
 
 cudaError_t launch_gate_topk(const float* scores, int B, int Hkv, int rows, int C, int causal,
-                             int K, float* gates, int32_t* idx, cudaStream_t stream) {
+                             int K, int phi, float* gates, int32_t* idx, cudaStream_t stream) {
   const long long total = (long long)B * Hkv * rows;
   if (total == 0) return cudaSuccess;
   const int maxlen = causal ? min(rows - 1, C) : C;
   if (maxlen <= kWarpCap) {
     const long long grid = (total + kWarpRowsPerCta - 1) / kWarpRowsPerCta;
     gate_topk_warp_kernel<<<(unsigned)grid, 32 * kWarpRowsPerCta, 0, stream>>>(
-        scores, (int)total, rows, C, causal, K, gates, idx);
+        scores, (int)total, rows, C, causal, K, phi, gates, idx);
     note_launches(1);
+  } else if (launch_cluster_topk(scores, total, rows, C, causal, K, phi, gates, idx, stream)) {
+    // one launch: a cluster of chunk CTAs per row
   } else if (C <= 2048) {
     // One block per row sorts the whole row.
     const int Lp = pow2_at_least(C), threads = min(1024, Lp);
     const size_t smem = (size_t)Lp * sizeof(uint64_t);
     if (Lp / threads == 1)
       gate_topk_chunk_kernel<true, 1><<<(unsigned)total, threads, smem, stream>>>(
-          scores, rows, C, causal, K, 1, min(K, Lp), gates, idx);
+          scores, rows, C, causal, K, 1, min(K, Lp), phi, gates, idx);
     else
       gate_topk_chunk_kernel<true, 2><<<(unsigned)total, threads, smem, stream>>>(
-          scores, rows, C, causal, K, 1, min(K, Lp), gates, idx);
+          scores, rows, C, causal, K, 1, min(K, Lp), phi, gates, idx);
     note_launches(1);
   } else {
     // The shortest chunk (a power of two from 512) whose candidates fit the
@@ -568,7 +762,8 @@ cudaError_t launch_gate_topk(const float* scores, int B, int Hkv, int rows, int 
       if (smem + kStaticSmem > 48 * 1024)
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e == cudaSuccess)
-        kern<<<grid, threads, smem, stream>>>(scores, rows, C, causal, K, chunks, kc, gates, idx);
+        kern<<<grid, threads, smem, stream>>>(scores, rows, C, causal, K, chunks, kc, phi, gates,
+                                              idx);
     };
     switch (E) {
       case 1: chunk(gate_topk_chunk_kernel<false, 1>); break;
@@ -586,7 +781,7 @@ cudaError_t launch_gate_topk(const float* scores, int B, int Hkv, int rows, int 
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
       if (e == cudaSuccess)
         kern<<<(unsigned)total, mthreads, msmem, stream>>>(scores, rows, C, causal, K, chunks, kc,
-                                                           gates, idx);
+                                                           phi, gates, idx);
     };
     switch (ME) {
       case 1: merge(gate_topk_merge_kernel<1>); break;

@@ -84,7 +84,80 @@ AttnShape make_shape(int B, int Hq, int Hkv, int T, int d, int b, int K, float s
   s.K = dense ? 0 : K;
   s.scale = resolve_scale(scale, d);
   s.dense = dense;
+  s.outer = false;
+  s.phi = SAS_PHI_SOFTMAX;
   return s;
+}
+
+bool valid_phi(int phi) {
+  return phi == SAS_PHI_SOFTMAX || phi == SAS_PHI_SIGMOID || phi == SAS_PHI_RAW;
+}
+bool valid_gating(int g) { return g == SAS_GATE_INNER || g == SAS_GATE_OUTER; }
+
+sas_status_t gate_topk_impl(const float* scores, int B, int Hkv, int rows, int C, int causal,
+                            int K, int phi, float* gates, int32_t* idx, cudaStream_t stream) {
+  if (B < 0 || Hkv < 0 || rows < 0) return SAS_ERR_INVALID_ARG;
+  if (C < 0 || K < 1 || (causal != 0 && causal != 1)) return SAS_ERR_INVALID_ARG;
+  if (!valid_phi(phi)) return SAS_ERR_INVALID_ARG;
+  if (causal && rows != C) return SAS_ERR_INVALID_ARG;
+  if (C > 262144 || K > 256) return SAS_ERR_UNSUPPORTED;
+  if ((long long)B * Hkv * rows == 0) return SAS_OK;
+  if (!idx || (C > 0 && (!scores || !gates))) return SAS_ERR_INVALID_ARG;
+  if (!aligned(scores, 4) || !aligned(gates, 4) || !aligned(idx, 4)) return SAS_ERR_INVALID_ARG;
+  if ((long long)B * Hkv * rows > (1ll << 31) - 1) return SAS_ERR_UNSUPPORTED;
+  return cuda_status(launch_gate_topk(scores, B, Hkv, rows, C, causal, K, phi, gates, idx, stream));
+}
+
+sas_status_t attn_fwd_impl(sas_dtype_t dtype, const void* q, const void* k, const void* v,
+                           const int32_t* idx, const float* gates, int B, int Hq, int Hkv, int T,
+                           int d, int b, int K, float scale, int gating, void* o, float* lse,
+                           cudaStream_t stream) {
+  sas_status_t st = check_attn(dtype, B, Hq, Hkv, T, d, b, K, false, scale);
+  if (st != SAS_OK) return st;
+  if (!valid_gating(gating)) return SAS_ERR_INVALID_ARG;
+  if (B == 0) return SAS_OK;
+  if (!q || !k || !v || !idx || !o || !lse) return SAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4) || !aligned(idx, 4) || (gates && !aligned(gates, 4)))
+    return SAS_ERR_INVALID_ARG;
+  DevCtx ctx;
+  if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
+  AttnShape s = make_shape(B, Hq, Hkv, T, d, b, K, scale, false);
+  s.outer = gating == SAS_GATE_OUTER;
+  if (tc_fwd_supported(dtype, s))
+    return cuda_status(launch_attn_fwd_tc(s, q, k, v, idx, gates, o, lse, ctx, stream));
+  return cuda_status(launch_attn_fwd_simt(dtype, s, q, k, v, idx, gates, o, lse, ctx, stream));
+}
+
+sas_status_t attn_bwd_impl(sas_dtype_t dtype, const void* q, const void* k, const void* v,
+                           const void* o, const float* lse, const void* dO, const int32_t* idx,
+                           const float* gates, int B, int Hq, int Hkv, int T, int d, int b, int K,
+                           float scale, int phi, int gating, void* dq, void* dk, void* dv,
+                           float* dscores, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  sas_status_t st = check_attn(dtype, B, Hq, Hkv, T, d, b, K, false, scale);
+  if (st != SAS_OK) return st;
+  if (!valid_phi(phi) || !valid_gating(gating)) return SAS_ERR_INVALID_ARG;
+  if (B == 0) return SAS_OK;
+  if (!q || !k || !v || !o || !lse || !dO || !idx || !dq || !dk || !dv)
+    return SAS_ERR_INVALID_ARG;
+  if (!gates && dscores) return SAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(dO, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+      !aligned(lse, 4) || !aligned(idx, 4) || (gates && !aligned(gates, 4)) ||
+      (dscores && !aligned(dscores, 4)))
+    return SAS_ERR_INVALID_ARG;
+  AttnShape s = make_shape(B, Hq, Hkv, T, d, b, K, scale, false);
+  s.outer = gating == SAS_GATE_OUTER;
+  s.phi = phi;
+  const size_t need = bwd_workspace_layout(s, tc_bwd_supported(dtype, s)).total;
+  if (!ws || ws_bytes < need || !aligned(ws, 256)) return SAS_ERR_WORKSPACE;
+  DevCtx ctx;
+  if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
+  if (tc_bwd_supported(dtype, s))
+    return cuda_status(launch_attn_bwd_tc(s, q, k, v, lse, dO, idx, gates, dq, dk, dv, dscores,
+                                          ws, ctx, stream));
+  return cuda_status(launch_attn_bwd_simt(dtype, s, q, k, v, o, lse, dO, idx, gates, dq, dk, dv,
+                                          dscores, ws, ctx, stream));
 }
 
 sas_status_t check_decode(sas_dtype_t dt, int B, int Hq, int Hkv, int L, int Lcap, int d, int b,
@@ -118,6 +191,7 @@ DecodeShape make_decode(int B, int Hq, int Hkv, int L, int Lcap, int d, int b, i
   s.C = (L - 1) / b;
   s.dense = dense;
   s.use_gates = dense ? 0 : (use_gates != 0);
+  s.paged = false;
   decode_plan(s);
   return s;
 }
@@ -193,34 +267,29 @@ sas_status_t sas_selftest_wait_timeout(sas_stream_t stream) {
 
 sas_status_t sas_gate_topk(const float* scores, int B, int Hkv, int rows, int C, int causal,
                            int K, float* gates, int32_t* idx, sas_stream_t stream) {
-  if (B < 0 || Hkv < 0 || rows < 0) return SAS_ERR_INVALID_ARG;
-  if (C < 0 || K < 1 || (causal != 0 && causal != 1)) return SAS_ERR_INVALID_ARG;
-  if (causal && rows != C) return SAS_ERR_INVALID_ARG;
-  if (C > 262144 || K > 256) return SAS_ERR_UNSUPPORTED;
-  if ((long long)B * Hkv * rows == 0) return SAS_OK;
-  if (!idx || (C > 0 && (!scores || !gates))) return SAS_ERR_INVALID_ARG;
-  if (!aligned(scores, 4) || !aligned(gates, 4) || !aligned(idx, 4)) return SAS_ERR_INVALID_ARG;
-  if ((long long)B * Hkv * rows > (1ll << 31) - 1) return SAS_ERR_UNSUPPORTED;
-  return cuda_status(launch_gate_topk(scores, B, Hkv, rows, C, causal, K, gates, idx, stream));
+  return gate_topk_impl(scores, B, Hkv, rows, C, causal, K, SAS_PHI_SOFTMAX, gates, idx, stream);
+}
+
+sas_status_t sas_gate_topk_phi(const float* scores, int B, int Hkv, int rows, int C, int causal,
+                               int K, sas_phi_t phi, float* gates, int32_t* idx,
+                               sas_stream_t stream) {
+  return gate_topk_impl(scores, B, Hkv, rows, C, causal, K, (int)phi, gates, idx, stream);
 }
 
 sas_status_t sas_attn_fwd(sas_dtype_t dtype, const void* q, const void* k, const void* v,
                           const int32_t* idx, const float* gates, int B, int Hq, int Hkv, int T,
                           int d, int b, int K, float scale, void* o, float* lse,
                           sas_stream_t stream) {
-  sas_status_t st = check_attn(dtype, B, Hq, Hkv, T, d, b, K, false, scale);
-  if (st != SAS_OK) return st;
-  if (B == 0) return SAS_OK;
-  if (!q || !k || !v || !idx || !o || !lse) return SAS_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
-      !aligned(lse, 4) || !aligned(idx, 4) || (gates && !aligned(gates, 4)))
-    return SAS_ERR_INVALID_ARG;
-  DevCtx ctx;
-  if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
-  const AttnShape s = make_shape(B, Hq, Hkv, T, d, b, K, scale, false);
-  if (tc_fwd_supported(dtype, s))
-    return cuda_status(launch_attn_fwd_tc(s, q, k, v, idx, gates, o, lse, ctx, stream));
-  return cuda_status(launch_attn_fwd_simt(dtype, s, q, k, v, idx, gates, o, lse, ctx, stream));
+  return attn_fwd_impl(dtype, q, k, v, idx, gates, B, Hq, Hkv, T, d, b, K, scale, SAS_GATE_INNER,
+                       o, lse, stream);
+}
+
+sas_status_t sas_attn_fwd_gated(sas_dtype_t dtype, const void* q, const void* k, const void* v,
+                                const int32_t* idx, const float* gates, int B, int Hq, int Hkv,
+                                int T, int d, int b, int K, float scale, sas_gating_t gating,
+                                void* o, float* lse, sas_stream_t stream) {
+  return attn_fwd_impl(dtype, q, k, v, idx, gates, B, Hq, Hkv, T, d, b, K, scale, (int)gating, o,
+                       lse, stream);
 }
 
 size_t sas_attn_bwd_workspace_size(sas_dtype_t dtype, int B, int Hq, int Hkv, int T, int d, int b,
@@ -235,27 +304,18 @@ sas_status_t sas_attn_bwd(sas_dtype_t dtype, const void* q, const void* k, const
                           const float* gates, int B, int Hq, int Hkv, int T, int d, int b, int K,
                           float scale, void* dq, void* dk, void* dv, float* dscores, void* ws,
                           size_t ws_bytes, sas_stream_t stream) {
-  sas_status_t st = check_attn(dtype, B, Hq, Hkv, T, d, b, K, false, scale);
-  if (st != SAS_OK) return st;
-  if (B == 0) return SAS_OK;
-  if (!q || !k || !v || !o || !lse || !dO || !idx || !dq || !dk || !dv)
-    return SAS_ERR_INVALID_ARG;
-  if (!gates && dscores) return SAS_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
-      !aligned(dO, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
-      !aligned(lse, 4) || !aligned(idx, 4) || (gates && !aligned(gates, 4)) ||
-      (dscores && !aligned(dscores, 4)))
-    return SAS_ERR_INVALID_ARG;
-  const AttnShape s = make_shape(B, Hq, Hkv, T, d, b, K, scale, false);
-  const size_t need = bwd_workspace_layout(s, tc_bwd_supported(dtype, s)).total;
-  if (!ws || ws_bytes < need || !aligned(ws, 256)) return SAS_ERR_WORKSPACE;
-  DevCtx ctx;
-  if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
-  if (tc_bwd_supported(dtype, s))
-    return cuda_status(launch_attn_bwd_tc(s, q, k, v, lse, dO, idx, gates, dq, dk, dv, dscores,
-                                          ws, ctx, stream));
-  return cuda_status(launch_attn_bwd_simt(dtype, s, q, k, v, o, lse, dO, idx, gates, dq, dk, dv,
-                                          dscores, ws, ctx, stream));
+  return attn_bwd_impl(dtype, q, k, v, o, lse, dO, idx, gates, B, Hq, Hkv, T, d, b, K, scale,
+                       SAS_PHI_SOFTMAX, SAS_GATE_INNER, dq, dk, dv, dscores, ws, ws_bytes, stream);
+}
+
+sas_status_t sas_attn_bwd_gated(sas_dtype_t dtype, const void* q, const void* k, const void* v,
+                                const void* o, const float* lse, const void* dO,
+                                const int32_t* idx, const float* gates, int B, int Hq, int Hkv,
+                                int T, int d, int b, int K, float scale, sas_phi_t phi,
+                                sas_gating_t gating, void* dq, void* dk, void* dv,
+                                float* dscores, void* ws, size_t ws_bytes, sas_stream_t stream) {
+  return attn_bwd_impl(dtype, q, k, v, o, lse, dO, idx, gates, B, Hq, Hkv, T, d, b, K, scale,
+                       (int)phi, (int)gating, dq, dk, dv, dscores, ws, ws_bytes, stream);
 }
 
 size_t sas_decode_workspace_size(int B, int Hq, int Hkv, int L, int d, int b, int K) {
@@ -308,6 +368,44 @@ sas_status_t sas_decode_noalloc(sas_dtype_t dtype, const void* q, const void* kc
 }
 
 size_t sas_decode_noalloc_max_scratch(void) { return decode_noalloc_capacity(); }
+
+size_t sas_decode_paged_workspace_size(int B, int Hq, int Hkv, int max_len, int d, int b, int K) {
+  return sas_decode_workspace_size(B, Hq, Hkv, max_len, d, b, K);
+}
+
+sas_status_t sas_decode_paged(sas_dtype_t dtype, const void* q, const void* kpages,
+                              const void* vpages, const int32_t* page_indptr,
+                              const int32_t* page_indices, const int32_t* seq_lens,
+                              const int32_t* idx, const float* gates, int use_gates, int B, int Hq,
+                              int Hkv, int num_pages, int page_size, int max_len, int d, int b,
+                              int K, float scale, void* o, void* ws, size_t ws_bytes,
+                              sas_stream_t stream) {
+  sas_status_t st = check_decode(dtype, B, Hq, Hkv, max_len, max_len, d, b, K, false, scale);
+  if (st != SAS_OK) return st;
+  if (num_pages < 1 || page_size < 1) return SAS_ERR_INVALID_ARG;
+  if (page_size < 16 || (page_size & (page_size - 1)) != 0 || page_size > (1 << 20))
+    return SAS_ERR_UNSUPPORTED;
+  if ((long long)num_pages * Hkv > 0x7fffffffLL) return SAS_ERR_UNSUPPORTED;
+  if (dtype != SAS_BF16 || d != 128 || b != 64) return SAS_ERR_UNSUPPORTED;
+  if (B == 0) return SAS_OK;
+  if (!q || !kpages || !vpages || !page_indptr || !page_indices || !seq_lens || !idx || !o)
+    return SAS_ERR_INVALID_ARG;
+  if (use_gates && !gates && (max_len - 1) / b > 0) return SAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(kpages, 16) || !aligned(vpages, 16) || !aligned(o, 16) ||
+      !aligned(idx, 4) || !aligned(page_indptr, 4) || !aligned(page_indices, 4) ||
+      !aligned(seq_lens, 4) || (gates && !aligned(gates, 4)))
+    return SAS_ERR_INVALID_ARG;
+  DecodeShape s = make_decode(B, Hq, Hkv, max_len, max_len, d, b, K, scale, false, use_gates);
+  s.paged = true;
+  if (!tc_decode_supported(dtype, s)) return SAS_ERR_UNSUPPORTED;
+  if (s.splits > 1 && (!ws || ws_bytes < decode_workspace_bytes(s) || !aligned(ws, 256)))
+    return SAS_ERR_WORKSPACE;
+  DevCtx ctx;
+  if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
+  const PagedArgs pa = {page_indptr, page_indices, seq_lens, page_size, num_pages};
+  return cuda_status(
+      launch_decode_paged_tc(s, pa, q, kpages, vpages, idx, gates, o, ws, ctx, stream));
+}
 
 sas_status_t sas_dense_fwd(sas_dtype_t dtype, const void* q, const void* k, const void* v, int B,
                            int Hq, int Hkv, int T, int d, int b, float scale, void* o, float* lse,

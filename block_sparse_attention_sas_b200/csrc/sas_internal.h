@@ -16,8 +16,9 @@ struct DevCtx;
 // Adds n to the library's launch counter (sas_launch_count).
 void note_launches(int n);
 
+// phi: a sas_phi_t value.
 cudaError_t launch_gate_topk(const float* scores, int B, int Hkv, int rows, int C, int causal,
-                             int K, float* gates, int32_t* idx, cudaStream_t stream);
+                             int K, int phi, float* gates, int32_t* idx, cudaStream_t stream);
 
 // Problem description shared by the attention launchers.
 struct AttnShape {
@@ -25,6 +26,8 @@ struct AttnShape {
   float scale;   // already resolved (> 0)
   int N;         // ceil(T / b)
   bool dense;    // every history block, no idx / gates
+  bool outer;    // outer gating (gate after the softmax); inner otherwise
+  int phi;       // gate activation (sas_phi_t) for the d scores Jacobian
 };
 
 // Workspace carve-up of the backward pass (byte offsets, 256-aligned).
@@ -53,7 +56,8 @@ cudaError_t launch_attn_bwd_tc(const AttnShape& s, const void* q, const void* k,
 // Shared pieces of the backward (defined with the SIMT kernels).
 cudaError_t launch_bwd_csr(const AttnShape& s, const int32_t* idx, int32_t* off, int32_t* list,
                            const DevCtx& ctx, cudaStream_t stream);
-// da holds RC row chunks per (head, query block, slot).
+// da holds RC row chunks per (head, query block, slot); s.phi picks the
+// Jacobian of the gate activation.
 cudaError_t launch_bwd_jacobian(const AttnShape& s, const float* da, const int32_t* idx,
                                 const float* gates, float* dscores, int RC, cudaStream_t stream);
 // 3-D TMA map over a [planes][rows][128] bf16 tensor, 64x64 boxes, 128-byte swizzle.
@@ -74,6 +78,19 @@ struct DecodeShape {
   int use_gates;
   int splits;   // CTAs per (batch, kv head)
   int bps;      // blocks per split
+  bool cluster; // (tensor-core decode) a unit's splits form one cluster
+  bool paged;   // the cache is paged (L = the longest sequence, C its history)
+};
+
+// Page table of a paged KV cache: sequence bi owns the pages
+// indices[indptr[bi] .. indptr[bi + 1]) in logical order and has lens[bi]
+// tokens; token t sits at row t % P of its (t / P)-th page.
+struct PagedArgs {
+  const int32_t* indptr;
+  const int32_t* indices;
+  const int32_t* lens;
+  int P;          // tokens per page: a power of two, at least 16
+  int num_pages;
 };
 void decode_plan(DecodeShape& s);  // fills splits / bps
 size_t decode_workspace_bytes(const DecodeShape& s);
@@ -86,12 +103,19 @@ bool tc_decode_supported(sas_dtype_t dt, const DecodeShape& s);
 cudaError_t launch_decode_tc(const DecodeShape& s, const void* q, const void* kc, const void* vc,
                              const int32_t* idx, const float* gates, void* o, void* ws,
                              const DevCtx& ctx, cudaStream_t stream);
+// The same over a paged cache (s.paged; kpages / vpages [num_pages, Hkv, P, d]).
+cudaError_t launch_decode_paged_tc(const DecodeShape& s, const PagedArgs& pa, const void* q,
+                                   const void* kpages, const void* vpages, const int32_t* idx,
+                                   const float* gates, void* o, void* ws, const DevCtx& ctx,
+                                   cudaStream_t stream);
 // The same map with 64 x 64 x 2 boxes (two consecutive planes per box).
 cudaError_t make_tmap_bf16_2planes(void* map, const void* ptr, int rows, int planes);
 // 3-D TMA map over planes of `pitch_rows` rows, the first `rows` of each mapped.
 cudaError_t make_tmap_bf16_rows8(void* map_out, const void* ptr, int rows);
 cudaError_t make_tmap_bf16_pitched(void* map, const void* ptr, int rows, int pitch_rows,
                                    int planes);
+// Map over [planes][rows][128] bf16 with 64 x box_rows x 1 boxes (pages).
+cudaError_t make_tmap_bf16_box(void* map, const void* ptr, int rows, int planes, int box_rows);
 // Fixed-size device scratch for sas_decode_noalloc (no allocation involved).
 size_t decode_noalloc_capacity();
 cudaError_t decode_noalloc_scratch(void** out);

@@ -230,3 +230,49 @@ def small_decode_config(B=1, Hq=2, Hkv=1, L=100, d=16, b=16, K=2, dtype="f32",
                         score_std=2.0, seed=0) -> DecodeConfig:
     return DecodeConfig(f"adhoc-decode B{B} Hq{Hq}/Hkv{Hkv} L{L} d{d} b{b} K{K} {dtype}", B,
                         Hq, Hkv, L, d, b, K, dtype, score_std=score_std, seed=seed)
+
+
+@dataclass
+class PagedDecodeInputs:
+    q: np.ndarray             # [B, Hq, d]
+    kpages: np.ndarray        # [num_pages, Hkv, P, d]
+    vpages: np.ndarray        # [num_pages, Hkv, P, d]
+    page_indptr: np.ndarray   # [B + 1] int32
+    page_indices: np.ndarray  # [page_indptr[-1]] int32, a random placement
+    seq_lens: np.ndarray      # [B] int32
+    scores: np.ndarray        # [B, Hkv, Cmax] float32; row bi meaningful for its own C
+    meta: dict = field(default_factory=dict)
+
+
+def make_paged_decode_inputs(B: int, Hq: int, Hkv: int, lens, d: int, b: int, P: int,
+                             dtype: str = "bf16", score_std: float = 2.0, spare_pages: int = 5,
+                             seed: int = 0) -> PagedDecodeInputs:
+    """A paged KV cache for decode tests: ragged sequence lengths, pages
+    placed at random physical slots (plus unused spare pages, filled with NaN
+    so that a read of one shows), the last page of a sequence partly used."""
+    root = np.random.SeedSequence(seed)
+    s_q, s_k, s_v, s_s, s_p = root.spawn(5)
+    bf = dtype == "bf16"
+    lens = np.asarray(lens, np.int32)
+    npages = [(int(L) + P - 1) // P for L in lens]
+    total = sum(npages) + spare_pages
+    q = normal(s_q, (B, Hq, d), bf16=bf)
+    kp = normal(s_k, (total, Hkv, P, d), bf16=bf)
+    vp = normal(s_v, (total, Hkv, P, d), bf16=bf)
+    perm = np.random.default_rng(s_p).permutation(total).astype(np.int32)
+    indptr = np.concatenate([[0], np.cumsum(npages)]).astype(np.int32)
+    indices = perm[:indptr[-1]].copy()
+    used = np.zeros(total, bool)
+    used[indices] = True
+    kp[~used] = np.nan
+    vp[~used] = np.nan
+    # rows past each sequence's end in its last page: NaN as well
+    for bi, L in enumerate(lens):
+        last = indices[indptr[bi + 1] - 1]
+        tail = int(L) - (npages[bi] - 1) * P
+        kp[last, :, tail:] = np.nan
+        vp[last, :, tail:] = np.nan
+    Cmax = max(1, (int(lens.max()) - 1) // b)
+    scores = normal(s_s, (B, Hkv, Cmax), std=score_std)
+    return PagedDecodeInputs(q, kp, vp, indptr, indices, lens, scores,
+                             meta={"seed": seed, "P": P})

@@ -71,6 +71,35 @@ typedef enum {
   SAS_ERR_DEVICE = 6       /* (device) a device-side check failed, e.g. idx out of range */
 } sas_status_t;
 
+/*
+ * Gate variants: the two ablation axes of the method. [picx] Methodology,
+ * Eq. 4 leaves the activation phi open; the [review] Summary compares the
+ * method's softmax with sigmoid and raw-logit gates, and inner with outer
+ * gating; [picx] Gradient Analysis, Eq. 5 gives the gate gradient of both
+ * gatings. The pages print no formula for the variants; this library reads
+ * them as:
+ *   SAS_PHI_SOFTMAX  g = softmax(s) over the valid history (Eq. 6; the method)
+ *   SAS_PHI_SIGMOID  g_m = 1 / (1 + exp(-s_m)), elementwise, not normalised
+ *   SAS_PHI_RAW      log g_m = s_m (stored as g_m = exp(s_m); needs s < 88)
+ *   SAS_GATE_INNER   log g enters the logits: o = softmax(q K^T scale + log g) V
+ *                    (Eq. 9; the method)
+ *   SAS_GATE_OUTER   the gate scales the softmax weights after normalisation:
+ *                    o_i = sum_t g_{m(t)} p_it v_t with p = softmax(q K^T scale)
+ *                    over the same keys (g = 1 on the current block); lse is
+ *                    that of the ungated logits
+ * Top-K is over the scores for every phi (each is increasing).
+ */
+typedef enum {
+  SAS_PHI_SOFTMAX = 0,
+  SAS_PHI_SIGMOID = 1,
+  SAS_PHI_RAW = 2
+} sas_phi_t;
+
+typedef enum {
+  SAS_GATE_INNER = 0,
+  SAS_GATE_OUTER = 1
+} sas_gating_t;
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* sas_status_string(sas_status_t status);
 
@@ -152,6 +181,38 @@ sas_status_t sas_attn_bwd(sas_dtype_t dtype, const void* q, const void* k, const
                           size_t ws_bytes, sas_stream_t stream);
 
 /*
+ * Gate-variant forms of the three training calls ([review] Summary; [picx]
+ * Eq. 4 and Eq. 5; readings above). Arguments, layouts and errors are those
+ * of the calls without the suffix, which are the (SAS_PHI_SOFTMAX,
+ * SAS_GATE_INNER) case.
+ *   sas_gate_topk_phi: gates g = phi(s) (the selection does not depend on phi).
+ *   sas_attn_fwd_gated: gating selects inner (Eq. 9) or outer gating; gates
+ *     as written by sas_gate_topk_phi with any phi (NULL: gates off, where
+ *     both gatings are plain block-sparse attention).
+ *   sas_attn_bwd_gated: the backward of sas_attn_fwd_gated with the same
+ *     gating, o and lse; dscores through the Jacobian of phi:
+ *       softmax: dscores[j,k] = [k in I_j] da_k - g_k sum_{m in I_j} da_m
+ *       sigmoid: dscores[j,k] = [k in I_j] da_k (1 - g_k)
+ *       raw:     dscores[j,k] = [k in I_j] da_k
+ *     with da_m = dL/dlog g_m: the sum of dS over the tile for inner gating,
+ *     the sum of g_m p dP (Eq. 5, outer form, times g_m) for outer gating.
+ *     Workspace: sas_attn_bwd_workspace_size() of the same shape.
+ */
+sas_status_t sas_gate_topk_phi(const float* scores, int B, int Hkv, int rows, int C, int causal,
+                               int K, sas_phi_t phi, float* gates, int32_t* idx,
+                               sas_stream_t stream);
+sas_status_t sas_attn_fwd_gated(sas_dtype_t dtype, const void* q, const void* k, const void* v,
+                                const int32_t* idx, const float* gates, int B, int Hq, int Hkv,
+                                int T, int d, int b, int K, float scale, sas_gating_t gating,
+                                void* o, float* lse, sas_stream_t stream);
+sas_status_t sas_attn_bwd_gated(sas_dtype_t dtype, const void* q, const void* k, const void* v,
+                                const void* o, const float* lse, const void* dO,
+                                const int32_t* idx, const float* gates, int B, int Hq, int Hkv,
+                                int T, int d, int b, int K, float scale, sas_phi_t phi,
+                                sas_gating_t gating, void* dq, void* dk, void* dv,
+                                float* dscores, void* ws, size_t ws_bytes, sas_stream_t stream);
+
+/*
  * sas_decode - one query token per sequence over a KV cache, selected blocks
  * plus the current block ([picx] Eq. 2 with use_gates = 0, Eq. 9 with
  * use_gates = 1; [review] Summary: gates are dropped at inference while the
@@ -212,6 +273,38 @@ sas_status_t sas_decode_noalloc(sas_dtype_t dtype, const void* q, const void* kc
                                 int use_gates, int B, int Hq, int Hkv, int L, int Lcap, int d,
                                 int b, int K, float scale, void* o, sas_stream_t stream);
 size_t sas_decode_noalloc_max_scratch(void);
+
+/*
+ * sas_decode_paged - sas_decode over a paged KV cache, the layout the pages'
+ * deployment decodes from ([picx] Efficiency Benefits: an SGLang backend
+ * with FlashInfer kernels, GQA with per-group selection). The pages fix no
+ * layout; this call reads it as:
+ *   kpages, vpages [num_pages, Hkv, P, d] (dtype), P = page_size tokens per
+ *     page. Sequence bi owns the pages page_indices[page_indptr[bi] ..
+ *     page_indptr[bi + 1]) in logical order; its token t sits at row t % P
+ *     of its (t / P)-th page. Pages may be shared or in any order.
+ *   seq_lens [B] int32: tokens of each sequence (1 <= L_bi <= max_len); the
+ *     last page may be partly used (rows past L_bi are never read into o).
+ *   The query of sequence bi sits at L_bi - 1; its current block is
+ *   cb = floor((L_bi - 1)/b) and idx[bi] selects among its cb history blocks.
+ *   gates [B, Hkv, Cmax] fp32 with Cmax = floor((max_len - 1)/b) (row bi
+ *     valid for its first cb entries); read only when use_gates != 0.
+ *   page_indptr [B + 1], page_indices, seq_lens, idx: device int32.
+ *   The result equals sas_decode on each sequence's gathered contiguous cache.
+ *   Limits: bf16, d = 128, b = 64, G <= 8, P a power of two >= 16
+ *   (SAS_ERR_UNSUPPORTED otherwise). A length, page entry or idx entry out
+ *   of range is skipped and reported as SAS_ERR_DEVICE.
+ *   ws / ws_bytes: at least sas_decode_paged_workspace_size() bytes, as for
+ *   sas_decode.
+ */
+size_t sas_decode_paged_workspace_size(int B, int Hq, int Hkv, int max_len, int d, int b, int K);
+sas_status_t sas_decode_paged(sas_dtype_t dtype, const void* q, const void* kpages,
+                              const void* vpages, const int32_t* page_indptr,
+                              const int32_t* page_indices, const int32_t* seq_lens,
+                              const int32_t* idx, const float* gates, int use_gates, int B, int Hq,
+                              int Hkv, int num_pages, int page_size, int max_len, int d, int b,
+                              int K, float scale, void* o, void* ws, size_t ws_bytes,
+                              sas_stream_t stream);
 
 /*
  * Dense comparison kernels ([picx] Eq. 1 with a causal mask): every block is

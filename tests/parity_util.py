@@ -11,6 +11,8 @@ Tolerances (stated by the workload definitions, read as follows):
 """
 from __future__ import annotations
 
+import os
+
 import numpy as np
 import torch
 
@@ -33,6 +35,16 @@ def host(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
+def _log(name, dtype, stored, err, l2, scale):
+    """Appends the measured margin of a check to $SAS_PARITY_LOG (if set)."""
+    path = os.environ.get("SAS_PARITY_LOG")
+    if path:
+        test = os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0]
+        with open(path, "a") as f:
+            f.write(f"{test}\t{name}\t{dtype}/{stored}\terr={err:.4e}\tl2={l2:.4e}\t"
+                    f"max|y|={scale:.3e}\n")
+
+
 def check(name: str, got, want, dtype: str, stored: str | None = None):
     """Compare at the workload's tolerance. `stored` is the dtype the library
     writes the tensor in (defaults to the workload dtype); the half-ulp
@@ -46,11 +58,13 @@ def check(name: str, got, want, dtype: str, stored: str | None = None):
     scale = np.abs(want).max() if want.size else 0.0
     if dtype == "f32":
         rel = err.max() / max(scale, 1e-30) if want.size else 0.0
+        _log(name, dtype, stored, rel, rel, scale)
         assert rel <= F32_NORMWISE, f"{name}: normwise rel err {rel:.3e} > {F32_NORMWISE}"
         return rel
     ulp = BF16_RTOL_ULP if stored == "bf16" else 0.0
     excess = (err - ulp * np.abs(want)).max() if want.size else 0.0
     l2 = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
+    _log(name, dtype, stored, excess, l2, scale)
     assert excess <= BF16_ATOL, f"{name}: max abs err {excess:.3e} > {BF16_ATOL} (stored {stored})"
     assert l2 <= BF16_REL_L2, f"{name}: rel L2 err {l2:.3e} > {BF16_REL_L2}"
     return l2

@@ -120,3 +120,16 @@ def test_decode_rejects(raw):
 def test_wait_limit_setter_is_host_only(raw):
     raw.LIB.sas_set_wait_limit(1000)
     raw.LIB.sas_set_wait_limit(0)
+
+
+def test_gate_variant_arguments_are_checked(raw):
+    """Unknown gate activations or gatings are rejected before any launch."""
+    L = raw.LIB
+    st = L.sas_gate_topk_phi(FAKE, 1, 1, 4, 4, 1, 2, 3, FAKE, FAKE, None)
+    assert st == 1
+    a = (1, FAKE, FAKE, FAKE, FAKE, None, 1, 4, 2, 128, 128, 64, 2, 0.0)
+    assert L.sas_attn_fwd_gated(*a, 2, FAKE, FAKE, None) == 1
+    assert L.sas_attn_fwd_gated(*a, -1, FAKE, FAKE, None) == 1
+    b = (1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 4, 2, 128, 128, 64, 2, 0.0)
+    assert L.sas_attn_bwd_gated(*b, 5, 0, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None) == 1
+    assert L.sas_attn_bwd_gated(*b, 0, 9, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None) == 1
