@@ -36,6 +36,7 @@
 // prefetch) is done, so that prologue overlaps the tail of the Top-K.
 // Every wait is bounded.
 #include <math.h>
+#include <stddef.h>
 
 #include <mutex>
 
@@ -73,7 +74,8 @@ struct Ctl {
   int abort, nblk;
   int blocks[kMaxSlotsPerSplit];
   float bias[kMaxSlotsPerSplit];  // log2-domain gate bias
-  union {
+  // 16-byte aligned: the cluster merge moves part_o rows as float4.
+  union alignas(16) {
     struct {
       float wgt[kMaxG * 64];  // merge weights of the last CTA
       // This split's partial for the cluster merge: unnormalised o per head.
@@ -91,6 +93,8 @@ struct Ctl {
   float mw[16], ml[16];  // the cluster's (max, sum) of the head being merged
 };
 constexpr size_t kSmem = kOffCtl + sizeof(Ctl) + 1024;
+static_assert(kOffCtl % 16 == 0 && offsetof(Ctl, part_o) % 16 == 0 && (kD * 4) % 16 == 0,
+              "the float4 accesses of part_o need 16-byte alignment");
 
 template <int G>
 __global__ void __launch_bounds__(kThreads, 2)

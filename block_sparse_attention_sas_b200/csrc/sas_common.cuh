@@ -99,6 +99,7 @@ __device__ __forceinline__ bool mbar_wait(const DevCtx& c, uint64_t* bar, uint32
 // hardware co-schedules a cluster's CTAs, so the barrier always completes
 // once each of them has arrived.
 __device__ __forceinline__ void cluster_sync_all() {
+  __syncwarp();  // the .aligned forms need the whole warp converged
   asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
                "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
