@@ -362,6 +362,11 @@ def run_ours(args):
         other_train.append(run_train_line(S, torch, dev, W.QWEN3_8B_TRAIN, flush, peaks,
                                           max(3, min(args.steps, 10)), 2, rank))
 
+    # ---- the dense causal comparison on the same layer (speedup denominator)
+    dense_line = None
+    if not args.no_dense:
+        dense_line = run_dense_line(S, torch, dev, cfg, d, flush, peaks, step_ms)
+
     # ---- roofline of the dominant call of the training step
     dom = max(k_ms, key=k_ms.get)
     dom_flops = {"sas_attn_fwd": f_fwd, "sas_attn_bwd": f_bwd}.get(dom, 0.0)
@@ -388,6 +393,7 @@ def run_ours(args):
         "clocks": clocks,
         "decode": decode_lines,
         "train_other": other_train,
+        "dense_train": dense_line,
         "wall_s_timed": t_wall,
     }
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -514,6 +520,40 @@ def run_train_line(S, torch, dev, cfg, flush, peaks, steps, warmup, rank):
     return {"workload": cfg.name, "ms_per_step": ms, "gate_fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
             "TFLOP/s": tf, "frac": tf / peaks["bf16_tflops"],
             "algorithmic_tflop_per_step": (f_fwd + f_bwd) / 1e12}
+
+
+def run_dense_line(S, torch, dev, cfg, d, flush, peaks, sparse_ms):
+    """Dense causal attention (every block, no gates) forward + backward on
+    the same inputs through sas_dense_fwd / sas_dense_bwd, device-timed (L2
+    flushed before each step); the sparse step's speedup over it."""
+    stream = torch.cuda.current_stream(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(3)]
+
+    def one(ev=None):
+        if ev:
+            ev[0].record(stream)
+        o, lse = S.dense_fwd(d["q"], d["k"], d["v"], b=cfg.b)
+        if ev:
+            ev[1].record(stream)
+        S.dense_bwd(d["q"], d["k"], d["v"], o, lse, d["dO"], b=cfg.b)
+        if ev:
+            ev[2].record(stream)
+
+    one()
+    for e in evs:
+        flush.zero_()
+        torch.cuda._sleep(HEAD_START_CYCLES)
+        one(e)
+    torch.cuda.synchronize(dev)
+    fwd_ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
+    pairs = attended_pairs(cfg.B, cfg.Hq, cfg.T, cfg.b, cfg.N)
+    flops = 14 * cfg.d * pairs
+    tf = flops / ((fwd_ms + bwd_ms) * 1e-3) / 1e12
+    return {"workload": cfg.name + " dense causal", "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+            "ms_per_step": fwd_ms + bwd_ms, "algorithmic_tflop_per_step": flops / 1e12,
+            "TFLOP/s": tf, "frac": tf / peaks["bf16_tflops"],
+            "speedup_sparse_step": (fwd_ms + bwd_ms) / sparse_ms}
 
 
 def bench_decode(S, torch, dev, stream, flush, peaks, args, rank):
@@ -704,6 +744,7 @@ def main():
     ap.add_argument("--profile-train", type=int, default=0, metavar="T",
                     help="run only the training step at sequence length T (for profiling)")
     ap.add_argument("--no-8b", action="store_true", help="skip the Qwen3-8B training line")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense training line")
     ap.add_argument("--dry-run", action="store_true",
                     help="CPU only: exercise the rank launch and timing reduction on gloo")
     args = ap.parse_args()

@@ -797,7 +797,7 @@ BwdWorkspace bwd_workspace_layout(const AttnShape& s, bool tc) {
   // dS tiles of every (query block, 128-row tile, slot) for the dq kernel:
   // [B][Hkv][N][G/2][K + 1][128][64] bf16 (slot K: the current block).
   L.off_ds = off;
-  if (tc)
+  if (tc && !s.dense)  // the dense comparison recomputes dS for dq instead
     off = align256(off + sizeof(uint16_t) * (size_t)s.B * s.Hkv * s.N * (s.Hq / s.Hkv / 2) *
                              (s.K + 1) * 128 * 64);
   L.total = off;

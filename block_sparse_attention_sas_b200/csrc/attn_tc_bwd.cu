@@ -95,11 +95,15 @@ tc_bwd_d_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   Ctl& c = *reinterpret_cast<Ctl*>(base + kOffCtl);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int j = blockIdx.x, kvh = blockIdx.y / TILES, u = blockIdx.y % TILES, bi = blockIdx.z;
+  // Dense: every history block, the longest query blocks first.
+  const int j = s.dense ? s.N - 1 - (int)blockIdx.x : (int)blockIdx.x;
+  const int kvh = blockIdx.y / TILES, u = blockIdx.y % TILES, bi = blockIdx.z;
   const int G = 2 * TILES;
   const int h0 = kvh * G + 2 * u;  // the tile's two heads: h0, h0 + 1
   const long long irow = ((long long)(bi * s.Hkv + kvh) * s.N + j);
   volatile int* abort = &c.abort;
+  // Block n of the list: the selected blocks then j; dense: 0 .. j.
+  auto blk = [&](int n) -> int { return s.dense ? n : c.blocks[n]; };
 
   const int quarter = warp & 3;
   const int rowi = quarter * 32 + lane;
@@ -139,17 +143,20 @@ tc_bwd_d_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tma_prefetch_desc(&tm_v);
     }
     __syncwarp();
-    const int n = warp_build_list(idx + irow * s.K, gates ? gates + irow * s.N : nullptr, s.K, j,
-                                  0, c.blocks, nullptr, c.bias, ctx);
-    if (lane == 0) {
-      c.blocks[n] = j;
-      c.bias[n] = 0.f;
-      c.nblk = n + 1;
+    int n = j;
+    if (!s.dense) {
+      n = warp_build_list(idx + irow * s.K, gates ? gates + irow * s.N : nullptr, s.K, j, 0,
+                          c.blocks, nullptr, c.bias, ctx);
+      if (lane == 0) {
+        c.blocks[n] = j;
+        c.bias[n] = 0.f;
+      }
     }
+    if (lane == 0) c.nblk = n + 1;
     __syncwarp();
     if (lane == 0) {
       for (; issued < n + 1 && issued < 1; ++issued) {  // stage 1 holds dO until it is in TMEM
-        const int m = c.blocks[issued];
+        const int m = blk(issued);
         unsigned char* kv = base + kOffKV + issued * 32768;
         mbar_arrive_expect_tx(&c.kv_full[issued], 32768);
         for (int h2 = 0; h2 < 2; ++h2) {
@@ -177,7 +184,7 @@ tc_bwd_d_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int n = issued; go && n < nblk; ++n) {
         const int st = n & 1;
         if (n >= 2 && !wait_or_abort(ctx, &c.kv_empty[st], ((n - 2) >> 1) & 1, abort)) break;
-        const int m = c.blocks[n];
+        const int m = blk(n);
         unsigned char* kv = base + kOffKV + st * 32768;
         mbar_arrive_expect_tx(&c.kv_full[st], 32768);
         for (int h2 = 0; h2 < 2; ++h2) {
@@ -248,8 +255,8 @@ tc_bwd_d_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         break;
       }
       fence_after_sync();
-      const int m = c.blocks[n];
-      const float bias = c.bias[n];
+      const int m = blk(n);
+      const float bias = s.dense ? 0.f : c.bias[n];
       const bool cur = (n == nblk - 1);
       const int kvalid = min(kB, s.T - m * kB);
       const float off = live ? bias - lse2 : -INFINITY;
@@ -308,6 +315,319 @@ tc_bwd_d_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (warp == 1) {
     fence_after_sync();
     tmem_dealloc(tmem, kTmemColsD);
+  }
+}
+
+// ============================================================================
+// Kernel R: dq with S and dP recomputed, for problems whose dS tiles are not
+// kept (the dense comparison, where they would take B*Hkv*N*N*(G/2)*16 KB).
+// ============================================================================
+// One CTA per (query block j, 128-row tile of two heads, KV head, batch),
+// laid out as the D kernel: Q and dO are copied into TMEM (the A operand of
+// S and dP), K/V stream through a two-stage ring. Per block: S and dP into
+// TMEM; the elementwise warps form dS = P (dP - D) as bf16 in a swizzled
+// shared tile; dQ += dS K (four M=128 N=128 MMAs, K read as an MN-major
+// operand) accumulates in TMEM, and the block's stage is freed once those
+// MMAs are done. The epilogue scales dQ and stores it.
+namespace kr {
+constexpr int kThreadsR = 256;   // warp 0 producer + list, warp 1 MMA, warps 4-7 rows
+constexpr uint32_t kTmemColsR = 512;
+constexpr uint32_t kColQ = 0, kColDO = 64, kColS = 128, kColDP = 192, kColDQ = 256;
+constexpr uint32_t kOffStage = 0;       // Q: [k half][128 rows][128 B]; dO in KV stage 1
+constexpr uint32_t kOffKV = 32768;      // 2 stages x (K halves, V halves)
+constexpr uint32_t kOffDS = kOffKV + 2 * 32768;  // dS: [128 rows][128 B]
+constexpr uint32_t kOffCtl = kOffDS + 16384;
+struct Ctl {
+  uint64_t qd_full, qd_free, kv_full[2], kv_empty[2], s_full, dp_full, ds_full, ds_free, dq_done,
+      drain;
+  uint32_t tmem_base;
+  int abort, nblk;
+  int blocks[kMaxList];
+  float bias[kMaxList];
+};
+constexpr size_t kSmem = kOffCtl + sizeof(Ctl) + 1024;
+}  // namespace kr
+
+template <int TILES>
+__global__ void __launch_bounds__(kr::kThreadsR, 1)
+tc_bwd_dq_recompute_kernel(const __grid_constant__ CUtensorMap tm_q,
+                           const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_v,
+                           const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ lse,
+                           const float* __restrict__ Dv, const int32_t* __restrict__ idx,
+                           const float* __restrict__ gates, AttnShape s,
+                           __nv_bfloat16* __restrict__ dq, DevCtx ctx) {
+  using namespace kr;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  unsigned char* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const uint32_t sbase = smem_u32(base);
+  Ctl& c = *reinterpret_cast<Ctl*>(base + kOffCtl);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int j = s.dense ? s.N - 1 - (int)blockIdx.x : (int)blockIdx.x;
+  const int kvh = blockIdx.y / TILES, u = blockIdx.y % TILES, bi = blockIdx.z;
+  const int G = 2 * TILES;
+  const int h0 = kvh * G + 2 * u;
+  const long long irow = ((long long)(bi * s.Hkv + kvh) * s.N + j);
+  volatile int* abort = &c.abort;
+  auto blk = [&](int n) -> int { return s.dense ? n : c.blocks[n]; };
+
+  const int quarter = warp & 3;
+  const int rowi = quarter * 32 + lane;
+  const int r = rowi & 63;
+  const int qrow = j * kB + r;
+  const bool live = qrow < s.T;
+  const long long hrow = (long long)(bi * s.Hq + h0 + (rowi >> 6)) * s.T + qrow;
+  float lse2 = 0.f, Di = 0.f;
+  if (warp >= 4 && live) {
+    lse2 = lse[hrow] * kLog2e;
+    Di = Dv[hrow];
+  }
+
+  int issued = 0;
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_init(&c.qd_full, 1);
+      mbar_init(&c.qd_free, 4);
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&c.kv_full[i], 5);  // expect-tx arrival + one per elementwise warp
+        mbar_init(&c.kv_empty[i], 1);
+      }
+      mbar_init(&c.s_full, 1);
+      mbar_init(&c.dp_full, 1);
+      mbar_init(&c.ds_full, 4);
+      mbar_init(&c.ds_free, 1);
+      mbar_init(&c.dq_done, 1);
+      mbar_init(&c.drain, 1);
+      fence_mbar_init();
+      c.abort = 0;
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_do);
+      mbar_arrive_expect_tx(&c.qd_full, 8 * 8192);
+      for (int h2 = 0; h2 < 2; ++h2)
+        for (int kb = 0; kb < 2; ++kb) {
+          tma_load_3d(base + kOffStage + kb * 16384 + h2 * 8192, &tm_q, kb * 64, j * kB,
+                      bi * s.Hq + h0 + h2, &c.qd_full);
+          tma_load_3d(base + kOffKV + 32768 + kb * 16384 + h2 * 8192, &tm_do, kb * 64, j * kB,
+                      bi * s.Hq + h0 + h2, &c.qd_full);
+        }
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
+    __syncwarp();
+    int n = j;
+    if (!s.dense) {
+      n = warp_build_list(idx + irow * s.K, gates ? gates + irow * s.N : nullptr, s.K, j, 0,
+                          c.blocks, nullptr, c.bias, ctx);
+      if (lane == 0) {
+        c.blocks[n] = j;
+        c.bias[n] = 0.f;
+      }
+    }
+    if (lane == 0) c.nblk = n + 1;
+    __syncwarp();
+    if (lane == 0) {
+      for (; issued < n + 1 && issued < 1; ++issued) {  // stage 1 holds dO until it is in TMEM
+        const int m = blk(issued);
+        unsigned char* kv = base + kOffKV + issued * 32768;
+        mbar_arrive_expect_tx(&c.kv_full[issued], 32768);
+        for (int h2 = 0; h2 < 2; ++h2) {
+          tma_load_3d(kv + h2 * 8192, &tm_k, h2 * 64, m * kB, bi * s.Hkv + kvh, &c.kv_full[issued]);
+          tma_load_3d(kv + 16384 + h2 * 8192, &tm_v, h2 * 64, m * kB, bi * s.Hkv + kvh,
+                      &c.kv_full[issued]);
+        }
+      }
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(&c.tmem_base, kTmemColsR);
+    tmem_relinquish();
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = c.tmem_base;
+  const int nblk = c.nblk;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      bool go = wait_or_abort(ctx, &c.qd_free, 0, abort);
+      for (int n = issued; go && n < nblk; ++n) {
+        const int st = n & 1;
+        if (n >= 2 && !wait_or_abort(ctx, &c.kv_empty[st], ((n - 2) >> 1) & 1, abort)) break;
+        const int m = blk(n);
+        unsigned char* kv = base + kOffKV + st * 32768;
+        mbar_arrive_expect_tx(&c.kv_full[st], 32768);
+        for (int h2 = 0; h2 < 2; ++h2) {
+          tma_load_3d(kv + h2 * 8192, &tm_k, h2 * 64, m * kB, bi * s.Hkv + kvh, &c.kv_full[st]);
+          tma_load_3d(kv + 16384 + h2 * 8192, &tm_v, h2 * 64, m * kB, bi * s.Hkv + kvh,
+                      &c.kv_full[st]);
+        }
+        issued = n + 1;
+      }
+      (void)mbar_wait(ctx, &c.qd_full, 0);
+      if (*abort)
+        for (int n = max(0, issued - 2); n < issued; ++n)
+          (void)mbar_wait(ctx, &c.kv_full[n & 1], (n >> 1) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16(128, 64, false, false);
+      const uint32_t id_q = idesc_bf16(128, 128, false, true);
+      const uint64_t dkv0 = sdesc_sw128(sbase + kOffKV, 16, 1024);
+      const uint64_t dds0 = sdesc_sw128(sbase + kOffDS, 16, 1024);          // dS, K-major
+      const uint64_t dkb0 = sdesc_sw128(sbase + kOffKV, 8192, 1024);        // K as MN-major B
+      // S/dP of block n + 1 are issued as soon as the row warps hold S/dP(n)
+      // in registers, so they run while dS(n) is formed.
+      auto issue_sdp = [&](int n) -> bool {
+        const int st = n & 1;
+        if (!wait_or_abort(ctx, &c.kv_full[st], (n >> 1) & 1, abort)) return false;
+        fence_after_sync();
+        const uint64_t kd = dkv0 + ((st * 32768) >> 4);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_bf16_ts(tmem + kColS, tmem + kColQ + ks * 8,
+                      kd + (((ks >> 2) * 8192 + (ks & 3) * 32) >> 4), id_s, ks > 0);
+        mma_commit(&c.s_full);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_bf16_ts(tmem + kColDP, tmem + kColDO + ks * 8,
+                      kd + ((16384 + (ks >> 2) * 8192 + (ks & 3) * 32) >> 4), id_s, ks > 0);
+        mma_commit(&c.dp_full);
+        return true;
+      };
+      bool ok = nblk > 0 && issue_sdp(0);
+      for (int n = 0; ok && n < nblk; ++n) {
+        const int st = n & 1;
+        if (n + 1 < nblk && !issue_sdp(n + 1)) break;
+        if (!wait_or_abort(ctx, &c.ds_full, n & 1, abort)) break;
+        fence_after_sync();
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_bf16_ss(tmem + kColDQ, dds0 + ((ks * 32) >> 4),
+                      dkb0 + ((st * 32768 + ks * 2048) >> 4), id_q, (n > 0 || ks > 0));
+        mma_commit(&c.ds_free);
+        mma_commit(&c.kv_empty[st]);
+      }
+      mma_commit(&c.dq_done);
+      if (*abort) {
+        mma_commit(&c.drain);
+        (void)mbar_wait(ctx, &c.drain, 0);
+      }
+    }
+  } else if (warp >= 4) {
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    const float sc = s.scale * kLog2e;
+    const uint64_t sc2 = f2u(sc, sc);
+    bool ok = warp_wait(ctx, &c.qd_full, 0, abort);
+    if (ok) {
+      tile_row_to_tmem(base + kOffStage, rowi, tl + kColQ);
+      tile_row_to_tmem(base + kOffKV + 32768, rowi, tl + kColDO);
+      tmem_st_wait();
+    }
+    fence_before_sync();
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&c.qd_free);     // stage 1 may take block 1
+      mbar_arrive(&c.kv_full[0]);  // Q, dO in TMEM: S/dP(0) may start
+    }
+    unsigned char* dsrow = base + kOffDS + rowi * 128;
+    for (int n = 0; ok && n < nblk; ++n) {
+      if (!warp_wait(ctx, &c.s_full, n & 1, abort)) {
+        ok = false;
+        break;
+      }
+      fence_after_sync();
+      const int m = blk(n);
+      const float bias = s.dense ? 0.f : c.bias[n];
+      const bool cur = (n == nblk - 1);
+      const int kvalid = min(kB, s.T - m * kB);
+      const float dinv = s.outer ? fminf(ex2(-bias), 3.0e38f) : 1.f;
+      const float off = live ? bias - lse2 : -INFINITY;
+      const uint64_t off2 = f2u(off, off);
+      float pf[64];
+      {
+        uint32_t sr[64];
+        tmem_ld32(tl + kColS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(tl + kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_ld_wait();
+        if (cur || kvalid < kB) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i)
+            if (i >= kvalid || (cur && i > r)) sr[i] = __float_as_uint(-INFINITY);
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const uint64_t a2 = ffma2(f2u(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
+                                    sc2, off2);
+          const uint64_t p2 = ((i & 3) == 3) ? ex2_poly2(a2) : f2u(ex2(lo_f(a2)), ex2(hi_f(a2)));
+          pf[2 * i] = lo_f(p2);
+          pf[2 * i + 1] = hi_f(p2);
+        }
+      }
+      if (!warp_wait(ctx, &c.dp_full, n & 1, abort)) {
+        ok = false;
+        break;
+      }
+      fence_after_sync();
+      uint32_t pr[64];
+      tmem_ld32(tl + kColDP, *reinterpret_cast<uint32_t(*)[32]>(&pr[0]));
+      tmem_ld32(tl + kColDP + 32, *reinterpret_cast<uint32_t(*)[32]>(&pr[32]));
+      tmem_ld_wait();
+      // S/dP(n) are in registers: S/dP(n + 1) may overwrite the accumulators.
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0 && n + 1 < nblk) mbar_arrive(&c.kv_full[(n + 1) & 1]);
+      uint32_t dd[32];
+      const uint64_t negD = f2u(-Di * dinv, -Di * dinv);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const uint64_t dp2 = f2u(__uint_as_float(pr[2 * i]), __uint_as_float(pr[2 * i + 1]));
+        const uint64_t ds2 = fmul2(f2u(pf[2 * i], pf[2 * i + 1]), fadd2(dp2, negD));
+        dd[i] = pack_bf16(lo_f(ds2), hi_f(ds2));
+      }
+      // The dS tile is free once dQ(n - 1) has read it.
+      if (n >= 1 && !warp_wait(ctx, &c.ds_free, (n - 1) & 1, abort)) {
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch)
+        *reinterpret_cast<uint4*>(dsrow + ((ch ^ (rowi & 7)) << 4)) =
+            make_uint4(dd[4 * ch], dd[4 * ch + 1], dd[4 * ch + 2], dd[4 * ch + 3]);
+      fence_proxy_async_smem();
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&c.ds_full);
+    }
+    if (ok && warp_wait(ctx, &c.dq_done, 0, abort)) {
+      fence_after_sync();
+      __nv_bfloat16* drow = dq + hrow * kD;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t ov[32];
+        tmem_ld32(tl + kColDQ + ch * 32, ov);
+        tmem_ld_wait();
+        if (live) {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 v;
+            v.x = pack_bf16(__uint_as_float(ov[8 * q4 + 0]) * s.scale, __uint_as_float(ov[8 * q4 + 1]) * s.scale);
+            v.y = pack_bf16(__uint_as_float(ov[8 * q4 + 2]) * s.scale, __uint_as_float(ov[8 * q4 + 3]) * s.scale);
+            v.z = pack_bf16(__uint_as_float(ov[8 * q4 + 4]) * s.scale, __uint_as_float(ov[8 * q4 + 5]) * s.scale);
+            v.w = pack_bf16(__uint_as_float(ov[8 * q4 + 6]) * s.scale, __uint_as_float(ov[8 * q4 + 7]) * s.scale);
+            *reinterpret_cast<uint4*>(drow + ch * 32 + q4 * 8) = v;
+          }
+        }
+      }
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after_sync();
+    tmem_dealloc(tmem, kTmemColsR);
   }
 }
 
@@ -581,12 +901,17 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t sbase = smem_u32(base);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int unit = order[blockIdx.x];
-  const int m = unit % s.N, bh = unit / s.N, kvh = bh % s.Hkv, bi = bh / s.Hkv;
+  // Dense: key block m is attended by every query block j >= m; the units
+  // go longest list (smallest m) first without a reverse index.
+  const int BH = s.B * s.Hkv;
+  const int unit = s.dense ? 0 : order[blockIdx.x];
+  const int m = s.dense ? (int)blockIdx.x / BH : unit % s.N;
+  const int bh = s.dense ? (int)blockIdx.x % BH : unit / s.N;
+  const int kvh = bh % s.Hkv, bi = bh / s.Hkv;
   const int G = 2 * TILES;
-  const int lo = csr_off[(long long)bh * (s.N + 1) + m];
-  const int nl = csr_off[(long long)bh * (s.N + 1) + m + 1] - lo;
-  const int32_t* lst = csr_list + (long long)bh * s.N * s.K + lo;
+  const int lo = s.dense ? 0 : csr_off[(long long)bh * (s.N + 1) + m];
+  const int nl = s.dense ? s.N - 1 - m : csr_off[(long long)bh * (s.N + 1) + m + 1] - lo;
+  const int32_t* lst = s.dense ? nullptr : csr_list + (long long)bh * s.N * s.K + lo;
   const int nsteps = (1 + nl) * TILES;
   // Step s covers tile (s % TILES) of query block j(s): first the diagonal
   // block m, then the selecting blocks in ascending order (entry / K of the
@@ -639,13 +964,16 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
     // The reverse list in a register window (lane l holds entry win_lo + l),
     // with the next window already in flight.
     int win_lo = 0;
-    int win = lane < nl ? lst[lane] : 0;
-    int win_next = 32 + lane < nl ? lst[32 + lane] : 0;
+    int win = (lst && lane < nl) ? lst[lane] : 0;
+    int win_next = (lst && 32 + lane < nl) ? lst[32 + lane] : 0;
     auto prefetch = [&](int st_i) -> Pre {
       Pre p;
       const int jj = st_i / TILES, u = st_i % TILES;
       int j = m, slot = s.K;  // the diagonal step's tile sits after the K slots
-      if (jj > 0) {
+      if (jj > 0 && s.dense) {
+        j = m + jj;
+        slot = 0;
+      } else if (jj > 0) {
         const int ix = jj - 1;
         while (ix >= win_lo + 32) {
           win = win_next;
@@ -808,8 +1136,10 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (!wait_or_abort(ctx, &c.pds_full[b], ph, abort)) break;
         const int j = c.buf_j[b], slot = c.buf_slot[b];
         const long long tile = (((long long)bh * s.N + j) * TILES + u) * (s.K + 1) + slot;
-        bulk_s2g(ds_out + tile * (128 * 64), base + kOffPD + b * 32768 + 16384, 16384);
-        bulk_commit();
+        if (ds_out != nullptr) {  // the dense comparison keeps no tiles
+          bulk_s2g(ds_out + tile * (128 * 64), base + kOffPD + b * 32768 + 16384, 16384);
+          bulk_commit();
+        }
         if (da != nullptr && !wait_or_abort(ctx, &c.da_full[b], ph, abort)) break;
         if (da != nullptr && slot < s.K) {
 #pragma unroll
@@ -960,7 +1290,7 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
 
 bool tc_bwd_supported(sas_dtype_t dt, const AttnShape& s) {
   const int G = s.Hq / s.Hkv;
-  return dt == SAS_BF16 && s.d == kD && s.b == kB && (G == 2 || G == 4) && !s.dense;
+  return dt == SAS_BF16 && s.d == kD && s.b == kB && (G == 2 || G == 4);
 }
 
 cudaError_t launch_attn_bwd_tc(const AttnShape& s, const void* q, const void* k, const void* v,
@@ -986,6 +1316,40 @@ cudaError_t launch_attn_bwd_tc(const AttnShape& s, const void* q, const void* k,
   CUtensorMap tq2, tdo2;  // 64 x 64 x 2 boxes for the dK/dV kernel's 128-row tiles
   if ((e = make_tmap_bf16_2planes(&tq2, q, s.T, s.B * s.Hq)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16_2planes(&tdo2, dO, s.T, s.B * s.Hq)) != cudaSuccess) return e;
+  if (s.dense) {
+    // Every block: no reverse index, no dS tiles (dq recomputes them), no da.
+    {
+      dim3 grid(s.N, s.Hkv * tiles, s.B);
+      auto kern = tiles == 2 ? tc_bwd_d_kernel<2> : tc_bwd_d_kernel<1>;
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kd::kSmem);
+      if (e != cudaSuccess) return e;
+      kern<<<grid, kd::kThreadsD, kd::kSmem, st>>>(tq, tk, tv, tdo, lse, nullptr, nullptr, s, Dv,
+                                                   ctx);
+      note_launches(1);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    {
+      dim3 grid(s.N * s.Hkv * s.B);
+      auto kern = tiles == 2 ? tc_bwd_dkdv_kernel<2, false> : tc_bwd_dkdv_kernel<1, false>;
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kb_::kSmem);
+      if (e != cudaSuccess) return e;
+      kern<<<grid, kb_::kThreadsB, kb_::kSmem, st>>>(tq2, tk, tv, tdo2, lse, Dv, nullptr, nullptr,
+                                                     nullptr, nullptr, s, (__nv_bfloat16*)dk,
+                                                     (__nv_bfloat16*)dv, nullptr, nullptr, ctx);
+      note_launches(1);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    {
+      dim3 grid(s.N, s.Hkv * tiles, s.B);
+      auto kern = tiles == 2 ? tc_bwd_dq_recompute_kernel<2> : tc_bwd_dq_recompute_kernel<1>;
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kr::kSmem);
+      if (e != cudaSuccess) return e;
+      kern<<<grid, kr::kThreadsR, kr::kSmem, st>>>(tq, tk, tv, tdo, lse, Dv, nullptr, nullptr, s,
+                                                   (__nv_bfloat16*)dq, ctx);
+      note_launches(1);
+      return cudaGetLastError();
+    }
+  }
   if ((e = launch_bwd_csr(s, idx, coff, clist, ctx, st)) != cudaSuccess) return e;
   {
     const size_t smem = sizeof(int32_t) * ((size_t)s.N + 1);

@@ -95,7 +95,9 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   Ctl& c = *reinterpret_cast<Ctl*>(base + kOffCtl);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int j = blockIdx.x, kvh = blockIdx.y, bi = blockIdx.z;
+  // Dense: the longest query blocks (most keys) start first.
+  const int j = s.dense ? s.N - 1 - (int)blockIdx.x : (int)blockIdx.x;
+  const int kvh = blockIdx.y, bi = blockIdx.z;
   const int G = 2 * TILES;
   const long long irow = ((long long)(bi * s.Hkv + kvh) * s.N + j);
 
@@ -123,15 +125,20 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   }
   if (warp == 0) {
     // Attended blocks in order: block j (bias 0, the largest logits in
-    // expectation), then the selected history blocks in slot order.
+    // expectation), then the selected history blocks in slot order. The
+    // dense comparison attends block j, then 0 .. j-1 (no list needed).
     __syncwarp();
-    if (lane == 0) {
-      c.blocks[0] = j;
-      c.bias[0] = 0.f;
+    if (s.dense) {
+      if (lane == 0) c.nblk = j + 1;
+    } else {
+      if (lane == 0) {
+        c.blocks[0] = j;
+        c.bias[0] = 0.f;
+      }
+      const int n = warp_build_list(idx + irow * s.K, gates ? gates + irow * s.N : nullptr, s.K,
+                                    j, 1, c.blocks, nullptr, c.bias, ctx);
+      if (lane == 0) c.nblk = n;
     }
-    const int n = warp_build_list(idx + irow * s.K, gates ? gates + irow * s.N : nullptr, s.K, j,
-                                  1, c.blocks, nullptr, c.bias, ctx);
-    if (lane == 0) c.nblk = n;
   }
   if (warp == 1) {
     tmem_alloc(&c.tmem_base, kTmemCols);
@@ -159,7 +166,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (n >= kStages &&
             !wait_or_abort(ctx, &empty[st], ((n - kStages) / kStages) & 1, abort))
           break;
-        const int m = c.blocks[n];
+        const int m = s.dense ? (n == 0 ? j : n - 1) : c.blocks[n];
         unsigned char* dst = base + off + st * kKVBytes;
         mbar_arrive_expect_tx(&full[st], kKVBytes);
         for (int h2 = 0; h2 < 2; ++h2)
@@ -266,10 +273,11 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       // S(n) is in registers: S(n + 1) may overwrite the accumulator.
       if (lane == 0 && n + 1 < nblk) mbar_arrive(&c.k_full[(n + 1) % kStages]);
 
-      const int m = c.blocks[n];
+      const int m = s.dense ? (n == 0 ? j : n - 1) : c.blocks[n];
       // Inner gating: log2 g joins the logits. Outer: P is scaled by g.
-      const float bias = OUTER ? 0.f : c.bias[n];
-      const float wgt = OUTER ? ex2(c.bias[n]) : 1.f;
+      const float gb = s.dense ? 0.f : c.bias[n];
+      const float bias = OUTER ? 0.f : gb;
+      const float wgt = OUTER ? ex2(gb) : 1.f;
       const bool cur = (n == 0);
       const int kvalid = min(kB, s.T - m * kB);   // keys of the block inside the sequence
       // Full history blocks need no mask; the current block (causal) and a
@@ -507,7 +515,7 @@ cudaError_t make_tmap_bf16_box(void* map_out, const void* ptr, int rows, int pla
 
 bool tc_fwd_supported(sas_dtype_t dt, const AttnShape& s) {
   const int G = s.Hq / s.Hkv;
-  return dt == SAS_BF16 && s.d == kD && s.b == kB && (G == 2 || G == 4) && !s.dense;
+  return dt == SAS_BF16 && s.d == kD && s.b == kB && (G == 2 || G == 4);
 }
 
 cudaError_t launch_attn_fwd_tc(const AttnShape& s, const void* q, const void* k, const void* v,

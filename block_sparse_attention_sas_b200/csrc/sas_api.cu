@@ -419,11 +419,14 @@ sas_status_t sas_dense_fwd(sas_dtype_t dtype, const void* q, const void* k, cons
   DevCtx ctx;
   if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
   const AttnShape s = make_shape(B, Hq, Hkv, T, d, b, 0, scale, true);
+  if (tc_fwd_supported(dtype, s))
+    return cuda_status(launch_attn_fwd_tc(s, q, k, v, nullptr, nullptr, o, lse, ctx, stream));
   return cuda_status(launch_attn_fwd_simt(dtype, s, q, k, v, nullptr, nullptr, o, lse, ctx, stream));
 }
 
 size_t sas_dense_bwd_workspace_size(int B, int Hq, int Hkv, int T, int d, int b) {
   if (check_attn(SAS_BF16, B, Hq, Hkv, T, d, b, 0, true, 1.f) != SAS_OK) return 0;
+  // The general layout covers the tensor-core one (D first, no dS tiles).
   return bwd_workspace_layout(make_shape(B, Hq, Hkv, T, d, b, 0, 1.f, true), false).total;
 }
 
@@ -444,6 +447,9 @@ sas_status_t sas_dense_bwd(sas_dtype_t dtype, const void* q, const void* k, cons
   if (!ws || ws_bytes < need || !aligned(ws, 256)) return SAS_ERR_WORKSPACE;
   DevCtx ctx;
   if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
+  if (tc_bwd_supported(dtype, s))
+    return cuda_status(launch_attn_bwd_tc(s, q, k, v, lse, dO, nullptr, nullptr, dq, dk, dv,
+                                          nullptr, ws, ctx, stream));
   return cuda_status(launch_attn_bwd_simt(dtype, s, q, k, v, o, lse, dO, nullptr, nullptr, dq, dk,
                                           dv, nullptr, ws, ctx, stream));
 }

@@ -39,7 +39,10 @@ notes with its reason):
     the C = floor((L-1)/b) blocks before it are the history.
 
 All arithmetic is float64; inputs (fp32 or bf16 values) convert to float64
-exactly. Parity of every function here is pinned by tests against closed
+exactly. The optional ``operands="bf16"`` of the attention functions rounds
+the weights P and dL/dX to bf16 where they enter a product, as the operands
+of a bf16 tensor-core kernel are: the tests use it only to measure the
+rounding floor of such arithmetic, never as the reference result. Parity of every function here is pinned by tests against closed
 forms, brute force, library special cases and finite differences.
 """
 from __future__ import annotations
@@ -108,6 +111,25 @@ def gate_topk(scores, K: int, causal: bool = True):
 # Key set of one query block (Eq. 3 selection + the always-retained block)
 # ---------------------------------------------------------------------------
 
+def round_bf16(x) -> np.ndarray:
+    """x rounded to bfloat16 and returned as float64: first to float32
+    (nearest), then to the 8-bit-mantissa bfloat16 grid (nearest, ties to even
+    on the 16 dropped bits). This is the data path of a bf16 MMA operand
+    formed in fp32 registers. Used only to measure the rounding floor of
+    bf16-operand arithmetic (``operands="bf16"`` below), never for results."""
+    f = np.asarray(x, np.float64).astype(np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    keep = (u >> 16) & 1
+    r = (((u + 0x7FFF + keep) >> 16) << 16).astype(np.uint32)
+    out = r.view(np.float32).astype(np.float64)
+    return np.where(np.isfinite(f), out, f.astype(np.float64))
+
+
+def _ops(a, operands):
+    """An MMA operand as the arithmetic under test sees it."""
+    return round_bf16(a) if operands == "bf16" else a
+
+
 def _key_set(j: int, b: int, T: int, sel_row, logg_row, use_gates: bool):
     """Columns and additive biases for query block j.
 
@@ -157,10 +179,13 @@ def _default_scale(d, scale):
 # Forward (Eq. 9)
 # ---------------------------------------------------------------------------
 
-def attn_fwd_block(q, k, v, idx, logg, bi, kvh, j, b, scale=0.0, use_gates=True):
+def attn_fwd_block(q, k, v, idx, logg, bi, kvh, j, b, scale=0.0, use_gates=True,
+                   operands=None):
     """Eq. 9 for the G query heads of KV head ``kvh`` and the rows of block j.
 
-    Returns (o [G, rows, d], lse [G, rows]) in float64.
+    Returns (o [G, rows, d], lse [G, rows]) in float64. With operands="bf16"
+    the weights P enter P V rounded to bf16 (the error floor of bf16-operand
+    arithmetic; the method's result is operands=None).
     """
     q, k, v = np.asarray(q), np.asarray(k), np.asarray(v)
     Hq, T, d = q.shape[1], q.shape[2], q.shape[3]
@@ -178,12 +203,12 @@ def attn_fwd_block(q, k, v, idx, logg, bi, kvh, j, b, scale=0.0, use_gates=True)
         X = _block_logits(_f64(q[bi, h, r0:r1]), Kc, bias, nh, scale, r0, j * b)
         lse = _lse_rows(X)
         P = np.exp(X - lse[:, None])
-        O[g] = P @ Vc
+        O[g] = _ops(P, operands) @ Vc
         L[g] = lse
     return O, L
 
 
-def attn_fwd(q, k, v, idx, logg, b, scale=0.0, use_gates=True):
+def attn_fwd(q, k, v, idx, logg, b, scale=0.0, use_gates=True, operands=None):
     """Eq. 9 over every query block. Returns (o [B,Hq,T,d], lse [B,Hq,T])."""
     B, Hq, T, d = np.shape(q)
     Hkv = np.shape(k)[1]
@@ -194,7 +219,8 @@ def attn_fwd(q, k, v, idx, logg, b, scale=0.0, use_gates=True):
     for bi in range(B):
         for kvh in range(Hkv):
             for j in range(N):
-                O, L = attn_fwd_block(q, k, v, idx, logg, bi, kvh, j, b, scale, use_gates)
+                O, L = attn_fwd_block(q, k, v, idx, logg, bi, kvh, j, b, scale, use_gates,
+                                      operands)
                 r0, r1 = j * b, min(T, (j + 1) * b)
                 o[bi, kvh * G:(kvh + 1) * G, r0:r1] = O
                 lse[bi, kvh * G:(kvh + 1) * G, r0:r1] = L
@@ -205,7 +231,8 @@ def attn_fwd(q, k, v, idx, logg, b, scale=0.0, use_gates=True):
 # Backward: chain rule through Eq. 9, then Eq. 5 (inner) and the Eq. 6 Jacobian
 # ---------------------------------------------------------------------------
 
-def attn_bwd_block(q, k, v, dO, idx, logg, bi, kvh, j, b, scale=0.0, use_gates=True):
+def attn_bwd_block(q, k, v, dO, idx, logg, bi, kvh, j, b, scale=0.0, use_gates=True,
+                   operands=None):
     """Gradients contributed by query block j of KV head ``kvh``.
 
     For the loss L = sum(o * dO): returns a dict with
@@ -215,6 +242,8 @@ def attn_bwd_block(q, k, v, dO, idx, logg, bi, kvh, j, b, scale=0.0, use_gates=T
     where dL/dX = P * (dP - rowsum(P * dP)) is the softmax Jacobian applied to
     dP = dO V^T, and da_m sums dL/dX over block m's columns, all rows and all
     G heads (log g_m enters every logit of block m, shared by the group).
+    operands="bf16" rounds P and dL/dX to bf16 where they enter the products
+    (dv, dq, dk), the floor of bf16-operand arithmetic; da stays exact.
     """
     q, k, v, dO = np.asarray(q), np.asarray(k), np.asarray(v), np.asarray(dO)
     Hq, T, d = q.shape[1], q.shape[2], q.shape[3]
@@ -237,9 +266,10 @@ def attn_bwd_block(q, k, v, dO, idx, logg, bi, kvh, j, b, scale=0.0, use_gates=T
         P = np.exp(X - _lse_rows(X)[:, None])
         dP = dOb @ Vc.T
         dX = P * (dP - (P * dP).sum(axis=1, keepdims=True))
-        dq[g] = scale * (dX @ Kc)
-        dk_c += scale * (dX.T @ Qb)
-        dv_c += P.T @ dOb
+        dXo = _ops(dX, operands)
+        dq[g] = scale * (dXo @ Kc)
+        dk_c += scale * (dXo.T @ Qb)
+        dv_c += _ops(P, operands).T @ dOb
         dX_hist += dX[:, :nh].sum(axis=0)
     da = {}
     pos = 0
@@ -267,7 +297,7 @@ def dscores_row(da: dict, gates_row, n: int) -> np.ndarray:
     return out
 
 
-def attn_bwd(q, k, v, dO, idx, gates, logg, b, scale=0.0, use_gates=True):
+def attn_bwd(q, k, v, dO, idx, gates, logg, b, scale=0.0, use_gates=True, operands=None):
     """Full backward. Returns (dq, dk, dv, dscores) in float64.
 
     dscores has the shape of the training score tensor [B, Hkv, N, N]: row j
@@ -284,7 +314,8 @@ def attn_bwd(q, k, v, dO, idx, gates, logg, b, scale=0.0, use_gates=True):
     for bi in range(B):
         for kvh in range(Hkv):
             for j in range(N):
-                r = attn_bwd_block(q, k, v, dO, idx, logg, bi, kvh, j, b, scale, use_gates)
+                r = attn_bwd_block(q, k, v, dO, idx, logg, bi, kvh, j, b, scale, use_gates,
+                                   operands)
                 r0, r1 = j * b, min(T, (j + 1) * b)
                 dq[bi, kvh * G:(kvh + 1) * G, r0:r1] = r["dq"]
                 np.add.at(dk[bi, kvh], r["cols"], r["dk_c"])
@@ -359,7 +390,7 @@ def dscores_row_phi(da: dict, s_row, n: int, phi: str) -> np.ndarray:
     return out
 
 
-def attn_bwd_phi(q, k, v, dO, idx, scores, b, phi: str, scale=0.0):
+def attn_bwd_phi(q, k, v, dO, idx, scores, b, phi: str, scale=0.0, operands=None):
     """Inner gating (Eq. 9) with gates from ``phi``: (dq, dk, dv, dscores)."""
     _, logg, _ = gate_topk_phi(scores, idx.shape[-1], phi)
     B, Hq, T, d = np.shape(q)
@@ -373,7 +404,8 @@ def attn_bwd_phi(q, k, v, dO, idx, scores, b, phi: str, scale=0.0):
     for bi in range(B):
         for kvh in range(Hkv):
             for j in range(N):
-                r = attn_bwd_block(q, k, v, dO, idx, logg, bi, kvh, j, b, scale)
+                r = attn_bwd_block(q, k, v, dO, idx, logg, bi, kvh, j, b, scale,
+                                   operands=operands)
                 r0, r1 = j * b, min(T, (j + 1) * b)
                 dq[bi, kvh * G:(kvh + 1) * G, r0:r1] = r["dq"]
                 np.add.at(dk[bi, kvh], r["cols"], r["dk_c"])
@@ -393,7 +425,7 @@ def _col_gates(j, b, T, sel_row, gates_row):
     return np.asarray(w)
 
 
-def attn_fwd_outer_block(q, k, v, idx, gates, bi, kvh, j, b, scale=0.0):
+def attn_fwd_outer_block(q, k, v, idx, gates, bi, kvh, j, b, scale=0.0, operands=None):
     """Outer gating for the G heads of KV head ``kvh`` and block j's rows:
     o = (P * w) V with P the ungated softmax and w the per-column gates.
     Returns (o [G, rows, d], lse [G, rows]) where lse is the ungated one."""
@@ -410,12 +442,12 @@ def attn_fwd_outer_block(q, k, v, idx, gates, bi, kvh, j, b, scale=0.0):
     for g in range(G):
         X = _block_logits(_f64(q[bi, kvh * G + g, r0:r1]), Kc, bias, nh, scale, r0, j * b)
         lse = _lse_rows(X)
-        O[g] = (np.exp(X - lse[:, None]) * w[None, :]) @ Vc
+        O[g] = _ops(np.exp(X - lse[:, None]) * w[None, :], operands) @ Vc
         L[g] = lse
     return O, L
 
 
-def attn_fwd_outer(q, k, v, idx, gates, b, scale=0.0):
+def attn_fwd_outer(q, k, v, idx, gates, b, scale=0.0, operands=None):
     """Outer gating over every query block: (o [B,Hq,T,d], lse [B,Hq,T])."""
     B, Hq, T, d = np.shape(q)
     Hkv = np.shape(k)[1]
@@ -426,14 +458,14 @@ def attn_fwd_outer(q, k, v, idx, gates, b, scale=0.0):
     for bi in range(B):
         for kvh in range(Hkv):
             for j in range(N):
-                O, L = attn_fwd_outer_block(q, k, v, idx, gates, bi, kvh, j, b, scale)
+                O, L = attn_fwd_outer_block(q, k, v, idx, gates, bi, kvh, j, b, scale, operands)
                 r0, r1 = j * b, min(T, (j + 1) * b)
                 o[bi, kvh * G:(kvh + 1) * G, r0:r1] = O
                 lse[bi, kvh * G:(kvh + 1) * G, r0:r1] = L
     return o, lse
 
 
-def attn_bwd_outer_block(q, k, v, dO, idx, gates, bi, kvh, j, b, scale=0.0):
+def attn_bwd_outer_block(q, k, v, dO, idx, gates, bi, kvh, j, b, scale=0.0, operands=None):
     """Gradients of L = sum(o * dO) under outer gating from query block j.
 
     With W = P * w: dv += W^T dO; dL/dP = w * dP (dP = dO V^T), so the
@@ -461,9 +493,10 @@ def attn_bwd_outer_block(q, k, v, dO, idx, gates, bi, kvh, j, b, scale=0.0):
         dP = dOb @ Vc.T
         wdP = dP * w[None, :]
         dX = P * (wdP - (P * wdP).sum(axis=1, keepdims=True))
-        dq[g] = scale * (dX @ Kc)
-        dk_c += scale * (dX.T @ Qb)
-        dv_c += (P * w[None, :]).T @ dOb
+        dXo = _ops(dX, operands)
+        dq[g] = scale * (dXo @ Kc)
+        dk_c += scale * (dXo.T @ Qb)
+        dv_c += _ops(P * w[None, :], operands).T @ dOb
         pdp_hist += (P * dP)[:, :nh].sum(axis=0)
     da, pos = {}, 0
     for m in idx[bi, kvh, j]:
@@ -505,7 +538,8 @@ def gate_grad_eq5_outer(q, k, v, dO, idx, gates, bi, kvh, j, b, scale=0.0):
     return out
 
 
-def attn_bwd_outer(q, k, v, dO, idx, scores, b, phi: str = "softmax", scale=0.0):
+def attn_bwd_outer(q, k, v, dO, idx, scores, b, phi: str = "softmax", scale=0.0,
+                   operands=None):
     """Outer gating with gates from ``phi``: (dq, dk, dv, dscores)."""
     gates, _, _ = gate_topk_phi(scores, idx.shape[-1], phi)
     B, Hq, T, d = np.shape(q)
@@ -519,7 +553,8 @@ def attn_bwd_outer(q, k, v, dO, idx, scores, b, phi: str = "softmax", scale=0.0)
     for bi in range(B):
         for kvh in range(Hkv):
             for j in range(N):
-                r = attn_bwd_outer_block(q, k, v, dO, idx, gates, bi, kvh, j, b, scale)
+                r = attn_bwd_outer_block(q, k, v, dO, idx, gates, bi, kvh, j, b, scale,
+                                         operands)
                 r0, r1 = j * b, min(T, (j + 1) * b)
                 dq[bi, kvh * G:(kvh + 1) * G, r0:r1] = r["dq"]
                 np.add.at(dk[bi, kvh], r["cols"], r["dk_c"])

@@ -45,10 +45,13 @@ def _log(name, dtype, stored, err, l2, scale):
                     f"max|y|={scale:.3e}\n")
 
 
-def check(name: str, got, want, dtype: str, stored: str | None = None):
+def check(name: str, got, want, dtype: str, stored: str | None = None, floor=None):
     """Compare at the workload's tolerance. `stored` is the dtype the library
     writes the tensor in (defaults to the workload dtype); the half-ulp
-    allowance applies only to bf16-stored tensors."""
+    allowance applies only to bf16-stored tensors. `floor` (bf16 workloads):
+    per element |emulated - exact|, where `emulated` is the oracle with its
+    MMA operands (P, dS) rounded to bf16; twice it is allowed on top of the
+    2e-2 bound, since no bf16-operand arithmetic can avoid that rounding."""
     stored = dtype if stored is None else stored
     got = np.asarray(got, np.float64)
     want = np.asarray(want, np.float64)
@@ -62,12 +65,20 @@ def check(name: str, got, want, dtype: str, stored: str | None = None):
         assert rel <= F32_NORMWISE, f"{name}: normwise rel err {rel:.3e} > {F32_NORMWISE}"
         return rel
     ulp = BF16_RTOL_ULP if stored == "bf16" else 0.0
-    excess = (err - ulp * np.abs(want)).max() if want.size else 0.0
+    allow = ulp * np.abs(want)
+    if floor is not None:
+        allow = allow + 2.0 * np.asarray(floor, np.float64)
+    excess = (err - allow).max() if want.size else 0.0
     l2 = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
     _log(name, dtype, stored, excess, l2, scale)
     assert excess <= BF16_ATOL, f"{name}: max abs err {excess:.3e} > {BF16_ATOL} (stored {stored})"
     assert l2 <= BF16_REL_L2, f"{name}: rel L2 err {l2:.3e} > {BF16_REL_L2}"
     return l2
+
+
+def floor_of(exact, emulated):
+    """Per-element rounding floor of bf16-operand arithmetic."""
+    return np.abs(np.asarray(emulated, np.float64) - np.asarray(exact, np.float64))
 
 
 def oracle_gates_slice(scores, bi, kvh, K, causal=True):
@@ -76,17 +87,18 @@ def oracle_gates_slice(scores, bi, kvh, K, causal=True):
     return g[0, 0], lg[0, 0], ix[0, 0]
 
 
-def oracle_fwd_rows(x, b, K, bi, kvh, j, use_gates=True, cache=None):
+def oracle_fwd_rows(x, b, K, bi, kvh, j, use_gates=True, cache=None, operands=None):
     """Oracle o [G, rows, d] and lse [G, rows] for query block j of (bi, kvh)."""
     g, lg, ix = cache if cache is not None else oracle_gates_slice(x.scores, bi, kvh, K)
     idx = np.zeros((bi + 1, kvh + 1) + ix.shape, np.int32)
     idx[bi, kvh] = ix
     logg = np.zeros((bi + 1, kvh + 1) + lg.shape)
     logg[bi, kvh] = lg
-    return O.attn_fwd_block(x.q, x.k, x.v, idx, logg, bi, kvh, j, b, use_gates=use_gates)
+    return O.attn_fwd_block(x.q, x.k, x.v, idx, logg, bi, kvh, j, b, use_gates=use_gates,
+                            operands=operands)
 
 
-def oracle_bwd_sample(x, b, K, bi, kvh, js, ms, use_gates=True, cache=None):
+def oracle_bwd_sample(x, b, K, bi, kvh, js, ms, use_gates=True, cache=None, operands=None):
     """Oracle gradients for sampled query blocks js (dq rows, dscores rows) and
     sampled key blocks ms (dk, dv rows; summed over every query block whose
     key set contains block m)."""
@@ -99,7 +111,8 @@ def oracle_bwd_sample(x, b, K, bi, kvh, js, ms, use_gates=True, cache=None):
     N = ix.shape[0]
     out = {"dq": {}, "ds": {}, "dk": {}, "dv": {}}
     for j in js:
-        r = O.attn_bwd_block(x.q, x.k, x.v, x.dO, idx, logg, bi, kvh, j, b, use_gates=use_gates)
+        r = O.attn_bwd_block(x.q, x.k, x.v, x.dO, idx, logg, bi, kvh, j, b, use_gates=use_gates,
+                             operands=operands)
         out["dq"][j] = r["dq"]
         if use_gates:
             out["ds"][j] = np.concatenate([O.dscores_row(r["da"], g[j], j), np.zeros(N - j)])
@@ -111,7 +124,7 @@ def oracle_bwd_sample(x, b, K, bi, kvh, js, ms, use_gates=True, cache=None):
             if j != m and m not in set(int(t) for t in ix[j]):
                 continue
             r = O.attn_bwd_block(x.q, x.k, x.v, x.dO, idx, logg, bi, kvh, j, b,
-                                 use_gates=use_gates)
+                                 use_gates=use_gates, operands=operands)
             sel = (r["cols"] >= m * b) & (r["cols"] < m * b + rows)
             dk += r["dk_c"][sel]
             dv += r["dv_c"][sel]

@@ -91,7 +91,8 @@ def test_decode_paged_bad_page_is_reported(cuda_lib):
     idx, gates, _, _ = _select(cuda_lib, x, K, b)
     q, kp, vp, ip, ix, ln = _paged_tensors(x)
     ix_bad = ix.clone()
-    ix_bad[1] = kp.shape[0] + 7  # a page past the pool
+    # the last page of sequence 0 holds its current block, which is always read
+    ix_bad[int(x.page_indptr[1]) - 1] = kp.shape[0] + 7  # a page past the pool
     cuda_lib.device_error()
     cuda_lib.decode_paged(q, kp, vp, ip, ix_bad, ln, idx, gates, False, b, max_len=500)
     st, raw = cuda_lib.device_error()

@@ -11,7 +11,7 @@ import torch
 
 from block_sparse_attention_sas_b200 import workloads as W
 from oracle import sas_oracle as O
-from tests.parity_util import check, dev, host, oracle_bwd_sample, oracle_fwd_rows, \
+from tests.parity_util import check, dev, floor_of, host, oracle_bwd_sample, oracle_fwd_rows, \
     oracle_gates_slice
 
 pytestmark = pytest.mark.gpu
@@ -82,11 +82,18 @@ def _full_compare(lib, cfg, use_gates=True):
     o, lse = O.attn_fwd(x.q, x.k, x.v, ix, lg, cfg.b, use_gates=use_gates)
     dq, dk, dv, ds = O.attn_bwd(x.q, x.k, x.v, x.dO, ix, g, lg, cfg.b, use_gates=use_gates)
     dt = cfg.dtype
-    check("o", host(r["o"]), o, dt)
+    fl = {n: None for n in ("o", "dq", "dk", "dv")}
+    if dt == "bf16":  # the rounding floor of bf16 MMA operands
+        oe, _ = O.attn_fwd(x.q, x.k, x.v, ix, lg, cfg.b, use_gates=use_gates, operands="bf16")
+        e = O.attn_bwd(x.q, x.k, x.v, x.dO, ix, g, lg, cfg.b, use_gates=use_gates,
+                       operands="bf16")
+        fl = {"o": floor_of(o, oe), "dq": floor_of(dq, e[0]), "dk": floor_of(dk, e[1]),
+              "dv": floor_of(dv, e[2])}
+    check("o", host(r["o"]), o, dt, floor=fl["o"])
     check("lse", host(r["lse"]), lse, dt, stored="f32")
-    check("dq", host(r["dq"]), dq, dt)
-    check("dk", host(r["dk"]), dk, dt)
-    check("dv", host(r["dv"]), dv, dt)
+    check("dq", host(r["dq"]), dq, dt, floor=fl["dq"])
+    check("dk", host(r["dk"]), dk, dt, floor=fl["dk"])
+    check("dv", host(r["dv"]), dv, dt, floor=fl["dv"])
     if use_gates:
         check("dscores", host(r["ds"]), ds, dt, stored="f32")
     else:
@@ -132,19 +139,25 @@ def test_train_full_size_sampled(cuda_lib, name):
         check("gates", host(r["gates"][bi, kvh]), cache[0], "f32")
         for j in js:
             o, lse = oracle_fwd_rows(x, b, cfg.K, bi, kvh, j, cache=cache)
+            oe, _ = oracle_fwd_rows(x, b, cfg.K, bi, kvh, j, cache=cache, operands="bf16")
             sl = slice(j * b, (j + 1) * b)
-            check(f"o[{j}]", host(r["o"][bi, kvh * G:(kvh + 1) * G, sl]), o, cfg.dtype)
+            check(f"o[{j}]", host(r["o"][bi, kvh * G:(kvh + 1) * G, sl]), o, cfg.dtype,
+                  floor=floor_of(o, oe))
             check(f"lse[{j}]", host(r["lse"][bi, kvh * G:(kvh + 1) * G, sl]), lse, cfg.dtype,
                   stored="f32")
         ob = oracle_bwd_sample(x, b, cfg.K, bi, kvh, js, ms, cache=cache)
+        eb = oracle_bwd_sample(x, b, cfg.K, bi, kvh, js, ms, cache=cache, operands="bf16")
         for j in js:
             sl = slice(j * b, (j + 1) * b)
-            check(f"dq[{j}]", host(r["dq"][bi, kvh * G:(kvh + 1) * G, sl]), ob["dq"][j], cfg.dtype)
+            check(f"dq[{j}]", host(r["dq"][bi, kvh * G:(kvh + 1) * G, sl]), ob["dq"][j], cfg.dtype,
+                  floor=floor_of(ob["dq"][j], eb["dq"][j]))
             check(f"ds[{j}]", host(r["ds"][bi, kvh, j]), ob["ds"][j], cfg.dtype, stored="f32")
         for m in ms:
             sl = slice(m * b, (m + 1) * b)
-            check(f"dk[{m}]", host(r["dk"][bi, kvh, sl]), ob["dk"][m], cfg.dtype)
-            check(f"dv[{m}]", host(r["dv"][bi, kvh, sl]), ob["dv"][m], cfg.dtype)
+            check(f"dk[{m}]", host(r["dk"][bi, kvh, sl]), ob["dk"][m], cfg.dtype,
+                  floor=floor_of(ob["dk"][m], eb["dk"][m]))
+            check(f"dv[{m}]", host(r["dv"][bi, kvh, sl]), ob["dv"][m], cfg.dtype,
+                  floor=floor_of(ob["dv"][m], eb["dv"][m]))
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
@@ -156,20 +169,71 @@ def test_train_reverse_index_past_1024_blocks(cuda_lib, dtype):
     _full_compare(cuda_lib, cfg, True)
 
 
-def test_dense_matches_all_blocks_selected(cuda_lib):
-    cfg = W.small_train_config(B=1, Hq=4, Hkv=2, T=300, d=128, b=64, K=8, dtype="bf16")
+@pytest.mark.parametrize("kw", [
+    dict(B=1, Hq=4, Hkv=2, T=300, d=128, b=64, K=8, dtype="bf16"),     # tensor cores, G = 2
+    dict(B=2, Hq=8, Hkv=2, T=1000, d=128, b=64, K=8, dtype="bf16"),    # tensor cores, G = 4
+    dict(B=1, Hq=2, Hkv=2, T=200, d=64, b=16, K=8, dtype="bf16"),      # general kernels
+])
+def test_dense_matches_all_blocks_selected(cuda_lib, kw):
+    cfg = W.small_train_config(**kw)
+    x = W.make_train_inputs(cfg)
+    q, k, v, dO = (dev(a, "bf16") for a in (x.q, x.k, x.v, x.dO))
+    o, lse = cuda_lib.dense_fwd(q, k, v, b=cfg.b)
+    dq, dk, dv = cuda_lib.dense_bwd(q, k, v, o, lse, dO, b=cfg.b)
+    torch.cuda.synchronize()
+    assert cuda_lib.device_error()[0] == 0
+    oo, ol = O.dense_fwd(x.q, x.k, x.v, cfg.b)
+    idx = O.all_blocks_idx(cfg.B, cfg.Hkv, cfg.N)
+    odq, odk, odv, _ = O.attn_bwd(x.q, x.k, x.v, x.dO, idx, None, None, cfg.b, use_gates=False)
+    oe, _ = O.attn_fwd(x.q, x.k, x.v, idx, None, cfg.b, use_gates=False, operands="bf16")
+    e = O.attn_bwd(x.q, x.k, x.v, x.dO, idx, None, None, cfg.b, use_gates=False, operands="bf16")
+    check("dense o", host(o), oo, "bf16", floor=floor_of(oo, oe))
+    check("dense lse", host(lse), ol, "bf16", stored="f32")
+    check("dense dq", host(dq), odq, "bf16", floor=floor_of(odq, e[0]))
+    check("dense dk", host(dk), odk, "bf16", floor=floor_of(odk, e[1]))
+    check("dense dv", host(dv), odv, "bf16", floor=floor_of(odv, e[2]))
+
+
+@pytest.mark.slow
+def test_dense_long_sequence_sampled(cuda_lib):
+    """N = 300 blocks (more than a sparse block list holds): dense forward and
+    backward on the tensor cores, checked on sampled query and key blocks
+    against the oracle's all-blocks selection."""
+    cfg = W.small_train_config(B=1, Hq=4, Hkv=1, T=19200, d=128, b=64, K=8, dtype="bf16")
     x = W.make_train_inputs(cfg)
     q, k, v, dO = (dev(a, "bf16") for a in (x.q, x.k, x.v, x.dO))
     o, lse = cuda_lib.dense_fwd(q, k, v, b=64)
     dq, dk, dv = cuda_lib.dense_bwd(q, k, v, o, lse, dO, b=64)
-    oo, ol = O.dense_fwd(x.q, x.k, x.v, 64)
-    idx = O.all_blocks_idx(1, 2, cfg.N)
-    odq, odk, odv, _ = O.attn_bwd(x.q, x.k, x.v, x.dO, idx, None, None, 64, use_gates=False)
-    check("dense o", host(o), oo, "bf16")
-    check("dense lse", host(lse), ol, "bf16", stored="f32")
-    check("dense dq", host(dq), odq, "bf16")
-    check("dense dk", host(dk), odk, "bf16")
-    check("dense dv", host(dv), odv, "bf16")
+    torch.cuda.synchronize()
+    assert cuda_lib.device_error()[0] == 0
+    N = cfg.N
+    idx = O.all_blocks_idx(1, 1, N)
+    logg = np.zeros((1, 1, N, N))
+    for j in (0, 1, 150, N - 1):
+        oo, ol = O.attn_fwd_block(x.q, x.k, x.v, idx, logg, 0, 0, j, 64, use_gates=False)
+        oe, _ = O.attn_fwd_block(x.q, x.k, x.v, idx, logg, 0, 0, j, 64, use_gates=False,
+                                 operands="bf16")
+        sl = slice(j * 64, (j + 1) * 64)
+        check(f"dense o[{j}]", host(o[0, :, sl]), oo, "bf16", floor=floor_of(oo, oe))
+        check(f"dense lse[{j}]", host(lse[0, :, sl]), ol, "bf16", stored="f32")
+        r = O.attn_bwd_block(x.q, x.k, x.v, x.dO, idx, logg, 0, 0, j, 64, use_gates=False)
+        re_ = O.attn_bwd_block(x.q, x.k, x.v, x.dO, idx, logg, 0, 0, j, 64, use_gates=False,
+                               operands="bf16")
+        check(f"dense dq[{j}]", host(dq[0, :, sl]), r["dq"], "bf16",
+              floor=floor_of(r["dq"], re_["dq"]))
+    for m in (N - 1, N - 3):
+        acc = {op: [np.zeros((64, 128)), np.zeros((64, 128))] for op in (None, "bf16")}
+        for j in range(m, N):
+            for op in (None, "bf16"):
+                r = O.attn_bwd_block(x.q, x.k, x.v, x.dO, idx, logg, 0, 0, j, 64,
+                                     use_gates=False, operands=op)
+                sel = (r["cols"] >= m * 64) & (r["cols"] < (m + 1) * 64)
+                acc[op][0] += r["dk_c"][sel]
+                acc[op][1] += r["dv_c"][sel]
+        sl = slice(m * 64, (m + 1) * 64)
+        (dkm, dvm), (dke, dve) = acc[None], acc["bf16"]
+        check(f"dense dk[{m}]", host(dk[0, 0, sl]), dkm, "bf16", floor=floor_of(dkm, dke))
+        check(f"dense dv[{m}]", host(dv[0, 0, sl]), dvm, "bf16", floor=floor_of(dvm, dve))
 
 
 # ------------------------------------------------------------------ decode

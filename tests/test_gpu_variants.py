@@ -14,7 +14,7 @@ import torch
 
 from block_sparse_attention_sas_b200 import workloads as W
 from oracle import sas_oracle as O
-from tests.parity_util import check, dev, host
+from tests.parity_util import check, dev, floor_of, host
 
 pytestmark = pytest.mark.gpu
 
@@ -60,11 +60,16 @@ def test_inner_gating_with_phi(cuda_lib, kw, phi):
     oo, ol = O.attn_fwd(x.q, x.k, x.v, ix, lg, cfg.b)
     odq, odk, odv, ods = O.attn_bwd_phi(x.q, x.k, x.v, x.dO, ix, x.scores, cfg.b, phi)
     dt = cfg.dtype
-    check("o", host(o), oo, dt)
+    fl = [None] * 4
+    if dt == "bf16":  # the rounding floor of bf16 MMA operands
+        oe, _ = O.attn_fwd(x.q, x.k, x.v, ix, lg, cfg.b, operands="bf16")
+        e = O.attn_bwd_phi(x.q, x.k, x.v, x.dO, ix, x.scores, cfg.b, phi, operands="bf16")
+        fl = [floor_of(oo, oe), floor_of(odq, e[0]), floor_of(odk, e[1]), floor_of(odv, e[2])]
+    check("o", host(o), oo, dt, floor=fl[0])
     check("lse", host(lse), ol, dt, stored="f32")
-    check("dq", host(dq), odq, dt)
-    check("dk", host(dk), odk, dt)
-    check("dv", host(dv), odv, dt)
+    check("dq", host(dq), odq, dt, floor=fl[1])
+    check("dk", host(dk), odk, dt, floor=fl[2])
+    check("dv", host(dv), odv, dt, floor=fl[3])
     check(f"dscores ({phi})", host(ds), ods, dt, stored="f32")
 
 
@@ -83,11 +88,16 @@ def test_outer_gating(cuda_lib, kw, phi):
     oo, ol = O.attn_fwd_outer(x.q, x.k, x.v, ix, og, cfg.b)
     odq, odk, odv, ods = O.attn_bwd_outer(x.q, x.k, x.v, x.dO, ix, x.scores, cfg.b, phi)
     dt = cfg.dtype
-    check("o (outer)", host(o), oo, dt)
+    fl = [None] * 4
+    if dt == "bf16":
+        oe, _ = O.attn_fwd_outer(x.q, x.k, x.v, ix, og, cfg.b, operands="bf16")
+        e = O.attn_bwd_outer(x.q, x.k, x.v, x.dO, ix, x.scores, cfg.b, phi, operands="bf16")
+        fl = [floor_of(oo, oe), floor_of(odq, e[0]), floor_of(odk, e[1]), floor_of(odv, e[2])]
+    check("o (outer)", host(o), oo, dt, floor=fl[0])
     check("lse (outer)", host(lse), ol, dt, stored="f32")
-    check("dq (outer)", host(dq), odq, dt)
-    check("dk (outer)", host(dk), odk, dt)
-    check("dv (outer)", host(dv), odv, dt)
+    check("dq (outer)", host(dq), odq, dt, floor=fl[1])
+    check("dk (outer)", host(dk), odk, dt, floor=fl[2])
+    check("dv (outer)", host(dv), odv, dt, floor=fl[3])
     check(f"dscores (outer, {phi})", host(ds), ods, dt, stored="f32")
 
 

@@ -400,3 +400,16 @@ def test_attended_pairs_brute_force():
         assert O.attended_pairs(1, 1, T, b, K) == cnt
     # the two bf16 training layers
     assert O.attended_pairs(1, 32, 16384, 64, 16) * 4 * 128 == pytest.approx(0.2745e12, rel=1e-3)
+
+
+def test_round_bf16_matches_torch_conversion():
+    """The bf16 rounding the oracle uses to measure operand-rounding floors is
+    torch's float32 -> bfloat16 conversion (nearest, ties to even)."""
+    import torch
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.integers(-8, 8, 20000),
+                        [0.0, -0.0, 1.0, 1.00390625, 1.01171875, 3.0e38, -3.0e38, 1e-40]])
+    # exact ties between two bf16 neighbours: both directions of ties-to-even
+    x = np.concatenate([x, 1.0 + (2 * np.arange(64) + 1) * 2.0 ** -9])
+    want = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).float().double().numpy()
+    np.testing.assert_array_equal(O.round_bf16(x), want)
