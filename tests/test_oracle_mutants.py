@@ -91,8 +91,8 @@ def _sigmoid_log_gate_sign(s_row, n, phi):
     return ORIG_V["log_gates_row_phi"](s_row, n, phi)
 
 
-def _outer_da_without_gate(q, k, v, dO, idx, gates, bi, kvh, j, b, scale=0.0):
-    r = ORIG_V["attn_bwd_outer_block"](q, k, v, dO, idx, gates, bi, kvh, j, b, scale)
+def _outer_da_without_gate(q, k, v, dO, idx, gates, bi, kvh, j, b, scale=0.0, operands=None):
+    r = ORIG_V["attn_bwd_outer_block"](q, k, v, dO, idx, gates, bi, kvh, j, b, scale, operands)
     r["da"] = {m: a / float(gates[bi, kvh, j, m]) for m, a in r["da"].items()}
     return r
 
