@@ -55,6 +55,10 @@ SIGNATURES = {
     "sas_decode_paged_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "sas_decode_paged": (_i, [_i, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i,
                               _i, _i, _i, _f, _p, _p, _sz, _p]),
+    "sas_selector_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "sas_selector_scores": (_i, [_i, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _p, _sz, _p]),
+    "sas_block_summaries": (_i, [_i, _p, _i, _i, _i, _i, _i, _i, _p, _p]),
+    "sas_selector_scores_decode": (_i, [_i, _p, _p, _i, _i, _i, _i, _i, _f, _p, _p]),
     "sas_dense_fwd": (_i, [_i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p]),
     "sas_dense_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "sas_dense_bwd": (_i, [_i, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p,
@@ -272,6 +276,48 @@ def decode_paged(q, kpages, vpages, page_indptr, page_indices, seq_lens, idx, ga
                                 int(use_gates), B, Hq, Hkv, num_pages, P, max_len, d, b, K, scale,
                                 _ptr(o), _ptr(ws), ws.numel(), _stream(q.device)))
     return o
+
+
+def selector_scores(q, k, b: int, scale: float = 0.0):
+    """Pooled-summary selector scores [B,Hkv,N,N] fp32 of q [B,Hq,T,d], k [B,Hkv,T,d]."""
+    _need(q, "q")
+    _need(k, "k", q.dtype)
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    N = (T + b - 1) // b
+    s = torch.empty((B, Hkv, N, N), dtype=torch.float32, device=q.device)
+    nbytes = LIB.sas_selector_workspace_size(B, Hkv, T, d, b)
+    ws = _workspace("selector", nbytes, q.device, zero=False)
+    _check("sas_selector_scores",
+           LIB.sas_selector_scores(_dtype(q), _ptr(q), _ptr(k), B, Hq, Hkv, T, d, b, scale,
+                                   _ptr(s), _ptr(ws), ws.numel(), _stream(q.device)))
+    return s
+
+
+def block_summaries(kcache, b: int, L: int | None = None):
+    """Mean key of each full history block of a cache [B,Hkv,Lcap,d] -> [B,Hkv,C,d] fp32."""
+    _need(kcache, "kcache")
+    B, Hkv, Lcap, d = kcache.shape
+    L = Lcap if L is None else L
+    C = (L - 1) // b
+    kbar = torch.empty((B, Hkv, C, d), dtype=torch.float32, device=kcache.device)
+    _check("sas_block_summaries",
+           LIB.sas_block_summaries(_dtype(kcache), _ptr(kcache), B, Hkv, L, Lcap, d, b,
+                                   _ptr(kbar), _stream(kcache.device)))
+    return kbar
+
+
+def selector_scores_decode(q, kbar, scale: float = 0.0):
+    """Decode selector scores [B,Hkv,C] of q [B,Hq,d] against kbar [B,Hkv,C,d]."""
+    _need(q, "q")
+    _need(kbar, "kbar", torch.float32)
+    B, Hq, d = q.shape
+    Hkv, C = kbar.shape[1], kbar.shape[2]
+    s = torch.empty((B, Hkv, C), dtype=torch.float32, device=q.device)
+    _check("sas_selector_scores_decode",
+           LIB.sas_selector_scores_decode(_dtype(q), _ptr(q), _ptr(kbar), B, Hq, Hkv, C, d,
+                                          scale, _ptr(s), _stream(q.device)))
+    return s
 
 
 def dense_fwd(q, k, v, b: int = 64, scale: float = 0.0):

@@ -407,6 +407,64 @@ sas_status_t sas_decode_paged(sas_dtype_t dtype, const void* q, const void* kpag
       launch_decode_paged_tc(s, pa, q, kpages, vpages, idx, gates, o, ws, ctx, stream));
 }
 
+size_t sas_selector_workspace_size(int B, int Hkv, int T, int d, int b) {
+  if (B < 0 || Hkv < 1 || T < 1 || (d != 64 && d != 128) || b < 1) return 0;
+  const size_t N = ((size_t)T + b - 1) / b;
+  return 2 * ((sizeof(float) * (size_t)B * Hkv * N * d + 255) & ~(size_t)255);
+}
+
+sas_status_t sas_selector_scores(sas_dtype_t dtype, const void* q, const void* k, int B, int Hq,
+                                 int Hkv, int T, int d, int b, float scale, float* scores,
+                                 void* ws, size_t ws_bytes, sas_stream_t stream) {
+  sas_status_t st = check_attn(dtype, B, Hq, Hkv, T, d, b, 1, false, scale);
+  if (st != SAS_OK) return st;
+  if (B == 0) return SAS_OK;
+  if (!q || !k || !scores) return SAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(scores, 4)) return SAS_ERR_INVALID_ARG;
+  if ((long long)B * Hkv > 65535) return SAS_ERR_UNSUPPORTED;  // grid dimension
+  const size_t need = sas_selector_workspace_size(B, Hkv, T, d, b);
+  if (!ws || ws_bytes < need || !aligned(ws, 256)) return SAS_ERR_WORKSPACE;
+  const int N = (T + b - 1) / b;
+  float* qbar = static_cast<float*>(ws);
+  float* kbar = reinterpret_cast<float*>(static_cast<char*>(ws) + need / 2);
+  const int G = Hq / Hkv;
+  cudaError_t e = launch_block_summaries(dtype, q, B * Hkv, G, T, T, b, N, d, qbar, stream);
+  if (e == cudaSuccess)
+    e = launch_block_summaries(dtype, k, B * Hkv, 1, T, T, b, N, d, kbar, stream);
+  if (e == cudaSuccess)
+    e = launch_selector_scores(qbar, kbar, B * Hkv, N, d, resolve_scale(scale, d), scores,
+                               stream);
+  return cuda_status(e);
+}
+
+sas_status_t sas_block_summaries(sas_dtype_t dtype, const void* kcache, int B, int Hkv, int L,
+                                 int Lcap, int d, int b, float* kbar, sas_stream_t stream) {
+  sas_status_t st = check_decode(dtype, B, Hkv, Hkv, L, Lcap, d, b, 1, false, 1.f);
+  if (st != SAS_OK) return st;
+  const int C = (L - 1) / b;
+  if (B == 0 || C == 0) return SAS_OK;
+  if (!kcache || !kbar) return SAS_ERR_INVALID_ARG;
+  if (!aligned(kcache, 16) || !aligned(kbar, 4)) return SAS_ERR_INVALID_ARG;
+  if ((long long)B * Hkv > 65535) return SAS_ERR_UNSUPPORTED;  // grid dimension
+  return cuda_status(
+      launch_block_summaries(dtype, kcache, B * Hkv, 1, C * b, Lcap, b, C, d, kbar, stream));
+}
+
+sas_status_t sas_selector_scores_decode(sas_dtype_t dtype, const void* q, const float* kbar, int B,
+                                        int Hq, int Hkv, int C, int d, float scale, float* scores,
+                                        sas_stream_t stream) {
+  if (!valid_dtype(dtype)) return SAS_ERR_INVALID_ARG;
+  if (B < 0 || Hq < 1 || Hkv < 1 || C < 0 || Hq % Hkv != 0 || !isfinite(scale))
+    return SAS_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SAS_ERR_UNSUPPORTED;
+  if (B > 65535 || (long long)B * Hkv > 65535) return SAS_ERR_UNSUPPORTED;
+  if (B == 0 || C == 0) return SAS_OK;
+  if (!q || !kbar || !scores) return SAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(kbar, 4) || !aligned(scores, 4)) return SAS_ERR_INVALID_ARG;
+  return cuda_status(launch_selector_scores_decode(dtype, q, kbar, B * Hkv, Hq / Hkv, C, d,
+                                                   resolve_scale(scale, d), scores, stream));
+}
+
 sas_status_t sas_dense_fwd(sas_dtype_t dtype, const void* q, const void* k, const void* v, int B,
                            int Hq, int Hkv, int T, int d, int b, float scale, void* o, float* lse,
                            sas_stream_t stream) {

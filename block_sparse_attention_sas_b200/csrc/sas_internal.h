@@ -122,4 +122,16 @@ cudaError_t decode_noalloc_scratch(void** out);
 
 cudaError_t launch_wait_selftest(const DevCtx& ctx, cudaStream_t stream);
 
+// Block-selector scores (selector.cu). Summaries: mean over each block's rows
+// of `group` consecutive planes ([planes_out * group][pitch rows][d], the
+// first `rows` valid) into out [planes_out][N][d] fp32.
+cudaError_t launch_block_summaries(sas_dtype_t dt, const void* x, int planes_out, int group,
+                                   int rows, int pitch, int b, int N, int d, float* out,
+                                   cudaStream_t st);
+cudaError_t launch_selector_scores(const float* qbar, const float* kbar, int units, int N, int d,
+                                   float scale, float* scores, cudaStream_t st);
+cudaError_t launch_selector_scores_decode(sas_dtype_t dt, const void* q, const float* kbar,
+                                          int units, int G, int C, int d, float scale,
+                                          float* scores, cudaStream_t st);
+
 }  // namespace sas

@@ -307,6 +307,36 @@ sas_status_t sas_decode_paged(sas_dtype_t dtype, const void* q, const void* kpag
                               sas_stream_t stream);
 
 /*
+ * Block-selector scores from pooled block summaries. [review] Frequently
+ * asked questions: the selector (the AttnGate architecture) works from
+ * pooling-based block summaries and scores history blocks per query block and
+ * KV-head group; the pages give neither its layers nor its weights. These
+ * calls compute the weight-free reading: a block's key summary is the mean of
+ * its keys (a partial last block: of its valid rows), a query block's
+ * summary the mean of its rows over the G heads of the group, and
+ *   scores[b, kvh, j, m] = scale * qbar_j . kbar_m  for m < j, 0 for m >= j
+ * (the mean of the attention logits over every row/head/key pair of the two
+ * blocks), fp32, ready for sas_gate_topk. scale <= 0 selects 1/sqrt(d).
+ *   sas_selector_scores: q [B, Hq, T, d], k [B, Hkv, T, d] (dtype) ->
+ *     scores [B, Hkv, N, N]; workspace sas_selector_workspace_size() bytes
+ *     (256-byte aligned; contents on entry do not matter).
+ *   sas_block_summaries: the key summaries of the C = floor((L-1)/b) full
+ *     history blocks of a cache [B, Hkv, Lcap, d] -> kbar [B, Hkv, C, d] fp32
+ *     (a server keeps these and adds one whenever a block fills).
+ *   sas_selector_scores_decode: q [B, Hq, d] (the token at L-1), kbar as
+ *     above -> scores [B, Hkv, C]: qbar is the mean of the group's G heads.
+ */
+size_t sas_selector_workspace_size(int B, int Hkv, int T, int d, int b);
+sas_status_t sas_selector_scores(sas_dtype_t dtype, const void* q, const void* k, int B, int Hq,
+                                 int Hkv, int T, int d, int b, float scale, float* scores,
+                                 void* ws, size_t ws_bytes, sas_stream_t stream);
+sas_status_t sas_block_summaries(sas_dtype_t dtype, const void* kcache, int B, int Hkv, int L,
+                                 int Lcap, int d, int b, float* kbar, sas_stream_t stream);
+sas_status_t sas_selector_scores_decode(sas_dtype_t dtype, const void* q, const float* kbar, int B,
+                                        int Hq, int Hkv, int C, int d, float scale, float* scores,
+                                        sas_stream_t stream);
+
+/*
  * Dense comparison kernels ([picx] Eq. 1 with a causal mask): every block is
  * attended, no gates. Same layouts and conventions as the sparse calls; the
  * block size b only sets the kernels' tiling (use 64 unless d or T call for

@@ -709,6 +709,62 @@ def dense_decode(q, kcache, vcache, scale=0.0):
 
 
 # ---------------------------------------------------------------------------
+# Block-selector scores from pooled block summaries
+# ---------------------------------------------------------------------------
+# The evolve.pub review (Frequently asked questions) says the selector (the
+# AttnGate architecture it shares with SeerAttention-R) works from
+# "pooling-based block summaries" and scores history blocks per query block
+# and KV-head group; no page gives its layers or weights. Reading (weight-free,
+# the plainest one the pages support): a block's key summary is the mean of
+# its keys, a query block's summary the mean of its query rows over the G
+# heads of the group, and the score is their scaled dot product,
+#   s[j, m] = scale * qbar_j . kbar_m   for history blocks m < j (0 otherwise),
+# with scale = 1/sqrt(d) as in the attention logits. At decode the query
+# summary is the mean of the G heads' single query token.
+
+def block_summaries(x, b):
+    """Mean over each block's rows (the last block may be partial):
+    x [..., T, d] -> [..., N, d] float64."""
+    x = _f64(x)
+    T = x.shape[-2]
+    N = (T + b - 1) // b
+    out = np.empty(x.shape[:-2] + (N, x.shape[-1]))
+    for m in range(N):
+        out[..., m, :] = x[..., m * b:min(T, (m + 1) * b), :].mean(axis=-2)
+    return out
+
+
+def selector_scores(q, k, b, scale=0.0):
+    """Training scores [B, Hkv, N, N] (row j meaningful for m < j, 0 elsewhere)."""
+    q, k = _f64(q), _f64(k)
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    scale = _default_scale(d, scale)
+    qbar = block_summaries(q.reshape(B, Hkv, G, T, d), b).mean(axis=2)  # [B, Hkv, N, d]
+    kbar = block_summaries(k, b)                                          # [B, Hkv, N, d]
+    N = kbar.shape[2]
+    s = np.zeros((B, Hkv, N, N))
+    for j in range(N):
+        s[:, :, j, :j] = scale * np.einsum("bhd,bhmd->bhm", qbar[:, :, j], kbar[:, :, :j])
+    return s
+
+
+def selector_scores_decode(q, kcache, L, b, scale=0.0):
+    """Decode scores [B, Hkv, C] over the C = floor((L-1)/b) history blocks of
+    a cache holding L tokens; q [B, Hq, d] is the token at L-1."""
+    q, kc = _f64(q), _f64(kcache)
+    B, Hq, d = q.shape
+    Hkv = kc.shape[1]
+    G = Hq // Hkv
+    scale = _default_scale(d, scale)
+    C = (L - 1) // b
+    qbar = q.reshape(B, Hkv, G, d).mean(axis=2)
+    kbar = block_summaries(kc[:, :, :C * b], b) if C else np.zeros((B, Hkv, 0, d))
+    return scale * np.einsum("bhd,bhmd->bhm", qbar, kbar)
+
+
+# ---------------------------------------------------------------------------
 # Algorithmic work counts (for throughput figures, not for any result)
 # ---------------------------------------------------------------------------
 

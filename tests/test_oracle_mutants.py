@@ -15,6 +15,7 @@ from oracle import sas_oracle as O
 from tests import test_oracle as P
 from tests import test_oracle_variants as V
 from tests import test_oracle_paged as PG
+from tests import test_oracle_selector as SEL
 
 
 def _no_scale(d, scale):
@@ -104,6 +105,14 @@ def _current_block_gated(j, b, T, sel_row, gates_row):
     return w
 
 
+ORIG_S = O.block_summaries
+
+
+def _summaries_summed(x, b):
+    """Block summaries as sums instead of means."""
+    return ORIG_S(x, b) * b
+
+
 def _pin(fn, *args):
     def run():
         fn(*args)
@@ -137,6 +146,9 @@ MUTANTS = {
     "outer gate on the current block": ("_col_gates", _current_block_gated,
                                         [V.test_outer_with_unit_gates_is_ungated_sparse_attention,
                                          V.test_outer_backward_matches_autograd]),
+    "selector: summed instead of mean-pooled": ("block_summaries", _summaries_summed,
+                                                [SEL.test_scores_equal_mean_of_pair_logits,
+                                                 SEL.test_constant_and_partial_blocks]),
     "paged: pages in reverse order": ("decode_paged", _paged_pages_reversed,
                                       [PG.test_uniform_lengths_equal_contiguous_decode,
                                        PG.test_full_selection_is_attention_of_the_last_token]),
