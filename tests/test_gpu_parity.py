@@ -19,6 +19,18 @@ pytestmark = pytest.mark.gpu
 
 # --------------------------------------------------------------------- gates
 
+@pytest.mark.parametrize("C,K", [(1023, 32), (8191, 64), (3000, 64)])
+def test_gate_topk_skewed_rows(cuda_lib, C, K):
+    """Rows whose largest scores all sit in the entries one lane of a warp
+    reads (indices = 0 mod 32): the lanes' own two largest then say little
+    about the row, so far more than 256 entries pass the first threshold and
+    the warp falls back to sorting its whole chunk."""
+    rng = np.random.default_rng(C)
+    s = (rng.standard_normal((1, 2, 3, C)) * 0.1).astype(np.float32)
+    s[..., ::32] += 5.0 + rng.standard_normal(s[..., ::32].shape).astype(np.float32)
+    _gate_case(cuda_lib, s, K, False)
+
+
 def _gate_case(lib, scores, K, causal):
     g, ix = lib.gate_topk(dev(scores, "f32"), K, causal=causal)
     og, _, oi = O.gate_topk(scores, K, causal=causal)
@@ -46,6 +58,9 @@ def test_gate_topk_decode_configs(cuda_lib, name):
     # fallback), chunked rows with heavy ties, chunked causal rows, many chunks
     (2049, 8, False, 0), (2048, 256, False, 0), (9000, 256, False, 2), (2100, 16, True, 0),
     (20000, 64, False, 0),
+    # decode-sized rows (warp-threshold path): 1, 2, 4 and 8 warps per row, ties
+    (1023, 32, False, 0), (8191, 64, False, 0), (4096, 64, False, 1), (1800, 64, True, 0),
+    (600, 1, False, 3), (7000, 33, False, 2),
 ])
 def test_gate_topk_edges(cuda_lib, C, K, causal, levels):
     rng = np.random.default_rng(C * 7 + K)
