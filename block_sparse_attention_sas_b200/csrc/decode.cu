@@ -447,13 +447,17 @@ cudaError_t decode_g(const DecodeShape& s, const void* q, const void* kc, const 
 }  // namespace
 
 void decode_plan(DecodeShape& s) {
-  // One wave of CTAs, about one per SM (148): the tensor-core decode keeps
-  // six 32 KB stages in flight per CTA, one CTA per SM. A sparse call keeps
-  // at most 16 splits per (batch, KV head) so that they merge inside one
-  // cluster; the dense comparison may use up to kMaxSplits.
+  // CTAs in one wave (148 SMs, two CTAs each). A sparse call's lists are
+  // short (tens of blocks per (batch, KV head)): about 1.5 CTAs per SM gave
+  // the shortest times there (fewer, longer CTAs pay less prologue and merge
+  // per block; 1 and 2 per SM were slower for the Qwen3-14B 512K or the
+  // Qwen3-4B 64K decode), and at most 16 splits per unit, so that they merge
+  // inside one cluster. The dense comparison streams long lists, two per SM.
+  // One CTA per SM with twice the stages was slower for both: each CTA's
+  // S -> softmax -> PV chain, not the bytes in flight, sets the pace.
   const int nslots = s.dense ? s.C + 1 : s.K + 1;
   const int units = s.B * s.Hkv;
-  const int target = 148;
+  const int target = s.dense ? 2 * 148 : 3 * 148 / 2;
   int splits = target / units;
   splits = max(1, min(splits, min(nslots, s.dense ? kMaxSplits : 16)));
   int bps = (nslots + splits - 1) / splits;

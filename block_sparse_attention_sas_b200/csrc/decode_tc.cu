@@ -13,7 +13,7 @@
 //
 // One CTA per (split, KV head, batch); a split is a run of block slots.
 //   warp 2  list of the split's blocks, TMA producer: Q once, then K and V of
-//           each block into a six-stage ring (32 KB a stage)
+//           each block into a three-stage ring (32 KB a stage)
 //   warp 1  MMA issuer: S(n+1) is issued before PV(n) so the softmax of block
 //           n overlaps the next QK^T
 //   warp 0  softmax, one thread per query row (TMEM lane): masks keys past
@@ -22,7 +22,8 @@
 //           per-row reference max: P = 2^(s * scale + bias - m_ref) stays
 //           below 2^8 and O is rescaled in TMEM only when a row max rises
 //           past that, so the softmax of block n + 1 never waits for PV(n)
-// TMEM: S[2] at columns 0 / 64, O at 128 (256 columns). Cache rows past L lie outside the tensor map and are read as zeros.
+// TMEM: S[2] at columns 0 / 64, O at 128 (256 columns, so two CTAs share an
+// SM: one's softmax chain overlaps the other's). Cache rows past L lie outside the tensor map and are read as zeros.
 // The splits of one (batch, KV head) merge their partial (max, sum, o) by
 // log-sum-exp. Up to 16 splits run as one thread-block cluster: each CTA
 // leaves its partial in its shared memory and, after a cluster barrier, CTA
@@ -59,10 +60,7 @@ constexpr int kMaxSlotsPerSplit = 512;
 constexpr int kMaxClusterSplits = 16;  // largest (non-portable) cluster
 
 // Shared memory (offsets from a 1024-byte aligned base).
-// Six 32 KB K/V stages and one CTA per SM: a sparse decode CTA streams only
-// a few tens of blocks, and under load a stage takes microseconds to land,
-// so the bytes in flight (148 SMs x 192 KB) set its speed.
-constexpr int kStages = 6;
+constexpr int kStages = 3;  // 32 KB K/V stages; two CTAs share an SM
 constexpr uint32_t kOffQ = 0;           // [k half][8 rows][128 B]
 constexpr uint32_t kOffKV = 2048;       // stages x (K halves 16 KB, V halves 16 KB)
 constexpr uint32_t kOffCtl = kOffKV + kStages * 32768;
@@ -99,7 +97,7 @@ static_assert(kOffCtl % 16 == 0 && offsetof(Ctl, part_o) % 16 == 0 && (kD * 4) %
               "the float4 accesses of part_o need 16-byte alignment");
 
 template <int G>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ idx,
                  const float* __restrict__ gates, DecodeShape s, __nv_bfloat16* __restrict__ o,

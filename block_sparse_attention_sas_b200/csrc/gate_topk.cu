@@ -337,35 +337,6 @@ __device__ __forceinline__ void warp_sort_cand(const uint64_t* cand, int m, uint
     if (e * 32 + lane < k) out[e * 32 + lane] = w[e];
 }
 
-// The last stage of a descending bitonic sort: turns a bitonic sequence of
-// 32 * EW keys (lane l holds indices e * 32 + l in w[e]) into a sorted one.
-template <int EW>
-__device__ __forceinline__ void warp_bitonic_merge_desc(uint64_t (&w)[EW]) {
-  const int lane = threadIdx.x & 31;
-  constexpr int n = 32 * EW;
-#pragma unroll
-  for (int j = n >> 1; j > 0; j >>= 1) {
-    if (j >= 32) {
-#pragma unroll
-      for (int e = 0; e < EW; ++e) {
-        const int pe = e ^ (j >> 5);
-        if (pe > e && w[e] < w[pe]) {
-          const uint64_t t = w[e];
-          w[e] = w[pe];
-          w[pe] = t;
-        }
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < EW; ++e) {
-        const uint64_t o = __shfl_xor_sync(0xffffffffu, w[e], j);
-        const bool keep_max = (lane & j) == 0;
-        w[e] = keep_max ? (w[e] > o ? w[e] : o) : (w[e] < o ? w[e] : o);
-      }
-    }
-  }
-}
-
 constexpr int kBins = 4096;     // histogram over the top 12 bits of a key
 constexpr int kCandCap = 256;   // candidates sorted by one warp
 
@@ -567,180 +538,181 @@ gate_topk_merge_kernel(const float* __restrict__ scores, int rows, int C, int ca
 }
 
 // ---------------------------------------------------------------------------
-// Decode rows (up to 8192 entries, K <= 64): warp-threshold selection, one
-// launch, no histogram. W warps share a row, each owning 1024 entries (32 per
-// lane). Each lane keeps its two largest composites; sorting the warp's 64
-// lane-tops gives tau, the k-th largest of them (k = the warp's selection
-// size). Those 64 are entries of the chunk, so at least k composites are
-// >= tau, and only those (usually a few more than k) are compacted with
-// ballots and sorted in registers. Rarely (adversarial rows) more than 256
-// pass; the warp then sorts its whole chunk. The W sorted lists of a row are
-// merged pairwise (a list and the reversed other form a bitonic sequence).
-// Composites are distinct, so the order is exact, ties to the lower index.
+// Decode-sized rows (513 .. 8192 entries): one CTA of 256 threads per row,
+// thread t holding entries [t EPT, (t + 1) EPT). The row's max M and min come
+// from one reduction, the gate softmax's sum from a second. Selection without
+// sorting the row: a 256-bucket histogram of (M - s) in steps of 1/32 finds
+// the bucket b* holding the k-th largest score (when that lies more than 8
+// below M, a second histogram spreads the rest of the row's range over 256
+// buckets). Every score in a bucket up to b* is a candidate -- a superset of
+// the top k, usually a few more than k -- and each candidate is placed by its
+// rank among the candidates under the composite order (descending score,
+// ties to the lower index), which is its rank in the row. More than 1024
+// candidates (mass ties) make the block sort the whole row instead.
 // ---------------------------------------------------------------------------
-constexpr int kWtChunk = 1024;  // entries per warp
-constexpr int kWtCand = 256;    // candidates one warp sorts
-constexpr int kWtMaxK = 64;
+constexpr int kBkThreads = 256;
+constexpr int kBkCand = 1024;
+constexpr float kBkStep = 32.f;  // level-1 buckets per unit of score below the max
 
-template <int EW>
-__device__ __forceinline__ void wt_sort_keep(uint64_t* cand, int m, int k) {
-  const int lane = threadIdx.x & 31;
-  uint64_t w[EW];
-#pragma unroll
-  for (int e = 0; e < EW; ++e) w[e] = e * 32 + lane < m ? cand[e * 32 + lane] : 0ull;
-  warp_sort_desc<EW>(w);
-  __syncwarp();
-#pragma unroll
-  for (int e = 0; e < EW; ++e)
-    if (e * 32 + lane < k) cand[e * 32 + lane] = w[e];
-  __syncwarp();
-}
-
-template <int W>
-__global__ void __launch_bounds__(32 * W * (W >= 4 ? 1 : 4 / W))
-gate_topk_wt_kernel(const float* __restrict__ scores, long long total_rows, int rows, int C,
-                    int causal, int K, int phi, float* __restrict__ gates,
-                    int32_t* __restrict__ idx) {
-  constexpr int R = W >= 4 ? 1 : 4 / W;  // rows per CTA
-  __shared__ uint64_t s_cand[W * R][kWtCand];
-  __shared__ float s_red[W * R][2];
-  __shared__ int s_cnt[W * R];
+template <int EPT>
+__global__ void __launch_bounds__(kBkThreads)
+gate_topk_bucket_kernel(const float* __restrict__ scores, int rows, int C, int causal, int K,
+                        int phi, float* __restrict__ gates, int32_t* __restrict__ idx) {
+  extern __shared__ uint64_t s_sort[];  // EPT * 256 keys; used only by the fallback
+  __shared__ int s_hist[256];
+  __shared__ uint64_t s_cand[kBkCand];
+  __shared__ float s_red[3][8];
+  __shared__ int s_m, s_b1, s_b2, s_before;
   grid_launch_dependents();  // a dependent decode may start its prologue
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rl = warp / W, w = warp % W;
-  const long long row = (long long)blockIdx.x * R + rl;
-  const bool row_ok = row < total_rows;
-  const int r = row_ok ? (int)(row % rows) : 0;
-  const int n = row_ok ? (causal ? min(r, C) : C) : 0;
-  const int lo = w * kWtChunk;
-  const int nw = max(0, min(n - lo, kWtChunk));
-  const float* srow = scores + (row_ok ? row : 0) * (long long)C;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long row = blockIdx.x;
+  const int r = (int)(row % rows);
+  const int n = causal ? min(r, C) : C;
+  const float* srow = scores + row * (long long)C;
+  const int i0 = tid * EPT;
 
-  // ---- the chunk, its max and sum of exp (the gate softmax partials)
-  float f[32];
-  float mx = -INFINITY;
+  float f[EPT];
+  float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
-  for (int e = 0; e < 32; ++e) {
-    f[e] = (e * 32 + lane < nw) ? srow[lo + e * 32 + lane] : -INFINITY;
-    mx = fmaxf(mx, f[e]);
+  for (int e = 0; e < EPT; ++e) {
+    const bool ok = i0 + e < n;
+    f[e] = ok ? srow[i0 + e] : -INFINITY;
+    if (ok) {
+      mx = fmaxf(mx, f[e]);
+      mn = fminf(mn, f[e]);
+    }
   }
   mx = warp_max(mx);
+  mn = -warp_max(-mn);
+  if (lane == 0) {
+    s_red[0][warp] = mx;
+    s_red[1][warp] = mn;
+  }
+  __syncthreads();
+  float M = -INFINITY, Mn = INFINITY;
+#pragma unroll
+  for (int x = 0; x < 8; ++x) {
+    M = fmaxf(M, s_red[0][x]);
+    Mn = fminf(Mn, s_red[1][x]);
+  }
   float sum = 0.f;
 #pragma unroll
-  for (int e = 0; e < 32; ++e)
-    if (e * 32 + lane < nw) sum += expf(f[e] - mx);
+  for (int e = 0; e < EPT; ++e)
+    if (i0 + e < n) sum += expf(f[e] - M);
   sum = warp_sum(sum);
-  if (lane == 0) {
-    s_red[warp][0] = mx;
-    s_red[warp][1] = sum;
-  }
-
-  // ---- tau from the lanes' two largest composites
-  const int kk = min(K, nw);
-  uint64_t t0 = 0ull, t1 = 0ull;
-#pragma unroll
-  for (int e = 0; e < 32; ++e) {
-    const uint64_t key = (e * 32 + lane < nw) ? ckey(f[e], lo + e * 32 + lane) : 0ull;
-    if (key > t0) {
-      t1 = t0;
-      t0 = key;
-    } else if (key > t1) {
-      t1 = key;
-    }
-  }
-  uint64_t tau = ~0ull;
-  if (kk > 0) {
-    uint64_t v[2] = {t0, t1};
-    warp_sort_desc<2>(v);
-    const int p = kk - 1;
-    tau = __shfl_sync(0xffffffffu, (p >> 5) ? v[1] : v[0], p & 31);
-  }
-
-  // ---- candidates >= tau, in index order
-  uint64_t* cand = s_cand[warp];
-  int m = 0;
-  const uint32_t lt = (1u << lane) - 1u;
-#pragma unroll
-  for (int e = 0; e < 32; ++e) {
-    const uint64_t key = (e * 32 + lane < nw) ? ckey(f[e], lo + e * 32 + lane) : 0ull;
-    const bool pred = key >= tau;
-    const uint32_t mask = __ballot_sync(0xffffffffu, pred);
-    const int pos = m + __popc(mask & lt);
-    if (pred && pos < kWtCand) cand[pos] = key;
-    m += __popc(mask);
-  }
-  __syncwarp();
-  if (kk > 0) {
-    if (m <= 64) wt_sort_keep<2>(cand, m, kk);
-    else if (m <= 128) wt_sort_keep<4>(cand, m, kk);
-    else if (m <= kWtCand) wt_sort_keep<8>(cand, m, kk);
-    else {
-      // More than 256 passed: sort the whole chunk.
-      uint64_t all[32];
-#pragma unroll
-      for (int e = 0; e < 32; ++e)
-        all[e] = (e * 32 + lane < nw) ? ckey(f[e], lo + e * 32 + lane) : 0ull;
-      warp_sort_desc<32>(all);
-#pragma unroll
-      for (int e = 0; e < 32; ++e)
-        if (e * 32 + lane < kk) cand[e * 32 + lane] = all[e];
-      __syncwarp();
-    }
-  }
-  if (lane == 0) s_cnt[warp] = kk;
+  if (lane == 0) s_red[2][warp] = sum;
+  if (tid < 256) s_hist[tid] = 0;
+  if (tid == 0) s_m = 0;
   __syncthreads();
-
-  // ---- the row's LSE (warp order) and this warp's gates
-  float M = -INFINITY, S = 0.f;
+  float S = 0.f;
 #pragma unroll
-  for (int x = 0; x < W; ++x) M = fmaxf(M, s_red[rl * W + x][0]);
-#pragma unroll
-  for (int x = 0; x < W; ++x) {
-    const float ss = s_red[rl * W + x][1];
-    if (ss > 0.f) S += ss * expf(s_red[rl * W + x][0] - M);
-  }
+  for (int x = 0; x < 8; ++x) S += s_red[2][x];
   const float lse = M + logf(S);
-  if (row_ok) {
-    float* grow = gates + row * (long long)C;
+  float* grow = gates + row * (long long)C;
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const int gi = lo + e * 32 + lane;
-      if (gi < C) grow[gi] = gi < n ? gate_of(f[e], lse, phi) : 0.f;
+  for (int e = 0; e < EPT; ++e) {
+    const int i = i0 + e;
+    if (i < C) grow[i] = i < n ? gate_of(f[e], lse, phi) : 0.f;
+  }
+  const int kk = min(K, n);
+  int32_t* out = idx + row * (long long)K;
+  for (int p = kk + tid; p < K; p += kBkThreads) out[p] = -1;
+  if (kk == 0) return;  // uniform over the CTA
+
+  // ---- level 1: buckets of width 1/32 below the max (bucket 255: the rest)
+  auto b1_of = [&](float x) -> int { return min(255, (int)((M - x) * kBkStep)); };
+#pragma unroll
+  for (int e = 0; e < EPT; ++e)
+    if (i0 + e < n) atomicAdd(&s_hist[b1_of(f[e])], 1);
+  __syncthreads();
+  // Warp 0 finds the first bucket whose running count reaches the target.
+  auto find_bucket = [&](int target, int& bstar, int& before) {
+    int h[8], tot = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      h[i] = s_hist[lane * 8 + i];
+      tot += h[i];
+    }
+    int incl = tot;  // inclusive prefix over lanes
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - tot, b = -1, bef = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (b < 0 && run + h[i] >= target) {
+        b = lane * 8 + i;
+        bef = run;
+      }
+      run += h[i];
+    }
+    const uint32_t hit = __ballot_sync(0xffffffffu, b >= 0);
+    const int src = __ffs(hit) - 1;  // the lowest lane holds the first such bucket
+    bstar = __shfl_sync(0xffffffffu, b, src);
+    before = __shfl_sync(0xffffffffu, bef, src);
+  };
+  if (warp == 0) {
+    int bs, bf;
+    find_bucket(kk, bs, bf);
+    if (lane == 0) {
+      s_b1 = bs;
+      s_before = bf;
+      s_b2 = 255;
     }
   }
-
-  // ---- pairwise merge of the row's sorted lists
+  __syncthreads();
+  const int b1 = s_b1;
+  // ---- level 2 (rare): the k-th largest lies in the overflow bucket; spread
+  // [min, M - 255/32) over 256 buckets, highest first.
+  const float top2 = M - 255.f / kBkStep;
+  const float inv2 = (top2 > Mn) ? 255.f / (top2 - Mn) : 0.f;
+  auto b2_of = [&](float x) -> int { return min(255, max(0, (int)((top2 - x) * inv2))); };
+  if (b1 == 255) {
+    const int need = kk - s_before;
+    if (tid < 256) s_hist[tid] = 0;
+    __syncthreads();
 #pragma unroll
-  for (int step = 1; step < W; step <<= 1) {
-    if ((w % (2 * step)) == 0 && w + step < W) {
-      uint64_t* a = s_cand[warp];
-      const uint64_t* b = s_cand[warp + step];
-      const int na = s_cnt[warp], nb = s_cnt[warp + step];
-      uint64_t v[4];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int i = e * 32 + lane;
-        v[e] = i < na ? a[i] : 0ull;
-        const int jb = 63 - i;  // b reversed into slots 64..127
-        v[e + 2] = jb < nb ? b[jb] : 0ull;
-      }
-      // Slots 0..63: a (descending, zero-padded); slot 64 + i: b[63 - i], so
-      // the 128 slots fall then rise: a bitonic sequence.
-      warp_bitonic_merge_desc<4>(v);
-      const int nk = min(K, na + nb);
-      __syncwarp();
-#pragma unroll
-      for (int e = 0; e < 2; ++e)
-        if (e * 32 + lane < nk) a[e * 32 + lane] = v[e];
-      if (lane == 0) s_cnt[warp] = nk;
+    for (int e = 0; e < EPT; ++e)
+      if (i0 + e < n && b1_of(f[e]) == 255) atomicAdd(&s_hist[b2_of(f[e])], 1);
+    __syncthreads();
+    if (warp == 0) {
+      int bs, bf;
+      find_bucket(need, bs, bf);
+      if (lane == 0) s_b2 = bs;
     }
     __syncthreads();
   }
+  const int b2 = s_b2;
 
-  if (w == 0 && row_ok) {
-    const int kr = min(K, n);
-    int32_t* out = idx + row * (long long)K;
-    for (int p = lane; p < K; p += 32) out[p] = p < kr ? ckey_index(s_cand[warp][p]) : -1;
+  // ---- candidates: every score in a bucket up to the k-th's
+#pragma unroll
+  for (int e = 0; e < EPT; ++e) {
+    if (i0 + e >= n) continue;
+    const int bb = b1_of(f[e]);
+    if (bb < b1 || (bb == b1 && (b1 < 255 || b2_of(f[e]) <= b2))) {
+      const int p = atomicAdd(&s_m, 1);
+      if (p < kBkCand) s_cand[p] = ckey(f[e], i0 + e);
+    }
+  }
+  __syncthreads();
+  const int m = s_m;
+  if (m <= kBkCand) {
+    // rank of each candidate among the candidates = its rank in the row
+    for (int p = tid; p < m; p += kBkThreads) {
+      const uint64_t key = s_cand[p];
+      int rank = 0;
+      for (int q = 0; q < m; ++q) rank += s_cand[q] > key;
+      if (rank < kk) out[rank] = ckey_index(key);
+    }
+  } else {
+    // mass ties: sort the whole row (every thread's keys) in shared memory
+    uint64_t v[EPT];
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) v[e] = (i0 + e < n) ? ckey(f[e], i0 + e) : 0ull;
+    block_sort_desc<EPT>(v, s_sort);
+    for (int p = tid; p < kk; p += kBkThreads) out[p] = ckey_index(s_sort[p]);
   }
 }
 
@@ -933,17 +905,16 @@ cudaError_t launch_gate_topk(const float* scores, int B, int Hkv, int rows, int 
     gate_topk_warp_kernel<<<(unsigned)grid, 32 * kWarpRowsPerCta, 0, stream>>>(
         scores, (int)total, rows, C, causal, K, phi, gates, idx);
     note_launches(1);
-  } else if (K <= kWtMaxK && C <= 8 * kWtChunk) {
-    // Decode-sized rows: warp-threshold selection, W warps per row.
-    const int W = C <= kWtChunk ? 1 : C <= 2 * kWtChunk ? 2 : C <= 4 * kWtChunk ? 4 : 8;
-    const int R = W >= 4 ? 1 : 4 / W;
-    const unsigned grid = (unsigned)((total + R - 1) / R);
-    switch (W) {
-      case 1: gate_topk_wt_kernel<1><<<grid, 32 * W * R, 0, stream>>>(scores, total, rows, C, causal, K, phi, gates, idx); break;
-      case 2: gate_topk_wt_kernel<2><<<grid, 32 * W * R, 0, stream>>>(scores, total, rows, C, causal, K, phi, gates, idx); break;
-      case 4: gate_topk_wt_kernel<4><<<grid, 32 * W * R, 0, stream>>>(scores, total, rows, C, causal, K, phi, gates, idx); break;
-      default: gate_topk_wt_kernel<8><<<grid, 32 * W * R, 0, stream>>>(scores, total, rows, C, causal, K, phi, gates, idx); break;
-    }
+  } else if (C <= 32 * kBkThreads) {
+    // Decode-sized rows: one CTA per row, bucket selection.
+    const int EPT = C <= 4 * kBkThreads ? 4 : C <= 8 * kBkThreads ? 8 : C <= 16 * kBkThreads ? 16 : 32;
+    const size_t smem = (size_t)EPT * kBkThreads * sizeof(uint64_t);  // the fallback's sort
+    auto kern = EPT == 4 ? gate_topk_bucket_kernel<4> : EPT == 8 ? gate_topk_bucket_kernel<8>
+              : EPT == 16 ? gate_topk_bucket_kernel<16> : gate_topk_bucket_kernel<32>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)total, kBkThreads, smem, stream>>>(scores, rows, C, causal, K, phi, gates, idx);
     note_launches(1);
   } else if (launch_cluster_topk(scores, total, rows, C, causal, K, phi, gates, idx, stream)) {
     // one launch: a cluster of chunk CTAs per row

@@ -19,6 +19,15 @@ pytestmark = pytest.mark.gpu
 
 # --------------------------------------------------------------------- gates
 
+@pytest.mark.parametrize("C,K,spread", [(1023, 32, 20.0), (8191, 64, 30.0), (5000, 256, 3.0)])
+def test_gate_topk_wide_rows(cuda_lib, C, K, spread):
+    """Rows whose k-th largest score lies far below the maximum (a wide
+    spread, or a large k): the selection's second histogram level."""
+    rng = np.random.default_rng(C + K)
+    s = (rng.standard_normal((2, 1, 2, C)) * spread).astype(np.float32)
+    _gate_case(cuda_lib, s, K, False)
+
+
 @pytest.mark.parametrize("C,K", [(1023, 32), (8191, 64), (3000, 64)])
 def test_gate_topk_skewed_rows(cuda_lib, C, K):
     """Rows whose largest scores all sit in the entries one lane of a warp
