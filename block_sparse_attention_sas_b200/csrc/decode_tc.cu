@@ -312,10 +312,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
     }
   } else if (warp == kSoftmaxWarp) {
-    // Thread `lane` owns query row `lane` of the tile (head lane < G).
+    // Lane l owns query row l % 8 (the 8-row Q box repeats down the tile, so
+    // lanes l, l + 8, l + 16, l + 24 hold the same S row) and, as lane group
+    // g = l / 8, the 16 columns 16 g .. 16 g + 15 of every block: each group
+    // is a split of its own (running max, sum and O in its TMEM lane; P is
+    // zero outside its columns) and the four are merged at the end. So a lane
+    // forms 16 probabilities per block, not 64.
     constexpr float kLazy = 8.f;  // log2 headroom of P over the reference max
     const float sc = s.scale * kLog2e;
     const uint32_t tl = tmem;  // lanes 0..31
+    const int grp = lane >> 3;
+    const bool row_live = (lane & 7) < G;
     for (int n = 0; n < nblk; ++n) {
       const int st = n & 1;
       if (!warp_wait(ctx, &c.s_full[st], (n >> 1) & 1, abort)) {
@@ -326,31 +333,29 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const int m = c.blocks[n];
       const float bias = c.bias[n];
       const int kvalid = min(kB, c.Lseq - m * kB);
-      // Two passes over the two 32-column halves of S: the row max first,
-      // then p = 2^(s*scale + bias - m_ref) as bf16 into the S columns
-      // already read (P(n) takes columns 0..31).
-      float smax = -INFINITY;
+      // This group's 16 columns of S (the ld is warp-wide; each group keeps its own).
+      float sv[16];
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         uint32_t sr[32];
         tmem_ld32(tl + kColS + st * 64 + hf * 32, sr);
         tmem_ld_wait();
-        float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          const bool v0 = hf * 32 + i < kvalid, v1 = hf * 32 + i + 1 < kvalid;
-          const bool v2 = hf * 32 + i + 2 < kvalid, v3 = hf * 32 + i + 3 < kvalid;
-          m0 = fmax3(m0, v0 ? __uint_as_float(sr[i]) : -INFINITY,
-                     v1 ? __uint_as_float(sr[i + 1]) : -INFINITY);
-          m1 = fmax3(m1, v2 ? __uint_as_float(sr[i + 2]) : -INFINITY,
-                     v3 ? __uint_as_float(sr[i + 3]) : -INFINITY);
+        for (int i = 0; i < 16; ++i) {
+          if (grp == 2 * hf) sv[i] = __uint_as_float(sr[i]);
+          else if (grp == 2 * hf + 1) sv[i] = __uint_as_float(sr[16 + i]);
         }
-        smax = fmax3(smax, m0, m1);
+      }
+      float smax = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if (16 * grp + i >= kvalid) sv[i] = -INFINITY;
+        smax = fmaxf(smax, sv[i]);
       }
       const float mx = (smax == -INFINITY) ? -INFINITY : fmaf(smax, sc, bias);
       // Reference update: the first finite max sets it (nothing accumulated
-      // for the row yet); a max more than kLazy above it rescales O.
-      const bool need = lane < G && m_run != -INFINITY && mx > m_run + kLazy;
+      // for the lane yet); a max more than kLazy above it rescales O.
+      const bool need = row_live && m_run != -INFINITY && mx > m_run + kLazy;
       if (m_run == -INFINITY) m_run = mx;
       if (__any_sync(0xffffffffu, need)) {
         // O must hold every PV issued so far. Seeing S(n) complete already
@@ -381,26 +386,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const float off = (m_run == -INFINITY) ? -INFINITY : bias - m_run;
       const uint64_t sc2 = f2u(sc, sc), off2 = f2u(off, off);
       uint64_t accp = 0;
+      uint32_t pk8[8], pk[32];
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t sr[32], pk[16];
-        tmem_ld32(tl + kColS + st * 64 + hf * 32, sr);
-        tmem_ld_wait();
-        if (kvalid < kB) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (hf * 32 + i >= kvalid) sr[i] = __float_as_uint(-INFINITY);
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const uint64_t a = ffma2(f2u(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
-                                   sc2, off2);
-          const float p0 = ex2(lo_f(a)), p1 = ex2(hi_f(a));
-          accp = fadd2(accp, f2u(p0, p1));
-          pk[i] = pack_bf16(p0, p1);
-        }
-        tmem_st16(tl + kColS + st * 64 + hf * 16, pk);
+      for (int i = 0; i < 8; ++i) {
+        const uint64_t a = ffma2(f2u(sv[2 * i], sv[2 * i + 1]), sc2, off2);
+        const float p0 = ex2(lo_f(a)), p1 = ex2(hi_f(a));
+        accp = fadd2(accp, f2u(p0, p1));
+        pk8[i] = pack_bf16(p0, p1);
       }
+      // P(n) into the S columns already read: word w holds columns 2w, 2w + 1,
+      // so this group's words are 8 g .. 8 g + 7 and the rest are zero.
+#pragma unroll
+      for (int w = 0; w < 32; ++w) pk[w] = ((w >> 3) == grp) ? pk8[w & 7] : 0u;
+      tmem_st32(tl + kColS + st * 64, pk);
       l_run += lo_f(accp) + hi_f(accp);
       if (s.paged && kvalid < kB) {
         // Rows past the sequence in a page hold other tokens or stale data:
@@ -437,6 +435,25 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           for (int i = 0; i < 32; ++i) acc[ch * 32 + i] = __uint_as_float(ov[i]);
         }
       }
+    }
+    // Merge the four column groups of each row (lanes l, l ^ 8, l ^ 16,
+    // l ^ 24) by log-sum-exp; every lane of the row ends with the result.
+    {
+      float Mr = fmaxf(m_run, __shfl_xor_sync(0xffffffffu, m_run, 8));
+      Mr = fmaxf(Mr, __shfl_xor_sync(0xffffffffu, Mr, 16));
+      const float wgt = (m_run == -INFINITY) ? 0.f : ex2(m_run - Mr);
+      float lt = wgt * l_run;
+      lt += __shfl_xor_sync(0xffffffffu, lt, 8);
+      lt += __shfl_xor_sync(0xffffffffu, lt, 16);
+#pragma unroll
+      for (int i = 0; i < kD; ++i) {
+        float a = wgt * acc[i];
+        a += __shfl_xor_sync(0xffffffffu, a, 8);
+        a += __shfl_xor_sync(0xffffffffu, a, 16);
+        acc[i] = a;
+      }
+      m_run = Mr;
+      l_run = lt;
     }
   }
   fence_before_sync();
