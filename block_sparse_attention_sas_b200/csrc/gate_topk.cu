@@ -539,12 +539,14 @@ gate_topk_merge_kernel(const float* __restrict__ scores, int rows, int C, int ca
 
 // ---------------------------------------------------------------------------
 // Decode-sized rows (513 .. 8192 entries): one CTA of 256 threads per row,
-// thread t holding entries [t EPT, (t + 1) EPT). The row's max M and min come
+// thread t holding entries t + 256 e (coalesced loads). The row's max M and min come
 // from one reduction, the gate softmax's sum from a second. Selection without
 // sorting the row: a 256-bucket histogram of (M - s) in steps of 1/32 finds
 // the bucket b* holding the k-th largest score (when that lies more than 8
 // below M, a second histogram spreads the rest of the row's range over 256
-// buckets). Every score in a bucket up to b* is a candidate -- a superset of
+// buckets). Histogram adds are combined per warp and bucket, and the
+// overflow bucket is never counted (its count is the rest of the row). Every
+// score in a bucket up to b* is a candidate -- a superset of
 // the top k, usually a few more than k -- and each candidate is placed by its
 // rank among the candidates under the composite order (descending score,
 // ties to the lower index), which is its rank in the row. More than 1024
@@ -569,14 +571,15 @@ gate_topk_bucket_kernel(const float* __restrict__ scores, int rows, int C, int c
   const int r = (int)(row % rows);
   const int n = causal ? min(r, C) : C;
   const float* srow = scores + row * (long long)C;
-  const int i0 = tid * EPT;
+  // entry of slot e: tid + 256 e
+  auto ix = [&](int e) -> int { return tid + kBkThreads * e; };
 
   float f[EPT];
   float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
   for (int e = 0; e < EPT; ++e) {
-    const bool ok = i0 + e < n;
-    f[e] = ok ? srow[i0 + e] : -INFINITY;
+    const bool ok = ix(e) < n;
+    f[e] = ok ? srow[ix(e)] : -INFINITY;
     if (ok) {
       mx = fmaxf(mx, f[e]);
       mn = fminf(mn, f[e]);
@@ -598,7 +601,7 @@ gate_topk_bucket_kernel(const float* __restrict__ scores, int rows, int C, int c
   float sum = 0.f;
 #pragma unroll
   for (int e = 0; e < EPT; ++e)
-    if (i0 + e < n) sum += expf(f[e] - M);
+    if (ix(e) < n) sum += expf(f[e] - M);
   sum = warp_sum(sum);
   if (lane == 0) s_red[2][warp] = sum;
   if (tid < 256) s_hist[tid] = 0;
@@ -611,7 +614,7 @@ gate_topk_bucket_kernel(const float* __restrict__ scores, int rows, int C, int c
   float* grow = gates + row * (long long)C;
 #pragma unroll
   for (int e = 0; e < EPT; ++e) {
-    const int i = i0 + e;
+    const int i = ix(e);
     if (i < C) grow[i] = i < n ? gate_of(f[e], lse, phi) : 0.f;
   }
   const int kk = min(K, n);
@@ -622,8 +625,11 @@ gate_topk_bucket_kernel(const float* __restrict__ scores, int rows, int C, int c
   // ---- level 1: buckets of width 1/32 below the max (bucket 255: the rest)
   auto b1_of = [&](float x) -> int { return min(255, (int)((M - x) * kBkStep)); };
 #pragma unroll
-  for (int e = 0; e < EPT; ++e)
-    if (i0 + e < n) atomicAdd(&s_hist[b1_of(f[e])], 1);
+  for (int e = 0; e < EPT; ++e) {
+    const int bb = ix(e) < n ? b1_of(f[e]) : 255;
+    warp_hist_add(s_hist, (uint32_t)bb, bb < 255);
+  }
+  if (tid == 0) s_hist[255] = 0;  // never counted: the rest of the row
   __syncthreads();
   // Warp 0 finds the first bucket whose running count reaches the target.
   auto find_bucket = [&](int target, int& bstar, int& before) {
@@ -654,6 +660,14 @@ gate_topk_bucket_kernel(const float* __restrict__ scores, int rows, int C, int c
     before = __shfl_sync(0xffffffffu, bef, src);
   };
   if (warp == 0) {
+    // bucket 255 holds whatever the first 255 buckets do not
+    int cnt = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) cnt += (lane * 8 + i < 255) ? s_hist[lane * 8 + i] : 0;
+    cnt = warp_sum(cnt);
+    __syncwarp();
+    if (lane == 31) s_hist[255] = n - cnt;
+    __syncwarp();
     int bs, bf;
     find_bucket(kk, bs, bf);
     if (lane == 0) {
@@ -674,8 +688,10 @@ gate_topk_bucket_kernel(const float* __restrict__ scores, int rows, int C, int c
     if (tid < 256) s_hist[tid] = 0;
     __syncthreads();
 #pragma unroll
-    for (int e = 0; e < EPT; ++e)
-      if (i0 + e < n && b1_of(f[e]) == 255) atomicAdd(&s_hist[b2_of(f[e])], 1);
+    for (int e = 0; e < EPT; ++e) {
+      const bool in = ix(e) < n && b1_of(f[e]) == 255;
+      warp_hist_add(s_hist, in ? (uint32_t)b2_of(f[e]) : 0u, in);
+    }
     __syncthreads();
     if (warp == 0) {
       int bs, bf;
@@ -689,12 +705,15 @@ gate_topk_bucket_kernel(const float* __restrict__ scores, int rows, int C, int c
   // ---- candidates: every score in a bucket up to the k-th's
 #pragma unroll
   for (int e = 0; e < EPT; ++e) {
-    if (i0 + e >= n) continue;
-    const int bb = b1_of(f[e]);
-    if (bb < b1 || (bb == b1 && (b1 < 255 || b2_of(f[e]) <= b2))) {
-      const int p = atomicAdd(&s_m, 1);
-      if (p < kBkCand) s_cand[p] = ckey(f[e], i0 + e);
-    }
+    const int bb = ix(e) < n ? b1_of(f[e]) : 256;
+    const bool take = bb < b1 || (bb == b1 && (b1 < 255 || b2_of(f[e]) <= b2));
+    // one atomic per warp: lanes place themselves after the warp's base
+    const uint32_t mask = __ballot_sync(0xffffffffu, take);
+    int basep = 0;
+    if (lane == 0 && mask) basep = atomicAdd(&s_m, __popc(mask));
+    basep = __shfl_sync(0xffffffffu, basep, 0);
+    const int p = basep + __popc(mask & ((1u << lane) - 1u));
+    if (take && p < kBkCand) s_cand[p] = ckey(f[e], ix(e));
   }
   __syncthreads();
   const int m = s_m;
@@ -710,7 +729,7 @@ gate_topk_bucket_kernel(const float* __restrict__ scores, int rows, int C, int c
     // mass ties: sort the whole row (every thread's keys) in shared memory
     uint64_t v[EPT];
 #pragma unroll
-    for (int e = 0; e < EPT; ++e) v[e] = (i0 + e < n) ? ckey(f[e], i0 + e) : 0ull;
+    for (int e = 0; e < EPT; ++e) v[e] = (ix(e) < n) ? ckey(f[e], ix(e)) : 0ull;
     block_sort_desc<EPT>(v, s_sort);
     for (int p = tid; p < kk; p += kBkThreads) out[p] = ckey_index(s_sort[p]);
   }
