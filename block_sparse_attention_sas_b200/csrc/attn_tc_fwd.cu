@@ -41,25 +41,53 @@ using namespace tc;
 
 constexpr int kD = 128;          // head dim
 constexpr int kB = 64;           // block size (keys per K/V block, rows per head)
-constexpr int kThreads = 384;    // 12 warps
-constexpr int kFirstSoftmaxWarp = 4;
-constexpr int kStages = 3;        // K ring and V ring depth
-constexpr uint32_t kTmemCols = 512;
-
-// Shared-memory carve-up (offsets from a 1024-byte aligned base).
-constexpr uint32_t kQBytes = 2 * 2 * 128 * 128;     // [tile][k half][128 rows][128 B]
 constexpr uint32_t kKVBytes = 2 * 64 * 128;         // one K or V block: [d half][64 rows][128 B]
-constexpr uint32_t kPBytes = 2 * 128 * 128;         // [tile][128 rows][128 B]
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kQBytes;
-constexpr uint32_t kOffV = kOffK + kStages * kKVBytes;
-constexpr uint32_t kOffP = kOffV + kStages * kKVBytes;
-constexpr uint32_t kOffCtl = kOffP + kPBytes;       // barriers and the block list
 constexpr int kMaxList = 257;                        // K <= 256 selected + current
 
+// Resources per CTA for TILES 128-row query tiles (the G heads of a KV head
+// are split into G/2 tiles of two heads).
+//   TILES = 2: 384 threads, 3-stage K and V rings, 512 TMEM columns (Q[t] at
+//              64 t, S[t] at 128 + 64 t, O[t] at 256 + 128 t): one CTA per SM,
+//              both tiles share every K/V block.
+//   TILES = 1: 224 threads, 2-stage rings, 256 TMEM columns (Q 0, S 64,
+//              O 128) and P in the Q staging area (free once Q is in TMEM):
+//              about 99 KB, two CTAs per SM, so one CTA's prologue, softmax
+//              and epilogue overlap the other's MMAs.
+template <int TILES> struct FwdLayout;
+template <> struct FwdLayout<2> {
+  static constexpr int kThreads = 384, kStages = 3, kMaxRegs = 168;
+  // warp roles: K producer, MMA issuer, V producer, first softmax warp
+  static constexpr int kWarpK = 0, kWarpMMA = 1, kWarpV = 2, kSoftFirst = 4;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kOffQ = 0;                       // [tile][k half][128 rows][128 B]
+  static constexpr uint32_t kOffK = kOffQ + 2 * 2 * 128 * 128;
+  static constexpr uint32_t kOffV = kOffK + kStages * kKVBytes;
+  static constexpr uint32_t kOffP = kOffV + kStages * kKVBytes;  // [tile][128 rows][128 B]
+  static constexpr uint32_t kOffCtl = kOffP + 2 * 128 * 128;
+  __device__ static uint32_t q_col(int t) { return t * 64; }
+  __device__ static uint32_t s_col(int t) { return 128 + t * 64; }
+  __device__ static uint32_t o_col(int t) { return 256 + t * 128; }
+};
+template <> struct FwdLayout<1> {
+  // The softmax warps come first (TMEM lane quarter = warp % 4): 7 warps,
+  // so two CTAs per SM leave each thread about 146 registers.
+  static constexpr int kThreads = 224, kStages = 2, kMaxRegs = 144;  // 2 x 7 warps x 144 <= 64K
+  static constexpr int kWarpK = 4, kWarpMMA = 5, kWarpV = 6, kSoftFirst = 0;
+  static constexpr uint32_t kTmemCols = 256;
+  static constexpr uint32_t kOffQ = 0;                       // [k half][128 rows][128 B]
+  static constexpr uint32_t kOffP = 0;                       // P reuses Q's first half
+  static constexpr uint32_t kOffK = 2 * 128 * 128;
+  static constexpr uint32_t kOffV = kOffK + kStages * kKVBytes;
+  static constexpr uint32_t kOffCtl = kOffV + kStages * kKVBytes;
+  __device__ static uint32_t q_col(int) { return 0; }
+  __device__ static uint32_t s_col(int) { return 64; }
+  __device__ static uint32_t o_col(int) { return 128; }
+};
+
+template <int ST>
 struct Ctl {
   uint64_t q_full;
-  uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
+  uint64_t k_full[ST], k_empty[ST], v_full[ST], v_empty[ST];
   // One barrier for both tiles where they move in step (fewer waits and
   // commits on the MMA thread, whose overhead sits on the critical path).
   // k_full[st] also takes one arrival per softmax warp once it is done with
@@ -74,31 +102,34 @@ struct Ctl {
   int blocks[kMaxList];
   float bias[kMaxList];  // log2-domain gate bias of each attended block
 };
-constexpr size_t kSmemBytes = kOffCtl + sizeof(Ctl) + 1024;  // + alignment slack
-
-// TMEM columns: Q[tile] (A operand, bf16 pairs) at tile*64, S[tile] at
-// 128 + tile*64, O[tile] at 256 + tile*128.
-__device__ __forceinline__ uint32_t q_col(int t) { return t * 64; }
-__device__ __forceinline__ uint32_t s_col(int t) { return 128 + t * 64; }
-__device__ __forceinline__ uint32_t o_col(int t) { return 256 + t * 128; }
+template <int TILES>
+constexpr size_t fwd_smem_bytes() {
+  return FwdLayout<TILES>::kOffCtl + sizeof(Ctl<FwdLayout<TILES>::kStages>) + 1024;  // + alignment
+}
+static_assert(2 * (fwd_smem_bytes<1>() + 1024) <= 228 * 1024, "two one-tile CTAs per SM");
 
 template <int TILES, bool OUTER>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(FwdLayout<TILES>::kThreads) __maxnreg__(FwdLayout<TILES>::kMaxRegs)
 tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ idx,
               const float* __restrict__ gates, AttnShape s, __nv_bfloat16* __restrict__ o,
               float* __restrict__ lse, DevCtx ctx) {
+  using L = FwdLayout<TILES>;
+  constexpr int kStages = L::kStages;
+  constexpr uint32_t kOffQ = L::kOffQ, kOffK = L::kOffK, kOffV = L::kOffV, kOffP = L::kOffP;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   unsigned char* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   const uint32_t sbase = smem_u32(base);
-  Ctl& c = *reinterpret_cast<Ctl*>(base + kOffCtl);
+  Ctl<kStages>& c = *reinterpret_cast<Ctl<kStages>*>(base + L::kOffCtl);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // Dense: the longest query blocks (most keys) start first.
   const int j = s.dense ? s.N - 1 - (int)blockIdx.x : (int)blockIdx.x;
-  const int kvh = blockIdx.y, bi = blockIdx.z;
-  const int G = 2 * TILES;
+  // blockIdx.y: KV head and, with TILES = 1, which of its G/2 tiles.
+  const int G = s.Hq / s.Hkv;
+  const int tpk = G / (2 * TILES);  // CTAs per KV head
+  const int kvh = blockIdx.y / tpk, u0 = (blockIdx.y % tpk) * TILES, bi = blockIdx.z;
   const long long irow = ((long long)(bi * s.Hkv + kvh) * s.N + j);
 
   if (tid == 0) {
@@ -121,7 +152,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       for (int hh = 0; hh < 2; ++hh)
         for (int kb = 0; kb < 2; ++kb)
           tma_load_3d(base + kOffQ + t * 32768 + kb * 16384 + hh * 8192, &tm_q, kb * 64, j * kB,
-                      bi * s.Hq + kvh * G + 2 * t + hh, &c.q_full);
+                      bi * s.Hq + kvh * G + 2 * (u0 + t) + hh, &c.q_full);
   }
   if (warp == 0) {
     // Attended blocks in order: block j (bias 0, the largest logits in
@@ -141,7 +172,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
   }
   if (warp == 1) {
-    tmem_alloc(&c.tmem_base, kTmemCols);
+    tmem_alloc(&c.tmem_base, L::kTmemCols);
     tmem_relinquish();
   }
   fence_before_sync();
@@ -151,10 +182,10 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const int nblk = c.nblk;
   volatile int* abort = &c.abort;
 
-  if (warp == 0 || warp == 2) {
+  if (warp == L::kWarpK || warp == L::kWarpV) {
     // ------------------------------------------------------------ producers
     if (lane == 0) {
-      const bool kside = (warp == 0);
+      const bool kside = (warp == L::kWarpK);
       const CUtensorMap* map = kside ? &tm_k : &tm_v;
       uint64_t* full = kside ? c.k_full : c.v_full;
       uint64_t* empty = kside ? c.k_empty : c.v_empty;
@@ -180,7 +211,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           (void)mbar_wait(ctx, &full[n % kStages], (n / kStages) & 1);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == L::kWarpMMA) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16(128, 64, false, false);
@@ -203,7 +234,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int t = 0; t < TILES; ++t) {
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
-            mma_bf16_ts(tmem + s_col(t), tmem + q_col(t) + ks * 8,
+            mma_bf16_ts(tmem + L::s_col(t), tmem + L::q_col(t) + ks * 8,
                         adv(kd, (ks >> 2) * 8192 + (ks & 3) * 32), id_s, ks > 0);
         }
         mma_commit(&c.s_full);
@@ -222,7 +253,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           const uint64_t pd = adv(pdesc0, t * 16384);
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
-            mma_bf16_ss(tmem + o_col(t), adv(pd, ks * 32), adv(vd, ks * 2048), id_o,
+            mma_bf16_ss(tmem + L::o_col(t), adv(pd, ks * 32), adv(vd, ks * 2048), id_o,
                         (n > 0 || ks > 0));
         }
         mma_commit(&c.pv_done);
@@ -234,13 +265,13 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         (void)mbar_wait(ctx, &c.drain, 0);
       }
     }
-  } else if (warp >= kFirstSoftmaxWarp) {
+  } else if (warp >= L::kSoftFirst && warp < L::kSoftFirst + 4 * TILES) {
     // ------------------------------------------------------------ softmax
-    const int t = (warp - kFirstSoftmaxWarp) >> 2;
+    const int t = (warp - L::kSoftFirst) >> 2;
     const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
     const int rowi = quarter * 32 + lane;         // row of the M-tile (TMEM lane)
     const int hh = rowi >> 6, r = rowi & 63;
-    const int head = kvh * G + 2 * t + hh;
+    const int head = kvh * G + 2 * (u0 + t) + hh;
     const int qrow = j * kB + r;
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
     const float sc = s.scale * kLog2e;
@@ -251,7 +282,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       if (!__all_sync(0xffffffffu, wait_or_abort(ctx, &c.q_full, 0, abort))) {
         ok = false;
       } else {
-        tile_row_to_tmem(base + kOffQ + t * 32768, rowi, tl + q_col(t));
+        tile_row_to_tmem(base + kOffQ + t * 32768, rowi, tl + L::q_col(t));
         tmem_st_wait();
         fence_before_sync();
         __syncwarp();
@@ -265,8 +296,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       }
       fence_after_sync();
       uint32_t sr[64];
-      tmem_ld32(tl + s_col(t), *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tl + s_col(t) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(tl + L::s_col(t), *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tl + L::s_col(t) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_ld_wait();
       fence_before_sync();
       __syncwarp();
@@ -311,11 +342,11 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
           uint32_t ov[32];
-          tmem_ld32(tl + o_col(t) + ch * 32, ov);
+          tmem_ld32(tl + L::o_col(t) + ch * 32, ov);
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-          tmem_st32(tl + o_col(t) + ch * 32, ov);
+          tmem_st32(tl + L::o_col(t) + ch * 32, ov);
         }
         tmem_st_wait();
         l *= alpha;
@@ -384,7 +415,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
           uint32_t ov[32];
-          tmem_ld32(tl + o_col(t) + ch * 32, ov);
+          tmem_ld32(tl + L::o_col(t) + ch * 32, ov);
           tmem_ld_wait();
           if (write) {
 #pragma unroll
@@ -406,7 +437,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   __syncthreads();
   if (warp == 1) {
     fence_after_sync();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, L::kTmemCols);
   }
 }
 
@@ -527,13 +558,27 @@ cudaError_t launch_attn_fwd_tc(const AttnShape& s, const void* q, const void* k,
   if ((e = make_tmap_bf16(&tk, k, s.T, s.B * s.Hkv)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16(&tv, v, s.T, s.B * s.Hkv)) != cudaSuccess) return e;
   const int G = s.Hq / s.Hkv;
-  dim3 grid(s.N, s.Hkv, s.B);
   const bool outer = s.outer && gates != nullptr;  // no gates: both gatings coincide
-  auto kern = G == 4 ? (outer ? tc_fwd_kernel<2, true> : tc_fwd_kernel<2, false>)
-                     : (outer ? tc_fwd_kernel<1, true> : tc_fwd_kernel<1, false>);
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-  if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, idx, gates, s, (__nv_bfloat16*)o, lse, ctx);
+  // One 128-row tile (two heads) per CTA, two CTAs per SM (kFwdTiles = 1), or
+  // both tiles of a G = 4 group in one CTA (kFwdTiles = 2).
+  constexpr int kFwdTiles = 1;
+  const int tiles = (G == 4 && kFwdTiles == 2) ? 2 : 1;
+  dim3 grid(s.N, s.Hkv * (G / (2 * tiles)), s.B);
+  if (tiles == 2) {
+    auto kern = outer ? tc_fwd_kernel<2, true> : tc_fwd_kernel<2, false>;
+    const size_t smem = fwd_smem_bytes<2>();
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, FwdLayout<2>::kThreads, smem, st>>>(tq, tk, tv, idx, gates, s,
+                                                     (__nv_bfloat16*)o, lse, ctx);
+  } else {
+    auto kern = outer ? tc_fwd_kernel<1, true> : tc_fwd_kernel<1, false>;
+    const size_t smem = fwd_smem_bytes<1>();
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, FwdLayout<1>::kThreads, smem, st>>>(tq, tk, tv, idx, gates, s,
+                                                     (__nv_bfloat16*)o, lse, ctx);
+  }
   note_launches(1);
   return cudaGetLastError();
 }
