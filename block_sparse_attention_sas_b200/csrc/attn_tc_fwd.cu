@@ -48,11 +48,11 @@ constexpr int kMaxList = 257;                        // K <= 256 selected + curr
 // are split into G/2 tiles of two heads).
 //   TILES = 2: 384 threads, 3-stage K and V rings, 512 TMEM columns (Q[t] at
 //              64 t, S[t] at 128 + 64 t, O[t] at 256 + 128 t): one CTA per SM,
-//              both tiles share every K/V block.
+//              both tiles share every K/V block (G = 4).
 //   TILES = 1: 224 threads, 2-stage rings, 256 TMEM columns (Q 0, S 64,
 //              O 128) and P in the Q staging area (free once Q is in TMEM):
 //              about 99 KB, two CTAs per SM, so one CTA's prologue, softmax
-//              and epilogue overlap the other's MMAs.
+//              and epilogue overlap the other's MMAs (G = 2).
 template <int TILES> struct FwdLayout;
 template <> struct FwdLayout<2> {
   static constexpr int kThreads = 384, kStages = 3, kMaxRegs = 168;
@@ -559,10 +559,11 @@ cudaError_t launch_attn_fwd_tc(const AttnShape& s, const void* q, const void* k,
   if ((e = make_tmap_bf16(&tv, v, s.T, s.B * s.Hkv)) != cudaSuccess) return e;
   const int G = s.Hq / s.Hkv;
   const bool outer = s.outer && gates != nullptr;  // no gates: both gatings coincide
-  // One 128-row tile (two heads) per CTA, two CTAs per SM (kFwdTiles = 1), or
-  // both tiles of a G = 4 group in one CTA (kFwdTiles = 2).
-  constexpr int kFwdTiles = 1;
-  const int tiles = (G == 4 && kFwdTiles == 2) ? 2 : 1;
+  // G = 4: both tiles of the group in one CTA, sharing every K/V block (one
+  // tile per CTA, two CTAs per SM, measured 0.58 ms against 0.41 ms on the
+  // Qwen3-4B layer: the K/V blocks are then fetched twice and the rings are
+  // shallower). G = 2: one tile per CTA, two CTAs per SM.
+  const int tiles = G == 4 ? 2 : 1;
   dim3 grid(s.N, s.Hkv * (G / (2 * tiles)), s.B);
   if (tiles == 2) {
     auto kern = outer ? tc_fwd_kernel<2, true> : tc_fwd_kernel<2, false>;
