@@ -538,49 +538,183 @@ gate_topk_merge_kernel(const float* __restrict__ scores, int rows, int C, int ca
 }
 
 // ---------------------------------------------------------------------------
-// Decode-sized rows (513 .. 8192 entries): one CTA of 256 threads per row,
-// thread t holding entries t + 256 e (coalesced loads). The row's max M and min come
-// from one reduction, the gate softmax's sum from a second. Selection without
-// sorting the row: a 256-bucket histogram of (M - s) in steps of 1/32 finds
-// the bucket b* holding the k-th largest score (when that lies more than 8
-// below M, a second histogram spreads the rest of the row's range over 256
-// buckets). Histogram adds are combined per warp and bucket, and the
-// overflow bucket is never counted (its count is the rest of the row). Every
-// score in a bucket up to b* is a candidate -- a superset of
-// the top k, usually a few more than k -- and each candidate is placed by its
-// rank among the candidates under the composite order (descending score,
-// ties to the lower index), which is its rank in the row. More than 1024
-// candidates (mass ties) make the block sort the whole row instead.
+// Decode-sized rows (513 .. 8192 entries): a thread-block cluster of CS CTAs
+// per row, CTA r holding the 512 entries [512 r, 512 r + 512), two per
+// thread. Selection without sorting the row:
+//  1. each CTA's (max, min, sum of exp) are read by every CTA of the cluster
+//     through distributed shared memory (one round trip, lane x reading rank
+//     x); every CTA forms the row's max M and LSE alike;
+//  2. each CTA histograms its chunk over 64 buckets of (M - s) in steps of
+//     1/8 (bucket 63: everything further down, never counted: its count is
+//     the rest of the row) and adds the histogram into every CTA's copy of
+//     the row's histogram (remote reductions, no round trip); after a
+//     cluster barrier each CTA finds b*, the bucket holding the k-th largest
+//     score, in its own copy. When that is bucket 63, a second histogram
+//     spreads [min, M - 63/8] over 64 buckets the same way;
+//  3. every score in a bucket up to b* is a candidate -- a superset of the
+//     top k, usually a few more than k. Each warp reserves room in rank 0's
+//     list with one remote atomic and stores its candidates there; rank 0
+//     places each by its rank among them under the composite order
+//     (descending score, ties to the lower index), which is its rank in the
+//     row.
+// More than 1024 candidates (mass ties, known from the histogram) switch the
+// cluster to an exact path: each CTA selects its chunk's best k and stores
+// them in rank 0's list, which rank 0 places by rank. The gates are written
+// last, so that no cluster barrier waits for those stores.
 // ---------------------------------------------------------------------------
-constexpr int kBkThreads = 256;
-constexpr int kBkCand = 1024;
-constexpr float kBkStep = 32.f;  // level-1 buckets per unit of score below the max
+constexpr int kCbThreads = 256;
+constexpr int kCbChunk = 512;   // entries per CTA
+constexpr int kCbMaxCta = 16;   // rows up to 8192 entries
+constexpr int kCbCand = 1024;   // candidates rank 0 places by rank
+constexpr int kNB = 64;         // buckets per histogram level
+constexpr float kBkStep = 8.f;  // level-1 buckets per unit of score below the max
 
-template <int EPT>
-__global__ void __launch_bounds__(kBkThreads)
-gate_topk_bucket_kernel(const float* __restrict__ scores, int rows, int C, int causal, int K,
-                        int phi, float* __restrict__ gates, int32_t* __restrict__ idx) {
-  extern __shared__ uint64_t s_sort[];  // EPT * 256 keys; used only by the fallback
-  __shared__ int s_hist[256];
-  __shared__ uint64_t s_cand[kBkCand];
-  __shared__ float s_red[3][8];
-  __shared__ int s_m, s_b1, s_b2, s_before;
+struct CbShared {
+  float part[3];                  // this chunk's max, min, sum of exp (relative to its max)
+  int hist[kNB];                  // this chunk's histogram
+  unsigned int row_hist[2][kNB];  // the row's, levels 1 and 2 (the cluster adds into it)
+  unsigned int nlist;             // rank 0: keys in its list
+  uint64_t best[kCbChunk];        // the exact path: this chunk's best, sorted
+  float red[2][8];
+  int wsum[8];
+  float M, Mn, lse;
+  int bstar, before, upto;
+  TopkScratch ts;  // the exact path
+};
+
+__device__ __forceinline__ float fast_gate(float sc, float lse, int phi) {
+  if (phi == SAS_PHI_SIGMOID) return 1.f / (1.f + __expf(-sc));
+  if (phi == SAS_PHI_RAW) return __expf(sc);
+  return __expf(sc - lse);
+}
+
+// Finds, in the row histogram h, the bucket holding the target-th entry in
+// bucket order (warp 0; lane l sums buckets 2l and 2l + 1). `rest` >= 0
+// gives the last bucket the count `rest` minus the other buckets' total (a
+// bucket no CTA counts). Returns the bucket; *before / *upto = entries in
+// the buckets before it / up to and including it. Every thread calls it;
+// the result is the same in every CTA.
+__device__ int find_bucket(const unsigned int* h, int target, int rest, CbShared& sh, int* before,
+                           int* upto) {
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int c0 = (int)h[2 * lane];
+    int c1 = (rest >= 0 && lane == 31) ? 0 : (int)h[2 * lane + 1];
+    int inc = c0 + c1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    const int tot = __shfl_sync(0xffffffffu, inc, 31);
+    if (rest >= 0 && lane == 31) {  // the uncounted bucket takes the rest
+      c1 = rest - tot;
+      inc = rest;
+    }
+    const int ex = inc - c0 - c1;  // entries before bucket 2 lane
+    if (ex < target && ex + c0 >= target) {
+      sh.bstar = 2 * lane;
+      sh.before = ex;
+      sh.upto = ex + c0;
+    } else if (ex + c0 < target && inc >= target) {
+      sh.bstar = 2 * lane + 1;
+      sh.before = ex + c0;
+      sh.upto = inc;
+    }
+  }
+  __syncthreads();
+  *before = sh.before;
+  *upto = sh.upto;
+  return sh.bstar;  // rewritten only after a later barrier
+}
+
+// Adds this CTA's histogram (sh.hist) into the row histogram `dst` of every
+// CTA of the cluster (thread t: bucket t % 64 into ranks t / 64, t / 64 + 4,
+// ...), then clears sh.hist.
+__device__ __forceinline__ void push_hist(CbShared& sh, unsigned int* dst, int CS) {
+  const int tid = threadIdx.x, bkt = tid & (kNB - 1);
+  __syncthreads();  // the local histogram is complete
+  const unsigned int v = (unsigned int)sh.hist[bkt];
+  if (v)
+    for (int x = tid / kNB; x < CS; x += kCbThreads / kNB)
+      dsmem_red_add_u32(dsmem_addr(&dst[bkt], (uint32_t)x), v);
+  __syncthreads();  // read before cleared
+  if (tid < kNB) sh.hist[tid] = 0;
+}
+
+// Places keys[0, m) by rank (keys equal to 0 are empty slots): out[rank] =
+// index for the kk best. Short lists: a group of tpc threads per key splits
+// the comparisons; long lists: four keys per thread, one pass over the list.
+__device__ __forceinline__ void place_by_rank(const uint64_t* keys, int m, int kk, int32_t* out) {
+  const int tid = threadIdx.x;
+  if (m <= kCbThreads) {
+    int tpc = 1;
+    while (tpc < 8 && 2 * tpc * m <= kCbThreads) tpc *= 2;
+    const int p = tid / tpc, part = tid % tpc;
+    const uint64_t mine = p < m ? keys[p] : 0ull;
+    int rk = 0;
+#pragma unroll 4
+    for (int q = part; q < m; q += tpc) rk += keys[q] > mine;
+    for (int o = 1; o < tpc; o <<= 1) rk += __shfl_xor_sync(0xffffffffu, rk, o);
+    if (part == 0 && mine != 0ull && rk < kk) out[rk] = ckey_index(mine);
+    return;
+  }
+  for (int p0 = tid; p0 < m; p0 += 4 * kCbThreads) {
+    uint64_t mine[4];
+    int rk[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int p = p0 + u * kCbThreads;
+      mine[u] = p < m ? keys[p] : 0ull;
+      rk[u] = 0;
+    }
+    for (int q = 0; q < m; ++q) {
+      const uint64_t y = keys[q];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) rk[u] += y > mine[u];
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (mine[u] != 0ull && rk[u] < kk) out[rk[u]] = ckey_index(mine[u]);
+  }
+}
+
+__global__ void __launch_bounds__(kCbThreads)
+gate_topk_cbucket_kernel(const float* __restrict__ scores, int rows, int C, int causal, int K,
+                         int CS, int phi, float* __restrict__ gates, int32_t* __restrict__ idx) {
+  // rank 0's list: the candidates, or CS chunks' best kk on the exact path
+  extern __shared__ uint64_t s_list[];
+  __shared__ CbShared sh;
   grid_launch_dependents();  // a dependent decode may start its prologue
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const long long row = blockIdx.x;
+  const uint32_t rank = cluster_rank();
+  const long long row = blockIdx.x / CS;
   const int r = (int)(row % rows);
   const int n = causal ? min(r, C) : C;
+  const int kk = min(K, n);  // the same in every CTA of the cluster
+  const int lo = (int)rank * kCbChunk;
   const float* srow = scores + row * (long long)C;
-  // entry of slot e: tid + 256 e
-  auto ix = [&](int e) -> int { return tid + kBkThreads * e; };
+  float* grow = gates + row * (long long)C;
+  int32_t* out = idx + row * (long long)K;
+  if (kk == 0) {  // an empty history (the whole cluster): gates 0, no selection
+    for (int e = 0; e < 2; ++e) {
+      const int i = lo + tid + kCbThreads * e;
+      if (i < C) grow[i] = 0.f;
+    }
+    if (rank == 0)
+      for (int p = tid; p < K; p += kCbThreads) out[p] = -1;
+    return;
+  }
 
-  float f[EPT];
+  float f[2];
+  bool ok[2];
   float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
-  for (int e = 0; e < EPT; ++e) {
-    const bool ok = ix(e) < n;
-    f[e] = ok ? srow[ix(e)] : -INFINITY;
-    if (ok) {
+  for (int e = 0; e < 2; ++e) {
+    const int i = lo + tid + kCbThreads * e;
+    ok[e] = i < n;
+    f[e] = ok[e] ? srow[i] : -INFINITY;
+    if (ok[e]) {
       mx = fmaxf(mx, f[e]);
       mn = fminf(mn, f[e]);
     }
@@ -588,150 +722,130 @@ gate_topk_bucket_kernel(const float* __restrict__ scores, int rows, int C, int c
   mx = warp_max(mx);
   mn = -warp_max(-mn);
   if (lane == 0) {
-    s_red[0][warp] = mx;
-    s_red[1][warp] = mn;
+    sh.red[0][warp] = mx;
+    sh.red[1][warp] = mn;
   }
+  if (tid < kNB) {
+    sh.hist[tid] = 0;
+    sh.row_hist[0][tid] = 0u;
+    sh.row_hist[1][tid] = 0u;
+  }
+  if (tid == 0) sh.nlist = 0u;
   __syncthreads();
-  float M = -INFINITY, Mn = INFINITY;
+  float cm = -INFINITY, cmn = INFINITY;
 #pragma unroll
   for (int x = 0; x < 8; ++x) {
-    M = fmaxf(M, s_red[0][x]);
-    Mn = fminf(Mn, s_red[1][x]);
+    cm = fmaxf(cm, sh.red[0][x]);
+    cmn = fminf(cmn, sh.red[1][x]);
   }
   float sum = 0.f;
 #pragma unroll
-  for (int e = 0; e < EPT; ++e)
-    if (ix(e) < n) sum += expf(f[e] - M);
+  for (int e = 0; e < 2; ++e)
+    if (ok[e]) sum += __expf(f[e] - cm);
   sum = warp_sum(sum);
-  if (lane == 0) s_red[2][warp] = sum;
-  if (tid < 256) s_hist[tid] = 0;
-  if (tid == 0) s_m = 0;
+  if (lane == 0) sh.wsum[warp] = __float_as_int(sum);
   __syncthreads();
-  float S = 0.f;
+  if (tid == 0) {
+    float t = 0.f;
 #pragma unroll
-  for (int x = 0; x < 8; ++x) S += s_red[2][x];
-  const float lse = M + logf(S);
-  float* grow = gates + row * (long long)C;
-#pragma unroll
-  for (int e = 0; e < EPT; ++e) {
-    const int i = ix(e);
-    if (i < C) grow[i] = i < n ? gate_of(f[e], lse, phi) : 0.f;
+    for (int x = 0; x < 8; ++x) t += __int_as_float(sh.wsum[x]);
+    sh.part[0] = cm;
+    sh.part[1] = cmn;
+    sh.part[2] = t;
   }
-  const int kk = min(K, n);
-  int32_t* out = idx + row * (long long)K;
-  for (int p = kk + tid; p < K; p += kBkThreads) out[p] = -1;
-  if (kk == 0) return;  // uniform over the CTA
+  // (1) the partials are written and every CTA's row histograms and list
+  // counter are cleared before anyone adds into them
+  cluster_sync_all();
 
-  // ---- level 1: buckets of width 1/32 below the max (bucket 255: the rest)
-  auto b1_of = [&](float x) -> int { return min(255, (int)((M - x) * kBkStep)); };
-#pragma unroll
-  for (int e = 0; e < EPT; ++e) {
-    const int bb = ix(e) < n ? b1_of(f[e]) : 255;
-    warp_hist_add(s_hist, (uint32_t)bb, bb < 255);
-  }
-  if (tid == 0) s_hist[255] = 0;  // never counted: the rest of the row
-  __syncthreads();
-  // Warp 0 finds the first bucket whose running count reaches the target.
-  auto find_bucket = [&](int target, int& bstar, int& before) {
-    int h[8], tot = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      h[i] = s_hist[lane * 8 + i];
-      tot += h[i];
-    }
-    int incl = tot;  // inclusive prefix over lanes
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int run = incl - tot, b = -1, bef = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (b < 0 && run + h[i] >= target) {
-        b = lane * 8 + i;
-        bef = run;
-      }
-      run += h[i];
-    }
-    const uint32_t hit = __ballot_sync(0xffffffffu, b >= 0);
-    const int src = __ffs(hit) - 1;  // the lowest lane holds the first such bucket
-    bstar = __shfl_sync(0xffffffffu, b, src);
-    before = __shfl_sync(0xffffffffu, bef, src);
-  };
   if (warp == 0) {
-    // bucket 255 holds whatever the first 255 buckets do not
-    int cnt = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) cnt += (lane * 8 + i < 255) ? s_hist[lane * 8 + i] : 0;
-    cnt = warp_sum(cnt);
-    __syncwarp();
-    if (lane == 31) s_hist[255] = n - cnt;
-    __syncwarp();
-    int bs, bf;
-    find_bucket(kk, bs, bf);
+    float pm = -INFINITY, pmn = INFINITY, ps = 0.f;
+    if (lane < CS) {
+      pm = dsmem_ld_f32(dsmem_addr(&sh.part[0], (uint32_t)lane));
+      pmn = dsmem_ld_f32(dsmem_addr(&sh.part[1], (uint32_t)lane));
+      ps = dsmem_ld_f32(dsmem_addr(&sh.part[2], (uint32_t)lane));
+    }
+    const float M = warp_max(pm);
+    const float Mn = -warp_max(-pmn);
+    const float S = warp_sum(ps > 0.f ? ps * __expf(pm - M) : 0.f);
     if (lane == 0) {
-      s_b1 = bs;
-      s_before = bf;
-      s_b2 = 255;
+      sh.M = M;
+      sh.Mn = Mn;
+      sh.lse = M + __logf(S);
     }
   }
   __syncthreads();
-  const int b1 = s_b1;
-  // ---- level 2 (rare): the k-th largest lies in the overflow bucket; spread
-  // [min, M - 255/32) over 256 buckets, highest first.
-  const float top2 = M - 255.f / kBkStep;
-  const float inv2 = (top2 > Mn) ? 255.f / (top2 - Mn) : 0.f;
-  auto b2_of = [&](float x) -> int { return min(255, max(0, (int)((top2 - x) * inv2))); };
-  if (b1 == 255) {
-    const int need = kk - s_before;
-    if (tid < 256) s_hist[tid] = 0;
-    __syncthreads();
-#pragma unroll
-    for (int e = 0; e < EPT; ++e) {
-      const bool in = ix(e) < n && b1_of(f[e]) == 255;
-      warp_hist_add(s_hist, in ? (uint32_t)b2_of(f[e]) : 0u, in);
-    }
-    __syncthreads();
-    if (warp == 0) {
-      int bs, bf;
-      find_bucket(need, bs, bf);
-      if (lane == 0) s_b2 = bs;
-    }
-    __syncthreads();
-  }
-  const int b2 = s_b2;
+  const float M = sh.M, Mn = sh.Mn;
 
-  // ---- candidates: every score in a bucket up to the k-th's
+  // ---- level 1: 1/8-wide buckets below the max; the last is never counted
+  auto b1_of = [&](float x) -> int { return (int)fminf((M - x) * kBkStep, (float)(kNB - 1)); };
 #pragma unroll
-  for (int e = 0; e < EPT; ++e) {
-    const int bb = ix(e) < n ? b1_of(f[e]) : 256;
-    const bool take = bb < b1 || (bb == b1 && (b1 < 255 || b2_of(f[e]) <= b2));
-    // one atomic per warp: lanes place themselves after the warp's base
-    const uint32_t mask = __ballot_sync(0xffffffffu, take);
-    int basep = 0;
-    if (lane == 0 && mask) basep = atomicAdd(&s_m, __popc(mask));
-    basep = __shfl_sync(0xffffffffu, basep, 0);
-    const int p = basep + __popc(mask & ((1u << lane) - 1u));
-    if (take && p < kBkCand) s_cand[p] = ckey(f[e], ix(e));
+  for (int e = 0; e < 2; ++e)
+    if (ok[e]) {
+      const int bb = b1_of(f[e]);
+      if (bb < kNB - 1) atomicAdd(&sh.hist[bb], 1);
+    }
+  push_hist(sh, sh.row_hist[0], CS);
+  cluster_sync_all();  // (2) the row histogram is complete in every CTA
+  int before, upto;
+  const int b1 = find_bucket(sh.row_hist[0], kk, n, sh, &before, &upto);
+
+  // ---- level 2 (rare: the k-th score lies 63/8 or more below the max):
+  // 64 buckets spread over [Mn, M - 63/8]
+  const float top2 = M - (float)(kNB - 1) / kBkStep;
+  const float inv2 = top2 > Mn ? (float)(kNB - 1) / (top2 - Mn) : 0.f;
+  auto b2_of = [&](float x) -> int {
+    return (int)fminf(fmaxf((top2 - x) * inv2, 0.f), (float)(kNB - 1));
+  };
+  int b2 = kNB - 1;
+  int ncand = upto;
+  if (b1 == kNB - 1) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+      if (ok[e] && b1_of(f[e]) == kNB - 1) atomicAdd(&sh.hist[b2_of(f[e])], 1);
+    push_hist(sh, sh.row_hist[1], CS);
+    cluster_sync_all();  // (2b)
+    int before2, upto2;
+    b2 = find_bucket(sh.row_hist[1], kk - before, -1, sh, &before2, &upto2);
+    ncand = before + upto2;
   }
-  __syncthreads();
-  const int m = s_m;
-  if (m <= kBkCand) {
-    // rank of each candidate among the candidates = its rank in the row
-    for (int p = tid; p < m; p += kBkThreads) {
-      const uint64_t key = s_cand[p];
-      int rank = 0;
-      for (int q = 0; q < m; ++q) rank += s_cand[q] > key;
-      if (rank < kk) out[rank] = ckey_index(key);
+
+  const uint32_t list0 = dsmem_addr(s_list, 0u), nlist0 = dsmem_addr(&sh.nlist, 0u);
+  const bool exact = ncand > kCbCand;
+  if (!exact) {
+    // ---- this chunk's candidates into rank 0's list
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int bb = ok[e] ? b1_of(f[e]) : kNB;
+      const bool take = bb < b1 || (bb == b1 && (b1 < kNB - 1 || b2_of(f[e]) <= b2));
+      const uint32_t mask = __ballot_sync(0xffffffffu, take);
+      if (mask == 0u) continue;
+      uint32_t slot = 0u;
+      if (lane == 0) slot = dsmem_atom_add_u32(nlist0, (uint32_t)__popc(mask));
+      slot = __shfl_sync(0xffffffffu, slot, 0) + (uint32_t)__popc(mask & ((1u << lane) - 1u));
+      if (take) dsmem_st_u64(list0 + 8u * slot, ckey(f[e], lo + tid + kCbThreads * e));
     }
   } else {
-    // mass ties: sort the whole row (every thread's keys) in shared memory
-    uint64_t v[EPT];
+    // ---- exact path (mass ties): each chunk's best kk into rank 0's list,
+    // at rank * kk (empty slots 0)
+    const int len = max(0, min(n - lo, kCbChunk));
+    const int kc = min(kk, len);
+    uint64_t v[2];
 #pragma unroll
-    for (int e = 0; e < EPT; ++e) v[e] = (ix(e) < n) ? ckey(f[e], ix(e)) : 0ull;
-    block_sort_desc<EPT>(v, s_sort);
-    for (int p = tid; p < kk; p += kBkThreads) out[p] = ckey_index(s_sort[p]);
+    for (int e = 0; e < 2; ++e) v[e] = ok[e] ? ckey(f[e], lo + tid + kCbThreads * e) : 0ull;
+    if (kc > 0) block_topk<2>(v, kc, sh.ts, sh.best);  // the best kc, sorted, in sh.best
+    for (int p = tid; p < kk; p += kCbThreads)
+      dsmem_st_u64(list0 + 8u * (uint32_t)(rank * kk + p), p < kc ? sh.best[p] : 0ull);
+  }
+  cluster_sync_all();  // (3) rank 0 holds the list; no CTA touches another's memory after this
+  if (rank == 0) {
+    place_by_rank(s_list, exact ? CS * kk : (int)sh.nlist, kk, out);
+    for (int p = kk + tid; p < K; p += kCbThreads) out[p] = -1;
+  }
+  const float lse = sh.lse;
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int i = lo + tid + kCbThreads * e;
+    if (i < C) grow[i] = i < n ? fast_gate(f[e], lse, phi) : 0.f;
   }
 }
 
@@ -858,6 +972,54 @@ int pow2_at_least(int x) {
   return p;
 }
 
+// The bucket-selection cluster kernel for rows of up to 16 * 512 entries,
+// when the device holds such a cluster; false leaves the row to other paths.
+bool launch_cbucket_topk(const float* scores, long long total, int rows, int C, int causal, int K,
+                         int phi, float* gates, int32_t* idx, cudaStream_t stream) {
+  if (C > kCbMaxCta * kCbChunk || total * kCbMaxCta > 0x7fffffffLL) return false;
+  const int CS = (C + kCbChunk - 1) / kCbChunk;
+  if (CS < 2) return false;
+  // rank 0's gather buffer: the bucket path's candidates, or the exact path's CS * K
+  const size_t smem = (size_t)max(kCbCand, CS * K) * sizeof(uint64_t);
+  auto kern = gate_topk_cbucket_kernel;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(total * CS));
+  cfg.blockDim = dim3(kCbThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static std::mutex mu;
+  static signed char fits[kCbMaxCta + 1] = {};
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (fits[CS] == 0) {
+      bool ok = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)(kCbMaxCta * 256 * sizeof(uint64_t))) == cudaSuccess;
+      if (ok && CS > 8)
+        ok = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+             cudaSuccess;
+      int nclusters = 0;
+      if (ok) ok = cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) == cudaSuccess;
+      fits[CS] = (ok && nclusters > 0) ? 1 : -1;
+      (void)cudaGetLastError();
+    }
+    if (fits[CS] < 0) return false;
+  }
+  if (cudaLaunchKernelEx(&cfg, kern, scores, rows, C, causal, K, CS, phi, gates, idx) !=
+      cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  note_launches(1);
+  return true;
+}
+
 // Launches the cluster kernel when the row fits (C <= 16 chunks of 4096) and
 // the device can hold such a cluster; returns false (nothing launched) to
 // leave the row to the two-launch path.
@@ -924,17 +1086,8 @@ cudaError_t launch_gate_topk(const float* scores, int B, int Hkv, int rows, int 
     gate_topk_warp_kernel<<<(unsigned)grid, 32 * kWarpRowsPerCta, 0, stream>>>(
         scores, (int)total, rows, C, causal, K, phi, gates, idx);
     note_launches(1);
-  } else if (C <= 32 * kBkThreads) {
-    // Decode-sized rows: one CTA per row, bucket selection.
-    const int EPT = C <= 4 * kBkThreads ? 4 : C <= 8 * kBkThreads ? 8 : C <= 16 * kBkThreads ? 16 : 32;
-    const size_t smem = (size_t)EPT * kBkThreads * sizeof(uint64_t);  // the fallback's sort
-    auto kern = EPT == 4 ? gate_topk_bucket_kernel<4> : EPT == 8 ? gate_topk_bucket_kernel<8>
-              : EPT == 16 ? gate_topk_bucket_kernel<16> : gate_topk_bucket_kernel<32>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    kern<<<(unsigned)total, kBkThreads, smem, stream>>>(scores, rows, C, causal, K, phi, gates, idx);
-    note_launches(1);
+  } else if (launch_cbucket_topk(scores, total, rows, C, causal, K, phi, gates, idx, stream)) {
+    // decode-sized rows: a cluster per row, bucket selection
   } else if (launch_cluster_topk(scores, total, rows, C, causal, K, phi, gates, idx, stream)) {
     // one launch: a cluster of chunk CTAs per row
   } else if (C <= 2048) {

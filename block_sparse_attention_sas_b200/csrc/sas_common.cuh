@@ -132,6 +132,19 @@ __device__ __forceinline__ uint64_t dsmem_ld_u64(uint32_t a) {
   asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(a) : "memory");
   return v;
 }
+__device__ __forceinline__ void dsmem_st_u64(uint32_t a, uint64_t v) {
+  asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(a), "l"(v) : "memory");
+}
+// Adds v to the u32 at a (no return value: the store-like form).
+__device__ __forceinline__ void dsmem_red_add_u32(uint32_t a, uint32_t v) {
+  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+// Adds v to the u32 at a and returns the value it held before.
+__device__ __forceinline__ uint32_t dsmem_atom_add_u32(uint32_t a, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(a), "r"(v) : "memory");
+  return old;
+}
 __device__ __forceinline__ float4 dsmem_ld_f32x4(uint32_t a) {
   float4 v;
   asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
