@@ -49,6 +49,17 @@ L2_FLUSH_BYTES = 256 << 20
 HEAD_START_CYCLES = 2_000_000
 
 
+# DRAM bytes (read + write) per call from ncu (dram__bytes_read.sum +
+# dram__bytes_write.sum summed over the call's D, dK/dV and dq kernels, one
+# --set full capture each of `bench.py --profile-train 8192`), for the
+# kernels as they stand. The capture ran the same layer at T = 8192; the
+# figure is scaled to T = 16384 by the attended pairs (536.1 M / 259.1 M),
+# which every kernel's work follows.
+MEASURED_TRAFFIC = {
+    ("qwen3-4b-train B1 Hq32/Hkv8 T16384 d128 b64 K16", "sas_attn_bwd"): 2023.9e6 * 536084480 / 259129344,
+}
+
+
 def attended_pairs(B, Hq, T, b, K):
     """Sum over query rows of the keys each row attends (selected blocks + causal current)."""
     N = (T + b - 1) // b
@@ -374,7 +385,9 @@ def run_ours(args):
     roof = {"kernel": dom, "bound": "tensor", "achieved": achieved,
             "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
             "frac": (achieved / peaks["bf16_tflops"]) if achieved else None,
-            "traffic": None, "peak_source": peaks["source"] + " (burst bf16 dense)"}
+            "traffic": MEASURED_TRAFFIC.get((cfg.name, dom)),
+            "traffic_unit": "bytes per call",
+            "peak_source": peaks["source"] + " (burst bf16 dense)"}
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -585,23 +598,50 @@ def bench_decode(S, torch, dev, stream, flush, peaks, args, rank):
                 ev[2].record(stream)
             return o
 
+        def two(ev):  # gate_topk then decode, no event between them
+            ev[0].record(stream)
+            gates, idx = S.gate_topk(t["s"], cfg.K, causal=False)
+            S.decode(t["q"], t["kc"], t["vc"], idx[:, :, 0], gates[:, :, 0], use_gates, cfg.b,
+                     L=cfg.L)
+            ev[1].record(stream)
+
+        s3 = t["s"][:, :, 0]
+
+        def fused(ev):  # the one call: selection inside the decode's launch
+            ev[0].record(stream)
+            S.decode_select(t["q"], t["kc"], t["vc"], s3, cfg.K, use_gates, cfg.b, L=cfg.L)
+            ev[1].record(stream)
+
         for _ in range(max(3, args.warmup)):
             one()
         reps = max(10, args.steps)
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
-        for i in range(reps):
-            flush.zero_()
-            torch.cuda._sleep(HEAD_START_CYCLES)
-            one(evs[i])
-        torch.cuda.synchronize(dev)
+
+        def timed(fn, nev):
+            evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(reps)]
+            for i in range(reps):
+                flush.zero_()
+                torch.cuda._sleep(HEAD_START_CYCLES)
+                fn(evs[i])
+            torch.cuda.synchronize(dev)
+            return evs
+
+        evs = timed(one, 3)
         topk_us = 1e3 * statistics.median(e[0].elapsed_time(e[1]) for e in evs)
         dec_us = 1e3 * statistics.median(e[1].elapsed_time(e[2]) for e in evs)
+        evs = timed(two, 2)
+        two_us = 1e3 * statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+        for _ in range(3):
+            fused([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+        evs = timed(fused, 2)
+        step_us = 1e3 * statistics.median(e[0].elapsed_time(e[1]) for e in evs)
         nbytes = decode_bytes(cfg)
         gbs = nbytes / (dec_us * 1e-6) / 1e9
-        line = {"workload": cfg.name, "use_gates": use_gates, "decode_us": dec_us,
-                "gate_topk_us": topk_us, "step_us": dec_us + topk_us,
-                "selected_bytes": nbytes, "GB/s": gbs,
-                "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+        line = {"workload": cfg.name, "use_gates": use_gates,
+                "step_us": step_us, "step": "sas_decode_select (gates, Top-K and decode, one call)",
+                "decode_us": dec_us, "gate_topk_us": topk_us, "two_launch_step_us": two_us,
+                "selected_bytes": nbytes, "GB/s": gbs, "step_GB/s": nbytes / (step_us * 1e-6) / 1e9,
+                "roofline": {"kernel": "decode_tc_kernel (sas_decode)", "bound": "hbm",
+                             "achieved": gbs, "peak": peaks["hbm_gbs"],
                              "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
                              "peak_source": peaks["source"] + " (copy bandwidth)"}}
         if use_gates == 0:
@@ -617,7 +657,7 @@ def bench_decode(S, torch, dev, stream, flush, peaks, args, rank):
             dbytes = decode_bytes(cfg, dense=True)
             line["dense"] = {"decode_us": dense_us, "bytes": dbytes,
                              "GB/s": dbytes / (dense_us * 1e-6) / 1e9,
-                             "speedup_sparse_step": dense_us / (dec_us + topk_us)}
+                             "speedup_sparse_step": dense_us / step_us}
         out.append(line)
     return out
 
@@ -658,6 +698,34 @@ def run_profile_train(args):
     torch.cuda.synchronize(dev)
     st, raw = S.device_error()
     print(json.dumps({"profile_train": cfg.name, "steps": args.warmup + args.steps,
+                      "device_error": st}), flush=True)
+    if st != 0:
+        raise SystemExit(1)
+
+
+def run_profile_decode(args):
+    """The decode step of one preset (sas_decode_select, gates on), warm-up
+    plus `steps` calls with the L2 flushed before each, untimed, for kernel
+    captures."""
+    import torch
+    from block_sparse_attention_sas_b200 import _lib as S
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cfg = W.PRESETS[args.profile_decode]
+    x = W.make_decode_inputs(cfg)
+    bf = torch.bfloat16
+    q = torch.from_numpy(x.q).to(bf).to(dev)
+    kc = torch.from_numpy(x.kcache).to(bf).to(dev)
+    vc = torch.from_numpy(x.vcache).to(bf).to(dev)
+    sc = torch.from_numpy(x.scores).to(dev)
+    del x
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup + args.steps):
+        flush.zero_()
+        S.decode_select(q, kc, vc, sc, cfg.K, True, cfg.b, L=cfg.L)
+    torch.cuda.synchronize(dev)
+    st, raw = S.device_error()
+    print(json.dumps({"profile_decode": cfg.name, "steps": args.warmup + args.steps,
                       "device_error": st}), flush=True)
     if st != 0:
         raise SystemExit(1)
@@ -743,6 +811,9 @@ def main():
                     help="time only the decode path of one preset (for profiling)")
     ap.add_argument("--profile-train", type=int, default=0, metavar="T",
                     help="run only the training step at sequence length T (for profiling)")
+    ap.add_argument("--profile-decode", default=None, metavar="PRESET",
+                    help="only run the decode step (sas_decode_select) warmup + steps times, "
+                         "untimed, for kernel captures")
     ap.add_argument("--no-8b", action="store_true", help="skip the Qwen3-8B training line")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense training line")
     ap.add_argument("--dry-run", action="store_true",
@@ -760,6 +831,8 @@ def main():
         run_decode_only(args)
     elif args.profile_train:
         run_profile_train(args)
+    elif args.profile_decode:
+        run_profile_decode(args)
     else:
         run_ours(args)
 

@@ -49,6 +49,9 @@ SIGNATURES = {
     "sas_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "sas_decode": (_i, [_i, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p,
                         _sz, _p]),
+    "sas_decode_select_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "sas_decode_select": (_i, [_i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p,
+                               _p, _p, _sz, _p]),
     "sas_decode_noalloc": (_i, [_i, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                                 _p, _p]),
     "sas_decode_noalloc_max_scratch": (_sz, []),
@@ -231,6 +234,33 @@ def decode(q, kcache, vcache, idx, gates, use_gates: bool, b: int, L: int | None
     _check("sas_decode", LIB.sas_decode(_dtype(q), _ptr(q), _ptr(kcache), _ptr(vcache), _ptr(idx),
                                         _ptr(gates), int(use_gates), B, Hq, Hkv, L, Lcap, d, b, K,
                                         scale, _ptr(o), _ptr(ws), ws.numel(), _stream(q.device)))
+    return o
+
+
+def decode_select(q, kcache, vcache, scores, K: int, use_gates: bool, b: int,
+                  L: int | None = None, scale: float = 0.0, o=None, gates=None, idx=None):
+    """One decode step from the selector scores [B,Hkv,C] (C = (L-1)//b):
+    gates and Top-K, then the decode; one launch where the shape allows.
+    gates [B,Hkv,C] / idx [B,Hkv,K], when given, receive the selection."""
+    for n, t in (("q", q), ("kcache", kcache), ("vcache", vcache)):
+        _need(t, n, q.dtype)
+    _need(scores, "scores", torch.float32)
+    B, Hq, d = q.shape
+    Hkv, Lcap = kcache.shape[1], kcache.shape[2]
+    L = Lcap if L is None else L
+    if o is None:
+        o = torch.empty_like(q)
+    if gates is not None:
+        _need(gates, "gates", torch.float32)
+    if idx is not None:
+        _need(idx, "idx", torch.int32)
+    nbytes = LIB.sas_decode_select_workspace_size(B, Hq, Hkv, L, d, b, K)
+    ws = _workspace("decode_select", nbytes, q.device, zero=False)
+    _check("sas_decode_select",
+           LIB.sas_decode_select(_dtype(q), _ptr(q), _ptr(kcache), _ptr(vcache), _ptr(scores),
+                                 int(use_gates), B, Hq, Hkv, L, Lcap, d, b, K, scale, _ptr(o),
+                                 _ptr(gates), _ptr(idx), _ptr(ws), ws.numel(),
+                                 _stream(q.device)))
     return o
 
 

@@ -42,6 +42,7 @@
 
 #include "sas_internal.h"
 #include "tc_common.cuh"
+#include "topk_select.cuh"
 
 namespace sas {
 namespace {
@@ -96,13 +97,27 @@ constexpr size_t kSmem = kOffCtl + sizeof(Ctl) + 1024;
 static_assert(kOffCtl % 16 == 0 && offsetof(Ctl, part_o) % 16 == 0 && (kD * 4) % 16 == 0,
               "the float4 accesses of part_o need 16-byte alignment");
 
-template <int G>
+// The fused selection (gates and Top-K of the unit's score row, then the
+// decode of the selected blocks in the same launch). Its scratch lives in the
+// K/V ring, which no load touches before the block lists exist.
+struct SelArgs {
+  bool on;              // select in the launch (else idx / gates are given)
+  const float* scores;  // [B * Hkv][C] selector scores (null when C == 0)
+  float* gates_out;     // [B * Hkv][C] or nullptr
+  int32_t* idx_out;     // [B * Hkv][K] or nullptr
+  int chunk;            // entries of the row per split (<= 512)
+};
+constexpr uint32_t kOffSelList = (sizeof(SelShared) + 127) & ~127u;  // from kOffKV
+static_assert(kOffSelList + 16 * 256 * 8 <= kStages * 32768,
+              "the selection scratch and list fit in the K/V ring");
+
+template <int G, bool SEL>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ idx,
                  const float* __restrict__ gates, DecodeShape s, __nv_bfloat16* __restrict__ o,
                  float* __restrict__ ws_ml, float* __restrict__ ws_o, uint32_t* __restrict__ ws_cnt,
-                 PagedArgs pa, DevCtx ctx) {
+                 PagedArgs pa, SelArgs sa, DevCtx ctx) {
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   unsigned char* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -159,7 +174,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       Cq = seq_ok ? (Lq - 1) / kB : 0;
     }
     int n = 0;
-    for (int sb = sl0; seq_ok && sb < sl1; sb += 32) {
+    for (int sb = sl0; !SEL && seq_ok && sb < sl1; sb += 32) {
       const int sl = sb + lane;
       int m = -1;
       float bias = 0.f;
@@ -204,13 +219,68 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       n += __popc(mask);
     }
     if (lane == 0) {
-      c.nblk = n;
+      if (!SEL) c.nblk = n;
       c.Lseq = Lq;
     }
   }
   if (warp == 1) {
     tmem_alloc(&c.tmem_base, kTmemCols);
     tmem_relinquish();
+  }
+  if constexpr (SEL) {
+    // ---- the unit's gates and Top-K, selected by its splits together
+    // (cluster_select); rank 0 stores each selected block, with its bias,
+    // into the control block of the split that owns its slot.
+    grid_dependency_wait();  // the scores may come from the previous grid
+    const int CS = s.splits, C = s.C, kk = min(s.K, C);
+    SelShared& sh = *reinterpret_cast<SelShared*>(base + kOffKV);
+    uint64_t* list = reinterpret_cast<uint64_t*>(base + kOffKV + kOffSelList);
+    const int lo = split * sa.chunk;
+    const float* srow = sa.scores + (long long)unit * C;
+    float f[4];
+    bool okf[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = lo + tid + kThreads * e;
+      okf[e] = i < C && i < lo + sa.chunk;
+      f[e] = okf[e] ? srow[i] : -INFINITY;
+    }
+    float lse = 0.f;
+    if (kk > 0) {  // the same in every split of the unit
+      const int m = cluster_select<kThreads, 4>(f, okf, lo, sa.chunk, C, kk, CS, sh, list);
+      lse = sh.lse;
+      if (split == 0) {
+        int32_t* iout = sa.idx_out ? sa.idx_out + (long long)unit * s.K : nullptr;
+        place_by_rank<kThreads>(list, m, kk, [&](int rk, uint64_t key) {
+          const int owner = rk / s.bps, pos = rk - owner * s.bps;
+          const int blk = ckey_index(key);
+          const float bias = s.use_gates ? (ckey_score(key) - lse) * kLog2e : 0.f;
+          dsmem_st_u32(dsmem_addr(&c.blocks[pos], (uint32_t)owner), (uint32_t)blk);
+          dsmem_st_f32(dsmem_addr(&c.bias[pos], (uint32_t)owner), bias);
+          if (iout) iout[rk] = blk;
+        });
+      }
+    }
+    if (split == 0 && sa.idx_out)
+      for (int p = kk + tid; p < s.K; p += kThreads) sa.idx_out[(long long)unit * s.K + p] = -1;
+    // This split's list: its selected slots [sl0, min(sl1, kk)), then the
+    // current block (slot K) when the split holds that slot.
+    if (tid == 0) {
+      int nb = max(0, min(sl1, kk) - sl0);
+      if (s.K >= sl0 && s.K < sl1) {
+        c.blocks[nb] = C;
+        c.bias[nb] = 0.f;
+        ++nb;
+      }
+      c.nblk = nb;
+    }
+    sel_sync(CS);  // (4) every split's list is complete
+    if (sa.gates_out) {
+      float* grow = sa.gates_out + (long long)unit * C;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (okf[e]) grow[lo + tid + kThreads * e] = fast_gate(f[e], lse, SAS_PHI_SOFTMAX);
+    }
   }
   fence_before_sync();
   __syncthreads();
@@ -592,15 +662,16 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 // Launch through cudaLaunchKernelEx: as a programmatic dependent of the
 // previous grid (its prologue overlaps that grid's tail), and with the
 // unit's splits as one cluster when s.cluster is set.
-template <int G>
+template <int G, bool SEL>
 cudaError_t launch_g(const DecodeShape& s, const CUtensorMap& tq, const CUtensorMap& tk,
                      const CUtensorMap& tv, const int32_t* idx, const float* gates, void* o,
                      float* ws_ml, float* ws_o, uint32_t* ws_cnt, const PagedArgs& pa,
-                     const DevCtx& ctx, cudaStream_t st, bool pdl) {
-  auto kern = decode_tc_kernel<G>;
+                     const SelArgs& sa, const DevCtx& ctx, cudaStream_t st, bool pdl) {
+  auto kern = decode_tc_kernel<G, SEL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
   if (e != cudaSuccess) return e;
-  if (s.cluster && s.splits > 8) {
+  const bool cluster = s.cluster || SEL;  // a fused selection always runs as one cluster
+  if (cluster && s.splits > 8) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
   }
@@ -616,7 +687,7 @@ cudaError_t launch_g(const DecodeShape& s, const CUtensorMap& tq, const CUtensor
     attr[na].val.programmaticStreamSerializationAllowed = 1;
     ++na;
   }
-  if (s.cluster) {
+  if (cluster) {
     attr[na].id = cudaLaunchAttributeClusterDimension;
     attr[na].val.clusterDim.x = (unsigned)s.splits;
     attr[na].val.clusterDim.y = 1;
@@ -626,7 +697,7 @@ cudaError_t launch_g(const DecodeShape& s, const CUtensorMap& tq, const CUtensor
   cfg.attrs = attr;
   cfg.numAttrs = na;
   e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, idx, gates, s, (__nv_bfloat16*)o, ws_ml, ws_o,
-                         ws_cnt, pa, ctx);
+                         ws_cnt, pa, sa, ctx);
   if (e == cudaSuccess) note_launches(1);
   return e;
 }
@@ -639,7 +710,7 @@ bool cluster_fits(int splits) {
   static signed char fits[17] = {};
   std::lock_guard<std::mutex> lk(mu);
   if (fits[splits] == 0) {
-    auto kern = decode_tc_kernel<G>;
+    auto kern = decode_tc_kernel<G, false>;
     bool ok = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem) ==
               cudaSuccess;
     if (ok && splits > 8)
@@ -668,8 +739,14 @@ template <int G>
 cudaError_t launch_any(DecodeShape s, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, const int32_t* idx, const float* gates, void* o,
                        float* ws_ml, float* ws_o, uint32_t* ws_cnt, const PagedArgs& pa,
-                       const DevCtx& ctx, cudaStream_t st) {
+                       const SelArgs& sa, const DevCtx& ctx, cudaStream_t st) {
   s.cluster = s.splits >= 2 && s.splits <= kMaxClusterSplits && cluster_fits<G>(s.splits);
+  if (sa.on) {
+    // The fused selection needs the unit's splits in one cluster.
+    if (!s.cluster && s.splits != 1) return cudaErrorNotSupported;
+    return launch_g<G, true>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, sa, ctx, st,
+                             true);
+  }
   if (!s.cluster && s.splits > 1) {
     // Tickets start at zero on every call, whatever the workspace held before.
     cudaError_t e = cudaMemsetAsync(ws_cnt, 0, sizeof(uint32_t) * (size_t)s.B * s.Hkv, st);
@@ -679,7 +756,8 @@ cudaError_t launch_any(DecodeShape s, const CUtensorMap& tq, const CUtensorMap& 
   // Only a kernel may precede a programmatic dependent: after the memset the
   // launch is an ordinary one.
   const bool pdl = s.cluster || s.splits == 1;
-  return launch_g<G>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, ctx, st, pdl);
+  return launch_g<G, false>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, sa, ctx, st,
+                            pdl);
 }
 
 }  // namespace
@@ -693,8 +771,8 @@ bool tc_decode_supported(sas_dtype_t dt, const DecodeShape& s) {
 namespace {
 cudaError_t launch_tc_maps(const DecodeShape& s, const CUtensorMap& tq, const CUtensorMap& tk,
                            const CUtensorMap& tv, const PagedArgs& pa, const int32_t* idx,
-                           const float* gates, void* o, void* ws, const DevCtx& ctx,
-                           cudaStream_t st) {
+                           const float* gates, void* o, void* ws, const SelArgs& sa,
+                           const DevCtx& ctx, cudaStream_t st) {
   char* w = static_cast<char*>(ws);
   const size_t parts = (size_t)s.B * s.Hq * s.splits;
   float* ws_ml = reinterpret_cast<float*>(w);
@@ -702,14 +780,22 @@ cudaError_t launch_tc_maps(const DecodeShape& s, const CUtensorMap& tq, const CU
   uint32_t* ws_cnt = reinterpret_cast<uint32_t*>(
       reinterpret_cast<char*>(ws_o) + ((parts * s.d * sizeof(float) + 255) & ~(size_t)255));
   switch (s.Hq / s.Hkv) {
-    case 1: return launch_any<1>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, ctx, st);
-    case 2: return launch_any<2>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, ctx, st);
-    case 3: return launch_any<3>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, ctx, st);
-    case 4: return launch_any<4>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, ctx, st);
-    case 5: return launch_any<5>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, ctx, st);
-    case 6: return launch_any<6>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, ctx, st);
-    case 7: return launch_any<7>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, ctx, st);
-    case 8: return launch_any<8>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, ctx, st);
+    case 1:
+      return launch_any<1>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, sa, ctx, st);
+    case 2:
+      return launch_any<2>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, sa, ctx, st);
+    case 3:
+      return launch_any<3>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, sa, ctx, st);
+    case 4:
+      return launch_any<4>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, sa, ctx, st);
+    case 5:
+      return launch_any<5>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, sa, ctx, st);
+    case 6:
+      return launch_any<6>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, sa, ctx, st);
+    case 7:
+      return launch_any<7>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, sa, ctx, st);
+    case 8:
+      return launch_any<8>(s, tq, tk, tv, idx, gates, o, ws_ml, ws_o, ws_cnt, pa, sa, ctx, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -726,7 +812,24 @@ cudaError_t launch_decode_tc(const DecodeShape& s, const void* q, const void* kc
   if ((e = make_tmap_bf16_pitched(&tk, kc, s.L, s.Lcap, s.B * s.Hkv)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16_pitched(&tv, vc, s.L, s.Lcap, s.B * s.Hkv)) != cudaSuccess) return e;
   const PagedArgs none = {nullptr, nullptr, nullptr, 0, 0};
-  return launch_tc_maps(s, tq, tk, tv, none, idx, gates, o, ws, ctx, st);
+  const SelArgs nosel = {false, nullptr, nullptr, nullptr, 0};
+  return launch_tc_maps(s, tq, tk, tv, none, idx, gates, o, ws, nosel, ctx, st);
+}
+
+cudaError_t launch_decode_select_tc(const DecodeShape& s, const void* q, const void* kc,
+                                    const void* vc, const float* scores, float* gates_out,
+                                    int32_t* idx_out, void* o, void* ws, const DevCtx& ctx,
+                                    cudaStream_t st) {
+  if (s.dense || s.paged || s.splits > kSelMaxCta || s.C > 512 * s.splits || s.K > 256)
+    return cudaErrorNotSupported;
+  CUtensorMap tq, tk, tv;
+  cudaError_t e;
+  if ((e = make_tmap_bf16_rows8(&tq, q, s.B * s.Hq)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_pitched(&tk, kc, s.L, s.Lcap, s.B * s.Hkv)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_pitched(&tv, vc, s.L, s.Lcap, s.B * s.Hkv)) != cudaSuccess) return e;
+  const PagedArgs none = {nullptr, nullptr, nullptr, 0, 0};
+  const SelArgs sa = {true, scores, gates_out, idx_out, (s.C + s.splits - 1) / s.splits};
+  return launch_tc_maps(s, tq, tk, tv, none, nullptr, nullptr, o, ws, sa, ctx, st);
 }
 
 cudaError_t launch_decode_paged_tc(const DecodeShape& s, const PagedArgs& pa, const void* q,
@@ -742,7 +845,8 @@ cudaError_t launch_decode_paged_tc(const DecodeShape& s, const PagedArgs& pa, co
     return e;
   if ((e = make_tmap_bf16_box(&tv, vpages, pa.P, pa.num_pages * s.Hkv, rows)) != cudaSuccess)
     return e;
-  return launch_tc_maps(s, tq, tk, tv, pa, idx, gates, o, ws, ctx, st);
+  const SelArgs nosel = {false, nullptr, nullptr, nullptr, 0};
+  return launch_tc_maps(s, tq, tk, tv, pa, idx, gates, o, ws, nosel, ctx, st);
 }
 
 }  // namespace sas

@@ -27,17 +27,10 @@
 
 #include "sas_common.cuh"
 #include "sas_internal.h"
+#include "topk_select.cuh"
 
 namespace sas {
 namespace {
-
-// Order-preserving map fp32 -> uint32 (larger float -> larger key); -0.0 is
-// folded onto +0.0 so that the two compare equal, as fp32 values do.
-__device__ __forceinline__ uint32_t fkey(float f) {
-  uint32_t u = __float_as_uint(f);
-  if (u == 0x80000000u) u = 0u;
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
@@ -211,13 +204,6 @@ gate_topk_warp_kernel(const float* __restrict__ scores, int total_rows, int rows
 constexpr int kMaxChunk = 8192;       // longest chunk (64 KB of keys)
 constexpr int kMaxCandidates = 8192;  // chunks x per-chunk candidates
 
-__device__ __forceinline__ uint64_t ckey(float f, int i) {
-  return ((uint64_t)fkey(f) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)i);
-}
-__device__ __forceinline__ int ckey_index(uint64_t c) {
-  return (int)(0xFFFFFFFFu - (uint32_t)(c & 0xFFFFFFFFu));
-}
-
 // Block reductions for any multiple of 32 threads up to 1024 (red: 32 floats).
 __device__ __forceinline__ float block_max(float x, float* red) {
   x = warp_max(x);
@@ -236,180 +222,9 @@ __device__ __forceinline__ float block_sum(float x, float* red) {
   return warp_sum(lane < (int)(blockDim.x >> 5) ? red[lane] : 0.f);
 }
 
-// Sorts the block's E * blockDim.x keys (a power of two) in descending
-// order with a bitonic network; thread t holds the keys at indices
-// e * blockDim.x + t in v[e]. Stages whose partners are less than 32 apart
-// exchange through warp shuffles (no barrier); the wider ones go through
-// sm (E * blockDim.x keys). On return the sorted keys are in sm.
-template <int E>
-__device__ void block_sort_desc(uint64_t (&v)[E], uint64_t* sm) {
-  const int bd = blockDim.x, tid = threadIdx.x, n = E * bd;
-  bool in_smem = false;
-  for (int k = 2; k <= n; k <<= 1)
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      if (j >= 32) {
-        if (!in_smem) {
-          __syncthreads();  // every thread has read sm into registers
-#pragma unroll
-          for (int e = 0; e < E; ++e) sm[e * bd + tid] = v[e];
-          __syncthreads();
-          in_smem = true;
-        }
-        for (int i = tid; i < n; i += bd) {
-          const int p = i ^ j;
-          if (p > i) {
-            const uint64_t a = sm[i], b = sm[p];
-            if (((i & k) == 0) ? (a < b) : (a > b)) {
-              sm[i] = b;
-              sm[p] = a;
-            }
-          }
-        }
-        __syncthreads();
-      } else {
-        if (in_smem) {
-#pragma unroll
-          for (int e = 0; e < E; ++e) v[e] = sm[e * bd + tid];
-          in_smem = false;
-        }
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          const int i = e * bd + tid;
-          const uint64_t o = __shfl_xor_sync(0xffffffffu, v[e], j);
-          // the lower index of a pair keeps the larger key in a descending run
-          const bool keep_max = ((i & j) == 0) == ((i & k) == 0);
-          v[e] = keep_max ? (v[e] > o ? v[e] : o) : (v[e] < o ? v[e] : o);
-        }
-      }
-    }
-  if (!in_smem) {
-    __syncthreads();
-#pragma unroll
-    for (int e = 0; e < E; ++e) sm[e * bd + tid] = v[e];
-  }
-  __syncthreads();
-}
-
-// Sorts one warp's 32 * EW keys in descending order in registers (lane l
-// holds indices e * 32 + l in w[e]); every lane of the warp calls it.
-template <int EW>
-__device__ __forceinline__ void warp_sort_desc(uint64_t (&w)[EW]) {
-  const int lane = threadIdx.x & 31;
-  constexpr int n = 32 * EW;
-#pragma unroll
-  for (int k = 2; k <= n; k <<= 1)
-#pragma unroll
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      if (j >= 32) {
-#pragma unroll
-        for (int e = 0; e < EW; ++e) {
-          const int pe = e ^ (j >> 5);
-          if (pe > e) {
-            const bool desc = ((e * 32 + lane) & k) == 0;
-            const uint64_t a = w[e], b = w[pe];
-            if (desc ? (a < b) : (a > b)) {
-              w[e] = b;
-              w[pe] = a;
-            }
-          }
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < EW; ++e) {
-          const int i = e * 32 + lane;
-          const uint64_t o = __shfl_xor_sync(0xffffffffu, w[e], j);
-          const bool keep_max = ((i & j) == 0) == ((i & k) == 0);
-          w[e] = keep_max ? (w[e] > o ? w[e] : o) : (w[e] < o ? w[e] : o);
-        }
-      }
-    }
-}
-
-template <int EW>
-__device__ __forceinline__ void warp_sort_cand(const uint64_t* cand, int m, uint64_t* out, int k) {
-  const int lane = threadIdx.x & 31;
-  uint64_t w[EW];
-#pragma unroll
-  for (int e = 0; e < EW; ++e) w[e] = e * 32 + lane < m ? cand[e * 32 + lane] : 0ull;
-  warp_sort_desc<EW>(w);
-#pragma unroll
-  for (int e = 0; e < EW; ++e)
-    if (e * 32 + lane < k) out[e * 32 + lane] = w[e];
-}
-
-constexpr int kBins = 4096;     // histogram over the top 12 bits of a key
-constexpr int kCandCap = 256;   // candidates sorted by one warp
-
-struct TopkScratch {
-  int hist[kBins];
-  uint64_t cand[kCandCap];
-  int warp_tot[32];
-  int ncand, bin, above;
-};
 // Static shared memory of the chunk and merge kernels (scratch + reduction),
 // counted against the 48 KB a launch gets without opting in.
 constexpr size_t kStaticSmem = sizeof(TopkScratch) + 32 * sizeof(float) + 64;
-
-// Leaves the k largest of the block's keys (v[e], E per thread; 0 = empty),
-// in descending order, in sm[0, k). Radix filter: a histogram over the top
-// 12 bits of the keys finds the bin b holding the k-th largest; every key in
-// a bin above b is in, and the rest come from bin b, so the keys in bins >= b
-// are the candidates. Up to 256 candidates are sorted by one warp; past that
-// (heavy ties) the block sorts all its keys. 1 <= k; every thread calls it.
-template <int E>
-__device__ void block_topk(uint64_t (&v)[E], int k, TopkScratch& ts, uint64_t* sm) {
-  const int tid = threadIdx.x, bd = blockDim.x, lane = tid & 31, w = tid >> 5;
-  for (int i = tid; i < kBins; i += bd) ts.hist[i] = 0;
-  if (tid == 0) {
-    ts.ncand = 0;
-    ts.bin = 0;  // always overwritten: the block holds at least k keys
-    ts.above = 0;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int e = 0; e < E; ++e)
-    if (v[e] != 0ull) atomicAdd(&ts.hist[(int)(v[e] >> 52)], 1);
-  __syncthreads();
-  // Suffix counts: thread t owns bins [t W, t W + W).
-  const int W = kBins / bd, b0 = tid * W;
-  int local = 0;
-  for (int x = 0; x < W; ++x) local += ts.hist[b0 + x];
-  int suf = local;  // over this warp's lanes >= lane
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int y = __shfl_down_sync(0xffffffffu, suf, off);
-    if (lane + off < 32) suf += y;
-  }
-  if (lane == 0) ts.warp_tot[w] = suf;
-  __syncthreads();
-  int running = suf - local;
-  for (int x = w + 1; x < (bd >> 5); ++x) running += ts.warp_tot[x];
-  for (int x = W - 1; x >= 0; --x) {
-    const int h = ts.hist[b0 + x];
-    if (running < k && running + h >= k) {
-      ts.bin = b0 + x;
-      ts.above = running;
-    }
-    running += h;
-  }
-  __syncthreads();
-  const int b = ts.bin, m = ts.above + ts.hist[b];
-  if (m <= kCandCap) {
-#pragma unroll
-    for (int e = 0; e < E; ++e)
-      if (v[e] != 0ull && (int)(v[e] >> 52) >= b) ts.cand[atomicAdd(&ts.ncand, 1)] = v[e];
-    __syncthreads();
-    if (w == 0) {
-      if (m <= 32) warp_sort_cand<1>(ts.cand, m, sm, k);
-      else if (m <= 64) warp_sort_cand<2>(ts.cand, m, sm, k);
-      else if (m <= 128) warp_sort_cand<4>(ts.cand, m, sm, k);
-      else warp_sort_cand<8>(ts.cand, m, sm, k);
-    }
-    __syncthreads();
-  } else {
-    block_sort_desc<E>(v, sm);
-  }
-}
 
 // Writes g = exp(s - lse) for i < n and 0 past n, over [0, C) of one row
 // (float4 accesses when both rows are 16-byte aligned).
@@ -540,153 +355,21 @@ gate_topk_merge_kernel(const float* __restrict__ scores, int rows, int C, int ca
 // ---------------------------------------------------------------------------
 // Decode-sized rows (513 .. 8192 entries): a thread-block cluster of CS CTAs
 // per row, CTA r holding the 512 entries [512 r, 512 r + 512), two per
-// thread. Selection without sorting the row:
-//  1. each CTA's (max, min, sum of exp) are read by every CTA of the cluster
-//     through distributed shared memory (one round trip, lane x reading rank
-//     x); every CTA forms the row's max M and LSE alike;
-//  2. each CTA histograms its chunk over 64 buckets of (M - s) in steps of
-//     1/8 (bucket 63: everything further down, never counted: its count is
-//     the rest of the row) and adds the histogram into every CTA's copy of
-//     the row's histogram (remote reductions, no round trip); after a
-//     cluster barrier each CTA finds b*, the bucket holding the k-th largest
-//     score, in its own copy. When that is bucket 63, a second histogram
-//     spreads [min, M - 63/8] over 64 buckets the same way;
-//  3. every score in a bucket up to b* is a candidate -- a superset of the
-//     top k, usually a few more than k. Each warp reserves room in rank 0's
-//     list with one remote atomic and stores its candidates there; rank 0
-//     places each by its rank among them under the composite order
-//     (descending score, ties to the lower index), which is its rank in the
-//     row.
-// More than 1024 candidates (mass ties, known from the histogram) switch the
-// cluster to an exact path: each CTA selects its chunk's best k and stores
-// them in rank 0's list, which rank 0 places by rank. The gates are written
-// last, so that no cluster barrier waits for those stores.
+// thread, selects the row with cluster_select (bucket histograms exchanged
+// over distributed shared memory; candidates placed by rank at rank 0). The
+// gates are written last, so that no cluster barrier waits for those stores.
 // ---------------------------------------------------------------------------
 constexpr int kCbThreads = 256;
-constexpr int kCbChunk = 512;   // entries per CTA
-constexpr int kCbMaxCta = 16;   // rows up to 8192 entries
-constexpr int kCbCand = 1024;   // candidates rank 0 places by rank
-constexpr int kNB = 64;         // buckets per histogram level
-constexpr float kBkStep = 8.f;  // level-1 buckets per unit of score below the max
-
-struct CbShared {
-  float part[3];                  // this chunk's max, min, sum of exp (relative to its max)
-  int hist[kNB];                  // this chunk's histogram
-  unsigned int row_hist[2][kNB];  // the row's, levels 1 and 2 (the cluster adds into it)
-  unsigned int nlist;             // rank 0: keys in its list
-  uint64_t best[kCbChunk];        // the exact path: this chunk's best, sorted
-  float red[2][8];
-  int wsum[8];
-  float M, Mn, lse;
-  int bstar, before, upto;
-  TopkScratch ts;  // the exact path
-};
-
-__device__ __forceinline__ float fast_gate(float sc, float lse, int phi) {
-  if (phi == SAS_PHI_SIGMOID) return 1.f / (1.f + __expf(-sc));
-  if (phi == SAS_PHI_RAW) return __expf(sc);
-  return __expf(sc - lse);
-}
-
-// Finds, in the row histogram h, the bucket holding the target-th entry in
-// bucket order (warp 0; lane l sums buckets 2l and 2l + 1). `rest` >= 0
-// gives the last bucket the count `rest` minus the other buckets' total (a
-// bucket no CTA counts). Returns the bucket; *before / *upto = entries in
-// the buckets before it / up to and including it. Every thread calls it;
-// the result is the same in every CTA.
-__device__ int find_bucket(const unsigned int* h, int target, int rest, CbShared& sh, int* before,
-                           int* upto) {
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    const int c0 = (int)h[2 * lane];
-    int c1 = (rest >= 0 && lane == 31) ? 0 : (int)h[2 * lane + 1];
-    int inc = c0 + c1;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += y;
-    }
-    const int tot = __shfl_sync(0xffffffffu, inc, 31);
-    if (rest >= 0 && lane == 31) {  // the uncounted bucket takes the rest
-      c1 = rest - tot;
-      inc = rest;
-    }
-    const int ex = inc - c0 - c1;  // entries before bucket 2 lane
-    if (ex < target && ex + c0 >= target) {
-      sh.bstar = 2 * lane;
-      sh.before = ex;
-      sh.upto = ex + c0;
-    } else if (ex + c0 < target && inc >= target) {
-      sh.bstar = 2 * lane + 1;
-      sh.before = ex + c0;
-      sh.upto = inc;
-    }
-  }
-  __syncthreads();
-  *before = sh.before;
-  *upto = sh.upto;
-  return sh.bstar;  // rewritten only after a later barrier
-}
-
-// Adds this CTA's histogram (sh.hist) into the row histogram `dst` of every
-// CTA of the cluster (thread t: bucket t % 64 into ranks t / 64, t / 64 + 4,
-// ...), then clears sh.hist.
-__device__ __forceinline__ void push_hist(CbShared& sh, unsigned int* dst, int CS) {
-  const int tid = threadIdx.x, bkt = tid & (kNB - 1);
-  __syncthreads();  // the local histogram is complete
-  const unsigned int v = (unsigned int)sh.hist[bkt];
-  if (v)
-    for (int x = tid / kNB; x < CS; x += kCbThreads / kNB)
-      dsmem_red_add_u32(dsmem_addr(&dst[bkt], (uint32_t)x), v);
-  __syncthreads();  // read before cleared
-  if (tid < kNB) sh.hist[tid] = 0;
-}
-
-// Places keys[0, m) by rank (keys equal to 0 are empty slots): out[rank] =
-// index for the kk best. Short lists: a group of tpc threads per key splits
-// the comparisons; long lists: four keys per thread, one pass over the list.
-__device__ __forceinline__ void place_by_rank(const uint64_t* keys, int m, int kk, int32_t* out) {
-  const int tid = threadIdx.x;
-  if (m <= kCbThreads) {
-    int tpc = 1;
-    while (tpc < 8 && 2 * tpc * m <= kCbThreads) tpc *= 2;
-    const int p = tid / tpc, part = tid % tpc;
-    const uint64_t mine = p < m ? keys[p] : 0ull;
-    int rk = 0;
-#pragma unroll 4
-    for (int q = part; q < m; q += tpc) rk += keys[q] > mine;
-    for (int o = 1; o < tpc; o <<= 1) rk += __shfl_xor_sync(0xffffffffu, rk, o);
-    if (part == 0 && mine != 0ull && rk < kk) out[rk] = ckey_index(mine);
-    return;
-  }
-  for (int p0 = tid; p0 < m; p0 += 4 * kCbThreads) {
-    uint64_t mine[4];
-    int rk[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int p = p0 + u * kCbThreads;
-      mine[u] = p < m ? keys[p] : 0ull;
-      rk[u] = 0;
-    }
-    for (int q = 0; q < m; ++q) {
-      const uint64_t y = keys[q];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) rk[u] += y > mine[u];
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (mine[u] != 0ull && rk[u] < kk) out[rk[u]] = ckey_index(mine[u]);
-  }
-}
+constexpr int kCbChunk = 512;  // entries per CTA
 
 __global__ void __launch_bounds__(kCbThreads)
 gate_topk_cbucket_kernel(const float* __restrict__ scores, int rows, int C, int causal, int K,
                          int CS, int phi, float* __restrict__ gates, int32_t* __restrict__ idx) {
   // rank 0's list: the candidates, or CS chunks' best kk on the exact path
   extern __shared__ uint64_t s_list[];
-  __shared__ CbShared sh;
+  __shared__ SelShared sh;
   grid_launch_dependents();  // a dependent decode may start its prologue
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const uint32_t rank = cluster_rank();
   const long long row = blockIdx.x / CS;
   const int r = (int)(row % rows);
@@ -705,142 +388,21 @@ gate_topk_cbucket_kernel(const float* __restrict__ scores, int rows, int C, int 
       for (int p = tid; p < K; p += kCbThreads) out[p] = -1;
     return;
   }
-
   float f[2];
   bool ok[2];
-  float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     const int i = lo + tid + kCbThreads * e;
     ok[e] = i < n;
     f[e] = ok[e] ? srow[i] : -INFINITY;
-    if (ok[e]) {
-      mx = fmaxf(mx, f[e]);
-      mn = fminf(mn, f[e]);
-    }
   }
-  mx = warp_max(mx);
-  mn = -warp_max(-mn);
-  if (lane == 0) {
-    sh.red[0][warp] = mx;
-    sh.red[1][warp] = mn;
-  }
-  if (tid < kNB) {
-    sh.hist[tid] = 0;
-    sh.row_hist[0][tid] = 0u;
-    sh.row_hist[1][tid] = 0u;
-  }
-  if (tid == 0) sh.nlist = 0u;
-  __syncthreads();
-  float cm = -INFINITY, cmn = INFINITY;
-#pragma unroll
-  for (int x = 0; x < 8; ++x) {
-    cm = fmaxf(cm, sh.red[0][x]);
-    cmn = fminf(cmn, sh.red[1][x]);
-  }
-  float sum = 0.f;
-#pragma unroll
-  for (int e = 0; e < 2; ++e)
-    if (ok[e]) sum += __expf(f[e] - cm);
-  sum = warp_sum(sum);
-  if (lane == 0) sh.wsum[warp] = __float_as_int(sum);
-  __syncthreads();
-  if (tid == 0) {
-    float t = 0.f;
-#pragma unroll
-    for (int x = 0; x < 8; ++x) t += __int_as_float(sh.wsum[x]);
-    sh.part[0] = cm;
-    sh.part[1] = cmn;
-    sh.part[2] = t;
-  }
-  // (1) the partials are written and every CTA's row histograms and list
-  // counter are cleared before anyone adds into them
-  cluster_sync_all();
-
-  if (warp == 0) {
-    float pm = -INFINITY, pmn = INFINITY, ps = 0.f;
-    if (lane < CS) {
-      pm = dsmem_ld_f32(dsmem_addr(&sh.part[0], (uint32_t)lane));
-      pmn = dsmem_ld_f32(dsmem_addr(&sh.part[1], (uint32_t)lane));
-      ps = dsmem_ld_f32(dsmem_addr(&sh.part[2], (uint32_t)lane));
-    }
-    const float M = warp_max(pm);
-    const float Mn = -warp_max(-pmn);
-    const float S = warp_sum(ps > 0.f ? ps * __expf(pm - M) : 0.f);
-    if (lane == 0) {
-      sh.M = M;
-      sh.Mn = Mn;
-      sh.lse = M + __logf(S);
-    }
-  }
-  __syncthreads();
-  const float M = sh.M, Mn = sh.Mn;
-
-  // ---- level 1: 1/8-wide buckets below the max; the last is never counted
-  auto b1_of = [&](float x) -> int { return (int)fminf((M - x) * kBkStep, (float)(kNB - 1)); };
-#pragma unroll
-  for (int e = 0; e < 2; ++e)
-    if (ok[e]) {
-      const int bb = b1_of(f[e]);
-      if (bb < kNB - 1) atomicAdd(&sh.hist[bb], 1);
-    }
-  push_hist(sh, sh.row_hist[0], CS);
-  cluster_sync_all();  // (2) the row histogram is complete in every CTA
-  int before, upto;
-  const int b1 = find_bucket(sh.row_hist[0], kk, n, sh, &before, &upto);
-
-  // ---- level 2 (rare: the k-th score lies 63/8 or more below the max):
-  // 64 buckets spread over [Mn, M - 63/8]
-  const float top2 = M - (float)(kNB - 1) / kBkStep;
-  const float inv2 = top2 > Mn ? (float)(kNB - 1) / (top2 - Mn) : 0.f;
-  auto b2_of = [&](float x) -> int {
-    return (int)fminf(fmaxf((top2 - x) * inv2, 0.f), (float)(kNB - 1));
-  };
-  int b2 = kNB - 1;
-  int ncand = upto;
-  if (b1 == kNB - 1) {
-#pragma unroll
-    for (int e = 0; e < 2; ++e)
-      if (ok[e] && b1_of(f[e]) == kNB - 1) atomicAdd(&sh.hist[b2_of(f[e])], 1);
-    push_hist(sh, sh.row_hist[1], CS);
-    cluster_sync_all();  // (2b)
-    int before2, upto2;
-    b2 = find_bucket(sh.row_hist[1], kk - before, -1, sh, &before2, &upto2);
-    ncand = before + upto2;
-  }
-
-  const uint32_t list0 = dsmem_addr(s_list, 0u), nlist0 = dsmem_addr(&sh.nlist, 0u);
-  const bool exact = ncand > kCbCand;
-  if (!exact) {
-    // ---- this chunk's candidates into rank 0's list
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int bb = ok[e] ? b1_of(f[e]) : kNB;
-      const bool take = bb < b1 || (bb == b1 && (b1 < kNB - 1 || b2_of(f[e]) <= b2));
-      const uint32_t mask = __ballot_sync(0xffffffffu, take);
-      if (mask == 0u) continue;
-      uint32_t slot = 0u;
-      if (lane == 0) slot = dsmem_atom_add_u32(nlist0, (uint32_t)__popc(mask));
-      slot = __shfl_sync(0xffffffffu, slot, 0) + (uint32_t)__popc(mask & ((1u << lane) - 1u));
-      if (take) dsmem_st_u64(list0 + 8u * slot, ckey(f[e], lo + tid + kCbThreads * e));
-    }
-  } else {
-    // ---- exact path (mass ties): each chunk's best kk into rank 0's list,
-    // at rank * kk (empty slots 0)
-    const int len = max(0, min(n - lo, kCbChunk));
-    const int kc = min(kk, len);
-    uint64_t v[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) v[e] = ok[e] ? ckey(f[e], lo + tid + kCbThreads * e) : 0ull;
-    if (kc > 0) block_topk<2>(v, kc, sh.ts, sh.best);  // the best kc, sorted, in sh.best
-    for (int p = tid; p < kk; p += kCbThreads)
-      dsmem_st_u64(list0 + 8u * (uint32_t)(rank * kk + p), p < kc ? sh.best[p] : 0ull);
-  }
-  cluster_sync_all();  // (3) rank 0 holds the list; no CTA touches another's memory after this
+  const int m = cluster_select<kCbThreads, 2>(f, ok, lo, kCbChunk, n, kk, CS, sh, s_list);
   if (rank == 0) {
-    place_by_rank(s_list, exact ? CS * kk : (int)sh.nlist, kk, out);
+    place_by_rank<kCbThreads>(s_list, m, kk,
+                              [&](int rk, uint64_t key) { out[rk] = ckey_index(key); });
     for (int p = kk + tid; p < K; p += kCbThreads) out[p] = -1;
   }
+  // The gates go last, so that no cluster barrier waits for these stores.
   const float lse = sh.lse;
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
@@ -976,11 +538,11 @@ int pow2_at_least(int x) {
 // when the device holds such a cluster; false leaves the row to other paths.
 bool launch_cbucket_topk(const float* scores, long long total, int rows, int C, int causal, int K,
                          int phi, float* gates, int32_t* idx, cudaStream_t stream) {
-  if (C > kCbMaxCta * kCbChunk || total * kCbMaxCta > 0x7fffffffLL) return false;
+  if (C > kSelMaxCta * kCbChunk || total * kSelMaxCta > 0x7fffffffLL) return false;
   const int CS = (C + kCbChunk - 1) / kCbChunk;
   if (CS < 2) return false;
   // rank 0's gather buffer: the bucket path's candidates, or the exact path's CS * K
-  const size_t smem = (size_t)max(kCbCand, CS * K) * sizeof(uint64_t);
+  const size_t smem = (size_t)max(kSelCand, CS * K) * sizeof(uint64_t);
   auto kern = gate_topk_cbucket_kernel;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(total * CS));
@@ -995,12 +557,12 @@ bool launch_cbucket_topk(const float* scores, long long total, int rows, int C, 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   static std::mutex mu;
-  static signed char fits[kCbMaxCta + 1] = {};
+  static signed char fits[kSelMaxCta + 1] = {};
   {
     std::lock_guard<std::mutex> lk(mu);
     if (fits[CS] == 0) {
       bool ok = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)(kCbMaxCta * 256 * sizeof(uint64_t))) == cudaSuccess;
+                                     (int)(kSelMaxCta * 256 * sizeof(uint64_t))) == cudaSuccess;
       if (ok && CS > 8)
         ok = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
              cudaSuccess;

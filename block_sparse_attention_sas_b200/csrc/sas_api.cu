@@ -343,6 +343,57 @@ sas_status_t sas_decode(sas_dtype_t dtype, const void* q, const void* kcache, co
   return cuda_status(launch_decode(dtype, s, q, kcache, vcache, idx, gates, o, ws, ctx, stream));
 }
 
+// Workspace of sas_decode_select: the decode's, then room for the gates and
+// the Top-K indices when the caller does not keep them and the selection
+// runs as its own launch.
+static size_t select_ws_parts(const DecodeShape& s, size_t* off_g, size_t* off_i) {
+  const size_t a = (decode_workspace_bytes(s) + 255) & ~(size_t)255;
+  const size_t g = ((size_t)s.B * s.Hkv * s.C * sizeof(float) + 255) & ~(size_t)255;
+  const size_t i = ((size_t)s.B * s.Hkv * s.K * sizeof(int32_t) + 255) & ~(size_t)255;
+  *off_g = a;
+  *off_i = a + g;
+  return a + g + i;
+}
+
+size_t sas_decode_select_workspace_size(int B, int Hq, int Hkv, int L, int d, int b, int K) {
+  if (check_decode(SAS_BF16, B, Hq, Hkv, L, L, d, b, K, false, 1.f) != SAS_OK) return 0;
+  size_t og, oi;
+  return select_ws_parts(make_decode(B, Hq, Hkv, L, L, d, b, K, 1.f, false, 0), &og, &oi);
+}
+
+sas_status_t sas_decode_select(sas_dtype_t dtype, const void* q, const void* kcache,
+                               const void* vcache, const float* scores, int use_gates, int B,
+                               int Hq, int Hkv, int L, int Lcap, int d, int b, int K, float scale,
+                               void* o, float* gates, int32_t* idx, void* ws, size_t ws_bytes,
+                               sas_stream_t stream) {
+  sas_status_t st = check_decode(dtype, B, Hq, Hkv, L, Lcap, d, b, K, false, scale);
+  if (st != SAS_OK) return st;
+  if (B == 0) return SAS_OK;
+  const int C = (L - 1) / b;
+  if (!q || !kcache || !vcache || !o || (!scores && C > 0)) return SAS_ERR_INVALID_ARG;
+  if (C > 262144) return SAS_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(kcache, 16) || !aligned(vcache, 16) || !aligned(o, 16) ||
+      (scores && !aligned(scores, 4)) || (gates && !aligned(gates, 4)) || (idx && !aligned(idx, 4)))
+    return SAS_ERR_INVALID_ARG;
+  const DecodeShape s = make_decode(B, Hq, Hkv, L, Lcap, d, b, K, scale, false, use_gates);
+  size_t og, oi;
+  const size_t need = select_ws_parts(s, &og, &oi);
+  if (!ws || ws_bytes < need || !aligned(ws, 256)) return SAS_ERR_WORKSPACE;
+  DevCtx ctx;
+  if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
+  if (tc_decode_supported(dtype, s)) {
+    const cudaError_t e =
+        launch_decode_select_tc(s, q, kcache, vcache, scores, gates, idx, o, ws, ctx, stream);
+    if (e != cudaErrorNotSupported) return cuda_status(e);
+  }
+  // Two launches: the gates and Top-K of the rows, then the decode.
+  float* g = gates ? gates : reinterpret_cast<float*>(static_cast<char*>(ws) + og);
+  int32_t* ix = idx ? idx : reinterpret_cast<int32_t*>(static_cast<char*>(ws) + oi);
+  cudaError_t e = launch_gate_topk(scores, B, Hkv, 1, C, 0, K, SAS_PHI_SOFTMAX, g, ix, stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  return cuda_status(launch_decode(dtype, s, q, kcache, vcache, ix, g, o, ws, ctx, stream));
+}
+
 sas_status_t sas_decode_noalloc(sas_dtype_t dtype, const void* q, const void* kcache,
                                 const void* vcache, const int32_t* idx, const float* gates,
                                 int use_gates, int B, int Hq, int Hkv, int L, int Lcap, int d,

@@ -100,6 +100,14 @@ cudaError_t launch_decode(sas_dtype_t dt, const DecodeShape& s, const void* q, c
 
 // Tensor-core (tcgen05) decode: bf16 cache, d = 128, b = 64, G <= 8.
 bool tc_decode_supported(sas_dtype_t dt, const DecodeShape& s);
+// The tensor-core decode with the gates and Top-K of the unit's selector
+// scores [B * Hkv][C] computed in the same launch (softmax gates); gates_out /
+// idx_out may be null. cudaErrorNotSupported when the shape does not allow
+// it (a unit's row must fit its splits' cluster, 512 entries a split).
+cudaError_t launch_decode_select_tc(const DecodeShape& s, const void* q, const void* kc,
+                                    const void* vc, const float* scores, float* gates_out,
+                                    int32_t* idx_out, void* o, void* ws, const DevCtx& ctx,
+                                    cudaStream_t st);
 cudaError_t launch_decode_tc(const DecodeShape& s, const void* q, const void* kc, const void* vc,
                              const int32_t* idx, const float* gates, void* o, void* ws,
                              const DevCtx& ctx, cudaStream_t stream);

@@ -240,6 +240,35 @@ sas_status_t sas_decode(sas_dtype_t dtype, const void* q, const void* kcache, co
                         void* ws, size_t ws_bytes, sas_stream_t stream);
 
 /*
+ * sas_decode_select - one decode step from the selector scores: the gates
+ * and Top-K of each (batch, KV head) row of history blocks, then sas_decode
+ * with them ([picx] Methodology Eq. 4-6 and Eq. 9; the selection the
+ * evolve.pub review's Summary keeps at inference). Equal to sas_gate_topk on
+ * scores viewed as [B][Hkv][1][C] (causal = 0, softmax gates) followed by
+ * sas_decode with its idx and gates.
+ *   scores   [B][Hkv][C] fp32, C = (L - 1) / b (may be NULL when C == 0).
+ *   gates    [B][Hkv][C] fp32 output, or NULL (not stored).
+ *   idx      [B][Hkv][K] int32 output, or NULL (not stored).
+ *   The other arguments are those of sas_decode. ws: at least
+ *   sas_decode_select_workspace_size(B, Hq, Hkv, L, d, b, K) bytes, 256-byte
+ *   aligned, owned by the caller, free once the call's work on `stream` is
+ *   done.
+ * With the tensor-core decode (bf16, d = 128, b = 64, G <= 8) and each row
+ * short enough for its splits (C <= 512 x splits, splits <= 16), the
+ * selection runs in the decode's own launch: the splits of a (batch, KV head)
+ * form one thread-block cluster that selects the row, and each split then
+ * streams its share of the selected blocks. Otherwise it is two launches.
+ * Errors: those of sas_gate_topk and sas_decode; a bad argument is reported
+ * before any launch.
+ */
+size_t sas_decode_select_workspace_size(int B, int Hq, int Hkv, int L, int d, int b, int K);
+sas_status_t sas_decode_select(sas_dtype_t dtype, const void* q, const void* kcache,
+                               const void* vcache, const float* scores, int use_gates, int B,
+                               int Hq, int Hkv, int L, int Lcap, int d, int b, int K, float scale,
+                               void* o, float* gates, int32_t* idx, void* ws, size_t ws_bytes,
+                               sas_stream_t stream);
+
+/*
  * sas_decode_noalloc - sas_decode for callers that cannot allocate device
  * memory. Some callers cannot call cudaMalloc or take a workspace from their
  * framework at the point where they decode: an inference server or plugin

@@ -1,0 +1,71 @@
+"""GPU parity of sas_decode_select (the gates and Top-K of the selector
+scores, then the decode, in one call) against the float64 oracle: the same
+Top-K indices and gates as the oracle's gate_topk, and its decode of the
+selected blocks. Tensor-core shapes run the selection inside the decode's
+own launch (a cluster of the unit's splits); the others take two launches.
+"""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_sas_b200 import workloads as W
+from oracle import sas_oracle as O
+from tests.parity_util import check, dev, host
+
+pytestmark = pytest.mark.gpu
+
+
+def _select_case(lib, dc, use_gates, scores=None):
+    x = W.make_decode_inputs(dc)
+    s = x.scores if scores is None else scores
+    q, kc, vc = (dev(a, dc.dtype) for a in (x.q, x.kcache, x.vcache))
+    g = torch.full((dc.B, dc.Hkv, dc.C), float("nan"), device="cuda")
+    ix = torch.full((dc.B, dc.Hkv, dc.K), -7, dtype=torch.int32, device="cuda")
+    sd = dev(s, "f32")
+    lib.device_error()
+    o = lib.decode_select(q, kc, vc, sd, dc.K, use_gates, dc.b, L=dc.L, gates=g, idx=ix)
+    o2 = lib.decode_select(q, kc, vc, sd, dc.K, use_gates, dc.b, L=dc.L)
+    torch.cuda.synchronize()
+    assert lib.device_error()[0] == 0
+    og, olg, oi = O.gate_topk(s[:, :, None, :], dc.K, causal=False)
+    np.testing.assert_array_equal(ix.cpu().numpy(), oi[:, :, 0])
+    check("gates", host(g), og[:, :, 0], "f32")
+    want = O.decode(x.q, x.kcache, x.vcache, oi[:, :, 0], olg[:, :, 0], dc.b, use_gates=use_gates)
+    check("decode_select o", host(o), want, dc.dtype)
+    # the optional outputs change nothing in o
+    assert torch.equal(o, o2)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(B=2, Hq=8, Hkv=2, L=5000, d=128, b=64, K=16, dtype="bf16"),    # G = 4, 9 splits
+    dict(B=1, Hq=10, Hkv=2, L=20000, d=128, b=64, K=64, dtype="bf16"),  # G = 5, 13 splits
+    dict(B=3, Hq=24, Hkv=3, L=40000, d=128, b=64, K=32, dtype="bf16"),  # G = 8
+    dict(B=2, Hq=4, Hkv=2, L=300, d=128, b=64, K=8, dtype="bf16"),      # K > C
+    dict(B=1, Hq=8, Hkv=1, L=64, d=128, b=64, K=2, dtype="bf16"),       # no history
+    dict(B=1, Hq=2, Hkv=1, L=3000, d=128, b=64, K=256, dtype="bf16"),   # K = 256
+    dict(B=2, Hq=4, Hkv=2, L=1000, d=128, b=64, K=4, dtype="f32"),      # two launches
+    dict(B=3, Hq=5, Hkv=1, L=777, d=64, b=16, K=9, dtype="bf16"),       # two launches
+])
+@pytest.mark.parametrize("use_gates", [False, True])
+def test_decode_select_small(cuda_lib, kw, use_gates):
+    _select_case(cuda_lib, W.small_decode_config(**kw), use_gates)
+
+
+@pytest.mark.parametrize("C,levels", [(1000, 1), (3000, 1), (3000, 2), (2500, 0)])
+def test_decode_select_ties_and_spread(cuda_lib, C, levels):
+    """Mass ties (every score equal: the long placement, and past 1024
+    candidates the per-chunk exact path), two levels, and a wide spread
+    (the k-th score more than 63/8 below the max: the second histogram)."""
+    dc = W.small_decode_config(B=1, Hq=4, Hkv=1, L=C * 64 + 1, d=128, b=64, K=32, dtype="bf16")
+    rng = np.random.default_rng(C + levels)
+    if levels:
+        s = rng.integers(0, levels, (1, 1, C)).astype(np.float32)
+    else:
+        s = (rng.standard_normal((1, 1, C)) * 40.0).astype(np.float32)
+    _select_case(cuda_lib, dc, True, scores=s)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,use_gates", [("qwen3-4b-decode", 1), ("qwen3-14b-decode", 0)])
+def test_decode_select_full_size(cuda_lib, name, use_gates):
+    _select_case(cuda_lib, W.PRESETS[name], bool(use_gates))
