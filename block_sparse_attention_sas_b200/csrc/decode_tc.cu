@@ -90,8 +90,7 @@ struct Ctl {
   int last;
   int Lseq;  // tokens of this unit's sequence
   // Running max (log2 domain) and sum of this split's partial per head.
-  float part_m[kMaxG], part_l[kMaxG];
-  float mw[16], ml[16];  // the cluster's (max, sum) of the head being merged
+  float2 part_ml[kMaxG];  // (max, sum) per head
 };
 constexpr size_t kSmem = kOffCtl + sizeof(Ctl) + 1024;
 static_assert(kOffCtl % 16 == 0 && offsetof(Ctl, part_o) % 16 == 0 && (kD * 4) % 16 == 0,
@@ -542,34 +541,38 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
       for (int q4 = 0; q4 < kD / 4; ++q4)
         dst[q4] = make_float4(acc[4 * q4], acc[4 * q4 + 1], acc[4 * q4 + 2], acc[4 * q4 + 3]);
-      c.part_m[lane] = good ? m_run : -INFINITY;
-      c.part_l[lane] = good ? l_run : 0.f;
+      c.part_ml[lane] = good ? make_float2(m_run, l_run) : make_float2(-INFINITY, 0.f);
     }
     cluster_sync_all();
     const int P = s.splits;
     for (int g = split; g < G; g += P) {
-      // (max, sum) of every split for head g, then the weighted sum of the
-      // partial o rows; thread t owns columns 4t .. 4t + 3 (t < 32).
-      if (tid < P) {
-        c.mw[tid] = dsmem_ld_f32(dsmem_addr(&c.part_m[g], (uint32_t)tid));
-        c.ml[tid] = dsmem_ld_f32(dsmem_addr(&c.part_l[g], (uint32_t)tid));
-      }
-      __syncthreads();
-      float M = -INFINITY;
-      for (int x = 0; x < P; ++x) M = fmaxf(M, c.mw[x]);
-      float Lsum = 0.f;
-      for (int x = 0; x < P; ++x)
-        if (c.mw[x] != -INFINITY) Lsum += ex2(c.mw[x] - M) * c.ml[x];
+      // Thread t (t < 32) owns columns 4t .. 4t + 3 of head g: it issues the
+      // loads of every split's (max, sum) and partial columns at once (one
+      // round trip through distributed shared memory), then merges them.
       if (tid < kD / 4) {
+        float2 ml[kMaxClusterSplits];
+        float4 v[kMaxClusterSplits];
+#pragma unroll
+        for (int x = 0; x < kMaxClusterSplits; ++x)
+          if (x < P) {
+            ml[x] = dsmem_ld_f32x2(dsmem_addr(&c.part_ml[g], (uint32_t)x));
+            v[x] = dsmem_ld_f32x4(dsmem_addr(&c.part_o[g][4 * tid], (uint32_t)x));
+          }
+        float M = -INFINITY;
+#pragma unroll
+        for (int x = 0; x < kMaxClusterSplits; ++x)
+          if (x < P) M = fmaxf(M, ml[x].x);
+        float Lsum = 0.f;
         float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int x = 0; x < P; ++x) {
-          if (c.mw[x] == -INFINITY) continue;
-          const float f = ex2(c.mw[x] - M);
-          const float4 v = dsmem_ld_f32x4(dsmem_addr(&c.part_o[g][4 * tid], (uint32_t)x));
-          a.x = fmaf(f, v.x, a.x);
-          a.y = fmaf(f, v.y, a.y);
-          a.z = fmaf(f, v.z, a.z);
-          a.w = fmaf(f, v.w, a.w);
+#pragma unroll
+        for (int x = 0; x < kMaxClusterSplits; ++x) {
+          if (x >= P || ml[x].x == -INFINITY) continue;
+          const float f = ex2(ml[x].x - M);
+          Lsum = fmaf(f, ml[x].y, Lsum);
+          a.x = fmaf(f, v[x].x, a.x);
+          a.y = fmaf(f, v[x].y, a.y);
+          a.z = fmaf(f, v[x].z, a.z);
+          a.w = fmaf(f, v[x].w, a.w);
         }
         const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
         uint2 pk;
@@ -577,7 +580,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         pk.y = pack_bf16(a.z * inv, a.w * inv);
         *reinterpret_cast<uint2*>(o + (hbase + g) * kD + 4 * tid) = pk;
       }
-      __syncthreads();
     }
     // Every rank's shared memory stays alive until all reads above are done.
     cluster_sync_all();
@@ -816,12 +818,16 @@ cudaError_t launch_decode_tc(const DecodeShape& s, const void* q, const void* kc
   return launch_tc_maps(s, tq, tk, tv, none, idx, gates, o, ws, nosel, ctx, st);
 }
 
-cudaError_t launch_decode_select_tc(const DecodeShape& s, const void* q, const void* kc,
+cudaError_t launch_decode_select_tc(const DecodeShape& s0, const void* q, const void* kc,
                                     const void* vc, const float* scores, float* gates_out,
                                     int32_t* idx_out, void* o, void* ws, const DevCtx& ctx,
                                     cudaStream_t st) {
-  if (s.dense || s.paged || s.splits > kSelMaxCta || s.C > 512 * s.splits || s.K > 256)
-    return cudaErrorNotSupported;
+  // A row longer than 512 entries a split widens the cluster: the extra
+  // CTAs (slot ranges past the last slot) help select and stream nothing.
+  DecodeShape s = s0;
+  const int need = (s.C + 511) / 512;
+  if (need > s.splits) s.splits = need;
+  if (s.dense || s.paged || s.splits > kSelMaxCta || s.K > 256) return cudaErrorNotSupported;
   CUtensorMap tq, tk, tv;
   cudaError_t e;
   if ((e = make_tmap_bf16_rows8(&tq, q, s.B * s.Hq)) != cudaSuccess) return e;

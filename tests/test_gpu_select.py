@@ -43,6 +43,7 @@ def _select_case(lib, dc, use_gates, scores=None):
     dict(B=2, Hq=4, Hkv=2, L=300, d=128, b=64, K=8, dtype="bf16"),      # K > C
     dict(B=1, Hq=8, Hkv=1, L=64, d=128, b=64, K=2, dtype="bf16"),       # no history
     dict(B=1, Hq=2, Hkv=1, L=3000, d=128, b=64, K=256, dtype="bf16"),   # K = 256
+    dict(B=1, Hq=4, Hkv=1, L=70401, d=128, b=64, K=1, dtype="bf16"),    # row wider than its splits
     dict(B=2, Hq=4, Hkv=2, L=1000, d=128, b=64, K=4, dtype="f32"),      # two launches
     dict(B=3, Hq=5, Hkv=1, L=777, d=64, b=16, K=9, dtype="bf16"),       # two launches
 ])
