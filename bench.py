@@ -447,7 +447,6 @@ def run_e2e(S, torch, dev, h, d, step, args, world, flops):
     outs = None
     in_ev = [torch.cuda.Event() for _ in range(2)]
     done_ev = [torch.cuda.Event() for _ in range(2)]
-    back_ev = [torch.cuda.Event() for _ in range(2)]
     names = ("o", "dq", "dk", "dv", "dscores")
     K = args.steps
     h2d = sum(t.numel() * t.element_size() for t in h.values())
@@ -471,12 +470,12 @@ def run_e2e(S, torch, dev, h, d, step, args, world, flops):
             if outs is None:
                 outs = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in res]
                         for _ in range(2)]
-            if i >= 2:
-                back_ev[b].synchronize()  # the host has the results of step i - 2
+            # outs[b] was last written by the copy-out of step i - 2, earlier
+            # on this same stream: no host wait, so the host keeps queueing
+            # the next step's copy-in while this copy-out runs.
             for dst, src in zip(outs[b], res):
                 dst.copy_(src, non_blocking=True)
                 src.record_stream(s_out)
-            back_ev[b].record(s_out)
 
     for i in range(2):
         one(i)

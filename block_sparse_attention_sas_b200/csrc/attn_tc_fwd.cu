@@ -55,7 +55,7 @@ constexpr int kMaxList = 257;                        // K <= 256 selected + curr
 //              and epilogue overlap the other's MMAs (G = 2).
 template <int TILES> struct FwdLayout;
 template <> struct FwdLayout<2> {
-  static constexpr int kThreads = 384, kStages = 3, kMaxRegs = 168;
+  static constexpr int kThreads = 384, kStages = 3;
   // warp roles: K producer, MMA issuer, V producer, first softmax warp
   static constexpr int kWarpK = 0, kWarpMMA = 1, kWarpV = 2, kSoftFirst = 4;
   static constexpr uint32_t kTmemCols = 512;
@@ -71,7 +71,7 @@ template <> struct FwdLayout<2> {
 template <> struct FwdLayout<1> {
   // The softmax warps come first (TMEM lane quarter = warp % 4): 7 warps,
   // so two CTAs per SM leave each thread about 146 registers.
-  static constexpr int kThreads = 224, kStages = 2, kMaxRegs = 144;  // 2 x 7 warps x 144 <= 64K
+  static constexpr int kThreads = 224, kStages = 2;
   static constexpr int kWarpK = 4, kWarpMMA = 5, kWarpV = 6, kSoftFirst = 0;
   static constexpr uint32_t kTmemCols = 256;
   static constexpr uint32_t kOffQ = 0;                       // [k half][128 rows][128 B]
@@ -108,12 +108,15 @@ constexpr size_t fwd_smem_bytes() {
 }
 static_assert(2 * (fwd_smem_bytes<1>() + 1024) <= 228 * 1024, "two one-tile CTAs per SM");
 
+// The kernel body; the two entry points below differ only in their register
+// budget (the tensor maps stay kernel parameters, passed by reference).
 template <int TILES, bool OUTER>
-__global__ void __launch_bounds__(FwdLayout<TILES>::kThreads) __maxnreg__(FwdLayout<TILES>::kMaxRegs)
-tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-              const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ idx,
-              const float* __restrict__ gates, AttnShape s, __nv_bfloat16* __restrict__ o,
-              float* __restrict__ lse, DevCtx ctx) {
+__device__ __forceinline__ void tc_fwd_body(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                                            const CUtensorMap& tm_v,
+                                            const int32_t* __restrict__ idx,
+                                            const float* __restrict__ gates, const AttnShape& s,
+                                            __nv_bfloat16* __restrict__ o,
+                                            float* __restrict__ lse, const DevCtx& ctx) {
   using L = FwdLayout<TILES>;
   constexpr int kStages = L::kStages;
   constexpr uint32_t kOffQ = L::kOffQ, kOffK = L::kOffK, kOffV = L::kOffV, kOffP = L::kOffP;
@@ -127,8 +130,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   // Dense: the longest query blocks (most keys) start first.
   const int j = s.dense ? s.N - 1 - (int)blockIdx.x : (int)blockIdx.x;
   // blockIdx.y: KV head and, with TILES = 1, which of its G/2 tiles.
-  const int G = s.Hq / s.Hkv;
-  const int tpk = G / (2 * TILES);  // CTAs per KV head
+  const int G = TILES == 2 ? 4 : s.Hq / s.Hkv;  // two tiles: G = 4
+  const int tpk = TILES == 2 ? 1 : G / 2;        // CTAs per KV head
   const int kvh = blockIdx.y / tpk, u0 = (blockIdx.y % tpk) * TILES, bi = blockIdx.z;
   const long long irow = ((long long)(bi * s.Hkv + kvh) * s.N + j);
 
@@ -441,6 +444,28 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   }
 }
 
+// Two tiles (G = 4): one CTA per SM, up to 168 registers a thread.
+template <bool OUTER>
+__global__ void __launch_bounds__(FwdLayout<2>::kThreads, 1)
+tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ idx,
+              const float* __restrict__ gates, AttnShape s, __nv_bfloat16* __restrict__ o,
+              float* __restrict__ lse, DevCtx ctx) {
+  tc_fwd_body<2, OUTER>(tm_q, tm_k, tm_v, idx, gates, s, o, lse, ctx);
+}
+
+// One tile (G = 2): two CTAs per SM, 144 registers a thread (2 x 7 warps x
+// 144 <= 64K).
+template <bool OUTER>
+__global__ void __maxnreg__(144)
+tc_fwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q,
+                   const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ idx,
+                   const float* __restrict__ gates, AttnShape s, __nv_bfloat16* __restrict__ o,
+                   float* __restrict__ lse, DevCtx ctx) {
+  tc_fwd_body<1, OUTER>(tm_q, tm_k, tm_v, idx, gates, s, o, lse, ctx);
+}
+
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -566,14 +591,14 @@ cudaError_t launch_attn_fwd_tc(const AttnShape& s, const void* q, const void* k,
   const int tiles = G == 4 ? 2 : 1;
   dim3 grid(s.N, s.Hkv * (G / (2 * tiles)), s.B);
   if (tiles == 2) {
-    auto kern = outer ? tc_fwd_kernel<2, true> : tc_fwd_kernel<2, false>;
+    auto kern = outer ? tc_fwd_kernel<true> : tc_fwd_kernel<false>;
     const size_t smem = fwd_smem_bytes<2>();
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, FwdLayout<2>::kThreads, smem, st>>>(tq, tk, tv, idx, gates, s,
                                                      (__nv_bfloat16*)o, lse, ctx);
   } else {
-    auto kern = outer ? tc_fwd_kernel<1, true> : tc_fwd_kernel<1, false>;
+    auto kern = outer ? tc_fwd_tile_kernel<true> : tc_fwd_tile_kernel<false>;
     const size_t smem = fwd_smem_bytes<1>();
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
