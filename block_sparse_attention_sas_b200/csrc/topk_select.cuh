@@ -474,8 +474,18 @@ __device__ __forceinline__ void place_by_rank(const uint64_t* keys, int m, int k
     const int p = tid / tpc, part = tid % tpc;
     const uint64_t mine = p < m ? keys[p] : 0ull;
     int rk = 0;
-#pragma unroll 4
-    for (int q = part; q < m; q += tpc) rk += keys[q] > mine;
+    // Eight loads in flight, then eight comparisons (0 past the list: never
+    // above a key that is placed).
+    for (int q0 = part; q0 < m; q0 += 8 * tpc) {
+      uint64_t y[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int q = q0 + u * tpc;
+        y[u] = q < m ? keys[q] : 0ull;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) rk += y[u] > mine;
+    }
     for (int o = 1; o < tpc; o <<= 1) rk += __shfl_xor_sync(0xffffffffu, rk, o);
     if (part == 0 && mine != 0ull && rk < kk) emit(rk, mine);
     return;
