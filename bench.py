@@ -2,9 +2,10 @@
 
 One step = one pass of the training hot path over one synthetic batch of the
 Qwen3-4B-shaped layer (B=1, 32 q heads / 8 KV heads, d=128, T=16384, b=64,
-K=16): gate softmax + Top-K (sas_gate_topk), the gated sparse forward
-(sas_attn_fwd) and its backward into q, k, v and the selector scores
-(sas_attn_bwd). `value` is the algorithmic fwd+bwd TFLOP/s of the whole job
+K=16): gate softmax + Top-K (sas_gate_topk), the gated sparse forward and
+its backward into q, k, v and the selector scores, as the pair that carries
+the forward's output residual (sas_attn_fwd_res / sas_attn_bwd_res: the same
+results, the backward's row sums from o and the residual). `value` is the algorithmic fwd+bwd TFLOP/s of the whole job
 (14*d FLOPs per attended (query, key) pair per query head; dense and skipped
 work never counted). Beside it the line reports the decode hot path (one token
 per sequence over 64K and 512K caches, gates off and on) in GB/s of selected
@@ -315,10 +316,11 @@ def run_ours(args):
         gates, idx = S.gate_topk(inp["scores"], cfg.K, causal=True)
         if ev:
             ev[1].record(stream)
-        o, lse = S.attn_fwd(inp["q"], inp["k"], inp["v"], idx, gates, cfg.b)
+        o, o_res, lse = S.attn_fwd_res(inp["q"], inp["k"], inp["v"], idx, gates, cfg.b)
         if ev:
             ev[2].record(stream)
-        dq, dk, dv, ds = S.attn_bwd(inp["q"], inp["k"], inp["v"], o, lse, inp["dO"], idx, gates,
+        dq, dk, dv, ds = S.attn_bwd_res(inp["q"], inp["k"], inp["v"], o, o_res, lse, inp["dO"],
+                                        idx, gates,
                                     cfg.b)
         if ev:
             ev[3].record(stream)
@@ -351,7 +353,7 @@ def run_ours(args):
     per = [[e[a].elapsed_time(e[a + 1]) for a in range(3)] for e in evs]  # ms
     step_ms = sum(sum(p) for p in per) / args.steps
     k_ms = {n: sum(p[i] for p in per) / args.steps for i, n in
-            enumerate(("sas_gate_topk", "sas_attn_fwd", "sas_attn_bwd"))}
+            enumerate(("sas_gate_topk", "sas_attn_fwd_res", "sas_attn_bwd_res"))}
     step_ms_max = D.max_over_ranks(step_ms, dev)
     value = world * (f_fwd + f_bwd) / (step_ms_max * 1e-3) / 1e12
 
@@ -380,7 +382,7 @@ def run_ours(args):
 
     # ---- roofline of the dominant call of the training step
     dom = max(k_ms, key=k_ms.get)
-    dom_flops = {"sas_attn_fwd": f_fwd, "sas_attn_bwd": f_bwd}.get(dom, 0.0)
+    dom_flops = {"sas_attn_fwd_res": f_fwd, "sas_attn_bwd_res": f_bwd}.get(dom, 0.0)
     achieved = dom_flops / (k_ms[dom] * 1e-3) / 1e12 if dom_flops else None
     roof = {"kernel": dom, "bound": "tensor", "achieved": achieved,
             "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
@@ -512,10 +514,10 @@ def run_train_line(S, torch, dev, cfg, flush, peaks, steps, warmup, rank):
         if ev:
             ev[0].record(stream)
         gates, idx = S.gate_topk(t["scores"], cfg.K, causal=True)
-        o, lse = S.attn_fwd(t["q"], t["k"], t["v"], idx, gates, cfg.b)
+        o, o_res, lse = S.attn_fwd_res(t["q"], t["k"], t["v"], idx, gates, cfg.b)
         if ev:
             ev[1].record(stream)
-        S.attn_bwd(t["q"], t["k"], t["v"], o, lse, t["dO"], idx, gates, cfg.b)
+        S.attn_bwd_res(t["q"], t["k"], t["v"], o, o_res, lse, t["dO"], idx, gates, cfg.b)
         if ev:
             ev[2].record(stream)
 
@@ -697,8 +699,8 @@ def run_profile_train(args):
     scores = torch.from_numpy(x.scores).to(dev)
     for _ in range(args.warmup + args.steps):
         gates, idx = S.gate_topk(scores, cfg.K)
-        o, lse = S.attn_fwd(t["q"], t["k"], t["v"], idx, gates, cfg.b)
-        S.attn_bwd(t["q"], t["k"], t["v"], o, lse, t["dO"], idx, gates, cfg.b)
+        o, o_res, lse = S.attn_fwd_res(t["q"], t["k"], t["v"], idx, gates, cfg.b)
+        S.attn_bwd_res(t["q"], t["k"], t["v"], o, o_res, lse, t["dO"], idx, gates, cfg.b)
     torch.cuda.synchronize(dev)
     st, raw = S.device_error()
     print(json.dumps({"profile_train": cfg.name, "steps": args.warmup + args.steps,

@@ -42,6 +42,10 @@ SIGNATURES = {
                                 _p, _p]),
     "sas_attn_bwd_gated": (_i, [_i, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i,
                                 _f, _i, _i, _p, _p, _p, _p, _p, _sz, _p]),
+    "sas_attn_fwd_res": (_i, [_i, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p,
+                              _p]),
+    "sas_attn_bwd_res": (_i, [_i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i,
+                              _f, _p, _p, _p, _p, _p, _sz, _p]),
     "sas_attn_fwd": (_i, [_i, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p]),
     "sas_attn_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i]),
     "sas_attn_bwd": (_i, [_i, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f,
@@ -214,6 +218,49 @@ def attn_bwd(q, k, v, o, lse, dO, idx, gates, b: int, scale: float = 0.0,
                                       scale, PHI[phi], GATING[gating], _ptr(dq), _ptr(dk),
                                       _ptr(dv), _ptr(ds), _ptr(ws), ws.numel(),
                                       _stream(q.device)))
+    return dq, dk, dv, ds
+
+
+def attn_fwd_res(q, k, v, idx, gates, b: int, scale: float = 0.0):
+    """Forward that also returns o's residual (o + o_res = the fp32 output).
+    Returns (o, o_res, lse); tensor-core shapes only."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, q.dtype)
+    _need(idx, "idx", torch.int32)
+    if gates is not None:
+        _need(gates, "gates", torch.float32)
+    B, Hq, T, d = q.shape
+    Hkv, K = k.shape[1], idx.shape[-1]
+    o, o_res = torch.empty_like(q), torch.empty_like(q)
+    lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    _check("sas_attn_fwd_res",
+           LIB.sas_attn_fwd_res(_dtype(q), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(gates), B,
+                                Hq, Hkv, T, d, b, K, scale, _ptr(o), _ptr(o_res), _ptr(lse),
+                                _stream(q.device)))
+    return o, o_res, lse
+
+
+def attn_bwd_res(q, k, v, o, o_res, lse, dO, idx, gates, b: int, scale: float = 0.0,
+                 want_dscores: bool = True):
+    """Backward with D from o and its residual. Returns (dq, dk, dv, dscores or None)."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("o_res", o_res), ("dO", dO)):
+        _need(t, n, q.dtype)
+    _need(lse, "lse", torch.float32)
+    _need(idx, "idx", torch.int32)
+    B, Hq, T, d = q.shape
+    Hkv, K = k.shape[1], idx.shape[-1]
+    N = (T + b - 1) // b
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ds = None
+    if gates is not None and want_dscores:
+        ds = torch.empty((B, Hkv, N, N), dtype=torch.float32, device=q.device)
+    nbytes = LIB.sas_attn_bwd_workspace_size(_dtype(q), B, Hq, Hkv, T, d, b, K)
+    ws = _workspace("bwd", nbytes, q.device, zero=False)
+    _check("sas_attn_bwd_res",
+           LIB.sas_attn_bwd_res(_dtype(q), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(o_res),
+                                _ptr(lse), _ptr(dO), _ptr(idx), _ptr(gates), B, Hq, Hkv, T, d, b,
+                                K, scale, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ds), _ptr(ws),
+                                ws.numel(), _stream(q.device)))
     return dq, dk, dv, ds
 
 

@@ -1293,10 +1293,49 @@ bool tc_bwd_supported(sas_dtype_t dt, const AttnShape& s) {
   return dt == SAS_BF16 && s.d == kD && s.b == kB && (G == 2 || G == 4);
 }
 
+namespace {
+// D_i = dO_i . (o_i + o_res_i) for every query row: one warp per row, four
+// columns a lane, rows in the [B][Hq][T] order of the D array. With the
+// forward's residual, o + o_res carries its fp32 output (P entered PV as two
+// bf16 terms), so this is Sum_t P_it dP_it to fp32 rounding.
+__global__ void __launch_bounds__(256)
+d_from_o_kernel(const __nv_bfloat16* __restrict__ dO, const __nv_bfloat16* __restrict__ o,
+                const __nv_bfloat16* __restrict__ o_res, long long rows, float* __restrict__ Dv) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long r = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
+       r += warps) {
+    const long long off = r * kD + lane * 4;
+    const uint2 a = __ldg(reinterpret_cast<const uint2*>(dO + off));
+    const uint2 b = __ldg(reinterpret_cast<const uint2*>(o + off));
+    const uint2 c = __ldg(reinterpret_cast<const uint2*>(o_res + off));
+    auto lo = [](uint32_t x) { return __uint_as_float(x << 16); };
+    auto hi = [](uint32_t x) { return __uint_as_float(x & 0xffff0000u); };
+    float acc = lo(a.x) * (lo(b.x) + lo(c.x));
+    acc = fmaf(hi(a.x), hi(b.x) + hi(c.x), acc);
+    acc = fmaf(lo(a.y), lo(b.y) + lo(c.y), acc);
+    acc = fmaf(hi(a.y), hi(b.y) + hi(c.y), acc);
+    acc = warp_sum(acc);
+    if (lane == 0) Dv[r] = acc;
+  }
+}
+
+cudaError_t launch_d_from_o(const AttnShape& s, const void* dO, const void* o, const void* o_res,
+                            float* Dv, cudaStream_t st) {
+  const long long rows = (long long)s.B * s.Hq * s.T;
+  const long long want = (rows + 7) / 8;
+  const int grid = (int)(want < 148 * 8 ? want : 148 * 8);
+  d_from_o_kernel<<<grid, 256, 0, st>>>((const __nv_bfloat16*)dO, (const __nv_bfloat16*)o,
+                                        (const __nv_bfloat16*)o_res, rows, Dv);
+  note_launches(1);
+  return cudaGetLastError();
+}
+}  // namespace
+
 cudaError_t launch_attn_bwd_tc(const AttnShape& s, const void* q, const void* k, const void* v,
-                               const float* lse, const void* dO, const int32_t* idx,
-                               const float* gates, void* dq, void* dk, void* dv, float* dscores,
-                               void* ws, const DevCtx& ctx, cudaStream_t st) {
+                               const void* o, const void* o_res, const float* lse, const void* dO,
+                               const int32_t* idx, const float* gates, void* dq, void* dk, void* dv,
+                               float* dscores, void* ws, const DevCtx& ctx, cudaStream_t st) {
   const BwdWorkspace L = bwd_workspace_layout(s, true);
   char* w = static_cast<char*>(ws);
   float* Dv = reinterpret_cast<float*>(w + L.off_D);
@@ -1318,7 +1357,9 @@ cudaError_t launch_attn_bwd_tc(const AttnShape& s, const void* q, const void* k,
   if ((e = make_tmap_bf16_2planes(&tdo2, dO, s.T, s.B * s.Hq)) != cudaSuccess) return e;
   if (s.dense) {
     // Every block: no reverse index, no dS tiles (dq recomputes them), no da.
-    {
+    if (o_res) {
+      if ((e = launch_d_from_o(s, dO, o, o_res, Dv, st)) != cudaSuccess) return e;
+    } else {
       dim3 grid(s.N, s.Hkv * tiles, s.B);
       auto kern = tiles == 2 ? tc_bwd_d_kernel<2> : tc_bwd_d_kernel<1>;
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kd::kSmem);
@@ -1359,7 +1400,9 @@ cudaError_t launch_attn_bwd_tc(const AttnShape& s, const void* q, const void* k,
     note_launches(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  {  // D
+  if (o_res) {  // D from the forward's output and its residual
+    if ((e = launch_d_from_o(s, dO, o, o_res, Dv, st)) != cudaSuccess) return e;
+  } else {  // D, recomputed exactly
     dim3 grid(s.N, s.Hkv * tiles, s.B);
     auto kern = tiles == 2 ? tc_bwd_d_kernel<2> : tc_bwd_d_kernel<1>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kd::kSmem);

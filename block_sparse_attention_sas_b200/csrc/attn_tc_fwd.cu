@@ -64,6 +64,9 @@ template <> struct FwdLayout<2> {
   static constexpr uint32_t kOffV = kOffK + kStages * kKVBytes;
   static constexpr uint32_t kOffP = kOffV + kStages * kKVBytes;  // [tile][128 rows][128 B]
   static constexpr uint32_t kOffCtl = kOffP + 2 * 128 * 128;
+  // With the residual output, the low half of P: tile t at kOffPlo + 16 KB t,
+  // in the Q staging area (free once every Q row is in TMEM, before S(0)).
+  static constexpr uint32_t kOffPlo = kOffQ;
   __device__ static uint32_t q_col(int t) { return t * 64; }
   __device__ static uint32_t s_col(int t) { return 128 + t * 64; }
   __device__ static uint32_t o_col(int t) { return 256 + t * 128; }
@@ -79,6 +82,7 @@ template <> struct FwdLayout<1> {
   static constexpr uint32_t kOffK = 2 * 128 * 128;
   static constexpr uint32_t kOffV = kOffK + kStages * kKVBytes;
   static constexpr uint32_t kOffCtl = kOffV + kStages * kKVBytes;
+  static constexpr uint32_t kOffPlo = 128 * 128;  // Q's second half
   __device__ static uint32_t q_col(int) { return 0; }
   __device__ static uint32_t s_col(int) { return 64; }
   __device__ static uint32_t o_col(int) { return 128; }
@@ -110,12 +114,16 @@ static_assert(2 * (fwd_smem_bytes<1>() + 1024) <= 228 * 1024, "two one-tile CTAs
 
 // The kernel body; the two entry points below differ only in their register
 // budget (the tensor maps stay kernel parameters, passed by reference).
-template <int TILES, bool OUTER>
+// RES: P enters PV as two bf16 terms (P = P_hi + P_lo, each rounded to
+// bf16), so O accumulates the fp32 product; o is written rounded to bf16 and
+// o_res = o_fp32 - o as the bf16 residual (the backward's D = dO . (o + o_res)).
+template <int TILES, bool OUTER, bool RES>
 __device__ __forceinline__ void tc_fwd_body(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                                             const CUtensorMap& tm_v,
                                             const int32_t* __restrict__ idx,
                                             const float* __restrict__ gates, const AttnShape& s,
                                             __nv_bfloat16* __restrict__ o,
+                                            __nv_bfloat16* __restrict__ o_res,
                                             float* __restrict__ lse, const DevCtx& ctx) {
   using L = FwdLayout<TILES>;
   constexpr int kStages = L::kStages;
@@ -225,6 +233,7 @@ __device__ __forceinline__ void tc_fwd_body(const CUtensorMap& tm_q, const CUten
       // address field (addresses stay below 256 KB, so no carry leaves it).
       const uint64_t kdesc0 = sdesc_sw128(sbase + kOffK, 16, 1024);
       const uint64_t pdesc0 = sdesc_sw128(sbase + kOffP, 16, 1024);
+      const uint64_t pldesc0 = sdesc_sw128(sbase + L::kOffPlo, 16, 1024);
       const uint64_t vdesc0 = sdesc_sw128(sbase + kOffV, 8192, 1024);
       auto adv = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
       auto issue_s = [&](int n) -> bool {
@@ -258,6 +267,12 @@ __device__ __forceinline__ void tc_fwd_body(const CUtensorMap& tm_q, const CUten
           for (int ks = 0; ks < 4; ++ks)
             mma_bf16_ss(tmem + L::o_col(t), adv(pd, ks * 32), adv(vd, ks * 2048), id_o,
                         (n > 0 || ks > 0));
+          if (RES) {  // + P_lo V
+            const uint64_t pl = adv(pldesc0, t * 16384);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+              mma_bf16_ss(tmem + L::o_col(t), adv(pl, ks * 32), adv(vd, ks * 2048), id_o, true);
+          }
         }
         mma_commit(&c.pv_done);
         mma_commit(&c.v_empty[st]);
@@ -360,6 +375,7 @@ __device__ __forceinline__ void tc_fwd_body(const CUtensorMap& tm_q, const CUten
       const uint64_t sc2 = f2u(sc, sc), off2 = f2u(off, off);
       uint64_t acc0 = 0, acc1 = 0;
       uint32_t pk[32];
+      uint32_t pl[RES ? 32 : 1];
 #pragma unroll
       for (int i = 0; i < 32; i += 2) {
         const uint64_t a0 = ffma2(f2u(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
@@ -386,6 +402,12 @@ __device__ __forceinline__ void tc_fwd_body(const CUtensorMap& tm_q, const CUten
         } else {
           pk[i] = pack_bf16(p0, p1);
           pk[i + 1] = pack_bf16(p2, p3);
+          if (RES) {  // what the bf16 rounding of P dropped, as a second bf16 term
+            pl[i] = pack_bf16(p0 - __uint_as_float(pk[i] << 16),
+                              p1 - __uint_as_float(pk[i] & 0xffff0000u));
+            pl[i + 1] = pack_bf16(p2 - __uint_as_float(pk[i + 1] << 16),
+                                  p3 - __uint_as_float(pk[i + 1] & 0xffff0000u));
+          }
         }
       }
       const uint64_t accs = fadd2(acc0, acc1);
@@ -402,6 +424,14 @@ __device__ __forceinline__ void tc_fwd_body(const CUtensorMap& tm_q, const CUten
         uint4 v = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
         *reinterpret_cast<uint4*>(prow + ((ch ^ (rowi & 7)) << 4)) = v;
       }
+      if (RES) {
+        unsigned char* lrow = base + L::kOffPlo + t * 16384 + rowi * 128;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          uint4 v = make_uint4(pl[4 * ch], pl[4 * ch + 1], pl[4 * ch + 2], pl[4 * ch + 3]);
+          *reinterpret_cast<uint4*>(lrow + ((ch ^ (rowi & 7)) << 4)) = v;
+        }
+      }
       fence_proxy_async_smem();
       fence_before_sync();
       __syncwarp();
@@ -414,7 +444,8 @@ __device__ __forceinline__ void tc_fwd_body(const CUtensorMap& tm_q, const CUten
         fence_after_sync();
         const float inv = 1.f / l;
         const bool write = qrow < s.T;
-        __nv_bfloat16* orow = o + ((long long)(bi * s.Hq + head) * s.T + qrow) * kD;
+        const long long ooff = ((long long)(bi * s.Hq + head) * s.T + qrow) * kD;
+        __nv_bfloat16* orow = o + ooff;
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
           uint32_t ov[32];
@@ -423,12 +454,25 @@ __device__ __forceinline__ void tc_fwd_body(const CUtensorMap& tm_q, const CUten
           if (write) {
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
+              float x[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(ov[8 * q4 + e]) * inv;
               uint4 v;
-              v.x = pack_bf16(__uint_as_float(ov[8 * q4 + 0]) * inv, __uint_as_float(ov[8 * q4 + 1]) * inv);
-              v.y = pack_bf16(__uint_as_float(ov[8 * q4 + 2]) * inv, __uint_as_float(ov[8 * q4 + 3]) * inv);
-              v.z = pack_bf16(__uint_as_float(ov[8 * q4 + 4]) * inv, __uint_as_float(ov[8 * q4 + 5]) * inv);
-              v.w = pack_bf16(__uint_as_float(ov[8 * q4 + 6]) * inv, __uint_as_float(ov[8 * q4 + 7]) * inv);
+              v.x = pack_bf16(x[0], x[1]);
+              v.y = pack_bf16(x[2], x[3]);
+              v.z = pack_bf16(x[4], x[5]);
+              v.w = pack_bf16(x[6], x[7]);
               *reinterpret_cast<uint4*>(orow + ch * 32 + q4 * 8) = v;
+              if (RES) {
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                uint32_t rr[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  rr[e] = pack_bf16(x[2 * e] - __uint_as_float(w[e] << 16),
+                                    x[2 * e + 1] - __uint_as_float(w[e] & 0xffff0000u));
+                *reinterpret_cast<uint4*>(o_res + ooff + ch * 32 + q4 * 8) =
+                    make_uint4(rr[0], rr[1], rr[2], rr[3]);
+              }
             }
           }
         }
@@ -445,25 +489,25 @@ __device__ __forceinline__ void tc_fwd_body(const CUtensorMap& tm_q, const CUten
 }
 
 // Two tiles (G = 4): one CTA per SM, up to 168 registers a thread.
-template <bool OUTER>
+template <bool OUTER, bool RES>
 __global__ void __launch_bounds__(FwdLayout<2>::kThreads, 1)
 tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ idx,
               const float* __restrict__ gates, AttnShape s, __nv_bfloat16* __restrict__ o,
-              float* __restrict__ lse, DevCtx ctx) {
-  tc_fwd_body<2, OUTER>(tm_q, tm_k, tm_v, idx, gates, s, o, lse, ctx);
+              __nv_bfloat16* __restrict__ o_res, float* __restrict__ lse, DevCtx ctx) {
+  tc_fwd_body<2, OUTER, RES>(tm_q, tm_k, tm_v, idx, gates, s, o, o_res, lse, ctx);
 }
 
 // One tile (G = 2): two CTAs per SM, 144 registers a thread (2 x 7 warps x
 // 144 <= 64K).
-template <bool OUTER>
+template <bool OUTER, bool RES>
 __global__ void __maxnreg__(144)
 tc_fwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ idx,
                    const float* __restrict__ gates, AttnShape s, __nv_bfloat16* __restrict__ o,
-                   float* __restrict__ lse, DevCtx ctx) {
-  tc_fwd_body<1, OUTER>(tm_q, tm_k, tm_v, idx, gates, s, o, lse, ctx);
+                   __nv_bfloat16* __restrict__ o_res, float* __restrict__ lse, DevCtx ctx) {
+  tc_fwd_body<1, OUTER, RES>(tm_q, tm_k, tm_v, idx, gates, s, o, o_res, lse, ctx);
 }
 
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -575,8 +619,8 @@ bool tc_fwd_supported(sas_dtype_t dt, const AttnShape& s) {
 }
 
 cudaError_t launch_attn_fwd_tc(const AttnShape& s, const void* q, const void* k, const void* v,
-                               const int32_t* idx, const float* gates, void* o, float* lse,
-                               const DevCtx& ctx, cudaStream_t st) {
+                               const int32_t* idx, const float* gates, void* o, void* o_res,
+                               float* lse, const DevCtx& ctx, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
   cudaError_t e;
   if ((e = make_tmap_bf16(&tq, q, s.T, s.B * s.Hq)) != cudaSuccess) return e;
@@ -584,6 +628,7 @@ cudaError_t launch_attn_fwd_tc(const AttnShape& s, const void* q, const void* k,
   if ((e = make_tmap_bf16(&tv, v, s.T, s.B * s.Hkv)) != cudaSuccess) return e;
   const int G = s.Hq / s.Hkv;
   const bool outer = s.outer && gates != nullptr;  // no gates: both gatings coincide
+  const bool res = o_res != nullptr;               // inner gating only (checked by the caller)
   // G = 4: both tiles of the group in one CTA, sharing every K/V block (one
   // tile per CTA, two CTAs per SM, measured 0.58 ms against 0.41 ms on the
   // Qwen3-4B layer: the K/V blocks are then fetched twice and the rings are
@@ -591,19 +636,23 @@ cudaError_t launch_attn_fwd_tc(const AttnShape& s, const void* q, const void* k,
   const int tiles = G == 4 ? 2 : 1;
   dim3 grid(s.N, s.Hkv * (G / (2 * tiles)), s.B);
   if (tiles == 2) {
-    auto kern = outer ? tc_fwd_kernel<true> : tc_fwd_kernel<false>;
+    auto kern = outer ? tc_fwd_kernel<true, false>
+                      : (res ? tc_fwd_kernel<false, true> : tc_fwd_kernel<false, false>);
     const size_t smem = fwd_smem_bytes<2>();
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, FwdLayout<2>::kThreads, smem, st>>>(tq, tk, tv, idx, gates, s,
-                                                     (__nv_bfloat16*)o, lse, ctx);
+                                                     (__nv_bfloat16*)o, (__nv_bfloat16*)o_res,
+                                                     lse, ctx);
   } else {
-    auto kern = outer ? tc_fwd_tile_kernel<true> : tc_fwd_tile_kernel<false>;
+    auto kern = outer ? tc_fwd_tile_kernel<true, false>
+                      : (res ? tc_fwd_tile_kernel<false, true> : tc_fwd_tile_kernel<false, false>);
     const size_t smem = fwd_smem_bytes<1>();
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, FwdLayout<1>::kThreads, smem, st>>>(tq, tk, tv, idx, gates, s,
-                                                     (__nv_bfloat16*)o, lse, ctx);
+                                                     (__nv_bfloat16*)o, (__nv_bfloat16*)o_res,
+                                                     lse, ctx);
   }
   note_launches(1);
   return cudaGetLastError();

@@ -110,8 +110,8 @@ sas_status_t gate_topk_impl(const float* scores, int B, int Hkv, int rows, int C
 
 sas_status_t attn_fwd_impl(sas_dtype_t dtype, const void* q, const void* k, const void* v,
                            const int32_t* idx, const float* gates, int B, int Hq, int Hkv, int T,
-                           int d, int b, int K, float scale, int gating, void* o, float* lse,
-                           cudaStream_t stream) {
+                           int d, int b, int K, float scale, int gating, void* o, void* o_res,
+                           float* lse, cudaStream_t stream) {
   sas_status_t st = check_attn(dtype, B, Hq, Hkv, T, d, b, K, false, scale);
   if (st != SAS_OK) return st;
   if (!valid_gating(gating)) return SAS_ERR_INVALID_ARG;
@@ -124,13 +124,18 @@ sas_status_t attn_fwd_impl(sas_dtype_t dtype, const void* q, const void* k, cons
   if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
   AttnShape s = make_shape(B, Hq, Hkv, T, d, b, K, scale, false);
   s.outer = gating == SAS_GATE_OUTER;
+  if (o_res) {  // the residual output: tensor-core forward, inner gating
+    if (!aligned(o_res, 16)) return SAS_ERR_INVALID_ARG;
+    if (!tc_fwd_supported(dtype, s) || s.outer) return SAS_ERR_UNSUPPORTED;
+  }
   if (tc_fwd_supported(dtype, s))
-    return cuda_status(launch_attn_fwd_tc(s, q, k, v, idx, gates, o, lse, ctx, stream));
+    return cuda_status(launch_attn_fwd_tc(s, q, k, v, idx, gates, o, o_res, lse, ctx, stream));
   return cuda_status(launch_attn_fwd_simt(dtype, s, q, k, v, idx, gates, o, lse, ctx, stream));
 }
 
 sas_status_t attn_bwd_impl(sas_dtype_t dtype, const void* q, const void* k, const void* v,
-                           const void* o, const float* lse, const void* dO, const int32_t* idx,
+                           const void* o, const void* o_res, const float* lse, const void* dO,
+                           const int32_t* idx,
                            const float* gates, int B, int Hq, int Hkv, int T, int d, int b, int K,
                            float scale, int phi, int gating, void* dq, void* dk, void* dv,
                            float* dscores, void* ws, size_t ws_bytes, cudaStream_t stream) {
@@ -149,13 +154,17 @@ sas_status_t attn_bwd_impl(sas_dtype_t dtype, const void* q, const void* k, cons
   AttnShape s = make_shape(B, Hq, Hkv, T, d, b, K, scale, false);
   s.outer = gating == SAS_GATE_OUTER;
   s.phi = phi;
+  if (o_res) {  // D from o and the forward's residual: tensor-core path, inner gating
+    if (!aligned(o_res, 16)) return SAS_ERR_INVALID_ARG;
+    if (!tc_bwd_supported(dtype, s) || s.outer) return SAS_ERR_UNSUPPORTED;
+  }
   const size_t need = bwd_workspace_layout(s, tc_bwd_supported(dtype, s)).total;
   if (!ws || ws_bytes < need || !aligned(ws, 256)) return SAS_ERR_WORKSPACE;
   DevCtx ctx;
   if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
   if (tc_bwd_supported(dtype, s))
-    return cuda_status(launch_attn_bwd_tc(s, q, k, v, lse, dO, idx, gates, dq, dk, dv, dscores,
-                                          ws, ctx, stream));
+    return cuda_status(launch_attn_bwd_tc(s, q, k, v, o, o_res, lse, dO, idx, gates, dq, dk, dv,
+                                          dscores, ws, ctx, stream));
   return cuda_status(launch_attn_bwd_simt(dtype, s, q, k, v, o, lse, dO, idx, gates, dq, dk, dv,
                                           dscores, ws, ctx, stream));
 }
@@ -281,7 +290,7 @@ sas_status_t sas_attn_fwd(sas_dtype_t dtype, const void* q, const void* k, const
                           int d, int b, int K, float scale, void* o, float* lse,
                           sas_stream_t stream) {
   return attn_fwd_impl(dtype, q, k, v, idx, gates, B, Hq, Hkv, T, d, b, K, scale, SAS_GATE_INNER,
-                       o, lse, stream);
+                       o, nullptr, lse, stream);
 }
 
 sas_status_t sas_attn_fwd_gated(sas_dtype_t dtype, const void* q, const void* k, const void* v,
@@ -289,7 +298,7 @@ sas_status_t sas_attn_fwd_gated(sas_dtype_t dtype, const void* q, const void* k,
                                 int T, int d, int b, int K, float scale, sas_gating_t gating,
                                 void* o, float* lse, sas_stream_t stream) {
   return attn_fwd_impl(dtype, q, k, v, idx, gates, B, Hq, Hkv, T, d, b, K, scale, (int)gating, o,
-                       lse, stream);
+                       nullptr, lse, stream);
 }
 
 size_t sas_attn_bwd_workspace_size(sas_dtype_t dtype, int B, int Hq, int Hkv, int T, int d, int b,
@@ -304,8 +313,9 @@ sas_status_t sas_attn_bwd(sas_dtype_t dtype, const void* q, const void* k, const
                           const float* gates, int B, int Hq, int Hkv, int T, int d, int b, int K,
                           float scale, void* dq, void* dk, void* dv, float* dscores, void* ws,
                           size_t ws_bytes, sas_stream_t stream) {
-  return attn_bwd_impl(dtype, q, k, v, o, lse, dO, idx, gates, B, Hq, Hkv, T, d, b, K, scale,
-                       SAS_PHI_SOFTMAX, SAS_GATE_INNER, dq, dk, dv, dscores, ws, ws_bytes, stream);
+  return attn_bwd_impl(dtype, q, k, v, o, nullptr, lse, dO, idx, gates, B, Hq, Hkv, T, d, b, K,
+                       scale, SAS_PHI_SOFTMAX, SAS_GATE_INNER, dq, dk, dv, dscores, ws, ws_bytes,
+                       stream);
 }
 
 sas_status_t sas_attn_bwd_gated(sas_dtype_t dtype, const void* q, const void* k, const void* v,
@@ -314,8 +324,28 @@ sas_status_t sas_attn_bwd_gated(sas_dtype_t dtype, const void* q, const void* k,
                                 int T, int d, int b, int K, float scale, sas_phi_t phi,
                                 sas_gating_t gating, void* dq, void* dk, void* dv,
                                 float* dscores, void* ws, size_t ws_bytes, sas_stream_t stream) {
-  return attn_bwd_impl(dtype, q, k, v, o, lse, dO, idx, gates, B, Hq, Hkv, T, d, b, K, scale,
-                       (int)phi, (int)gating, dq, dk, dv, dscores, ws, ws_bytes, stream);
+  return attn_bwd_impl(dtype, q, k, v, o, nullptr, lse, dO, idx, gates, B, Hq, Hkv, T, d, b, K,
+                       scale, (int)phi, (int)gating, dq, dk, dv, dscores, ws, ws_bytes, stream);
+}
+
+sas_status_t sas_attn_fwd_res(sas_dtype_t dtype, const void* q, const void* k, const void* v,
+                              const int32_t* idx, const float* gates, int B, int Hq, int Hkv, int T,
+                              int d, int b, int K, float scale, void* o, void* o_res, float* lse,
+                              sas_stream_t stream) {
+  if (!o_res && B > 0) return SAS_ERR_INVALID_ARG;
+  return attn_fwd_impl(dtype, q, k, v, idx, gates, B, Hq, Hkv, T, d, b, K, scale, SAS_GATE_INNER,
+                       o, o_res, lse, stream);
+}
+
+sas_status_t sas_attn_bwd_res(sas_dtype_t dtype, const void* q, const void* k, const void* v,
+                              const void* o, const void* o_res, const float* lse, const void* dO,
+                              const int32_t* idx, const float* gates, int B, int Hq, int Hkv,
+                              int T, int d, int b, int K, float scale, void* dq, void* dk, void* dv,
+                              float* dscores, void* ws, size_t ws_bytes, sas_stream_t stream) {
+  if (!o_res && B > 0) return SAS_ERR_INVALID_ARG;
+  return attn_bwd_impl(dtype, q, k, v, o, o_res, lse, dO, idx, gates, B, Hq, Hkv, T, d, b, K,
+                       scale, SAS_PHI_SOFTMAX, SAS_GATE_INNER, dq, dk, dv, dscores, ws, ws_bytes,
+                       stream);
 }
 
 size_t sas_decode_workspace_size(int B, int Hq, int Hkv, int L, int d, int b, int K) {
@@ -529,7 +559,8 @@ sas_status_t sas_dense_fwd(sas_dtype_t dtype, const void* q, const void* k, cons
   if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
   const AttnShape s = make_shape(B, Hq, Hkv, T, d, b, 0, scale, true);
   if (tc_fwd_supported(dtype, s))
-    return cuda_status(launch_attn_fwd_tc(s, q, k, v, nullptr, nullptr, o, lse, ctx, stream));
+    return cuda_status(launch_attn_fwd_tc(s, q, k, v, nullptr, nullptr, o, nullptr, lse, ctx,
+                                          stream));
   return cuda_status(launch_attn_fwd_simt(dtype, s, q, k, v, nullptr, nullptr, o, lse, ctx, stream));
 }
 
@@ -557,7 +588,7 @@ sas_status_t sas_dense_bwd(sas_dtype_t dtype, const void* q, const void* k, cons
   DevCtx ctx;
   if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
   if (tc_bwd_supported(dtype, s))
-    return cuda_status(launch_attn_bwd_tc(s, q, k, v, lse, dO, nullptr, nullptr, dq, dk, dv,
+    return cuda_status(launch_attn_bwd_tc(s, q, k, v, o, nullptr, lse, dO, nullptr, nullptr, dq, dk, dv,
                                           nullptr, ws, ctx, stream));
   return cuda_status(launch_attn_bwd_simt(dtype, s, q, k, v, o, lse, dO, nullptr, nullptr, dq, dk,
                                           dv, nullptr, ws, ctx, stream));

@@ -43,16 +43,20 @@ cudaError_t launch_attn_fwd_simt(sas_dtype_t dt, const AttnShape& s, const void*
                                  float* lse, const DevCtx& ctx, cudaStream_t stream);
 // Tensor-core (tcgen05) forward: bf16, d = 128, b = 64, G in {2, 4}.
 bool tc_fwd_supported(sas_dtype_t dt, const AttnShape& s);
+// o_res (nullable, inner gating only): the forward also writes o's bf16
+// residual o_fp32 - o, with P split in two bf16 terms in the PV product.
 cudaError_t launch_attn_fwd_tc(const AttnShape& s, const void* q, const void* k, const void* v,
-                               const int32_t* idx, const float* gates, void* o, float* lse,
-                               const DevCtx& ctx, cudaStream_t stream);
+                               const int32_t* idx, const float* gates, void* o, void* o_res,
+                               float* lse, const DevCtx& ctx, cudaStream_t stream);
 
 // Tensor-core (tcgen05) backward for the same shapes as the forward.
 bool tc_bwd_supported(sas_dtype_t dt, const AttnShape& s);
+// o / o_res (both or neither): D = dO . (o + o_res) in one memory-bound pass
+// instead of the exact recomputation (inner gating).
 cudaError_t launch_attn_bwd_tc(const AttnShape& s, const void* q, const void* k, const void* v,
-                               const float* lse, const void* dO, const int32_t* idx,
-                               const float* gates, void* dq, void* dk, void* dv, float* dscores,
-                               void* ws, const DevCtx& ctx, cudaStream_t stream);
+                               const void* o, const void* o_res, const float* lse, const void* dO,
+                               const int32_t* idx, const float* gates, void* dq, void* dk, void* dv,
+                               float* dscores, void* ws, const DevCtx& ctx, cudaStream_t stream);
 // Shared pieces of the backward (defined with the SIMT kernels).
 cudaError_t launch_bwd_csr(const AttnShape& s, const int32_t* idx, int32_t* off, int32_t* list,
                            const DevCtx& ctx, cudaStream_t stream);

@@ -213,6 +213,37 @@ sas_status_t sas_attn_bwd_gated(sas_dtype_t dtype, const void* q, const void* k,
                                 float* dscores, void* ws, size_t ws_bytes, sas_stream_t stream);
 
 /*
+ * The training pair with the forward's output residual: the same results as
+ * sas_attn_fwd / sas_attn_bwd, with the backward's row sums
+ * D_i = sum_t P_it dP_it taken in one pass over dO, o and o_res instead of a
+ * recomputation of every attended tile. This is a library variant; the
+ * method's pages fix no kernel split of the backward.
+ *   sas_attn_fwd_res: also writes o_res [B, Hq, T, d] (dtype), the part of
+ *     the fp32 output that rounding o to the dtype drops: o + o_res is the
+ *     output to fp32 rounding. For this the probabilities enter the P.V
+ *     product as two bf16 terms (P = P_hi + P_lo), so that product is the
+ *     fp32 one; o itself is the same up to that rounding.
+ *   sas_attn_bwd_res: the backward with D_i = dO_i . (o_i + o_res_i), which
+ *     equals sum_t P_it dP_it to fp32 rounding. Taking D from the stored bf16
+ *     o alone would move dq by more than the bf16 tolerance on rows that
+ *     attend a few large-logit keys; with the residual it does not.
+ *   Both: bf16, d = 128, b = 64, G = Hq / Hkv of 2 or 4 (the tensor-core
+ *   path), inner gating; any other shape returns SAS_ERR_UNSUPPORTED. o_res
+ *   is 16-byte aligned and not NULL (SAS_ERR_INVALID_ARG). Other arguments,
+ *   layouts, the workspace and the errors are those of sas_attn_fwd /
+ *   sas_attn_bwd.
+ */
+sas_status_t sas_attn_fwd_res(sas_dtype_t dtype, const void* q, const void* k, const void* v,
+                              const int32_t* idx, const float* gates, int B, int Hq, int Hkv, int T,
+                              int d, int b, int K, float scale, void* o, void* o_res, float* lse,
+                              sas_stream_t stream);
+sas_status_t sas_attn_bwd_res(sas_dtype_t dtype, const void* q, const void* k, const void* v,
+                              const void* o, const void* o_res, const float* lse, const void* dO,
+                              const int32_t* idx, const float* gates, int B, int Hq, int Hkv,
+                              int T, int d, int b, int K, float scale, void* dq, void* dk, void* dv,
+                              float* dscores, void* ws, size_t ws_bytes, sas_stream_t stream);
+
+/*
  * sas_decode - one query token per sequence over a KV cache, selected blocks
  * plus the current block ([picx] Eq. 2 with use_gates = 0, Eq. 9 with
  * use_gates = 1; [review] Summary: gates are dropped at inference while the
