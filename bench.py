@@ -666,8 +666,83 @@ def bench_decode(S, torch, dev, stream, flush, peaks, args, rank):
             line["dense"] = {"decode_us": dense_us, "bytes": dbytes,
                              "GB/s": dbytes / (dense_us * 1e-6) / 1e9,
                              "speedup_sparse_step": dense_us / step_us}
+            line["paged"] = bench_paged(S, torch, dev, stream, flush, t, cfg, use_gates, reps)
+            line["with_selector"] = bench_selector_step(S, torch, dev, stream, flush, t, cfg,
+                                                        use_gates, reps)
         out.append(line)
     return out
+
+
+def bench_paged(S, torch, dev, stream, flush, t, cfg, use_gates, reps, P=16):
+    """The same decode over a paged copy of the caches (P-token pages placed
+    in a seeded random order): sas_decode_paged with the same selection,
+    timed like the contiguous decode; its output must equal the contiguous
+    one."""
+    B, Hkv, L, d = t["kc"].shape
+    npp = L // P
+    perm = torch.randperm(B * npp, generator=torch.Generator().manual_seed(cfg.seed + 17))
+    kp = torch.empty((B * npp, Hkv, P, d), dtype=t["kc"].dtype, device=dev)
+    vp = torch.empty_like(kp)
+    pd = perm.to(dev)
+    kp[pd] = t["kc"].view(B, Hkv, npp, P, d).permute(0, 2, 1, 3, 4).reshape(B * npp, Hkv, P, d)
+    vp[pd] = t["vc"].view(B, Hkv, npp, P, d).permute(0, 2, 1, 3, 4).reshape(B * npp, Hkv, P, d)
+    indptr = torch.arange(0, B * npp + 1, npp, dtype=torch.int32, device=dev)
+    indices = pd.to(torch.int32)
+    lens = torch.full((B,), cfg.L, dtype=torch.int32, device=dev)
+    gates, idx = S.gate_topk(t["s"], cfg.K, causal=False)
+    ix, g = idx[:, :, 0].contiguous(), gates[:, :, 0].contiguous()
+
+    def call():
+        return S.decode_paged(t["q"], kp, vp, indptr, indices, lens, ix, g, use_gates, cfg.b,
+                              max_len=cfg.L)
+
+    o_ref = S.decode(t["q"], t["kc"], t["vc"], ix, g, use_gates, cfg.b, L=cfg.L)
+    o_pg = call()
+    torch.cuda.synchronize(dev)
+    same = bool(torch.equal(o_ref, o_pg))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+    for i in range(reps):
+        flush.zero_()
+        torch.cuda._sleep(HEAD_START_CYCLES)
+        evs[i][0].record(stream)
+        call()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    us = 1e3 * statistics.median(a.elapsed_time(b) for a, b in evs)
+    nbytes = decode_bytes(cfg)
+    del kp, vp
+    torch.cuda.empty_cache()
+    return {"page_tokens": P, "pages": B * npp, "order": "seeded random permutation",
+            "decode_us": us, "GB/s": nbytes / (us * 1e-6) / 1e9,
+            "equals_contiguous_decode": same}
+
+
+def bench_selector_step(S, torch, dev, stream, flush, t, cfg, use_gates, reps):
+    """The decode step with the weight-free block selector in front: the
+    scores of q against the history blocks' mean keys (kept per block, so
+    computed once here, as a serving loop would keep them), then the fused
+    selection and decode."""
+    kbar = S.block_summaries(t["kc"], cfg.b, L=cfg.L)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+    for i in range(reps + 3):
+        flush.zero_()
+        torch.cuda._sleep(HEAD_START_CYCLES)
+        ev = evs[i - 3] if i >= 3 else None
+        if ev:
+            ev[0].record(stream)
+        sc = S.selector_scores_decode(t["q"], kbar)
+        if ev:
+            ev[1].record(stream)
+        S.decode_select(t["q"], t["kc"], t["vc"], sc, cfg.K, use_gates, cfg.b, L=cfg.L)
+        if ev:
+            ev[2].record(stream)
+    torch.cuda.synchronize(dev)
+    sel = 1e3 * statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+    step = 1e3 * statistics.median(e[0].elapsed_time(e[2]) for e in evs)
+    del kbar
+    return {"selector_scores_us": sel, "step_us": step,
+            "step": "sas_selector_scores_decode + sas_decode_select",
+            "block_summaries": "computed once (a serving loop adds one per filled block)"}
 
 
 def run_decode_only(args):

@@ -78,27 +78,59 @@ scores_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar, in
 }
 
 // Decode scores of one (batch, KV head): qbar = the mean of the G query heads,
-// s[m] = scale * qbar . kbar_m for m < C. One warp per history block.
-template <typename T>
+// s[m] = scale * qbar . kbar_m for m < C. A CTA takes 64 history blocks (8
+// per warp), so the query mean is formed once per 64 blocks; a lane reads
+// d / 32 consecutive columns of a block (one vector load when kbar is
+// 16-byte aligned), and the eight blocks of a warp are in flight together.
+template <typename T, int D, bool VEC>
 __global__ void __launch_bounds__(256)
-decode_scores_kernel(const T* __restrict__ q, const float* __restrict__ kbar, int G, int C, int d,
+decode_scores_kernel(const T* __restrict__ q, const float* __restrict__ kbar, int G, int C,
                      float scale, float* __restrict__ s) {
-  __shared__ float qb[128];
+  constexpr int W = D / 32;  // columns a lane
+  __shared__ __align__(16) float qb[D];
   const int u = blockIdx.y;  // batch * Hkv + kvh
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+  for (int c = threadIdx.x; c < D; c += blockDim.x) {
     float a = 0.f;
-    for (int g = 0; g < G; ++g) a += ld_f(q + ((long long)u * G + g) * d + c);
+    for (int g = 0; g < G; ++g) a += ld_f(q + ((long long)u * G + g) * D + c);
     qb[c] = a / (float)G;
   }
   __syncthreads();
   const int lane = threadIdx.x & 31;
-  const int m = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (m >= C) return;
-  const float* kr = kbar + ((long long)u * C + m) * d;
-  float a = 0.f;
-  for (int c = lane; c < d; c += 32) a = fmaf(qb[c], kr[c], a);
-  a = warp_sum(a);
-  if (lane == 0) s[(long long)u * C + m] = a * scale;
+  const int m0 = blockIdx.x * 64 + (threadIdx.x >> 5) * 8;
+  float qv[W];
+#pragma unroll
+  for (int w = 0; w < W; ++w) qv[w] = qb[lane * W + w];
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int m = m0 + i;
+    float kv[W];
+    if (m < C) {
+      const float* kr = kbar + ((long long)u * C + m) * D + lane * W;
+      if (VEC && W == 4) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(kr));
+        kv[0] = v.x;
+        kv[1 % W] = v.y;
+        kv[2 % W] = v.z;
+        kv[3 % W] = v.w;
+      } else {
+#pragma unroll
+        for (int w = 0; w < W; ++w) kv[w] = __ldg(kr + w);
+      }
+    } else {
+#pragma unroll
+      for (int w = 0; w < W; ++w) kv[w] = 0.f;
+    }
+    float a = 0.f;
+#pragma unroll
+    for (int w = 0; w < W; ++w) a = fmaf(qv[w], kv[w], a);
+    acc[i] = a;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float a = warp_sum(acc[i]);
+    if (lane == 0 && m0 + i < C) s[(long long)u * C + m0 + i] = a * scale;
+  }
 }
 
 template <typename T>
@@ -137,13 +169,26 @@ cudaError_t launch_selector_scores_decode(sas_dtype_t dt, const void* q, const f
                                           int units, int G, int C, int d, float scale,
                                           float* scores, cudaStream_t st) {
   if (units == 0 || C == 0) return cudaSuccess;
-  dim3 grid((C + 7) / 8, units);
-  if (dt == SAS_F32)
-    decode_scores_kernel<float><<<grid, 256, 0, st>>>((const float*)q, kbar, G, C, d, scale,
-                                                       scores);
-  else
-    decode_scores_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)q, kbar, G,
-                                                               C, d, scale, scores);
+  dim3 grid((C + 63) / 64, units);
+  const bool vec = (reinterpret_cast<uintptr_t>(kbar) & 15) == 0;
+  auto go = [&](auto kern, const auto* qq) {
+    kern<<<grid, 256, 0, st>>>(qq, kbar, G, C, scale, scores);
+  };
+  if (dt == SAS_F32) {
+    const float* qq = (const float*)q;
+    if (d == 128)
+      vec ? go(decode_scores_kernel<float, 128, true>, qq)
+          : go(decode_scores_kernel<float, 128, false>, qq);
+    else
+      go(decode_scores_kernel<float, 64, false>, qq);
+  } else {
+    const __nv_bfloat16* qq = (const __nv_bfloat16*)q;
+    if (d == 128)
+      vec ? go(decode_scores_kernel<__nv_bfloat16, 128, true>, qq)
+          : go(decode_scores_kernel<__nv_bfloat16, 128, false>, qq);
+    else
+      go(decode_scores_kernel<__nv_bfloat16, 64, false>, qq);
+  }
   note_launches(1);
   return cudaGetLastError();
 }

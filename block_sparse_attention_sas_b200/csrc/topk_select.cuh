@@ -222,8 +222,9 @@ __device__ __forceinline__ float fast_gate(float sc, float lse, int phi) {
 //     through distributed shared memory (one round trip, lane x reading rank
 //     x); every CTA forms the row's max M and LSE alike;
 //  2. each CTA histograms its chunk over 64 buckets of (M - s) in steps of
-//     1/8 (bucket 63: everything further down, never counted: its count is
-//     the rest of the row) and adds the histogram into every CTA's copy of
+//     1/8, or of (M - min) / 63 when the row's scores span less than 63/8
+//     (bucket 63: everything further down, never counted: its count is the
+//     rest of the row) and adds the histogram into every CTA's copy of
 //     the row's histogram (remote reductions, no round trip); after a
 //     cluster barrier each CTA finds b*, the bucket holding the k-th largest
 //     score, in its own copy. When that is bucket 63, a second histogram
@@ -240,7 +241,7 @@ __device__ __forceinline__ float fast_gate(float sc, float lse, int phi) {
 constexpr int kSelMaxCta = 16;   // rows up to 16 chunks
 constexpr int kSelCand = 1024;   // candidates rank 0 places by rank
 constexpr int kSelNB = 64;       // buckets per histogram level
-constexpr float kSelStep = 8.f;  // level-1 buckets per unit of score below the max
+constexpr float kSelStep = 8.f;  // level-1 buckets per unit of score below the max (at least)
 
 struct SelShared {
   float part[3];                     // this chunk's max, min, sum of exp (relative to its max)
@@ -396,9 +397,15 @@ __device__ int cluster_select(const float (&f)[E], const bool (&ok)[E], int lo, 
   __syncthreads();
   const float M = sh.M, Mn = sh.Mn;
 
-  // ---- level 1: 1/8-wide buckets below the max; the last is never counted
+  // ---- level 1: 1/8-wide buckets below the max (finer when the row's
+  // scores span less: 63 buckets then cover the span); the last is never
+  // counted. The width comes from M and Mn, so it is the same in every CTA.
+  const float span = M - Mn;
+  const float step = (span > 0.f && span < (float)(kSelNB - 1) / kSelStep)
+                         ? (float)(kSelNB - 1) / span
+                         : kSelStep;
   auto b1_of = [&](float x) -> int {
-    return (int)fminf((M - x) * kSelStep, (float)(kSelNB - 1));
+    return (int)fminf((M - x) * step, (float)(kSelNB - 1));
   };
 #pragma unroll
   for (int e = 0; e < E; ++e)
@@ -413,7 +420,7 @@ __device__ int cluster_select(const float (&f)[E], const bool (&ok)[E], int lo, 
 
   // ---- level 2 (rare: the k-th score lies 63/8 or more below the max):
   // 64 buckets spread over [Mn, M - 63/8]
-  const float top2 = M - (float)(kSelNB - 1) / kSelStep;
+  const float top2 = M - (float)(kSelNB - 1) / step;
   const float inv2 = top2 > Mn ? (float)(kSelNB - 1) / (top2 - Mn) : 0.f;
   auto b2_of = [&](float x) -> int {
     return (int)fminf(fmaxf((top2 - x) * inv2, 0.f), (float)(kSelNB - 1));

@@ -28,6 +28,17 @@ def test_gate_topk_wide_rows(cuda_lib, C, K, spread):
     _gate_case(cuda_lib, s, K, False)
 
 
+@pytest.mark.parametrize("C,K", [(1023, 32), (8191, 64), (3000, 100)])
+def test_gate_topk_narrow_rows(cuda_lib, C, K):
+    """Rows whose scores span far less than one unit (std 0.01, as the
+    weight-free selector gives on random data): the selection's buckets
+    narrow to the row's span instead of sending every entry to the exact
+    path."""
+    rng = np.random.default_rng(C + 3 * K)
+    s = (rng.standard_normal((2, 1, 2, C)) * 0.01).astype(np.float32)
+    _gate_case(cuda_lib, s, K, False)
+
+
 @pytest.mark.parametrize("C,K", [(1023, 32), (8191, 64), (3000, 64)])
 def test_gate_topk_skewed_rows(cuda_lib, C, K):
     """Rows whose largest scores all sit in the entries one lane of a warp

@@ -52,17 +52,20 @@ def test_decode_select_small(cuda_lib, kw, use_gates):
     _select_case(cuda_lib, W.small_decode_config(**kw), use_gates)
 
 
-@pytest.mark.parametrize("C,levels", [(1000, 1), (3000, 1), (3000, 2), (2500, 0)])
+@pytest.mark.parametrize("C,levels", [(1000, 1), (3000, 1), (3000, 2), (2500, 0), (2500, -1)])
 def test_decode_select_ties_and_spread(cuda_lib, C, levels):
     """Mass ties (every score equal: the long placement, and past 1024
-    candidates the per-chunk exact path), two levels, and a wide spread
-    (the k-th score more than 63/8 below the max: the second histogram)."""
+    candidates the per-chunk exact path), two levels, a wide spread (the
+    k-th score more than 63/8 below the max: the second histogram), and a
+    narrow one (std 0.01: buckets narrowed to the row's span)."""
     dc = W.small_decode_config(B=1, Hq=4, Hkv=1, L=C * 64 + 1, d=128, b=64, K=32, dtype="bf16")
     rng = np.random.default_rng(C + levels)
-    if levels:
+    if levels > 0:
         s = rng.integers(0, levels, (1, 1, C)).astype(np.float32)
-    else:
+    elif levels == 0:
         s = (rng.standard_normal((1, 1, C)) * 40.0).astype(np.float32)
+    else:
+        s = (rng.standard_normal((1, 1, C)) * 0.01).astype(np.float32)
     _select_case(cuda_lib, dc, True, scores=s)
 
 
