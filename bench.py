@@ -717,11 +717,29 @@ def bench_paged(S, torch, dev, stream, flush, t, cfg, use_gates, reps, P=16):
             "equals_contiguous_decode": same}
 
 
+def _time_us(torch, stream, flush, reps, fn):
+    """Median device time (µs) of fn() on `stream`: 3 untimed calls, then
+    `reps` calls, each after an L2 flush and a head start of the stream."""
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+    for i in range(reps + 3):
+        flush.zero_()
+        torch.cuda._sleep(HEAD_START_CYCLES)
+        ev = evs[i - 3] if i >= 3 else None
+        if ev:
+            ev[0].record(stream)
+        fn()
+        if ev:
+            ev[1].record(stream)
+    torch.cuda.synchronize()
+    return 1e3 * statistics.median(a.elapsed_time(b) for a, b in evs)
+
+
 def bench_selector_step(S, torch, dev, stream, flush, t, cfg, use_gates, reps):
     """The decode step with the weight-free block selector in front: the
     scores of q against the history blocks' mean keys (kept per block, so
     computed once here, as a serving loop would keep them), then the fused
-    selection and decode."""
+    selection and decode; and the same step as one call that forms the
+    scores itself (sas_decode_select_pooled)."""
     kbar = S.block_summaries(t["kc"], cfg.b, L=cfg.L)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
     for i in range(reps + 3):
@@ -739,9 +757,12 @@ def bench_selector_step(S, torch, dev, stream, flush, t, cfg, use_gates, reps):
     torch.cuda.synchronize(dev)
     sel = 1e3 * statistics.median(e[0].elapsed_time(e[1]) for e in evs)
     step = 1e3 * statistics.median(e[0].elapsed_time(e[2]) for e in evs)
+    pooled = _time_us(torch, stream, flush, reps, lambda: S.decode_select_pooled(
+        t["q"], t["kc"], t["vc"], kbar, cfg.K, use_gates, cfg.b, L=cfg.L))
     del kbar
-    return {"selector_scores_us": sel, "step_us": step,
-            "step": "sas_selector_scores_decode + sas_decode_select",
+    return {"selector_scores_us": sel, "two_call_step_us": step, "step_us": pooled,
+            "step": "sas_decode_select_pooled (scores, selection and decode in one call)",
+            "two_call_step": "sas_selector_scores_decode + sas_decode_select",
             "block_summaries": "computed once (a serving loop adds one per filled block)"}
 
 

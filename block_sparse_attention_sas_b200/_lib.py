@@ -56,6 +56,9 @@ SIGNATURES = {
     "sas_decode_select_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "sas_decode_select": (_i, [_i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p,
                                _p, _p, _sz, _p]),
+    "sas_decode_select_pooled_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "sas_decode_select_pooled": (_i, [_i, _p, _p, _p, _p, _f, _i, _i, _i, _i, _i, _i, _i, _i, _i,
+                                      _f, _p, _p, _p, _p, _sz, _p]),
     "sas_decode_noalloc": (_i, [_i, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                                 _p, _p]),
     "sas_decode_noalloc_max_scratch": (_sz, []),
@@ -308,6 +311,37 @@ def decode_select(q, kcache, vcache, scores, K: int, use_gates: bool, b: int,
                                  int(use_gates), B, Hq, Hkv, L, Lcap, d, b, K, scale, _ptr(o),
                                  _ptr(gates), _ptr(idx), _ptr(ws), ws.numel(),
                                  _stream(q.device)))
+    return o
+
+
+def decode_select_pooled(q, kcache, vcache, kbar, K: int, use_gates: bool, b: int,
+                         L: int | None = None, scale: float = 0.0, sel_scale: float = 0.0,
+                         o=None, gates=None, idx=None):
+    """decode_select with the pooled selector's scores formed from the key
+    summaries kbar [B,Hkv,C,d] (fp32) and the query: one launch where the
+    shape allows."""
+    for n, t in (("q", q), ("kcache", kcache), ("vcache", vcache)):
+        _need(t, n, q.dtype)
+    B, Hq, d = q.shape
+    Hkv, Lcap = kcache.shape[1], kcache.shape[2]
+    L = Lcap if L is None else L
+    if kbar is not None:  # None: the library reports the missing summaries
+        _need(kbar, "kbar", torch.float32)
+        if tuple(kbar.shape) != (B, Hkv, (L - 1) // b, d):
+            raise ValueError(f"kbar must be [B, Hkv, (L-1)//b, d], got {tuple(kbar.shape)}")
+    if o is None:
+        o = torch.empty_like(q)
+    if gates is not None:
+        _need(gates, "gates", torch.float32)
+    if idx is not None:
+        _need(idx, "idx", torch.int32)
+    nbytes = LIB.sas_decode_select_pooled_workspace_size(B, Hq, Hkv, L, d, b, K)
+    ws = _workspace("decode_select", nbytes, q.device, zero=False)
+    _check("sas_decode_select_pooled",
+           LIB.sas_decode_select_pooled(_dtype(q), _ptr(q), _ptr(kcache), _ptr(vcache),
+                                        _ptr(kbar), sel_scale, int(use_gates), B, Hq, Hkv, L,
+                                        Lcap, d, b, K, scale, _ptr(o), _ptr(gates), _ptr(idx),
+                                        _ptr(ws), ws.numel(), _stream(q.device)))
     return o
 
 

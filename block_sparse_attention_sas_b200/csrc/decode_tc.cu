@@ -91,6 +91,7 @@ struct Ctl {
   int Lseq;  // tokens of this unit's sequence
   // Running max (log2 domain) and sum of this split's partial per head.
   float2 part_ml[kMaxG];  // (max, sum) per head
+  uint64_t sel_full[3];   // the pooled selector's staged key summaries
 };
 constexpr size_t kSmem = kOffCtl + sizeof(Ctl) + 1024;
 static_assert(kOffCtl % 16 == 0 && offsetof(Ctl, part_o) % 16 == 0 && (kD * 4) % 16 == 0,
@@ -101,7 +102,12 @@ static_assert(kOffCtl % 16 == 0 && offsetof(Ctl, part_o) % 16 == 0 && (kD * 4) %
 // K/V ring, which no load touches before the block lists exist.
 struct SelArgs {
   bool on;              // select in the launch (else idx / gates are given)
-  const float* scores;  // [B * Hkv][C] selector scores (null when C == 0)
+  const float* scores;  // [B * Hkv][C] selector scores (null when C == 0, or pooled)
+  // Pooled selector (kbar != nullptr): the scores are formed in the launch,
+  // s_m = sel_scale * qbar . kbar_m, qbar the mean of the unit's query heads.
+  const float* kbar;          // [B * Hkv][C][128] fp32 block means, 16-byte aligned
+  const __nv_bfloat16* q;     // [B * Hq][128]
+  float sel_scale;
   float* gates_out;     // [B * Hkv][C] or nullptr
   int32_t* idx_out;     // [B * Hkv][K] or nullptr
   int chunk;            // entries of the row per split (<= 512)
@@ -109,6 +115,16 @@ struct SelArgs {
 constexpr uint32_t kOffSelList = (sizeof(SelShared) + 127) & ~127u;  // from kOffKV
 static_assert(kOffSelList + 16 * 256 * 8 <= kStages * 32768,
               "the selection scratch and list fit in the K/V ring");
+// The pooled selector stages the key summaries of its entries through the
+// ring (free until the selection's first cluster barrier: no CTA touches
+// another's shared memory before it) in kSelBufs pieces of kSelRows rows,
+// then keeps qbar and the 512 scores after them.
+constexpr int kSelRows = 60;
+constexpr int kSelBufs = 3;
+constexpr uint32_t kSelPiece = kSelRows * kD * 4;
+constexpr uint32_t kOffSelScores = kSelBufs * kSelPiece;  // from kOffKV
+static_assert(kOffSelScores + (kD + 512) * 4 <= kStages * 32768 && kSelPiece % 16 == 0,
+              "the staged summaries, qbar and the scores fit in the K/V ring");
 
 template <int G, bool SEL>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -238,11 +254,78 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const float* srow = sa.scores + (long long)unit * C;
     float f[4];
     bool okf[4];
+    if (sa.kbar) {
+      // The pooled selector's scores of this split's entries: qbar (the mean
+      // of the unit's G query heads) against each block's mean key. The
+      // summaries arrive by bulk copies, up to three pieces in flight; a warp
+      // takes a row at a time, a lane four columns of it.
+      static_assert(kThreads == kD, "one thread per column of qbar");
+      float* qb = reinterpret_cast<float*>(base + kOffKV + kOffSelScores);
+      float* scr = qb + kD;
+      const float* kb = sa.kbar + ((long long)unit * C + lo) * kD;
+      const int here = max(0, min(sa.chunk, C - lo));
+      const int npieces = (here + kSelRows - 1) / kSelRows;
+      auto issue = [&](int p) {
+        const uint32_t bytes = (uint32_t)min(kSelRows, here - p * kSelRows) * kD * 4;
+        uint64_t* bar = &c.sel_full[p % kSelBufs];
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_g2s(base + kOffKV + (p % kSelBufs) * kSelPiece, kb + (long long)p * kSelRows * kD,
+                 bytes, bar);
+      };
+      if (tid == 0) {
+        for (int i = 0; i < kSelBufs; ++i) mbar_init(&c.sel_full[i], 1);
+        fence_mbar_init();
+        for (int p = 0; p < min(kSelBufs, npieces); ++p) issue(p);
+      }
+      {
+        float a = 0.f;
+        for (int g = 0; g < G; ++g) a += __bfloat162float(sa.q[(hbase + g) * kD + tid]);
+        qb[tid] = a / (float)G;
+      }
+      __syncthreads();
+      const float4 qv = reinterpret_cast<const float4*>(qb)[lane];
+      for (int p = 0; p < npieces; ++p) {
+        const int rows = min(kSelRows, here - p * kSelRows);
+        if (!mbar_wait(ctx, &c.sel_full[p % kSelBufs], (p / kSelBufs) & 1)) *abort = 1;
+        const float4* buf =
+            reinterpret_cast<const float4*>(base + kOffKV + (p % kSelBufs) * kSelPiece);
+        for (int r0 = warp * 4; r0 < rows; r0 += 4 * kWarps) {
+          float acc[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int i = lo + tid + kThreads * e;
-      okf[e] = i < C && i < lo + sa.chunk;
-      f[e] = okf[e] ? srow[i] : -INFINITY;
+          for (int u = 0; u < 4; ++u) {
+            const float4 v = r0 + u < rows ? buf[(r0 + u) * (kD / 4) + lane]
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+            float a = 0.f;  // the standalone selector kernel's order of terms
+            a = fmaf(qv.x, v.x, a);
+            a = fmaf(qv.y, v.y, a);
+            a = fmaf(qv.z, v.z, a);
+            acc[u] = fmaf(qv.w, v.w, a);
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float a = warp_sum(acc[u]);
+            if (lane == 0 && r0 + u < rows) scr[p * kSelRows + r0 + u] = a * sa.sel_scale;
+          }
+        }
+        __syncthreads();  // every read of the piece is done: its buffer takes the next
+        if (tid == 0 && p + kSelBufs < npieces) {
+          fence_proxy_async_smem();
+          issue(p + kSelBufs);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = lo + tid + kThreads * e;
+        okf[e] = i < C && i < lo + sa.chunk;
+        f[e] = okf[e] ? scr[tid + kThreads * e] : -INFINITY;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = lo + tid + kThreads * e;
+        okf[e] = i < C && i < lo + sa.chunk;
+        f[e] = okf[e] ? srow[i] : -INFINITY;
+      }
     }
     float lse = 0.f;
     if (kk > 0) {  // the same in every split of the unit
@@ -814,14 +897,14 @@ cudaError_t launch_decode_tc(const DecodeShape& s, const void* q, const void* kc
   if ((e = make_tmap_bf16_pitched(&tk, kc, s.L, s.Lcap, s.B * s.Hkv)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16_pitched(&tv, vc, s.L, s.Lcap, s.B * s.Hkv)) != cudaSuccess) return e;
   const PagedArgs none = {nullptr, nullptr, nullptr, 0, 0};
-  const SelArgs nosel = {false, nullptr, nullptr, nullptr, 0};
+  const SelArgs nosel = {false, nullptr, nullptr, nullptr, 0.f, nullptr, nullptr, 0};
   return launch_tc_maps(s, tq, tk, tv, none, idx, gates, o, ws, nosel, ctx, st);
 }
 
 cudaError_t launch_decode_select_tc(const DecodeShape& s0, const void* q, const void* kc,
-                                    const void* vc, const float* scores, float* gates_out,
-                                    int32_t* idx_out, void* o, void* ws, const DevCtx& ctx,
-                                    cudaStream_t st) {
+                                    const void* vc, const float* scores, const float* kbar,
+                                    float sel_scale, float* gates_out, int32_t* idx_out, void* o,
+                                    void* ws, const DevCtx& ctx, cudaStream_t st) {
   // A row longer than 512 entries a split widens the cluster: the extra
   // CTAs (slot ranges past the last slot) help select and stream nothing.
   DecodeShape s = s0;
@@ -834,7 +917,8 @@ cudaError_t launch_decode_select_tc(const DecodeShape& s0, const void* q, const 
   if ((e = make_tmap_bf16_pitched(&tk, kc, s.L, s.Lcap, s.B * s.Hkv)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16_pitched(&tv, vc, s.L, s.Lcap, s.B * s.Hkv)) != cudaSuccess) return e;
   const PagedArgs none = {nullptr, nullptr, nullptr, 0, 0};
-  const SelArgs sa = {true, scores, gates_out, idx_out, (s.C + s.splits - 1) / s.splits};
+  const SelArgs sa = {true,      scores,  kbar,    (const __nv_bfloat16*)q, sel_scale,
+                      gates_out, idx_out, (s.C + s.splits - 1) / s.splits};
   return launch_tc_maps(s, tq, tk, tv, none, nullptr, nullptr, o, ws, sa, ctx, st);
 }
 
@@ -851,7 +935,7 @@ cudaError_t launch_decode_paged_tc(const DecodeShape& s, const PagedArgs& pa, co
     return e;
   if ((e = make_tmap_bf16_box(&tv, vpages, pa.P, pa.num_pages * s.Hkv, rows)) != cudaSuccess)
     return e;
-  const SelArgs nosel = {false, nullptr, nullptr, nullptr, 0};
+  const SelArgs nosel = {false, nullptr, nullptr, nullptr, 0.f, nullptr, nullptr, 0};
   return launch_tc_maps(s, tq, tk, tv, pa, idx, gates, o, ws, nosel, ctx, st);
 }
 

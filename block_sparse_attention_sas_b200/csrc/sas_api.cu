@@ -391,37 +391,88 @@ size_t sas_decode_select_workspace_size(int B, int Hq, int Hkv, int L, int d, in
   return select_ws_parts(make_decode(B, Hq, Hkv, L, L, d, b, K, 1.f, false, 0), &og, &oi);
 }
 
-sas_status_t sas_decode_select(sas_dtype_t dtype, const void* q, const void* kcache,
-                               const void* vcache, const float* scores, int use_gates, int B,
-                               int Hq, int Hkv, int L, int Lcap, int d, int b, int K, float scale,
-                               void* o, float* gates, int32_t* idx, void* ws, size_t ws_bytes,
-                               sas_stream_t stream) {
+// The fused step and its two-launch fallback. kbar (nullable): the scores
+// are the pooled selector's, formed in the launch (or, on the fallback, by
+// the selector kernel into the workspace's scores part at off_s).
+static sas_status_t decode_select_impl(sas_dtype_t dtype, const void* q, const void* kcache,
+                                       const void* vcache, const float* scores, const float* kbar,
+                                       float sel_scale, size_t off_s, int use_gates, int B,
+                                       int Hq, int Hkv, int L, int Lcap, int d, int b, int K,
+                                       float scale, void* o, float* gates, int32_t* idx, void* ws,
+                                       size_t ws_bytes, sas_stream_t stream) {
   sas_status_t st = check_decode(dtype, B, Hq, Hkv, L, Lcap, d, b, K, false, scale);
   if (st != SAS_OK) return st;
   if (B == 0) return SAS_OK;
   const int C = (L - 1) / b;
-  if (!q || !kcache || !vcache || !o || (!scores && C > 0)) return SAS_ERR_INVALID_ARG;
+  if (!q || !kcache || !vcache || !o || (!scores && !kbar && C > 0)) return SAS_ERR_INVALID_ARG;
   if (C > 262144) return SAS_ERR_UNSUPPORTED;
   if (!aligned(q, 16) || !aligned(kcache, 16) || !aligned(vcache, 16) || !aligned(o, 16) ||
-      (scores && !aligned(scores, 4)) || (gates && !aligned(gates, 4)) || (idx && !aligned(idx, 4)))
+      (scores && !aligned(scores, 4)) || (kbar && !aligned(kbar, 4)) ||
+      (gates && !aligned(gates, 4)) || (idx && !aligned(idx, 4)))
     return SAS_ERR_INVALID_ARG;
   const DecodeShape s = make_decode(B, Hq, Hkv, L, Lcap, d, b, K, scale, false, use_gates);
   size_t og, oi;
-  const size_t need = select_ws_parts(s, &og, &oi);
+  const size_t need = select_ws_parts(s, &og, &oi) +
+                      (kbar ? (((size_t)B * Hkv * C * sizeof(float) + 255) & ~(size_t)255) : 0);
   if (!ws || ws_bytes < need || !aligned(ws, 256)) return SAS_ERR_WORKSPACE;
   DevCtx ctx;
   if (device_ctx(ctx) != cudaSuccess) return SAS_ERR_CUDA;
-  if (tc_decode_supported(dtype, s)) {
-    const cudaError_t e =
-        launch_decode_select_tc(s, q, kcache, vcache, scores, gates, idx, o, ws, ctx, stream);
+  if (tc_decode_supported(dtype, s) && (!kbar || aligned(kbar, 16))) {
+    const cudaError_t e = launch_decode_select_tc(s, q, kcache, vcache, scores, kbar, sel_scale,
+                                                  gates, idx, o, ws, ctx, stream);
     if (e != cudaErrorNotSupported) return cuda_status(e);
   }
-  // Two launches: the gates and Top-K of the rows, then the decode.
+  // Two or three launches: the pooled selector's scores (when asked for),
+  // the gates and Top-K of the rows, then the decode.
+  if (kbar && C > 0) {
+    float* sc = reinterpret_cast<float*>(static_cast<char*>(ws) + off_s);
+    const cudaError_t e = launch_selector_scores_decode(dtype, q, kbar, B * Hkv, Hq / Hkv, C, d,
+                                                        sel_scale, sc, stream);
+    if (e != cudaSuccess) return cuda_status(e);
+    scores = sc;
+  }
   float* g = gates ? gates : reinterpret_cast<float*>(static_cast<char*>(ws) + og);
   int32_t* ix = idx ? idx : reinterpret_cast<int32_t*>(static_cast<char*>(ws) + oi);
   cudaError_t e = launch_gate_topk(scores, B, Hkv, 1, C, 0, K, SAS_PHI_SOFTMAX, g, ix, stream);
   if (e != cudaSuccess) return cuda_status(e);
   return cuda_status(launch_decode(dtype, s, q, kcache, vcache, ix, g, o, ws, ctx, stream));
+}
+
+sas_status_t sas_decode_select(sas_dtype_t dtype, const void* q, const void* kcache,
+                               const void* vcache, const float* scores, int use_gates, int B,
+                               int Hq, int Hkv, int L, int Lcap, int d, int b, int K, float scale,
+                               void* o, float* gates, int32_t* idx, void* ws, size_t ws_bytes,
+                               sas_stream_t stream) {
+  return decode_select_impl(dtype, q, kcache, vcache, scores, nullptr, 0.f, 0, use_gates, B, Hq,
+                            Hkv, L, Lcap, d, b, K, scale, o, gates, idx, ws, ws_bytes, stream);
+}
+
+size_t sas_decode_select_pooled_workspace_size(int B, int Hq, int Hkv, int L, int d, int b, int K) {
+  if (check_decode(SAS_BF16, B, Hq, Hkv, L, L, d, b, K, false, 1.f) != SAS_OK) return 0;
+  size_t og, oi;
+  const DecodeShape s = make_decode(B, Hq, Hkv, L, L, d, b, K, 1.f, false, 0);
+  return select_ws_parts(s, &og, &oi) +
+         (((size_t)B * Hkv * s.C * sizeof(float) + 255) & ~(size_t)255);
+}
+
+sas_status_t sas_decode_select_pooled(sas_dtype_t dtype, const void* q, const void* kcache,
+                                      const void* vcache, const float* kbar, float sel_scale,
+                                      int use_gates, int B, int Hq, int Hkv, int L, int Lcap, int d,
+                                      int b, int K, float scale, void* o, float* gates,
+                                      int32_t* idx, void* ws, size_t ws_bytes,
+                                      sas_stream_t stream) {
+  const sas_status_t st = check_decode(dtype, B, Hq, Hkv, L, Lcap, d, b, K, false, scale);
+  if (st != SAS_OK) return st;
+  if (!isfinite(sel_scale)) return SAS_ERR_INVALID_ARG;
+  if (B == 0) return SAS_OK;
+  if ((L - 1) / b > 0 && !kbar) return SAS_ERR_INVALID_ARG;
+  if ((long long)B * Hkv > 65535) return SAS_ERR_UNSUPPORTED;  // the selector kernel's grid
+  size_t og, oi;
+  const size_t off_s = select_ws_parts(make_decode(B, Hq, Hkv, L, Lcap, d, b, K, 1.f, false, 0),
+                                       &og, &oi);
+  return decode_select_impl(dtype, q, kcache, vcache, nullptr, kbar, resolve_scale(sel_scale, d),
+                            off_s, use_gates, B, Hq, Hkv, L, Lcap, d, b, K, scale, o, gates, idx,
+                            ws, ws_bytes, stream);
 }
 
 sas_status_t sas_decode_noalloc(sas_dtype_t dtype, const void* q, const void* kcache,

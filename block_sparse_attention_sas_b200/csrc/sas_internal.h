@@ -108,10 +108,12 @@ bool tc_decode_supported(sas_dtype_t dt, const DecodeShape& s);
 // scores [B * Hkv][C] computed in the same launch (softmax gates); gates_out /
 // idx_out may be null. cudaErrorNotSupported when the shape does not allow
 // it (a unit's row must fit its splits' cluster, 512 entries a split).
+// kbar (nullable, with sel_scale): the scores come from the pooled selector
+// in the same launch (scores is then unused).
 cudaError_t launch_decode_select_tc(const DecodeShape& s, const void* q, const void* kc,
-                                    const void* vc, const float* scores, float* gates_out,
-                                    int32_t* idx_out, void* o, void* ws, const DevCtx& ctx,
-                                    cudaStream_t st);
+                                    const void* vc, const float* scores, const float* kbar,
+                                    float sel_scale, float* gates_out, int32_t* idx_out, void* o,
+                                    void* ws, const DevCtx& ctx, cudaStream_t st);
 cudaError_t launch_decode_tc(const DecodeShape& s, const void* q, const void* kc, const void* vc,
                              const int32_t* idx, const float* gates, void* o, void* ws,
                              const DevCtx& ctx, cudaStream_t stream);

@@ -300,6 +300,33 @@ sas_status_t sas_decode_select(sas_dtype_t dtype, const void* q, const void* kca
                                sas_stream_t stream);
 
 /*
+ * sas_decode_select_pooled - sas_decode_select whose scores are the
+ * weight-free pooled selector's (sas_selector_scores_decode below), formed
+ * from the key summaries instead of being passed in:
+ *   scores[b, kvh, m] = sel_scale * qbar . kbar[b, kvh, m],
+ *   qbar = the mean of q over the group's G heads; sel_scale <= 0 selects
+ *   1/sqrt(d).
+ * Equal to sas_selector_scores_decode followed by sas_decode_select.
+ *   kbar [B][Hkv][C][d] fp32 (sas_block_summaries' output; may be NULL when
+ *   C == 0). The other arguments are those of sas_decode_select; ws: at
+ *   least sas_decode_select_pooled_workspace_size(B, Hq, Hkv, L, d, b, K)
+ *   bytes, 256-byte aligned, owned by the caller.
+ * Where sas_decode_select runs in one launch and kbar is 16-byte aligned,
+ * the scores are formed in that launch too: each split of the cluster scores
+ * its own entries of the row before the selection. Otherwise the selector
+ * kernel writes them into the workspace first.
+ * Errors: those of sas_decode_select and sas_selector_scores_decode
+ * (B x Hkv > 65535 is SAS_ERR_UNSUPPORTED).
+ */
+size_t sas_decode_select_pooled_workspace_size(int B, int Hq, int Hkv, int L, int d, int b, int K);
+sas_status_t sas_decode_select_pooled(sas_dtype_t dtype, const void* q, const void* kcache,
+                                      const void* vcache, const float* kbar, float sel_scale,
+                                      int use_gates, int B, int Hq, int Hkv, int L, int Lcap, int d,
+                                      int b, int K, float scale, void* o, float* gates,
+                                      int32_t* idx, void* ws, size_t ws_bytes,
+                                      sas_stream_t stream);
+
+/*
  * sas_decode_noalloc - sas_decode for callers that cannot allocate device
  * memory. Some callers cannot call cudaMalloc or take a workspace from their
  * framework at the point where they decode: an inference server or plugin
