@@ -824,13 +824,17 @@ def run_profile_decode(args):
     sc = torch.from_numpy(x.scores).to(dev)
     del x
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    kbar = S.block_summaries(kc, cfg.b, L=cfg.L) if args.pooled else None
     for _ in range(args.warmup + args.steps):
         flush.zero_()
-        S.decode_select(q, kc, vc, sc, cfg.K, True, cfg.b, L=cfg.L)
+        if args.pooled:
+            S.decode_select_pooled(q, kc, vc, kbar, cfg.K, True, cfg.b, L=cfg.L)
+        else:
+            S.decode_select(q, kc, vc, sc, cfg.K, True, cfg.b, L=cfg.L)
     torch.cuda.synchronize(dev)
     st, raw = S.device_error()
-    print(json.dumps({"profile_decode": cfg.name, "steps": args.warmup + args.steps,
-                      "device_error": st}), flush=True)
+    print(json.dumps({"profile_decode": cfg.name, "pooled": bool(args.pooled),
+                      "steps": args.warmup + args.steps, "device_error": st}), flush=True)
     if st != 0:
         raise SystemExit(1)
 
@@ -918,6 +922,9 @@ def main():
     ap.add_argument("--profile-decode", default=None, metavar="PRESET",
                     help="only run the decode step (sas_decode_select) warmup + steps times, "
                          "untimed, for kernel captures")
+    ap.add_argument("--pooled", action="store_true",
+                    help="with --profile-decode: sas_decode_select_pooled (the selector's "
+                         "scores formed in the launch from the block means)")
     ap.add_argument("--no-8b", action="store_true", help="skip the Qwen3-8B training line")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense training line")
     ap.add_argument("--dry-run", action="store_true",
