@@ -1257,25 +1257,38 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
       }
     }
+    // Epilogue: thread rowi holds dimension d = rowi; group grp the keys
+    // 32 grp .. 32 grp + 31. The key block's dV and dK rows are contiguous
+    // 16 KB ranges of dv and dk, so they are staged as [key][d] bf16 tiles in
+    // the first Q/dO stage (no MMA reads it after acc_done, no load fills it)
+    // and leave in two bulk copies. Every elementwise warp reaches the
+    // barrier; the copies go only when no wait of the CTA gave up.
+    unsigned char* st_dv = base + kOffQD;
+    unsigned char* st_dk = base + kOffQD + 16384;
     if (ok && warp_wait(ctx, &c.acc_done, 0, abort)) {
-      // Epilogue: thread rowi holds dimension d = rowi; group g the keys 32g .. 32g + 31.
       fence_after_sync();
       const int d = rowi;
-      const long long kb0 = ((long long)bh * s.T + (long long)m * kB) * kD;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
-        __nv_bfloat16* out = which == 0 ? dv : dk;
+        __nv_bfloat16* t = reinterpret_cast<__nv_bfloat16*>(which == 0 ? st_dv : st_dk);
         const float mul = which == 0 ? 1.f : s.scale;
         uint32_t v[32];
         tmem_ld32(tl + (which == 0 ? kColDV : kColDK) + grp * 32, v);
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int key = grp * 32 + i;
-          if (i < kvalid) out[kb0 + (long long)key * kD + d] =
-              __float2bfloat16_rn(__uint_as_float(v[i]) * mul);
-        }
+        for (int i = 0; i < 32; ++i)
+          t[(grp * 32 + i) * kD + d] = __float2bfloat16_rn(__uint_as_float(v[i]) * mul);
       }
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(1, 32 * 8);
+    if (warp == 4 && lane == 0 && *abort == 0) {
+      const long long kb0 = ((long long)bh * s.T + (long long)m * kB) * kD;
+      const uint32_t bytes = (uint32_t)min(kB, s.T - m * kB) * kD * 2;
+      bulk_s2g(dv + kb0, st_dv, bytes);
+      bulk_s2g(dk + kb0, st_dk, bytes);
+      bulk_commit();
+      bulk_wait_read_all();
     }
   }
   fence_before_sync();

@@ -202,6 +202,12 @@ __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// Barrier `id` (1..15; 0 is __syncthreads') among `nthreads` threads of the
+// CTA, whole warps, every one of which must reach it.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // Prefetch one tile of a 3D tensor map into L2: no shared-memory destination
 // and no completion to wait for (a later load of the same tile hits L2).
 __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2) {
