@@ -53,13 +53,13 @@ HEAD_START_CYCLES = 2_000_000
 # DRAM bytes (read + write) per call from ncu (dram__bytes_read.sum +
 # dram__bytes_write.sum summed over the call's kernels, one --set full capture
 # each of `bench.py --profile-train 8192`), for the kernels as they stand:
-# the backward with the residual D pass is D-from-o 206.1 MB, dK/dV 1241.5 MB
+# the backward with the residual D pass is D-from-o 206.1 MB, dK/dV 1229.5 MB
 # and dq 608.6 MB per call at T = 8192. The capture ran the same layer at
 # T = 8192; the figure is scaled to T = 16384 by the attended pairs
 # (536.1 M / 259.1 M), which every kernel's work follows.
 MEASURED_TRAFFIC = {
     ("qwen3-4b-train B1 Hq32/Hkv8 T16384 d128 b64 K16", "sas_attn_bwd_res"):
-        (206.1e6 + 1241.5e6 + 608.6e6) * 536084480 / 259129344,
+        (206.1e6 + 1229.5e6 + 608.6e6) * 536084480 / 259129344,
 }
 
 
