@@ -91,6 +91,38 @@ __device__ __forceinline__ float gate_of(float sc, float lse, int phi) {
 constexpr int kWarpRowsPerCta = 8;
 constexpr int kWarpCap = 512;   // longest row handled by one warp
 constexpr int kMaxK = 256;
+constexpr int kArgmaxMaxK = 64;  // largest K taken by rounds of warp argmax
+
+// Small K: the k largest of a row of n <= 32 E entries by k rounds of warp
+// argmax. Each lane holds E composite keys, the score's order-preserving key
+// above the complement of the index, so the larger composite is the higher
+// score and, among equal scores, the lower index; no two entries share one,
+// and round t yields the entry of rank t. Empty slots hold 0, below every
+// composite of a valid entry (whose low word is at least ~511).
+template <int E>
+__device__ __forceinline__ void warp_argmax_topk(const float* v, int n, int k, int lane,
+                                                 int32_t* out) {
+  uint64_t key[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = lane + 32 * e;
+    key[e] = i < n ? ((uint64_t)fkey(v[i]) << 32) | (uint64_t)(~(uint32_t)i) : 0ull;
+  }
+  for (int t = 0; t < k; ++t) {
+    uint64_t m = key[0];
+#pragma unroll
+    for (int e = 1; e < E; ++e) m = key[e] > m ? key[e] : m;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const uint64_t o = __shfl_xor_sync(0xffffffffu, m, off);
+      m = o > m ? o : m;
+    }
+    if (lane == 0) out[t] = (int32_t)(~(uint32_t)m);
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+      if (key[e] == m) key[e] = 0ull;
+  }
+}
 
 // ---------------------------------------------------------------------------
 // One warp per row.
@@ -130,7 +162,13 @@ gate_topk_warp_kernel(const float* __restrict__ scores, int total_rows, int rows
   for (int i = lane; i < C; i += 32) g[i] = (i < n) ? gate_of(v[i], lse, phi) : 0.f;
 
   const int k = min(K, n);
-  if (k > 0) {
+  if (k > 0 && K <= kArgmaxMaxK) {
+    __syncwarp();  // the row's scores in v are visible to every lane
+    if (n <= 256)
+      warp_argmax_topk<8>(v, n, k, lane, out);
+    else
+      warp_argmax_topk<16>(v, n, k, lane, out);
+  } else if (k > 0) {
     // ---- tau = k-th largest key: radix select, four 8-bit digits
     int* hist = s_hist[w];
     uint32_t tau = 0, mask = 0;
