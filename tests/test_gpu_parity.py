@@ -81,6 +81,11 @@ def test_gate_topk_decode_configs(cuda_lib, name):
     # decode-sized rows (warp-threshold path): 1, 2, 4 and 8 warps per row, ties
     (1023, 32, False, 0), (8191, 64, False, 0), (4096, 64, False, 1), (1800, 64, True, 0),
     (600, 1, False, 3), (7000, 33, False, 2),
+    # rows of one warp on either side of the argmax path's K bound (K <= 64:
+    # rounds of warp argmax; K = 65: the radix select), with ties, and a
+    # full 512-entry row (16 keys a lane)
+    (300, 64, True, 2), (300, 65, True, 2), (257, 64, True, 3), (512, 64, False, 0),
+    (512, 17, False, 2),
 ])
 def test_gate_topk_edges(cuda_lib, C, K, causal, levels):
     rng = np.random.default_rng(C * 7 + K)

@@ -133,6 +133,26 @@ def test_decode_select_pooled(cuda_lib, kw, use_gates):
     _pooled_case(cuda_lib, W.small_decode_config(**kw), use_gates)
 
 
+def test_decode_select_pooled_unaligned_kbar(cuda_lib):
+    """Key summaries that are not 16-byte aligned take the three-launch
+    path (the selector kernel, then the selection and the decode); the
+    results equal the fused call's."""
+    dc = W.small_decode_config(B=2, Hq=8, Hkv=2, L=5000, d=128, b=64, K=16, dtype="bf16")
+    x = W.make_decode_inputs(dc)
+    q, kc, vc = (dev(a, dc.dtype) for a in (x.q, x.kcache, x.vcache))
+    kbar = cuda_lib.block_summaries(kc, dc.b, L=dc.L)
+    store = torch.empty(kbar.numel() + 1, dtype=torch.float32, device="cuda")
+    shifted = store[1:].view(kbar.shape)  # 4 bytes past a 16-byte boundary
+    shifted.copy_(kbar)
+    assert shifted.data_ptr() % 16 == 4
+    ix1 = torch.empty((dc.B, dc.Hkv, dc.K), dtype=torch.int32, device="cuda")
+    ix2 = torch.empty_like(ix1)
+    o1 = cuda_lib.decode_select_pooled(q, kc, vc, kbar, dc.K, True, dc.b, L=dc.L, idx=ix1)
+    o2 = cuda_lib.decode_select_pooled(q, kc, vc, shifted, dc.K, True, dc.b, L=dc.L, idx=ix2)
+    torch.cuda.synchronize()
+    assert torch.equal(ix1, ix2) and torch.equal(o1, o2)
+
+
 def test_decode_select_pooled_rejects(cuda_lib):
     """A missing kbar with history, a non-finite selector scale and a kbar of
     the wrong shape are argument errors raised before any launch."""
