@@ -251,7 +251,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     SelShared& sh = *reinterpret_cast<SelShared*>(base + kOffKV);
     uint64_t* list = reinterpret_cast<uint64_t*>(base + kOffKV + kOffSelList);
     const int lo = split * sa.chunk;
-    const float* srow = sa.scores + (long long)unit * C;
     float f[4];
     bool okf[4];
     if (sa.kbar) {
@@ -320,6 +319,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         f[e] = okf[e] ? scr[tid + kThreads * e] : -INFINITY;
       }
     } else {
+      const float* srow = C > 0 ? sa.scores + (long long)unit * C : nullptr;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int i = lo + tid + kThreads * e;
