@@ -673,6 +673,23 @@ def bench_decode(S, torch, dev, stream, flush, peaks, args, rank):
     return out
 
 
+def paged_copy(torch, dev, kc, vc, cfg, P=16):
+    """A paged copy of contiguous caches [B, Hkv, L, d]: P-token pages placed
+    in a seeded random order, with their page table and lengths."""
+    B, Hkv, L, d = kc.shape
+    npp = L // P
+    perm = torch.randperm(B * npp, generator=torch.Generator().manual_seed(cfg.seed + 17))
+    kp = torch.empty((B * npp, Hkv, P, d), dtype=kc.dtype, device=dev)
+    vp = torch.empty_like(kp)
+    pd = perm.to(dev)
+    kp[pd] = kc.view(B, Hkv, npp, P, d).permute(0, 2, 1, 3, 4).reshape(B * npp, Hkv, P, d)
+    vp[pd] = vc.view(B, Hkv, npp, P, d).permute(0, 2, 1, 3, 4).reshape(B * npp, Hkv, P, d)
+    indptr = torch.arange(0, B * npp + 1, npp, dtype=torch.int32, device=dev)
+    indices = pd.to(torch.int32)
+    lens = torch.full((B,), cfg.L, dtype=torch.int32, device=dev)
+    return kp, vp, indptr, indices, lens
+
+
 def bench_paged(S, torch, dev, stream, flush, t, cfg, use_gates, reps, P=16):
     """The same decode over a paged copy of the caches (P-token pages placed
     in a seeded random order): sas_decode_paged with the same selection,
@@ -680,15 +697,7 @@ def bench_paged(S, torch, dev, stream, flush, t, cfg, use_gates, reps, P=16):
     one."""
     B, Hkv, L, d = t["kc"].shape
     npp = L // P
-    perm = torch.randperm(B * npp, generator=torch.Generator().manual_seed(cfg.seed + 17))
-    kp = torch.empty((B * npp, Hkv, P, d), dtype=t["kc"].dtype, device=dev)
-    vp = torch.empty_like(kp)
-    pd = perm.to(dev)
-    kp[pd] = t["kc"].view(B, Hkv, npp, P, d).permute(0, 2, 1, 3, 4).reshape(B * npp, Hkv, P, d)
-    vp[pd] = t["vc"].view(B, Hkv, npp, P, d).permute(0, 2, 1, 3, 4).reshape(B * npp, Hkv, P, d)
-    indptr = torch.arange(0, B * npp + 1, npp, dtype=torch.int32, device=dev)
-    indices = pd.to(torch.int32)
-    lens = torch.full((B,), cfg.L, dtype=torch.int32, device=dev)
+    kp, vp, indptr, indices, lens = paged_copy(torch, dev, t["kc"], t["vc"], cfg, P)
     gates, idx = S.gate_topk(t["s"], cfg.K, causal=False)
     ix, g = idx[:, :, 0].contiguous(), gates[:, :, 0].contiguous()
 
@@ -808,9 +817,10 @@ def run_profile_train(args):
 
 
 def run_profile_decode(args):
-    """The decode step of one preset (sas_decode_select, gates on), warm-up
-    plus `steps` calls with the L2 flushed before each, untimed, for kernel
-    captures."""
+    """The decode step of one preset, gates on, warm-up plus `steps` calls
+    with the L2 flushed before each, untimed, for kernel captures: the fused
+    step (sas_decode_select) by default, or the pooled call, the two-call
+    step with the standalone selector, or the paged decode."""
     import torch
     from block_sparse_attention_sas_b200 import _lib as S
     dev = torch.device("cuda", 0)
@@ -824,16 +834,27 @@ def run_profile_decode(args):
     sc = torch.from_numpy(x.scores).to(dev)
     del x
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    kbar = S.block_summaries(kc, cfg.b, L=cfg.L) if args.pooled else None
+    kbar = S.block_summaries(kc, cfg.b, L=cfg.L) if (args.pooled or args.two_call) else None
+    if args.paged:
+        kp, vp, indptr, indices, lens = paged_copy(torch, dev, kc, vc, cfg)
+        gates, idx = S.gate_topk(sc[:, :, None, :].contiguous(), cfg.K, causal=False)
+        ix, g = idx[:, :, 0].contiguous(), gates[:, :, 0].contiguous()
     for _ in range(args.warmup + args.steps):
         flush.zero_()
-        if args.pooled:
+        if args.paged:
+            S.decode_paged(q, kp, vp, indptr, indices, lens, ix, g, True, cfg.b, max_len=cfg.L)
+        elif args.pooled:
             S.decode_select_pooled(q, kc, vc, kbar, cfg.K, True, cfg.b, L=cfg.L)
+        elif args.two_call:
+            s2 = S.selector_scores_decode(q, kbar)
+            S.decode_select(q, kc, vc, s2, cfg.K, True, cfg.b, L=cfg.L)
         else:
             S.decode_select(q, kc, vc, sc, cfg.K, True, cfg.b, L=cfg.L)
     torch.cuda.synchronize(dev)
     st, raw = S.device_error()
-    print(json.dumps({"profile_decode": cfg.name, "pooled": bool(args.pooled),
+    mode = ("paged" if args.paged else "pooled" if args.pooled else
+            "two_call" if args.two_call else "fused")
+    print(json.dumps({"profile_decode": cfg.name, "mode": mode,
                       "steps": args.warmup + args.steps, "device_error": st}), flush=True)
     if st != 0:
         raise SystemExit(1)
@@ -925,6 +946,12 @@ def main():
     ap.add_argument("--pooled", action="store_true",
                     help="with --profile-decode: sas_decode_select_pooled (the selector's "
                          "scores formed in the launch from the block means)")
+    ap.add_argument("--two-call", action="store_true",
+                    help="with --profile-decode: sas_selector_scores_decode, then "
+                         "sas_decode_select")
+    ap.add_argument("--paged", action="store_true",
+                    help="with --profile-decode: sas_decode_paged over a paged copy of the "
+                         "caches (16-token pages in a seeded random order)")
     ap.add_argument("--no-8b", action="store_true", help="skip the Qwen3-8B training line")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense training line")
     ap.add_argument("--dry-run", action="store_true",
