@@ -382,6 +382,11 @@ def run_ours(args):
     if not args.no_dense:
         dense_line = run_dense_line(S, torch, dev, cfg, d, flush, peaks, step_ms)
 
+    # ---- the gate variants on the same layer
+    variant_lines = None
+    if not args.no_variants:
+        variant_lines = run_variant_lines(S, torch, dev, cfg, d, flush, peaks)
+
     # ---- roofline of the dominant call of the training step
     dom = max(k_ms, key=k_ms.get)
     dom_flops = {"sas_attn_fwd_res": f_fwd, "sas_attn_bwd_res": f_bwd}.get(dom, 0.0)
@@ -411,6 +416,7 @@ def run_ours(args):
         "decode": decode_lines,
         "train_other": other_train,
         "dense_train": dense_line,
+        "train_variants": variant_lines,
         "wall_s_timed": t_wall,
     }
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -541,6 +547,41 @@ def run_train_line(S, torch, dev, cfg, flush, peaks, steps, warmup, rank):
     return {"workload": cfg.name, "ms_per_step": ms, "gate_fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
             "TFLOP/s": tf, "frac": tf / peaks["bf16_tflops"],
             "algorithmic_tflop_per_step": (f_fwd + f_bwd) / 1e12}
+
+
+def run_variant_lines(S, torch, dev, cfg, d, flush, peaks):
+    """The training step of the same layer with the ablation variants' gates
+    (phi: sigmoid or raw logits; outer gating), through sas_gate_topk_phi,
+    sas_attn_fwd_gated and sas_attn_bwd_gated, device-timed (L2 flushed
+    before each step); the plain softmax / inner pair (sas_attn_fwd +
+    sas_attn_bwd) beside them on the same box."""
+    stream = torch.cuda.current_stream(dev)
+    f_fwd, f_bwd = train_flops(cfg)
+    out = []
+    for phi, gating in (("softmax", "inner"), ("sigmoid", "inner"), ("raw", "inner"),
+                        ("softmax", "outer")):
+        def one(ev=None):
+            if ev:
+                ev[0].record(stream)
+            gates, idx = S.gate_topk(d["scores"], cfg.K, causal=True, phi=phi)
+            o, lse = S.attn_fwd(d["q"], d["k"], d["v"], idx, gates, cfg.b, gating=gating)
+            S.attn_bwd(d["q"], d["k"], d["v"], o, lse, d["dO"], idx, gates, cfg.b, phi=phi,
+                       gating=gating)
+            if ev:
+                ev[1].record(stream)
+
+        one()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(3)]
+        for e in evs:
+            flush.zero_()
+            torch.cuda._sleep(HEAD_START_CYCLES)
+            one(e)
+        torch.cuda.synchronize(dev)
+        ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+        out.append({"phi": phi, "gating": gating, "ms_per_step": ms,
+                    "TFLOP/s": (f_fwd + f_bwd) / (ms * 1e-3) / 1e12})
+    return {"workload": cfg.name, "pair": "sas_attn_fwd(_gated) + sas_attn_bwd(_gated), D "
+            "recomputed (the residual pair takes softmax / inner gating only)", "lines": out}
 
 
 def run_dense_line(S, torch, dev, cfg, d, flush, peaks, sparse_ms):
@@ -953,6 +994,8 @@ def main():
                     help="with --profile-decode: sas_decode_paged over a paged copy of the "
                          "caches (16-token pages in a seeded random order)")
     ap.add_argument("--no-8b", action="store_true", help="skip the Qwen3-8B training line")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the gate-variant training lines")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense training line")
     ap.add_argument("--dry-run", action="store_true",
                     help="CPU only: exercise the rank launch and timing reduction on gloo")
