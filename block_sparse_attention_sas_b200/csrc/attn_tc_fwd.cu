@@ -437,46 +437,73 @@ __device__ __forceinline__ void tc_fwd_body(const CUtensorMap& tm_q, const CUten
       __syncwarp();
       if (lane == 0) mbar_arrive(&c.v_full[n % kStages]);  // P(n) is ready for PV(n)
     }
-    if (ok && t < TILES) {
-      // ---- epilogue: O / l and the log-sum-exp
+    if (t < TILES) {
+      // ---- epilogue: O / l and the log-sum-exp. Each head's 64 rows of o
+      // (and of o_res) are one contiguous 16 KB range, so the tile stages
+      // its rows as bf16 in shared memory that no MMA or load touches after
+      // the last PV (o in the tile's share of the Q area, o_res in the K/V
+      // rings) and writes each range with one bulk copy. A lane writes the
+      // four 16-byte chunks of a 64-byte group in a rotated order, so eight
+      // lanes of a phase spread over four bank groups. Every softmax warp of
+      // the tile reaches the barrier; the copies go only when no wait of the
+      // CTA gave up.
       const int nl = nblk - 1;
-      if (__all_sync(0xffffffffu, wait_or_abort(ctx, &c.pv_done, nl & 1, abort))) {
+      unsigned char* so = base + L::kOffQ + t * 32768 + rowi * 256;
+      unsigned char* sr = base + L::kOffK + t * 32768 + rowi * 256;
+      if (ok && __all_sync(0xffffffffu, wait_or_abort(ctx, &c.pv_done, nl & 1, abort))) {
         fence_after_sync();
         const float inv = 1.f / l;
-        const bool write = qrow < s.T;
-        const long long ooff = ((long long)(bi * s.Hq + head) * s.T + qrow) * kD;
-        __nv_bfloat16* orow = o + ooff;
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
           uint32_t ov[32];
           tmem_ld32(tl + L::o_col(t) + ch * 32, ov);
           tmem_ld_wait();
-          if (write) {
+          uint4 vo[4], vr[4];
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              float x[8];
+          for (int q4 = 0; q4 < 4; ++q4) {
+            float x[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(ov[8 * q4 + e]) * inv;
-              uint4 v;
-              v.x = pack_bf16(x[0], x[1]);
-              v.y = pack_bf16(x[2], x[3]);
-              v.z = pack_bf16(x[4], x[5]);
-              v.w = pack_bf16(x[6], x[7]);
-              *reinterpret_cast<uint4*>(orow + ch * 32 + q4 * 8) = v;
-              if (RES) {
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                uint32_t rr[4];
+            for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(ov[8 * q4 + e]) * inv;
+            vo[q4].x = pack_bf16(x[0], x[1]);
+            vo[q4].y = pack_bf16(x[2], x[3]);
+            vo[q4].z = pack_bf16(x[4], x[5]);
+            vo[q4].w = pack_bf16(x[6], x[7]);
+            if (RES) {
+              const uint32_t w[4] = {vo[q4].x, vo[q4].y, vo[q4].z, vo[q4].w};
+              uint32_t rr[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                  rr[e] = pack_bf16(x[2 * e] - __uint_as_float(w[e] << 16),
-                                    x[2 * e + 1] - __uint_as_float(w[e] & 0xffff0000u));
-                *reinterpret_cast<uint4*>(o_res + ooff + ch * 32 + q4 * 8) =
-                    make_uint4(rr[0], rr[1], rr[2], rr[3]);
-              }
+              for (int e = 0; e < 4; ++e)
+                rr[e] = pack_bf16(x[2 * e] - __uint_as_float(w[e] << 16),
+                                  x[2 * e + 1] - __uint_as_float(w[e] & 0xffff0000u));
+              vr[q4] = make_uint4(rr[0], rr[1], rr[2], rr[3]);
+            }
+          }
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const int q4 = (k4 + lane) & 3;
+            const uint4 a = q4 == 0 ? vo[0] : q4 == 1 ? vo[1] : q4 == 2 ? vo[2] : vo[3];
+            *reinterpret_cast<uint4*>(so + (ch * 4 + q4) * 16) = a;
+            if (RES) {
+              const uint4 b2 = q4 == 0 ? vr[0] : q4 == 1 ? vr[1] : q4 == 2 ? vr[2] : vr[3];
+              *reinterpret_cast<uint4*>(sr + (ch * 4 + q4) * 16) = b2;
             }
           }
         }
-        if (write) lse[(long long)(bi * s.Hq + head) * s.T + qrow] = (m_used + log2f(l)) * kLn2;
+        if (qrow < s.T)
+          lse[(long long)(bi * s.Hq + head) * s.T + qrow] = (m_used + log2f(l)) * kLn2;
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1 + t, 128);
+      if (rowi == 0 && *abort == 0) {
+        const uint32_t bytes = (uint32_t)min(kB, s.T - j * kB) * kD * 2;
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const long long goff =
+              ((long long)(bi * s.Hq + kvh * G + 2 * (u0 + t) + h2) * s.T + (long long)j * kB) * kD;
+          bulk_s2g(o + goff, base + L::kOffQ + t * 32768 + h2 * 16384, bytes);
+          if (RES) bulk_s2g(o_res + goff, base + L::kOffK + t * 32768 + h2 * 16384, bytes);
+        }
+        bulk_commit();
+        bulk_wait_read_all();
       }
     }
   }
