@@ -95,8 +95,9 @@ tc_bwd_d_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   Ctl& c = *reinterpret_cast<Ctl*>(base + kOffCtl);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // Dense: every history block, the longest query blocks first.
-  const int j = s.dense ? s.N - 1 - (int)blockIdx.x : (int)blockIdx.x;
+  // The longest query blocks first (in the dense comparison, every history
+  // block), so the short ones fill the last wave.
+  const int j = s.N - 1 - (int)blockIdx.x;
   const int kvh = blockIdx.y / TILES, u = blockIdx.y % TILES, bi = blockIdx.z;
   const int G = 2 * TILES;
   const int h0 = kvh * G + 2 * u;  // the tile's two heads: h0, h0 + 1
@@ -365,7 +366,7 @@ tc_bwd_dq_recompute_kernel(const __grid_constant__ CUtensorMap tm_q,
   Ctl& c = *reinterpret_cast<Ctl*>(base + kOffCtl);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int j = s.dense ? s.N - 1 - (int)blockIdx.x : (int)blockIdx.x;
+  const int j = s.N - 1 - (int)blockIdx.x;  // longest query blocks first
   const int kvh = blockIdx.y / TILES, u = blockIdx.y % TILES, bi = blockIdx.z;
   const int G = 2 * TILES;
   const int h0 = kvh * G + 2 * u;
@@ -667,7 +668,10 @@ tc_bwd_dq_kernel(const __nv_bfloat16* __restrict__ ds, const __grid_constant__ C
   Ctl& c = *reinterpret_cast<Ctl*>(base + kOffCtl);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int j = blockIdx.x, kvh = blockIdx.y / TILES, u = blockIdx.y % TILES, bi = blockIdx.z;
+  // The longest query blocks (most attended blocks) start first, so the
+  // short ones fill the last wave.
+  const int j = s.N - 1 - (int)blockIdx.x;
+  const int kvh = blockIdx.y / TILES, u = blockIdx.y % TILES, bi = blockIdx.z;
   const int G = 2 * TILES;
   const int h0 = kvh * G + 2 * u;
   const long long irow = ((long long)(bi * s.Hkv + kvh) * s.N + j);

@@ -135,8 +135,10 @@ __device__ __forceinline__ void tc_fwd_body(const CUtensorMap& tm_q, const CUten
   Ctl<kStages>& c = *reinterpret_cast<Ctl<kStages>*>(base + L::kOffCtl);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // Dense: the longest query blocks (most keys) start first.
-  const int j = s.dense ? s.N - 1 - (int)blockIdx.x : (int)blockIdx.x;
+  // The longest query blocks (most keys) start first, so the short ones
+  // (fewer than K history blocks to attend, or the dense comparison's
+  // early blocks) fill the last wave.
+  const int j = s.N - 1 - (int)blockIdx.x;
   // blockIdx.y: KV head and, with TILES = 1, which of its G/2 tiles.
   const int G = TILES == 2 ? 4 : s.Hq / s.Hkv;  // two tiles: G = 4
   const int tpk = TILES == 2 ? 1 : G / 2;        // CTAs per KV head
